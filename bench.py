@@ -1,0 +1,414 @@
+"""Benchmark of the single-GPU MoE layer (route -> dispatch -> expert MLP -> combine).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mixtral] [--impl ours|reference]
+
+One step = one moe_layer_forward over one batch of T tokens of the workload
+(default: the Mixtral-shaped layer, T=4096, H=4096, E=8, top-2, F=14336, bf16).
+Inputs are synthetic and seeded. Rank 0 prints one JSON line.
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
+on the launching stream; L2 is flushed (a 256 MB write) before every step,
+outside the events. A barrier and a device synchronisation bracket the timed
+region; with several ranks every rank runs its own replica of the layer on its
+own tokens (weak scaling, no data-path collective) and the time is the maximum
+over ranks. `e2e` repeats the measurement through the same C ABI call with the
+step's inputs copied from pinned host memory and the output copied back inside
+the timed region. A second pass calls the four piecewise entry points with
+events between them to attribute time to route, dispatch, expert MLP and
+combine; the expert MLP (the grouped GEMMs, the dominant cost) gives `roofline`.
+
+`--impl reference` times the CPU oracle on this host's cores instead, on a
+bounded sample of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+METRIC = "MoE layer tokens/s on 1 B200; dispatch/combine HBM GB/s & GEMM % of roofline"
+KERNELS_PER_STEP = 7   # route x3, dispatch, gate/up GEMM, down GEMM, combine
+
+
+def load_peaks():
+    if os.path.exists(PEAKS_PATH):
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        p["source"] = "measured"
+        return p
+    p = dict(FALLBACK_PEAKS)
+    p["source"] = "fallback"
+    return p
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+class Clocks:
+    """Samples nvidia-smi during the timed region (clocks and throttle reasons)."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 8:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+
+        def num(s):
+            try:
+                return float(s)
+            except ValueError:
+                return float("nan")
+        sm = np.array([num(r[0]) for r in rows])
+        mx = np.array([num(r[1]) for r in rows])
+        pw = np.array([num(r[2]) for r in rows])
+        loaded = pw >= np.nanmax(pw) * 0.5 if np.isfinite(pw).any() else np.ones(len(rows), bool)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[4 + i]
+                          and not r[4 + i].startswith("Not")})
+        return {"sm_mhz": float(np.nanmedian(sm[loaded])) if loaded.any() else float(np.nanmedian(sm)),
+                "sm_max_mhz": float(np.nanmax(mx)), "samples": len(rows), "reasons": reasons}
+
+
+def flush_l2(buf: torch.Tensor):
+    buf.add_(1)
+
+
+class Layer:
+    """Device-resident inputs, weights and workspace of one replica."""
+
+    def __init__(self, wl: W.Workload, seed: int, device):
+        import combine_moe_route_13_b200 as M
+        self.M = M
+        self.wl = wl
+        self.C = M.moe_capacity(wl.T, wl.K, wl.E, wl.cf)
+        self.cfg = M.make_config(wl.T, wl.H, wl.E, wl.K, wl.F, wl.S, self.C, wl.row_align, wl.act)
+        st = M.moe_check_config(self.cfg)
+        if st != M.MOE_OK:
+            raise SystemExit(f"unsupported workload: {M.status_string(st)}")
+        self.inp = W.make_inputs(wl, seed=seed, device=device)
+        self.ws = M.alloc_workspace(M.moe_workspace_bytes(self.cfg), device)
+        self.out = torch.empty(wl.T, wl.H, dtype=wl.torch_act, device=device)
+        self.aux = None
+
+    def forward(self):
+        self.aux = self.M.moe_layer_forward(self.cfg, self.inp["logits"], self.inp["x"],
+                                            self.inp["w_gu"], self.inp["w_d"], self.out, self.ws)
+
+    def views(self):
+        return self.M.layer_views(self.cfg, self.ws, self.aux)
+
+
+def time_steps(fn, steps, warmup, flush_buf, stream):
+    for _ in range(warmup):
+        flush_l2(flush_buf)
+        fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for a, b in evs:
+        flush_l2(flush_buf)
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def phase_times(layer: Layer, steps, flush_buf, stream):
+    """Per-phase device times (ms, mean over steps) through the piecewise entry points."""
+    M = layer.M
+    v = layer.views()
+    cfg, inp = layer.cfg, layer.inp
+    names = ("route", "dispatch", "expert_mlp", "combine")
+    calls = (
+        lambda: M.moe_route_topk(cfg, inp["logits"], v["topk_idx"], v["topk_w"], v["expert_counts"],
+                                 v["overflow"], v["expert_offsets"], v["segment_offsets"],
+                                 v["token_slot"], v["row_src"], v["totals"], layer.ws),
+        lambda: M.moe_dispatch(cfg, inp["x"], v["token_slot"], v["xp"]),
+        lambda: M.moe_expert_mlp(cfg, v["xp"], v["expert_offsets"], v["expert_counts"],
+                                 inp["w_gu"], inp["w_d"], v["h"], v["y"], layer.ws),
+        lambda: M.moe_combine(cfg, v["y"], v["token_slot"], v["topk_w"], layer.out),
+    )
+    acc = {n: [] for n in names}
+    for _ in range(steps + 1):
+        flush_l2(flush_buf)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
+        ev[0].record(stream)
+        for i, c in enumerate(calls):
+            c()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        for i, n in enumerate(names):
+            acc[n].append(ev[i].elapsed_time(ev[i + 1]))
+    return {n: float(np.mean(acc[n][1:])) for n in names}   # first pass is a warm-up
+
+
+def e2e_steps(layer: Layer, steps, warmup, flush_buf, stream):
+    """Same layer through the same C call, inputs from pinned host memory, output back to host."""
+    inp = layer.inp
+    h_logits = inp["logits"].cpu().pin_memory()
+    h_x = inp["x"].cpu().pin_memory()
+    h_out = torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory()
+    d_logits = torch.empty_like(inp["logits"])
+    d_x = torch.empty_like(inp["x"])
+    M, cfg = layer.M, layer.cfg
+
+    def step():
+        d_logits.copy_(h_logits, non_blocking=True)
+        d_x.copy_(h_x, non_blocking=True)
+        M.moe_layer_forward(cfg, d_logits, d_x, inp["w_gu"], inp["w_d"], layer.out, layer.ws)
+        h_out.copy_(layer.out, non_blocking=True)
+
+    times = time_steps(step, steps, warmup, flush_buf, stream)
+    h2d = h_logits.numel() * 4 + h_x.numel() * h_x.element_size()
+    d2h = h_out.numel() * h_out.element_size()
+    return times, h2d, d2h
+
+
+def algorithmic(layer: Layer, totals):
+    wl = layer.wl
+    s = 4 if wl.act == "f32" else 2
+    N = int(totals[1])
+    T, H, F, K, E = wl.T, wl.H, wl.F, wl.K, wl.E
+    return {
+        "N": N,
+        "mlp_flops": 6.0 * N * H * F,
+        "dispatch_bytes": (T + N) * H * s + T * K * 4,
+        "combine_bytes": (N + T) * H * s + T * K * 8,
+        "route_bytes": T * E * 4 + T * K * 12,
+    }
+
+
+def cpu_oracle_sample(wl: W.Workload, tokens: int, seed: int, inp_host=None):
+    """The oracle's whole layer on the first `tokens` tokens of the workload
+    (capacity scaled to that batch). Returns (seconds, tokens)."""
+    from oracle import moe_oracle as O
+    import torch as _t
+    if inp_host is None:
+        inp_host = W.make_inputs(wl, seed=seed, device="cpu")
+
+    def np_act(t):
+        t = t.contiguous()
+        return t.view(_t.int16).numpy().view(np.uint16) if t.dtype == _t.bfloat16 else t.numpy()
+
+    lg = inp_host["logits"][:tokens].numpy()
+    x = np_act(inp_host["x"][:tokens])
+    w_gu, w_d = np_act(inp_host["w_gu"]), np_act(inp_host["w_d"])
+    C = O.capacity(tokens, wl.K, wl.E, wl.cf)
+    t0 = time.perf_counter()
+    O.layer_forward(lg, x, w_gu, w_d, wl.K, C, wl.row_align, wl.S, wl.act)
+    return time.perf_counter() - t0, tokens
+
+
+def cpu_cores():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = max((i.get("num_threads", 1) for i in info), default=1)
+        return int(n)
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+def run_reference(args, wl: W.Workload, world, rank):
+    if rank != 0:
+        return 0
+    tokens = args.cpu_tokens
+    inp_host = W.make_inputs(wl, seed=0, device="cpu")
+    for _ in range(args.warmup):
+        cpu_oracle_sample(wl, tokens, 0, inp_host)
+    secs = [cpu_oracle_sample(wl, tokens, 0, inp_host)[0] for _ in range(args.steps)]
+    ms = float(np.mean(secs)) * 1e3
+    value = tokens / (ms / 1e3)
+    cores = cpu_cores()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.act,
+        "data": "synthetic", "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E,
+                                        "K": wl.K, "F": wl.F, "S": wl.S, "cf": wl.cf},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"whole layer (float64 numpy oracle) on the first {tokens} "
+                                   f"tokens of the workload per step, capacity scaled to that batch"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=16)
+    ap.add_argument("--warmup", type=int, default=4)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mixtral", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--cpu-tokens", type=int, default=256,
+                    help="tokens of the CPU-oracle sample per step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        raise SystemExit("--warmup must be >= 3")
+    wl = W.WORKLOADS[args.workload]
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, wl, world, rank)
+
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    device = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(device)
+    peaks = load_peaks()
+
+    layer = Layer(wl, seed=rank, device=device)
+    flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+
+    layer.forward()
+    torch.cuda.synchronize()
+    st = layer.M.moe_get_device_status(layer.ws)
+    if st != layer.M.MOE_OK:
+        raise SystemExit(f"device status after the first step: {layer.M.status_string(st)}")
+    totals = layer.views()["totals"].cpu().tolist()
+    alg = algorithmic(layer, totals)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    clocks = Clocks(device.index if device.index is not None else 0)
+    barrier()
+    clocks.start()
+    times = time_steps(layer.forward, args.steps, args.warmup, flush_buf, stream)
+    barrier()
+    clk = clocks.stop()
+    total_ms = float(np.sum(times))
+    if world > 1:
+        t = torch.tensor([total_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms = total_ms / args.steps
+    value = world * wl.T / (ms / 1e3)
+
+    e2e_t, h2d, d2h = e2e_steps(layer, args.steps, args.warmup, flush_buf, stream)
+    e2e_ms = float(np.sum(e2e_t))
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_ms /= args.steps
+
+    ph = phase_times(layer, max(args.steps // 2, 3), flush_buf, stream)
+    st = layer.M.moe_get_device_status(layer.ws)
+    if st != layer.M.MOE_OK:
+        raise SystemExit(f"device status after timing: {layer.M.status_string(st)}")
+
+    hbm = peaks["hbm_gbs"]
+    tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    mlp_tflops = alg["mlp_flops"] / (ph["expert_mlp"] * 1e-3) / 1e12
+    kernels = {
+        "route_us": ph["route"] * 1e3,
+        "dispatch_us": ph["dispatch"] * 1e3,
+        "dispatch_gbs": alg["dispatch_bytes"] / (ph["dispatch"] * 1e-3) / 1e9,
+        "expert_mlp_us": ph["expert_mlp"] * 1e3,
+        "expert_mlp_tflops": mlp_tflops,
+        "combine_us": ph["combine"] * 1e3,
+        "combine_gbs": alg["combine_bytes"] / (ph["combine"] * 1e-3) / 1e9,
+    }
+    kernels["dispatch_hbm_frac"] = kernels["dispatch_gbs"] / hbm
+    kernels["combine_hbm_frac"] = kernels["combine_gbs"] / hbm
+    kernels["expert_mlp_tensor_frac_burst"] = mlp_tflops / peaks["bf16_tflops"]
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        secs, tok = cpu_oracle_sample(wl, args.cpu_tokens, 0)
+        cpu = {"value": tok / secs, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+               "sample": f"whole layer (float64 numpy oracle) on the first {tok} tokens of the "
+                         f"workload, capacity scaled to that batch; {secs:.1f} s"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.act == "bf16" else "f32",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "K": wl.K, "F": wl.F,
+                   "S": wl.S, "cf": wl.cf, "capacity": layer.C, "row_align": wl.row_align,
+                   "effective_tokens": alg["N"], "overflow": int(totals[2]),
+                   "l2": "flushed (256 MB write) before every step", "parallelism": f"replicas{world}"},
+        "e2e": {"value": world * wl.T / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "roofline": {"bound": "tensor", "kernel": "expert_mlp (gate/up + down grouped GEMMs)",
+                     "achieved": mlp_tflops, "peak": tensor_peak, "unit": "TFLOP/s",
+                     "frac": mlp_tflops / tensor_peak,
+                     "peak_kind": f"bf16_tflops_sustained ({peaks['source']})", "traffic": None},
+        "kernels": kernels,
+        "effective_tokens_per_s": world * alg["N"] / (ms / 1e3),
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

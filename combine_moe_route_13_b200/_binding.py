@@ -1,0 +1,268 @@
+"""ctypes binding of libmoe.so: the C entry points under the same names.
+
+Argument marshalling only: every step of the layer runs in the library's
+CUDA kernels. torch tensors supply device memory and the stream; each
+function checks dtype, device and contiguity, passes raw pointers and raises
+MoeError on a non-OK status. There is no fallback: if the library is missing
+or fails to load, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoe.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED = 2
+MOE_ERR_WORKSPACE = 3
+MOE_ERR_CUDA = 4
+MOE_ERR_TIMEOUT = 5
+MOE_ERR_DEVICE_INPUT = 6
+MOE_F32 = 0
+MOE_BF16 = 1
+MOE_FLAG_NONE = 0
+
+# every symbol declared in include/moe.h
+EXPORTS = ("moe_capacity", "moe_max_rows", "moe_check_config", "moe_route_workspace_bytes",
+           "moe_workspace_bytes", "moe_workspace_init", "moe_route_topk", "moe_dispatch",
+           "moe_expert_mlp", "moe_combine", "moe_layer_forward", "moe_get_device_status",
+           "moe_status_string", "moe_version")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} (status {code})")
+
+
+class MoeConfig(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("K", ctypes.c_int32), ("F", ctypes.c_int32), ("S", ctypes.c_int32),
+                ("capacity", ctypes.c_int32), ("row_align", ctypes.c_int32),
+                ("act_dtype", ctypes.c_int32)]
+
+    def __repr__(self):
+        return ("MoeConfig(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")")
+
+
+class MoeLayerAux(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "topk_idx", "expert_counts", "overflow", "expert_offsets", "segment_offsets",
+        "token_slot", "row_src", "totals", "topk_w", "xp", "h", "y")]
+
+
+_P = ctypes.c_void_p
+_CFG = ctypes.POINTER(MoeConfig)
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libmoe.so is not built ({LIB_PATH}); run "
+                          "`python -m combine_moe_route_13_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    sig = {
+        "moe_capacity": (ctypes.c_int32, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_double]),
+        "moe_max_rows": (ctypes.c_int64, [_CFG]),
+        "moe_check_config": (ctypes.c_int, [_CFG]),
+        "moe_route_workspace_bytes": (ctypes.c_size_t, [_CFG]),
+        "moe_workspace_bytes": (ctypes.c_size_t, [_CFG, ctypes.c_uint32]),
+        "moe_workspace_init": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
+        "moe_route_topk": (ctypes.c_int, [_CFG] + [_P] * 10 + [_P, ctypes.c_size_t, _P]),
+        "moe_dispatch": (ctypes.c_int, [_CFG, _P, _P, _P, _P]),
+        "moe_expert_mlp": (ctypes.c_int, [_CFG] + [_P] * 7 + [_P, ctypes.c_size_t, _P]),
+        "moe_combine": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P]),
+        "moe_layer_forward": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, ctypes.c_uint32, _P,
+                                             ctypes.c_size_t, ctypes.POINTER(MoeLayerAux), _P]),
+        "moe_get_device_status": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int), _P]),
+        "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "moe_version": (ctypes.c_int32, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+LIB = _load()
+
+
+def status_string(code: int) -> str:
+    return LIB.moe_status_string(int(code)).decode()
+
+
+def _check(code: int, where: str):
+    if code != MOE_OK:
+        raise MoeError(code, where)
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: torch.Tensor | None, dtype=None, name="tensor") -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    return t.data_ptr()
+
+
+def make_config(T, H, E, K, F, S, capacity, row_align=128, act="bf16") -> MoeConfig:
+    return MoeConfig(int(T), int(H), int(E), int(K), int(F), int(S), int(capacity),
+                     int(row_align), MOE_F32 if act in ("f32", torch.float32, MOE_F32) else MOE_BF16)
+
+
+def act_dtype(cfg: MoeConfig) -> torch.dtype:
+    return torch.float32 if cfg.act_dtype == MOE_F32 else torch.bfloat16
+
+
+# ---------------------------------------------------------------- entry points
+
+def moe_capacity(T: int, K: int, E: int, cf: float) -> int:
+    return int(LIB.moe_capacity(T, K, E, float(cf)))
+
+
+def moe_max_rows(cfg: MoeConfig) -> int:
+    return int(LIB.moe_max_rows(ctypes.byref(cfg)))
+
+
+def moe_check_config(cfg: MoeConfig) -> int:
+    return int(LIB.moe_check_config(ctypes.byref(cfg)))
+
+
+def moe_route_workspace_bytes(cfg: MoeConfig) -> int:
+    return int(LIB.moe_route_workspace_bytes(ctypes.byref(cfg)))
+
+
+def moe_workspace_bytes(cfg: MoeConfig, flags: int = MOE_FLAG_NONE) -> int:
+    return int(LIB.moe_workspace_bytes(ctypes.byref(cfg), flags))
+
+
+def moe_workspace_init(ws: torch.Tensor, stream=None):
+    _check(LIB.moe_workspace_init(_ptr(ws, name="ws"), ws.numel() * ws.element_size(),
+                                  _stream(stream)), "moe_workspace_init")
+
+
+def moe_route_topk(cfg, logits, topk_idx, topk_w, expert_counts, overflow, expert_offsets,
+                   segment_offsets, token_slot, row_src, totals, ws, stream=None):
+    i32 = torch.int32
+    _check(LIB.moe_route_topk(
+        ctypes.byref(cfg), _ptr(logits, torch.float32, "logits"), _ptr(topk_idx, i32, "topk_idx"),
+        _ptr(topk_w, torch.float32, "topk_w"), _ptr(expert_counts, i32, "expert_counts"),
+        _ptr(overflow, i32, "overflow"), _ptr(expert_offsets, i32, "expert_offsets"),
+        _ptr(segment_offsets, i32, "segment_offsets"), _ptr(token_slot, i32, "token_slot"),
+        _ptr(row_src, i32, "row_src"), _ptr(totals, i32, "totals"), _ptr(ws, name="ws"),
+        ws.numel() * ws.element_size(), _stream(stream)), "moe_route_topk")
+
+
+def moe_dispatch(cfg, x, token_slot, xp, stream=None):
+    dt = act_dtype(cfg)
+    _check(LIB.moe_dispatch(ctypes.byref(cfg), _ptr(x, dt, "x"),
+                            _ptr(token_slot, torch.int32, "token_slot"), _ptr(xp, dt, "xp"),
+                            _stream(stream)), "moe_dispatch")
+
+
+def moe_expert_mlp(cfg, xp, expert_offsets, expert_counts, w_gu, w_d, h, y, ws, stream=None):
+    dt = act_dtype(cfg)
+    _check(LIB.moe_expert_mlp(
+        ctypes.byref(cfg), _ptr(xp, dt, "xp"), _ptr(expert_offsets, torch.int32, "expert_offsets"),
+        _ptr(expert_counts, torch.int32, "expert_counts"), _ptr(w_gu, dt, "w_gu"),
+        _ptr(w_d, dt, "w_d"), _ptr(h, dt, "h"), _ptr(y, dt, "y"), _ptr(ws, name="ws"),
+        ws.numel() * ws.element_size(), _stream(stream)), "moe_expert_mlp")
+
+
+def moe_combine(cfg, y, token_slot, topk_w, out, stream=None):
+    dt = act_dtype(cfg)
+    _check(LIB.moe_combine(ctypes.byref(cfg), _ptr(y, dt, "y"),
+                           _ptr(token_slot, torch.int32, "token_slot"),
+                           _ptr(topk_w, torch.float32, "topk_w"), _ptr(out, dt, "out"),
+                           _stream(stream)), "moe_combine")
+
+
+def moe_layer_forward(cfg, logits, x, w_gu, w_d, out, ws, flags=MOE_FLAG_NONE, stream=None):
+    """Runs the fused layer; returns a MoeLayerAux with the workspace pointers of
+    the intermediates (see layer_views)."""
+    dt = act_dtype(cfg)
+    aux = MoeLayerAux()
+    _check(LIB.moe_layer_forward(
+        ctypes.byref(cfg), _ptr(logits, torch.float32, "logits"), _ptr(x, dt, "x"),
+        _ptr(w_gu, dt, "w_gu"), _ptr(w_d, dt, "w_d"), _ptr(out, dt, "out"), flags,
+        _ptr(ws, name="ws"), ws.numel() * ws.element_size(), ctypes.byref(aux), _stream(stream)),
+        "moe_layer_forward")
+    return aux
+
+
+def moe_get_device_status(ws, stream=None) -> int:
+    st = ctypes.c_int(0)
+    _check(LIB.moe_get_device_status(_ptr(ws, name="ws"), ctypes.byref(st), _stream(stream)),
+           "moe_get_device_status")
+    return int(st.value)
+
+
+def moe_version() -> int:
+    return int(LIB.moe_version())
+
+
+# ---------------------------------------------------------------- conveniences
+
+def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A zeroed byte workspace (torch allocations are 256-byte aligned)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def alloc_route_outputs(cfg: MoeConfig, device="cuda") -> dict:
+    i32 = dict(dtype=torch.int32, device=device)
+    R = moe_max_rows(cfg)
+    return {
+        "topk_idx": torch.empty(cfg.T, cfg.K, **i32),
+        "topk_w": torch.empty(cfg.T, cfg.K, dtype=torch.float32, device=device),
+        "expert_counts": torch.empty(cfg.E, **i32),
+        "overflow": torch.empty(cfg.E, **i32),
+        "expert_offsets": torch.empty(cfg.E + 1, **i32),
+        "segment_offsets": torch.empty(cfg.S + 1, **i32),
+        "token_slot": torch.empty(cfg.T, cfg.K, **i32),
+        "row_src": torch.empty(max(R, 1), **i32),
+        "totals": torch.empty(4, **i32),
+    }
+
+
+def layer_views(cfg: MoeConfig, ws: torch.Tensor, aux: MoeLayerAux) -> dict:
+    """torch views of the intermediates that moe_layer_forward left in ws."""
+    base = ws.data_ptr()
+    R = moe_max_rows(cfg)
+    dt = act_dtype(cfg)
+    es = 4 if dt == torch.float32 else 2
+
+    def view(ptr, nbytes, dtype, shape):
+        off = ptr - base
+        return ws[off:off + nbytes].view(dtype).view(shape)
+
+    TK = cfg.T * cfg.K
+    return {
+        "topk_idx": view(aux.topk_idx, TK * 4, torch.int32, (cfg.T, cfg.K)),
+        "topk_w": view(aux.topk_w, TK * 4, torch.float32, (cfg.T, cfg.K)),
+        "expert_counts": view(aux.expert_counts, cfg.E * 4, torch.int32, (cfg.E,)),
+        "overflow": view(aux.overflow, cfg.E * 4, torch.int32, (cfg.E,)),
+        "expert_offsets": view(aux.expert_offsets, (cfg.E + 1) * 4, torch.int32, (cfg.E + 1,)),
+        "segment_offsets": view(aux.segment_offsets, (cfg.S + 1) * 4, torch.int32, (cfg.S + 1,)),
+        "token_slot": view(aux.token_slot, TK * 4, torch.int32, (cfg.T, cfg.K)),
+        "row_src": view(aux.row_src, R * 4, torch.int32, (R,)),
+        "totals": view(aux.totals, 16, torch.int32, (4,)),
+        "xp": view(aux.xp, R * cfg.H * es, dt, (R, cfg.H)),
+        "h": view(aux.h, R * cfg.F * es, dt, (R, cfg.F)),
+        "y": view(aux.y, R * cfg.H * es, dt, (R, cfg.H)),
+    }

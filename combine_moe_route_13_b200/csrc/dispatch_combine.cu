@@ -1,0 +1,178 @@
+// Dispatch (scatter of token rows into the expert-grouped buffer) and combine
+// (weighted gather-sum back to token order).
+//
+// Dispatch follows the pplx-kernels page ("Dispatch"): every token row is
+// copied to the rows its experts own in the grouped-GEMM input. Combine
+// follows its "Combine" section and the EFA page's receiver-side accumulation
+// ("Диспетчеризация и комбинирование"): a token's K expert outputs are read
+// back and summed with the router weights.
+//
+// Both are pure HBM streams. One block per token row; each thread moves
+// 16-byte vectors (8 bf16 or 4 fp32), several per iteration so that enough
+// loads are in flight. A dispatched row is read once and written K times;
+// a combined row reads its K expert rows and is written once.
+#include <algorithm>
+
+#include <cuda_bf16.h>
+
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int DC_THREADS = 128;
+constexpr int DC_UNROLL = 4;
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) { return __ldcs(p); }
+
+__global__ void __launch_bounds__(DC_THREADS)
+dispatch_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ token_slot,
+                uint4* __restrict__ xp, int K, int row_vecs) {
+  __shared__ int s_slot[MAX_K];
+  __shared__ int s_any;
+  const int t = blockIdx.x;
+  if (threadIdx.x == 0) s_any = 0;
+  __syncthreads();
+  if (threadIdx.x < K) {
+    const int s = token_slot[(size_t)t * K + threadIdx.x];
+    s_slot[threadIdx.x] = s;
+    if (s >= 0) atomicOr(&s_any, 1);
+  }
+  __syncthreads();
+  if (!s_any) return;   // every assignment of this token overflowed: nothing to copy
+  const uint4* src = x + (size_t)t * row_vecs;
+  for (int v0 = threadIdx.x; v0 < row_vecs; v0 += DC_THREADS * DC_UNROLL) {
+    uint4 d[DC_UNROLL];
+#pragma unroll
+    for (int u = 0; u < DC_UNROLL; ++u) {
+      const int v = v0 + u * DC_THREADS;
+      if (v < row_vecs) d[u] = ld_stream(src + v);
+    }
+    for (int k = 0; k < K; ++k) {
+      const int s = s_slot[k];
+      if (s < 0) continue;
+      uint4* dst = xp + (size_t)s * row_vecs;
+#pragma unroll
+      for (int u = 0; u < DC_UNROLL; ++u) {
+        const int v = v0 + u * DC_THREADS;
+        if (v < row_vecs) dst[v] = d[u];
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4& q, float (&f)[8]) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+// out[t] = sum_k w[t,k] * y[slot[t,k]] with fp32 accumulation in k order.
+template <bool BF16>
+__global__ void __launch_bounds__(DC_THREADS)
+combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ token_slot,
+               const float* __restrict__ topk_w, uint4* __restrict__ out, int K, int row_vecs) {
+  __shared__ int s_slot[MAX_K];
+  __shared__ float s_w[MAX_K];
+  const int t = blockIdx.x;
+  if (threadIdx.x < K) {
+    s_slot[threadIdx.x] = token_slot[(size_t)t * K + threadIdx.x];
+    s_w[threadIdx.x] = topk_w[(size_t)t * K + threadIdx.x];
+  }
+  __syncthreads();
+  constexpr int LANES = BF16 ? 8 : 4;
+  uint4* dst = out + (size_t)t * row_vecs;
+  for (int v0 = threadIdx.x; v0 < row_vecs; v0 += DC_THREADS * 2) {
+    float acc[2][LANES];
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int i = 0; i < LANES; ++i) acc[u][i] = 0.f;
+    int k = 0;
+    // groups of 4 experts: issue the loads, then accumulate in k order
+    for (; k < K; k += 4) {
+      uint4 d[4][2];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int s = (k + j < K) ? s_slot[k + j] : -1;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int v = v0 + u * DC_THREADS;
+          if (s >= 0 && v < row_vecs) d[j][u] = __ldg(y + (size_t)s * row_vecs + v);
+          else d[j][u] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (k + j >= K || s_slot[k + j] < 0) continue;
+        const float wk = s_w[k + j];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (BF16) {
+            float f[8];
+            unpack_bf16x8(d[j][u], f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[u][i] = fmaf(wk, f[i], acc[u][i]);
+          } else {
+            acc[u][0] = fmaf(wk, __uint_as_float(d[j][u].x), acc[u][0]);
+            acc[u][1] = fmaf(wk, __uint_as_float(d[j][u].y), acc[u][1]);
+            acc[u][2] = fmaf(wk, __uint_as_float(d[j][u].z), acc[u][2]);
+            acc[u][3] = fmaf(wk, __uint_as_float(d[j][u].w), acc[u][3]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int v = v0 + u * DC_THREADS;
+      if (v >= row_vecs) continue;
+      uint4 o;
+      if (BF16) {
+        o.x = pack_bf16x2(acc[u][0], acc[u][1]);
+        o.y = pack_bf16x2(acc[u][2], acc[u][3]);
+        o.z = pack_bf16x2(acc[u][4], acc[u][5]);
+        o.w = pack_bf16x2(acc[u][6], acc[u][7]);
+      } else {
+        o.x = __float_as_uint(acc[u][0]);
+        o.y = __float_as_uint(acc[u][1]);
+        o.z = __float_as_uint(acc[u][2]);
+        o.w = __float_as_uint(acc[u][3]);
+      }
+      __stcs(dst + v, o);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t* slot, void* xp,
+                            cudaStream_t s) {
+  if (c.T == 0) return cudaSuccess;
+  const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
+  dispatch_kernel<<<c.T, DC_THREADS, 0, s>>>(static_cast<const uint4*>(x), slot,
+                                             static_cast<uint4*>(xp), c.K, row_vecs);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const moe_config_t& c, const void* y, const int32_t* slot,
+                           const float* w, void* out, cudaStream_t s) {
+  if (c.T == 0) return cudaSuccess;
+  const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
+  if (c.act_dtype == MOE_BF16)
+    combine_kernel<true><<<c.T, DC_THREADS, 0, s>>>(static_cast<const uint4*>(y), slot, w,
+                                                    static_cast<uint4*>(out), c.K, row_vecs);
+  else
+    combine_kernel<false><<<c.T, DC_THREADS, 0, s>>>(static_cast<const uint4*>(y), slot, w,
+                                                     static_cast<uint4*>(out), c.K, row_vecs);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,240 @@
+// extern "C" entry points of libmoe.so: argument validation, workspace layout
+// and the launch order of the layer. Every entry point only launches kernels
+// on the caller's stream; none allocates, frees or synchronises (except
+// moe_get_device_status, which exists to synchronise).
+#include <algorithm>
+#include <climits>
+#include <cmath>
+
+#include "moe_internal.h"
+
+namespace moe {
+
+int64_t max_rows(const moe_config_t& c) {
+  return std::min<int64_t>((int64_t)c.T * c.K, (int64_t)c.E * c.capacity) +
+         (int64_t)c.E * (c.row_align - 1);
+}
+
+static moe_status_t basic_checks(const moe_config_t* c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->T < 0 || c->H < 1 || c->E < 1 || c->K < 1 || c->F < 1 || c->S < 1) return MOE_ERR_INVALID_ARG;
+  if (c->K > c->E || c->E % c->S != 0 || c->capacity < 0 || c->row_align < 1)
+    return MOE_ERR_INVALID_ARG;
+  if (c->act_dtype != MOE_F32 && c->act_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (c->E > MAX_E || c->K > MAX_K || c->row_align > 1024) return MOE_ERR_UNSUPPORTED;
+  if ((int64_t)c->T * c->K > INT_MAX / 2) return MOE_ERR_UNSUPPORTED;
+  if (max_rows(*c) > INT_MAX / 2) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status_t validate(const moe_config_t* c, bool need_mlp) {
+  moe_status_t st = basic_checks(c);
+  if (st != MOE_OK) return st;
+  const int sz = act_size(c->act_dtype);
+  if (((int64_t)c->H * sz) % 16 != 0 || ((int64_t)c->F * sz) % 16 != 0) return MOE_ERR_UNSUPPORTED;
+  if (need_mlp && c->act_dtype == MOE_BF16) {
+    if (c->H % 64 != 0 || c->F % 64 != 0) return MOE_ERR_UNSUPPORTED;
+    if ((int64_t)c->E * 2 * c->F > INT_MAX / 2 || (int64_t)c->E * c->H > INT_MAX / 2)
+      return MOE_ERR_UNSUPPORTED;
+  }
+  if (need_mlp && c->act_dtype == MOE_F32 && ceil_div(max_rows(*c), 32) + c->E > 65535)
+    return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+WsLayout ws_layout(const moe_config_t& c) {
+  WsLayout L;
+  const int64_t nblk = ceil_div(c.T, ROUTE_TB);
+  const int64_t TK = (int64_t)c.T * c.K;
+  const int64_t R = max_rows(c);
+  const size_t as = act_size(c.act_dtype);
+  size_t p = 256;   // status word region
+  L.blk_cnt = p;   p += align256((size_t)std::max<int64_t>(nblk, 1) * c.E * 4);
+  L.route_end = p;
+  L.topk_idx = p;  p += align256((size_t)TK * 4);
+  L.topk_w = p;    p += align256((size_t)TK * 4);
+  L.counts = p;    p += align256((size_t)c.E * 4);
+  L.overflow = p;  p += align256((size_t)c.E * 4);
+  L.offsets = p;   p += align256((size_t)(c.E + 1) * 4);
+  L.segoff = p;    p += align256((size_t)(c.S + 1) * 4);
+  L.totals = p;    p += align256(16);
+  L.slot = p;      p += align256((size_t)TK * 4);
+  L.row_src = p;   p += align256((size_t)R * 4);
+  L.xp = p;        p += align256((size_t)R * c.H * as);
+  L.h = p;         p += align256((size_t)R * c.F * as);
+  L.y = p;         p += align256((size_t)R * c.H * as);
+  L.total = p;
+  return L;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int32_t moe_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_TIMEOUT: return "a bounded wait inside a kernel gave up";
+    case MOE_ERR_DEVICE_INPUT: return "a device-side table held an out-of-range value";
+  }
+  return "unknown status";
+}
+
+int32_t moe_capacity(int32_t T, int32_t K, int32_t E, double cf) {
+  if (T < 0 || K < 1 || E < 1) return -1;
+  if (cf < 0) return T;
+  const double c = std::ceil(cf * (double)T * (double)K / (double)E);
+  if (!(c <= (double)INT_MAX)) return -1;
+  return (int32_t)c;
+}
+
+int64_t moe_max_rows(const moe_config_t* cfg) {
+  if (basic_checks(cfg) != MOE_OK) return -1;
+  return max_rows(*cfg);
+}
+
+moe_status_t moe_check_config(const moe_config_t* cfg) { return validate(cfg, true); }
+
+size_t moe_route_workspace_bytes(const moe_config_t* cfg) {
+  if (basic_checks(cfg) != MOE_OK) return 0;
+  return ws_layout(*cfg).route_end;
+}
+
+size_t moe_workspace_bytes(const moe_config_t* cfg, uint32_t flags) {
+  (void)flags;
+  if (basic_checks(cfg) != MOE_OK) return 0;
+  return ws_layout(*cfg).total;
+}
+
+moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < 256 || (reinterpret_cast<uintptr_t>(ws) & 255u)) return MOE_ERR_WORKSPACE;
+  return cuda_status(cudaMemsetAsync(ws, 0, 4, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_route_topk(const moe_config_t* cfg, const float* logits, int32_t* topk_idx,
+                            float* topk_w, int32_t* expert_counts, int32_t* overflow,
+                            int32_t* expert_offsets, int32_t* segment_offsets,
+                            int32_t* token_slot, int32_t* row_src, int32_t* totals, void* ws,
+                            size_t ws_bytes, void* stream) {
+  moe_status_t st = validate(cfg, false);
+  if (st != MOE_OK) return st;
+  if (!expert_counts || !overflow || !expert_offsets || !segment_offsets || !totals)
+    return MOE_ERR_INVALID_ARG;
+  if (cfg->T > 0 && (!logits || !topk_idx || !topk_w || !token_slot)) return MOE_ERR_INVALID_ARG;
+  const int64_t R = max_rows(*cfg);
+  if (R > 0 && !row_src) return MOE_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(*cfg);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < L.route_end)
+    return MOE_ERR_WORKSPACE;
+  int32_t* blk = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + L.blk_cnt);
+  return cuda_status(launch_route(*cfg, logits, topk_idx, topk_w, expert_counts, overflow,
+                                  expert_offsets, segment_offsets, token_slot, row_src, totals,
+                                  blk, R, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* token_slot,
+                          void* xp, void* stream) {
+  moe_status_t st = validate(cfg, false);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x || !token_slot || !xp) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(xp)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_dispatch(*cfg, x, token_slot, xp, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_expert_mlp(const moe_config_t* cfg, const void* xp,
+                            const int32_t* expert_offsets, const int32_t* expert_counts,
+                            const void* w_gu, const void* w_d, void* h, void* y, void* ws,
+                            size_t ws_bytes, void* stream) {
+  moe_status_t st = validate(cfg, true);
+  if (st != MOE_OK) return st;
+  const int64_t R = max_rows(*cfg);
+  if (R == 0) return MOE_OK;
+  if (!xp || !expert_offsets || !expert_counts || !w_gu || !w_d || !h || !y)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(xp) || !aligned16(w_gu) || !aligned16(w_d) || !aligned16(h) || !aligned16(y))
+    return MOE_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < 256) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cfg->act_dtype == MOE_F32)
+    return cuda_status(launch_mlp_f32(*cfg, static_cast<const float*>(xp), expert_offsets,
+                                      expert_counts, static_cast<const float*>(w_gu),
+                                      static_cast<const float*>(w_d), static_cast<float*>(h),
+                                      static_cast<float*>(y), R, s));
+  return launch_mlp_bf16_tc(*cfg, xp, expert_offsets, expert_counts, w_gu, w_d, h, y, R,
+                            static_cast<uint32_t*>(ws), s);
+}
+
+moe_status_t moe_combine(const moe_config_t* cfg, const void* y, const int32_t* token_slot,
+                         const float* topk_w, void* out, void* stream) {
+  moe_status_t st = validate(cfg, false);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!y || !token_slot || !topk_w || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(
+      launch_combine(*cfg, y, token_slot, topk_w, out, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_layer_forward(const moe_config_t* cfg, const float* logits, const void* x,
+                               const void* w_gu, const void* w_d, void* out, uint32_t flags,
+                               void* ws, size_t ws_bytes, moe_layer_aux_t* aux, void* stream) {
+  moe_status_t st = validate(cfg, true);
+  if (st != MOE_OK) return st;
+  if (flags != MOE_FLAG_NONE) return MOE_ERR_UNSUPPORTED;
+  if (cfg->T > 0 && (!logits || !x || !out)) return MOE_ERR_INVALID_ARG;
+  if (!w_gu || !w_d) return MOE_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(*cfg);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  char* b = static_cast<char*>(ws);
+  moe_layer_aux_t a;
+  a.topk_idx = reinterpret_cast<int32_t*>(b + L.topk_idx);
+  a.topk_w = reinterpret_cast<float*>(b + L.topk_w);
+  a.expert_counts = reinterpret_cast<int32_t*>(b + L.counts);
+  a.overflow = reinterpret_cast<int32_t*>(b + L.overflow);
+  a.expert_offsets = reinterpret_cast<int32_t*>(b + L.offsets);
+  a.segment_offsets = reinterpret_cast<int32_t*>(b + L.segoff);
+  a.totals = reinterpret_cast<int32_t*>(b + L.totals);
+  a.token_slot = reinterpret_cast<int32_t*>(b + L.slot);
+  a.row_src = reinterpret_cast<int32_t*>(b + L.row_src);
+  a.xp = b + L.xp;
+  a.h = b + L.h;
+  a.y = b + L.y;
+  if (aux) *aux = a;
+  st = moe_route_topk(cfg, logits, a.topk_idx, a.topk_w, a.expert_counts, a.overflow,
+                      a.expert_offsets, a.segment_offsets, a.token_slot, a.row_src, a.totals, ws,
+                      ws_bytes, stream);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  st = moe_dispatch(cfg, x, a.token_slot, a.xp, stream);
+  if (st != MOE_OK) return st;
+  st = moe_expert_mlp(cfg, a.xp, a.expert_offsets, a.expert_counts, w_gu, w_d, a.h, a.y, ws,
+                      ws_bytes, stream);
+  if (st != MOE_OK) return st;
+  return moe_combine(cfg, a.y, a.token_slot, a.topk_w, out, stream);
+}
+
+moe_status_t moe_get_device_status(void* ws, moe_status_t* status, void* stream) {
+  if (!ws || !status) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, ws, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  *status = static_cast<moe_status_t>(v);
+  if (cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,64 @@
+// Internal declarations shared by the CUDA sources of libmoe.so.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// Tokens handled by one block of the route kernel. The per-block expert
+// bitmap has ROUTE_TB/32 words per expert.
+constexpr int ROUTE_TB = 128;
+constexpr int ROUTE_THREADS = 256;
+constexpr int MAX_E = 1024;
+constexpr int MAX_K = 32;
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline int act_size(int32_t act) { return act == MOE_F32 ? 4 : 2; }
+
+// Byte offsets of every region in a workspace. The first 256 bytes hold the
+// status word (uint32 at offset 0).
+struct WsLayout {
+  size_t status = 0;
+  size_t blk_cnt = 0;      // [nblk, E] int32: per-block histograms, then bases
+  size_t route_end = 0;    // bytes needed by moe_route_topk
+  size_t topk_idx = 0, topk_w = 0, counts = 0, overflow = 0, offsets = 0;
+  size_t segoff = 0, totals = 0, slot = 0, row_src = 0;
+  size_t xp = 0, h = 0, y = 0;
+  size_t total = 0;        // bytes needed by moe_layer_forward
+};
+
+WsLayout ws_layout(const moe_config_t& c);
+int64_t max_rows(const moe_config_t& c);
+moe_status_t validate(const moe_config_t* c, bool need_mlp);
+
+// ---- launchers (return cudaGetLastError() of their launches) ----
+cudaError_t launch_route(const moe_config_t& c, const float* logits, int32_t* topk_idx,
+                         float* topk_w, int32_t* counts, int32_t* overflow, int32_t* offsets,
+                         int32_t* segoff, int32_t* slot, int32_t* row_src, int32_t* totals,
+                         int32_t* blk_cnt, int64_t R_max, cudaStream_t s);
+
+cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t* slot, void* xp,
+                            cudaStream_t s);
+
+cudaError_t launch_combine(const moe_config_t& c, const void* y, const int32_t* slot,
+                           const float* w, void* out, cudaStream_t s);
+
+// fp32 CUDA-core grouped SwiGLU (gate/up then down).
+cudaError_t launch_mlp_f32(const moe_config_t& c, const float* xp, const int32_t* offsets,
+                           const int32_t* counts, const float* w_gu, const float* w_d, float* h,
+                           float* y, int64_t R_max, cudaStream_t s);
+
+// bf16 tcgen05 grouped SwiGLU (gate/up then down). Returns a moe status.
+moe_status_t launch_mlp_bf16_tc(const moe_config_t& c, const void* xp, const int32_t* offsets,
+                                const int32_t* counts, const void* w_gu, const void* w_d,
+                                void* h, void* y, int64_t R_max, uint32_t* status,
+                                cudaStream_t s);
+
+}  // namespace moe

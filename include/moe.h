@@ -1,0 +1,201 @@
+/*
+ * moe.h -- C ABI of libmoe.so: the single-GPU MoE expert layer on B200 (sm_100a).
+ *
+ *   route (top-K + softmax weights, histogram, capacity/overflow, owner-aligned
+ *   offsets, permutation) -> dispatch -> grouped SwiGLU expert MLP -> combine
+ *
+ * The operations follow the pages this library is built from:
+ *   - "Efficient and portable Mixture-of-Experts communication" (pplx-kernels):
+ *     "Introductie" (router distribution, top-K, weighted average of expert
+ *     outputs), "Dispatch" (pack tokens per expert, record the return address),
+ *     "Combine" (gather 16-bit expert outputs, weighted average at the receiver).
+ *   - "Enabling trillion-parameter models on AWS EFA": "Диспетчеризация и
+ *     комбинирование" (count tokens per expert with shared-memory atomics in a
+ *     block, cumulative sum -> offsets, pack contiguously), "MoE all-to-all через
+ *     EFA" (grouped GEMM between dispatch and combine).
+ *   - "MoE Expert Parallel Benchmark", Step 2: overflow = max(assigned - capacity, 0),
+ *     effective tokens = sum(assigned - overflow).
+ *   - "Mixture-of-Experts acceleration through overlap": remote-owner-aligned
+ *     layout (each tile belongs to exactly one owner segment).
+ *
+ * Conventions for every entry point
+ *   - Pointers named as device buffers are CUDA device pointers to row-major,
+ *     contiguous data on the current device. The caller owns and allocates all
+ *     of them; the library never allocates or frees device memory and keeps no
+ *     per-call state on the host.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream). Every call is asynchronous on that stream and never synchronises
+ *     the host, except moe_get_device_status.
+ *   - The return value reports argument, configuration, workspace and launch
+ *     errors, detected before or at launch. Errors found by a kernel while it
+ *     runs (a bounded wait that gave up, an expert id out of range in a
+ *     caller-supplied table) are recorded in the workspace's status word and
+ *     read with moe_get_device_status.
+ *   - Shapes the kernels do not support return MOE_ERR_UNSUPPORTED; nothing is
+ *     ever computed another way.
+ *
+ * Symbols: T tokens, H hidden size, E experts, K experts per token, F SwiGLU
+ * width, S owner segments, C capacity per expert, A row alignment, R_max rows
+ * of the dispatch buffer (moe_max_rows).
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* null pointer, negative size, inconsistent config */
+  MOE_ERR_UNSUPPORTED = 2,   /* valid config the kernels do not implement */
+  MOE_ERR_WORKSPACE = 3,     /* workspace missing, misaligned or too small */
+  MOE_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+  MOE_ERR_TIMEOUT = 5,       /* device status: a bounded wait in a kernel gave up */
+  MOE_ERR_DEVICE_INPUT = 6   /* device status: a caller table held an out-of-range id */
+} moe_status_t;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
+
+/* Layer configuration. Limits: T >= 0; H >= 1; 1 <= E <= 1024; 1 <= K <= min(E, 32);
+ * F >= 1; S >= 1 and E % S == 0 (owner segment s holds experts [s*E/S, (s+1)*E/S));
+ * capacity >= 0 (the per-expert limit C, see moe_capacity); 1 <= row_align <= 1024
+ * (every expert's rows start at a multiple of A inside the dispatch buffer);
+ * act_dtype is the dtype of x, the weights, xp, h, y and out.
+ * Rows must be 16-byte multiples: H*sizeof(act) % 16 == 0, F*sizeof(act) % 16 == 0.
+ * The bf16 expert MLP (tensor cores) also needs H % 64 == 0 and F % 64 == 0. */
+typedef struct {
+  int32_t T, H, E, K, F, S;
+  int32_t capacity;
+  int32_t row_align;
+  int32_t act_dtype;
+} moe_config_t;
+
+/* Pointers into the workspace where moe_layer_forward keeps the intermediates.
+ * Filled by moe_layer_forward (host-side writes only) so that a caller can read
+ * the route outputs, the dispatch buffer and the expert outputs afterwards. */
+typedef struct {
+  int32_t *topk_idx, *expert_counts, *overflow, *expert_offsets, *segment_offsets;
+  int32_t *token_slot, *row_src, *totals;
+  float *topk_w;
+  void *xp, *h, *y;
+} moe_layer_aux_t;
+
+#define MOE_FLAG_NONE 0u
+
+/* C = ceil(cf * T * K / E), computed in double precision; cf < 0 means no limit
+ * and returns T (a token picks an expert at most once). Returns -1 if T < 0,
+ * K < 1 or E < 1. ("MoE Expert Parallel Benchmark", Step 2, fixes capacity as the
+ * per-expert, per-step limit; the capacity-factor formula is this library's
+ * reading.) */
+int32_t moe_capacity(int32_t T, int32_t K, int32_t E, double cf);
+
+/* R_max = min(T*K, E*C) + E*(A-1): rows of the dispatch buffer xp (and of h, y
+ * and row_src). Every kept assignment gets one row and each expert adds at most
+ * A-1 rows of alignment padding (a fixed worst-case bound, as the pplx-kernels
+ * page sizes its receive buffers, "Draagbare kernels"). Returns -1 for an
+ * invalid config. */
+int64_t moe_max_rows(const moe_config_t* cfg);
+
+/* MOE_OK if cfg is valid and supported, else the status moe_layer_forward
+ * would return for it. */
+moe_status_t moe_check_config(const moe_config_t* cfg);
+
+/* Bytes of workspace needed by moe_route_topk (per-block histograms and the
+ * status word). */
+size_t moe_route_workspace_bytes(const moe_config_t* cfg);
+
+/* Bytes of workspace needed by moe_layer_forward: the route workspace plus
+ * every intermediate (route outputs, xp, h, y), each 256-byte aligned. */
+size_t moe_workspace_bytes(const moe_config_t* cfg, uint32_t flags);
+
+/* Zero the workspace's status word (and nothing else). Call once after
+ * allocating a workspace; asynchronous on `stream`. */
+moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Route: steps "top-K + weights", "histogram + capacity + overflow" and
+ * "owner-aligned offsets + permutation".
+ *   logits          [T,E] fp32, device, read only. Any bias is already added.
+ *   topk_idx        [T,K] int32 out: experts by (logit descending, index ascending).
+ *   topk_w          [T,K] fp32 out: softmax over the K selected logits.
+ *   expert_counts   [E]   int32 out: assignments per expert (the histogram).
+ *   overflow        [E]   int32 out: max(count - C, 0).
+ *   expert_offsets  [E+1] int32 out: off[0]=0, off[e+1]=off[e]+roundup(min(count,C), A).
+ *   segment_offsets [S+1] int32 out: off[s*E/S].
+ *   token_slot      [T,K] int32 out: row of (t,k) in xp, or -1 if it overflowed.
+ *                   The first C assignments of each expert in token order are kept.
+ *   row_src         [R_max] int32 out: t*K+k for each kept row, -1 on padding rows.
+ *   totals          [4]   int32 out: {T*K, effective N, total overflow, R = off[E]}.
+ *   ws, ws_bytes    workspace of at least moe_route_workspace_bytes(cfg) bytes,
+ *                   256-byte aligned; contents need not be initialised except the
+ *                   status word (moe_workspace_init).
+ * All outputs are written in full; the results are deterministic. */
+moe_status_t moe_route_topk(const moe_config_t* cfg, const float* logits,
+                            int32_t* topk_idx, float* topk_w, int32_t* expert_counts,
+                            int32_t* overflow, int32_t* expert_offsets,
+                            int32_t* segment_offsets, int32_t* token_slot,
+                            int32_t* row_src, int32_t* totals,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* Dispatch ("Dispatch" of the pplx-kernels page): xp[token_slot[t,k]] = x[t],
+ * a bit copy, for every (t,k) with token_slot >= 0.
+ *   x          [T,H] act, device, read only.
+ *   token_slot [T,K] int32 from moe_route_topk.
+ *   xp         [R_max,H] act out; rows no slot points at are not written. */
+moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* token_slot,
+                          void* xp, void* stream);
+
+/* Grouped SwiGLU expert MLP. For every expert e and every row r in
+ * [off_e, off_e + min(count_e, C)):
+ *   h[r] = silu(xp[r] Wg_e^T) * (xp[r] Wu_e^T)   (fp32 accumulate, rounded to act)
+ *   y[r] = h[r] W_d,e^T                          (fp32 accumulate, rounded to act)
+ *   xp             [R_max,H] act.
+ *   expert_offsets [E+1] int32, expert_counts [E] int32 (raw counts; the kept
+ *                  count min(count, C) is derived on the device).
+ *   w_gu           [E,2F,H] act: rows 0..F-1 are Wg_e, rows F..2F-1 are Wu_e.
+ *   w_d            [E,H,F] act.
+ *   h              [R_max,F] act out (scratch for the second GEMM), y [R_max,H] act out.
+ *   Rows outside every expert's kept range are not written.
+ *   ws, ws_bytes   any workspace with a status word (at least 256 bytes).
+ * bf16 runs on tcgen05 tensor cores (TMA-fed persistent grouped GEMM); fp32 runs
+ * on a CUDA-core FFMA grouped GEMM (fp32 inputs, no TF32). */
+moe_status_t moe_expert_mlp(const moe_config_t* cfg, const void* xp,
+                            const int32_t* expert_offsets, const int32_t* expert_counts,
+                            const void* w_gu, const void* w_d, void* h, void* y,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* Combine ("Combine" of the pplx-kernels page): out[t] = sum over k in order of
+ * topk_w[t,k] * y[token_slot[t,k]] for slots >= 0, fp32 accumulation, rounded
+ * once to act. Dropped assignments contribute zero (no renormalisation); a token
+ * with every assignment dropped gets zeros.
+ *   y [R_max,H] act, token_slot [T,K] int32, topk_w [T,K] fp32, out [T,H] act. */
+moe_status_t moe_combine(const moe_config_t* cfg, const void* y, const int32_t* token_slot,
+                         const float* topk_w, void* out, void* stream);
+
+/* The whole layer on `stream`: route -> dispatch -> expert MLP -> combine, with
+ * every intermediate in the workspace (moe_workspace_bytes). `aux` may be NULL;
+ * otherwise it receives the workspace pointers of the intermediates. No host
+ * synchronisation: the per-expert counts stay on the device. */
+moe_status_t moe_layer_forward(const moe_config_t* cfg, const float* logits, const void* x,
+                               const void* w_gu, const void* w_d, void* out,
+                               uint32_t flags, void* ws, size_t ws_bytes,
+                               moe_layer_aux_t* aux, void* stream);
+
+/* Synchronise `stream`, read the workspace's status word into *status and reset
+ * it to MOE_OK. Returns MOE_ERR_CUDA if the synchronisation or copy failed. */
+moe_status_t moe_get_device_status(void* ws, moe_status_t* status, void* stream);
+
+/* Static text for a status code. */
+const char* moe_status_string(moe_status_t status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int32_t moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */

@@ -1,0 +1,122 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every symbol include/moe.h declares, and its host-only functions (capacity,
+sizes, validation, status strings) behave as documented."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import combine_moe_route_13_b200 as M
+from oracle import moe_oracle as O
+import workloads as W
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "moe.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert len(names) >= 14
+    lib = ctypes.CDLL(M.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(M.EXPORTS) == names
+
+
+def test_version():
+    assert M.moe_version() == 10000
+
+
+@pytest.mark.parametrize("name", list(W.WORKLOADS))
+def test_capacity_matches_oracle(name):
+    w = W.WORKLOADS[name]
+    assert M.moe_capacity(w.T, w.K, w.E, w.cf) == O.capacity(w.T, w.K, w.E, w.cf)
+
+
+def test_capacity_edge_cases():
+    assert M.moe_capacity(10, 3, 4, 1.0) == 8
+    assert M.moe_capacity(10, 3, 4, -1.0) == 10
+    assert M.moe_capacity(0, 3, 4, 1.0) == 0
+    assert M.moe_capacity(-1, 3, 4, 1.0) == -1
+    assert M.moe_capacity(10, 0, 4, 1.0) == -1
+
+
+def cfg_of(w, **kw):
+    C = O.capacity(w.T, w.K, w.E, w.cf)
+    d = dict(T=w.T, H=w.H, E=w.E, K=w.K, F=w.F, S=w.S, capacity=C, row_align=w.row_align, act=w.act)
+    d.update(kw)
+    return M.make_config(**d)
+
+
+@pytest.mark.parametrize("name", list(W.WORKLOADS))
+def test_sizes_match_oracle(name):
+    w = W.WORKLOADS[name]
+    cfg = cfg_of(w)
+    C = cfg.capacity
+    assert M.moe_max_rows(cfg) == O.max_rows(w.T, w.K, w.E, C, w.row_align)
+    assert M.moe_check_config(cfg) == M.MOE_OK
+    R = M.moe_max_rows(cfg)
+    s = 4 if w.act == "f32" else 2
+    need = R * (2 * w.H + w.F) * s
+    assert M.moe_workspace_bytes(cfg) >= need
+    assert 256 < M.moe_route_workspace_bytes(cfg) < M.moe_workspace_bytes(cfg)
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("K", 0, M.MOE_ERR_INVALID_ARG), ("K", 9, M.MOE_ERR_INVALID_ARG),      # K > E
+    ("S", 3, M.MOE_ERR_INVALID_ARG),                                       # E % S != 0
+    ("capacity", -1, M.MOE_ERR_INVALID_ARG), ("row_align", 0, M.MOE_ERR_INVALID_ARG),
+    ("T", -5, M.MOE_ERR_INVALID_ARG), ("act_dtype", 7, M.MOE_ERR_INVALID_ARG),
+    ("H", 4100, M.MOE_ERR_UNSUPPORTED),                                    # bf16 GEMM needs H % 64
+    ("F", 100, M.MOE_ERR_UNSUPPORTED), ("row_align", 4096, M.MOE_ERR_UNSUPPORTED),
+])
+def test_invalid_configs_are_rejected(field, value, code):
+    cfg = cfg_of(W.WORKLOADS["mixtral"])
+    setattr(cfg, field, value)
+    assert M.moe_check_config(cfg) == code
+
+
+def test_too_many_experts_unsupported():
+    cfg = M.make_config(T=16, H=64, E=2048, K=2, F=64, S=1, capacity=4)
+    assert M.moe_check_config(cfg) == M.MOE_ERR_UNSUPPORTED
+    cfg = M.make_config(T=16, H=64, E=64, K=33, F=64, S=1, capacity=4)
+    assert M.moe_check_config(cfg) == M.MOE_ERR_UNSUPPORTED
+
+
+def test_entry_points_reject_bad_arguments_before_any_launch():
+    lib = M.LIB
+    cfg = cfg_of(W.WORKLOADS["tiny"])
+    nul = None
+    # null config
+    assert lib.moe_dispatch(None, nul, nul, nul, nul) == M.MOE_ERR_INVALID_ARG
+    # null buffers
+    assert lib.moe_dispatch(ctypes.byref(cfg), nul, nul, nul, nul) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine(ctypes.byref(cfg), nul, nul, nul, nul, nul) == M.MOE_ERR_INVALID_ARG
+    # a missing or misaligned workspace
+    fake = ctypes.c_void_p(0x10000)
+    args = [ctypes.byref(cfg)] + [fake] * 10 + [None, 0, None]
+    assert lib.moe_route_topk(*args) == M.MOE_ERR_WORKSPACE
+    args = [ctypes.byref(cfg)] + [fake] * 10 + [ctypes.c_void_p(0x10010), 1 << 30, None]
+    assert lib.moe_route_topk(*args) == M.MOE_ERR_WORKSPACE
+    small = M.moe_route_workspace_bytes(cfg) - 256
+    args = [ctypes.byref(cfg)] + [fake] * 10 + [fake, small, None]
+    assert lib.moe_route_topk(*args) == M.MOE_ERR_WORKSPACE
+    # layer: flags that are not defined
+    assert lib.moe_layer_forward(ctypes.byref(cfg), fake, fake, fake, fake, fake, 7, fake,
+                                 1 << 40, None, None) == M.MOE_ERR_UNSUPPORTED
+    assert lib.moe_workspace_init(None, 0, None) == M.MOE_ERR_WORKSPACE
+    st = ctypes.c_int(0)
+    assert lib.moe_get_device_status(None, ctypes.byref(st), None) == M.MOE_ERR_INVALID_ARG
+
+
+def test_status_strings():
+    for code in range(7):
+        s = M.status_string(code)
+        assert s and s != "unknown status"
+    assert M.status_string(99) == "unknown status"

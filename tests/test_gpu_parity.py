@@ -1,0 +1,246 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Integer outputs (routing indices, counts, overflow, offsets, the permutation,
+the dispatched rows) must match bit for bit; router weights within 2e-6
+relative; expert MLP and combine outputs within max|err| <= 1e-2 * rms(ref)
+for bf16 and max|err| <= 1e-5 * max|ref| for fp32.
+"""
+import numpy as np
+import pytest
+import torch
+
+import combine_moe_route_13_b200 as M
+from oracle import moe_oracle as O
+import workloads as W
+from _gpu_common import (act_np, assert_close_act, assert_route_equal, cfg_for, host,
+                         run_route)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def logits_for(T, E, kind, seed):
+    g = torch.Generator().manual_seed(seed)
+    if kind == "tied":
+        return W.tied_logits(T, E, 3, g)
+    lg = torch.randn(T, E, generator=g)
+    if kind == "zipf":
+        lg += 2.0 * torch.log(torch.arange(1, E + 1, dtype=torch.float64) ** -1.2).float()
+    if kind == "bias":
+        lg += torch.randn(E, generator=g) * 0.1
+    if kind == "hot":
+        lg[:, 0] += 2.0
+    return lg
+
+
+ROUTE_CASES = [
+    # T, E, K, S, cf, A, logits
+    (64, 8, 2, 2, 1.25, 1, "normal"),
+    (300, 8, 2, 8, 1.25, 128, "normal"),
+    (1000, 17, 5, 1, 0.7, 4, "normal"),
+    (1024, 256, 8, 8, 1.5, 128, "bias"),
+    (4097, 64, 6, 8, 1.0, 128, "zipf"),
+    (513, 384, 8, 16, 1.25, 128, "normal"),
+    (200, 1024, 32, 4, 2.0, 8, "normal"),
+    (256, 32, 32, 4, 1.0, 1, "normal"),
+    (300, 12, 3, 3, 1.0, 1, "tied"),
+    (128, 8, 2, 2, 0.0, 1, "normal"),
+    (100, 8, 1, 1, -1.0, 1, "normal"),
+    (0, 8, 2, 2, 1.0, 4, "normal"),
+    (5000, 1, 1, 1, 1.0, 128, "normal"),
+    (777, 40, 4, 5, 0.9, 32, "hot"),
+]
+
+
+@pytest.mark.parametrize("T,E,K,S,cf,A,kind", ROUTE_CASES)
+def test_route_bit_exact(cuda_ok, T, E, K, S, cf, A, kind):
+    C = O.capacity(T, K, E, cf)
+    lg = logits_for(T, E, kind, T * 7 + E)
+    cfg = cfg_for(T, 64, E, K, 64, S, C, A, "bf16")
+    gpu = host(run_route(cfg, lg.to(DEV)))
+    ref = O.route(lg.numpy(), K, C, A, S)
+    assert_route_equal(gpu, ref, ref["R_max"])
+
+
+def test_route_is_deterministic(cuda_ok):
+    T, E, K, S, A = 4096, 64, 6, 8, 128
+    lg = logits_for(T, E, "zipf", 3).to(DEV)
+    cfg = cfg_for(T, 64, E, K, 64, S, O.capacity(T, K, E, 1.0), A, "bf16")
+    a, b = host(run_route(cfg, lg)), host(run_route(cfg, lg))
+    for k in a:
+        assert np.array_equal(a[k], b[k]), k
+
+
+@pytest.mark.parametrize("act", ["bf16", "f32"])
+@pytest.mark.parametrize("T,H,E,K,S,cf,A", [
+    (300, 256, 8, 2, 2, 1.0, 128), (1000, 128, 17, 5, 1, 0.7, 4), (64, 7168, 4, 2, 2, 1.0, 1)])
+def test_dispatch_bit_exact(cuda_ok, act, T, H, E, K, S, cf, A):
+    C = O.capacity(T, K, E, cf)
+    lg = logits_for(T, E, "hot", 11)
+    cfg = cfg_for(T, H, E, K, 64, S, C, A, act)
+    r = run_route(cfg, lg.to(DEV))
+    dt = torch.float32 if act == "f32" else torch.bfloat16
+    x = torch.randn(T, H, generator=torch.Generator().manual_seed(5)).to(dt).to(DEV)
+    R = M.moe_max_rows(cfg)
+    xp = torch.full((R, H), 7, dtype=x.dtype, device=DEV)    # sentinel in unwritten rows
+    M.moe_dispatch(cfg, x, r["token_slot"], xp)
+    torch.cuda.synchronize()
+    ref = O.dispatch(act_np(x), r["token_slot"].cpu().numpy(), R)
+    rs = r["row_src"].cpu().numpy()[:R]
+    kept = rs >= 0
+    assert np.array_equal(act_np(xp)[kept], ref[kept])
+    # rows no slot points at are left untouched
+    untouched = act_np(xp)[~kept]
+    sentinel = act_np(torch.full((1, H), 7, dtype=x.dtype))
+    assert np.all(untouched == sentinel)
+
+
+@pytest.mark.parametrize("act,K", [("bf16", 1), ("bf16", 2), ("bf16", 4), ("bf16", 8),
+                                   ("f32", 1), ("f32", 2)])
+def test_round_trip_identity_experts_bit_exact(cuda_ok, act, K):
+    # y := xp (identity experts), weights summing to 1 in binary (K = 1, or equal
+    # logits so that w = 1/K), no drops: combine(dispatch(x)) == x bit for bit.
+    # Exact only while every partial sum k*x/K is exact in the fp32 accumulator:
+    # any K <= 32 for bf16 rows (8 significant bits), K <= 2 for fp32 rows.
+    T, H, E, S = 513, 512, 8, 2
+    g = torch.Generator().manual_seed(2)
+    lg = torch.randn(T, E, generator=g) - 10.0
+    for t in range(T):   # K experts per token share the largest logit
+        lg[t, torch.randperm(E, generator=g)[:K]] = 1.0
+    cfg = cfg_for(T, H, E, K, 64, S, T, 8, act)
+    r = run_route(cfg, lg.to(DEV))
+    w = r["topk_w"].cpu()
+    assert torch.all(w == 1.0 / K)
+    dt = torch.float32 if act == "f32" else torch.bfloat16
+    x = torch.randn(T, H, generator=torch.Generator().manual_seed(3)).to(dt).to(DEV)
+    xp = torch.zeros(M.moe_max_rows(cfg), H, dtype=dt, device=DEV)
+    out = torch.empty_like(x)
+    M.moe_dispatch(cfg, x, r["token_slot"], xp)
+    M.moe_combine(cfg, xp, r["token_slot"], r["topk_w"], out)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16) if dt == torch.bfloat16 else out.view(torch.int32),
+                       x.view(torch.int16) if dt == torch.bfloat16 else x.view(torch.int32))
+
+
+@pytest.mark.parametrize("act", ["bf16", "f32"])
+@pytest.mark.parametrize("T,H,E,K,cf", [(300, 256, 8, 2, 1.0), (777, 1024, 40, 6, 0.8),
+                                        (50, 7168, 384, 8, 1.25), (64, 128, 8, 2, 0.0)])
+def test_combine_matches_explicit_weighted_sum(cuda_ok, act, T, H, E, K, cf):
+    C = O.capacity(T, K, E, cf)
+    lg = logits_for(T, E, "hot", 13)
+    cfg = cfg_for(T, H, E, K, 64, 1, C, 16, act)
+    r = run_route(cfg, lg.to(DEV))
+    R = M.moe_max_rows(cfg)
+    dt = torch.float32 if act == "f32" else torch.bfloat16
+    y = torch.randn(max(R, 1), H, generator=torch.Generator().manual_seed(4)).to(dt).to(DEV)
+    out = torch.empty(T, H, dtype=dt, device=DEV)
+    M.moe_combine(cfg, y, r["token_slot"], r["topk_w"], out)
+    torch.cuda.synchronize()
+    ref = O.combine(act_np(y), r["token_slot"].cpu().numpy(), r["topk_w"].cpu().numpy(), act)
+    assert_close_act(act_np(out), ref, act, "combine")
+    if C == 0:
+        assert torch.all(out == 0)
+
+
+MLP_CASES = [
+    # T, H, E, K, F, S, cf, A, logits
+    (256, 256, 4, 2, 256, 2, 1.25, 128, "normal"),
+    (300, 320, 6, 2, 192, 3, 1.0, 1, "normal"),        # N tails, tiles straddling experts
+    (1000, 512, 16, 4, 128, 4, 0.5, 128, "hot"),       # overflow
+    (130, 128, 2, 1, 64, 1, -1.0, 8, "normal"),
+    (600, 256, 8, 2, 384, 8, 2.0, 128, "zipf"),        # empty experts
+    (128, 64, 64, 8, 64, 8, 2.0, 16, "normal"),        # many tiny experts
+    (1200, 1024, 8, 2, 1024, 2, 1.25, 128, "normal"),  # several M and N tiles per expert
+]
+
+
+def _run_mlp(T, H, E, K, F, S, cf, A, kind, act):
+    C = O.capacity(T, K, E, cf)
+    lg = logits_for(T, E, kind, T + H + F)
+    cfg = cfg_for(T, H, E, K, F, S, C, A, act)
+    wl = W.small_case(T, H, E, K, F, S, cf, act, A)
+    inp = W.make_inputs(wl, seed=T + E, device=DEV)
+    r = run_route(cfg, lg.to(DEV))
+    R = M.moe_max_rows(cfg)
+    dt = wl.torch_act
+    xp = torch.zeros(R, H, dtype=dt, device=DEV)
+    h = torch.zeros(R, F, dtype=dt, device=DEV)
+    y = torch.zeros(R, H, dtype=dt, device=DEV)
+    ws = M.alloc_workspace(256)
+    M.moe_dispatch(cfg, inp["x"], r["token_slot"], xp)
+    M.moe_expert_mlp(cfg, xp, r["expert_offsets"], r["expert_counts"], inp["w_gu"], inp["w_d"],
+                     h, y, ws)
+    assert M.moe_get_device_status(ws) == M.MOE_OK
+    return cfg, r, inp, xp, h, y
+
+
+@pytest.mark.parametrize("T,H,E,K,F,S,cf,A,kind", MLP_CASES)
+def test_expert_mlp_bf16(cuda_ok, T, H, E, K, F, S, cf, A, kind):
+    cfg, r, inp, xp, h, y = _run_mlp(T, H, E, K, F, S, cf, A, kind, "bf16")
+    off = r["expert_offsets"].cpu().numpy()
+    kept = np.minimum(r["expert_counts"].cpu().numpy(), cfg.capacity)
+    xp_n, h_n, y_n = act_np(xp), act_np(h), act_np(y)
+    w_gu, w_d = act_np(inp["w_gu"]), act_np(inp["w_d"])
+    rows = np.concatenate([np.arange(off[e], off[e] + kept[e]) for e in range(E)] + [np.zeros(0, int)])
+    ref_h = np.zeros((len(rows), F), np.uint16)
+    ref_y = np.zeros((len(rows), H), np.uint16)
+    p = 0
+    for e in range(E):
+        n = int(kept[e])
+        if n:
+            he, ye = O.expert_mlp_rows(xp_n[off[e]:off[e] + n], w_gu[e], w_d[e], O.ACT_BF16)
+            ref_h[p:p + n], ref_y[p:p + n] = he, ye
+            p += n
+    assert_close_act(h_n[rows], ref_h, O.ACT_BF16, "h")
+    assert_close_act(y_n[rows], ref_y, O.ACT_BF16, "y")
+
+
+def test_expert_mlp_f32_tiny(cuda_ok):
+    w = W.WORKLOADS["tiny"]
+    cfg, r, inp, xp, h, y = _run_mlp(w.T, w.H, w.E, w.K, w.F, w.S, w.cf, 1, "normal", "f32")
+    ref_h, ref_y = O.expert_mlp(act_np(xp), r["expert_offsets"].cpu().numpy(),
+                                np.minimum(r["expert_counts"].cpu().numpy(), cfg.capacity),
+                                act_np(inp["w_gu"]), act_np(inp["w_d"]), O.ACT_F32)
+    rs = r["row_src"].cpu().numpy()[:M.moe_max_rows(cfg)]
+    kept = rs >= 0
+    assert_close_act(act_np(h)[kept], ref_h[kept], O.ACT_F32, "h")
+    assert_close_act(act_np(y)[kept], ref_y[kept], O.ACT_F32, "y")
+
+
+def _layer(wl, C, seed=0):
+    inp = W.make_inputs(wl, seed=seed, device=DEV)
+    cfg = cfg_for(wl.T, wl.H, wl.E, wl.K, wl.F, wl.S, C, wl.row_align, wl.act)
+    ws = M.alloc_workspace(M.moe_workspace_bytes(cfg))
+    out = torch.empty(wl.T, wl.H, dtype=wl.torch_act, device=DEV)
+    aux = M.moe_layer_forward(cfg, inp["logits"], inp["x"], inp["w_gu"], inp["w_d"], out, ws)
+    assert M.moe_get_device_status(ws) == M.MOE_OK
+    return cfg, inp, out, M.layer_views(cfg, ws, aux)
+
+
+@pytest.mark.parametrize("wl", [
+    W.WORKLOADS["tiny"],
+    W.small_case(512, 256, 8, 2, 256, 2, 1.25, "bf16", 128),
+    W.small_case(700, 384, 12, 3, 192, 4, 0.8, "bf16", 1, bias="zipf1.2"),
+    W.small_case(300, 128, 16, 4, 128, 8, 1.0, "f32", 4),
+], ids=lambda w: w.name)
+def test_layer_forward_end_to_end(cuda_ok, wl):
+    C = O.capacity(wl.T, wl.K, wl.E, wl.cf)
+    cfg, inp, out, v = _layer(wl, C)
+    ref_out, ref = O.layer_forward(inp["logits"].cpu().numpy(), act_np(inp["x"]),
+                                   act_np(inp["w_gu"]), act_np(inp["w_d"]), wl.K, C,
+                                   wl.row_align, wl.S, wl.act)
+    assert_route_equal(host({k: v[k] for k in ("topk_idx", "topk_w", "expert_counts", "overflow",
+                                                "expert_offsets", "segment_offsets", "token_slot",
+                                                "row_src", "totals")}), ref, ref["R_max"])
+    kept = ref["row_src"] >= 0
+    assert np.array_equal(act_np(v["xp"])[kept], ref["xp"][kept])
+    assert_close_act(act_np(v["y"])[kept], ref["y"][kept], wl.act, "y")
+    assert_close_act(act_np(out), ref_out, wl.act, "out")
+
+
+def test_empty_batch(cuda_ok):
+    wl = W.small_case(0, 128, 8, 2, 128, 2, 1.0, "bf16", 128)
+    cfg, inp, out, v = _layer(wl, 0)
+    assert v["totals"].cpu().tolist() == [0, 0, 0, 0]
+    assert torch.all(v["expert_counts"] == 0)
+    assert torch.all(v["row_src"] == -1)
