@@ -63,7 +63,7 @@ _CFG = ctypes.POINTER(MoeConfig)
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"libmoe.so is not built ({LIB_PATH}); run "
-                          "`python -m combine_moe_route_13_b200.build`")
+                          "`python combine_moe_route_13_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     sig = {
         "moe_capacity": (ctypes.c_int32, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_double]),

@@ -1,6 +1,9 @@
 """Build libmoe.so in-tree with nvcc for sm_100a.
 
-    python -m combine_moe_route_13_b200.build [--force] [--verbose]
+    python combine_moe_route_13_b200/build.py [--force] [--verbose] [--ptxas-info]
+
+(run as a script: importing the package loads the library, which may not
+exist yet)
 
 The library is written next to this file so that it travels with the source
 tree. Rebuilds only when a source or header is newer than the library.
