@@ -31,7 +31,7 @@ MOE_FLAG_NONE = 0
 EXPORTS = ("moe_capacity", "moe_max_rows", "moe_check_config", "moe_route_workspace_bytes",
            "moe_workspace_bytes", "moe_workspace_init", "moe_route_topk", "moe_dispatch",
            "moe_expert_mlp", "moe_combine", "moe_layer_forward", "moe_get_device_status",
-           "moe_status_string", "moe_version")
+           "moe_status_string", "moe_version", "moe_route_topk_noalloc")
 
 
 class MoeError(RuntimeError):
@@ -81,6 +81,7 @@ def _load():
         "moe_get_device_status": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int), _P]),
         "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "moe_version": (ctypes.c_int32, []),
+        "moe_route_topk_noalloc": (ctypes.c_int, [_CFG] + [_P] * 10 + [_P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -167,6 +168,21 @@ def moe_route_topk(cfg, logits, topk_idx, topk_w, expert_counts, overflow, exper
         _ptr(segment_offsets, i32, "segment_offsets"), _ptr(token_slot, i32, "token_slot"),
         _ptr(row_src, i32, "row_src"), _ptr(totals, i32, "totals"), _ptr(ws, name="ws"),
         ws.numel() * ws.element_size(), _stream(stream)), "moe_route_topk")
+
+
+def moe_route_topk_noalloc(cfg, logits, topk_idx, topk_w, expert_counts, overflow,
+                           expert_offsets, segment_offsets, token_slot, row_src, totals,
+                           stream=None):
+    """moe_route_topk without a workspace (for callers that cannot allocate):
+    the scratch is a fixed 1 MiB device array inside the library."""
+    i32 = torch.int32
+    _check(LIB.moe_route_topk_noalloc(
+        ctypes.byref(cfg), _ptr(logits, torch.float32, "logits"), _ptr(topk_idx, i32, "topk_idx"),
+        _ptr(topk_w, torch.float32, "topk_w"), _ptr(expert_counts, i32, "expert_counts"),
+        _ptr(overflow, i32, "overflow"), _ptr(expert_offsets, i32, "expert_offsets"),
+        _ptr(segment_offsets, i32, "segment_offsets"), _ptr(token_slot, i32, "token_slot"),
+        _ptr(row_src, i32, "row_src"), _ptr(totals, i32, "totals"), _stream(stream)),
+        "moe_route_topk_noalloc")
 
 
 def moe_dispatch(cfg, x, token_slot, xp, stream=None):

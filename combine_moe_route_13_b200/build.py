@@ -20,7 +20,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmoe.so")
-SOURCES = ["moe_abi.cu", "route.cu", "dispatch_combine.cu", "gemm_simt.cu", "gemm_tc.cu"]
+SOURCES = ["moe_abi.cu", "route.cu", "dispatch_combine.cu", "gemm_simt.cu", "gemm_tc.cu",
+           "route_noalloc.cu"]
 HEADERS = [os.path.join(CSRC, "moe_internal.h"), os.path.join(ROOT, "include", "moe.h")]
 GENCODE = "arch=compute_100a,code=sm_100a"
 

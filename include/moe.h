@@ -140,6 +140,36 @@ moe_status_t moe_route_topk(const moe_config_t* cfg, const float* logits,
                             int32_t* row_src, int32_t* totals,
                             void* ws, size_t ws_bytes, void* stream);
 
+/* Bytes of the fixed device scratch area used by moe_route_topk_noalloc. */
+#define MOE_NOALLOC_SCRATCH_BYTES (1u << 20)
+
+/* moe_route_topk for callers that cannot allocate device memory (no counterpart
+ * on the pages; an addition of this library).
+ * Some callers cannot call cudaMalloc or hand out a workspace: code that runs
+ * inside another framework's allocator, plug-ins that receive only their input
+ * and output buffers, or code paths where an allocation could fail at a bad
+ * moment. This entry point takes the same arguments as moe_route_topk without
+ * ws/ws_bytes and produces identical results. Its scratch (the per-block expert
+ * histograms, ceil(T/128) * E * 4 bytes) lives in a fixed device array of
+ * MOE_NOALLOC_SCRATCH_BYTES (1 MiB) inside the library, which every GPU that
+ * loads the library holds until the process exits.
+ *   - It calls no cudaMalloc, cudaFree or allocating library routine.
+ *   - Configurations needing more scratch than 1 MiB (ceil(T/128) * E > 262144)
+ *     return MOE_ERR_WORKSPACE and launch nothing.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) and caches it; make that first call before any
+ *     stream capture on that device.
+ *   - Every call shares the one array, which keeps the last call's contents;
+ *     the kernels write every scratch entry before reading it, so nothing needs
+ *     to start at zero. Calls whose kernels overlap on the GPU (different
+ *     streams, or threads without ordering between them) race on the array and
+ *     give wrong results: serialise them. */
+moe_status_t moe_route_topk_noalloc(const moe_config_t* cfg, const float* logits,
+                                    int32_t* topk_idx, float* topk_w, int32_t* expert_counts,
+                                    int32_t* overflow, int32_t* expert_offsets,
+                                    int32_t* segment_offsets, int32_t* token_slot,
+                                    int32_t* row_src, int32_t* totals, void* stream);
+
 /* Dispatch ("Dispatch" of the pplx-kernels page): xp[token_slot[t,k]] = x[t],
  * a bit copy, for every (t,k) with token_slot >= 0.
  *   x          [T,H] act, device, read only.
