@@ -119,6 +119,17 @@ class Clocks:
                 "sm_max_mhz": float(np.nanmax(mx)), "samples": len(rows), "reasons": reasons}
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The maximum of x over all ranks (identity with one rank). The tensor
+    lives on `device`: CUDA under NCCL, CPU under gloo."""
+    if world <= 1:
+        return float(x)
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def flush_l2(buf: torch.Tensor):
     buf.add_(1)
 
@@ -335,21 +346,12 @@ def main(argv=None):
     times = time_steps(layer.forward, args.steps, args.warmup, flush_buf, stream)
     barrier()
     clk = clocks.stop()
-    total_ms = float(np.sum(times))
-    if world > 1:
-        t = torch.tensor([total_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(np.sum(times)), world, device)
     ms = total_ms / args.steps
     value = world * wl.T / (ms / 1e3)
 
     e2e_t, h2d, d2h = e2e_steps(layer, args.steps, args.warmup, flush_buf, stream)
-    e2e_ms = float(np.sum(e2e_t))
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_ms /= args.steps
+    e2e_ms = max_over_ranks(float(np.sum(e2e_t)), world, device) / args.steps
 
     ph = phase_times(layer, max(args.steps // 2, 3), flush_buf, stream)
     st = layer.M.moe_get_device_status(layer.ws)

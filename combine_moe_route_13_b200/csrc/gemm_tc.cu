@@ -5,26 +5,36 @@
 // "Результаты экспериментов": one grouped GEMM instead of many small ones),
 // written as a persistent kernel that walks every expert's tiles without a
 // relaunch (the producer of "Mixture-of-Experts acceleration through
-// overlap"). With the row alignment A = 128 every M tile lies inside one
-// expert, hence inside one owner segment (the remote-owner-aligned layout of
-// the same page); with any other A a tile starts at its expert's first row and
-// rows past the expert's end are computed but never stored.
+// overlap"). With the row alignment A = 128 every 128-row half tile lies inside
+// one expert, hence inside one owner segment (the remote-owner-aligned layout
+// of the same page); with any other A a tile starts at its expert's first row
+// and rows past the expert's end are computed but never stored.
 //
 // Two launches:
 //   MODE 0: [g | u] = xp W_gu[e]^T  (N = 128 gate + 128 up columns, one MMA of
 //           N = 256), epilogue h = silu(g) * u rounded to bf16.
 //   MODE 1: y = h W_d[e]^T (N = 256 columns), epilogue rounds to bf16.
 //
-// Per CTA (one per SM, persistent, static round-robin over tiles):
-//   warp 0     TMA producer: A box [128 rows x 64 k] and two B boxes
-//              [128 rows x 64 k], 128-byte swizzle, into a 4-stage ring.
-//   warp 1     MMA issuer: 4 x tcgen05.mma (M=128, N=256, K=16) per stage,
-//              fp32 accumulators in TMEM, two 256-column buffers so that the
-//              epilogue of one tile overlaps the MMAs of the next.
-//   warps 2-5  epilogue: tcgen05.ld rows from TMEM (each warp owns the 32
-//              TMEM lanes of its sub-partition), SwiGLU / rounding, stores.
-// Tile order: expert-major, then N tile, then M tile, so that the CTAs running
-// at the same time share an expert's rows of xp and each weight slab in L2.
+// CG = 2 (used): a cluster of two CTAs on two SMs shares one
+// tcgen05.mma.cta_group::2 of M = 256, N = 256. Each CTA loads its own 128 rows
+// of A and its own 128 rows (half of N) of B, so a CTA moves 32 KB per k step
+// instead of 48 KB and six stages fit in shared memory. Each CTA's TMEM holds
+// the 128 x 256 fp32 accumulator of its own rows. CG = 1: one CTA, M = 128,
+// both B halves loaded by the CTA, four stages.
+//
+// Roles per CTA (one CTA per SM, persistent, static round-robin over tiles):
+//   warp 0     TMA producer (128-byte swizzled boxes [64 k x 128 rows]);
+//   warp 1     MMA issuer (one thread of the cluster's first CTA) and TMEM
+//              allocation; two 256-column accumulators so that the epilogue
+//              of one tile overlaps the MMAs of the next;
+//   warps 2-5  epilogue: tcgen05.ld of its TMEM sub-partition's 32 lanes,
+//              SwiGLU / rounding, stores.
+// Barriers: the producers of both CTAs signal the leader's "full" barrier;
+// the leader's commits signal "empty" and "TMEM full" in both CTAs; both
+// CTAs' epilogues signal the leader's "TMEM empty".
+// Tile order: expert-major, then N tile, then M tile, so that the clusters
+// running at the same time share an expert's rows of xp and each weight slab
+// in L2.
 //
 // Every wait on an mbarrier is bounded (globaltimer deadline). On expiry the
 // kernel records MOE_ERR_TIMEOUT in the status word, all roles leave their
@@ -42,27 +52,34 @@
 namespace moe {
 namespace tc {
 
-constexpr int BM = 128;                     // tile rows = TMEM lanes
+constexpr int BM = 128;                     // rows per CTA = TMEM lanes
 constexpr int BK = 64;                      // k per stage: one 128-byte swizzle row of bf16
 constexpr int UMMA_N = 256;                 // N of one MMA
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;        // 16 KB
-constexpr int B_HALF_BYTES = 128 * BK * 2;  // 16 KB
-constexpr int STAGE_BYTES = A_BYTES + 2 * B_HALF_BYTES;
+constexpr int BOX_BYTES = 128 * BK * 2;     // one TMA box: 128 rows x 64 k, 16 KB
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr unsigned long long WAIT_NS = 2000000000ull;   // 2 s
 constexpr unsigned long long DRAIN_NS = 200000000ull;   // 0.2 s
 
-// Instruction descriptor of tcgen05.mma.kind::f16: D fp32 (bits 4-5 = 1),
-// A bf16 (bits 7-9 = 1), B bf16 (bits 10-12 = 1), both K-major (bits 15, 16 = 0),
-// N >> 3 at bits 17-22, M >> 4 at bits 24-28.
-constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
-                           ((uint32_t)(UMMA_N >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+template <int CG>
+struct Cfg {
+  static constexpr int B_BOXES = 3 - CG;                    // B boxes loaded per CTA
+  static constexpr int STAGE_BYTES = BOX_BYTES * (1 + B_BOXES);
+  static constexpr int STAGES = CG == 2 ? 6 : 4;
+  static constexpr int TILE_ROWS = BM * CG;                 // rows per tile (per cluster)
+  // Instruction descriptor of tcgen05.mma.kind::f16: D fp32 (bits 4-5 = 1),
+  // A bf16 (bits 7-9 = 1), B bf16 (bits 10-12 = 1), both K-major (bits 15,
+  // 16 = 0), N >> 3 at bits 17-22, M >> 4 at bits 24-28 (M = 128 per CTA).
+  static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
+                                    ((uint32_t)(UMMA_N >> 3) << 17) |
+                                    ((uint32_t)((BM * CG) >> 4) << 24);
+};
+
+constexpr int MAX_STAGES = 6;
 
 struct Ctl {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[MAX_STAGES];
+  uint64_t empty[MAX_STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -71,14 +88,34 @@ struct Ctl {
   int wsum[8];
 };
 
+template <int CG>
 size_t smem_bytes(int E) {
-  return 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Ctl) + (size_t)(3 * E + 1) * 4;
+  return 1024 + (size_t)Cfg<CG>::STAGES * Cfg<CG>::STAGE_BYTES + sizeof(Ctl) +
+         (size_t)(3 * E + 1) * 4;
 }
 
 // ---------------------------------------------------------------- PTX helpers
 
 __device__ __forceinline__ uint32_t saddr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t a, uint32_t rank) {
+  uint32_t d;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(rank));
+  return d;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
 }
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -89,8 +126,14 @@ __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+__device__ __forceinline__ void mbar_arrive_local(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Arrive on a barrier given by its shared::cluster address (possibly in the peer CTA).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
+               : "memory");
 }
 
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
@@ -102,7 +145,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}\n"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
@@ -116,12 +159,12 @@ __device__ __forceinline__ unsigned long long globaltimer() {
   return t;
 }
 
-// Wait for the phase of `bar` with parity `parity`. Gives up when the CTA's
-// abort flag is raised or after `limit_ns`; a timeout raises the flag and
+// Slow path of wait_phase: keep polling until the phase completes, the CTA's
+// abort flag is raised, or `limit_ns` passes; a timeout raises the flag and
 // records MOE_ERR_TIMEOUT.
-__device__ __noinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                        uint32_t* status, unsigned long long limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+__device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity,
+                                             volatile int* abort_flag, uint32_t* status,
+                                             unsigned long long limit_ns) {
   const unsigned long long t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -136,32 +179,67 @@ __device__ __noinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile 
   }
 }
 
+// Wait for the phase of `bar` with parity `parity` (bounded, see wait_phase_slow).
+// The common case, a phase that has already completed, costs one try_wait.
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                           uint32_t* status, unsigned long long limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_phase_slow(bar, parity, abort_flag, status, limit_ns);
+}
+
+// TMA box load into this CTA's shared memory; completion is counted on `bar`,
+// a shared::cluster barrier address that may lie in the pair's first CTA.
+template <int CG>
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
                                             uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
+  if (CG == 2)
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+  else
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
 }
 
 __device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+template <int CG>
 __device__ __forceinline__ void tmem_alloc(uint32_t dst, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst),
-               "r"(ncols)
-               : "memory");
+  if (CG == 2)
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst),
+                 "r"(ncols)
+                 : "memory");
+  else
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst),
+                 "r"(ncols)
+                 : "memory");
 }
 
+template <int CG>
 __device__ __forceinline__ void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  if (CG == 2)
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  else
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
 }
 
+template <int CG>
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
+  if (CG == 2)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr),
+                 "r"(ncols)
+                 : "memory");
+  else
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr),
+                 "r"(ncols)
+                 : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -172,22 +250,39 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// Arrive once on `bar` when every tcgen05 operation this thread issued so far
-// has completed.
+// Arrive once on `bar` (at the same offset in both CTAs of the pair for
+// CG = 2) when every tcgen05 operation this thread issued so far has completed.
+template <int CG>
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar)
-               : "memory");
+  if (CG == 2)
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(bar),
+        "h"((uint16_t)3)
+        : "memory");
+  else
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar)
+                 : "memory");
 }
 
+template <int CG>
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                        uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(IDESC), "r"(accumulate)
-      : "memory");
+  if (CG == 2)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(Cfg<CG>::IDESC), "r"(accumulate)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(Cfg<CG>::IDESC), "r"(accumulate)
+        : "memory");
 }
 
 // 32 consecutive fp32 columns of this thread's TMEM lane.
@@ -201,6 +296,28 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
         "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+// 64 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+      "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]),
+        "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]),
+        "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),
+        "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]),
+        "=r"(r[62]), "=r"(r[63])
       : "r"(taddr));
 }
 
@@ -249,25 +366,30 @@ __device__ __forceinline__ void decode_tile(int tile, int NT, const int* P, int 
   m = local - n * mt;
 }
 
-template <int MODE>
+template <int MODE, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 __nv_bfloat16* __restrict__ out, int N_out, int Kdim, int b_rows_per_expert,
                 int b_second_off, const int32_t* __restrict__ offsets,
                 const int32_t* __restrict__ counts, int E, int C, long long R_max,
                 uint32_t* __restrict__ status) {
+  using CF = Cfg<CG>;
+  constexpr int STAGES = CF::STAGES;
   constexpr int BN_OUT = (MODE == 0) ? 128 : 256;   // output columns per tile
   constexpr int N_STEP = BN_OUT;                     // weight rows per n tile
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = saddr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (base - raw);
-  Ctl* ctl = reinterpret_cast<Ctl*>(smem + STAGES * STAGE_BYTES);
+  Ctl* ctl = reinterpret_cast<Ctl*>(smem + STAGES * CF::STAGE_BYTES);
   int* P = reinterpret_cast<int*>(ctl + 1);   // [E+1] M-tile prefix
   int* row_off = P + (E + 1);                 // [E]
   int* kept_s = row_off + E;                  // [E]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;   // position in the pair
+  const bool leader = rank == 0;
+  const int cluster_id = blockIdx.x / CG, n_clusters = gridDim.x / CG;
   const int NT = (N_out + BN_OUT - 1) / BN_OUT;
   const int KB = Kdim / BK;
   volatile int* abort_flag = &ctl->abort;
@@ -279,7 +401,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(saddr(&ctl->tfull[b]), 1);
-      mbar_init(saddr(&ctl->tempty[b]), 4);
+      mbar_init(saddr(&ctl->tempty[b]), 4 * CG);
     }
     mbar_init(saddr(&ctl->drain), 1);
     ctl->abort = 0;
@@ -288,8 +410,8 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     prefetch_map(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(saddr(&ctl->tmem_base), TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc<CG>(saddr(&ctl->tmem_base), TMEM_COLS);
+    tmem_relinquish<CG>();
   }
   {  // per-expert kept rows, first row and M-tile prefix (block scan)
     const int chunk = (E + NUM_THREADS - 1) / NUM_THREADS;
@@ -301,7 +423,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         const int k = max(0, min(counts[e], C));
         kept_s[e] = k;
         row_off[e] = offsets[e];
-        local += (k + BM - 1) / BM;
+        local += (k + CF::TILE_ROWS - 1) / CF::TILE_ROWS;
       }
     }
     int incl = local;
@@ -318,13 +440,14 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       const int e = e0 + i;
       if (e < E) {
         P[e] = run;
-        run += (kept_s[e] + BM - 1) / BM;
+        run += (kept_s[e] + CF::TILE_ROWS - 1) / CF::TILE_ROWS;
       }
     }
     if (threadIdx.x == NUM_THREADS - 1) P[E] = run;
   }
   tc_fence_before();
   __syncthreads();
+  if (CG == 2) cluster_sync();   // both CTAs' barriers exist before anyone signals them
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
   const int total = P[E] * NT;
@@ -332,12 +455,11 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   if (warp == 0) {
     if (lane == 0) {  // ------------------------------------------------ TMA producer
       int it = 0;
-      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      for (int tile = cluster_id; tile < total; tile += n_clusters) {
         int e, m, n;
         decode_tile(tile, NT, P, E, e, m, n);
-        const int a_row = row_off[e] + m * BM;
+        const int a_row = row_off[e] + m * CF::TILE_ROWS + (int)rank * BM;
         const int b_row0 = e * b_rows_per_expert + n * N_STEP;
-        const int b_row1 = b_row0 + b_second_off;
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % STAGES;
@@ -346,24 +468,31 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             ok = false;
             break;
           }
-          const uint32_t sa = base + s * STAGE_BYTES;
-          const uint32_t fb = saddr(&ctl->full[s]);
-          mbar_expect_tx(fb, STAGE_BYTES);
-          tma_load_2d(sa, &tmA, kb * BK, a_row, fb);
-          tma_load_2d(sa + A_BYTES, &tmB, kb * BK, b_row0, fb);
-          tma_load_2d(sa + A_BYTES + B_HALF_BYTES, &tmB, kb * BK, b_row1, fb);
+          const uint32_t sa = base + s * CF::STAGE_BYTES;
+          const uint32_t fb_local = saddr(&ctl->full[s]);
+          const uint32_t fb = (CG == 2) ? map_to_rank(fb_local, 0) : fb_local;
+          if (leader) mbar_expect_tx(fb_local, CF::STAGE_BYTES * CG);
+          tma_load_2d<CG>(sa, &tmA, kb * BK, a_row, fb);
+          if (CG == 2) {
+            tma_load_2d<CG>(sa + BOX_BYTES, &tmB, kb * BK, b_row0 + (int)rank * b_second_off, fb);
+          } else {
+            tma_load_2d<CG>(sa + BOX_BYTES, &tmB, kb * BK, b_row0, fb);
+            tma_load_2d<CG>(sa + 2 * BOX_BYTES, &tmB, kb * BK, b_row0 + b_second_off, fb);
+          }
         }
         if (!ok) break;
       }
       // the copies of the last STAGES stages must land before the CTA exits
-      for (int i = max(0, it - STAGES); i < it; ++i)
-        wait_phase(saddr(&ctl->full[i % STAGES]), (uint32_t)(i / STAGES) & 1u, abort_flag, status,
-                   DRAIN_NS);
+      // (the leader's barriers also count the peer's copies)
+      if (leader)
+        for (int i = max(0, it - STAGES); i < it; ++i)
+          wait_phase(saddr(&ctl->full[i % STAGES]), (uint32_t)(i / STAGES) & 1u, abort_flag,
+                     status, DRAIN_NS);
     }
   } else if (warp == 1) {
-    if (lane == 0) {  // ------------------------------------------------ MMA issuer
+    if (lane == 0 && leader) {  // ---------------------------------------- MMA issuer
       int it = 0, tcount = 0;
-      for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
+      for (int tile = cluster_id; tile < total; tile += n_clusters, ++tcount) {
         const int b = tcount & 1;
         const uint32_t tph = (uint32_t)(tcount >> 1) & 1u;
         if (!wait_phase(saddr(&ctl->tempty[b]), tph ^ 1u, abort_flag, status, WAIT_NS)) break;
@@ -378,30 +507,33 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             break;
           }
           tc_fence_after();
-          const uint32_t sa = base + s * STAGE_BYTES;
+          const uint32_t sa = base + s * CF::STAGE_BYTES;
           const uint64_t ad = sw128_desc(sa);
-          const uint64_t bd = sw128_desc(sa + A_BYTES);
+          const uint64_t bd = sw128_desc(sa + BOX_BYTES);
 #pragma unroll
           for (int j = 0; j < BK / 16; ++j)
-            tc_mma(d, ad + (uint64_t)(2 * j), bd + (uint64_t)(2 * j), (kb | j) != 0 ? 1u : 0u);
-          tc_commit(saddr(&ctl->empty[s]));
+            tc_mma<CG>(d, ad + (uint64_t)(2 * j), bd + (uint64_t)(2 * j), (kb | j) != 0 ? 1u : 0u);
+          tc_commit<CG>(saddr(&ctl->empty[s]));
         }
         if (!ok) break;
-        tc_commit(saddr(&ctl->tfull[b]));
+        tc_commit<CG>(saddr(&ctl->tfull[b]));
       }
       // every MMA this thread issued must finish before TMEM is released
-      tc_commit(saddr(&ctl->drain));
+      tc_commit<CG>(saddr(&ctl->drain));
       wait_phase(saddr(&ctl->drain), 0u, abort_flag, status, DRAIN_NS);
     }
   } else {  // -------------------------------------------------------- epilogue
     const int q = warp & 3;                 // TMEM sub-partition of this warp
-    const int r_in = q * 32 + lane;         // tile row handled by this thread
+    const int r_in = q * 32 + lane;         // row of this CTA's half tile
+    const uint32_t tempty0 = saddr(&ctl->tempty[0]);
+    const uint32_t tempty_leader0 = (CG == 2) ? map_to_rank(tempty0, 0) : tempty0;
     int tcount = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
+    for (int tile = cluster_id; tile < total; tile += n_clusters, ++tcount) {
       int e, m, n;
       decode_tile(tile, NT, P, E, e, m, n);
-      const int rows = min(BM, kept_s[e] - m * BM);
-      const long long grow = (long long)row_off[e] + m * BM + r_in;
+      const int first = m * CF::TILE_ROWS + (int)rank * BM;   // first row of this half tile
+      const int rows = min(BM, kept_s[e] - first);
+      const long long grow = (long long)row_off[e] + first + r_in;
       const int b = tcount & 1;
       const uint32_t tph = (uint32_t)(tcount >> 1) & 1u;
       int ok = 1;
@@ -419,16 +551,16 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       const uint32_t t0 = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * UMMA_N);
       if (MODE == 0) {
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t g[32], u[32];
-          tmem_ld32(t0 + (uint32_t)(c * 32), g);
-          tmem_ld32(t0 + 128u + (uint32_t)(c * 32), u);
+        for (int c = 0; c < 2; ++c) {   // 64 h columns: gate in [c*64, +64), up in [128 + c*64, +64)
+          uint32_t g[64], u[64];
+          tmem_ld64(t0 + (uint32_t)(c * 64), g);
+          tmem_ld64(t0 + 128u + (uint32_t)(c * 64), u);
           tmem_ld_wait();
-          const int col = n * BN_OUT + c * 32;
-          if (row_ok && col < N_out) {
+          const int col = n * BN_OUT + c * 64;
+          if (row_ok && col < N_out) {   // N_out % 64 == 0: a chunk is all in or all out
             uint4* dst = reinterpret_cast<uint4*>(orow + col);
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
+            for (int v = 0; v < 8; ++v) {
               uint4 o;
               o.x = pack_bf16x2(silu_mul(g[8 * v + 0], u[8 * v + 0]), silu_mul(g[8 * v + 1], u[8 * v + 1]));
               o.y = pack_bf16x2(silu_mul(g[8 * v + 2], u[8 * v + 2]), silu_mul(g[8 * v + 3], u[8 * v + 3]));
@@ -440,15 +572,15 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         }
       } else {
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          uint32_t a[32];
-          tmem_ld32(t0 + (uint32_t)(c * 32), a);
+        for (int c = 0; c < 4; ++c) {   // 64 y columns per chunk
+          uint32_t a[64];
+          tmem_ld64(t0 + (uint32_t)(c * 64), a);
           tmem_ld_wait();
-          const int col = n * BN_OUT + c * 32;
+          const int col = n * BN_OUT + c * 64;
           if (row_ok && col < N_out) {
             uint4* dst = reinterpret_cast<uint4*>(orow + col);
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
+            for (int v = 0; v < 8; ++v) {
               uint4 o;
               o.x = pack_bf16x2(__uint_as_float(a[8 * v + 0]), __uint_as_float(a[8 * v + 1]));
               o.y = pack_bf16x2(__uint_as_float(a[8 * v + 2]), __uint_as_float(a[8 * v + 3]));
@@ -461,15 +593,19 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(saddr(&ctl->tempty[b]));
+      if (lane == 0) {
+        const uint32_t tb = tempty_leader0 + (uint32_t)(b * sizeof(uint64_t));
+        if (CG == 2) mbar_arrive_cluster(tb); else mbar_arrive_local(tb);
+      }
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  if (CG == 2) cluster_sync();   // no CTA leaves while its peer may still signal it
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    tmem_dealloc<CG>(tmem, TMEM_COLS);
   }
 }
 
@@ -503,11 +639,74 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows) 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  return n;
+template <int MODE, int CG>
+void fill_launch(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr, int grid, size_t smem,
+                 cudaStream_t s) {
+  cfg = cudaLaunchConfig_t{};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CG;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+}
+
+// Co-resident CTAs (CG = 1) or 2-CTA clusters (CG = 2) of the kernel on this device.
+template <int CG>
+int resident_units(size_t smem) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  if (CG == 1) return sms;
+  cudaLaunchConfig_t q;
+  cudaLaunchAttribute attr[1];
+  fill_launch<0, CG>(q, attr, sms & ~1, smem, nullptr);
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, tc_grouped_gemm<0, CG>, &q) != cudaSuccess)
+    return 0;
+  return clusters;
+}
+
+template <int CG>
+moe_status_t launch_mlp(const moe_config_t& c, const void* xp, const int32_t* offsets,
+                        const int32_t* counts, const void* w_gu, const void* w_d, void* h,
+                        void* y, int64_t R_max, uint32_t* status, cudaStream_t s) {
+  CUtensorMap mx, mwgu, mh, mwd;
+  if (!make_map(&mx, xp, (uint64_t)c.H, (uint64_t)R_max) ||
+      !make_map(&mwgu, w_gu, (uint64_t)c.H, (uint64_t)c.E * 2 * c.F) ||
+      !make_map(&mh, h, (uint64_t)c.F, (uint64_t)R_max) ||
+      !make_map(&mwd, w_d, (uint64_t)c.F, (uint64_t)c.E * c.H))
+    return MOE_ERR_CUDA;
+  const size_t smem = smem_bytes<CG>(c.E);
+  if (cudaFuncSetAttribute(tc_grouped_gemm<0, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess ||
+      cudaFuncSetAttribute(tc_grouped_gemm<1, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int units = resident_units<CG>(smem);
+  if (units <= 0) return MOE_ERR_CUDA;
+  const int64_t mt_bound = ceil_div(R_max, Cfg<CG>::TILE_ROWS) + c.E;  // >= sum_e M tiles
+  const int64_t t0 = mt_bound * ceil_div(c.F, 128), t1 = mt_bound * ceil_div(c.H, 256);
+  const int g0 = (int)std::min<int64_t>(units, t0) * CG;
+  const int g1 = (int)std::min<int64_t>(units, t1) * CG;
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  fill_launch<0, CG>(cfg, attr, g0, smem, s);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, tc_grouped_gemm<0, CG>, mx, mwgu,
+                                     static_cast<__nv_bfloat16*>(h), c.F, c.H, 2 * c.F, c.F,
+                                     offsets, counts, c.E, c.capacity, (long long)R_max, status);
+  if (e == cudaSuccess) {
+    fill_launch<1, CG>(cfg, attr, g1, smem, s);
+    e = cudaLaunchKernelEx(&cfg, tc_grouped_gemm<1, CG>, mh, mwd, static_cast<__nv_bfloat16*>(y),
+                           c.H, c.F, c.H, 128, offsets, counts, c.E, c.capacity,
+                           (long long)R_max, status);
+  }
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace tc
@@ -516,32 +715,14 @@ moe_status_t launch_mlp_bf16_tc(const moe_config_t& c, const void* xp, const int
                                 const int32_t* counts, const void* w_gu, const void* w_d,
                                 void* h, void* y, int64_t R_max, uint32_t* status,
                                 cudaStream_t s) {
-  using namespace tc;
   if (R_max == 0) return MOE_OK;
-  CUtensorMap mx, mwgu, mh, mwd;
-  if (!make_map(&mx, xp, (uint64_t)c.H, (uint64_t)R_max) ||
-      !make_map(&mwgu, w_gu, (uint64_t)c.H, (uint64_t)c.E * 2 * c.F) ||
-      !make_map(&mh, h, (uint64_t)c.F, (uint64_t)R_max) ||
-      !make_map(&mwd, w_d, (uint64_t)c.F, (uint64_t)c.E * c.H))
-    return MOE_ERR_CUDA;
-  const int sms = sm_count();
-  if (sms <= 0) return MOE_ERR_CUDA;
-  const size_t smem = smem_bytes(c.E);
-  if (cudaFuncSetAttribute(tc_grouped_gemm<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess ||
-      cudaFuncSetAttribute(tc_grouped_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  const int64_t mt_bound = ceil_div(R_max, BM) + c.E;   // >= sum_e ceil(kept_e / BM)
-  const int64_t t0 = mt_bound * ceil_div(c.F, 128), t1 = mt_bound * ceil_div(c.H, 256);
-  const int g0 = (int)std::min<int64_t>(sms, t0), g1 = (int)std::min<int64_t>(sms, t1);
-  tc_grouped_gemm<0><<<g0, NUM_THREADS, smem, s>>>(
-      mx, mwgu, static_cast<__nv_bfloat16*>(h), c.F, c.H, 2 * c.F, c.F, offsets, counts, c.E,
-      c.capacity, (long long)R_max, status);
-  tc_grouped_gemm<1><<<g1, NUM_THREADS, smem, s>>>(
-      mh, mwd, static_cast<__nv_bfloat16*>(y), c.H, c.F, c.H, 128, offsets, counts, c.E,
-      c.capacity, (long long)R_max, status);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  // Tile shape from the expected rows per expert: 256-row pair tiles halve each
+  // CTA's operand traffic but waste up to 255 padded rows per expert, so small
+  // experts (decode-like batches) use 128-row single-CTA tiles.
+  const int64_t rows_per_expert = std::min<int64_t>((int64_t)c.T * c.K, (int64_t)c.E * c.capacity) / c.E;
+  if (rows_per_expert >= 192)
+    return tc::launch_mlp<2>(c, xp, offsets, counts, w_gu, w_d, h, y, R_max, status, s);
+  return tc::launch_mlp<1>(c, xp, offsets, counts, w_gu, w_d, h, y, R_max, status, s);
 }
 
 }  // namespace moe

@@ -10,10 +10,10 @@
 
 namespace moe {
 
-// Tokens handled by one block of the route kernel. The per-block expert
-// bitmap has ROUTE_TB/32 words per expert.
+// Tokens handled by one block of the route kernel (the unit of the per-block
+// expert histograms). The per-block expert bitmap has ROUTE_TB/32 words per
+// expert.
 constexpr int ROUTE_TB = 128;
-constexpr int ROUTE_THREADS = 256;
 constexpr int MAX_E = 1024;
 constexpr int MAX_K = 32;
 

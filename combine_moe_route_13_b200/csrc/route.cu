@@ -13,13 +13,18 @@
 // "Dispatch", notes that its own packing order is not).
 //
 // Three launches, no host synchronisation:
-//   route_topk_kernel  one warp per token: K rounds of a warp arg-max over the
-//                      token's E logits, softmax over the K winners, bitmap.
-//   route_scan_kernel  one block: per-expert scan over blocks, counts,
-//                      capacity/overflow ("MoE Expert Parallel Benchmark",
-//                      Step 2), aligned exclusive scan over experts, segments.
-//   route_slot_kernel  every assignment: slot = off[e] + rank if rank < C,
-//                      else -1; row_src back-map; padding rows of row_src = -1.
+//   route_topk_kernel  one warp per token (4-8 tokens per warp, the next
+//                      token's logits loaded while the current one is ranked):
+//                      K rounds of a warp arg-max over the token's E logits,
+//                      softmax over the K winners, bitmap.
+//   route_scan_kernel  one warp per expert: exclusive scan of the expert's
+//                      per-block counts, its total count and overflow
+//                      ("MoE Expert Parallel Benchmark", Step 2).
+//   route_slot_kernel  every block first scans the aligned kept counts over
+//                      the experts (block 0 stores the offsets, segment
+//                      offsets and totals); then every assignment gets
+//                      slot = off[e] + rank if rank < C, else -1, the row_src
+//                      back-map, and row_src padding rows get -1.
 #include <algorithm>
 #include <cfloat>
 #include <climits>
@@ -45,7 +50,17 @@ __device__ __forceinline__ bool better(const Cand& a, const Cand& b) {
 }
 
 template <int VPL>
-__global__ void __launch_bounds__(ROUTE_THREADS)
+__device__ __forceinline__ void load_logits(const float* __restrict__ row, int E, int lane,
+                                            float (&v)[VPL]) {
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) {
+    const int e = lane + 32 * j;
+    v[j] = (e < E) ? __ldg(row + e) : 0.f;
+  }
+}
+
+template <int VPL, int THREADS>
+__global__ void __launch_bounds__(THREADS)
 route_topk_kernel(const float* __restrict__ logits, int T, int E, int K,
                   int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                   int32_t* __restrict__ local_rank, int32_t* __restrict__ blk_cnt) {
@@ -59,22 +74,20 @@ route_topk_kernel(const float* __restrict__ logits, int T, int E, int K,
   __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nwarps = blockDim.x >> 5;
-  for (int tl = warp; tl < ntok; tl += nwarps) {
-    const int t = tb0 + tl;
-    const float* row = logits + (size_t)t * E;
-    float v[VPL];
-    uint32_t taken = 0u;
+  constexpr int NWARPS = THREADS / 32;
+  uint32_t invalid = 0u;   // bit j: element lane + 32 j does not exist
 #pragma unroll
-    for (int j = 0; j < VPL; ++j) {
-      const int e = lane + 32 * j;
-      if (e < E) {
-        v[j] = __ldg(row + e);
-      } else {
-        v[j] = 0.f;
-        taken |= 1u << j;
-      }
-    }
+  for (int j = 0; j < VPL; ++j)
+    if (lane + 32 * j >= E) invalid |= 1u << j;
+  float nxt[VPL];
+  if (warp < ntok) load_logits<VPL>(logits + (size_t)(tb0 + warp) * E, E, lane, nxt);
+  for (int tl = warp; tl < ntok; tl += NWARPS) {
+    const int t = tb0 + tl;
+    float v[VPL];
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) v[j] = nxt[j];
+    if (tl + NWARPS < ntok) load_logits<VPL>(logits + (size_t)(t + NWARPS) * E, E, lane, nxt);
+    uint32_t taken = invalid;
     float my_v = 0.f, v0 = 0.f;
     int my_i = 0;
     for (int k = 0; k < K; ++k) {
@@ -132,93 +145,113 @@ route_topk_kernel(const float* __restrict__ logits, int T, int E, int K,
   }
 }
 
-// Block-wide exclusive scan for blockDim.x == 1024 (32 warps).
-__device__ __forceinline__ int block_excl_scan_1024(int v, int* warp_tmp, int& total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = v;
+// One warp per expert: exclusive scan of the expert's per-block counts (in
+// place), its total count and its overflow.
+__global__ void __launch_bounds__(1024)
+route_scan_kernel(int nblk, int E, int C, int32_t* __restrict__ blk_cnt,
+                  int32_t* __restrict__ counts, int32_t* __restrict__ overflow) {
+  const int e = blockIdx.x * 32 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (e >= E) return;
+  const int per = (nblk + 31) / 32;            // consecutive blocks per lane
+  const int b0 = min(nblk, lane * per), b1 = min(nblk, b0 + per);
+  int local = 0;
+  for (int b = b0; b < b1; ++b) local += blk_cnt[(size_t)b * E + e];
+  int incl = local;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
     const int o = __shfl_up_sync(0xffffffffu, incl, off);
     if (lane >= off) incl += o;
   }
-  if (lane == 31) warp_tmp[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int w = warp_tmp[lane];
-    int wi = w;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int o = __shfl_up_sync(0xffffffffu, wi, off);
-      if (lane >= off) wi += o;
-    }
-    warp_tmp[lane] = wi - w;       // exclusive prefix of warp totals
-    if (lane == 31) warp_tmp[32] = wi;
+  int run = incl - local;
+  for (int b = b0; b < b1; ++b) {
+    const size_t p = (size_t)b * E + e;
+    const int c = blk_cnt[p];
+    blk_cnt[p] = run;
+    run += c;
   }
-  __syncthreads();
-  const int res = warp_tmp[warp] + incl - v;
-  total = warp_tmp[32];
-  __syncthreads();
-  return res;
+  if (lane == 31) {
+    counts[e] = incl;
+    overflow[e] = max(incl - C, 0);
+  }
 }
 
-__global__ void __launch_bounds__(1024)
-route_scan_kernel(int nblk, int E, int S, int C, int A, int TK, int32_t* __restrict__ blk_cnt,
-                  int32_t* __restrict__ counts, int32_t* __restrict__ overflow,
-                  int32_t* __restrict__ offsets, int32_t* __restrict__ segoff,
-                  int32_t* __restrict__ totals) {
-  __shared__ int warp_tmp[33];
-  __shared__ int off_s[MAX_E + 1];
-  const int e = threadIdx.x;
-  int cnt = 0;
-  if (e < E) {
-    // per-expert exclusive scan over the blocks, in place
-#pragma unroll 8
-    for (int b = 0; b < nblk; ++b) {
-      const size_t p = (size_t)b * E + e;
-      const int c = blk_cnt[p];
-      blk_cnt[p] = cnt;
-      cnt += c;
+// Exclusive scan of the experts' aligned kept counts, done by every block of
+// route_slot_kernel into shared memory (E <= 1024, 256 threads, 4 per thread).
+__device__ __forceinline__ void expert_offsets_smem(int E, int C, int A,
+                                                    const int32_t* __restrict__ counts,
+                                                    int* off_s, int* kept_s, int* warp_tmp,
+                                                    int& sum_kept) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int e0 = threadIdx.x * 4;
+  int pad[4], kp[4], local = 0, lk = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = e0 + i;
+    kp[i] = (e < E) ? min(counts[e], C) : 0;
+    pad[i] = (kp[i] + A - 1) / A * A;
+    local += pad[i];
+    lk += kp[i];
+  }
+  int incl = local, inck = lk;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, off);
+    const int ok = __shfl_up_sync(0xffffffffu, inck, off);
+    if (lane >= off) {
+      incl += o;
+      inck += ok;
     }
   }
-  const int kept = min(cnt, C);
-  const int ov = cnt - kept;
-  const int padded = (e < E) ? (kept + A - 1) / A * A : 0;
-  int sum_pad, sum_kept, sum_ov;
-  const int excl = block_excl_scan_1024(padded, warp_tmp, sum_pad);
-  block_excl_scan_1024(e < E ? kept : 0, warp_tmp, sum_kept);
-  block_excl_scan_1024(e < E ? ov : 0, warp_tmp, sum_ov);
-  if (e < E) {
-    counts[e] = cnt;
-    overflow[e] = ov;
-    offsets[e] = excl;
-    off_s[e] = excl;
-  }
-  if (e == 0) {
-    offsets[E] = sum_pad;
-    off_s[E] = sum_pad;
-    totals[0] = TK;
-    totals[1] = sum_kept;
-    totals[2] = sum_ov;
-    totals[3] = sum_pad;
+  if (lane == 31) {
+    warp_tmp[warp] = incl;
+    warp_tmp[8 + warp] = inck;
   }
   __syncthreads();
-  const int per = E / S;
-  for (int q = e; q <= S; q += blockDim.x) segoff[q] = off_s[q * per];
+  int base = 0, tot = 0, totk = 0;
+  for (int w = 0; w < 8; ++w) {
+    if (w < warp) base += warp_tmp[w];
+    tot += warp_tmp[w];
+    totk += warp_tmp[8 + w];
+  }
+  int run = base + incl - local;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = e0 + i;
+    if (e < E) {
+      off_s[e] = run;
+      kept_s[e] = kp[i];
+    }
+    run += pad[i];
+  }
+  if (threadIdx.x == 0) off_s[E] = tot;
+  sum_kept = totk;
+  __syncthreads();
 }
 
 __global__ void __launch_bounds__(256)
-route_slot_kernel(int T, int K, int E, int C, int64_t R_max,
+route_slot_kernel(int T, int K, int E, int S, int C, int A, int64_t R_max,
                   const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ blk_base,
-                  const int32_t* __restrict__ offsets, const int32_t* __restrict__ counts,
+                  const int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                  int32_t* __restrict__ segoff, int32_t* __restrict__ totals,
                   int32_t* __restrict__ slot, int32_t* __restrict__ row_src) {
   __shared__ int off_s[MAX_E + 1];
   __shared__ int kept_s[MAX_E];
-  for (int e = threadIdx.x; e <= E; e += blockDim.x) {
-    off_s[e] = offsets[e];
-    if (e < E) kept_s[e] = min(counts[e], C);
-  }
-  __syncthreads();
+  __shared__ int warp_tmp[16];
+  int sum_kept;
+  expert_offsets_smem(E, C, A, counts, off_s, kept_s, warp_tmp, sum_kept);
   const int64_t TK = (int64_t)T * K;
+  if (blockIdx.x == 0) {
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) offsets[e] = off_s[e];
+    const int per = E / S;
+    for (int q = threadIdx.x; q <= S; q += blockDim.x) segoff[q] = off_s[q * per];
+    if (threadIdx.x == 0) {
+      totals[0] = (int32_t)TK;
+      totals[1] = sum_kept;
+      totals[2] = (int32_t)TK - sum_kept;
+      totals[3] = off_s[E];
+    }
+  }
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < TK; i += stride) {
     const int t = (int)(i / K);
@@ -250,7 +283,9 @@ route_slot_kernel(int T, int K, int E, int C, int64_t R_max,
 template <int VPL>
 void launch_topk(int nblk, size_t smem, cudaStream_t s, const float* logits, int T, int E, int K,
                  int32_t* idx, float* w, int32_t* rank, int32_t* blk) {
-  route_topk_kernel<VPL><<<nblk, ROUTE_THREADS, smem, s>>>(logits, T, E, K, idx, w, rank, blk);
+  // 32 warps (4 tokens each) while the register budget allows, 16 for E > 512
+  constexpr int THREADS = VPL >= 32 ? 512 : 1024;
+  route_topk_kernel<VPL, THREADS><<<nblk, THREADS, smem, s>>>(logits, T, E, K, idx, w, rank, blk);
 }
 
 }  // namespace
@@ -270,12 +305,13 @@ cudaError_t launch_route(const moe_config_t& c, const float* logits, int32_t* to
     else if (vpl <= 16) launch_topk<16>(nblk, smem, s, logits, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
     else launch_topk<32>(nblk, smem, s, logits, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
   }
-  route_scan_kernel<<<1, 1024, 0, s>>>(nblk, c.E, c.S, c.capacity, c.row_align, c.T * c.K,
-                                       blk_cnt, counts, overflow, offsets, segoff, totals);
+  route_scan_kernel<<<(unsigned)ceil_div(c.E, 32), 1024, 0, s>>>(nblk, c.E, c.capacity, blk_cnt,
+                                                                 counts, overflow);
   const int64_t work = std::max<int64_t>((int64_t)c.T * c.K, R_max);
   int grid = (int)std::min<int64_t>(std::max<int64_t>(ceil_div(work, 256), 1), 148 * 8);
-  route_slot_kernel<<<grid, 256, 0, s>>>(c.T, c.K, c.E, c.capacity, R_max, topk_idx, blk_cnt,
-                                         offsets, counts, slot, row_src);
+  route_slot_kernel<<<grid, 256, 0, s>>>(c.T, c.K, c.E, c.S, c.capacity, c.row_align, R_max,
+                                         topk_idx, blk_cnt, counts, offsets, segoff, totals, slot,
+                                         row_src);
   return cudaGetLastError();
 }
 

@@ -151,6 +151,10 @@ MLP_CASES = [
     (600, 256, 8, 2, 384, 8, 2.0, 128, "zipf"),        # empty experts
     (128, 64, 64, 8, 64, 8, 2.0, 16, "normal"),        # many tiny experts
     (1200, 1024, 8, 2, 1024, 2, 1.25, 128, "normal"),  # several M and N tiles per expert
+    # >= 192 rows per expert: 256-row tiles on CTA pairs
+    (2048, 256, 4, 2, 192, 2, 1.25, 1, "normal"),      # pair tiles straddling experts, N tail
+    (1500, 320, 6, 2, 256, 3, 1.0, 128, "zipf"),       # odd 128-row blocks, small experts
+    (3000, 512, 12, 2, 320, 4, 2.0, 128, "hot"),       # one hot expert over many pair tiles
 ]
 
 
