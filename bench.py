@@ -131,7 +131,12 @@ def max_over_ranks(x: float, world: int, device) -> float:
 
 
 def flush_l2(buf: torch.Tensor):
+    """Evict L2 (a write larger than L2), then keep the GPU busy for ~0.2 ms
+    so that the host has queued the next step's launches before the GPU
+    reaches them: the timed region then holds device time only."""
     buf.add_(1)
+    if hasattr(torch.cuda, "_sleep"):
+        torch.cuda._sleep(400_000)
 
 
 class Layer:

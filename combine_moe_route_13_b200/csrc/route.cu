@@ -15,11 +15,13 @@
 // Three launches, no host synchronisation:
 //   route_topk_kernel  one warp per token (4-8 tokens per warp, the next
 //                      token's logits loaded while the current one is ranked):
-//                      K rounds of a warp arg-max over the token's E logits,
-//                      softmax over the K winners, bitmap.
+//                      K rounds of a warp arg-max over the token's E logits
+//                      (two redux.sync reductions per round on an
+//                      order-preserving integer key), softmax over the K
+//                      winners, bitmap, per-block counts [E][blocks].
 //   route_scan_kernel  one warp per expert: exclusive scan of the expert's
-//                      per-block counts, its total count and overflow
-//                      ("MoE Expert Parallel Benchmark", Step 2).
+//                      per-block counts (one coalesced row), its total count
+//                      and overflow ("MoE Expert Parallel Benchmark", Step 2).
 //   route_slot_kernel  every block first scans the aligned kept counts over
 //                      the experts (block 0 stores the offsets, segment
 //                      offsets and totals); then every assignment gets
@@ -37,16 +39,16 @@ namespace {
 
 constexpr int WORDS = ROUTE_TB / 32;   // bitmap words per expert
 
-struct Cand {
-  float v;
-  int i;   // INT_MAX: no candidate
-};
+// Order-preserving map of a float to uint32 (larger float -> larger key);
+// -0.0 is first folded into +0.0 so that the two compare equal, as floats do.
+// Keys of finite values and of -inf are > 0.
+__device__ __forceinline__ uint32_t order_key(float v) {
+  const uint32_t b = __float_as_uint(v + 0.0f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
 
-// Total order of the selection: larger logit first, then lower expert index.
-__device__ __forceinline__ bool better(const Cand& a, const Cand& b) {
-  if (a.i == INT_MAX) return false;
-  if (b.i == INT_MAX) return true;
-  return a.v > b.v || (a.v == b.v && a.i < b.i);
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
 template <int VPL>
@@ -88,32 +90,33 @@ route_topk_kernel(const float* __restrict__ logits, int T, int E, int K,
     for (int j = 0; j < VPL; ++j) v[j] = nxt[j];
     if (tl + NWARPS < ntok) load_logits<VPL>(logits + (size_t)(t + NWARPS) * E, E, lane, nxt);
     uint32_t taken = invalid;
+    uint32_t key[VPL];
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) key[j] = order_key(v[j]);
     float my_v = 0.f, v0 = 0.f;
     int my_i = 0;
     for (int k = 0; k < K; ++k) {
-      Cand c{0.f, INT_MAX};
+      // this lane's best remaining element: elements are visited in increasing
+      // index order, so a strict '>' keeps the lowest index among equal keys
+      uint32_t best = 0u;
+      int bi = INT_MAX;
 #pragma unroll
       for (int j = 0; j < VPL; ++j) {
-        // elements of a lane are visited in increasing index order, so a
-        // strict '>' keeps the lowest index among equal logits
-        if (!((taken >> j) & 1u) && (c.i == INT_MAX || v[j] > c.v)) {
-          c.v = v[j];
-          c.i = lane + 32 * j;
+        if (!((taken >> j) & 1u) && key[j] > best) {
+          best = key[j];
+          bi = lane + 32 * j;
         }
       }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        Cand o;
-        o.v = __shfl_xor_sync(0xffffffffu, c.v, off);
-        o.i = __shfl_xor_sync(0xffffffffu, c.i, off);
-        if (better(o, c)) c = o;
-      }
-      if (k == 0) v0 = c.v;
+      // the warp's largest key, then the lowest index holding it
+      const uint32_t m = __reduce_max_sync(0xffffffffu, best);
+      const int win = __reduce_min_sync(0xffffffffu, best == m ? bi : INT_MAX);
+      const float wv = key_value(m);
+      if (k == 0) v0 = wv;
       if (lane == k) {
-        my_v = c.v;
-        my_i = c.i;
+        my_v = wv;
+        my_i = win;
       }
-      if ((c.i & 31) == lane) taken |= 1u << (c.i >> 5);
+      if ((win & 31) == lane) taken |= 1u << (win >> 5);
     }
     // softmax over the K selected logits, shifted by the largest one
     const float ex = (lane < K) ? expf(my_v - v0) : 0.f;
@@ -133,7 +136,7 @@ route_topk_kernel(const float* __restrict__ logits, int T, int E, int K,
     int c = 0;
 #pragma unroll
     for (int q = 0; q < WORDS; ++q) c += __popc(bitmap[e * WORDS + q]);
-    blk_cnt[(size_t)blockIdx.x * E + e] = c;
+    blk_cnt[(size_t)e * gridDim.x + blockIdx.x] = c;
   }
   for (int i = threadIdx.x; i < ntok * K; i += blockDim.x) {
     const int tl = i / K;
@@ -145,34 +148,41 @@ route_topk_kernel(const float* __restrict__ logits, int T, int E, int K,
   }
 }
 
-// One warp per expert: exclusive scan of the expert's per-block counts (in
-// place), its total count and its overflow.
+// One warp per expert: exclusive scan, in place, of the expert's per-block
+// counts (row e of [E][nblk]), its total count and its overflow. Loads of
+// eight 32-block chunks are issued before they are scanned.
 __global__ void __launch_bounds__(1024)
 route_scan_kernel(int nblk, int E, int C, int32_t* __restrict__ blk_cnt,
                   int32_t* __restrict__ counts, int32_t* __restrict__ overflow) {
   const int e = blockIdx.x * 32 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (e >= E) return;
-  const int per = (nblk + 31) / 32;            // consecutive blocks per lane
-  const int b0 = min(nblk, lane * per), b1 = min(nblk, b0 + per);
-  int local = 0;
-  for (int b = b0; b < b1; ++b) local += blk_cnt[(size_t)b * E + e];
-  int incl = local;
+  int32_t* row = blk_cnt + (size_t)e * nblk;
+  constexpr int G = 8;
+  int carry = 0;
+  for (int c0 = 0; c0 < nblk; c0 += 32 * G) {
+    int v[G];
 #pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int o = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += o;
+    for (int g = 0; g < G; ++g) {
+      const int b = c0 + g * 32 + lane;
+      v[g] = (b < nblk) ? row[b] : 0;
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      int incl = v[g];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      const int b = c0 + g * 32 + lane;
+      if (b < nblk) row[b] = carry + incl - v[g];
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
   }
-  int run = incl - local;
-  for (int b = b0; b < b1; ++b) {
-    const size_t p = (size_t)b * E + e;
-    const int c = blk_cnt[p];
-    blk_cnt[p] = run;
-    run += c;
-  }
-  if (lane == 31) {
-    counts[e] = incl;
-    overflow[e] = max(incl - C, 0);
+  if (lane == 0) {
+    counts[e] = carry;
+    overflow[e] = max(carry - C, 0);
   }
 }
 
@@ -230,7 +240,7 @@ __device__ __forceinline__ void expert_offsets_smem(int E, int C, int A,
 }
 
 __global__ void __launch_bounds__(256)
-route_slot_kernel(int T, int K, int E, int S, int C, int A, int64_t R_max,
+route_slot_kernel(int T, int K, int E, int S, int C, int A, int nblk, int64_t R_max,
                   const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ blk_base,
                   const int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                   int32_t* __restrict__ segoff, int32_t* __restrict__ totals,
@@ -256,7 +266,7 @@ route_slot_kernel(int T, int K, int E, int S, int C, int A, int64_t R_max,
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < TK; i += stride) {
     const int t = (int)(i / K);
     const int e = topk_idx[i];
-    const int pos = blk_base[(size_t)(t / ROUTE_TB) * E + e] + slot[i];
+    const int pos = blk_base[(size_t)e * nblk + t / ROUTE_TB] + slot[i];
     int s = -1;
     if (pos < C) {
       s = off_s[e] + pos;
@@ -283,8 +293,9 @@ route_slot_kernel(int T, int K, int E, int S, int C, int A, int64_t R_max,
 template <int VPL>
 void launch_topk(int nblk, size_t smem, cudaStream_t s, const float* logits, int T, int E, int K,
                  int32_t* idx, float* w, int32_t* rank, int32_t* blk) {
-  // 32 warps (4 tokens each) while the register budget allows, 16 for E > 512
-  constexpr int THREADS = VPL >= 32 ? 512 : 1024;
+  // 32 warps (4 tokens each) while the register budget allows: 16 warps for
+  // E > 256, 8 for E > 512
+  constexpr int THREADS = VPL >= 32 ? 256 : (VPL >= 16 ? 512 : 1024);
   route_topk_kernel<VPL, THREADS><<<nblk, THREADS, smem, s>>>(logits, T, E, K, idx, w, rank, blk);
 }
 
@@ -309,7 +320,7 @@ cudaError_t launch_route(const moe_config_t& c, const float* logits, int32_t* to
                                                                  counts, overflow);
   const int64_t work = std::max<int64_t>((int64_t)c.T * c.K, R_max);
   int grid = (int)std::min<int64_t>(std::max<int64_t>(ceil_div(work, 256), 1), 148 * 8);
-  route_slot_kernel<<<grid, 256, 0, s>>>(c.T, c.K, c.E, c.S, c.capacity, c.row_align, R_max,
+  route_slot_kernel<<<grid, 256, 0, s>>>(c.T, c.K, c.E, c.S, c.capacity, c.row_align, nblk, R_max,
                                          topk_idx, blk_cnt, counts, offsets, segoff, totals, slot,
                                          row_src);
   return cudaGetLastError();
