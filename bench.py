@@ -80,7 +80,7 @@ class Clocks:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -231,14 +231,29 @@ def e2e_steps(layer: Layer, steps, warmup, flush_buf, stream):
     return times, h2d, d2h
 
 
-def algorithmic(layer: Layer, totals):
+def mlp_tile_rows(layer: Layer) -> int:
+    """Rows per grouped-GEMM tile the library picks for this shape (256-row
+    tiles on CTA pairs when the expected rows per expert are >= 192)."""
+    wl = layer.wl
+    if wl.act == "f32":
+        return 32
+    return 256 if min(wl.T * wl.K, wl.E * layer.C) // wl.E >= 192 else 128
+
+
+def algorithmic(layer: Layer, totals, counts):
     wl = layer.wl
     s = 4 if wl.act == "f32" else 2
     N = int(totals[1])
     T, H, F, K, E = wl.T, wl.H, wl.F, wl.K, wl.E
+    tr = mlp_tile_rows(layer)
+    kept = np.minimum(np.asarray(counts), layer.C)
+    executed = int(np.sum((kept + tr - 1) // tr * tr))
     return {
         "N": N,
+        "tile_rows": tr,
+        "executed_rows": executed,
         "mlp_flops": 6.0 * N * H * F,
+        "mlp_executed_flops": 6.0 * executed * H * F,
         "dispatch_bytes": (T + N) * H * s + T * K * 4,
         "combine_bytes": (N + T) * H * s + T * K * 8,
         "route_bytes": T * E * 4 + T * K * 12,
@@ -305,8 +320,8 @@ def run_reference(args, wl: W.Workload, world, rank):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=16)
-    ap.add_argument("--warmup", type=int, default=4)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mixtral", choices=sorted(W.WORKLOADS))
     ap.add_argument("--cpu-tokens", type=int, default=256,
@@ -338,7 +353,7 @@ def main(argv=None):
     if st != layer.M.MOE_OK:
         raise SystemExit(f"device status after the first step: {layer.M.status_string(st)}")
     totals = layer.views()["totals"].cpu().tolist()
-    alg = algorithmic(layer, totals)
+    alg = algorithmic(layer, totals, layer.views()["expert_counts"].cpu().numpy())
 
     def barrier():
         if world > 1:
@@ -378,6 +393,9 @@ def main(argv=None):
     kernels["dispatch_hbm_frac"] = kernels["dispatch_gbs"] / hbm
     kernels["combine_hbm_frac"] = kernels["combine_gbs"] / hbm
     kernels["expert_mlp_tensor_frac_burst"] = mlp_tflops / peaks["bf16_tflops"]
+    kernels["expert_mlp_executed_tflops"] = alg["mlp_executed_flops"] / (ph["expert_mlp"] * 1e-3) / 1e12
+    kernels["expert_mlp_tile_rows"] = alg["tile_rows"]
+    kernels["expert_mlp_executed_rows"] = alg["executed_rows"]
 
     if rank != 0:
         if world > 1:

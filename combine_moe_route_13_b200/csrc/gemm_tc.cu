@@ -28,7 +28,9 @@
 //              allocation; two 256-column accumulators so that the epilogue
 //              of one tile overlaps the MMAs of the next;
 //   warps 2-5  epilogue: tcgen05.ld of its TMEM sub-partition's 32 lanes,
-//              SwiGLU / rounding, stores.
+//              SwiGLU / rounding, then a 128 x 64 box staged in shared memory
+//              (128-byte swizzle) and written by a TMA store; half tiles that
+//              end inside an expert's last rows are stored row by row instead.
 // Barriers: the producers of both CTAs signal the leader's "full" barrier;
 // the leader's commits signal "empty" and "TMEM full" in both CTAs; both
 // CTAs' epilogues signal the leader's "TMEM empty".
@@ -88,10 +90,12 @@ struct Ctl {
   int wsum[8];
 };
 
+constexpr int STAGING_BYTES = 128 * 64 * 2;   // one 128-row x 64-column bf16 output box
+
 template <int CG>
 size_t smem_bytes(int E) {
-  return 1024 + (size_t)Cfg<CG>::STAGES * Cfg<CG>::STAGE_BYTES + sizeof(Ctl) +
-         (size_t)(3 * E + 1) * 4;
+  return 1024 + (size_t)Cfg<CG>::STAGES * Cfg<CG>::STAGE_BYTES + STAGING_BYTES + sizeof(Ctl) +
+         (size_t)(3 * E + 2) * 4;
 }
 
 // ---------------------------------------------------------------- PTX helpers
@@ -204,6 +208,38 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
         : "memory");
+}
+
+// TMA store of one staged box (shared memory -> global), tracked by bulk groups.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y, uint32_t src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(src)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Wait until the committed bulk stores have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// Wait until the committed bulk stores have completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to TMA.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Barrier among the four epilogue warps only.
+__device__ __forceinline__ void epilogue_bar() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
 }
 
 __device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
@@ -344,9 +380,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&b);
 }
 
+// silu(g) * u = g * u / (1 + exp(-g)), with the fast exponential and the fast
+// reciprocal-multiply division (the result is rounded to bf16 next). For very
+// negative g the denominator overflows to inf and the quotient is 0, which is
+// silu's limit.
 __device__ __forceinline__ float silu_mul(uint32_t g_bits, uint32_t u_bits) {
   const float g = __uint_as_float(g_bits);
-  return g / (1.0f + __expf(-g)) * __uint_as_float(u_bits);
+  return __fdividef(g * __uint_as_float(u_bits), 1.0f + __expf(-g));
 }
 
 // Tile t -> (expert, m tile, n tile). Expert e owns tiles [NT*P[e], NT*P[e+1])
@@ -369,7 +409,8 @@ __device__ __forceinline__ void decode_tile(int tile, int NT, const int* P, int 
 template <int MODE, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                __nv_bfloat16* __restrict__ out, int N_out, int Kdim, int b_rows_per_expert,
+                const __grid_constant__ CUtensorMap tmOut, __nv_bfloat16* __restrict__ out,
+                int N_out, int Kdim, int b_rows_per_expert,
                 int b_second_off, const int32_t* __restrict__ offsets,
                 const int32_t* __restrict__ counts, int E, int C, long long R_max,
                 uint32_t* __restrict__ status) {
@@ -381,10 +422,11 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   const uint32_t raw = saddr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (base - raw);
-  Ctl* ctl = reinterpret_cast<Ctl*>(smem + STAGES * CF::STAGE_BYTES);
+  const uint32_t staging = base + STAGES * CF::STAGE_BYTES;   // epilogue output box
+  Ctl* ctl = reinterpret_cast<Ctl*>(smem + STAGES * CF::STAGE_BYTES + STAGING_BYTES);
   int* P = reinterpret_cast<int*>(ctl + 1);   // [E+1] M-tile prefix
-  int* row_off = P + (E + 1);                 // [E]
-  int* kept_s = row_off + E;                  // [E]
+  int* row_off = P + (E + 1);                 // [E+1] first row of each expert, and R
+  int* kept_s = row_off + (E + 1);            // [E]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;   // position in the pair
@@ -408,6 +450,8 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     fence_mbar_init();
     prefetch_map(&tmA);
     prefetch_map(&tmB);
+    prefetch_map(&tmOut);
+    row_off[E] = offsets[E];
   }
   if (warp == 1) {
     tmem_alloc<CG>(saddr(&ctl->tmem_base), TMEM_COLS);
@@ -547,48 +591,66 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         atomicCAS(status, 0u, (uint32_t)MOE_ERR_DEVICE_INPUT);
         row_ok = false;
       }
+      // A half tile whose 128 rows all lie inside its expert's row range
+      // (alignment padding included, which no reader uses) leaves through a
+      // staged TMA store; otherwise each thread stores its own row if valid.
+      const long long row0 = (long long)row_off[e] + first;
+      const bool staged =
+          rows > 0 && row0 >= 0 && row0 + BM <= row_off[e + 1] && row0 + BM <= R_max;
       __nv_bfloat16* orow = out + (row_ok ? grow : 0) * (long long)N_out;
       const uint32_t t0 = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * UMMA_N);
-      if (MODE == 0) {
+      constexpr int CHUNKS = (MODE == 0) ? 2 : 4;   // 64 output columns each
 #pragma unroll 1
-        for (int c = 0; c < 2; ++c) {   // 64 h columns: gate in [c*64, +64), up in [128 + c*64, +64)
+      for (int c = 0; c < CHUNKS; ++c) {
+        uint4 o[8];
+        if (MODE == 0) {   // gate in TMEM columns [c*64, +64), up in [128 + c*64, +64)
           uint32_t g[64], u[64];
           tmem_ld64(t0 + (uint32_t)(c * 64), g);
           tmem_ld64(t0 + 128u + (uint32_t)(c * 64), u);
           tmem_ld_wait();
-          const int col = n * BN_OUT + c * 64;
-          if (row_ok && col < N_out) {   // N_out % 64 == 0: a chunk is all in or all out
-            uint4* dst = reinterpret_cast<uint4*>(orow + col);
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              uint4 o;
-              o.x = pack_bf16x2(silu_mul(g[8 * v + 0], u[8 * v + 0]), silu_mul(g[8 * v + 1], u[8 * v + 1]));
-              o.y = pack_bf16x2(silu_mul(g[8 * v + 2], u[8 * v + 2]), silu_mul(g[8 * v + 3], u[8 * v + 3]));
-              o.z = pack_bf16x2(silu_mul(g[8 * v + 4], u[8 * v + 4]), silu_mul(g[8 * v + 5], u[8 * v + 5]));
-              o.w = pack_bf16x2(silu_mul(g[8 * v + 6], u[8 * v + 6]), silu_mul(g[8 * v + 7], u[8 * v + 7]));
-              dst[v] = o;
-            }
+          for (int v = 0; v < 8; ++v) {
+            o[v].x = pack_bf16x2(silu_mul(g[8 * v + 0], u[8 * v + 0]), silu_mul(g[8 * v + 1], u[8 * v + 1]));
+            o[v].y = pack_bf16x2(silu_mul(g[8 * v + 2], u[8 * v + 2]), silu_mul(g[8 * v + 3], u[8 * v + 3]));
+            o[v].z = pack_bf16x2(silu_mul(g[8 * v + 4], u[8 * v + 4]), silu_mul(g[8 * v + 5], u[8 * v + 5]));
+            o[v].w = pack_bf16x2(silu_mul(g[8 * v + 6], u[8 * v + 6]), silu_mul(g[8 * v + 7], u[8 * v + 7]));
           }
-        }
-      } else {
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {   // 64 y columns per chunk
+        } else {
           uint32_t a[64];
           tmem_ld64(t0 + (uint32_t)(c * 64), a);
           tmem_ld_wait();
-          const int col = n * BN_OUT + c * 64;
-          if (row_ok && col < N_out) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + col);
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              uint4 o;
-              o.x = pack_bf16x2(__uint_as_float(a[8 * v + 0]), __uint_as_float(a[8 * v + 1]));
-              o.y = pack_bf16x2(__uint_as_float(a[8 * v + 2]), __uint_as_float(a[8 * v + 3]));
-              o.z = pack_bf16x2(__uint_as_float(a[8 * v + 4]), __uint_as_float(a[8 * v + 5]));
-              o.w = pack_bf16x2(__uint_as_float(a[8 * v + 6]), __uint_as_float(a[8 * v + 7]));
-              dst[v] = o;
-            }
+          for (int v = 0; v < 8; ++v) {
+            o[v].x = pack_bf16x2(__uint_as_float(a[8 * v + 0]), __uint_as_float(a[8 * v + 1]));
+            o[v].y = pack_bf16x2(__uint_as_float(a[8 * v + 2]), __uint_as_float(a[8 * v + 3]));
+            o[v].z = pack_bf16x2(__uint_as_float(a[8 * v + 4]), __uint_as_float(a[8 * v + 5]));
+            o[v].w = pack_bf16x2(__uint_as_float(a[8 * v + 6]), __uint_as_float(a[8 * v + 7]));
           }
+        }
+        const int col = n * BN_OUT + c * 64;
+        if (col >= N_out) continue;   // N_out % 64 == 0: a chunk is all in or all out
+        if (staged) {
+          if (threadIdx.x == 64) bulk_wait_read_all();   // the previous box has left smem
+          epilogue_bar();
+          // row r_in of the box, 16-byte chunk v at position v ^ (r_in % 8):
+          // the 128-byte swizzle the output tensor map uses
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const uint32_t a = staging + (uint32_t)(r_in * 128 + ((v ^ (r_in & 7)) << 4));
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(o[v].x),
+                         "r"(o[v].y), "r"(o[v].z), "r"(o[v].w)
+                         : "memory");
+          }
+          fence_proxy_async_smem();
+          epilogue_bar();
+          if (threadIdx.x == 64) {
+            tma_store_2d(&tmOut, col, (int)row0, staging);
+            bulk_commit();
+          }
+        } else if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + col);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) dst[v] = o[v];
         }
       }
       tc_fence_before();
@@ -598,6 +660,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         if (CG == 2) mbar_arrive_cluster(tb); else mbar_arrive_local(tb);
       }
     }
+    if (threadIdx.x == 64) bulk_wait_all();   // staged stores complete before the CTA exits
   }
 
   tc_fence_before();
@@ -676,11 +739,12 @@ template <int CG>
 moe_status_t launch_mlp(const moe_config_t& c, const void* xp, const int32_t* offsets,
                         const int32_t* counts, const void* w_gu, const void* w_d, void* h,
                         void* y, int64_t R_max, uint32_t* status, cudaStream_t s) {
-  CUtensorMap mx, mwgu, mh, mwd;
+  CUtensorMap mx, mwgu, mh, mwd, my;
   if (!make_map(&mx, xp, (uint64_t)c.H, (uint64_t)R_max) ||
       !make_map(&mwgu, w_gu, (uint64_t)c.H, (uint64_t)c.E * 2 * c.F) ||
       !make_map(&mh, h, (uint64_t)c.F, (uint64_t)R_max) ||
-      !make_map(&mwd, w_d, (uint64_t)c.F, (uint64_t)c.E * c.H))
+      !make_map(&mwd, w_d, (uint64_t)c.F, (uint64_t)c.E * c.H) ||
+      !make_map(&my, y, (uint64_t)c.H, (uint64_t)R_max))
     return MOE_ERR_CUDA;
   const size_t smem = smem_bytes<CG>(c.E);
   if (cudaFuncSetAttribute(tc_grouped_gemm<0, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -697,12 +761,12 @@ moe_status_t launch_mlp(const moe_config_t& c, const void* xp, const int32_t* of
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
   fill_launch<0, CG>(cfg, attr, g0, smem, s);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, tc_grouped_gemm<0, CG>, mx, mwgu,
+  cudaError_t e = cudaLaunchKernelEx(&cfg, tc_grouped_gemm<0, CG>, mx, mwgu, mh,
                                      static_cast<__nv_bfloat16*>(h), c.F, c.H, 2 * c.F, c.F,
                                      offsets, counts, c.E, c.capacity, (long long)R_max, status);
   if (e == cudaSuccess) {
     fill_launch<1, CG>(cfg, attr, g1, smem, s);
-    e = cudaLaunchKernelEx(&cfg, tc_grouped_gemm<1, CG>, mh, mwd, static_cast<__nv_bfloat16*>(y),
+    e = cudaLaunchKernelEx(&cfg, tc_grouped_gemm<1, CG>, mh, mwd, my, static_cast<__nv_bfloat16*>(y),
                            c.H, c.F, c.H, 128, offsets, counts, c.E, c.capacity,
                            (long long)R_max, status);
   }

@@ -188,7 +188,8 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
  *   w_gu           [E,2F,H] act: rows 0..F-1 are Wg_e, rows F..2F-1 are Wu_e.
  *   w_d            [E,H,F] act.
  *   h              [R_max,F] act out (scratch for the second GEMM), y [R_max,H] act out.
- *   Rows outside every expert's kept range are not written.
+ *   Rows outside every expert's kept range hold unspecified values afterwards
+ *   (an expert's alignment padding rows may be written; no reader uses them).
  *   ws, ws_bytes   any workspace with a status word (at least 256 bytes).
  * bf16 runs on tcgen05 tensor cores (TMA-fed persistent grouped GEMM); fp32 runs
  * on a CUDA-core FFMA grouped GEMM (fp32 inputs, no TF32). */
