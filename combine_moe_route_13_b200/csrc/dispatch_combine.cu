@@ -32,6 +32,8 @@ dispatch_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ token_s
   __shared__ int s_any;
   const int t = blockIdx.x;
   if (threadIdx.x == 0) s_any = 0;
+  pdl_wait();
+  pdl_trigger();
   __syncthreads();
   if (threadIdx.x < K) {
     const int s = token_slot[(size_t)t * K + threadIdx.x];
@@ -83,6 +85,8 @@ combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ token_sl
   __shared__ int s_slot[MAX_K];
   __shared__ float s_w[MAX_K];
   const int t = blockIdx.x;
+  pdl_wait();
+  pdl_trigger();
   if (threadIdx.x < K) {
     s_slot[threadIdx.x] = token_slot[(size_t)t * K + threadIdx.x];
     s_w[threadIdx.x] = topk_w[(size_t)t * K + threadIdx.x];
@@ -157,9 +161,8 @@ cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t*
                             cudaStream_t s) {
   if (c.T == 0) return cudaSuccess;
   const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
-  dispatch_kernel<<<c.T, DC_THREADS, 0, s>>>(static_cast<const uint4*>(x), slot,
-                                             static_cast<uint4*>(xp), c.K, row_vecs);
-  return cudaGetLastError();
+  return launch_pdl(dispatch_kernel, dim3(c.T), dim3(DC_THREADS), 0, s,
+                    static_cast<const uint4*>(x), slot, static_cast<uint4*>(xp), c.K, row_vecs);
 }
 
 cudaError_t launch_combine(const moe_config_t& c, const void* y, const int32_t* slot,
@@ -167,12 +170,11 @@ cudaError_t launch_combine(const moe_config_t& c, const void* y, const int32_t* 
   if (c.T == 0) return cudaSuccess;
   const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
   if (c.act_dtype == MOE_BF16)
-    combine_kernel<true><<<c.T, DC_THREADS, 0, s>>>(static_cast<const uint4*>(y), slot, w,
-                                                    static_cast<uint4*>(out), c.K, row_vecs);
-  else
-    combine_kernel<false><<<c.T, DC_THREADS, 0, s>>>(static_cast<const uint4*>(y), slot, w,
-                                                     static_cast<uint4*>(out), c.K, row_vecs);
-  return cudaGetLastError();
+    return launch_pdl(combine_kernel<true>, dim3(c.T), dim3(DC_THREADS), 0, s,
+                      static_cast<const uint4*>(y), slot, w, static_cast<uint4*>(out), c.K,
+                      row_vecs);
+  return launch_pdl(combine_kernel<false>, dim3(c.T), dim3(DC_THREADS), 0, s,
+                    static_cast<const uint4*>(y), slot, w, static_cast<uint4*>(out), c.K, row_vecs);
 }
 
 }  // namespace moe

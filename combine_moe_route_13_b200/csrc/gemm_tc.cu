@@ -451,12 +451,13 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     prefetch_map(&tmA);
     prefetch_map(&tmB);
     prefetch_map(&tmOut);
-    row_off[E] = offsets[E];
   }
   if (warp == 1) {
     tmem_alloc<CG>(saddr(&ctl->tmem_base), TMEM_COLS);
     tmem_relinquish<CG>();
   }
+  pdl_wait();      // everything above touched only this CTA's shared memory and TMEM
+  pdl_trigger();
   {  // per-expert kept rows, first row and M-tile prefix (block scan)
     const int chunk = (E + NUM_THREADS - 1) / NUM_THREADS;
     const int e0 = threadIdx.x * chunk;
@@ -487,7 +488,10 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         run += (kept_s[e] + CF::TILE_ROWS - 1) / CF::TILE_ROWS;
       }
     }
-    if (threadIdx.x == NUM_THREADS - 1) P[E] = run;
+    if (threadIdx.x == NUM_THREADS - 1) {
+      P[E] = run;
+      row_off[E] = offsets[E];
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -714,8 +718,10 @@ void fill_launch(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr, int grid, s
   attr[0].val.clusterDim.x = CG;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
 }
 
 // Co-resident CTAs (CG = 1) or 2-CTA clusters (CG = 2) of the kernel on this device.
@@ -727,8 +733,9 @@ int resident_units(size_t smem) {
     return 0;
   if (CG == 1) return sms;
   cudaLaunchConfig_t q;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   fill_launch<0, CG>(q, attr, sms & ~1, smem, nullptr);
+  q.numAttrs = 1;   // the cluster shape only
   int clusters = 0;
   if (cudaOccupancyMaxActiveClusters(&clusters, tc_grouped_gemm<0, CG>, &q) != cudaSuccess)
     return 0;
@@ -759,7 +766,7 @@ moe_status_t launch_mlp(const moe_config_t& c, const void* xp, const int32_t* of
   const int g0 = (int)std::min<int64_t>(units, t0) * CG;
   const int g1 = (int)std::min<int64_t>(units, t1) * CG;
   cudaLaunchConfig_t cfg;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   fill_launch<0, CG>(cfg, attr, g0, smem, s);
   cudaError_t e = cudaLaunchKernelEx(&cfg, tc_grouped_gemm<0, CG>, mx, mwgu, mh,
                                      static_cast<__nv_bfloat16*>(h), c.F, c.H, 2 * c.F, c.F,

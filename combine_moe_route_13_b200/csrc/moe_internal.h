@@ -3,6 +3,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 
 #include <cuda_runtime.h>
 
@@ -35,6 +36,35 @@ struct WsLayout {
 };
 
 WsLayout ws_layout(const moe_config_t& c);
+
+// Programmatic dependent launch. Every kernel of the layer is launched with
+// programmatic stream serialization, so its launch and on-chip prologue may
+// overlap the tail of the kernel before it in the stream. Each such kernel
+// calls pdl_wait() before its first global-memory access (read or write: the
+// previous kernel may still be reading a buffer this one overwrites) and
+// pdl_trigger() to let its own successor launch early.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+#ifdef __CUDACC__
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+#endif
 int64_t max_rows(const moe_config_t& c);
 moe_status_t validate(const moe_config_t* c, bool need_mlp);
 

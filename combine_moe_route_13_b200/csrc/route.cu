@@ -73,6 +73,8 @@ route_topk_kernel(const float* __restrict__ logits, int T, int E, int K,
   const int tb0 = blockIdx.x * ROUTE_TB;
   const int ntok = min(ROUTE_TB, T - tb0);
   for (int i = threadIdx.x; i < E * WORDS; i += blockDim.x) bitmap[i] = 0u;
+  pdl_wait();
+  pdl_trigger();
   __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -154,6 +156,8 @@ route_topk_kernel(const float* __restrict__ logits, int T, int E, int K,
 __global__ void __launch_bounds__(1024)
 route_scan_kernel(int nblk, int E, int C, int32_t* __restrict__ blk_cnt,
                   int32_t* __restrict__ counts, int32_t* __restrict__ overflow) {
+  pdl_wait();
+  pdl_trigger();
   const int e = blockIdx.x * 32 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (e >= E) return;
@@ -248,6 +252,8 @@ route_slot_kernel(int T, int K, int E, int S, int C, int A, int nblk, int64_t R_
   __shared__ int off_s[MAX_E + 1];
   __shared__ int kept_s[MAX_E];
   __shared__ int warp_tmp[16];
+  pdl_wait();
+  pdl_trigger();
   int sum_kept;
   expert_offsets_smem(E, C, A, counts, off_s, kept_s, warp_tmp, sum_kept);
   const int64_t TK = (int64_t)T * K;
@@ -291,12 +297,13 @@ route_slot_kernel(int T, int K, int E, int S, int C, int A, int nblk, int64_t R_
 }
 
 template <int VPL>
-void launch_topk(int nblk, size_t smem, cudaStream_t s, const float* logits, int T, int E, int K,
+cudaError_t launch_topk(int nblk, size_t smem, cudaStream_t s, const float* logits, int T, int E, int K,
                  int32_t* idx, float* w, int32_t* rank, int32_t* blk) {
   // 32 warps (4 tokens each) while the register budget allows: 16 warps for
   // E > 256, 8 for E > 512
   constexpr int THREADS = VPL >= 32 ? 256 : (VPL >= 16 ? 512 : 1024);
-  route_topk_kernel<VPL, THREADS><<<nblk, THREADS, smem, s>>>(logits, T, E, K, idx, w, rank, blk);
+  return launch_pdl(route_topk_kernel<VPL, THREADS>, dim3(nblk), dim3(THREADS), smem, s, logits, T,
+                    E, K, idx, w, rank, blk);
 }
 
 }  // namespace
@@ -309,21 +316,23 @@ cudaError_t launch_route(const moe_config_t& c, const float* logits, int32_t* to
   if (nblk > 0) {
     const size_t smem = (size_t)c.E * WORDS * 4 + (size_t)ROUTE_TB * c.K * 4;
     const int vpl = (int)ceil_div(c.E, 32);
-    if (vpl <= 1) launch_topk<1>(nblk, smem, s, logits, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
-    else if (vpl <= 2) launch_topk<2>(nblk, smem, s, logits, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
-    else if (vpl <= 4) launch_topk<4>(nblk, smem, s, logits, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
-    else if (vpl <= 8) launch_topk<8>(nblk, smem, s, logits, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
-    else if (vpl <= 16) launch_topk<16>(nblk, smem, s, logits, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
-    else launch_topk<32>(nblk, smem, s, logits, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
+    cudaError_t e;
+    if (vpl <= 1) e = launch_topk<1>(nblk, smem, s, logits, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
+    else if (vpl <= 2) e = launch_topk<2>(nblk, smem, s, logits, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
+    else if (vpl <= 4) e = launch_topk<4>(nblk, smem, s, logits, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
+    else if (vpl <= 8) e = launch_topk<8>(nblk, smem, s, logits, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
+    else if (vpl <= 16) e = launch_topk<16>(nblk, smem, s, logits, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
+    else e = launch_topk<32>(nblk, smem, s, logits, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
+    if (e != cudaSuccess) return e;
   }
-  route_scan_kernel<<<(unsigned)ceil_div(c.E, 32), 1024, 0, s>>>(nblk, c.E, c.capacity, blk_cnt,
-                                                                 counts, overflow);
+  cudaError_t e = launch_pdl(route_scan_kernel, dim3((unsigned)ceil_div(c.E, 32)), dim3(1024), 0, s,
+                             nblk, c.E, c.capacity, blk_cnt, counts, overflow);
+  if (e != cudaSuccess) return e;
   const int64_t work = std::max<int64_t>((int64_t)c.T * c.K, R_max);
   int grid = (int)std::min<int64_t>(std::max<int64_t>(ceil_div(work, 256), 1), 148 * 8);
-  route_slot_kernel<<<grid, 256, 0, s>>>(c.T, c.K, c.E, c.S, c.capacity, c.row_align, nblk, R_max,
-                                         topk_idx, blk_cnt, counts, offsets, segoff, totals, slot,
-                                         row_src);
-  return cudaGetLastError();
+  return launch_pdl(route_slot_kernel, dim3(grid), dim3(256), 0, s, c.T, c.K, c.E, c.S, c.capacity,
+                    c.row_align, nblk, R_max, (const int32_t*)topk_idx, (const int32_t*)blk_cnt,
+                    (const int32_t*)counts, offsets, segoff, totals, slot, row_src);
 }
 
 }  // namespace moe
