@@ -56,6 +56,23 @@ def load_peaks():
     return p
 
 
+def measured_traffic(workload: str):
+    """DRAM bytes per moe_expert_mlp call from the committed ncu capture of this
+    workload, or None when there is none or the GEMM source changed since."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(workload)
+        if not rec:
+            return None
+        with open(os.path.join(ROOT, rec["kernel_source"]), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+        return rec["traffic_bytes"] if sha.startswith(rec["sha256_prefix"]) else None
+    except (OSError, ValueError, KeyError):
+        return None
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -423,7 +440,9 @@ def main(argv=None):
         "roofline": {"bound": "tensor", "kernel": "expert_mlp (gate/up + down grouped GEMMs)",
                      "achieved": mlp_tflops, "peak": tensor_peak, "unit": "TFLOP/s",
                      "frac": mlp_tflops / tensor_peak,
-                     "peak_kind": f"bf16_tflops_sustained ({peaks['source']})", "traffic": None},
+                     "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
+                     "traffic": measured_traffic(wl.name),
+                     "traffic_unit": "bytes per moe_expert_mlp call (ncu dram read+write)"},
         "kernels": kernels,
         "effective_tokens_per_s": world * alg["N"] / (ms / 1e3),
         "clocks": clk,
