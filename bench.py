@@ -159,9 +159,10 @@ def flush_l2(buf: torch.Tensor):
 class Layer:
     """Device-resident inputs, weights and workspace of one replica."""
 
-    def __init__(self, wl: W.Workload, seed: int, device):
+    def __init__(self, wl: W.Workload, seed: int, device, overlap: bool = False):
         import combine_moe_route_13_b200 as M
         self.M = M
+        self.flags = M.MOE_FLAG_OVERLAP if overlap else M.MOE_FLAG_NONE
         self.wl = wl
         self.C = M.moe_capacity(wl.T, wl.K, wl.E, wl.cf)
         self.cfg = M.make_config(wl.T, wl.H, wl.E, wl.K, wl.F, wl.S, self.C, wl.row_align, wl.act)
@@ -175,7 +176,8 @@ class Layer:
 
     def forward(self):
         self.aux = self.M.moe_layer_forward(self.cfg, self.inp["logits"], self.inp["x"],
-                                            self.inp["w_gu"], self.inp["w_d"], self.out, self.ws)
+                                            self.inp["w_gu"], self.inp["w_d"], self.out, self.ws,
+                                            flags=self.flags)
 
     def views(self):
         return self.M.layer_views(self.cfg, self.ws, self.aux)
@@ -239,7 +241,8 @@ def e2e_steps(layer: Layer, steps, warmup, flush_buf, stream):
     def step():
         d_logits.copy_(h_logits, non_blocking=True)
         d_x.copy_(h_x, non_blocking=True)
-        M.moe_layer_forward(cfg, d_logits, d_x, inp["w_gu"], inp["w_d"], layer.out, layer.ws)
+        M.moe_layer_forward(cfg, d_logits, d_x, inp["w_gu"], inp["w_d"], layer.out, layer.ws,
+                            flags=layer.flags)
         h_out.copy_(layer.out, non_blocking=True)
 
     times = time_steps(step, steps, warmup, flush_buf, stream)
@@ -344,6 +347,8 @@ def main(argv=None):
     ap.add_argument("--cpu-tokens", type=int, default=256,
                     help="tokens of the CPU-oracle sample per step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--overlap", action="store_true",
+                    help="overlap the combine with the down GEMM (MOE_FLAG_OVERLAP)")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         raise SystemExit("--warmup must be >= 3")
@@ -360,7 +365,7 @@ def main(argv=None):
     torch.cuda.set_device(device)
     peaks = load_peaks()
 
-    layer = Layer(wl, seed=rank, device=device)
+    layer = Layer(wl, seed=rank, device=device, overlap=args.overlap)
     flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream()
 
@@ -433,7 +438,8 @@ def main(argv=None):
         "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "K": wl.K, "F": wl.F,
                    "S": wl.S, "cf": wl.cf, "capacity": layer.C, "row_align": wl.row_align,
                    "effective_tokens": alg["N"], "overflow": int(totals[2]),
-                   "l2": "flushed (256 MB write) before every step", "parallelism": f"replicas{world}"},
+                   "l2": "flushed (256 MB write) before every step", "parallelism": f"replicas{world}",
+                   "overlap": bool(args.overlap)},
         "e2e": {"value": world * wl.T / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": KERNELS_PER_STEP * args.steps,

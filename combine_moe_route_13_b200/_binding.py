@@ -26,12 +26,13 @@ MOE_ERR_DEVICE_INPUT = 6
 MOE_F32 = 0
 MOE_BF16 = 1
 MOE_FLAG_NONE = 0
+MOE_FLAG_OVERLAP = 1
 
 # every symbol declared in include/moe.h
 EXPORTS = ("moe_capacity", "moe_max_rows", "moe_check_config", "moe_route_workspace_bytes",
            "moe_workspace_bytes", "moe_workspace_init", "moe_route_topk", "moe_dispatch",
            "moe_expert_mlp", "moe_combine", "moe_layer_forward", "moe_get_device_status",
-           "moe_status_string", "moe_version", "moe_route_topk_noalloc")
+           "moe_status_string", "moe_version", "moe_route_topk_noalloc", "moe_combine_wait")
 
 
 class MoeError(RuntimeError):
@@ -82,6 +83,8 @@ def _load():
         "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "moe_version": (ctypes.c_int32, []),
         "moe_route_topk_noalloc": (ctypes.c_int, [_CFG] + [_P] * 10 + [_P]),
+        "moe_combine_wait": (ctypes.c_int, [_CFG, _P, _P, _P, _P, ctypes.c_uint32, _P,
+                                            ctypes.c_uint32, _P, ctypes.c_size_t, _P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -207,6 +210,21 @@ def moe_combine(cfg, y, token_slot, topk_w, out, stream=None):
                            _ptr(token_slot, torch.int32, "token_slot"),
                            _ptr(topk_w, torch.float32, "topk_w"), _ptr(out, dt, "out"),
                            _stream(stream)), "moe_combine")
+
+
+def moe_combine_wait(cfg, y, token_slot, topk_w, row_ready, ready_target, out, ws,
+                     timeout_us=2_000_000, stream=None):
+    dt = act_dtype(cfg)
+    _check(LIB.moe_combine_wait(
+        ctypes.byref(cfg), _ptr(y, dt, "y"), _ptr(token_slot, torch.int32, "token_slot"),
+        _ptr(topk_w, torch.float32, "topk_w"), _ptr(row_ready, (torch.int32, torch.uint32), "row_ready"),
+        int(ready_target), _ptr(out, dt, "out"), int(timeout_us), _ptr(ws, name="ws"),
+        ws.numel() * ws.element_size(), _stream(stream)), "moe_combine_wait")
+
+
+def ready_target(cfg: MoeConfig) -> int:
+    """Counter value at which a 128-row block of y is final (the down GEMM's N tiles)."""
+    return (cfg.H + 255) // 256
 
 
 def moe_layer_forward(cfg, logits, x, w_gu, w_d, out, ws, flags=MOE_FLAG_NONE, stream=None):

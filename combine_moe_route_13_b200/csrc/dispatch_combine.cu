@@ -155,6 +155,126 @@ combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ token_sl
   }
 }
 
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// The consumer half of the tile-signalled overlap ("Mixture-of-Experts
+// acceleration through overlap": tile-ready flags published by the GEMM,
+// consumed by a separate kernel as soon as they are set). Same arithmetic as
+// combine_kernel, but instead of waiting for the previous kernel to finish, a
+// token waits until the ready counter of the 128-row block of each of its
+// kept rows has reached `target` (acquire). The wait is bounded: after
+// `timeout_ns`, or once any block has given up, the block records
+// MOE_ERR_TIMEOUT and leaves its token's output unwritten.
+template <bool BF16>
+__global__ void __launch_bounds__(DC_THREADS)
+combine_wait_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ token_slot,
+                    const float* __restrict__ topk_w, uint4* __restrict__ out, int K,
+                    int row_vecs, const uint32_t* row_ready, uint32_t target,
+                    unsigned long long timeout_ns, uint32_t* status) {
+  __shared__ int s_slot[MAX_K];
+  __shared__ float s_w[MAX_K];
+  __shared__ int s_ok;
+  pdl_trigger();   // no griddepcontrol.wait: the ready counters carry the dependency
+  const int t = blockIdx.x;
+  if (threadIdx.x < K) {
+    s_slot[threadIdx.x] = token_slot[(size_t)t * K + threadIdx.x];
+    s_w[threadIdx.x] = topk_w[(size_t)t * K + threadIdx.x];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    const unsigned long long t0 = globaltimer();
+    for (int k = 0; k < K && ok; ++k) {
+      const int sl = s_slot[k];
+      if (sl < 0) continue;
+      const uint32_t* flag = row_ready + sl / READY_ROWS;
+      unsigned sleep_ns = 32;
+      while (ld_acquire(flag) < target) {
+        if (*(volatile uint32_t*)status != 0u || globaltimer() - t0 > timeout_ns) {
+          atomicCAS(status, 0u, (uint32_t)MOE_ERR_TIMEOUT);
+          ok = 0;
+          break;
+        }
+        __nanosleep(sleep_ns);
+        if (sleep_ns < 2048) sleep_ns *= 2;
+      }
+    }
+    s_ok = ok;
+  }
+  __syncthreads();
+  if (!s_ok) return;
+  constexpr int LANES = BF16 ? 8 : 4;
+  uint4* dst = out + (size_t)t * row_vecs;
+  for (int v0 = threadIdx.x; v0 < row_vecs; v0 += DC_THREADS * 2) {
+    float acc[2][LANES];
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int i = 0; i < LANES; ++i) acc[u][i] = 0.f;
+    for (int k = 0; k < K; k += 4) {
+      uint4 d[4][2];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int sl = (k + j < K) ? s_slot[k + j] : -1;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int v = v0 + u * DC_THREADS;
+          // coherent loads: these rows were written while this kernel ran
+          if (sl >= 0 && v < row_vecs) d[j][u] = y[(size_t)sl * row_vecs + v];
+          else d[j][u] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (k + j >= K || s_slot[k + j] < 0) continue;
+        const float wk = s_w[k + j];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (BF16) {
+            float f[8];
+            unpack_bf16x8(d[j][u], f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[u][i] = fmaf(wk, f[i], acc[u][i]);
+          } else {
+            acc[u][0] = fmaf(wk, __uint_as_float(d[j][u].x), acc[u][0]);
+            acc[u][1] = fmaf(wk, __uint_as_float(d[j][u].y), acc[u][1]);
+            acc[u][2] = fmaf(wk, __uint_as_float(d[j][u].z), acc[u][2]);
+            acc[u][3] = fmaf(wk, __uint_as_float(d[j][u].w), acc[u][3]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int v = v0 + u * DC_THREADS;
+      if (v >= row_vecs) continue;
+      uint4 o;
+      if (BF16) {
+        o.x = pack_bf16x2(acc[u][0], acc[u][1]);
+        o.y = pack_bf16x2(acc[u][2], acc[u][3]);
+        o.z = pack_bf16x2(acc[u][4], acc[u][5]);
+        o.w = pack_bf16x2(acc[u][6], acc[u][7]);
+      } else {
+        o.x = __float_as_uint(acc[u][0]);
+        o.y = __float_as_uint(acc[u][1]);
+        o.z = __float_as_uint(acc[u][2]);
+        o.w = __float_as_uint(acc[u][3]);
+      }
+      __stcs(dst + v, o);
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t* slot, void* xp,
@@ -175,6 +295,21 @@ cudaError_t launch_combine(const moe_config_t& c, const void* y, const int32_t* 
                       row_vecs);
   return launch_pdl(combine_kernel<false>, dim3(c.T), dim3(DC_THREADS), 0, s,
                     static_cast<const uint4*>(y), slot, w, static_cast<uint4*>(out), c.K, row_vecs);
+}
+
+cudaError_t launch_combine_wait(const moe_config_t& c, const void* y, const int32_t* slot,
+                                const float* w, const uint32_t* row_ready, uint32_t target,
+                                unsigned long long timeout_ns, uint32_t* status, void* out,
+                                cudaStream_t s) {
+  if (c.T == 0) return cudaSuccess;
+  const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
+  if (c.act_dtype == MOE_BF16)
+    return launch_pdl(combine_wait_kernel<true>, dim3(c.T), dim3(DC_THREADS), 0, s,
+                      static_cast<const uint4*>(y), slot, w, static_cast<uint4*>(out), c.K,
+                      row_vecs, row_ready, target, timeout_ns, status);
+  return launch_pdl(combine_wait_kernel<false>, dim3(c.T), dim3(DC_THREADS), 0, s,
+                    static_cast<const uint4*>(y), slot, w, static_cast<uint4*>(out), c.K,
+                    row_vecs, row_ready, target, timeout_ns, status);
 }
 
 }  // namespace moe

@@ -232,6 +232,17 @@ __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+// Order this thread's completed async-proxy (TMA) global writes before its
+// later generic-proxy accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// counter += 1 with release semantics at GPU scope.
+__device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // Make this thread's generic-proxy shared-memory writes visible to TMA.
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -413,7 +424,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 int N_out, int Kdim, int b_rows_per_expert,
                 int b_second_off, const int32_t* __restrict__ offsets,
                 const int32_t* __restrict__ counts, int E, int C, long long R_max,
-                uint32_t* __restrict__ status) {
+                uint32_t* __restrict__ status, uint32_t* __restrict__ row_ready) {
   using CF = Cfg<CG>;
   constexpr int STAGES = CF::STAGES;
   constexpr int BN_OUT = (MODE == 0) ? 128 : 256;   // output columns per tile
@@ -663,6 +674,19 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         const uint32_t tb = tempty_leader0 + (uint32_t)(b * sizeof(uint64_t));
         if (CG == 2) mbar_arrive_cluster(tb); else mbar_arrive_local(tb);
       }
+      if (row_ready != nullptr && rows > 0) {
+        // Publish this half tile: its 128 rows (one ready block: the rows are
+        // aligned to 128) have one more N tile stored. The staged TMA stores
+        // are waited for by their issuing thread and every thread fences its
+        // own stores before the barrier; the count is added with release.
+        __threadfence();
+        if (threadIdx.x == 64) {
+          bulk_wait_all();
+          fence_proxy_async_global();
+        }
+        epilogue_bar();
+        if (threadIdx.x == 64) red_release_add(row_ready + (row0 / READY_ROWS), 1u);
+      }
     }
     if (threadIdx.x == 64) bulk_wait_all();   // staged stores complete before the CTA exits
   }
@@ -745,7 +769,8 @@ int resident_units(size_t smem) {
 template <int CG>
 moe_status_t launch_mlp(const moe_config_t& c, const void* xp, const int32_t* offsets,
                         const int32_t* counts, const void* w_gu, const void* w_d, void* h,
-                        void* y, int64_t R_max, uint32_t* status, cudaStream_t s) {
+                        void* y, int64_t R_max, uint32_t* status, cudaStream_t s,
+                        uint32_t* row_ready) {
   CUtensorMap mx, mwgu, mh, mwd, my;
   if (!make_map(&mx, xp, (uint64_t)c.H, (uint64_t)R_max) ||
       !make_map(&mwgu, w_gu, (uint64_t)c.H, (uint64_t)c.E * 2 * c.F) ||
@@ -770,12 +795,13 @@ moe_status_t launch_mlp(const moe_config_t& c, const void* xp, const int32_t* of
   fill_launch<0, CG>(cfg, attr, g0, smem, s);
   cudaError_t e = cudaLaunchKernelEx(&cfg, tc_grouped_gemm<0, CG>, mx, mwgu, mh,
                                      static_cast<__nv_bfloat16*>(h), c.F, c.H, 2 * c.F, c.F,
-                                     offsets, counts, c.E, c.capacity, (long long)R_max, status);
+                                     offsets, counts, c.E, c.capacity, (long long)R_max, status,
+                                     (uint32_t*)nullptr);
   if (e == cudaSuccess) {
     fill_launch<1, CG>(cfg, attr, g1, smem, s);
     e = cudaLaunchKernelEx(&cfg, tc_grouped_gemm<1, CG>, mh, mwd, my, static_cast<__nv_bfloat16*>(y),
                            c.H, c.F, c.H, 128, offsets, counts, c.E, c.capacity,
-                           (long long)R_max, status);
+                           (long long)R_max, status, row_ready);
   }
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -785,15 +811,15 @@ moe_status_t launch_mlp(const moe_config_t& c, const void* xp, const int32_t* of
 moe_status_t launch_mlp_bf16_tc(const moe_config_t& c, const void* xp, const int32_t* offsets,
                                 const int32_t* counts, const void* w_gu, const void* w_d,
                                 void* h, void* y, int64_t R_max, uint32_t* status,
-                                cudaStream_t s) {
+                                cudaStream_t s, uint32_t* row_ready) {
   if (R_max == 0) return MOE_OK;
   // Tile shape from the expected rows per expert: 256-row pair tiles halve each
   // CTA's operand traffic but waste up to 255 padded rows per expert, so small
   // experts (decode-like batches) use 128-row single-CTA tiles.
   const int64_t rows_per_expert = std::min<int64_t>((int64_t)c.T * c.K, (int64_t)c.E * c.capacity) / c.E;
   if (rows_per_expert >= 192)
-    return tc::launch_mlp<2>(c, xp, offsets, counts, w_gu, w_d, h, y, R_max, status, s);
-  return tc::launch_mlp<1>(c, xp, offsets, counts, w_gu, w_d, h, y, R_max, status, s);
+    return tc::launch_mlp<2>(c, xp, offsets, counts, w_gu, w_d, h, y, R_max, status, s, row_ready);
+  return tc::launch_mlp<1>(c, xp, offsets, counts, w_gu, w_d, h, y, R_max, status, s, row_ready);
 }
 
 }  // namespace moe

@@ -60,6 +60,7 @@ WsLayout ws_layout(const moe_config_t& c) {
   L.totals = p;    p += align256(16);
   L.slot = p;      p += align256((size_t)TK * 4);
   L.row_src = p;   p += align256((size_t)R * 4);
+  L.row_ready = p; p += align256((size_t)ceil_div(R, READY_ROWS) * 4);
   L.xp = p;        p += align256((size_t)R * c.H * as);
   L.h = p;         p += align256((size_t)R * c.F * as);
   L.y = p;         p += align256((size_t)R * c.H * as);
@@ -188,12 +189,32 @@ moe_status_t moe_combine(const moe_config_t* cfg, const void* y, const int32_t* 
       launch_combine(*cfg, y, token_slot, topk_w, out, static_cast<cudaStream_t>(stream)));
 }
 
+moe_status_t moe_combine_wait(const moe_config_t* cfg, const void* y, const int32_t* token_slot,
+                              const float* topk_w, const uint32_t* row_ready,
+                              uint32_t ready_target, void* out, uint32_t timeout_us, void* ws,
+                              size_t ws_bytes, void* stream) {
+  moe_status_t st = validate(cfg, false);
+  if (st != MOE_OK) return st;
+  if (cfg->row_align % READY_ROWS != 0) return MOE_ERR_UNSUPPORTED;
+  if (cfg->T == 0) return MOE_OK;
+  if (!y || !token_slot || !topk_w || !row_ready || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < 256) return MOE_ERR_WORKSPACE;
+  return cuda_status(launch_combine_wait(*cfg, y, token_slot, topk_w, row_ready, ready_target,
+                                         (unsigned long long)timeout_us * 1000ull,
+                                         static_cast<uint32_t*>(ws), out,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
 moe_status_t moe_layer_forward(const moe_config_t* cfg, const float* logits, const void* x,
                                const void* w_gu, const void* w_d, void* out, uint32_t flags,
                                void* ws, size_t ws_bytes, moe_layer_aux_t* aux, void* stream) {
   moe_status_t st = validate(cfg, true);
   if (st != MOE_OK) return st;
-  if (flags != MOE_FLAG_NONE) return MOE_ERR_UNSUPPORTED;
+  if ((flags & ~MOE_FLAG_OVERLAP) != 0u) return MOE_ERR_UNSUPPORTED;
+  const bool overlap = (flags & MOE_FLAG_OVERLAP) != 0u;
+  if (overlap && (cfg->act_dtype != MOE_BF16 || cfg->row_align % READY_ROWS != 0))
+    return MOE_ERR_UNSUPPORTED;
   if (cfg->T > 0 && (!logits || !x || !out)) return MOE_ERR_INVALID_ARG;
   if (!w_gu || !w_d) return MOE_ERR_INVALID_ARG;
   const WsLayout L = ws_layout(*cfg);
@@ -213,17 +234,37 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const float* logits, con
   a.h = b + L.h;
   a.y = b + L.y;
   if (aux) *aux = a;
-  st = moe_route_topk(cfg, logits, a.topk_idx, a.topk_w, a.expert_counts, a.overflow,
-                      a.expert_offsets, a.segment_offsets, a.token_slot, a.row_src, a.totals, ws,
-                      ws_bytes, stream);
+  if (!overlap) {
+    st = moe_route_topk(cfg, logits, a.topk_idx, a.topk_w, a.expert_counts, a.overflow,
+                        a.expert_offsets, a.segment_offsets, a.token_slot, a.row_src, a.totals,
+                        ws, ws_bytes, stream);
+    if (st != MOE_OK) return st;
+    if (cfg->T == 0) return MOE_OK;
+    st = moe_dispatch(cfg, x, a.token_slot, a.xp, stream);
+    if (st != MOE_OK) return st;
+    st = moe_expert_mlp(cfg, a.xp, a.expert_offsets, a.expert_counts, w_gu, w_d, a.h, a.y, ws,
+                        ws_bytes, stream);
+    if (st != MOE_OK) return st;
+    return moe_combine(cfg, a.y, a.token_slot, a.topk_w, out, stream);
+  }
+  // Overlapped: the route also zeroes the ready counters, the down GEMM
+  // publishes them and the combine consumes them while the GEMM finishes.
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* ready = reinterpret_cast<uint32_t*>(b + L.row_ready);
+  uint32_t* status = static_cast<uint32_t*>(ws);
+  const int64_t R = max_rows(*cfg);
+  st = cuda_status(launch_route(*cfg, logits, a.topk_idx, a.topk_w, a.expert_counts, a.overflow,
+                                a.expert_offsets, a.segment_offsets, a.token_slot, a.row_src,
+                                a.totals, reinterpret_cast<int32_t*>(b + L.blk_cnt), R, s, ready));
   if (st != MOE_OK) return st;
   if (cfg->T == 0) return MOE_OK;
-  st = moe_dispatch(cfg, x, a.token_slot, a.xp, stream);
+  st = cuda_status(launch_dispatch(*cfg, x, a.token_slot, a.xp, s));
   if (st != MOE_OK) return st;
-  st = moe_expert_mlp(cfg, a.xp, a.expert_offsets, a.expert_counts, w_gu, w_d, a.h, a.y, ws,
-                      ws_bytes, stream);
+  st = launch_mlp_bf16_tc(*cfg, a.xp, a.expert_offsets, a.expert_counts, w_gu, w_d, a.h, a.y, R,
+                          status, s, ready);
   if (st != MOE_OK) return st;
-  return moe_combine(cfg, a.y, a.token_slot, a.topk_w, out, stream);
+  return cuda_status(launch_combine_wait(*cfg, a.y, a.token_slot, a.topk_w, ready,
+                                         ready_target(*cfg), WAIT_LIMIT_NS, status, out, s));
 }
 
 moe_status_t moe_get_device_status(void* ws, moe_status_t* status, void* stream) {

@@ -17,6 +17,10 @@ namespace moe {
 constexpr int ROUTE_TB = 128;
 constexpr int MAX_E = 1024;
 constexpr int MAX_K = 32;
+// Rows per ready counter of the overlapped combine (the GEMM half-tile height).
+constexpr int READY_ROWS = 128;
+// Bound of every wait in the kernels (ns).
+constexpr unsigned long long WAIT_LIMIT_NS = 2000000000ull;
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -30,7 +34,7 @@ struct WsLayout {
   size_t blk_cnt = 0;      // [nblk, E] int32: per-block histograms, then bases
   size_t route_end = 0;    // bytes needed by moe_route_topk
   size_t topk_idx = 0, topk_w = 0, counts = 0, overflow = 0, offsets = 0;
-  size_t segoff = 0, totals = 0, slot = 0, row_src = 0;
+  size_t segoff = 0, totals = 0, slot = 0, row_src = 0, row_ready = 0;
   size_t xp = 0, h = 0, y = 0;
   size_t total = 0;        // bytes needed by moe_layer_forward
 };
@@ -69,10 +73,13 @@ int64_t max_rows(const moe_config_t& c);
 moe_status_t validate(const moe_config_t* c, bool need_mlp);
 
 // ---- launchers (return cudaGetLastError() of their launches) ----
+// row_ready (optional): ceil(R_max / READY_ROWS) counters zeroed for the
+// overlapped combine.
 cudaError_t launch_route(const moe_config_t& c, const float* logits, int32_t* topk_idx,
                          float* topk_w, int32_t* counts, int32_t* overflow, int32_t* offsets,
                          int32_t* segoff, int32_t* slot, int32_t* row_src, int32_t* totals,
-                         int32_t* blk_cnt, int64_t R_max, cudaStream_t s);
+                         int32_t* blk_cnt, int64_t R_max, cudaStream_t s,
+                         uint32_t* row_ready = nullptr);
 
 cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t* slot, void* xp,
                             cudaStream_t s);
@@ -80,15 +87,28 @@ cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t*
 cudaError_t launch_combine(const moe_config_t& c, const void* y, const int32_t* slot,
                            const float* w, void* out, cudaStream_t s);
 
+// Combine that waits, token by token, for the ready counters of its rows to
+// reach `target` instead of for the previous kernel to finish.
+cudaError_t launch_combine_wait(const moe_config_t& c, const void* y, const int32_t* slot,
+                                const float* w, const uint32_t* row_ready, uint32_t target,
+                                unsigned long long timeout_ns, uint32_t* status, void* out,
+                                cudaStream_t s);
+
 // fp32 CUDA-core grouped SwiGLU (gate/up then down).
 cudaError_t launch_mlp_f32(const moe_config_t& c, const float* xp, const int32_t* offsets,
                            const int32_t* counts, const float* w_gu, const float* w_d, float* h,
                            float* y, int64_t R_max, cudaStream_t s);
 
 // bf16 tcgen05 grouped SwiGLU (gate/up then down). Returns a moe status.
+// row_ready (optional): the down GEMM adds 1 to the counter of a 128-row
+// block each time it has stored one of the block's N tiles (release), so
+// a block is final when its counter reaches ceil(H / 256).
 moe_status_t launch_mlp_bf16_tc(const moe_config_t& c, const void* xp, const int32_t* offsets,
                                 const int32_t* counts, const void* w_gu, const void* w_d,
                                 void* h, void* y, int64_t R_max, uint32_t* status,
-                                cudaStream_t s);
+                                cudaStream_t s, uint32_t* row_ready = nullptr);
+
+// Ready-counter target of the down GEMM (its number of N tiles).
+inline uint32_t ready_target(const moe_config_t& c) { return (uint32_t)ceil_div(c.H, 256); }
 
 }  // namespace moe

@@ -248,7 +248,8 @@ route_slot_kernel(int T, int K, int E, int S, int C, int A, int nblk, int64_t R_
                   const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ blk_base,
                   const int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                   int32_t* __restrict__ segoff, int32_t* __restrict__ totals,
-                  int32_t* __restrict__ slot, int32_t* __restrict__ row_src) {
+                  int32_t* __restrict__ slot, int32_t* __restrict__ row_src,
+                  uint32_t* __restrict__ row_ready, int64_t n_ready) {
   __shared__ int off_s[MAX_E + 1];
   __shared__ int kept_s[MAX_E];
   __shared__ int warp_tmp[16];
@@ -269,6 +270,8 @@ route_slot_kernel(int T, int K, int E, int S, int C, int A, int nblk, int64_t R_
     }
   }
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_ready; i += stride)
+    row_ready[i] = 0u;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < TK; i += stride) {
     const int t = (int)(i / K);
     const int e = topk_idx[i];
@@ -311,8 +314,10 @@ cudaError_t launch_topk(int nblk, size_t smem, cudaStream_t s, const float* logi
 cudaError_t launch_route(const moe_config_t& c, const float* logits, int32_t* topk_idx,
                          float* topk_w, int32_t* counts, int32_t* overflow, int32_t* offsets,
                          int32_t* segoff, int32_t* slot, int32_t* row_src, int32_t* totals,
-                         int32_t* blk_cnt, int64_t R_max, cudaStream_t s) {
+                         int32_t* blk_cnt, int64_t R_max, cudaStream_t s,
+                         uint32_t* row_ready) {
   const int nblk = (int)ceil_div(c.T, ROUTE_TB);
+  const int64_t n_ready = row_ready ? ceil_div(R_max, READY_ROWS) : 0;
   if (nblk > 0) {
     const size_t smem = (size_t)c.E * WORDS * 4 + (size_t)ROUTE_TB * c.K * 4;
     const int vpl = (int)ceil_div(c.E, 32);
@@ -332,7 +337,8 @@ cudaError_t launch_route(const moe_config_t& c, const float* logits, int32_t* to
   int grid = (int)std::min<int64_t>(std::max<int64_t>(ceil_div(work, 256), 1), 148 * 8);
   return launch_pdl(route_slot_kernel, dim3(grid), dim3(256), 0, s, c.T, c.K, c.E, c.S, c.capacity,
                     c.row_align, nblk, R_max, (const int32_t*)topk_idx, (const int32_t*)blk_cnt,
-                    (const int32_t*)counts, offsets, segoff, totals, slot, row_src);
+                    (const int32_t*)counts, offsets, segoff, totals, slot, row_src, row_ready,
+                    n_ready);
 }
 
 }  // namespace moe

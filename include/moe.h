@@ -85,6 +85,9 @@ typedef struct {
 } moe_layer_aux_t;
 
 #define MOE_FLAG_NONE 0u
+/* moe_layer_forward: overlap the combine with the down GEMM through per-block
+ * ready counters (see moe_combine_wait). bf16 only; row_align % 128 == 0. */
+#define MOE_FLAG_OVERLAP 1u
 
 /* C = ceil(cf * T * K / E), computed in double precision; cf < 0 means no limit
  * and returns T (a token picks an expert at most once). Returns -1 if T < 0,
@@ -206,10 +209,33 @@ moe_status_t moe_expert_mlp(const moe_config_t* cfg, const void* xp,
 moe_status_t moe_combine(const moe_config_t* cfg, const void* y, const int32_t* token_slot,
                          const float* topk_w, void* out, void* stream);
 
+/* The combine as the consumer of a tile-signalled overlap ("Mixture-of-Experts
+ * acceleration through overlap": the GEMM publishes tile-ready flags in its
+ * epilogue and a separate kernel starts on each tile as soon as its flag is set).
+ * Same result as moe_combine. Before reading the rows of token t, the kernel
+ * waits until row_ready[slot / 128] >= ready_target for every kept slot of t
+ * (acquire loads). moe_expert_mlp's down GEMM, run by moe_layer_forward with
+ * MOE_FLAG_OVERLAP, adds 1 to a block's counter per stored 256-column tile
+ * (release), so the target there is ceil(H / 256). The kernel does not wait for
+ * the previous kernel in the stream, so token_slot and topk_w must already be
+ * final when it starts; only the rows of y are waited for.
+ *   row_ready   [ceil(R_max / 128)] uint32, device.
+ *   timeout_us  bound of all waits; on expiry the kernel records MOE_ERR_TIMEOUT
+ *               in the workspace's status word (moe_get_device_status), stops
+ *               waiting everywhere and leaves the affected rows of out unwritten.
+ *   ws          a workspace holding the status word (at least 256 bytes).
+ * Requires row_align % 128 == 0 (every 128-row block belongs to one expert). */
+moe_status_t moe_combine_wait(const moe_config_t* cfg, const void* y, const int32_t* token_slot,
+                              const float* topk_w, const uint32_t* row_ready,
+                              uint32_t ready_target, void* out, uint32_t timeout_us, void* ws,
+                              size_t ws_bytes, void* stream);
+
 /* The whole layer on `stream`: route -> dispatch -> expert MLP -> combine, with
  * every intermediate in the workspace (moe_workspace_bytes). `aux` may be NULL;
  * otherwise it receives the workspace pointers of the intermediates. No host
- * synchronisation: the per-expert counts stay on the device. */
+ * synchronisation: the per-expert counts stay on the device. flags: MOE_FLAG_NONE,
+ * or MOE_FLAG_OVERLAP (the combine overlaps the down GEMM; bf16 with
+ * row_align % 128 == 0, else MOE_ERR_UNSUPPORTED; identical results). */
 moe_status_t moe_layer_forward(const moe_config_t* cfg, const float* logits, const void* x,
                                const void* w_gu, const void* w_d, void* out,
                                uint32_t flags, void* ws, size_t ws_bytes,

@@ -115,6 +115,21 @@ def test_entry_points_reject_bad_arguments_before_any_launch():
     assert lib.moe_get_device_status(None, ctypes.byref(st), None) == M.MOE_ERR_INVALID_ARG
 
 
+def test_overlap_flag_needs_bf16_and_128_row_alignment():
+    lib = M.LIB
+    fake = ctypes.c_void_p(0x10000)
+    for A, act in ((1, "bf16"), (64, "bf16"), (128, "f32")):
+        cfg = M.make_config(T=256, H=128, E=8, K=2, F=128, S=2, capacity=64, row_align=A, act=act)
+        assert lib.moe_layer_forward(ctypes.byref(cfg), fake, fake, fake, fake, fake,
+                                     M.MOE_FLAG_OVERLAP, fake, 1 << 40, None, None) == M.MOE_ERR_UNSUPPORTED
+    cfg = M.make_config(T=256, H=128, E=8, K=2, F=128, S=2, capacity=64, row_align=1)
+    assert lib.moe_combine_wait(ctypes.byref(cfg), fake, fake, fake, fake, 1, fake, 10, fake,
+                                256, None) == M.MOE_ERR_UNSUPPORTED
+    cfg.row_align = 128
+    assert lib.moe_combine_wait(ctypes.byref(cfg), fake, fake, fake, None, 1, fake, 10, fake,
+                                256, None) == M.MOE_ERR_INVALID_ARG
+
+
 def test_status_strings():
     for code in range(7):
         s = M.status_string(code)
