@@ -42,7 +42,7 @@ PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 METRIC = "MoE layer tokens/s on 1 B200; dispatch/combine HBM GB/s & GEMM % of roofline"
-KERNELS_PER_STEP = 7   # route x3, dispatch, gate/up GEMM, down GEMM, combine
+KERNELS_PER_STEP = 7   # route x3, dispatch, gate/up GEMM, down GEMM, combine (+1 with --router)
 
 
 def load_peaks():
@@ -159,25 +159,35 @@ def flush_l2(buf: torch.Tensor):
 class Layer:
     """Device-resident inputs, weights and workspace of one replica."""
 
-    def __init__(self, wl: W.Workload, seed: int, device, overlap: bool = False):
+    def __init__(self, wl: W.Workload, seed: int, device, overlap: bool = False,
+                 router: bool = False):
         import combine_moe_route_13_b200 as M
         self.M = M
         self.flags = M.MOE_FLAG_OVERLAP if overlap else M.MOE_FLAG_NONE
+        self.router = router
         self.wl = wl
         self.C = M.moe_capacity(wl.T, wl.K, wl.E, wl.cf)
         self.cfg = M.make_config(wl.T, wl.H, wl.E, wl.K, wl.F, wl.S, self.C, wl.row_align, wl.act)
         st = M.moe_check_config(self.cfg)
         if st != M.MOE_OK:
             raise SystemExit(f"unsupported workload: {M.status_string(st)}")
-        self.inp = W.make_inputs(wl, seed=seed, device=device)
+        self.inp = W.make_inputs(wl, seed=seed, device=device, router=router)
         self.ws = M.alloc_workspace(M.moe_workspace_bytes(self.cfg), device)
         self.out = torch.empty(wl.T, wl.H, dtype=wl.torch_act, device=device)
         self.aux = None
 
-    def forward(self):
-        self.aux = self.M.moe_layer_forward(self.cfg, self.inp["logits"], self.inp["x"],
-                                            self.inp["w_gu"], self.inp["w_d"], self.out, self.ws,
-                                            flags=self.flags)
+    def forward(self, x=None, logits=None):
+        x = self.inp["x"] if x is None else x
+        if self.router:   # from hidden states: router projection + selection-only bias
+            self.aux = self.M.moe_layer_forward_x(self.cfg, x, self.inp["w_g"],
+                                                  self.inp["sel_bias"], self.inp["w_gu"],
+                                                  self.inp["w_d"], self.out, self.ws,
+                                                  flags=self.flags)
+        else:
+            logits = self.inp["logits"] if logits is None else logits
+            self.aux = self.M.moe_layer_forward(self.cfg, logits, x, self.inp["w_gu"],
+                                                self.inp["w_d"], self.out, self.ws,
+                                                flags=self.flags)
 
     def views(self):
         return self.M.layer_views(self.cfg, self.ws, self.aux)
@@ -204,11 +214,16 @@ def phase_times(layer: Layer, steps, flush_buf, stream):
     M = layer.M
     v = layer.views()
     cfg, inp = layer.cfg, layer.inp
-    names = ("route", "dispatch", "expert_mlp", "combine")
+    names = ("router", "route", "dispatch", "expert_mlp", "combine")
+    logits = v["logits"] if layer.router else inp["logits"]
+    bias = inp["sel_bias"] if layer.router else None
     calls = (
-        lambda: M.moe_route_topk(cfg, inp["logits"], v["topk_idx"], v["topk_w"], v["expert_counts"],
-                                 v["overflow"], v["expert_offsets"], v["segment_offsets"],
-                                 v["token_slot"], v["row_src"], v["totals"], layer.ws),
+        (lambda: M.moe_router_logits(cfg, inp["x"], inp["w_g"], v["logits"], layer.ws))
+        if layer.router else (lambda: None),
+        lambda: M.moe_route_topk_biased(cfg, logits, bias, v["topk_idx"], v["topk_w"],
+                                        v["expert_counts"], v["overflow"], v["expert_offsets"],
+                                        v["segment_offsets"], v["token_slot"], v["row_src"],
+                                        v["totals"], layer.ws),
         lambda: M.moe_dispatch(cfg, inp["x"], v["token_slot"], v["xp"]),
         lambda: M.moe_expert_mlp(cfg, v["xp"], v["expert_offsets"], v["expert_counts"],
                                  inp["w_gu"], inp["w_d"], v["h"], v["y"], layer.ws),
@@ -239,14 +254,14 @@ def e2e_steps(layer: Layer, steps, warmup, flush_buf, stream):
     M, cfg = layer.M, layer.cfg
 
     def step():
-        d_logits.copy_(h_logits, non_blocking=True)
+        if not layer.router:
+            d_logits.copy_(h_logits, non_blocking=True)
         d_x.copy_(h_x, non_blocking=True)
-        M.moe_layer_forward(cfg, d_logits, d_x, inp["w_gu"], inp["w_d"], layer.out, layer.ws,
-                            flags=layer.flags)
+        layer.forward(x=d_x, logits=d_logits)
         h_out.copy_(layer.out, non_blocking=True)
 
     times = time_steps(step, steps, warmup, flush_buf, stream)
-    h2d = h_logits.numel() * 4 + h_x.numel() * h_x.element_size()
+    h2d = (0 if layer.router else h_logits.numel() * 4) + h_x.numel() * h_x.element_size()
     d2h = h_out.numel() * h_out.element_size()
     return times, h2d, d2h
 
@@ -347,6 +362,9 @@ def main(argv=None):
     ap.add_argument("--cpu-tokens", type=int, default=256,
                     help="tokens of the CPU-oracle sample per step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--router", action="store_true",
+                    help="start from hidden states: router projection x W_g^T and a "
+                         "selection-only bias (moe_layer_forward_x)")
     ap.add_argument("--overlap", action="store_true",
                     help="overlap the combine with the down GEMM (MOE_FLAG_OVERLAP)")
     args = ap.parse_args(argv)
@@ -365,7 +383,7 @@ def main(argv=None):
     torch.cuda.set_device(device)
     peaks = load_peaks()
 
-    layer = Layer(wl, seed=rank, device=device, overlap=args.overlap)
+    layer = Layer(wl, seed=rank, device=device, overlap=args.overlap, router=args.router)
     flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream()
 
@@ -404,6 +422,7 @@ def main(argv=None):
     tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     mlp_tflops = alg["mlp_flops"] / (ph["expert_mlp"] * 1e-3) / 1e12
     kernels = {
+        "router_us": ph["router"] * 1e3 if args.router else None,
         "route_us": ph["route"] * 1e3,
         "dispatch_us": ph["dispatch"] * 1e3,
         "dispatch_gbs": alg["dispatch_bytes"] / (ph["dispatch"] * 1e-3) / 1e9,
@@ -439,10 +458,10 @@ def main(argv=None):
                    "S": wl.S, "cf": wl.cf, "capacity": layer.C, "row_align": wl.row_align,
                    "effective_tokens": alg["N"], "overflow": int(totals[2]),
                    "l2": "flushed (256 MB write) before every step", "parallelism": f"replicas{world}",
-                   "overlap": bool(args.overlap)},
+                   "overlap": bool(args.overlap), "router_projection": bool(args.router)},
         "e2e": {"value": world * wl.T / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": (KERNELS_PER_STEP + (1 if args.router else 0)) * args.steps,
         "roofline": {"bound": "tensor", "kernel": "expert_mlp (gate/up + down grouped GEMMs)",
                      "achieved": mlp_tflops, "peak": tensor_peak, "unit": "TFLOP/s",
                      "frac": mlp_tflops / tensor_peak,

@@ -32,7 +32,8 @@ MOE_FLAG_OVERLAP = 1
 EXPORTS = ("moe_capacity", "moe_max_rows", "moe_check_config", "moe_route_workspace_bytes",
            "moe_workspace_bytes", "moe_workspace_init", "moe_route_topk", "moe_dispatch",
            "moe_expert_mlp", "moe_combine", "moe_layer_forward", "moe_get_device_status",
-           "moe_status_string", "moe_version", "moe_route_topk_noalloc", "moe_combine_wait")
+           "moe_status_string", "moe_version", "moe_route_topk_noalloc", "moe_combine_wait",
+           "moe_route_topk_biased", "moe_router_logits", "moe_layer_forward_x")
 
 
 class MoeError(RuntimeError):
@@ -54,7 +55,7 @@ class MoeConfig(ctypes.Structure):
 class MoeLayerAux(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "topk_idx", "expert_counts", "overflow", "expert_offsets", "segment_offsets",
-        "token_slot", "row_src", "totals", "topk_w", "xp", "h", "y")]
+        "token_slot", "row_src", "totals", "topk_w", "xp", "h", "y", "logits")]
 
 
 _P = ctypes.c_void_p
@@ -85,6 +86,11 @@ def _load():
         "moe_route_topk_noalloc": (ctypes.c_int, [_CFG] + [_P] * 10 + [_P]),
         "moe_combine_wait": (ctypes.c_int, [_CFG, _P, _P, _P, _P, ctypes.c_uint32, _P,
                                             ctypes.c_uint32, _P, ctypes.c_size_t, _P]),
+        "moe_route_topk_biased": (ctypes.c_int, [_CFG] + [_P] * 11 + [_P, ctypes.c_size_t, _P]),
+        "moe_router_logits": (ctypes.c_int, [_CFG, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+        "moe_layer_forward_x": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, ctypes.c_uint32,
+                                               _P, ctypes.c_size_t, ctypes.POINTER(MoeLayerAux),
+                                               _P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -171,6 +177,42 @@ def moe_route_topk(cfg, logits, topk_idx, topk_w, expert_counts, overflow, exper
         _ptr(segment_offsets, i32, "segment_offsets"), _ptr(token_slot, i32, "token_slot"),
         _ptr(row_src, i32, "row_src"), _ptr(totals, i32, "totals"), _ptr(ws, name="ws"),
         ws.numel() * ws.element_size(), _stream(stream)), "moe_route_topk")
+
+
+def moe_route_topk_biased(cfg, logits, sel_bias, topk_idx, topk_w, expert_counts, overflow,
+                          expert_offsets, segment_offsets, token_slot, row_src, totals, ws,
+                          stream=None):
+    i32 = torch.int32
+    _check(LIB.moe_route_topk_biased(
+        ctypes.byref(cfg), _ptr(logits, torch.float32, "logits"),
+        _ptr(sel_bias, torch.float32, "sel_bias"), _ptr(topk_idx, i32, "topk_idx"),
+        _ptr(topk_w, torch.float32, "topk_w"), _ptr(expert_counts, i32, "expert_counts"),
+        _ptr(overflow, i32, "overflow"), _ptr(expert_offsets, i32, "expert_offsets"),
+        _ptr(segment_offsets, i32, "segment_offsets"), _ptr(token_slot, i32, "token_slot"),
+        _ptr(row_src, i32, "row_src"), _ptr(totals, i32, "totals"), _ptr(ws, name="ws"),
+        ws.numel() * ws.element_size(), _stream(stream)), "moe_route_topk_biased")
+
+
+def moe_router_logits(cfg, x, w_g, logits, ws, stream=None):
+    dt = act_dtype(cfg)
+    _check(LIB.moe_router_logits(ctypes.byref(cfg), _ptr(x, dt, "x"), _ptr(w_g, dt, "w_g"),
+                                 _ptr(logits, torch.float32, "logits"), _ptr(ws, name="ws"),
+                                 ws.numel() * ws.element_size(), _stream(stream)),
+           "moe_router_logits")
+
+
+def moe_layer_forward_x(cfg, x, w_g, sel_bias, w_gu, w_d, out, ws, flags=MOE_FLAG_NONE,
+                        stream=None):
+    """The layer from hidden states (router projection included); returns a
+    MoeLayerAux like moe_layer_forward, with the logits' address."""
+    dt = act_dtype(cfg)
+    aux = MoeLayerAux()
+    _check(LIB.moe_layer_forward_x(
+        ctypes.byref(cfg), _ptr(x, dt, "x"), _ptr(w_g, dt, "w_g"),
+        _ptr(sel_bias, torch.float32, "sel_bias"), _ptr(w_gu, dt, "w_gu"), _ptr(w_d, dt, "w_d"),
+        _ptr(out, dt, "out"), flags, _ptr(ws, name="ws"), ws.numel() * ws.element_size(),
+        ctypes.byref(aux), _stream(stream)), "moe_layer_forward_x")
+    return aux
 
 
 def moe_route_topk_noalloc(cfg, logits, topk_idx, topk_w, expert_counts, overflow,
@@ -299,4 +341,5 @@ def layer_views(cfg: MoeConfig, ws: torch.Tensor, aux: MoeLayerAux) -> dict:
         "xp": view(aux.xp, R * cfg.H * es, dt, (R, cfg.H)),
         "h": view(aux.h, R * cfg.F * es, dt, (R, cfg.F)),
         "y": view(aux.y, R * cfg.H * es, dt, (R, cfg.H)),
+        "logits": view(aux.logits, TK // max(cfg.K, 1) * cfg.E * 4, torch.float32, (cfg.T, cfg.E)),
     }

@@ -105,7 +105,31 @@ simt_grouped_gemm(const float* __restrict__ A, int Kdim, const float* __restrict
   }
 }
 
+// Router projection for fp32 activations: one thread per logit, FFMA over H.
+__global__ void __launch_bounds__(256)
+router_logits_f32(const float* __restrict__ x, const float* __restrict__ w_g,
+                  float* __restrict__ logits, int T, int H, int E) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (int64_t)T * E) return;
+  const int t = (int)(i / E), e = (int)(i % E);
+  const float* xr = x + (int64_t)t * H;
+  const float* wr = w_g + (int64_t)e * H;
+  float acc = 0.f;
+  for (int h = 0; h < H; ++h) acc = fmaf(xr[h], wr[h], acc);
+  logits[i] = acc;
+}
+
 }  // namespace
+
+cudaError_t launch_router_f32(const moe_config_t& c, const float* x, const float* w_g,
+                              float* logits, cudaStream_t s) {
+  const int64_t n = (int64_t)c.T * c.E;
+  if (n == 0) return cudaSuccess;
+  return launch_pdl(router_logits_f32, dim3((unsigned)ceil_div(n, 256)), dim3(256), 0, s, x, w_g,
+                    logits, c.T, c.H, c.E);
+}
 
 cudaError_t launch_mlp_f32(const moe_config_t& c, const float* xp, const int32_t* offsets,
                            const int32_t* counts, const float* w_gu, const float* w_d, float* h,

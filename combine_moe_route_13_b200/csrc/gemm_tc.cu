@@ -420,14 +420,16 @@ __device__ __forceinline__ void decode_tile(int tile, int NT, const int* P, int 
 template <int MODE, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ CUtensorMap tmOut, __nv_bfloat16* __restrict__ out,
+                const __grid_constant__ CUtensorMap tmOut, void* __restrict__ out_v,
                 int N_out, int Kdim, int b_rows_per_expert,
                 int b_second_off, const int32_t* __restrict__ offsets,
                 const int32_t* __restrict__ counts, int E, int C, long long R_max,
-                uint32_t* __restrict__ status, uint32_t* __restrict__ row_ready) {
+                uint32_t* __restrict__ status, uint32_t* __restrict__ row_ready,
+                int dense_rows) {
   using CF = Cfg<CG>;
   constexpr int STAGES = CF::STAGES;
   constexpr int BN_OUT = (MODE == 0) ? 128 : 256;   // output columns per tile
+  __nv_bfloat16* __restrict__ out = static_cast<__nv_bfloat16*>(out_v);
   constexpr int N_STEP = BN_OUT;                     // weight rows per n tile
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = saddr(smem_raw);
@@ -476,9 +478,10 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     for (int i = 0; i < chunk; ++i) {
       const int e = e0 + i;
       if (e < E) {
-        const int k = max(0, min(counts[e], C));
+        // dense_rows > 0: one group of dense_rows rows starting at row 0
+        const int k = dense_rows > 0 ? dense_rows : max(0, min(counts[e], C));
         kept_s[e] = k;
-        row_off[e] = offsets[e];
+        row_off[e] = dense_rows > 0 ? 0 : offsets[e];
         local += (k + CF::TILE_ROWS - 1) / CF::TILE_ROWS;
       }
     }
@@ -501,7 +504,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     }
     if (threadIdx.x == NUM_THREADS - 1) {
       P[E] = run;
-      row_off[E] = offsets[E];
+      row_off[E] = dense_rows > 0 ? dense_rows : offsets[E];
     }
   }
   tc_fence_before();
@@ -610,11 +613,33 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       // (alignment padding included, which no reader uses) leaves through a
       // staged TMA store; otherwise each thread stores its own row if valid.
       const long long row0 = (long long)row_off[e] + first;
-      const bool staged =
-          rows > 0 && row0 >= 0 && row0 + BM <= row_off[e + 1] && row0 + BM <= R_max;
+      const bool staged = MODE != 2 && rows > 0 && row0 >= 0 && row0 + BM <= row_off[e + 1] &&
+                          row0 + BM <= R_max;
       __nv_bfloat16* orow = out + (row_ok ? grow : 0) * (long long)N_out;
       const uint32_t t0 = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * UMMA_N);
       constexpr int CHUNKS = (MODE == 0) ? 2 : 4;   // 64 output columns each
+      if (MODE == 2) {   // router logits: fp32 out, any number of columns
+        float* lrow = static_cast<float*>(out_v) + (row_ok ? grow : 0) * (long long)N_out;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t a[64];
+          tmem_ld64(t0 + (uint32_t)(c * 64), a);
+          tmem_ld_wait();
+          const int col = n * BN_OUT + c * 64;
+          if (!row_ok || col >= N_out) continue;
+          if (col + 64 <= N_out && (N_out & 3) == 0) {
+            float4* dst = reinterpret_cast<float4*>(lrow + col);
+#pragma unroll
+            for (int v = 0; v < 16; ++v)
+              dst[v] = make_float4(__uint_as_float(a[4 * v]), __uint_as_float(a[4 * v + 1]),
+                                   __uint_as_float(a[4 * v + 2]), __uint_as_float(a[4 * v + 3]));
+          } else {
+#pragma unroll
+            for (int j = 0; j < 64; ++j)
+              if (col + j < N_out) lrow[col + j] = __uint_as_float(a[j]);
+          }
+        }
+      } else
 #pragma unroll 1
       for (int c = 0; c < CHUNKS; ++c) {
         uint4 o[8];
@@ -748,8 +773,10 @@ void fill_launch(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr, int grid, s
   cfg.numAttrs = 2;
 }
 
-// Co-resident CTAs (CG = 1) or 2-CTA clusters (CG = 2) of the kernel on this device.
-template <int CG>
+// Co-resident CTAs (CG = 1) or 2-CTA clusters (CG = 2) of tc_grouped_gemm<MODE, CG>
+// with `smem` bytes of dynamic shared memory (its attribute must already allow
+// that much).
+template <int MODE, int CG>
 int resident_units(size_t smem) {
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -758,10 +785,10 @@ int resident_units(size_t smem) {
   if (CG == 1) return sms;
   cudaLaunchConfig_t q;
   cudaLaunchAttribute attr[2];
-  fill_launch<0, CG>(q, attr, sms & ~1, smem, nullptr);
+  fill_launch<MODE, CG>(q, attr, sms & ~1, smem, nullptr);
   q.numAttrs = 1;   // the cluster shape only
   int clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&clusters, tc_grouped_gemm<0, CG>, &q) != cudaSuccess)
+  if (cudaOccupancyMaxActiveClusters(&clusters, tc_grouped_gemm<MODE, CG>, &q) != cudaSuccess)
     return 0;
   return clusters;
 }
@@ -784,7 +811,7 @@ moe_status_t launch_mlp(const moe_config_t& c, const void* xp, const int32_t* of
       cudaFuncSetAttribute(tc_grouped_gemm<1, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return MOE_ERR_CUDA;
-  const int units = resident_units<CG>(smem);
+  const int units = resident_units<0, CG>(smem);
   if (units <= 0) return MOE_ERR_CUDA;
   const int64_t mt_bound = ceil_div(R_max, Cfg<CG>::TILE_ROWS) + c.E;  // >= sum_e M tiles
   const int64_t t0 = mt_bound * ceil_div(c.F, 128), t1 = mt_bound * ceil_div(c.H, 256);
@@ -793,20 +820,54 @@ moe_status_t launch_mlp(const moe_config_t& c, const void* xp, const int32_t* of
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[2];
   fill_launch<0, CG>(cfg, attr, g0, smem, s);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, tc_grouped_gemm<0, CG>, mx, mwgu, mh,
-                                     static_cast<__nv_bfloat16*>(h), c.F, c.H, 2 * c.F, c.F,
+  cudaError_t e = cudaLaunchKernelEx(&cfg, tc_grouped_gemm<0, CG>, mx, mwgu, mh, h, c.F, c.H,
+                                     2 * c.F, c.F,
                                      offsets, counts, c.E, c.capacity, (long long)R_max, status,
-                                     (uint32_t*)nullptr);
+                                     (uint32_t*)nullptr, 0);
   if (e == cudaSuccess) {
     fill_launch<1, CG>(cfg, attr, g1, smem, s);
-    e = cudaLaunchKernelEx(&cfg, tc_grouped_gemm<1, CG>, mh, mwd, my, static_cast<__nv_bfloat16*>(y),
-                           c.H, c.F, c.H, 128, offsets, counts, c.E, c.capacity,
-                           (long long)R_max, status, row_ready);
+    e = cudaLaunchKernelEx(&cfg, tc_grouped_gemm<1, CG>, mh, mwd, my, y, c.H, c.F, c.H, 128,
+                           offsets, counts, c.E, c.capacity,
+                           (long long)R_max, status, row_ready, 0);
   }
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Router projection as one dense group: logits[T,E] = x[T,H] w_g[E,H]^T.
+template <int CG>
+moe_status_t launch_router(const moe_config_t& c, const void* x, const void* w_g, float* logits,
+                           uint32_t* status, cudaStream_t s) {
+  CUtensorMap mx, mg;
+  if (!make_map(&mx, x, (uint64_t)c.H, (uint64_t)c.T) ||
+      !make_map(&mg, w_g, (uint64_t)c.H, (uint64_t)c.E))
+    return MOE_ERR_CUDA;
+  const size_t smem = smem_bytes<CG>(1);
+  if (cudaFuncSetAttribute(tc_grouped_gemm<2, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int units = resident_units<2, CG>(smem);
+  if (units <= 0) return MOE_ERR_CUDA;
+  const int64_t tiles = ceil_div(c.T, Cfg<CG>::TILE_ROWS) * ceil_div(c.E, 256);
+  const int grid = (int)std::min<int64_t>(units, tiles) * CG;
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[2];
+  fill_launch<2, CG>(cfg, attr, grid, smem, s);
+  // the output map argument is unused in this mode (fp32 rows are stored directly)
+  const cudaError_t e = cudaLaunchKernelEx(
+      &cfg, tc_grouped_gemm<2, CG>, mx, mg, mx, (void*)logits, c.E, c.H, 0, 128,
+      (const int32_t*)nullptr, (const int32_t*)nullptr, 1, c.T, (long long)c.T, status,
+      (uint32_t*)nullptr, c.T);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 }  // namespace tc
+
+moe_status_t launch_router_logits_tc(const moe_config_t& c, const void* x, const void* w_g,
+                                     float* logits, uint32_t* status, cudaStream_t s) {
+  if (c.T == 0) return MOE_OK;
+  if (c.T >= 256) return tc::launch_router<2>(c, x, w_g, logits, status, s);
+  return tc::launch_router<1>(c, x, w_g, logits, status, s);
+}
 
 moe_status_t launch_mlp_bf16_tc(const moe_config_t& c, const void* xp, const int32_t* offsets,
                                 const int32_t* counts, const void* w_gu, const void* w_d,

@@ -61,6 +61,7 @@ WsLayout ws_layout(const moe_config_t& c) {
   L.slot = p;      p += align256((size_t)TK * 4);
   L.row_src = p;   p += align256((size_t)R * 4);
   L.row_ready = p; p += align256((size_t)ceil_div(R, READY_ROWS) * 4);
+  L.logits = p;    p += align256((size_t)c.T * c.E * 4);
   L.xp = p;        p += align256((size_t)R * c.H * as);
   L.h = p;         p += align256((size_t)R * c.F * as);
   L.y = p;         p += align256((size_t)R * c.H * as);
@@ -124,11 +125,12 @@ moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   return cuda_status(cudaMemsetAsync(ws, 0, 4, static_cast<cudaStream_t>(stream)));
 }
 
-moe_status_t moe_route_topk(const moe_config_t* cfg, const float* logits, int32_t* topk_idx,
-                            float* topk_w, int32_t* expert_counts, int32_t* overflow,
-                            int32_t* expert_offsets, int32_t* segment_offsets,
-                            int32_t* token_slot, int32_t* row_src, int32_t* totals, void* ws,
-                            size_t ws_bytes, void* stream) {
+moe_status_t moe_route_topk_biased(const moe_config_t* cfg, const float* logits,
+                                   const float* sel_bias, int32_t* topk_idx, float* topk_w,
+                                   int32_t* expert_counts, int32_t* overflow,
+                                   int32_t* expert_offsets, int32_t* segment_offsets,
+                                   int32_t* token_slot, int32_t* row_src, int32_t* totals,
+                                   void* ws, size_t ws_bytes, void* stream) {
   moe_status_t st = validate(cfg, false);
   if (st != MOE_OK) return st;
   if (!expert_counts || !overflow || !expert_offsets || !segment_offsets || !totals)
@@ -142,7 +144,32 @@ moe_status_t moe_route_topk(const moe_config_t* cfg, const float* logits, int32_
   int32_t* blk = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + L.blk_cnt);
   return cuda_status(launch_route(*cfg, logits, topk_idx, topk_w, expert_counts, overflow,
                                   expert_offsets, segment_offsets, token_slot, row_src, totals,
-                                  blk, R, static_cast<cudaStream_t>(stream)));
+                                  blk, R, static_cast<cudaStream_t>(stream), nullptr, sel_bias));
+}
+
+moe_status_t moe_route_topk(const moe_config_t* cfg, const float* logits, int32_t* topk_idx,
+                            float* topk_w, int32_t* expert_counts, int32_t* overflow,
+                            int32_t* expert_offsets, int32_t* segment_offsets,
+                            int32_t* token_slot, int32_t* row_src, int32_t* totals, void* ws,
+                            size_t ws_bytes, void* stream) {
+  return moe_route_topk_biased(cfg, logits, nullptr, topk_idx, topk_w, expert_counts, overflow,
+                               expert_offsets, segment_offsets, token_slot, row_src, totals, ws,
+                               ws_bytes, stream);
+}
+
+moe_status_t moe_router_logits(const moe_config_t* cfg, const void* x, const void* w_g,
+                               float* logits, void* ws, size_t ws_bytes, void* stream) {
+  moe_status_t st = validate(cfg, true);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x || !w_g || !logits) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_g)) return MOE_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < 256) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cfg->act_dtype == MOE_F32)
+    return cuda_status(launch_router_f32(*cfg, static_cast<const float*>(x),
+                                         static_cast<const float*>(w_g), logits, s));
+  return launch_router_logits_tc(*cfg, x, w_g, logits, static_cast<uint32_t*>(ws), s);
 }
 
 moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* token_slot,
@@ -206,16 +233,23 @@ moe_status_t moe_combine_wait(const moe_config_t* cfg, const void* y, const int3
                                          static_cast<cudaStream_t>(stream)));
 }
 
-moe_status_t moe_layer_forward(const moe_config_t* cfg, const float* logits, const void* x,
-                               const void* w_gu, const void* w_d, void* out, uint32_t flags,
-                               void* ws, size_t ws_bytes, moe_layer_aux_t* aux, void* stream) {
+}  // extern "C"
+
+namespace moe {
+
+// The layer from router logits (written by the caller, or by the router
+// projection when x_for_router is set), with an optional selection bias.
+static moe_status_t layer_forward(const moe_config_t* cfg, const float* logits,
+                                  const float* sel_bias, const void* x, const void* w_g,
+                                  const void* w_gu, const void* w_d, void* out, uint32_t flags,
+                                  void* ws, size_t ws_bytes, moe_layer_aux_t* aux, void* stream) {
   moe_status_t st = validate(cfg, true);
   if (st != MOE_OK) return st;
   if ((flags & ~MOE_FLAG_OVERLAP) != 0u) return MOE_ERR_UNSUPPORTED;
   const bool overlap = (flags & MOE_FLAG_OVERLAP) != 0u;
   if (overlap && (cfg->act_dtype != MOE_BF16 || cfg->row_align % READY_ROWS != 0))
     return MOE_ERR_UNSUPPORTED;
-  if (cfg->T > 0 && (!logits || !x || !out)) return MOE_ERR_INVALID_ARG;
+  if (cfg->T > 0 && (!(logits || w_g) || !x || !out)) return MOE_ERR_INVALID_ARG;
   if (!w_gu || !w_d) return MOE_ERR_INVALID_ARG;
   const WsLayout L = ws_layout(*cfg);
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
@@ -233,38 +267,59 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const float* logits, con
   a.xp = b + L.xp;
   a.h = b + L.h;
   a.y = b + L.y;
+  a.logits = reinterpret_cast<float*>(b + L.logits);
   if (aux) *aux = a;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (w_g) {   // router projection into the workspace
+    st = moe_router_logits(cfg, x, w_g, a.logits, ws, ws_bytes, stream);
+    if (st != MOE_OK) return st;
+    logits = a.logits;
+  }
+  // Overlapped: the route also zeroes the ready counters, the down GEMM
+  // publishes them and the combine consumes them while the GEMM finishes.
+  uint32_t* ready = overlap ? reinterpret_cast<uint32_t*>(b + L.row_ready) : nullptr;
+  uint32_t* status = static_cast<uint32_t*>(ws);
+  const int64_t R = max_rows(*cfg);
+  st = cuda_status(launch_route(*cfg, logits, a.topk_idx, a.topk_w, a.expert_counts, a.overflow,
+                                a.expert_offsets, a.segment_offsets, a.token_slot, a.row_src,
+                                a.totals, reinterpret_cast<int32_t*>(b + L.blk_cnt), R, s, ready,
+                                sel_bias));
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  st = moe_dispatch(cfg, x, a.token_slot, a.xp, stream);
+  if (st != MOE_OK) return st;
   if (!overlap) {
-    st = moe_route_topk(cfg, logits, a.topk_idx, a.topk_w, a.expert_counts, a.overflow,
-                        a.expert_offsets, a.segment_offsets, a.token_slot, a.row_src, a.totals,
-                        ws, ws_bytes, stream);
-    if (st != MOE_OK) return st;
-    if (cfg->T == 0) return MOE_OK;
-    st = moe_dispatch(cfg, x, a.token_slot, a.xp, stream);
-    if (st != MOE_OK) return st;
     st = moe_expert_mlp(cfg, a.xp, a.expert_offsets, a.expert_counts, w_gu, w_d, a.h, a.y, ws,
                         ws_bytes, stream);
     if (st != MOE_OK) return st;
     return moe_combine(cfg, a.y, a.token_slot, a.topk_w, out, stream);
   }
-  // Overlapped: the route also zeroes the ready counters, the down GEMM
-  // publishes them and the combine consumes them while the GEMM finishes.
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint32_t* ready = reinterpret_cast<uint32_t*>(b + L.row_ready);
-  uint32_t* status = static_cast<uint32_t*>(ws);
-  const int64_t R = max_rows(*cfg);
-  st = cuda_status(launch_route(*cfg, logits, a.topk_idx, a.topk_w, a.expert_counts, a.overflow,
-                                a.expert_offsets, a.segment_offsets, a.token_slot, a.row_src,
-                                a.totals, reinterpret_cast<int32_t*>(b + L.blk_cnt), R, s, ready));
-  if (st != MOE_OK) return st;
-  if (cfg->T == 0) return MOE_OK;
-  st = cuda_status(launch_dispatch(*cfg, x, a.token_slot, a.xp, s));
-  if (st != MOE_OK) return st;
   st = launch_mlp_bf16_tc(*cfg, a.xp, a.expert_offsets, a.expert_counts, w_gu, w_d, a.h, a.y, R,
                           status, s, ready);
   if (st != MOE_OK) return st;
   return cuda_status(launch_combine_wait(*cfg, a.y, a.token_slot, a.topk_w, ready,
                                          ready_target(*cfg), WAIT_LIMIT_NS, status, out, s));
+}
+
+}  // namespace moe
+
+extern "C" {
+
+moe_status_t moe_layer_forward(const moe_config_t* cfg, const float* logits, const void* x,
+                               const void* w_gu, const void* w_d, void* out, uint32_t flags,
+                               void* ws, size_t ws_bytes, moe_layer_aux_t* aux, void* stream) {
+  if (cfg && cfg->T > 0 && !logits) return MOE_ERR_INVALID_ARG;
+  return layer_forward(cfg, logits, nullptr, x, nullptr, w_gu, w_d, out, flags, ws, ws_bytes, aux,
+                       stream);
+}
+
+moe_status_t moe_layer_forward_x(const moe_config_t* cfg, const void* x, const void* w_g,
+                                 const float* sel_bias, const void* w_gu, const void* w_d,
+                                 void* out, uint32_t flags, void* ws, size_t ws_bytes,
+                                 moe_layer_aux_t* aux, void* stream) {
+  if (!w_g) return MOE_ERR_INVALID_ARG;
+  return layer_forward(cfg, nullptr, sel_bias, x, w_g, w_gu, w_d, out, flags, ws, ws_bytes, aux,
+                       stream);
 }
 
 moe_status_t moe_get_device_status(void* ws, moe_status_t* status, void* stream) {

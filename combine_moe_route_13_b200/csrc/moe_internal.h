@@ -34,7 +34,7 @@ struct WsLayout {
   size_t blk_cnt = 0;      // [nblk, E] int32: per-block histograms, then bases
   size_t route_end = 0;    // bytes needed by moe_route_topk
   size_t topk_idx = 0, topk_w = 0, counts = 0, overflow = 0, offsets = 0;
-  size_t segoff = 0, totals = 0, slot = 0, row_src = 0, row_ready = 0;
+  size_t segoff = 0, totals = 0, slot = 0, row_src = 0, row_ready = 0, logits = 0;
   size_t xp = 0, h = 0, y = 0;
   size_t total = 0;        // bytes needed by moe_layer_forward
 };
@@ -79,7 +79,7 @@ cudaError_t launch_route(const moe_config_t& c, const float* logits, int32_t* to
                          float* topk_w, int32_t* counts, int32_t* overflow, int32_t* offsets,
                          int32_t* segoff, int32_t* slot, int32_t* row_src, int32_t* totals,
                          int32_t* blk_cnt, int64_t R_max, cudaStream_t s,
-                         uint32_t* row_ready = nullptr);
+                         uint32_t* row_ready = nullptr, const float* sel_bias = nullptr);
 
 cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t* slot, void* xp,
                             cudaStream_t s);
@@ -107,6 +107,13 @@ moe_status_t launch_mlp_bf16_tc(const moe_config_t& c, const void* xp, const int
                                 const int32_t* counts, const void* w_gu, const void* w_d,
                                 void* h, void* y, int64_t R_max, uint32_t* status,
                                 cudaStream_t s, uint32_t* row_ready = nullptr);
+
+// Router projection logits[T,E] = x[T,H] w_g[E,H]^T (fp32 out): tcgen05 for
+// bf16, FFMA for fp32.
+moe_status_t launch_router_logits_tc(const moe_config_t& c, const void* x, const void* w_g,
+                                     float* logits, uint32_t* status, cudaStream_t s);
+cudaError_t launch_router_f32(const moe_config_t& c, const float* x, const float* w_g,
+                              float* logits, cudaStream_t s);
 
 // Ready-counter target of the down GEMM (its number of N tiles).
 inline uint32_t ready_target(const moe_config_t& c) { return (uint32_t)ceil_div(c.H, 256); }

@@ -61,10 +61,10 @@ __device__ __forceinline__ void load_logits(const float* __restrict__ row, int E
   }
 }
 
-template <int VPL, int THREADS>
+template <int VPL, int THREADS, bool BIAS>
 __global__ void __launch_bounds__(THREADS)
-route_topk_kernel(const float* __restrict__ logits, int T, int E, int K,
-                  int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+route_topk_kernel(const float* __restrict__ logits, const float* __restrict__ sel_bias, int T,
+                  int E, int K, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                   int32_t* __restrict__ local_rank, int32_t* __restrict__ blk_cnt) {
   extern __shared__ uint32_t smem_u[];
   uint32_t* bitmap = smem_u;                                   // [E][WORDS]
@@ -83,6 +83,9 @@ route_topk_kernel(const float* __restrict__ logits, int T, int E, int K,
 #pragma unroll
   for (int j = 0; j < VPL; ++j)
     if (lane + 32 * j >= E) invalid |= 1u << j;
+  float bias[VPL];   // selection-only bias of this lane's experts
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) bias[j] = (BIAS && lane + 32 * j < E) ? sel_bias[lane + 32 * j] : 0.f;
   float nxt[VPL];
   if (warp < ntok) load_logits<VPL>(logits + (size_t)(tb0 + warp) * E, E, lane, nxt);
   for (int tl = warp; tl < ntok; tl += NWARPS) {
@@ -94,7 +97,7 @@ route_topk_kernel(const float* __restrict__ logits, int T, int E, int K,
     uint32_t taken = invalid;
     uint32_t key[VPL];
 #pragma unroll
-    for (int j = 0; j < VPL; ++j) key[j] = order_key(v[j]);
+    for (int j = 0; j < VPL; ++j) key[j] = order_key(BIAS ? v[j] + bias[j] : v[j]);
     float my_v = 0.f, v0 = 0.f;
     int my_i = 0;
     for (int k = 0; k < K; ++k) {
@@ -112,7 +115,16 @@ route_topk_kernel(const float* __restrict__ logits, int T, int E, int K,
       // the warp's largest key, then the lowest index holding it
       const uint32_t m = __reduce_max_sync(0xffffffffu, best);
       const int win = __reduce_min_sync(0xffffffffu, best == m ? bi : INT_MAX);
-      const float wv = key_value(m);
+      float wv;
+      if (BIAS) {   // the winner's unbiased logit, from the lane that holds it
+        float cand = 0.f;
+#pragma unroll
+        for (int j = 0; j < VPL; ++j)
+          if (j == (win >> 5)) cand = v[j];
+        wv = __shfl_sync(0xffffffffu, cand, win & 31);
+      } else {
+        wv = key_value(m);
+      }
       if (k == 0) v0 = wv;
       if (lane == k) {
         my_v = wv;
@@ -120,7 +132,10 @@ route_topk_kernel(const float* __restrict__ logits, int T, int E, int K,
       }
       if ((win & 31) == lane) taken |= 1u << (win >> 5);
     }
-    // softmax over the K selected logits, shifted by the largest one
+    // softmax over the K selected logits, shifted by the largest one (the
+    // first winner unless a selection bias reordered them)
+    if (BIAS)
+      v0 = key_value(__reduce_max_sync(0xffffffffu, lane < K ? order_key(my_v) : 0u));
     const float ex = (lane < K) ? expf(my_v - v0) : 0.f;
     float sum = ex;
 #pragma unroll
@@ -300,13 +315,17 @@ route_slot_kernel(int T, int K, int E, int S, int C, int A, int nblk, int64_t R_
 }
 
 template <int VPL>
-cudaError_t launch_topk(int nblk, size_t smem, cudaStream_t s, const float* logits, int T, int E, int K,
-                 int32_t* idx, float* w, int32_t* rank, int32_t* blk) {
+cudaError_t launch_topk(int nblk, size_t smem, cudaStream_t s, const float* logits,
+                        const float* sel_bias, int T, int E, int K, int32_t* idx, float* w,
+                        int32_t* rank, int32_t* blk) {
   // 32 warps (4 tokens each) while the register budget allows: 16 warps for
   // E > 256, 8 for E > 512
   constexpr int THREADS = VPL >= 32 ? 256 : (VPL >= 16 ? 512 : 1024);
-  return launch_pdl(route_topk_kernel<VPL, THREADS>, dim3(nblk), dim3(THREADS), smem, s, logits, T,
-                    E, K, idx, w, rank, blk);
+  if (sel_bias)
+    return launch_pdl(route_topk_kernel<VPL, THREADS, true>, dim3(nblk), dim3(THREADS), smem, s,
+                      logits, sel_bias, T, E, K, idx, w, rank, blk);
+  return launch_pdl(route_topk_kernel<VPL, THREADS, false>, dim3(nblk), dim3(THREADS), smem, s,
+                    logits, sel_bias, T, E, K, idx, w, rank, blk);
 }
 
 }  // namespace
@@ -315,19 +334,19 @@ cudaError_t launch_route(const moe_config_t& c, const float* logits, int32_t* to
                          float* topk_w, int32_t* counts, int32_t* overflow, int32_t* offsets,
                          int32_t* segoff, int32_t* slot, int32_t* row_src, int32_t* totals,
                          int32_t* blk_cnt, int64_t R_max, cudaStream_t s,
-                         uint32_t* row_ready) {
+                         uint32_t* row_ready, const float* sel_bias) {
   const int nblk = (int)ceil_div(c.T, ROUTE_TB);
   const int64_t n_ready = row_ready ? ceil_div(R_max, READY_ROWS) : 0;
   if (nblk > 0) {
     const size_t smem = (size_t)c.E * WORDS * 4 + (size_t)ROUTE_TB * c.K * 4;
     const int vpl = (int)ceil_div(c.E, 32);
     cudaError_t e;
-    if (vpl <= 1) e = launch_topk<1>(nblk, smem, s, logits, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
-    else if (vpl <= 2) e = launch_topk<2>(nblk, smem, s, logits, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
-    else if (vpl <= 4) e = launch_topk<4>(nblk, smem, s, logits, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
-    else if (vpl <= 8) e = launch_topk<8>(nblk, smem, s, logits, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
-    else if (vpl <= 16) e = launch_topk<16>(nblk, smem, s, logits, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
-    else e = launch_topk<32>(nblk, smem, s, logits, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
+    if (vpl <= 1) e = launch_topk<1>(nblk, smem, s, logits, sel_bias, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
+    else if (vpl <= 2) e = launch_topk<2>(nblk, smem, s, logits, sel_bias, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
+    else if (vpl <= 4) e = launch_topk<4>(nblk, smem, s, logits, sel_bias, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
+    else if (vpl <= 8) e = launch_topk<8>(nblk, smem, s, logits, sel_bias, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
+    else if (vpl <= 16) e = launch_topk<16>(nblk, smem, s, logits, sel_bias, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
+    else e = launch_topk<32>(nblk, smem, s, logits, sel_bias, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
     if (e != cudaSuccess) return e;
   }
   cudaError_t e = launch_pdl(route_scan_kernel, dim3((unsigned)ceil_div(c.E, 32)), dim3(1024), 0, s,

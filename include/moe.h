@@ -82,6 +82,7 @@ typedef struct {
   int32_t *token_slot, *row_src, *totals;
   float *topk_w;
   void *xp, *h, *y;
+  float *logits;   /* [T,E]: the router projection's output (moe_layer_forward_x only) */
 } moe_layer_aux_t;
 
 #define MOE_FLAG_NONE 0u
@@ -142,6 +143,29 @@ moe_status_t moe_route_topk(const moe_config_t* cfg, const float* logits,
                             int32_t* segment_offsets, int32_t* token_slot,
                             int32_t* row_src, int32_t* totals,
                             void* ws, size_t ws_bytes, void* stream);
+
+/* moe_route_topk with a selection-only bias. Experts are selected by the fp32 sum
+ * logits[t,e] + sel_bias[e], in the same order (larger first, then lower index);
+ * the weights are the softmax over the selected experts' unbiased logits. This is
+ * the bias-for-selection routing of DeepSeek-style routers, written with this
+ * library's weight rule. sel_bias: [E] fp32 device, or NULL (then identical to
+ * moe_route_topk). Other arguments as moe_route_topk. */
+moe_status_t moe_route_topk_biased(const moe_config_t* cfg, const float* logits,
+                                   const float* sel_bias, int32_t* topk_idx, float* topk_w,
+                                   int32_t* expert_counts, int32_t* overflow,
+                                   int32_t* expert_offsets, int32_t* segment_offsets,
+                                   int32_t* token_slot, int32_t* row_src, int32_t* totals,
+                                   void* ws, size_t ws_bytes, void* stream);
+
+/* Router projection: the small linear layer in front of the route ("Introductie"
+ * of the pplx-kernels page; the EFA page's introduction):
+ *   logits[t,e] = sum_h x[t,h] * w_g[e,h], fp32 accumulation, stored as fp32.
+ *   x [T,H] act, w_g [E,H] act, logits [T,E] fp32 out (device).
+ *   ws: any workspace with a status word (at least 256 bytes).
+ * bf16 runs on the tcgen05 tensor cores (a one-group instance of the grouped
+ * GEMM), fp32 on CUDA cores (FFMA). Same shape limits as moe_expert_mlp. */
+moe_status_t moe_router_logits(const moe_config_t* cfg, const void* x, const void* w_g,
+                               float* logits, void* ws, size_t ws_bytes, void* stream);
 
 /* Bytes of the fixed device scratch area used by moe_route_topk_noalloc. */
 #define MOE_NOALLOC_SCRATCH_BYTES (1u << 20)
@@ -240,6 +264,15 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const float* logits, con
                                const void* w_gu, const void* w_d, void* out,
                                uint32_t flags, void* ws, size_t ws_bytes,
                                moe_layer_aux_t* aux, void* stream);
+
+/* The layer from hidden states: moe_router_logits (into the workspace) ->
+ * moe_route_topk_biased -> dispatch -> expert MLP -> combine. w_g [E,H] act;
+ * sel_bias [E] fp32 or NULL. flags: MOE_FLAG_NONE or MOE_FLAG_OVERLAP, as for
+ * moe_layer_forward. aux->logits receives the logits' workspace address. */
+moe_status_t moe_layer_forward_x(const moe_config_t* cfg, const void* x, const void* w_g,
+                                 const float* sel_bias, const void* w_gu, const void* w_d,
+                                 void* out, uint32_t flags, void* ws, size_t ws_bytes,
+                                 moe_layer_aux_t* aux, void* stream);
 
 /* Synchronise `stream`, read the workspace's status word into *status and reset
  * it to MOE_OK. Returns MOE_ERR_CUDA if the synchronisation or copy failed. */

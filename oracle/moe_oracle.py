@@ -126,22 +126,32 @@ def max_rows(T: int, K: int, E: int, C: int, A: int) -> int:
 # Route: top-K and softmax weights
 # ----------------------------------------------------------------------------
 
-def route_topk(logits: np.ndarray, K: int):
+def router_logits(x: np.ndarray, w_g: np.ndarray, act: str) -> np.ndarray:
+    """The router's linear layer: logits[t,e] = sum_h x[t,h] * w_g[e,h]
+    (pplx-kernels page, "Introductie": a small linear layer gives the router's
+    distribution), exact float64 sums of the widened inputs, stored as fp32."""
+    return (act_to_f64(x, act) @ act_to_f64(w_g, act).T).astype(np.float32)
+
+
+def route_topk(logits: np.ndarray, K: int, sel_bias: np.ndarray | None = None):
     """Top-K experts per token and their weights.
 
-    Selection orders experts by (fp32 logit descending, index ascending); a
-    stable sort of the negated logits realises exactly that order.  The
-    weights are the softmax over the K selected logits, i.e. the router's
-    probability distribution renormalised to the chosen experts
-    (pplx-kernels page, "Introductie"): w_k = exp(l_k - l_0) / sum_j exp(l_j - l_0),
+    Selection orders experts by (fp32 key descending, index ascending) where
+    the key is the logit, or the fp32 sum logit + sel_bias[e] when a
+    selection-only bias is given; a stable sort of the negated keys realises
+    exactly that order.  The weights are the softmax over the K selected
+    (unbiased) logits, i.e. the router's probability distribution renormalised
+    to the chosen experts (pplx-kernels page, "Introductie"):
+    w_k = exp(l_k - m) / sum_j exp(l_j - m) with m the largest selected logit,
     in float64, stored as float32.
     """
     lg = np.asarray(logits, dtype=np.float32)
     T, E = lg.shape
-    order = np.argsort(-lg, axis=1, kind="stable")
+    key = lg if sel_bias is None else lg + np.asarray(sel_bias, dtype=np.float32)[None, :]
+    order = np.argsort(-key, axis=1, kind="stable")
     idx = order[:, :K].astype(np.int32)
     sel = np.take_along_axis(lg, idx, axis=1).astype(np.float64)
-    ex = np.exp(sel - sel[:, :1])
+    ex = np.exp(sel - sel.max(axis=1, keepdims=True))
     w = (ex / ex.sum(axis=1, keepdims=True)).astype(np.float32)
     return idx, w
 
@@ -217,12 +227,12 @@ def permutation(topk_idx: np.ndarray, E: int, C: int, off: np.ndarray, R_max: in
     return slot, row_src
 
 
-def route(logits: np.ndarray, K: int, C: int, A: int, S: int):
+def route(logits: np.ndarray, K: int, C: int, A: int, S: int, sel_bias: np.ndarray | None = None):
     """Steps a1-a3 together: top-K, histogram, capacity/overflow, offsets and
     the permutation.  Returns a dict of the route outputs."""
     lg = np.asarray(logits, dtype=np.float32)
     T, E = lg.shape
-    idx, w = route_topk(lg, K)
+    idx, w = route_topk(lg, K, sel_bias)
     cnt = expert_histogram(idx, E)
     kept, overflow, effective, total_overflow = capacity_overflow(cnt, C)
     off, seg = aligned_offsets(kept, A, S)

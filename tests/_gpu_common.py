@@ -95,3 +95,23 @@ def assert_close_act(gpu_act: np.ndarray, ref_act: np.ndarray, act: str, what: s
     else:
         bound = F32_TOL * np.abs(r).max()
         assert diff.max() <= bound, f"{what}: max|err| {diff.max():.3e} > {bound:.3e}"
+
+
+def assert_layer_stages(gpu: dict, gpu_out: np.ndarray, x: np.ndarray, w_gu: np.ndarray,
+                        w_d: np.ndarray, ref: dict, ref_out: np.ndarray, act: str):
+    """End-to-end check stage by stage, each against the oracle with the stated
+    tolerance: xp bit-exact; y against the oracle's MLP on the same rows; out
+    against the oracle's combine of the GPU's own y. (Comparing out with the
+    oracle's whole chain element-wise would compound two independent bf16
+    roundings, y's and out's.) The whole chain must also agree within a relative
+    Frobenius error of 1e-2."""
+    kept = ref["row_src"] >= 0
+    assert np.array_equal(gpu["xp"][kept], ref["xp"][kept])
+    h_ref, y_ref = O.expert_mlp(gpu["xp"], ref["expert_offsets"], ref["kept"], w_gu, w_d, act)
+    assert_close_act(gpu["y"][kept], y_ref[kept], act, "y")
+    out_from_gpu_y = O.combine(gpu["y"], ref["token_slot"], ref["topk_w"], act)
+    assert_close_act(gpu_out, out_from_gpu_y, act, "out")
+    g = O.act_to_f64(gpu_out, act)
+    r = O.act_to_f64(ref_out, act)
+    fro = np.sqrt(np.sum((g - r) ** 2)) / max(np.sqrt(np.sum(r * r)), 1e-300)
+    assert fro <= 1e-2, f"whole chain: relative Frobenius error {fro:.3e}"

@@ -451,3 +451,44 @@ def test_planted_mistakes_are_caught(monkeypatch):
     swapped = torch.cat([w_gu[0, F:], w_gu[0, :F]])                           # gate/up swapped
     h_sw, _ = O.expert_mlp_rows(x.numpy(), swapped.numpy(), w_d[0].numpy(), O.ACT_F32)
     assert not np.allclose(h_sw, ref, rtol=1e-3)
+
+
+# ----------------------------------------------------------------------------
+# router projection and the selection-only bias
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("act", [O.ACT_F32, O.ACT_BF16])
+def test_router_logits_equal_torch_matmul(act):
+    g = torch.Generator().manual_seed(21)
+    x = torch.randn(33, 96, generator=g)
+    w_g = torch.randn(13, 96, generator=g) / 10
+    if act == O.ACT_BF16:
+        x, w_g = x.to(torch.bfloat16), w_g.to(torch.bfloat16)
+        to_np = bf16_bits_of
+    else:
+        to_np = lambda t: t.numpy()  # noqa: E731
+    got = O.router_logits(to_np(x), to_np(w_g), act)
+    ref = (x.double() @ w_g.double().T).float().numpy()     # x W_g^T, not W_g x
+    assert got.dtype == np.float32 and got.shape == (33, 13)
+    assert np.array_equal(got, ref)
+
+
+def test_selection_bias_brute_force():
+    g = torch.Generator().manual_seed(22)
+    lg = torch.randn(60, 12, generator=g).numpy()
+    bias = (torch.randn(12, generator=g) * 0.7).numpy().astype(np.float32)
+    K = 4
+    idx, w = O.route_topk(lg, K, bias)
+    for t in range(60):
+        keys = [np.float32(lg[t, e]) + np.float32(bias[e]) for e in range(12)]
+        assert list(idx[t]) == brute_topk(keys, K)
+        sel = [float(lg[t, e]) for e in idx[t]]          # weights from the unbiased logits
+        m = max(sel)
+        ex = [math.exp(v - m) for v in sel]
+        assert np.allclose(w[t], [v / sum(ex) for v in ex], rtol=1e-7)
+    # a bias that reorders the experts changes the selection but not how weights are made
+    big = np.zeros(12, np.float32)
+    big[11] = 100.0
+    idx2, w2 = O.route_topk(lg, 1, big)
+    assert np.all(idx2[:, 0] == 11) and np.all(w2 == 1.0)
+    assert np.array_equal(O.route_topk(lg, K, np.zeros(12, np.float32))[0], O.route_topk(lg, K)[0])

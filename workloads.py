@@ -97,8 +97,12 @@ def _normal(shape, std, dtype, gen, device, chunk_elems=1 << 28):
     return out
 
 
-def make_inputs(w: Workload, seed: int = 0, device="cpu", weights: bool = True):
-    """Return dict(logits, x, w_gu, w_d) drawn in a fixed order from one seeded generator."""
+def make_inputs(w: Workload, seed: int = 0, device="cpu", weights: bool = True,
+                router: bool = False):
+    """Return dict(logits, x, w_gu, w_d) drawn in a fixed order from one seeded
+    generator; with router=True also the router weights w_g [E,H] ~ N(0, 1/H)
+    (so that x w_g^T has unit variance) and a selection-only bias sel_bias [E]
+    ~ N(0, 0.1^2), drawn after the others."""
     gen = torch.Generator(device=device)
     gen.manual_seed(seed)
     logits = make_router_logits(w, gen, device)
@@ -107,6 +111,9 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu", weights: bool = True):
     if weights:
         out["w_gu"] = _normal((w.E, 2 * w.F, w.H), 0.02, w.torch_act, gen, device)
         out["w_d"] = _normal((w.E, w.H, w.F), 0.02, w.torch_act, gen, device)
+    if router:
+        out["w_g"] = _normal((w.E, w.H), w.H ** -0.5, w.torch_act, gen, device)
+        out["sel_bias"] = torch.randn(w.E, generator=gen, device=device, dtype=torch.float32) * 0.1
     return out
 
 
