@@ -317,11 +317,14 @@ def expert_mlp(xp: np.ndarray, expert_offsets: np.ndarray, kept: np.ndarray,
 # Combine
 # ----------------------------------------------------------------------------
 
-def combine(y: np.ndarray, token_slot: np.ndarray, topk_w: np.ndarray, act: str) -> np.ndarray:
+def combine(y: np.ndarray, token_slot: np.ndarray, topk_w: np.ndarray, act: str,
+            y_shared: np.ndarray | None = None) -> np.ndarray:
     """out[t] = sum over k with slot[t,k] != -1 of w[t,k] * y[slot[t,k]], summed
-    in float64 in k order and rounded once to the activation dtype.  Dropped
+    in float64 in k order, plus the shared expert's output y_shared[t] (weight
+    1) when there is one, rounded once to the activation dtype.  Dropped
     assignments contribute nothing and the remaining weights are not
-    renormalised; a token with every assignment dropped gets zeros."""
+    renormalised; a token with every assignment dropped (and no shared
+    expert) gets zeros."""
     slot = np.asarray(token_slot)
     T, K = slot.shape
     H = y.shape[1]
@@ -331,6 +334,8 @@ def combine(y: np.ndarray, token_slot: np.ndarray, topk_w: np.ndarray, act: str)
         s = slot[:, k]
         m = s >= 0
         acc[m] += w[m, k][:, None] * act_to_f64(y[s[m]], act)
+    if y_shared is not None:
+        acc += act_to_f64(y_shared, act)
     return f64_to_act(acc, act)
 
 
@@ -338,11 +343,19 @@ def combine(y: np.ndarray, token_slot: np.ndarray, topk_w: np.ndarray, act: str)
 # The whole layer
 # ----------------------------------------------------------------------------
 
-def layer_forward(logits, x, w_gu, w_d, K: int, C: int, A: int, S: int, act: str):
-    """route -> dispatch -> expert MLP -> combine.  Returns (out, intermediates)."""
+def layer_forward(logits, x, w_gu, w_d, K: int, C: int, A: int, S: int, act: str,
+                  n_shared: int = 0):
+    """route -> dispatch -> expert MLP -> combine.  With n_shared = 1 the last
+    expert of w_gu / w_d is a shared expert that every token uses with weight 1
+    on top of its routed experts (its rows are the tokens themselves).
+    Returns (out, intermediates)."""
+    E_routed = w_gu.shape[0] - n_shared
     r = route(logits, K, C, A, S)
     xp = dispatch(x, r["token_slot"], r["R_max"])
-    h, y = expert_mlp(xp, r["expert_offsets"], r["kept"], w_gu, w_d, act)
-    out = combine(y, r["token_slot"], r["topk_w"], act)
-    r.update(xp=xp, h=h, y=y)
+    h, y = expert_mlp(xp, r["expert_offsets"], r["kept"], w_gu[:E_routed], w_d[:E_routed], act)
+    y_sh = None
+    if n_shared:
+        _, y_sh = expert_mlp_rows(x, w_gu[E_routed], w_d[E_routed], act)
+    out = combine(y, r["token_slot"], r["topk_w"], act, y_shared=y_sh)
+    r.update(xp=xp, h=h, y=y, y_shared=y_sh)
     return out, r

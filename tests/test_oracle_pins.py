@@ -492,3 +492,28 @@ def test_selection_bias_brute_force():
     idx2, w2 = O.route_topk(lg, 1, big)
     assert np.all(idx2[:, 0] == 11) and np.all(w2 == 1.0)
     assert np.array_equal(O.route_topk(lg, K, np.zeros(12, np.float32))[0], O.route_topk(lg, K)[0])
+
+
+# ----------------------------------------------------------------------------
+# shared expert
+# ----------------------------------------------------------------------------
+
+def test_shared_expert_adds_a_dense_swiglu_of_every_token():
+    # E routed experts with all-dropped routing (C = 0) leave only the shared
+    # expert: out must be torch's dense SwiGLU of x with the shared weights.
+    T, H, F, E = 21, 16, 24, 3
+    g = torch.Generator().manual_seed(31)
+    x = torch.randn(T, H, generator=g)
+    w_gu = torch.randn(E + 1, 2 * F, H, generator=g) * 0.3
+    w_d = torch.randn(E + 1, H, F, generator=g) * 0.3
+    lg = torch.randn(T, E, generator=g).numpy()
+    out, r = O.layer_forward(lg, x.numpy(), w_gu.numpy(), w_d.numpy(), 2, 0, 1, 1, O.ACT_F32,
+                             n_shared=1)
+    ref = torch_swiglu(x.double(), w_gu[E].double(), w_d[E].double()) @ w_d[E].double().T
+    assert np.allclose(out, ref.numpy(), rtol=1e-5, atol=1e-7)
+    # with routing kept, out = routed combine + shared output (the routed part unchanged)
+    out2, r2 = O.layer_forward(lg, x.numpy(), w_gu.numpy(), w_d.numpy(), 2, T, 1, 1, O.ACT_F32,
+                               n_shared=1)
+    routed = O.combine(r2["y"], r2["token_slot"], r2["topk_w"], O.ACT_F32)
+    assert np.allclose(out2, routed + r2["y_shared"], rtol=1e-5, atol=1e-6)
+    assert not np.allclose(out2, routed, rtol=1e-3)
