@@ -167,7 +167,8 @@ class Layer:
         self.router = router
         self.wl = wl
         self.C = M.moe_capacity(wl.T, wl.K, wl.E, wl.cf)
-        self.cfg = M.make_config(wl.T, wl.H, wl.E, wl.K, wl.F, wl.S, self.C, wl.row_align, wl.act)
+        self.cfg = M.make_config(wl.T, wl.H, wl.E, wl.K, wl.F, wl.S, self.C, wl.row_align, wl.act,
+                                 n_shared=wl.n_shared)
         st = M.moe_check_config(self.cfg)
         if st != M.MOE_OK:
             raise SystemExit(f"unsupported workload: {M.status_string(st)}")
@@ -282,15 +283,17 @@ def algorithmic(layer: Layer, totals, counts):
     T, H, F, K, E = wl.T, wl.H, wl.F, wl.K, wl.E
     tr = mlp_tile_rows(layer)
     kept = np.minimum(np.asarray(counts), layer.C)
-    executed = int(np.sum((kept + tr - 1) // tr * tr))
+    # the shared expert (if any) is one more group of T rows
+    Ns = wl.n_shared * T
+    executed = int(np.sum((kept + tr - 1) // tr * tr)) + (Ns + tr - 1) // tr * tr
     return {
         "N": N,
         "tile_rows": tr,
         "executed_rows": executed,
-        "mlp_flops": 6.0 * N * H * F,
+        "mlp_flops": 6.0 * (N + Ns) * H * F,
         "mlp_executed_flops": 6.0 * executed * H * F,
-        "dispatch_bytes": (T + N) * H * s + T * K * 4,
-        "combine_bytes": (N + T) * H * s + T * K * 8,
+        "dispatch_bytes": (T + N + Ns) * H * s + T * K * 4,
+        "combine_bytes": (N + Ns + T) * H * s + T * K * 8,
         "route_bytes": T * E * 4 + T * K * 12,
     }
 
@@ -312,7 +315,7 @@ def cpu_oracle_sample(wl: W.Workload, tokens: int, seed: int, inp_host=None):
     w_gu, w_d = np_act(inp_host["w_gu"]), np_act(inp_host["w_d"])
     C = O.capacity(tokens, wl.K, wl.E, wl.cf)
     t0 = time.perf_counter()
-    O.layer_forward(lg, x, w_gu, w_d, wl.K, C, wl.row_align, wl.S, wl.act)
+    O.layer_forward(lg, x, w_gu, w_d, wl.K, C, wl.row_align, wl.S, wl.act, n_shared=wl.n_shared)
     return time.perf_counter() - t0, tokens
 
 
@@ -367,10 +370,14 @@ def main(argv=None):
                          "selection-only bias (moe_layer_forward_x)")
     ap.add_argument("--overlap", action="store_true",
                     help="overlap the combine with the down GEMM (MOE_FLAG_OVERLAP)")
+    ap.add_argument("--shared", action="store_true",
+                    help="add one shared expert of the routed width (as DeepSeek-V3 and Kimi-K2 have)")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         raise SystemExit("--warmup must be >= 3")
     wl = W.WORKLOADS[args.workload]
+    if args.shared:
+        wl = wl.with_(name=wl.name + "_shared", n_shared=1)
     world, rank, local = dist_env()
     if args.impl == "reference":
         return run_reference(args, wl, world, rank)
@@ -458,7 +465,8 @@ def main(argv=None):
                    "S": wl.S, "cf": wl.cf, "capacity": layer.C, "row_align": wl.row_align,
                    "effective_tokens": alg["N"], "overflow": int(totals[2]),
                    "l2": "flushed (256 MB write) before every step", "parallelism": f"replicas{world}",
-                   "overlap": bool(args.overlap), "router_projection": bool(args.router)},
+                   "overlap": bool(args.overlap), "router_projection": bool(args.router),
+                   "n_shared": wl.n_shared},
         "e2e": {"value": world * wl.T / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": (KERNELS_PER_STEP + (1 if args.router else 0)) * args.steps,

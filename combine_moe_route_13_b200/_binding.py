@@ -46,7 +46,7 @@ class MoeConfig(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("E", ctypes.c_int32),
                 ("K", ctypes.c_int32), ("F", ctypes.c_int32), ("S", ctypes.c_int32),
                 ("capacity", ctypes.c_int32), ("row_align", ctypes.c_int32),
-                ("act_dtype", ctypes.c_int32)]
+                ("act_dtype", ctypes.c_int32), ("n_shared", ctypes.c_int32)]
 
     def __repr__(self):
         return ("MoeConfig(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")")
@@ -131,9 +131,15 @@ def _ptr(t: torch.Tensor | None, dtype=None, name="tensor") -> int | None:
     return t.data_ptr()
 
 
-def make_config(T, H, E, K, F, S, capacity, row_align=128, act="bf16") -> MoeConfig:
+def make_config(T, H, E, K, F, S, capacity, row_align=128, act="bf16", n_shared=0) -> MoeConfig:
     return MoeConfig(int(T), int(H), int(E), int(K), int(F), int(S), int(capacity),
-                     int(row_align), MOE_F32 if act in ("f32", torch.float32, MOE_F32) else MOE_BF16)
+                     int(row_align), MOE_F32 if act in ("f32", torch.float32, MOE_F32) else MOE_BF16,
+                     int(n_shared))
+
+
+def shared_row0(cfg: MoeConfig) -> int:
+    """First row of the shared expert in xp / h / y (the rows before it are routed)."""
+    return moe_max_rows(cfg) - cfg.n_shared * cfg.T
 
 
 def act_dtype(cfg: MoeConfig) -> torch.dtype:

@@ -10,7 +10,8 @@
 // Both are pure HBM streams. One block per token row; each thread moves
 // 16-byte vectors (8 bf16 or 4 fp32), several per iteration so that enough
 // loads are in flight. A dispatched row is read once and written K times;
-// a combined row reads its K expert rows and is written once.
+// a combined row reads its K expert rows and is written once. A shared
+// expert adds one row per token to both (its copy of x, its output row).
 #include <algorithm>
 
 #include <cuda_bf16.h>
@@ -27,10 +28,12 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) { return __ldcs(p); }
 
 __global__ void __launch_bounds__(DC_THREADS)
 dispatch_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ token_slot,
-                uint4* __restrict__ xp, int K, int row_vecs) {
-  __shared__ int s_slot[MAX_K];
+                uint4* __restrict__ xp, int K, int row_vecs, long long sh_row0) {
+  __shared__ int s_slot[MAX_K + 1];
   __shared__ int s_any;
   const int t = blockIdx.x;
+  // the shared expert's row of this token is one more destination
+  const int KD = sh_row0 >= 0 ? K + 1 : K;
   if (threadIdx.x == 0) s_any = 0;
   pdl_wait();
   pdl_trigger();
@@ -39,6 +42,9 @@ dispatch_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ token_s
     const int s = token_slot[(size_t)t * K + threadIdx.x];
     s_slot[threadIdx.x] = s;
     if (s >= 0) atomicOr(&s_any, 1);
+  } else if (threadIdx.x == K && KD > K) {
+    s_slot[K] = (int)(sh_row0 + t);
+    s_any = 1;
   }
   __syncthreads();
   if (!s_any) return;   // every assignment of this token overflowed: nothing to copy
@@ -50,7 +56,7 @@ dispatch_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ token_s
       const int v = v0 + u * DC_THREADS;
       if (v < row_vecs) d[u] = ld_stream(src + v);
     }
-    for (int k = 0; k < K; ++k) {
+    for (int k = 0; k < KD; ++k) {
       const int s = s_slot[k];
       if (s < 0) continue;
       uint4* dst = xp + (size_t)s * row_vecs;
@@ -77,11 +83,62 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&b);
 }
 
-// out[t] = sum_k w[t,k] * y[slot[t,k]] with fp32 accumulation in k order.
+template <bool BF16>
+using Acc = float[2][BF16 ? 8 : 4];   // the two 16-byte vectors a thread accumulates
+
+// acc += row (weight 1): the shared expert's term, after the routed ones.
+// COHERENT: plain loads, for rows written while the kernel runs.
+template <bool BF16, bool COHERENT>
+__device__ __forceinline__ void add_row(const uint4* row, int v0, int row_vecs, Acc<BF16>& acc) {
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int v = v0 + u * DC_THREADS;
+    if (v >= row_vecs) continue;
+    const uint4 d = COHERENT ? row[v] : __ldg(row + v);
+    if (BF16) {
+      float f[8];
+      unpack_bf16x8(d, f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[u][i] += f[i];
+    } else {
+      acc[u][0] += __uint_as_float(d.x);
+      acc[u][1] += __uint_as_float(d.y);
+      acc[u][2] += __uint_as_float(d.z);
+      acc[u][3] += __uint_as_float(d.w);
+    }
+  }
+}
+
+// Round the accumulators once to the activation dtype and store them.
+template <bool BF16>
+__device__ __forceinline__ void store_acc(uint4* dst, int v0, int row_vecs, const Acc<BF16>& acc) {
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int v = v0 + u * DC_THREADS;
+    if (v >= row_vecs) continue;
+    uint4 o;
+    if (BF16) {
+      o.x = pack_bf16x2(acc[u][0], acc[u][1]);
+      o.y = pack_bf16x2(acc[u][2], acc[u][3]);
+      o.z = pack_bf16x2(acc[u][4], acc[u][5]);
+      o.w = pack_bf16x2(acc[u][6], acc[u][7]);
+    } else {
+      o.x = __float_as_uint(acc[u][0]);
+      o.y = __float_as_uint(acc[u][1]);
+      o.z = __float_as_uint(acc[u][2]);
+      o.w = __float_as_uint(acc[u][3]);
+    }
+    __stcs(dst + v, o);
+  }
+}
+
+// out[t] = sum_k w[t,k] * y[slot[t,k]] with fp32 accumulation in k order,
+// plus y[sh_row0 + t] when sh_row0 >= 0 (the shared expert).
 template <bool BF16>
 __global__ void __launch_bounds__(DC_THREADS)
 combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ token_slot,
-               const float* __restrict__ topk_w, uint4* __restrict__ out, int K, int row_vecs) {
+               const float* __restrict__ topk_w, uint4* __restrict__ out, int K, int row_vecs,
+               long long sh_row0) {
   __shared__ int s_slot[MAX_K];
   __shared__ float s_w[MAX_K];
   const int t = blockIdx.x;
@@ -95,7 +152,7 @@ combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ token_sl
   constexpr int LANES = BF16 ? 8 : 4;
   uint4* dst = out + (size_t)t * row_vecs;
   for (int v0 = threadIdx.x; v0 < row_vecs; v0 += DC_THREADS * 2) {
-    float acc[2][LANES];
+    Acc<BF16> acc;
 #pragma unroll
     for (int u = 0; u < 2; ++u)
 #pragma unroll
@@ -134,24 +191,8 @@ combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ token_sl
         }
       }
     }
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int v = v0 + u * DC_THREADS;
-      if (v >= row_vecs) continue;
-      uint4 o;
-      if (BF16) {
-        o.x = pack_bf16x2(acc[u][0], acc[u][1]);
-        o.y = pack_bf16x2(acc[u][2], acc[u][3]);
-        o.z = pack_bf16x2(acc[u][4], acc[u][5]);
-        o.w = pack_bf16x2(acc[u][6], acc[u][7]);
-      } else {
-        o.x = __float_as_uint(acc[u][0]);
-        o.y = __float_as_uint(acc[u][1]);
-        o.z = __float_as_uint(acc[u][2]);
-        o.w = __float_as_uint(acc[u][3]);
-      }
-      __stcs(dst + v, o);
-    }
+    if (sh_row0 >= 0) add_row<BF16, false>(y + (size_t)(sh_row0 + t) * row_vecs, v0, row_vecs, acc);
+    store_acc<BF16>(dst, v0, row_vecs, acc);
   }
 }
 
@@ -179,22 +220,25 @@ template <bool BF16>
 __global__ void __launch_bounds__(DC_THREADS)
 combine_wait_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ token_slot,
                     const float* __restrict__ topk_w, uint4* __restrict__ out, int K,
-                    int row_vecs, const uint32_t* row_ready, uint32_t target,
+                    int row_vecs, long long sh_row0, const uint32_t* row_ready, uint32_t target,
                     unsigned long long timeout_ns, uint32_t* status) {
-  __shared__ int s_slot[MAX_K];
+  __shared__ int s_slot[MAX_K + 1];
   __shared__ float s_w[MAX_K];
   __shared__ int s_ok;
   pdl_trigger();   // no griddepcontrol.wait: the ready counters carry the dependency
   const int t = blockIdx.x;
+  const int KW = sh_row0 >= 0 ? K + 1 : K;   // rows to wait for, the shared one last
   if (threadIdx.x < K) {
     s_slot[threadIdx.x] = token_slot[(size_t)t * K + threadIdx.x];
     s_w[threadIdx.x] = topk_w[(size_t)t * K + threadIdx.x];
+  } else if (threadIdx.x == K && KW > K) {
+    s_slot[K] = (int)(sh_row0 + t);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = 1;
     const unsigned long long t0 = globaltimer();
-    for (int k = 0; k < K && ok; ++k) {
+    for (int k = 0; k < KW && ok; ++k) {
       const int sl = s_slot[k];
       if (sl < 0) continue;
       const uint32_t* flag = row_ready + sl / READY_ROWS;
@@ -216,7 +260,7 @@ combine_wait_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ tok
   constexpr int LANES = BF16 ? 8 : 4;
   uint4* dst = out + (size_t)t * row_vecs;
   for (int v0 = threadIdx.x; v0 < row_vecs; v0 += DC_THREADS * 2) {
-    float acc[2][LANES];
+    Acc<BF16> acc;
 #pragma unroll
     for (int u = 0; u < 2; ++u)
 #pragma unroll
@@ -254,62 +298,41 @@ combine_wait_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ tok
         }
       }
     }
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int v = v0 + u * DC_THREADS;
-      if (v >= row_vecs) continue;
-      uint4 o;
-      if (BF16) {
-        o.x = pack_bf16x2(acc[u][0], acc[u][1]);
-        o.y = pack_bf16x2(acc[u][2], acc[u][3]);
-        o.z = pack_bf16x2(acc[u][4], acc[u][5]);
-        o.w = pack_bf16x2(acc[u][6], acc[u][7]);
-      } else {
-        o.x = __float_as_uint(acc[u][0]);
-        o.y = __float_as_uint(acc[u][1]);
-        o.z = __float_as_uint(acc[u][2]);
-        o.w = __float_as_uint(acc[u][3]);
-      }
-      __stcs(dst + v, o);
-    }
+    if (sh_row0 >= 0) add_row<BF16, true>(y + (size_t)(sh_row0 + t) * row_vecs, v0, row_vecs, acc);
+    store_acc<BF16>(dst, v0, row_vecs, acc);
   }
 }
 
 }  // namespace
 
 cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t* slot, void* xp,
-                            cudaStream_t s) {
+                            int64_t sh_row0, cudaStream_t s) {
   if (c.T == 0) return cudaSuccess;
   const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
   return launch_pdl(dispatch_kernel, dim3(c.T), dim3(DC_THREADS), 0, s,
-                    static_cast<const uint4*>(x), slot, static_cast<uint4*>(xp), c.K, row_vecs);
+                    static_cast<const uint4*>(x), slot, static_cast<uint4*>(xp), c.K, row_vecs,
+                    (long long)sh_row0);
 }
 
 cudaError_t launch_combine(const moe_config_t& c, const void* y, const int32_t* slot,
-                           const float* w, void* out, cudaStream_t s) {
+                           const float* w, int64_t sh_row0, void* out, cudaStream_t s) {
   if (c.T == 0) return cudaSuccess;
   const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
-  if (c.act_dtype == MOE_BF16)
-    return launch_pdl(combine_kernel<true>, dim3(c.T), dim3(DC_THREADS), 0, s,
-                      static_cast<const uint4*>(y), slot, w, static_cast<uint4*>(out), c.K,
-                      row_vecs);
-  return launch_pdl(combine_kernel<false>, dim3(c.T), dim3(DC_THREADS), 0, s,
-                    static_cast<const uint4*>(y), slot, w, static_cast<uint4*>(out), c.K, row_vecs);
+  auto kernel = c.act_dtype == MOE_BF16 ? combine_kernel<true> : combine_kernel<false>;
+  return launch_pdl(kernel, dim3(c.T), dim3(DC_THREADS), 0, s, static_cast<const uint4*>(y), slot,
+                    w, static_cast<uint4*>(out), c.K, row_vecs, (long long)sh_row0);
 }
 
 cudaError_t launch_combine_wait(const moe_config_t& c, const void* y, const int32_t* slot,
-                                const float* w, const uint32_t* row_ready, uint32_t target,
-                                unsigned long long timeout_ns, uint32_t* status, void* out,
-                                cudaStream_t s) {
+                                const float* w, int64_t sh_row0, const uint32_t* row_ready,
+                                uint32_t target, unsigned long long timeout_ns, uint32_t* status,
+                                void* out, cudaStream_t s) {
   if (c.T == 0) return cudaSuccess;
   const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
-  if (c.act_dtype == MOE_BF16)
-    return launch_pdl(combine_wait_kernel<true>, dim3(c.T), dim3(DC_THREADS), 0, s,
-                      static_cast<const uint4*>(y), slot, w, static_cast<uint4*>(out), c.K,
-                      row_vecs, row_ready, target, timeout_ns, status);
-  return launch_pdl(combine_wait_kernel<false>, dim3(c.T), dim3(DC_THREADS), 0, s,
-                    static_cast<const uint4*>(y), slot, w, static_cast<uint4*>(out), c.K,
-                    row_vecs, row_ready, target, timeout_ns, status);
+  auto kernel = c.act_dtype == MOE_BF16 ? combine_wait_kernel<true> : combine_wait_kernel<false>;
+  return launch_pdl(kernel, dim3(c.T), dim3(DC_THREADS), 0, s, static_cast<const uint4*>(y), slot,
+                    w, static_cast<uint4*>(out), c.K, row_vecs, (long long)sh_row0, row_ready,
+                    target, timeout_ns, status);
 }
 
 }  // namespace moe

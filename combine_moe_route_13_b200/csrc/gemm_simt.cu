@@ -8,6 +8,8 @@
 //
 // Each block computes a BM x BN tile of one expert: grid.y enumerates the
 // experts' M tiles (an upper bound; surplus blocks exit), grid.x the N tiles.
+// A shared expert (sh_rows > 0) is group E: rows [sh_row0, sh_row0 + sh_rows)
+// with the weights of expert E.
 // GATE_UP: out = silu(A Wg^T) * (A Wu^T) with Wg, Wu the two halves of w_gu[e];
 // otherwise out = A W^T.
 #include <algorithm>
@@ -24,33 +26,34 @@ __global__ void __launch_bounds__(NT)
 simt_grouped_gemm(const float* __restrict__ A, int Kdim, const float* __restrict__ W,
                   int w_rows_per_expert, int up_off, int N_out, float* __restrict__ out,
                   const int32_t* __restrict__ offsets, const int32_t* __restrict__ counts, int E,
-                  int C) {
-  __shared__ int mt_prefix[MAX_E + 1];
+                  int C, int sh_rows, long long sh_row0) {
+  __shared__ int mt_prefix[MAX_E + 2];
   __shared__ float As[BK][BM + 1];
   __shared__ float Bg[BK][BN + 1];
   __shared__ float Bu[GATE_UP ? BK : 1][BN + 1];
   // M tiles of each expert and their prefix (serial: E is small on this path)
+  const int G = sh_rows > 0 ? E + 1 : E;   // groups
   if (threadIdx.x == 0) {
     int p = 0;
-    for (int e = 0; e < E; ++e) {
+    for (int e = 0; e < G; ++e) {
       mt_prefix[e] = p;
-      p += (min(counts[e], C) + BM - 1) / BM;
+      p += ((e < E ? min(counts[e], C) : sh_rows) + BM - 1) / BM;
     }
-    mt_prefix[E] = p;
+    mt_prefix[G] = p;
   }
   __syncthreads();
   const int mt = blockIdx.y;
-  if (mt >= mt_prefix[E]) return;
-  int lo = 0, hi = E;     // expert e with mt_prefix[e] <= mt < mt_prefix[e+1]
+  if (mt >= mt_prefix[G]) return;
+  int lo = 0, hi = G;     // group e with mt_prefix[e] <= mt < mt_prefix[e+1]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (mt_prefix[mid] <= mt) lo = mid; else hi = mid;
   }
   const int e = lo;   // experts without tiles never satisfy the strict upper bound
-  const int kept = min(counts[e], C);
+  const int kept = e < E ? min(counts[e], C) : sh_rows;
   const int r0 = (mt - mt_prefix[e]) * BM;          // first row inside the expert
   const int rows = min(BM, kept - r0);
-  const int64_t row_base = (int64_t)offsets[e] + r0;
+  const int64_t row_base = (e < E ? (int64_t)offsets[e] : (int64_t)sh_row0) + r0;
   const int n0 = blockIdx.x * BN;
   const float* We = W + (int64_t)e * w_rows_per_expert * Kdim;
 
@@ -134,14 +137,16 @@ cudaError_t launch_router_f32(const moe_config_t& c, const float* x, const float
 cudaError_t launch_mlp_f32(const moe_config_t& c, const float* xp, const int32_t* offsets,
                            const int32_t* counts, const float* w_gu, const float* w_d, float* h,
                            float* y, int64_t R_max, cudaStream_t s) {
-  const int64_t mt_bound = ceil_div(R_max, BM) + c.E;   // >= sum_e ceil(kept_e / BM)
+  const int64_t mt_bound = ceil_div(R_max, BM) + c.E + 1;   // >= sum_e ceil(kept_e / BM)
+  const int sh_rows = c.n_shared ? c.T : 0;
+  const long long sh_row0 = c.n_shared ? shared_row0(c) : 0;
   if (mt_bound == 0 || mt_bound > 65535) return mt_bound == 0 ? cudaSuccess : cudaErrorInvalidValue;
   dim3 g1((unsigned)ceil_div(c.F, BN), (unsigned)mt_bound);
   simt_grouped_gemm<true><<<g1, NT, 0, s>>>(xp, c.H, w_gu, 2 * c.F, c.F, c.F, h, offsets, counts,
-                                            c.E, c.capacity);
+                                            c.E, c.capacity, sh_rows, sh_row0);
   dim3 g2((unsigned)ceil_div(c.H, BN), (unsigned)mt_bound);
   simt_grouped_gemm<false><<<g2, NT, 0, s>>>(h, c.F, w_d, c.H, 0, c.H, y, offsets, counts, c.E,
-                                             c.capacity);
+                                             c.capacity, sh_rows, sh_row0);
   return cudaGetLastError();
 }
 

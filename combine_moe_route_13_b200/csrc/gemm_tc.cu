@@ -420,12 +420,12 @@ __device__ __forceinline__ void decode_tile(int tile, int NT, const int* P, int 
 template <int MODE, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ CUtensorMap tmOut, void* __restrict__ out_v,
-                int N_out, int Kdim, int b_rows_per_expert,
+                const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ CUtensorMap tmA2,
+                void* __restrict__ out_v, int N_out, int Kdim, int b_rows_per_expert,
                 int b_second_off, const int32_t* __restrict__ offsets,
                 const int32_t* __restrict__ counts, int E, int C, long long R_max,
                 uint32_t* __restrict__ status, uint32_t* __restrict__ row_ready,
-                int dense_rows) {
+                int dense_rows, int sh_rows, int sh_a_row, int sh_out_row) {
   using CF = Cfg<CG>;
   constexpr int STAGES = CF::STAGES;
   constexpr int BN_OUT = (MODE == 0) ? 128 : 256;   // output columns per tile
@@ -437,9 +437,12 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   uint8_t* smem = smem_raw + (base - raw);
   const uint32_t staging = base + STAGES * CF::STAGE_BYTES;   // epilogue output box
   Ctl* ctl = reinterpret_cast<Ctl*>(smem + STAGES * CF::STAGE_BYTES + STAGING_BYTES);
-  int* P = reinterpret_cast<int*>(ctl + 1);   // [E+1] M-tile prefix
-  int* row_off = P + (E + 1);                 // [E+1] first row of each expert, and R
-  int* kept_s = row_off + (E + 1);            // [E]
+  // Groups: the E routed experts, then (sh_rows > 0) the shared expert, whose
+  // sh_rows rows are read from tmA2 at row sh_a_row and written at sh_out_row.
+  const int G = sh_rows > 0 ? E + 1 : E;
+  int* P = reinterpret_cast<int*>(ctl + 1);   // [G+1] M-tile prefix
+  int* row_off = P + (G + 1);                 // [G+1] first output row of each group, and its end
+  int* kept_s = row_off + (G + 1);            // [G]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;   // position in the pair
@@ -464,6 +467,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     prefetch_map(&tmA);
     prefetch_map(&tmB);
     prefetch_map(&tmOut);
+    if (G > E) prefetch_map(&tmA2);
   }
   if (warp == 1) {
     tmem_alloc<CG>(saddr(&ctl->tmem_base), TMEM_COLS);
@@ -471,17 +475,19 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   }
   pdl_wait();      // everything above touched only this CTA's shared memory and TMEM
   pdl_trigger();
-  {  // per-expert kept rows, first row and M-tile prefix (block scan)
-    const int chunk = (E + NUM_THREADS - 1) / NUM_THREADS;
+  {  // per-group kept rows, first row and M-tile prefix (block scan)
+    const int chunk = (G + NUM_THREADS - 1) / NUM_THREADS;
     const int e0 = threadIdx.x * chunk;
     int local = 0;
     for (int i = 0; i < chunk; ++i) {
       const int e = e0 + i;
-      if (e < E) {
+      if (e < G) {
         // dense_rows > 0: one group of dense_rows rows starting at row 0
-        const int k = dense_rows > 0 ? dense_rows : max(0, min(counts[e], C));
+        const int k = dense_rows > 0 ? dense_rows
+                      : e < E        ? max(0, min(counts[e], C))
+                                     : sh_rows;
         kept_s[e] = k;
-        row_off[e] = dense_rows > 0 ? 0 : offsets[e];
+        row_off[e] = dense_rows > 0 ? 0 : (e < E ? offsets[e] : sh_out_row);
         local += (k + CF::TILE_ROWS - 1) / CF::TILE_ROWS;
       }
     }
@@ -497,14 +503,14 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     for (int w = 0; w < warp; ++w) run += ctl->wsum[w];
     for (int i = 0; i < chunk; ++i) {
       const int e = e0 + i;
-      if (e < E) {
+      if (e < G) {
         P[e] = run;
         run += (kept_s[e] + CF::TILE_ROWS - 1) / CF::TILE_ROWS;
       }
     }
     if (threadIdx.x == NUM_THREADS - 1) {
-      P[E] = run;
-      row_off[E] = dense_rows > 0 ? dense_rows : offsets[E];
+      P[G] = run;
+      row_off[G] = dense_rows > 0 ? dense_rows : (G > E ? sh_out_row + sh_rows : offsets[E]);
     }
   }
   tc_fence_before();
@@ -512,15 +518,17 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   if (CG == 2) cluster_sync();   // both CTAs' barriers exist before anyone signals them
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
-  const int total = P[E] * NT;
+  const int total = P[G] * NT;
 
   if (warp == 0) {
     if (lane == 0) {  // ------------------------------------------------ TMA producer
       int it = 0;
       for (int tile = cluster_id; tile < total; tile += n_clusters) {
         int e, m, n;
-        decode_tile(tile, NT, P, E, e, m, n);
-        const int a_row = row_off[e] + m * CF::TILE_ROWS + (int)rank * BM;
+        decode_tile(tile, NT, P, G, e, m, n);
+        const bool shared_group = e >= E;
+        const CUtensorMap* mapA = shared_group ? &tmA2 : &tmA;
+        const int a_row = (shared_group ? sh_a_row : row_off[e]) + m * CF::TILE_ROWS + (int)rank * BM;
         const int b_row0 = e * b_rows_per_expert + n * N_STEP;
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb, ++it) {
@@ -534,7 +542,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
           const uint32_t fb_local = saddr(&ctl->full[s]);
           const uint32_t fb = (CG == 2) ? map_to_rank(fb_local, 0) : fb_local;
           if (leader) mbar_expect_tx(fb_local, CF::STAGE_BYTES * CG);
-          tma_load_2d<CG>(sa, &tmA, kb * BK, a_row, fb);
+          tma_load_2d<CG>(sa, mapA, kb * BK, a_row, fb);
           if (CG == 2) {
             tma_load_2d<CG>(sa + BOX_BYTES, &tmB, kb * BK, b_row0 + (int)rank * b_second_off, fb);
           } else {
@@ -592,7 +600,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     int tcount = 0;
     for (int tile = cluster_id; tile < total; tile += n_clusters, ++tcount) {
       int e, m, n;
-      decode_tile(tile, NT, P, E, e, m, n);
+      decode_tile(tile, NT, P, G, e, m, n);
       const int first = m * CF::TILE_ROWS + (int)rank * BM;   // first row of this half tile
       const int rows = min(BM, kept_s[e] - first);
       const long long grow = (long long)row_off[e] + first + r_in;
@@ -797,15 +805,26 @@ template <int CG>
 moe_status_t launch_mlp(const moe_config_t& c, const void* xp, const int32_t* offsets,
                         const int32_t* counts, const void* w_gu, const void* w_d, void* h,
                         void* y, int64_t R_max, uint32_t* status, cudaStream_t s,
-                        uint32_t* row_ready) {
-  CUtensorMap mx, mwgu, mh, mwd, my;
+                        uint32_t* row_ready, const void* x_shared) {
+  const int n_sh = c.n_shared ? 1 : 0;
+  const int G = c.E + n_sh;   // routed experts + the shared expert (last in the weights)
+  CUtensorMap mx, mwgu, mh, mwd, my, mxs;
   if (!make_map(&mx, xp, (uint64_t)c.H, (uint64_t)R_max) ||
-      !make_map(&mwgu, w_gu, (uint64_t)c.H, (uint64_t)c.E * 2 * c.F) ||
+      !make_map(&mwgu, w_gu, (uint64_t)c.H, (uint64_t)G * 2 * c.F) ||
       !make_map(&mh, h, (uint64_t)c.F, (uint64_t)R_max) ||
-      !make_map(&mwd, w_d, (uint64_t)c.F, (uint64_t)c.E * c.H) ||
+      !make_map(&mwd, w_d, (uint64_t)c.F, (uint64_t)G * c.H) ||
       !make_map(&my, y, (uint64_t)c.H, (uint64_t)R_max))
     return MOE_ERR_CUDA;
-  const size_t smem = smem_bytes<CG>(c.E);
+  // The shared expert's gate/up rows: the caller's x, or xp's shared rows.
+  const int sh_rows = n_sh ? c.T : 0;
+  const int sh_row0 = n_sh ? (int)shared_row0(c) : 0;
+  int sh_a_row = sh_row0;
+  mxs = mx;
+  if (n_sh && x_shared) {
+    if (!make_map(&mxs, x_shared, (uint64_t)c.H, (uint64_t)c.T)) return MOE_ERR_CUDA;
+    sh_a_row = 0;
+  }
+  const size_t smem = smem_bytes<CG>(G);
   if (cudaFuncSetAttribute(tc_grouped_gemm<0, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess ||
       cudaFuncSetAttribute(tc_grouped_gemm<1, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -813,22 +832,22 @@ moe_status_t launch_mlp(const moe_config_t& c, const void* xp, const int32_t* of
     return MOE_ERR_CUDA;
   const int units = resident_units<0, CG>(smem);
   if (units <= 0) return MOE_ERR_CUDA;
-  const int64_t mt_bound = ceil_div(R_max, Cfg<CG>::TILE_ROWS) + c.E;  // >= sum_e M tiles
+  const int64_t mt_bound = ceil_div(R_max, Cfg<CG>::TILE_ROWS) + G;  // >= sum over groups of M tiles
   const int64_t t0 = mt_bound * ceil_div(c.F, 128), t1 = mt_bound * ceil_div(c.H, 256);
   const int g0 = (int)std::min<int64_t>(units, t0) * CG;
   const int g1 = (int)std::min<int64_t>(units, t1) * CG;
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[2];
   fill_launch<0, CG>(cfg, attr, g0, smem, s);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, tc_grouped_gemm<0, CG>, mx, mwgu, mh, h, c.F, c.H,
-                                     2 * c.F, c.F,
-                                     offsets, counts, c.E, c.capacity, (long long)R_max, status,
-                                     (uint32_t*)nullptr, 0);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, tc_grouped_gemm<0, CG>, mx, mwgu, mh, mxs, h, c.F,
+                                     c.H, 2 * c.F, c.F, offsets, counts, c.E, c.capacity,
+                                     (long long)R_max, status, (uint32_t*)nullptr, 0, sh_rows,
+                                     sh_a_row, sh_row0);
   if (e == cudaSuccess) {
     fill_launch<1, CG>(cfg, attr, g1, smem, s);
-    e = cudaLaunchKernelEx(&cfg, tc_grouped_gemm<1, CG>, mh, mwd, my, y, c.H, c.F, c.H, 128,
-                           offsets, counts, c.E, c.capacity,
-                           (long long)R_max, status, row_ready, 0);
+    e = cudaLaunchKernelEx(&cfg, tc_grouped_gemm<1, CG>, mh, mwd, my, mh, y, c.H, c.F, c.H, 128,
+                           offsets, counts, c.E, c.capacity, (long long)R_max, status, row_ready,
+                           0, sh_rows, sh_row0, sh_row0);
   }
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -854,9 +873,9 @@ moe_status_t launch_router(const moe_config_t& c, const void* x, const void* w_g
   fill_launch<2, CG>(cfg, attr, grid, smem, s);
   // the output map argument is unused in this mode (fp32 rows are stored directly)
   const cudaError_t e = cudaLaunchKernelEx(
-      &cfg, tc_grouped_gemm<2, CG>, mx, mg, mx, (void*)logits, c.E, c.H, 0, 128,
+      &cfg, tc_grouped_gemm<2, CG>, mx, mg, mx, mx, (void*)logits, c.E, c.H, 0, 128,
       (const int32_t*)nullptr, (const int32_t*)nullptr, 1, c.T, (long long)c.T, status,
-      (uint32_t*)nullptr, c.T);
+      (uint32_t*)nullptr, c.T, 0, 0, 0);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -872,15 +891,17 @@ moe_status_t launch_router_logits_tc(const moe_config_t& c, const void* x, const
 moe_status_t launch_mlp_bf16_tc(const moe_config_t& c, const void* xp, const int32_t* offsets,
                                 const int32_t* counts, const void* w_gu, const void* w_d,
                                 void* h, void* y, int64_t R_max, uint32_t* status,
-                                cudaStream_t s, uint32_t* row_ready) {
+                                cudaStream_t s, uint32_t* row_ready, const void* x_shared) {
   if (R_max == 0) return MOE_OK;
   // Tile shape from the expected rows per expert: 256-row pair tiles halve each
   // CTA's operand traffic but waste up to 255 padded rows per expert, so small
   // experts (decode-like batches) use 128-row single-CTA tiles.
   const int64_t rows_per_expert = std::min<int64_t>((int64_t)c.T * c.K, (int64_t)c.E * c.capacity) / c.E;
   if (rows_per_expert >= 192)
-    return tc::launch_mlp<2>(c, xp, offsets, counts, w_gu, w_d, h, y, R_max, status, s, row_ready);
-  return tc::launch_mlp<1>(c, xp, offsets, counts, w_gu, w_d, h, y, R_max, status, s, row_ready);
+    return tc::launch_mlp<2>(c, xp, offsets, counts, w_gu, w_d, h, y, R_max, status, s,
+                             row_ready, x_shared);
+  return tc::launch_mlp<1>(c, xp, offsets, counts, w_gu, w_d, h, y, R_max, status, s, row_ready,
+                           x_shared);
 }
 
 }  // namespace moe

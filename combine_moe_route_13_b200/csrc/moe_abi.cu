@@ -10,10 +10,20 @@
 
 namespace moe {
 
-int64_t max_rows(const moe_config_t& c) {
+int64_t routed_rows(const moe_config_t& c) {
   return std::min<int64_t>((int64_t)c.T * c.K, (int64_t)c.E * c.capacity) +
          (int64_t)c.E * (c.row_align - 1);
 }
+
+int64_t shared_row0(const moe_config_t& c) {
+  const int64_t r = routed_rows(c);
+  return c.n_shared ? ceil_div(r, READY_ROWS) * READY_ROWS : r;
+}
+
+int64_t max_rows(const moe_config_t& c) { return shared_row0(c) + (int64_t)c.n_shared * c.T; }
+
+// First shared-expert row for the kernels, or -1 without a shared expert.
+static int64_t sh_row0_or_none(const moe_config_t& c) { return c.n_shared ? shared_row0(c) : -1; }
 
 static moe_status_t basic_checks(const moe_config_t* c) {
   if (!c) return MOE_ERR_INVALID_ARG;
@@ -21,6 +31,7 @@ static moe_status_t basic_checks(const moe_config_t* c) {
   if (c->K > c->E || c->E % c->S != 0 || c->capacity < 0 || c->row_align < 1)
     return MOE_ERR_INVALID_ARG;
   if (c->act_dtype != MOE_F32 && c->act_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (c->n_shared != 0 && c->n_shared != 1) return MOE_ERR_INVALID_ARG;
   if (c->E > MAX_E || c->K > MAX_K || c->row_align > 1024) return MOE_ERR_UNSUPPORTED;
   if ((int64_t)c->T * c->K > INT_MAX / 2) return MOE_ERR_UNSUPPORTED;
   if (max_rows(*c) > INT_MAX / 2) return MOE_ERR_UNSUPPORTED;
@@ -34,10 +45,10 @@ moe_status_t validate(const moe_config_t* c, bool need_mlp) {
   if (((int64_t)c->H * sz) % 16 != 0 || ((int64_t)c->F * sz) % 16 != 0) return MOE_ERR_UNSUPPORTED;
   if (need_mlp && c->act_dtype == MOE_BF16) {
     if (c->H % 64 != 0 || c->F % 64 != 0) return MOE_ERR_UNSUPPORTED;
-    if ((int64_t)c->E * 2 * c->F > INT_MAX / 2 || (int64_t)c->E * c->H > INT_MAX / 2)
-      return MOE_ERR_UNSUPPORTED;
+    const int64_t ew = (int64_t)c->E + c->n_shared;   // experts in the weight arrays
+    if (ew * 2 * c->F > INT_MAX / 2 || ew * c->H > INT_MAX / 2) return MOE_ERR_UNSUPPORTED;
   }
-  if (need_mlp && c->act_dtype == MOE_F32 && ceil_div(max_rows(*c), 32) + c->E > 65535)
+  if (need_mlp && c->act_dtype == MOE_F32 && ceil_div(max_rows(*c), 32) + c->E + 1 > 65535)
     return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
@@ -179,7 +190,8 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
   if (cfg->T == 0) return MOE_OK;
   if (!x || !token_slot || !xp) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(xp)) return MOE_ERR_INVALID_ARG;
-  return cuda_status(launch_dispatch(*cfg, x, token_slot, xp, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_dispatch(*cfg, x, token_slot, xp, sh_row0_or_none(*cfg),
+                                     static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_expert_mlp(const moe_config_t* cfg, const void* xp,
@@ -212,8 +224,8 @@ moe_status_t moe_combine(const moe_config_t* cfg, const void* y, const int32_t* 
   if (cfg->T == 0) return MOE_OK;
   if (!y || !token_slot || !topk_w || !out) return MOE_ERR_INVALID_ARG;
   if (!aligned16(y) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
-  return cuda_status(
-      launch_combine(*cfg, y, token_slot, topk_w, out, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_combine(*cfg, y, token_slot, topk_w, sh_row0_or_none(*cfg), out,
+                                    static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_combine_wait(const moe_config_t* cfg, const void* y, const int32_t* token_slot,
@@ -227,7 +239,8 @@ moe_status_t moe_combine_wait(const moe_config_t* cfg, const void* y, const int3
   if (!y || !token_slot || !topk_w || !row_ready || !out) return MOE_ERR_INVALID_ARG;
   if (!aligned16(y) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < 256) return MOE_ERR_WORKSPACE;
-  return cuda_status(launch_combine_wait(*cfg, y, token_slot, topk_w, row_ready, ready_target,
+  return cuda_status(launch_combine_wait(*cfg, y, token_slot, topk_w, sh_row0_or_none(*cfg),
+                                         row_ready, ready_target,
                                          (unsigned long long)timeout_us * 1000ull,
                                          static_cast<uint32_t*>(ws), out,
                                          static_cast<cudaStream_t>(stream)));
@@ -286,18 +299,26 @@ static moe_status_t layer_forward(const moe_config_t* cfg, const float* logits,
                                 sel_bias));
   if (st != MOE_OK) return st;
   if (cfg->T == 0) return MOE_OK;
-  st = moe_dispatch(cfg, x, a.token_slot, a.xp, stream);
+  if (!aligned16(x) || !aligned16(out) || !aligned16(w_gu) || !aligned16(w_d))
+    return MOE_ERR_INVALID_ARG;
+  // bf16: the shared expert's gate/up GEMM reads x itself, so the dispatch
+  // copies only the routed rows
+  const bool bf16 = cfg->act_dtype == MOE_BF16;
+  const int64_t sh = sh_row0_or_none(*cfg);
+  st = cuda_status(launch_dispatch(*cfg, x, a.token_slot, a.xp, bf16 ? -1 : sh, s));
   if (st != MOE_OK) return st;
-  if (!overlap) {
-    st = moe_expert_mlp(cfg, a.xp, a.expert_offsets, a.expert_counts, w_gu, w_d, a.h, a.y, ws,
-                        ws_bytes, stream);
-    if (st != MOE_OK) return st;
-    return moe_combine(cfg, a.y, a.token_slot, a.topk_w, out, stream);
-  }
-  st = launch_mlp_bf16_tc(*cfg, a.xp, a.expert_offsets, a.expert_counts, w_gu, w_d, a.h, a.y, R,
-                          status, s, ready);
+  if (bf16)
+    st = launch_mlp_bf16_tc(*cfg, a.xp, a.expert_offsets, a.expert_counts, w_gu, w_d, a.h, a.y,
+                            R, status, s, ready, cfg->n_shared ? x : nullptr);
+  else
+    st = cuda_status(launch_mlp_f32(*cfg, static_cast<const float*>(a.xp), a.expert_offsets,
+                                    a.expert_counts, static_cast<const float*>(w_gu),
+                                    static_cast<const float*>(w_d), static_cast<float*>(a.h),
+                                    static_cast<float*>(a.y), R, s));
   if (st != MOE_OK) return st;
-  return cuda_status(launch_combine_wait(*cfg, a.y, a.token_slot, a.topk_w, ready,
+  if (!overlap)
+    return cuda_status(launch_combine(*cfg, a.y, a.token_slot, a.topk_w, sh, out, s));
+  return cuda_status(launch_combine_wait(*cfg, a.y, a.token_slot, a.topk_w, sh, ready,
                                          ready_target(*cfg), WAIT_LIMIT_NS, status, out, s));
 }
 

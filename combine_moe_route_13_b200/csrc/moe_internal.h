@@ -69,7 +69,11 @@ __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 #endif
+// Rows of xp, h, y and row_src: the routed rows, then (n_shared = 1) the
+// shared expert's T rows from shared_row0.
 int64_t max_rows(const moe_config_t& c);
+int64_t routed_rows(const moe_config_t& c);   // min(T*K, E*C) + E*(A-1)
+int64_t shared_row0(const moe_config_t& c);   // roundup(routed_rows, 128) with a shared expert
 moe_status_t validate(const moe_config_t* c, bool need_mlp);
 
 // ---- launchers (return cudaGetLastError() of their launches) ----
@@ -81,32 +85,39 @@ cudaError_t launch_route(const moe_config_t& c, const float* logits, int32_t* to
                          int32_t* blk_cnt, int64_t R_max, cudaStream_t s,
                          uint32_t* row_ready = nullptr, const float* sel_bias = nullptr);
 
+// sh_row0 >= 0: also copy x[t] to xp[sh_row0 + t] (the shared expert's rows).
 cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t* slot, void* xp,
-                            cudaStream_t s);
+                            int64_t sh_row0, cudaStream_t s);
 
+// sh_row0 >= 0: add y[sh_row0 + t] with weight 1 after the routed terms.
 cudaError_t launch_combine(const moe_config_t& c, const void* y, const int32_t* slot,
-                           const float* w, void* out, cudaStream_t s);
+                           const float* w, int64_t sh_row0, void* out, cudaStream_t s);
 
 // Combine that waits, token by token, for the ready counters of its rows to
 // reach `target` instead of for the previous kernel to finish.
 cudaError_t launch_combine_wait(const moe_config_t& c, const void* y, const int32_t* slot,
-                                const float* w, const uint32_t* row_ready, uint32_t target,
-                                unsigned long long timeout_ns, uint32_t* status, void* out,
-                                cudaStream_t s);
+                                const float* w, int64_t sh_row0, const uint32_t* row_ready,
+                                uint32_t target, unsigned long long timeout_ns, uint32_t* status,
+                                void* out, cudaStream_t s);
 
-// fp32 CUDA-core grouped SwiGLU (gate/up then down).
+// fp32 CUDA-core grouped SwiGLU (gate/up then down); with a shared expert
+// its rows [shared_row0, +T) of xp are included.
 cudaError_t launch_mlp_f32(const moe_config_t& c, const float* xp, const int32_t* offsets,
                            const int32_t* counts, const float* w_gu, const float* w_d, float* h,
                            float* y, int64_t R_max, cudaStream_t s);
 
 // bf16 tcgen05 grouped SwiGLU (gate/up then down). Returns a moe status.
+// With a shared expert, its T rows are one more group of the same GEMMs; its
+// gate/up input rows come from x_shared ([T,H], e.g. the layer input) when
+// given, else from xp's rows [shared_row0, +T).
 // row_ready (optional): the down GEMM adds 1 to the counter of a 128-row
 // block each time it has stored one of the block's N tiles (release), so
 // a block is final when its counter reaches ceil(H / 256).
 moe_status_t launch_mlp_bf16_tc(const moe_config_t& c, const void* xp, const int32_t* offsets,
                                 const int32_t* counts, const void* w_gu, const void* w_d,
                                 void* h, void* y, int64_t R_max, uint32_t* status,
-                                cudaStream_t s, uint32_t* row_ready = nullptr);
+                                cudaStream_t s, uint32_t* row_ready = nullptr,
+                                const void* x_shared = nullptr);
 
 // Router projection logits[T,E] = x[T,H] w_g[E,H]^T (fp32 out): tcgen05 for
 // bf16, FFMA for fp32.

@@ -26,7 +26,8 @@
 //                      the experts (block 0 stores the offsets, segment
 //                      offsets and totals); then every assignment gets
 //                      slot = off[e] + rank if rank < C, else -1, the row_src
-//                      back-map, and row_src padding rows get -1.
+//                      back-map; row_src padding rows get -1 and the shared
+//                      expert's rows (if any) T*K + t.
 #include <algorithm>
 #include <cfloat>
 #include <climits>
@@ -259,7 +260,7 @@ __device__ __forceinline__ void expert_offsets_smem(int E, int C, int A,
 }
 
 __global__ void __launch_bounds__(256)
-route_slot_kernel(int T, int K, int E, int S, int C, int A, int nblk, int64_t R_max,
+route_slot_kernel(int T, int K, int E, int S, int C, int A, int nblk, int64_t R_max, int64_t R_sh,
                   const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ blk_base,
                   const int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                   int32_t* __restrict__ segoff, int32_t* __restrict__ totals,
@@ -298,9 +299,14 @@ route_slot_kernel(int T, int K, int E, int S, int C, int A, int nblk, int64_t R_
     }
     slot[i] = s;
   }
-  // rows no assignment fills: each expert's alignment padding and the tail
+  // rows no assignment fills: each expert's alignment padding and the tail;
+  // from R_sh on, the shared expert's rows (one per token, id T*K + t)
   const int R = off_s[E];
   for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < R_max; r += stride) {
+    if (r >= R_sh) {
+      row_src[r] = (int32_t)(TK + (r - R_sh));
+      continue;
+    }
     bool pad = true;
     if (r < R) {
       int lo = 0, hi = E;   // largest e with off_s[e] <= r
@@ -355,7 +361,7 @@ cudaError_t launch_route(const moe_config_t& c, const float* logits, int32_t* to
   const int64_t work = std::max<int64_t>((int64_t)c.T * c.K, R_max);
   int grid = (int)std::min<int64_t>(std::max<int64_t>(ceil_div(work, 256), 1), 148 * 8);
   return launch_pdl(route_slot_kernel, dim3(grid), dim3(256), 0, s, c.T, c.K, c.E, c.S, c.capacity,
-                    c.row_align, nblk, R_max, (const int32_t*)topk_idx, (const int32_t*)blk_cnt,
+                    c.row_align, nblk, R_max, shared_row0(c), (const int32_t*)topk_idx, (const int32_t*)blk_cnt,
                     (const int32_t*)counts, offsets, segoff, totals, slot, row_src, row_ready,
                     n_ready);
 }

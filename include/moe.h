@@ -37,6 +37,15 @@
  * Symbols: T tokens, H hidden size, E experts, K experts per token, F SwiGLU
  * width, S owner segments, C capacity per expert, A row alignment, R_max rows
  * of the dispatch buffer (moe_max_rows).
+ *
+ * Shared expert (n_shared = 1): an expert that every token uses with weight 1
+ * next to its K routed experts (the shared experts whose multiplication the EFA
+ * page runs while the dispatch transfers are in flight, "Диспетчеризация и
+ * комбинирование"; the sum of routed and shared output is this library's
+ * reading). It is stored as expert E of the weight arrays (w_gu and w_d hold
+ * E + 1 experts, the shared one last, same F) and owns the T rows
+ * [R_sh, R_sh + T) of xp, h and y, one per token in token order, where
+ * R_sh = roundup(min(T*K, E*C) + E*(A-1), 128). Routing never selects it.
  */
 #ifndef MOE_H
 #define MOE_H
@@ -61,6 +70,7 @@ typedef enum {
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
 
 /* Layer configuration. Limits: T >= 0; H >= 1; 1 <= E <= 1024; 1 <= K <= min(E, 32);
+ * n_shared is 0 or 1 (a shared expert, see above);
  * F >= 1; S >= 1 and E % S == 0 (owner segment s holds experts [s*E/S, (s+1)*E/S));
  * capacity >= 0 (the per-expert limit C, see moe_capacity); 1 <= row_align <= 1024
  * (every expert's rows start at a multiple of A inside the dispatch buffer);
@@ -72,6 +82,7 @@ typedef struct {
   int32_t capacity;
   int32_t row_align;
   int32_t act_dtype;
+  int32_t n_shared;
 } moe_config_t;
 
 /* Pointers into the workspace where moe_layer_forward keeps the intermediates.
@@ -100,7 +111,8 @@ int32_t moe_capacity(int32_t T, int32_t K, int32_t E, double cf);
 /* R_max = min(T*K, E*C) + E*(A-1): rows of the dispatch buffer xp (and of h, y
  * and row_src). Every kept assignment gets one row and each expert adds at most
  * A-1 rows of alignment padding (a fixed worst-case bound, as the pplx-kernels
- * page sizes its receive buffers, "Draagbare kernels"). Returns -1 for an
+ * page sizes its receive buffers, "Draagbare kernels"). With n_shared = 1,
+ * R_max = R_sh + T (the shared expert's rows follow). Returns -1 for an
  * invalid config. */
 int64_t moe_max_rows(const moe_config_t* cfg);
 
@@ -131,7 +143,8 @@ moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
  *   segment_offsets [S+1] int32 out: off[s*E/S].
  *   token_slot      [T,K] int32 out: row of (t,k) in xp, or -1 if it overflowed.
  *                   The first C assignments of each expert in token order are kept.
- *   row_src         [R_max] int32 out: t*K+k for each kept row, -1 on padding rows.
+ *   row_src         [R_max] int32 out: t*K+k for each kept row, -1 on padding rows,
+ *                   T*K+t on the shared expert's row of token t (n_shared = 1).
  *   totals          [4]   int32 out: {T*K, effective N, total overflow, R = off[E]}.
  *   ws, ws_bytes    workspace of at least moe_route_workspace_bytes(cfg) bytes,
  *                   256-byte aligned; contents need not be initialised except the
@@ -198,7 +211,8 @@ moe_status_t moe_route_topk_noalloc(const moe_config_t* cfg, const float* logits
                                     int32_t* row_src, int32_t* totals, void* stream);
 
 /* Dispatch ("Dispatch" of the pplx-kernels page): xp[token_slot[t,k]] = x[t],
- * a bit copy, for every (t,k) with token_slot >= 0.
+ * a bit copy, for every (t,k) with token_slot >= 0, and xp[R_sh + t] = x[t]
+ * when n_shared = 1.
  *   x          [T,H] act, device, read only.
  *   token_slot [T,K] int32 from moe_route_topk.
  *   xp         [R_max,H] act out; rows no slot points at are not written. */
@@ -212,8 +226,9 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
  *   xp             [R_max,H] act.
  *   expert_offsets [E+1] int32, expert_counts [E] int32 (raw counts; the kept
  *                  count min(count, C) is derived on the device).
- *   w_gu           [E,2F,H] act: rows 0..F-1 are Wg_e, rows F..2F-1 are Wu_e.
- *   w_d            [E,H,F] act.
+ *   w_gu           [E+n_shared,2F,H] act: rows 0..F-1 are Wg_e, rows F..2F-1 are Wu_e.
+ *   w_d            [E+n_shared,H,F] act.
+ *   With n_shared = 1 the shared expert E also maps rows [R_sh, R_sh + T).
  *   h              [R_max,F] act out (scratch for the second GEMM), y [R_max,H] act out.
  *   Rows outside every expert's kept range hold unspecified values afterwards
  *   (an expert's alignment padding rows may be written; no reader uses them).
@@ -226,9 +241,10 @@ moe_status_t moe_expert_mlp(const moe_config_t* cfg, const void* xp,
                             void* ws, size_t ws_bytes, void* stream);
 
 /* Combine ("Combine" of the pplx-kernels page): out[t] = sum over k in order of
- * topk_w[t,k] * y[token_slot[t,k]] for slots >= 0, fp32 accumulation, rounded
- * once to act. Dropped assignments contribute zero (no renormalisation); a token
- * with every assignment dropped gets zeros.
+ * topk_w[t,k] * y[token_slot[t,k]] for slots >= 0, plus y[R_sh + t] when
+ * n_shared = 1, fp32 accumulation, rounded once to act. Dropped assignments
+ * contribute zero (no renormalisation); a token with every assignment dropped
+ * gets zeros (or its shared expert's output alone).
  *   y [R_max,H] act, token_slot [T,K] int32, topk_w [T,K] fp32, out [T,H] act. */
 moe_status_t moe_combine(const moe_config_t* cfg, const void* y, const int32_t* token_slot,
                          const float* topk_w, void* out, void* stream);
@@ -237,8 +253,8 @@ moe_status_t moe_combine(const moe_config_t* cfg, const void* y, const int32_t* 
  * acceleration through overlap": the GEMM publishes tile-ready flags in its
  * epilogue and a separate kernel starts on each tile as soon as its flag is set).
  * Same result as moe_combine. Before reading the rows of token t, the kernel
- * waits until row_ready[slot / 128] >= ready_target for every kept slot of t
- * (acquire loads). moe_expert_mlp's down GEMM, run by moe_layer_forward with
+ * waits until row_ready[slot / 128] >= ready_target for every kept slot of t,
+ * and for its shared row R_sh + t when n_shared = 1 (acquire loads). moe_expert_mlp's down GEMM, run by moe_layer_forward with
  * MOE_FLAG_OVERLAP, adds 1 to a block's counter per stored 256-column tile
  * (release), so the target there is ceil(H / 256). The kernel does not wait for
  * the previous kernel in the stream, so token_slot and topk_w must already be
@@ -257,7 +273,9 @@ moe_status_t moe_combine_wait(const moe_config_t* cfg, const void* y, const int3
 /* The whole layer on `stream`: route -> dispatch -> expert MLP -> combine, with
  * every intermediate in the workspace (moe_workspace_bytes). `aux` may be NULL;
  * otherwise it receives the workspace pointers of the intermediates. No host
- * synchronisation: the per-expert counts stay on the device. flags: MOE_FLAG_NONE,
+ * synchronisation: the per-expert counts stay on the device. With n_shared = 1 and
+ * bf16, the shared expert's GEMM reads its rows straight from x, so the shared
+ * rows of xp are not written. flags: MOE_FLAG_NONE,
  * or MOE_FLAG_OVERLAP (the combine overlaps the down GEMM; bf16 with
  * row_align % 128 == 0, else MOE_ERR_UNSUPPORTED; identical results). */
 moe_status_t moe_layer_forward(const moe_config_t* cfg, const float* logits, const void* x,

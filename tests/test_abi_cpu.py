@@ -68,6 +68,39 @@ def test_sizes_match_oracle(name):
     assert 256 < M.moe_route_workspace_bytes(cfg) < M.moe_workspace_bytes(cfg)
 
 
+@pytest.mark.parametrize("name", ["tiny", "mixtral", "dsv3", "kimi"])
+def test_sizes_with_a_shared_expert(name):
+    # moe.h: the shared expert's T rows start at the routed bound rounded up to
+    # 128 and R_max grows by them; routed sizes are unchanged.
+    w = W.WORKLOADS[name]
+    base = cfg_of(w)
+    cfg = cfg_of(w, n_shared=1)
+    R_r = O.max_rows(w.T, w.K, w.E, base.capacity, w.row_align)
+    R_sh = -(-R_r // 128) * 128
+    assert M.moe_max_rows(base) == R_r
+    assert M.moe_max_rows(cfg) == R_sh + w.T
+    assert M.shared_row0(cfg) == R_sh and M.shared_row0(base) == R_r
+    assert M.moe_check_config(cfg) == M.MOE_OK
+    assert M.moe_workspace_bytes(cfg) >= M.moe_workspace_bytes(base) + w.T * (2 * w.H + w.F) * (
+        4 if w.act == "f32" else 2)
+
+
+def test_n_shared_other_than_0_or_1_is_invalid():
+    cfg = cfg_of(W.WORKLOADS["tiny"], n_shared=2)
+    assert M.moe_check_config(cfg) == M.MOE_ERR_INVALID_ARG
+    cfg.n_shared = -1
+    assert M.moe_max_rows(cfg) == -1
+
+
+def test_config_struct_matches_header():
+    # the ctypes mirror of moe_config_t has the header's fields in order
+    src = open(HEADER).read()
+    body = re.search(r"typedef struct \{(.*?)\} moe_config_t;", src, re.S).group(1)
+    names = re.findall(r"\b([A-Za-z_]+)\s*[,;]", body)
+    assert [n for n, _ in M.MoeConfig._fields_] == names
+    assert ctypes.sizeof(M.MoeConfig) == 4 * len(names)
+
+
 @pytest.mark.parametrize("field,value,code", [
     ("K", 0, M.MOE_ERR_INVALID_ARG), ("K", 9, M.MOE_ERR_INVALID_ARG),      # K > E
     ("S", 3, M.MOE_ERR_INVALID_ARG),                                       # E % S != 0

@@ -8,6 +8,10 @@ launch configuration bench.py times).
   non-empty one and random ones; first, last and random rows of each) against
   the oracle's SwiGLU on the same xp rows;
 * combine: sampled tokens against the oracle's weighted sum of the GPU's y rows.
+
+DeepSeek-V3 and Kimi-K2 also run with their shared expert (n_shared = 1): its
+rows of h and y are sampled like an expert's, from x, and the combine adds
+them.
 """
 import numpy as np
 import pytest
@@ -23,12 +27,14 @@ ROUTE_KEYS = ("topk_idx", "topk_w", "expert_counts", "overflow", "expert_offsets
               "segment_offsets", "token_slot", "row_src", "totals")
 
 
-@pytest.mark.parametrize("name", ["mixtral", "dsv3", "skewed", "kimi"])
-def test_workload_full_size(cuda_ok, name):
-    wl = W.WORKLOADS[name]
+@pytest.mark.parametrize("name,n_shared", [("mixtral", 0), ("dsv3", 0), ("skewed", 0),
+                                           ("kimi", 0), ("dsv3", 1), ("kimi", 1)])
+def test_workload_full_size(cuda_ok, name, n_shared):
+    wl = W.WORKLOADS[name].with_(n_shared=n_shared)
     dev = torch.device("cuda")
     C = M.moe_capacity(wl.T, wl.K, wl.E, wl.cf)
-    cfg = M.make_config(wl.T, wl.H, wl.E, wl.K, wl.F, wl.S, C, wl.row_align, wl.act)
+    cfg = M.make_config(wl.T, wl.H, wl.E, wl.K, wl.F, wl.S, C, wl.row_align, wl.act,
+                        n_shared=n_shared)
     inp = W.make_inputs(wl, seed=0, device=dev)
     ws = M.alloc_workspace(M.moe_workspace_bytes(cfg), dev)
     out = torch.empty(wl.T, wl.H, dtype=wl.torch_act, device=dev)
@@ -41,8 +47,14 @@ def test_workload_full_size(cuda_ok, name):
     R_max = ref["R_max"]
     assert_route_equal(host({k: v[k] for k in ROUTE_KEYS}), ref, R_max)
 
+    R_sh = M.shared_row0(cfg)
+    if n_shared:   # the shared rows' ids, in full
+        assert torch.all(v["row_src"][R_max:R_sh] == -1)
+        assert torch.equal(v["row_src"][R_sh:].cpu(),
+                           torch.arange(wl.T, dtype=torch.int32) + wl.T * wl.K)
+
     # dispatch, in full on the device: xp[row] == x[row_src[row] // K]
-    rs = v["row_src"]
+    rs = v["row_src"][:R_max]
     rows = torch.nonzero(rs >= 0).squeeze(1)
     assert rows.numel() == int(ref["totals"][1])
     src_tok = (rs[rows] // wl.K).long()
@@ -65,6 +77,13 @@ def test_workload_full_size(cuda_ok, name):
         idx = torch.from_numpy(rws).to(dev)
         assert_close_act(act_np(v["h"][idx]), he, wl.act, f"h[e={e}]")
         assert_close_act(act_np(v["y"][idx]), ye, wl.act, f"y[e={e}]")
+    if n_shared:   # the shared expert's rows: first, last and random tokens, from x
+        tk = np.unique(np.concatenate([[0, 1, wl.T - 1], rng.integers(0, wl.T, 13)]))
+        he, ye = O.expert_mlp_rows(act_np(inp["x"][torch.from_numpy(tk).to(dev)]),
+                                   act_np(inp["w_gu"][wl.E]), act_np(inp["w_d"][wl.E]), wl.act)
+        idx = torch.from_numpy(R_sh + tk).to(dev)
+        assert_close_act(act_np(v["h"][idx]), he, wl.act, "h[shared]")
+        assert_close_act(act_np(v["y"][idx]), ye, wl.act, "y[shared]")
 
     # combine on sampled tokens, from the GPU's y
     toks = np.unique(np.concatenate([[0, wl.T - 1], rng.integers(0, wl.T, 254)]))
@@ -75,7 +94,8 @@ def test_workload_full_size(cuda_ok, name):
     slot_sub = np.where(slot >= 0, remap[np.maximum(slot, 0)], -1).astype(np.int32)
     y_sub = act_np(v["y"][torch.from_numpy(need).to(dev)]) if len(need) else \
         np.zeros((1, wl.H), np.uint16)
-    ref_out = O.combine(y_sub, slot_sub, ref["topk_w"][toks], wl.act)
+    y_sh = act_np(v["y"][torch.from_numpy(R_sh + toks).to(dev)]) if n_shared else None
+    ref_out = O.combine(y_sub, slot_sub, ref["topk_w"][toks], wl.act, y_shared=y_sh)
     got = act_np(out[torch.from_numpy(toks).to(dev)])
     assert_close_act(got, ref_out, wl.act, "out")
     del inp, ws, out

@@ -20,9 +20,14 @@ Value recipe (all from one ``torch.Generator`` seeded with ``seed``, drawn in
 this order): router logits N(0,1) [T,E] fp32; per-expert logit bias (dsv3:
 N(0, 0.1) with 0.1 the standard deviation; skewed: 2*ln(rank^-1.2) with rank
 e+1; others none) added to every token's logits; activations x N(0,1) [T,H];
-gate/up weights N(0, 0.02^2) [E,2F,H] (rows 0..F-1 gate, F..2F-1 up); down
-weights N(0, 0.02^2) [E,H,F].  Activations and weights are produced in the
+gate/up weights N(0, 0.02^2) [E',2F,H] (rows 0..F-1 gate, F..2F-1 up); down
+weights N(0, 0.02^2) [E',H,F], with E' = E + n_shared (a shared expert, when
+present, is the last one).  Activations and weights are produced in the
 workload's activation dtype.
+
+``with_(n_shared=1)`` adds one shared expert of the routed experts' width, as
+in DeepSeek-V3 and Kimi-K2 (one shared expert of width 2048 next to the routed
+ones).
 """
 from __future__ import annotations
 
@@ -44,6 +49,7 @@ class Workload:
     act: str              # "f32" or "bf16"
     bias: str = "none"    # "none" | "normal0.1" | "zipf1.2"
     row_align: int = 128  # A: expert start alignment inside the dispatch buffer
+    n_shared: int = 0     # 1: one shared expert every token uses with weight 1
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -109,17 +115,20 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu", weights: bool = True,
     x = _normal((w.T, w.H), 1.0, w.torch_act, gen, device)
     out = {"logits": logits, "x": x}
     if weights:
-        out["w_gu"] = _normal((w.E, 2 * w.F, w.H), 0.02, w.torch_act, gen, device)
-        out["w_d"] = _normal((w.E, w.H, w.F), 0.02, w.torch_act, gen, device)
+        ew = w.E + w.n_shared
+        out["w_gu"] = _normal((ew, 2 * w.F, w.H), 0.02, w.torch_act, gen, device)
+        out["w_d"] = _normal((ew, w.H, w.F), 0.02, w.torch_act, gen, device)
     if router:
         out["w_g"] = _normal((w.E, w.H), w.H ** -0.5, w.torch_act, gen, device)
         out["sel_bias"] = torch.randn(w.E, generator=gen, device=device, dtype=torch.float32) * 0.1
     return out
 
 
-def small_case(T, H, E, K, F, S, cf, act="bf16", row_align=128, bias="none") -> Workload:
+def small_case(T, H, E, K, F, S, cf, act="bf16", row_align=128, bias="none",
+               n_shared=0) -> Workload:
     """An ad-hoc workload for parity sweeps (ragged sizes, edge cases)."""
-    return Workload(f"case_T{T}_H{H}_E{E}_K{K}_F{F}", T, H, E, K, F, S, cf, act, bias, row_align)
+    name = f"case_T{T}_H{H}_E{E}_K{K}_F{F}" + ("_shared" if n_shared else "")
+    return Workload(name, T, H, E, K, F, S, cf, act, bias, row_align, n_shared)
 
 
 def tied_logits(T: int, E: int, levels: int, gen: torch.Generator, device="cpu") -> torch.Tensor:
@@ -132,7 +141,7 @@ def tied_logits(T: int, E: int, levels: int, gen: torch.Generator, device="cpu")
 def expected_bytes_gb(w: Workload) -> float:
     """Device memory held by the inputs, in GB (for sizing decisions)."""
     s = 4 if w.act == "f32" else 2
-    return (w.T * w.E * 4 + w.T * w.H * s + 3 * w.E * w.F * w.H * s) / 1e9
+    return (w.T * w.E * 4 + w.T * w.H * s + 3 * (w.E + w.n_shared) * w.F * w.H * s) / 1e9
 
 
 __all__ = ["Workload", "WORKLOADS", "make_inputs", "make_router_logits", "small_case",
