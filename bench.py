@@ -56,18 +56,26 @@ def load_peaks():
     return p
 
 
+def kernel_sources_sha(paths) -> str:
+    """sha256 of the concatenated sources (repo-relative paths), in order."""
+    import hashlib
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def measured_traffic(workload: str):
     """DRAM bytes per moe_expert_mlp call from the committed ncu capture of this
-    workload, or None when there is none or the GEMM source changed since."""
-    import hashlib
+    workload, or None when there is none or the GEMM sources changed since."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f).get(workload)
         if not rec:
             return None
-        with open(os.path.join(ROOT, rec["kernel_source"]), "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()
+        sha = kernel_sources_sha(rec["kernel_sources"])
         return rec["traffic_bytes"] if sha.startswith(rec["sha256_prefix"]) else None
     except (OSError, ValueError, KeyError):
         return None
