@@ -33,7 +33,9 @@ EXPORTS = ("moe_capacity", "moe_max_rows", "moe_check_config", "moe_route_worksp
            "moe_workspace_bytes", "moe_workspace_init", "moe_route_topk", "moe_dispatch",
            "moe_expert_mlp", "moe_combine", "moe_layer_forward", "moe_get_device_status",
            "moe_status_string", "moe_version", "moe_route_topk_noalloc", "moe_combine_wait",
-           "moe_route_topk_biased", "moe_router_logits", "moe_layer_forward_x")
+           "moe_route_topk_biased", "moe_router_logits", "moe_layer_forward_x",
+           "moe_fp8_scale_bytes", "moe_quantize_fp8", "moe_dispatch_fp8", "moe_expert_mlp_fp8",
+           "moe_layer_forward_fp8")
 
 
 class MoeError(RuntimeError):
@@ -55,7 +57,8 @@ class MoeConfig(ctypes.Structure):
 class MoeLayerAux(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "topk_idx", "expert_counts", "overflow", "expert_offsets", "segment_offsets",
-        "token_slot", "row_src", "totals", "topk_w", "xp", "h", "y", "logits")]
+        "token_slot", "row_src", "totals", "topk_w", "xp", "h", "y", "logits",
+        "xq", "xs", "hq", "hs")]
 
 
 _P = ctypes.c_void_p
@@ -91,6 +94,13 @@ def _load():
         "moe_layer_forward_x": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, ctypes.c_uint32,
                                                _P, ctypes.c_size_t, ctypes.POINTER(MoeLayerAux),
                                                _P]),
+        "moe_fp8_scale_bytes": (ctypes.c_int64, [ctypes.c_int64, ctypes.c_int64]),
+        "moe_quantize_fp8": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int64, _P, _P, _P]),
+        "moe_dispatch_fp8": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P]),
+        "moe_expert_mlp_fp8": (ctypes.c_int, [_CFG] + [_P] * 11 + [_P, ctypes.c_size_t, _P]),
+        "moe_layer_forward_fp8": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P,
+                                                 ctypes.c_uint32, _P, ctypes.c_size_t,
+                                                 ctypes.POINTER(MoeLayerAux), _P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -299,6 +309,77 @@ def moe_version() -> int:
     return int(LIB.moe_version())
 
 
+# ---------------------------------------------------------------- fp8 block-scaled path
+
+U8 = torch.uint8
+
+
+def moe_fp8_scale_bytes(rows: int, cols: int) -> int:
+    return int(LIB.moe_fp8_scale_bytes(int(rows), int(cols)))
+
+
+def moe_quantize_fp8(src, codes, scales, stream=None):
+    """Block-quantise a [rows, cols] bf16 tensor into codes (uint8, same shape) and scales."""
+    rows, cols = src.shape
+    _check(LIB.moe_quantize_fp8(_ptr(src, torch.bfloat16, "src"), rows, cols,
+                                _ptr(codes, U8, "codes"), _ptr(scales, U8, "scales"),
+                                _stream(stream)), "moe_quantize_fp8")
+
+
+def quantize_fp8(src: torch.Tensor, stream=None):
+    """Allocate and fill (codes, scales) for a bf16 tensor viewed as [-1, last dim]."""
+    m = src.reshape(-1, src.shape[-1])
+    codes = torch.empty(m.shape, dtype=U8, device=src.device)
+    scales = torch.empty(max(moe_fp8_scale_bytes(*m.shape), 16), dtype=U8, device=src.device)
+    moe_quantize_fp8(m, codes, scales, stream)
+    return codes.view(src.shape), scales
+
+
+def moe_dispatch_fp8(cfg, x, token_slot, xq, xs, stream=None):
+    _check(LIB.moe_dispatch_fp8(ctypes.byref(cfg), _ptr(x, torch.bfloat16, "x"),
+                                _ptr(token_slot, torch.int32, "token_slot"), _ptr(xq, U8, "xq"),
+                                _ptr(xs, U8, "xs"), _stream(stream)), "moe_dispatch_fp8")
+
+
+def moe_expert_mlp_fp8(cfg, xq, xs, expert_offsets, expert_counts, wq_gu, ws_gu, wq_d, ws_d,
+                       hq, hs, y, ws, stream=None):
+    i32 = torch.int32
+    _check(LIB.moe_expert_mlp_fp8(
+        ctypes.byref(cfg), _ptr(xq, U8, "xq"), _ptr(xs, U8, "xs"),
+        _ptr(expert_offsets, i32, "expert_offsets"), _ptr(expert_counts, i32, "expert_counts"),
+        _ptr(wq_gu, U8, "wq_gu"), _ptr(ws_gu, U8, "ws_gu"), _ptr(wq_d, U8, "wq_d"),
+        _ptr(ws_d, U8, "ws_d"), _ptr(hq, U8, "hq"), _ptr(hs, U8, "hs"),
+        _ptr(y, torch.bfloat16, "y"), _ptr(ws, name="ws"), ws.numel() * ws.element_size(),
+        _stream(stream)), "moe_expert_mlp_fp8")
+
+
+def moe_layer_forward_fp8(cfg, logits, x, wq_gu, ws_gu, wq_d, ws_d, out, ws,
+                          flags=MOE_FLAG_NONE, stream=None):
+    aux = MoeLayerAux()
+    _check(LIB.moe_layer_forward_fp8(
+        ctypes.byref(cfg), _ptr(logits, torch.float32, "logits"), _ptr(x, torch.bfloat16, "x"),
+        _ptr(wq_gu, U8, "wq_gu"), _ptr(ws_gu, U8, "ws_gu"), _ptr(wq_d, U8, "wq_d"),
+        _ptr(ws_d, U8, "ws_d"), _ptr(out, torch.bfloat16, "out"), flags, _ptr(ws, name="ws"),
+        ws.numel() * ws.element_size(), ctypes.byref(aux), _stream(stream)),
+        "moe_layer_forward_fp8")
+    return aux
+
+
+def fp8_views(cfg: MoeConfig, ws: torch.Tensor, aux: MoeLayerAux) -> dict:
+    """torch views of the fp8 intermediates moe_layer_forward_fp8 left in ws."""
+    base = ws.data_ptr()
+    R = moe_max_rows(cfg)
+
+    def view(ptr, nbytes, shape):
+        off = ptr - base
+        return ws[off:off + nbytes].view(shape)
+
+    return {"xq": view(aux.xq, R * cfg.H, (R, cfg.H)),
+            "xs": view(aux.xs, moe_fp8_scale_bytes(R, cfg.H), (-1,)),
+            "hq": view(aux.hq, R * cfg.F, (R, cfg.F)),
+            "hs": view(aux.hs, moe_fp8_scale_bytes(R, cfg.F), (-1,))}
+
+
 # ---------------------------------------------------------------- conveniences
 
 def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
@@ -330,6 +411,8 @@ def layer_views(cfg: MoeConfig, ws: torch.Tensor, aux: MoeLayerAux) -> dict:
     es = 4 if dt == torch.float32 else 2
 
     def view(ptr, nbytes, dtype, shape):
+        if ptr is None:   # not produced by this entry point (xp / h of the fp8 layer)
+            return None
         off = ptr - base
         return ws[off:off + nbytes].view(dtype).view(shape)
 

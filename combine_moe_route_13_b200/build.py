@@ -21,8 +21,9 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmoe.so")
 SOURCES = ["moe_abi.cu", "route.cu", "dispatch_combine.cu", "gemm_simt.cu", "gemm_tc.cu",
-           "route_noalloc.cu"]
-HEADERS = [os.path.join(CSRC, "moe_internal.h"), os.path.join(ROOT, "include", "moe.h")]
+           "route_noalloc.cu", "quant_fp8.cu", "gemm_fp8.cu"]
+HEADERS = [os.path.join(CSRC, h) for h in ("moe_internal.h", "tc_ptx.cuh", "fp8_util.cuh")] + \
+    [os.path.join(ROOT, "include", "moe.h")]
 GENCODE = "arch=compute_100a,code=sm_100a"
 
 

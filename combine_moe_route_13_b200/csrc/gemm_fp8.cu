@@ -1,0 +1,519 @@
+// fp8 block-scaled grouped SwiGLU expert MLP on the sm_100a tensor cores
+// (tcgen05.mma kind::mxf8f6f4 with UE8M0 block scales, TMEM, TMA).
+//
+// The grouped GEMM between dispatch and combine ("Enabling trillion-parameter
+// models on AWS EFA", "MoE all-to-all через EFA") fed by the fp8 block-scaled
+// dispatch payload of the same page's evaluation ("Оценка"). Both operands are
+// e4m3 with one power-of-two scale per 128 k values of a row (see
+// fp8_util.cuh); the tensor cores apply the scales themselves, one per 32 k
+// values, so the fp32 accumulator holds the exact sum of scaled products.
+//
+// Two launches, each a persistent grid of one CTA per SM walking the tiles of
+// every expert (same tile order as the bf16 kernel: expert, N tile, M tile):
+//   MODE 0: [g | u] = xq W_gu[e]^T (M = 128, N = 128 gate + 128 up columns),
+//           epilogue h = silu(g) * u, quantised to e4m3 with one scale per
+//           128 columns of a row (the tile's columns are exactly one scale
+//           block), codes by TMA store, scales to their chunk.
+//   MODE 1: y = hq W_d[e]^T (N = 256 columns), epilogue rounds to bf16.
+//
+// Per stage (128 k values = one 128-byte swizzle row of e4m3): TMA boxes of A
+// (128 rows) and B (2 x 128 rows), and three 512-byte scale chunks (A, B rows
+// 0-127, B rows 128-255) by bulk copy. The MMA thread moves the chunks into
+// TMEM with tcgen05.cp (32 rows x 16 bytes, replicated to the four lane
+// quarters) and issues four K = 32 MMAs, the j-th reading scale byte j.
+//
+// TMEM: the 256-column fp32 accumulator at column 0 (single buffer) and 12
+// scale columns per stage from column 256. To overlap one tile's epilogue with
+// the next tile's MMAs despite the single accumulator, the epilogue first
+// loads its whole row into registers and releases TMEM, then quantises /
+// rounds and stores.
+//
+// Every mbarrier wait is bounded as in the bf16 kernel.
+#include <algorithm>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include "fp8_util.cuh"
+#include "moe_internal.h"
+#include "tc_ptx.cuh"
+
+namespace moe {
+namespace tc {
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn();
+bool make_map(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows);
+}  // namespace tc
+
+namespace f8 {
+using namespace tc;
+
+constexpr int BM = 128;                         // rows per tile = TMEM lanes
+constexpr int BK = 128;                         // k per stage (bytes of a swizzle row)
+constexpr int UMMA_N = 256;
+constexpr int A_BYTES = BM * BK;                // 16 KB
+constexpr int B_HALF = 128 * BK;                // 16 KB
+constexpr int OPER_BYTES = A_BYTES + 2 * B_HALF;
+constexpr int SF_STAGE = 3 * SF_CHUNK;          // A, B rows 0-127, B rows 128-255
+constexpr int STAGES = 4;
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t SF_COL0 = 256;
+constexpr uint32_t SF_COLS = 12;                // per stage: 4 (A) + 8 (B)
+constexpr int STAGING_BYTES = 128 * 128;        // one 128-row x 128-byte output box
+constexpr unsigned long long WAIT_NS = 2000000000ull;
+constexpr unsigned long long DRAIN_NS = 200000000ull;
+
+struct Ctl {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull, tempty, drain;
+  uint32_t tmem_base;
+  int abort;
+  int wsum[8];
+};
+
+size_t smem_bytes(int E) {
+  return 1024 + (size_t)STAGES * (OPER_BYTES + SF_STAGE) + STAGING_BYTES + sizeof(Ctl) +
+         (size_t)(3 * E + 2) * 4;
+}
+
+// Instruction descriptor of tcgen05.mma.kind::mxf8f6f4.block_scale: B scale
+// byte j (bits 4-5), A and B e4m3 (format 0 at bits 7-9, 10-12), both
+// K-major, N >> 3 at bits 17-22, UE8M0 scales (bit 23), M >> 4 at bits 24-28,
+// A scale byte j (bits 29-30), dense K = 32 (bit 31 = 0).
+__host__ __device__ constexpr uint32_t idesc_fp8(uint32_t j) {
+  return (j << 4) | ((uint32_t)(UMMA_N >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24) |
+         (j << 29);
+}
+
+// Global -> shared bulk copy (no tensor map), completion counted on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// Shared-memory descriptor of a 32-row x 16-byte scale chunk: no swizzle,
+// 8-row core matrices of 128 bytes stacked 128 bytes apart (stride byte
+// offset); one core matrix wide, so the leading byte offset is not used.
+__device__ __forceinline__ uint64_t sf_desc(uint32_t a) {
+  uint64_t d = (uint64_t)((a >> 4) & 0x3FFFu);
+  d |= (uint64_t)(128u >> 4) << 16;
+  d |= (uint64_t)(128u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  return d;
+}
+
+// 32 rows x 128 bits of shared memory into 4 TMEM columns, the same rows in
+// each of the four 32-lane quarters.
+__device__ __forceinline__ void sf_copy(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
+__device__ __forceinline__ void mma_fp8(uint32_t d, uint64_t ad, uint64_t bd, uint32_t idesc,
+                                        uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::
+          "r"(d),
+      "l"(ad), "l"(bd), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+__device__ __forceinline__ float silu_mul(uint32_t g_bits, uint32_t u_bits) {
+  const float g = __uint_as_float(g_bits);
+  return __fdividef(g * __uint_as_float(u_bits), 1.0f + __expf(-g));
+}
+
+__device__ __forceinline__ int decode_tile(int tile, int NT, const int* P, int E, int& m, int& n) {
+  const int g = tile / NT;
+  int lo = 0, hi = E;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (P[mid] <= g) lo = mid; else hi = mid;
+  }
+  const int mt = P[lo + 1] - P[lo];
+  const int local = tile - NT * P[lo];
+  n = local / mt;
+  m = local - n * mt;
+  return lo;
+}
+
+// Write one 128-byte row of the output box into the staging buffer at the
+// position the 128-byte swizzle of the output tensor map expects.
+__device__ __forceinline__ void stage_row(uint32_t staging, int r, const uint4 (&o)[8]) {
+#pragma unroll
+  for (int v = 0; v < 8; ++v) {
+    const uint32_t a = staging + (uint32_t)(r * 128 + ((v ^ (r & 7)) << 4));
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(o[v].x), "r"(o[v].y),
+                 "r"(o[v].z), "r"(o[v].w)
+                 : "memory");
+  }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const __grid_constant__ CUtensorMap tmOut, const uint8_t* __restrict__ sfa,
+                 const uint8_t* __restrict__ sfb, void* __restrict__ out_v,
+                 uint8_t* __restrict__ out_sf, int N_out, int Kdim, int b_rows_per_expert,
+                 int b_second_off, const int32_t* __restrict__ offsets,
+                 const int32_t* __restrict__ counts, int E, int C, long long R_max,
+                 uint32_t* __restrict__ status) {
+  constexpr int BN_OUT = (MODE == 0) ? 128 : 256;   // output columns per tile
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = saddr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  const uint32_t sf_smem = base + STAGES * OPER_BYTES;          // scale chunks of each stage
+  const uint32_t staging = sf_smem + STAGES * SF_STAGE;         // 1024-aligned
+  Ctl* ctl = reinterpret_cast<Ctl*>(smem + (staging - base) + STAGING_BYTES);
+  int* P = reinterpret_cast<int*>(ctl + 1);   // [E+1] M-tile prefix
+  int* row_off = P + (E + 1);                 // [E+1] first row of each expert, and R
+  int* kept_s = row_off + (E + 1);            // [E]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int NT = (N_out + BN_OUT - 1) / BN_OUT;
+  const int KB = Kdim / BK;
+  volatile int* abort_flag = &ctl->abort;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(saddr(&ctl->full[s]), 1);
+      mbar_init(saddr(&ctl->empty[s]), 1);
+    }
+    mbar_init(saddr(&ctl->tfull), 1);
+    mbar_init(saddr(&ctl->tempty), 4);
+    mbar_init(saddr(&ctl->drain), 1);
+    ctl->abort = 0;
+    fence_mbar_init();
+    prefetch_map(&tmA);
+    prefetch_map(&tmB);
+    prefetch_map(&tmOut);
+  }
+  if (warp == 1) {
+    tmem_alloc<1>(saddr(&ctl->tmem_base), TMEM_COLS);
+    tmem_relinquish<1>();
+  }
+  pdl_wait();
+  pdl_trigger();
+  {  // per-expert kept rows, first row and M-tile prefix (block scan)
+    const int chunk = (E + NUM_THREADS - 1) / NUM_THREADS;
+    const int e0 = threadIdx.x * chunk;
+    int local = 0;
+    for (int i = 0; i < chunk; ++i) {
+      const int e = e0 + i;
+      if (e < E) {
+        const int k = max(0, min(counts[e], C));
+        kept_s[e] = k;
+        row_off[e] = offsets[e];
+        local += (k + BM - 1) / BM;
+      }
+    }
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    if (lane == 31) ctl->wsum[warp] = incl;
+    __syncthreads();
+    int run = incl - local;
+    for (int w = 0; w < warp; ++w) run += ctl->wsum[w];
+    for (int i = 0; i < chunk; ++i) {
+      const int e = e0 + i;
+      if (e < E) {
+        P[e] = run;
+        run += (kept_s[e] + BM - 1) / BM;
+      }
+    }
+    if (threadIdx.x == NUM_THREADS - 1) {
+      P[E] = run;
+      row_off[E] = offsets[E];
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+  const int total = P[E] * NT;
+
+  if (warp == 0) {
+    if (lane == 0) {  // ------------------------------------------------ TMA producer
+      int it = 0;
+      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        int m, n;
+        const int e = decode_tile(tile, NT, P, E, m, n);
+        const int a_row = row_off[e] + m * BM;           // a multiple of 128
+        const int b_row0 = e * b_rows_per_expert + n * BN_OUT * (MODE == 0 ? 1 : 1);
+        const uint8_t* sa_rows = sfa + (size_t)(a_row / 128) * KB * SF_CHUNK;
+        const uint8_t* sb0_rows = sfb + (size_t)(b_row0 / 128) * KB * SF_CHUNK;
+        const uint8_t* sb1_rows = sfb + (size_t)((b_row0 + b_second_off) / 128) * KB * SF_CHUNK;
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (!wait_phase(saddr(&ctl->empty[s]), ph ^ 1u, abort_flag, status, WAIT_NS)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = base + s * OPER_BYTES;
+          const uint32_t ss = sf_smem + s * SF_STAGE;
+          const uint32_t fb = saddr(&ctl->full[s]);
+          mbar_expect_tx(fb, OPER_BYTES + SF_STAGE);
+          tma_load_2d<1>(sa, &tmA, kb * BK, a_row, fb);
+          tma_load_2d<1>(sa + A_BYTES, &tmB, kb * BK, b_row0, fb);
+          tma_load_2d<1>(sa + A_BYTES + B_HALF, &tmB, kb * BK, b_row0 + b_second_off, fb);
+          bulk_load(ss, sa_rows + (size_t)kb * SF_CHUNK, SF_CHUNK, fb);
+          bulk_load(ss + SF_CHUNK, sb0_rows + (size_t)kb * SF_CHUNK, SF_CHUNK, fb);
+          bulk_load(ss + 2 * SF_CHUNK, sb1_rows + (size_t)kb * SF_CHUNK, SF_CHUNK, fb);
+        }
+        if (!ok) break;
+      }
+      for (int i = max(0, it - STAGES); i < it; ++i)
+        wait_phase(saddr(&ctl->full[i % STAGES]), (uint32_t)(i / STAGES) & 1u, abort_flag, status,
+                   DRAIN_NS);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {  // ---------------------------------------------- MMA issuer
+      int it = 0, tcount = 0;
+      for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
+        if (!wait_phase(saddr(&ctl->tempty), ((uint32_t)tcount & 1u) ^ 1u, abort_flag, status,
+                        WAIT_NS))
+          break;
+        tc_fence_after();
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (!wait_phase(saddr(&ctl->full[s]), ph, abort_flag, status, WAIT_NS)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = base + s * OPER_BYTES;
+          const uint32_t ss = sf_smem + s * SF_STAGE;
+          const uint32_t tsf = tmem + SF_COL0 + (uint32_t)s * SF_COLS;
+          sf_copy(tsf, sf_desc(ss));
+          sf_copy(tsf + 4, sf_desc(ss + SF_CHUNK));
+          sf_copy(tsf + 8, sf_desc(ss + 2 * SF_CHUNK));
+          const uint64_t ad = sw128_desc(sa);
+          const uint64_t bd = sw128_desc(sa + A_BYTES);
+#pragma unroll
+          for (uint32_t j = 0; j < 4; ++j)
+            mma_fp8(tmem, ad + 2 * j, bd + 2 * j, idesc_fp8(j), tsf | (j << 30),
+                    (tsf + 4) | (j << 30), (kb | (int)j) != 0 ? 1u : 0u);
+          tc_commit<1>(saddr(&ctl->empty[s]));
+        }
+        if (!ok) break;
+        tc_commit<1>(saddr(&ctl->tfull));
+      }
+      tc_commit<1>(saddr(&ctl->drain));
+      wait_phase(saddr(&ctl->drain), 0u, abort_flag, status, DRAIN_NS);
+    }
+  } else {  // -------------------------------------------------------- epilogue
+    const int q = warp & 3;                 // TMEM lane quarter of this warp
+    const int r_in = q * 32 + lane;         // row of the tile
+    const int KBo = N_out / FP8_BLOCK;      // scale blocks of an output row (MODE 0)
+    int tcount = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
+      int m, n;
+      const int e = decode_tile(tile, NT, P, E, m, n);
+      const int first = m * BM;
+      const int rows = min(BM, kept_s[e] - first);
+      const long long row0 = (long long)row_off[e] + first;
+      const long long grow = row0 + r_in;
+      int ok = 1;
+      if (lane == 0) ok = wait_phase(saddr(&ctl->tfull), (uint32_t)tcount & 1u, abort_flag, status,
+                                     WAIT_NS);
+      __syncwarp();
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      bool row_ok = r_in < rows;
+      if (row_ok && (grow < 0 || grow >= R_max)) {   // inconsistent offsets from the caller
+        atomicCAS(status, 0u, (uint32_t)MOE_ERR_DEVICE_INPUT);
+        row_ok = false;
+      }
+      // a 128-row tile inside its expert's row range (alignment padding
+      // included) leaves through staged TMA stores, otherwise row by row
+      const bool staged = rows > 0 && row0 >= 0 && row0 + BM <= row_off[e + 1] && row0 + BM <= R_max;
+      const uint32_t t0 = tmem + ((uint32_t)(q * 32) << 16);
+      if (MODE == 0) {
+        float h[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t g[32], u[32];
+          tmem_ld32(t0 + (uint32_t)(c * 32), g);
+          tmem_ld32(t0 + 128u + (uint32_t)(c * 32), u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) h[c * 32 + k] = silu_mul(g[k], u[k]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_local(saddr(&ctl->tempty));   // TMEM free for the next tile
+        float amax = 0.f;
+#pragma unroll
+        for (int k = 0; k < 128; ++k) amax = fmaxf(amax, fabsf(h[k]));
+        const int p = fp8_scale_exp(amax);
+        const float inv = fp8_inv_scale(p);
+        uint4 o[8];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const float* hv = h + 16 * v;
+          o[v].x = fp8x2(hv[0] * inv, hv[1] * inv) | (fp8x2(hv[2] * inv, hv[3] * inv) << 16);
+          o[v].y = fp8x2(hv[4] * inv, hv[5] * inv) | (fp8x2(hv[6] * inv, hv[7] * inv) << 16);
+          o[v].z = fp8x2(hv[8] * inv, hv[9] * inv) | (fp8x2(hv[10] * inv, hv[11] * inv) << 16);
+          o[v].w = fp8x2(hv[12] * inv, hv[13] * inv) | (fp8x2(hv[14] * inv, hv[15] * inv) << 16);
+        }
+        if (row_ok)
+          *reinterpret_cast<uint32_t*>(out_sf + sf_offset(grow, n, KBo)) =
+              (uint32_t)(p + 127) * 0x01010101u;
+        if (staged) {
+          if (threadIdx.x == 64) bulk_wait_read_all();   // the previous box has left smem
+          epilogue_bar();
+          stage_row(staging, r_in, o);
+          fence_proxy_async_smem();
+          epilogue_bar();
+          if (threadIdx.x == 64) {
+            tma_store_2d(&tmOut, n * BN_OUT, (int)row0, staging);
+            bulk_commit();
+          }
+        } else if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(out_v) + grow * N_out +
+                                                (long long)n * BN_OUT);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) dst[v] = o[v];
+        }
+      } else {
+        uint32_t pk[128];   // 256 bf16 of this row
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t a[64];
+          tmem_ld64(t0 + (uint32_t)(c * 64), a);
+          tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            pk[c * 32 + k] = pack_bf16x2(__uint_as_float(a[2 * k]), __uint_as_float(a[2 * k + 1]));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_local(saddr(&ctl->tempty));
+        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(out_v) + (row_ok ? grow : 0) * (long long)N_out;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int col = n * BN_OUT + c * 64;
+          if (col >= N_out) continue;   // N_out % 64 == 0: a chunk is all in or all out
+          uint4 o[8];
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            o[v] = make_uint4(pk[c * 32 + 4 * v], pk[c * 32 + 4 * v + 1], pk[c * 32 + 4 * v + 2],
+                              pk[c * 32 + 4 * v + 3]);
+          if (staged) {
+            if (threadIdx.x == 64) bulk_wait_read_all();
+            epilogue_bar();
+            stage_row(staging, r_in, o);
+            fence_proxy_async_smem();
+            epilogue_bar();
+            if (threadIdx.x == 64) {
+              tma_store_2d(&tmOut, col, (int)row0, staging);
+              bulk_commit();
+            }
+          } else if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + col);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) dst[v] = o[v];
+          }
+        }
+      }
+    }
+    if (threadIdx.x == 64) bulk_wait_all();   // staged stores complete before the CTA exits
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc<1>(tmem, TMEM_COLS);
+  }
+}
+
+// 2-D uint8 map over a row-major [rows, cols] byte matrix: box 128 x 128,
+// 128-byte swizzle, zeros outside.
+bool make_map_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols};
+  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE>
+cudaError_t launch_one(int grid, size_t smem, cudaStream_t s, const CUtensorMap& a,
+                       const CUtensorMap& b, const CUtensorMap& o, const uint8_t* sfa,
+                       const uint8_t* sfb, void* out, uint8_t* out_sf, int N_out, int Kdim,
+                       int b_rows, int b_second, const int32_t* offsets, const int32_t* counts,
+                       int E, int C, long long R_max, uint32_t* status) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fp8_grouped_gemm<MODE>, a, b, o, sfa, sfb, out, out_sf, N_out,
+                            Kdim, b_rows, b_second, offsets, counts, E, C, R_max, status);
+}
+
+}  // namespace f8
+
+moe_status_t launch_mlp_fp8(const moe_config_t& c, const uint8_t* xq, const uint8_t* xs,
+                            const int32_t* offsets, const int32_t* counts, const uint8_t* wq_gu,
+                            const uint8_t* ws_gu, const uint8_t* wq_d, const uint8_t* ws_d,
+                            uint8_t* hq, uint8_t* hs, void* y, int64_t R_max, uint32_t* status,
+                            cudaStream_t s) {
+  using namespace f8;
+  if (R_max == 0) return MOE_OK;
+  CUtensorMap mx, mwgu, mh, mwd, my;
+  if (!make_map_u8(&mx, xq, (uint64_t)c.H, (uint64_t)R_max) ||
+      !make_map_u8(&mwgu, wq_gu, (uint64_t)c.H, (uint64_t)c.E * 2 * c.F) ||
+      !make_map_u8(&mh, hq, (uint64_t)c.F, (uint64_t)R_max) ||
+      !make_map_u8(&mwd, wq_d, (uint64_t)c.F, (uint64_t)c.E * c.H) ||
+      !tc::make_map(&my, y, (uint64_t)c.H, (uint64_t)R_max))
+    return MOE_ERR_CUDA;
+  const size_t smem = smem_bytes(c.E);
+  if (cudaFuncSetAttribute(fp8_grouped_gemm<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess ||
+      cudaFuncSetAttribute(fp8_grouped_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int64_t mt_bound = ceil_div(R_max, BM) + c.E;   // >= sum_e M tiles
+  const int g0 = (int)std::min<int64_t>(sms, mt_bound * ceil_div(c.F, 128));
+  const int g1 = (int)std::min<int64_t>(sms, mt_bound * ceil_div(c.H, 256));
+  cudaError_t e = launch_one<0>(g0, smem, s, mx, mwgu, mh, xs, ws_gu, hq, hs, c.F, c.H, 2 * c.F,
+                                c.F, offsets, counts, c.E, c.capacity, (long long)R_max, status);
+  if (e == cudaSuccess)
+    e = launch_one<1>(g1, smem, s, mh, mwd, my, hs, ws_d, y, nullptr, c.H, c.F, c.H, 128, offsets,
+                      counts, c.E, c.capacity, (long long)R_max, status);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace moe

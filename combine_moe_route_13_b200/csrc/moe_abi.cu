@@ -6,6 +6,7 @@
 #include <climits>
 #include <cmath>
 
+#include "fp8_util.cuh"
 #include "moe_internal.h"
 
 namespace moe {
@@ -53,6 +54,15 @@ moe_status_t validate(const moe_config_t* c, bool need_mlp) {
   return MOE_OK;
 }
 
+moe_status_t validate_fp8(const moe_config_t* c) {
+  moe_status_t st = validate(c, true);
+  if (st != MOE_OK) return st;
+  if (c->act_dtype != MOE_BF16 || c->H % 256 != 0 || c->F % FP8_BLOCK != 0 ||
+      c->row_align % 128 != 0 || c->n_shared != 0 || c->E > 512)
+    return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
 WsLayout ws_layout(const moe_config_t& c) {
   WsLayout L;
   const int64_t nblk = ceil_div(c.T, ROUTE_TB);
@@ -76,6 +86,10 @@ WsLayout ws_layout(const moe_config_t& c) {
   L.xp = p;        p += align256((size_t)R * c.H * as);
   L.h = p;         p += align256((size_t)R * c.F * as);
   L.y = p;         p += align256((size_t)R * c.H * as);
+  if (c.H % FP8_BLOCK == 0 && c.F % FP8_BLOCK == 0) {   // scales of the fp8 variant
+    L.xs = p;      p += align256((size_t)sf_bytes(R, c.H));
+    L.hs = p;      p += align256((size_t)sf_bytes(R, c.F));
+  }
   L.total = p;
   return L;
 }
@@ -267,7 +281,7 @@ static moe_status_t layer_forward(const moe_config_t* cfg, const float* logits,
   const WsLayout L = ws_layout(*cfg);
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   char* b = static_cast<char*>(ws);
-  moe_layer_aux_t a;
+  moe_layer_aux_t a = {};
   a.topk_idx = reinterpret_cast<int32_t*>(b + L.topk_idx);
   a.topk_w = reinterpret_cast<float*>(b + L.topk_w);
   a.expert_counts = reinterpret_cast<int32_t*>(b + L.counts);
@@ -341,6 +355,100 @@ moe_status_t moe_layer_forward_x(const moe_config_t* cfg, const void* x, const v
   if (!w_g) return MOE_ERR_INVALID_ARG;
   return layer_forward(cfg, nullptr, sel_bias, x, w_g, w_gu, w_d, out, flags, ws, ws_bytes, aux,
                        stream);
+}
+
+int64_t moe_fp8_scale_bytes(int64_t rows, int64_t cols) {
+  if (rows < 0 || cols <= 0 || cols % FP8_BLOCK != 0) return -1;
+  return sf_bytes(rows, cols);
+}
+
+moe_status_t moe_quantize_fp8(const void* src, int64_t rows, int64_t cols, uint8_t* codes,
+                              uint8_t* scales, void* stream) {
+  if (rows < 0 || cols <= 0 || cols % FP8_BLOCK != 0) return MOE_ERR_INVALID_ARG;
+  if (rows > INT_MAX || cols > (int64_t)INT_MAX / 2) return MOE_ERR_UNSUPPORTED;
+  if (rows == 0) return MOE_OK;
+  if (!src || !codes || !scales || !aligned16(src) || !aligned16(codes) || !aligned16(scales))
+    return MOE_ERR_INVALID_ARG;
+  return cuda_status(
+      launch_quantize_fp8(src, rows, cols, codes, scales, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_dispatch_fp8(const moe_config_t* cfg, const void* x, const int32_t* token_slot,
+                              uint8_t* xq, uint8_t* xs, void* stream) {
+  moe_status_t st = validate_fp8(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x || !token_slot || !xq || !xs) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(xq) || !aligned16(xs)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(
+      launch_dispatch_fp8(*cfg, x, token_slot, xq, xs, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_expert_mlp_fp8(const moe_config_t* cfg, const uint8_t* xq, const uint8_t* xs,
+                                const int32_t* expert_offsets, const int32_t* expert_counts,
+                                const uint8_t* wq_gu, const uint8_t* ws_gu, const uint8_t* wq_d,
+                                const uint8_t* ws_d, uint8_t* hq, uint8_t* hs, void* y, void* ws,
+                                size_t ws_bytes, void* stream) {
+  moe_status_t st = validate_fp8(cfg);
+  if (st != MOE_OK) return st;
+  const int64_t R = max_rows(*cfg);
+  if (R == 0) return MOE_OK;
+  if (!xq || !xs || !expert_offsets || !expert_counts || !wq_gu || !ws_gu || !wq_d || !ws_d ||
+      !hq || !hs || !y)
+    return MOE_ERR_INVALID_ARG;
+  for (const void* p : {(const void*)xq, (const void*)xs, (const void*)wq_gu, (const void*)ws_gu,
+                        (const void*)wq_d, (const void*)ws_d, (const void*)hq, (const void*)hs,
+                        (const void*)y})
+    if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < 256) return MOE_ERR_WORKSPACE;
+  return launch_mlp_fp8(*cfg, xq, xs, expert_offsets, expert_counts, wq_gu, ws_gu, wq_d, ws_d, hq,
+                        hs, y, R, static_cast<uint32_t*>(ws), static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_layer_forward_fp8(const moe_config_t* cfg, const float* logits, const void* x,
+                                   const uint8_t* wq_gu, const uint8_t* ws_gu,
+                                   const uint8_t* wq_d, const uint8_t* ws_d, void* out,
+                                   uint32_t flags, void* ws, size_t ws_bytes,
+                                   moe_layer_aux_t* aux, void* stream) {
+  moe_status_t st = validate_fp8(cfg);
+  if (st != MOE_OK) return st;
+  if (flags != MOE_FLAG_NONE) return MOE_ERR_UNSUPPORTED;
+  if (cfg->T > 0 && (!logits || !x || !out)) return MOE_ERR_INVALID_ARG;
+  if (!wq_gu || !ws_gu || !wq_d || !ws_d) return MOE_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(*cfg);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  char* b = static_cast<char*>(ws);
+  moe_layer_aux_t a = {};
+  a.topk_idx = reinterpret_cast<int32_t*>(b + L.topk_idx);
+  a.topk_w = reinterpret_cast<float*>(b + L.topk_w);
+  a.expert_counts = reinterpret_cast<int32_t*>(b + L.counts);
+  a.overflow = reinterpret_cast<int32_t*>(b + L.overflow);
+  a.expert_offsets = reinterpret_cast<int32_t*>(b + L.offsets);
+  a.segment_offsets = reinterpret_cast<int32_t*>(b + L.segoff);
+  a.totals = reinterpret_cast<int32_t*>(b + L.totals);
+  a.token_slot = reinterpret_cast<int32_t*>(b + L.slot);
+  a.row_src = reinterpret_cast<int32_t*>(b + L.row_src);
+  a.y = b + L.y;
+  a.xq = reinterpret_cast<uint8_t*>(b + L.xp);
+  a.xs = reinterpret_cast<uint8_t*>(b + L.xs);
+  a.hq = reinterpret_cast<uint8_t*>(b + L.h);
+  a.hs = reinterpret_cast<uint8_t*>(b + L.hs);
+  if (aux) *aux = a;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t R = max_rows(*cfg);
+  st = cuda_status(launch_route(*cfg, logits, a.topk_idx, a.topk_w, a.expert_counts, a.overflow,
+                                a.expert_offsets, a.segment_offsets, a.token_slot, a.row_src,
+                                a.totals, reinterpret_cast<int32_t*>(b + L.blk_cnt), R, s));
+  if (st != MOE_OK || cfg->T == 0) return st;
+  if (!aligned16(x) || !aligned16(out) || !aligned16(wq_gu) || !aligned16(ws_gu) ||
+      !aligned16(wq_d) || !aligned16(ws_d))
+    return MOE_ERR_INVALID_ARG;
+  st = cuda_status(launch_dispatch_fp8(*cfg, x, a.token_slot, a.xq, a.xs, s));
+  if (st != MOE_OK) return st;
+  st = launch_mlp_fp8(*cfg, a.xq, a.xs, a.expert_offsets, a.expert_counts, wq_gu, ws_gu, wq_d,
+                      ws_d, a.hq, a.hs, a.y, R, static_cast<uint32_t*>(ws), s);
+  if (st != MOE_OK) return st;
+  return cuda_status(launch_combine(*cfg, a.y, a.token_slot, a.topk_w, -1, out, s));
 }
 
 moe_status_t moe_get_device_status(void* ws, moe_status_t* status, void* stream) {

@@ -36,6 +36,7 @@ struct WsLayout {
   size_t topk_idx = 0, topk_w = 0, counts = 0, overflow = 0, offsets = 0;
   size_t segoff = 0, totals = 0, slot = 0, row_src = 0, row_ready = 0, logits = 0;
   size_t xp = 0, h = 0, y = 0;
+  size_t xs = 0, hs = 0;   // fp8 scales (the fp8 codes xq, hq reuse the xp, h regions)
   size_t total = 0;        // bytes needed by moe_layer_forward
 };
 
@@ -125,6 +126,18 @@ moe_status_t launch_router_logits_tc(const moe_config_t& c, const void* x, const
                                      float* logits, uint32_t* status, cudaStream_t s);
 cudaError_t launch_router_f32(const moe_config_t& c, const float* x, const float* w_g,
                               float* logits, cudaStream_t s);
+
+// ---- fp8 block-scaled path ----
+moe_status_t validate_fp8(const moe_config_t* c);
+cudaError_t launch_quantize_fp8(const void* src, int64_t rows, int64_t cols, uint8_t* q,
+                                uint8_t* sf, cudaStream_t s);
+cudaError_t launch_dispatch_fp8(const moe_config_t& c, const void* x, const int32_t* slot,
+                                uint8_t* xq, uint8_t* xs, cudaStream_t s);
+moe_status_t launch_mlp_fp8(const moe_config_t& c, const uint8_t* xq, const uint8_t* xs,
+                            const int32_t* offsets, const int32_t* counts, const uint8_t* wq_gu,
+                            const uint8_t* ws_gu, const uint8_t* wq_d, const uint8_t* ws_d,
+                            uint8_t* hq, uint8_t* hs, void* y, int64_t R_max, uint32_t* status,
+                            cudaStream_t s);
 
 // Ready-counter target of the down GEMM (its number of N tiles).
 inline uint32_t ready_target(const moe_config_t& c) { return (uint32_t)ceil_div(c.H, 256); }

@@ -79,7 +79,7 @@ __device__ __forceinline__ unsigned long long globaltimer() {
 // Slow path of wait_phase: keep polling until the phase completes, the CTA's
 // abort flag is raised, or `limit_ns` passes; a timeout raises the flag and
 // records MOE_ERR_TIMEOUT.
-__device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity,
+static __device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity,
                                              volatile int* abort_flag, uint32_t* status,
                                              unsigned long long limit_ns) {
   const unsigned long long t0 = globaltimer();

@@ -94,6 +94,7 @@ typedef struct {
   float *topk_w;
   void *xp, *h, *y;
   float *logits;   /* [T,E]: the router projection's output (moe_layer_forward_x only) */
+  uint8_t *xq, *xs, *hq, *hs;   /* fp8 payload and its scales (moe_layer_forward_fp8 only) */
 } moe_layer_aux_t;
 
 #define MOE_FLAG_NONE 0u
@@ -291,6 +292,66 @@ moe_status_t moe_layer_forward_x(const moe_config_t* cfg, const void* x, const v
                                  const float* sel_bias, const void* w_gu, const void* w_d,
                                  void* out, uint32_t flags, void* ws, size_t ws_bytes,
                                  moe_layer_aux_t* aux, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * fp8 block-scaled variant ("Enabling trillion-parameter models on AWS EFA",
+ * "Оценка": fp8 with block scaling for the dispatch, bf16 for the combine; the
+ * pplx-kernels page, "Dispatch": tokens travel with their block scale factors).
+ *
+ * Format (the pages fix neither block shape nor scale encoding; this is the
+ * library's reading): e4m3 codes (round to nearest even); one scale per 128
+ * consecutive elements of a row along the contraction dimension; the scale is a
+ * power of two 2^p stored as the byte p + 127 (UE8M0), p the smallest integer
+ * >= -127 with max|block| <= 448 * 2^p.
+ * Scale layout (what the tensor cores read): for each block of 128 rows and each
+ * 128-element k block, a 512-byte chunk at ((r / 128) * (cols / 128) + kb) * 512;
+ * row r owns bytes 16*(r % 32) + 4*((r % 128) / 32) + {0,1,2,3} of it, all four
+ * holding its scale byte. A [rows, cols] matrix has moe_fp8_scale_bytes(rows, cols)
+ * bytes of scales; bytes of rows past `rows` are never written.
+ * The whole fp8 path requires bf16 activations, H % 256 == 0, F % 128 == 0,
+ * row_align % 128 == 0, n_shared == 0 and E <= 512 (else MOE_ERR_UNSUPPORTED).
+ * ------------------------------------------------------------------------- */
+
+/* ceil(rows / 128) * (cols / 128) * 512, or -1 if rows < 0 or cols is not a
+ * positive multiple of 128. */
+int64_t moe_fp8_scale_bytes(int64_t rows, int64_t cols);
+
+/* Block-quantise a [rows, cols] bf16 matrix (device, row-major; cols % 128 == 0):
+ * codes [rows, cols] e4m3 bytes, scales in the layout above. Used once for the
+ * expert weights: w_gu as [E*2F, H] and w_d as [E*H, F]. */
+moe_status_t moe_quantize_fp8(const void* src, int64_t rows, int64_t cols, uint8_t* codes,
+                              uint8_t* scales, void* stream);
+
+/* Dispatch with the fp8 payload: each token row of x [T,H] bf16 is quantised once
+ * and its codes and scales written to every kept row token_slot[t,k] of
+ * xq [R_max,H] (e4m3) and xs (moe_fp8_scale_bytes(R_max, H) bytes). Rows no slot
+ * points at are not written. */
+moe_status_t moe_dispatch_fp8(const moe_config_t* cfg, const void* x, const int32_t* token_slot,
+                              uint8_t* xq, uint8_t* xs, void* stream);
+
+/* Grouped SwiGLU on the fp8 payload (tcgen05 block-scaled MMA, fp32 accumulate):
+ * for every expert e and kept row r,
+ *   h[r] = silu(xq[r] Wg_e^T) * (xq[r] Wu_e^T), quantised to hq[r] (e4m3) and hs
+ *          (scales of the [R_max, F] matrix) from its fp32 value,
+ *   y[r] = hq[r] W_d,e^T rounded to bf16,
+ * with every operand taken as scale * e4m3 value. wq_gu [E,2F,H] e4m3 with scales
+ * ws_gu of the [E*2F, H] matrix; wq_d [E,H,F] with ws_d of [E*H, F] (from
+ * moe_quantize_fp8). y [R_max,H] bf16. ws: any workspace with a status word. */
+moe_status_t moe_expert_mlp_fp8(const moe_config_t* cfg, const uint8_t* xq, const uint8_t* xs,
+                                const int32_t* expert_offsets, const int32_t* expert_counts,
+                                const uint8_t* wq_gu, const uint8_t* ws_gu, const uint8_t* wq_d,
+                                const uint8_t* ws_d, uint8_t* hq, uint8_t* hs, void* y, void* ws,
+                                size_t ws_bytes, void* stream);
+
+/* The whole layer with the fp8 payload: route -> moe_dispatch_fp8 ->
+ * moe_expert_mlp_fp8 -> moe_combine (bf16), intermediates in the workspace
+ * (moe_workspace_bytes). flags must be MOE_FLAG_NONE. aux (optional) also gets
+ * xq, xs, hq, hs. */
+moe_status_t moe_layer_forward_fp8(const moe_config_t* cfg, const float* logits, const void* x,
+                                   const uint8_t* wq_gu, const uint8_t* ws_gu,
+                                   const uint8_t* wq_d, const uint8_t* ws_d, void* out,
+                                   uint32_t flags, void* ws, size_t ws_bytes,
+                                   moe_layer_aux_t* aux, void* stream);
 
 /* Synchronise `stream`, read the workspace's status word into *status and reset
  * it to MOE_OK. Returns MOE_ERR_CUDA if the synchronisation or copy failed. */

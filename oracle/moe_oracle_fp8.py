@@ -107,6 +107,13 @@ def dequantize_rows(codes: np.ndarray, p: np.ndarray) -> np.ndarray:
     return np.ldexp(vals, np.asarray(p)[:, :, None].astype(np.int32)).reshape(rows, K)
 
 
+def _scale_positions(rows: int, KB: int) -> np.ndarray:
+    """Byte offset of the first of the four copies of scale (r, kb): [rows, KB]."""
+    r = np.arange(rows, dtype=np.int64)[:, None]
+    kb = np.arange(KB, dtype=np.int64)[None, :]
+    return ((r // 128) * KB + kb) * 512 + 16 * (r % 32) + 4 * ((r % 128) // 32)
+
+
 def scales_blocked(p: np.ndarray, row_blocks: int | None = None, pad: int | None = None) -> np.ndarray:
     """The scale bytes (p + 127) in the byte layout the library's kernels read.
 
@@ -122,11 +129,9 @@ def scales_blocked(p: np.ndarray, row_blocks: int | None = None, pad: int | None
     rows, KB = p.shape
     RB = -(-rows // 128) if row_blocks is None else row_blocks
     out = np.full(RB * KB * 512, 0 if pad is None else pad, dtype=np.uint8)
-    for r in range(rows):
-        rb, i, j = r // 128, r % 32, (r % 128) // 32
-        for kb in range(KB):
-            base = (rb * KB + kb) * 512 + 16 * i + 4 * j
-            out[base:base + 4] = p[r, kb] + 127
+    pos = _scale_positions(rows, KB)
+    for s in range(4):
+        out[pos + s] = (p + 127).astype(np.uint8)
     return out
 
 
@@ -134,16 +139,12 @@ def scales_from_blocked(buf: np.ndarray, rows: int, KB: int) -> np.ndarray:
     """Inverse of scales_blocked for the first `rows` rows: p [rows, KB].
     Raises if a row's four copies of a scale disagree."""
     buf = np.asarray(buf, dtype=np.uint8)
-    p = np.empty((rows, KB), np.int64)
-    for r in range(rows):
-        rb, i, j = r // 128, r % 32, (r % 128) // 32
-        for kb in range(KB):
-            base = (rb * KB + kb) * 512 + 16 * i + 4 * j
-            q = buf[base:base + 4]
-            if not np.all(q == q[0]):
-                raise ValueError(f"row {r} block {kb}: scale copies differ {q.tolist()}")
-            p[r, kb] = int(q[0]) - 127
-    return p
+    pos = _scale_positions(rows, KB)
+    q = np.stack([buf[pos + s] for s in range(4)])
+    if not np.all(q == q[0]):
+        bad = np.argwhere(np.any(q != q[0], axis=0))[0]
+        raise ValueError(f"row {bad[0]} block {bad[1]}: scale copies differ {q[:, bad[0], bad[1]].tolist()}")
+    return q[0].astype(np.int64) - 127
 
 
 def dispatch_fp8(x_bf16: np.ndarray, token_slot: np.ndarray, R_max: int):

@@ -17,7 +17,7 @@ HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))
 def declared_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_library_exports_every_declared_symbol():
@@ -168,3 +168,42 @@ def test_status_strings():
         s = M.status_string(code)
         assert s and s != "unknown status"
     assert M.status_string(99) == "unknown status"
+
+
+def test_fp8_scale_bytes():
+    assert M.moe_fp8_scale_bytes(1, 128) == 512
+    assert M.moe_fp8_scale_bytes(128, 256) == 1024
+    assert M.moe_fp8_scale_bytes(129, 7168) == 2 * 56 * 512
+    assert M.moe_fp8_scale_bytes(0, 128) == 0
+    assert M.moe_fp8_scale_bytes(10, 100) == -1 and M.moe_fp8_scale_bytes(-1, 128) == -1
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(act="f32"), M.MOE_ERR_UNSUPPORTED),
+    (dict(H=4224), M.MOE_ERR_UNSUPPORTED),          # H % 256 != 0
+    (dict(F=14400), M.MOE_ERR_UNSUPPORTED),         # F % 128 != 0
+    (dict(row_align=64), M.MOE_ERR_UNSUPPORTED),
+    (dict(n_shared=1), M.MOE_ERR_UNSUPPORTED),
+    (dict(E=640, K=2, S=8), M.MOE_ERR_UNSUPPORTED),
+])
+def test_fp8_configs_outside_the_kernels_are_rejected(kw, code):
+    w = W.WORKLOADS["mixtral"]
+    cfg = cfg_of(w, **kw)
+    fake = ctypes.c_void_p(0x10000)
+    assert M.LIB.moe_layer_forward_fp8(ctypes.byref(cfg), fake, fake, fake, fake, fake, fake, fake,
+                                       0, fake, 1 << 40, None, None) == code
+    assert M.LIB.moe_dispatch_fp8(ctypes.byref(cfg), fake, fake, fake, fake, None) == code
+
+
+def test_fp8_entry_points_reject_bad_arguments():
+    lib = M.LIB
+    cfg = cfg_of(W.WORKLOADS["mixtral"])
+    fake = ctypes.c_void_p(0x10000)
+    assert lib.moe_quantize_fp8(fake, 10, 100, fake, fake, None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_quantize_fp8(None, 10, 128, fake, fake, None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_quantize_fp8(fake, 0, 128, None, None, None) == M.MOE_OK
+    assert lib.moe_dispatch_fp8(ctypes.byref(cfg), None, fake, fake, fake, None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_layer_forward_fp8(ctypes.byref(cfg), fake, fake, fake, fake, fake, fake, fake,
+                                     M.MOE_FLAG_OVERLAP, fake, 1 << 40, None, None) == M.MOE_ERR_UNSUPPORTED
+    assert lib.moe_layer_forward_fp8(ctypes.byref(cfg), fake, fake, fake, fake, fake, fake, fake,
+                                     0, fake, 1024, None, None) == M.MOE_ERR_WORKSPACE
