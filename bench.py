@@ -168,11 +168,12 @@ class Layer:
     """Device-resident inputs, weights and workspace of one replica."""
 
     def __init__(self, wl: W.Workload, seed: int, device, overlap: bool = False,
-                 router: bool = False):
+                 router: bool = False, fp8: bool = False):
         import combine_moe_route_13_b200 as M
         self.M = M
         self.flags = M.MOE_FLAG_OVERLAP if overlap else M.MOE_FLAG_NONE
         self.router = router
+        self.fp8 = fp8
         self.wl = wl
         self.C = M.moe_capacity(wl.T, wl.K, wl.E, wl.cf)
         self.cfg = M.make_config(wl.T, wl.H, wl.E, wl.K, wl.F, wl.S, self.C, wl.row_align, wl.act,
@@ -181,13 +182,20 @@ class Layer:
         if st != M.MOE_OK:
             raise SystemExit(f"unsupported workload: {M.status_string(st)}")
         self.inp = W.make_inputs(wl, seed=seed, device=device, router=router)
+        if fp8:   # weights quantised once, before any timing (a preparation step)
+            self.wq = M.quantize_fp8(self.inp["w_gu"]) + M.quantize_fp8(self.inp["w_d"])
+            del self.inp["w_gu"], self.inp["w_d"]
+            torch.cuda.synchronize()
         self.ws = M.alloc_workspace(M.moe_workspace_bytes(self.cfg), device)
         self.out = torch.empty(wl.T, wl.H, dtype=wl.torch_act, device=device)
         self.aux = None
 
     def forward(self, x=None, logits=None):
         x = self.inp["x"] if x is None else x
-        if self.router:   # from hidden states: router projection + selection-only bias
+        if self.fp8:
+            logits = self.inp["logits"] if logits is None else logits
+            self.aux = self.M.moe_layer_forward_fp8(self.cfg, logits, x, *self.wq, self.out, self.ws)
+        elif self.router:   # from hidden states: router projection + selection-only bias
             self.aux = self.M.moe_layer_forward_x(self.cfg, x, self.inp["w_g"],
                                                   self.inp["sel_bias"], self.inp["w_gu"],
                                                   self.inp["w_d"], self.out, self.ws,
@@ -226,6 +234,9 @@ def phase_times(layer: Layer, steps, flush_buf, stream):
     names = ("router", "route", "dispatch", "expert_mlp", "combine")
     logits = v["logits"] if layer.router else inp["logits"]
     bias = inp["sel_bias"] if layer.router else None
+    if layer.fp8:
+        f = M.fp8_views(cfg, layer.ws, layer.aux)
+        gq, gs, dq, ds = layer.wq
     calls = (
         (lambda: M.moe_router_logits(cfg, inp["x"], inp["w_g"], v["logits"], layer.ws))
         if layer.router else (lambda: None),
@@ -233,9 +244,14 @@ def phase_times(layer: Layer, steps, flush_buf, stream):
                                         v["expert_counts"], v["overflow"], v["expert_offsets"],
                                         v["segment_offsets"], v["token_slot"], v["row_src"],
                                         v["totals"], layer.ws),
-        lambda: M.moe_dispatch(cfg, inp["x"], v["token_slot"], v["xp"]),
-        lambda: M.moe_expert_mlp(cfg, v["xp"], v["expert_offsets"], v["expert_counts"],
-                                 inp["w_gu"], inp["w_d"], v["h"], v["y"], layer.ws),
+        (lambda: M.moe_dispatch_fp8(cfg, inp["x"], v["token_slot"], f["xq"], f["xs"]))
+        if layer.fp8 else (lambda: M.moe_dispatch(cfg, inp["x"], v["token_slot"], v["xp"])),
+        (lambda: M.moe_expert_mlp_fp8(cfg, f["xq"], f["xs"], v["expert_offsets"],
+                                      v["expert_counts"], gq, gs, dq, ds, f["hq"], f["hs"],
+                                      v["y"], layer.ws))
+        if layer.fp8 else
+        (lambda: M.moe_expert_mlp(cfg, v["xp"], v["expert_offsets"], v["expert_counts"],
+                                  inp["w_gu"], inp["w_d"], v["h"], v["y"], layer.ws)),
         lambda: M.moe_combine(cfg, v["y"], v["token_slot"], v["topk_w"], layer.out),
     )
     acc = {n: [] for n in names}
@@ -281,6 +297,8 @@ def mlp_tile_rows(layer: Layer) -> int:
     wl = layer.wl
     if wl.act == "f32":
         return 32
+    if layer.fp8:
+        return 128
     return 256 if min(wl.T * wl.K, wl.E * layer.C) // wl.E >= 192 else 128
 
 
@@ -300,7 +318,8 @@ def algorithmic(layer: Layer, totals, counts):
         "executed_rows": executed,
         "mlp_flops": 6.0 * (N + Ns) * H * F,
         "mlp_executed_flops": 6.0 * executed * H * F,
-        "dispatch_bytes": (T + N + Ns) * H * s + T * K * 4,
+        "dispatch_bytes": (T * H * s + (N + Ns) * H * (1 + 4 / 128) + T * K * 4) if layer.fp8
+        else (T + N + Ns) * H * s + T * K * 4,
         "combine_bytes": (N + Ns + T) * H * s + T * K * 8,
         "route_bytes": T * E * 4 + T * K * 12,
     }
@@ -324,6 +343,24 @@ def cpu_oracle_sample(wl: W.Workload, tokens: int, seed: int, inp_host=None):
     C = O.capacity(tokens, wl.K, wl.E, wl.cf)
     t0 = time.perf_counter()
     O.layer_forward(lg, x, w_gu, w_d, wl.K, C, wl.row_align, wl.S, wl.act, n_shared=wl.n_shared)
+    return time.perf_counter() - t0, tokens
+
+
+def cpu_oracle_sample_fp8(wl: W.Workload, tokens: int, layer: "Layer"):
+    """The fp8 oracle's whole layer on the first `tokens` tokens, with the
+    expert weights as the library quantised them (its quantiser is bit-exact
+    with the oracle's). Returns (seconds, tokens)."""
+    from oracle import moe_oracle as O
+    from oracle import moe_oracle_fp8 as Q
+    E, F, H = wl.E, wl.F, wl.H
+    gq, gs, dq, ds = (t.cpu().numpy() for t in layer.wq)
+    ge = Q.scales_from_blocked(gs, E * 2 * F, H // 128).reshape(E, 2 * F, H // 128)
+    de = Q.scales_from_blocked(ds, E * H, F // 128).reshape(E, H, F // 128)
+    lg = layer.inp["logits"][:tokens].cpu().numpy()
+    x = layer.inp["x"][:tokens].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    C = O.capacity(tokens, wl.K, wl.E, wl.cf)
+    t0 = time.perf_counter()
+    Q.layer_forward_fp8(lg, x, gq, ge, dq, de, wl.K, C, wl.row_align, wl.S)
     return time.perf_counter() - t0, tokens
 
 
@@ -378,6 +415,8 @@ def main(argv=None):
                          "selection-only bias (moe_layer_forward_x)")
     ap.add_argument("--overlap", action="store_true",
                     help="overlap the combine with the down GEMM (MOE_FLAG_OVERLAP)")
+    ap.add_argument("--fp8", action="store_true",
+                    help="fp8 block-scaled payload and expert GEMMs (moe_layer_forward_fp8)")
     ap.add_argument("--shared", action="store_true",
                     help="add one shared expert of the routed width (as DeepSeek-V3 and Kimi-K2 have)")
     args = ap.parse_args(argv)
@@ -386,6 +425,8 @@ def main(argv=None):
     wl = W.WORKLOADS[args.workload]
     if args.shared:
         wl = wl.with_(name=wl.name + "_shared", n_shared=1)
+    if args.fp8:
+        wl = wl.with_(name=wl.name + "_fp8")
     world, rank, local = dist_env()
     if args.impl == "reference":
         return run_reference(args, wl, world, rank)
@@ -398,7 +439,8 @@ def main(argv=None):
     torch.cuda.set_device(device)
     peaks = load_peaks()
 
-    layer = Layer(wl, seed=rank, device=device, overlap=args.overlap, router=args.router)
+    layer = Layer(wl, seed=rank, device=device, overlap=args.overlap, router=args.router,
+                  fp8=args.fp8)
     flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream()
 
@@ -435,6 +477,10 @@ def main(argv=None):
 
     hbm = peaks["hbm_gbs"]
     tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    peak_kind = f"bf16_tflops_sustained ({peaks['source']})"
+    if args.fp8:   # fp8 dense rate = 2 x bf16 (nominal 4.5 / 2.25 PFLOP/s)
+        tensor_peak *= 2.0
+        peak_kind += " x 2 (nominal fp8/bf16 ratio)"
     mlp_tflops = alg["mlp_flops"] / (ph["expert_mlp"] * 1e-3) / 1e12
     kernels = {
         "router_us": ph["router"] * 1e3 if args.router else None,
@@ -448,7 +494,7 @@ def main(argv=None):
     }
     kernels["dispatch_hbm_frac"] = kernels["dispatch_gbs"] / hbm
     kernels["combine_hbm_frac"] = kernels["combine_gbs"] / hbm
-    kernels["expert_mlp_tensor_frac_burst"] = mlp_tflops / peaks["bf16_tflops"]
+    kernels["expert_mlp_tensor_frac_burst"] = mlp_tflops / (peaks["bf16_tflops"] * (2.0 if args.fp8 else 1.0))
     kernels["expert_mlp_executed_tflops"] = alg["mlp_executed_flops"] / (ph["expert_mlp"] * 1e-3) / 1e12
     kernels["expert_mlp_tile_rows"] = alg["tile_rows"]
     kernels["expert_mlp_executed_rows"] = alg["executed_rows"]
@@ -460,28 +506,34 @@ def main(argv=None):
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        secs, tok = cpu_oracle_sample(wl, args.cpu_tokens, 0)
+        if args.fp8:
+            secs, tok = cpu_oracle_sample_fp8(wl, args.cpu_tokens, layer)
+        else:
+            secs, tok = cpu_oracle_sample(wl, args.cpu_tokens, 0)
         cpu = {"value": tok / secs, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
-               "sample": f"whole layer (float64 numpy oracle) on the first {tok} tokens of the "
-                         f"workload, capacity scaled to that batch; {secs:.1f} s"}
+               "sample": f"whole layer ({'fp8 ' if args.fp8 else ''}float64 numpy oracle) on the "
+                         f"first {tok} tokens of the workload, capacity scaled to that batch; "
+                         f"{secs:.1f} s"}
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.act == "bf16" else "f32",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": ("fp8" if args.fp8 else "bf16") if wl.act == "bf16" else "f32",
         "data": "synthetic",
         "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "K": wl.K, "F": wl.F,
                    "S": wl.S, "cf": wl.cf, "capacity": layer.C, "row_align": wl.row_align,
                    "effective_tokens": alg["N"], "overflow": int(totals[2]),
                    "l2": "flushed (256 MB write) before every step", "parallelism": f"replicas{world}",
                    "overlap": bool(args.overlap), "router_projection": bool(args.router),
-                   "n_shared": wl.n_shared},
+                   "n_shared": wl.n_shared,
+                   "payload": "e4m3, 1x128 blocks, UE8M0 scales; bf16 combine" if args.fp8 else wl.act},
         "e2e": {"value": world * wl.T / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": (KERNELS_PER_STEP + (1 if args.router else 0)) * args.steps,
         "roofline": {"bound": "tensor", "kernel": "expert_mlp (gate/up + down grouped GEMMs)",
                      "achieved": mlp_tflops, "peak": tensor_peak, "unit": "TFLOP/s",
                      "frac": mlp_tflops / tensor_peak,
-                     "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
+                     "peak_kind": peak_kind,
                      "traffic": measured_traffic(wl.name),
                      "traffic_unit": "bytes per moe_expert_mlp call (ncu dram read+write)"},
         "kernels": kernels,
