@@ -312,10 +312,17 @@ def algorithmic(layer: Layer, totals, counts):
     # the shared expert (if any) is one more group of T rows
     Ns = wl.n_shared * T
     executed = int(np.sum((kept + tr - 1) // tr * tr)) + (Ns + tr - 1) // tr * tr
+    # bytes the expert MLP must move at least: the weights of every expert that
+    # has rows (read once), its input rows, h written and read back, y written
+    ws_ = 1 if layer.fp8 else s           # weight / xp / h element size
+    active = int(np.count_nonzero(kept)) + wl.n_shared
+    mlp_bytes = (3 * active * H * F * ws_ * (1 + (4 / 128 if layer.fp8 else 0))
+                 + (N + Ns) * (H * ws_ + 2 * F * ws_ + H * s))
     return {
         "N": N,
         "tile_rows": tr,
         "executed_rows": executed,
+        "mlp_bytes": mlp_bytes,
         "mlp_flops": 6.0 * (N + Ns) * H * F,
         "mlp_executed_flops": 6.0 * executed * H * F,
         "dispatch_bytes": (T * H * s + (N + Ns) * H * (1 + 4 / 128) + T * K * 4) if layer.fp8
@@ -482,6 +489,9 @@ def main(argv=None):
         tensor_peak *= 2.0
         peak_kind += " x 2 (nominal fp8/bf16 ratio)"
     mlp_tflops = alg["mlp_flops"] / (ph["expert_mlp"] * 1e-3) / 1e12
+    mlp_gbs = alg["mlp_bytes"] / (ph["expert_mlp"] * 1e-3) / 1e9
+    # the binding roofline of the expert MLP: tensor time or HBM time, whichever is longer
+    hbm_bound = alg["mlp_bytes"] / (hbm * 1e9) > alg["mlp_flops"] / (tensor_peak * 1e12)
     kernels = {
         "router_us": ph["router"] * 1e3 if args.router else None,
         "route_us": ph["route"] * 1e3,
@@ -489,6 +499,7 @@ def main(argv=None):
         "dispatch_gbs": alg["dispatch_bytes"] / (ph["dispatch"] * 1e-3) / 1e9,
         "expert_mlp_us": ph["expert_mlp"] * 1e3,
         "expert_mlp_tflops": mlp_tflops,
+        "expert_mlp_gbs": mlp_gbs,
         "combine_us": ph["combine"] * 1e3,
         "combine_gbs": alg["combine_bytes"] / (ph["combine"] * 1e-3) / 1e9,
     }
@@ -530,10 +541,15 @@ def main(argv=None):
         "e2e": {"value": world * wl.T / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": (KERNELS_PER_STEP + (1 if args.router else 0)) * args.steps,
-        "roofline": {"bound": "tensor", "kernel": "expert_mlp (gate/up + down grouped GEMMs)",
-                     "achieved": mlp_tflops, "peak": tensor_peak, "unit": "TFLOP/s",
-                     "frac": mlp_tflops / tensor_peak,
-                     "peak_kind": peak_kind,
+        "roofline": ({"bound": "hbm", "kernel": "expert_mlp (gate/up + down grouped GEMMs)",
+                      "achieved": mlp_gbs, "peak": hbm, "unit": "GB/s", "frac": mlp_gbs / hbm,
+                      "peak_kind": f"hbm_gbs ({peaks['source']})",
+                      "tensor_frac": mlp_tflops / tensor_peak}
+                     if hbm_bound else
+                     {"bound": "tensor", "kernel": "expert_mlp (gate/up + down grouped GEMMs)",
+                      "achieved": mlp_tflops, "peak": tensor_peak, "unit": "TFLOP/s",
+                      "frac": mlp_tflops / tensor_peak, "peak_kind": peak_kind,
+                      "hbm_frac": mlp_gbs / hbm}) | {
                      "traffic": measured_traffic(wl.name),
                      "traffic_unit": "bytes per moe_expert_mlp call (ncu dram read+write)"},
         "kernels": kernels,
