@@ -8,9 +8,10 @@
 // (UE8M0), p the smallest integer >= -127 with amax <= 448 * 2^p.
 //
 // Scale bytes live in the layout the block-scaled MMA reads after a
-// tcgen05.cp of 32 rows x 16 bytes: for each block of 128 rows and each
-// 128-element k block a 512-byte chunk; row r owns bytes 16*(r%32) + 4*((r%128)/32)
-// + {0..3} of its chunk, all four holding its scale (one per 32-element part).
+// tcgen05.cp of 32 rows x 16 bytes: for each block of 128 rows and each group
+// of four 128-element k blocks a 512-byte chunk; row r's scale for k block kb
+// is byte 16*(r%32) + 4*((r%128)/32) + kb%4 of chunk (r/128, kb/4). One chunk
+// copy serves four k blocks: the MMA selects the byte with its scale-factor id.
 #pragma once
 
 #include <cstdint>
@@ -20,16 +21,17 @@
 namespace moe {
 
 constexpr int FP8_BLOCK = 128;     // elements per scale
-constexpr int SF_CHUNK = 512;      // scale bytes of 128 rows x one k block
+constexpr int SF_CHUNK = 512;      // scale bytes of 128 rows x four k blocks
 
-// Byte offset of row r's scales for k block kb (KB k blocks per row).
+// Byte offset of row r's scale for k block kb (KB k blocks per row).
 __host__ __device__ __forceinline__ int64_t sf_offset(int64_t r, int kb, int KB) {
-  return ((r / 128) * KB + kb) * SF_CHUNK + 16 * (r % 32) + 4 * ((r % 128) / 32);
+  const int KG = (KB + 3) / 4;
+  return ((r / 128) * KG + kb / 4) * SF_CHUNK + 16 * (r % 32) + 4 * ((r % 128) / 32) + kb % 4;
 }
 
 // Bytes of scales for a [rows, cols] matrix.
 __host__ __device__ __forceinline__ int64_t sf_bytes(int64_t rows, int64_t cols) {
-  return ((rows + 127) / 128) * (cols / FP8_BLOCK) * SF_CHUNK;
+  return ((rows + 127) / 128) * ((cols / FP8_BLOCK + 3) / 4) * SF_CHUNK;
 }
 
 #ifdef __CUDACC__

@@ -17,13 +17,17 @@
 //   MODE 1: y = hq W_d[e]^T (N = 256 columns), epilogue rounds to bf16.
 //
 // Per stage (128 k values = one 128-byte swizzle row of e4m3): TMA boxes of A
-// (128 rows) and B (2 x 128 rows), and three 512-byte scale chunks (A, B rows
-// 0-127, B rows 128-255) by bulk copy. The MMA thread moves the chunks into
-// TMEM with tcgen05.cp (32 rows x 16 bytes, replicated to the four lane
-// quarters) and issues four K = 32 MMAs, the j-th reading scale byte j.
+// (128 rows) and B (2 x 128 rows). A scale chunk covers four k blocks, so the
+// three chunks of a k group (A, B rows 0-127, B rows 128-255; 512 bytes each,
+// by bulk copy) ride with one stage in four: group 0 with the tile's first
+// stage, group g > 0 three stages before it is used (with stage 4g - 3). The
+// MMA thread moves them into TMEM with tcgen05.cp (32 rows x 16 bytes,
+// replicated to the four lane quarters) when they arrive, into one of two
+// scale slots, so that a copy's latency overlaps the previous group's MMAs;
+// each K = 32 MMA of k block kb reads scale byte kb % 4 (its scale-factor id).
 //
-// TMEM: the 256-column fp32 accumulator at column 0 (single buffer) and 12
-// scale columns per stage from column 256. To overlap one tile's epilogue with
+// TMEM: the 256-column fp32 accumulator at column 0 (single buffer) and two
+// 12-column scale slots from column 256. To overlap one tile's epilogue with
 // the next tile's MMAs despite the single accumulator, the epilogue first
 // loads its whole row into registers and releases TMEM, then quantises /
 // rounds and stores.
@@ -59,7 +63,7 @@ constexpr int STAGES = 4;
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL0 = 256;
-constexpr uint32_t SF_COLS = 12;                // per stage: 4 (A) + 8 (B)
+constexpr uint32_t SF_COLS = 12;                // per scale slot: 4 (A) + 8 (B)
 constexpr int STAGING_BYTES = 128 * 128;        // one 128-row x 128-byte output box
 constexpr unsigned long long WAIT_NS = 2000000000ull;
 constexpr unsigned long long DRAIN_NS = 200000000ull;
@@ -131,6 +135,13 @@ __device__ __forceinline__ float silu_mul(uint32_t g_bits, uint32_t u_bits) {
   return __fdividef(g * __uint_as_float(u_bits), 1.0f + __expf(-g));
 }
 
+// The k group whose scales ride with stage kb, or -1.
+__device__ __forceinline__ int sf_group_of_stage(int kb, int KG) {
+  if (kb == 0) return 0;
+  if ((kb & 3) == 1 && (kb >> 2) + 1 < KG) return (kb >> 2) + 1;
+  return -1;
+}
+
 __device__ __forceinline__ int decode_tile(int tile, int NT, const int* P, int E, int& m, int& n) {
   const int g = tile / NT;
   int lo = 0, hi = E;
@@ -181,6 +192,7 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int NT = (N_out + BN_OUT - 1) / BN_OUT;
   const int KB = Kdim / BK;
+  const int KG = (KB + 3) / 4;   // k groups (scale chunks per row block)
   volatile int* abort_flag = &ctl->abort;
 
   if (threadIdx.x == 0) {
@@ -251,10 +263,10 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         int m, n;
         const int e = decode_tile(tile, NT, P, E, m, n);
         const int a_row = row_off[e] + m * BM;           // a multiple of 128
-        const int b_row0 = e * b_rows_per_expert + n * BN_OUT * (MODE == 0 ? 1 : 1);
-        const uint8_t* sa_rows = sfa + (size_t)(a_row / 128) * KB * SF_CHUNK;
-        const uint8_t* sb0_rows = sfb + (size_t)(b_row0 / 128) * KB * SF_CHUNK;
-        const uint8_t* sb1_rows = sfb + (size_t)((b_row0 + b_second_off) / 128) * KB * SF_CHUNK;
+        const int b_row0 = e * b_rows_per_expert + n * BN_OUT;
+        const uint8_t* sa_rows = sfa + (size_t)(a_row / 128) * KG * SF_CHUNK;
+        const uint8_t* sb0_rows = sfb + (size_t)(b_row0 / 128) * KG * SF_CHUNK;
+        const uint8_t* sb1_rows = sfb + (size_t)((b_row0 + b_second_off) / 128) * KG * SF_CHUNK;
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % STAGES;
@@ -266,13 +278,16 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           const uint32_t sa = base + s * OPER_BYTES;
           const uint32_t ss = sf_smem + s * SF_STAGE;
           const uint32_t fb = saddr(&ctl->full[s]);
-          mbar_expect_tx(fb, OPER_BYTES + SF_STAGE);
+          const int sg = sf_group_of_stage(kb, KG);
+          mbar_expect_tx(fb, OPER_BYTES + (sg >= 0 ? SF_STAGE : 0));
           tma_load_2d<1>(sa, &tmA, kb * BK, a_row, fb);
           tma_load_2d<1>(sa + A_BYTES, &tmB, kb * BK, b_row0, fb);
           tma_load_2d<1>(sa + A_BYTES + B_HALF, &tmB, kb * BK, b_row0 + b_second_off, fb);
-          bulk_load(ss, sa_rows + (size_t)kb * SF_CHUNK, SF_CHUNK, fb);
-          bulk_load(ss + SF_CHUNK, sb0_rows + (size_t)kb * SF_CHUNK, SF_CHUNK, fb);
-          bulk_load(ss + 2 * SF_CHUNK, sb1_rows + (size_t)kb * SF_CHUNK, SF_CHUNK, fb);
+          if (sg >= 0) {
+            bulk_load(ss, sa_rows + (size_t)sg * SF_CHUNK, SF_CHUNK, fb);
+            bulk_load(ss + SF_CHUNK, sb0_rows + (size_t)sg * SF_CHUNK, SF_CHUNK, fb);
+            bulk_load(ss + 2 * SF_CHUNK, sb1_rows + (size_t)sg * SF_CHUNK, SF_CHUNK, fb);
+          }
         }
         if (!ok) break;
       }
@@ -299,16 +314,22 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           tc_fence_after();
           const uint32_t sa = base + s * OPER_BYTES;
           const uint32_t ss = sf_smem + s * SF_STAGE;
-          const uint32_t tsf = tmem + SF_COL0 + (uint32_t)s * SF_COLS;
-          sf_copy(tsf, sf_desc(ss));
-          sf_copy(tsf + 4, sf_desc(ss + SF_CHUNK));
-          sf_copy(tsf + 8, sf_desc(ss + 2 * SF_CHUNK));
+          const int sg = sf_group_of_stage(kb, KG);
+          if (sg >= 0) {   // this stage brought the scales of k group sg
+            const uint32_t slot = tmem + SF_COL0 + (uint32_t)(sg & 1) * SF_COLS;
+            sf_copy(slot, sf_desc(ss));
+            sf_copy(slot + 4, sf_desc(ss + SF_CHUNK));
+            sf_copy(slot + 8, sf_desc(ss + 2 * SF_CHUNK));
+          }
+          const uint32_t cur = tmem + SF_COL0 + (uint32_t)((kb >> 2) & 1) * SF_COLS;
+          const uint32_t sel = (uint32_t)(kb & 3);   // scale byte of this k block
+          const uint32_t idesc = idesc_fp8(sel);
           const uint64_t ad = sw128_desc(sa);
           const uint64_t bd = sw128_desc(sa + A_BYTES);
 #pragma unroll
           for (uint32_t j = 0; j < 4; ++j)
-            mma_fp8(tmem, ad + 2 * j, bd + 2 * j, idesc_fp8(j), tsf | (j << 30),
-                    (tsf + 4) | (j << 30), (kb | (int)j) != 0 ? 1u : 0u);
+            mma_fp8(tmem, ad + 2 * j, bd + 2 * j, idesc, cur | (sel << 30),
+                    (cur + 4) | (sel << 30), (kb | (int)j) != 0 ? 1u : 0u);
           tc_commit<1>(saddr(&ctl->empty[s]));
         }
         if (!ok) break;
@@ -373,9 +394,7 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           o[v].z = fp8x2(hv[8] * inv, hv[9] * inv) | (fp8x2(hv[10] * inv, hv[11] * inv) << 16);
           o[v].w = fp8x2(hv[12] * inv, hv[13] * inv) | (fp8x2(hv[14] * inv, hv[15] * inv) << 16);
         }
-        if (row_ok)
-          *reinterpret_cast<uint32_t*>(out_sf + sf_offset(grow, n, KBo)) =
-              (uint32_t)(p + 127) * 0x01010101u;
+        if (row_ok) out_sf[sf_offset(grow, n, KBo)] = (uint8_t)(p + 127);
         if (staged) {
           if (threadIdx.x == 64) bulk_wait_read_all();   // the previous box has left smem
           epilogue_bar();

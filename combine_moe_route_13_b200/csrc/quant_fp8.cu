@@ -11,7 +11,7 @@
 // vector v = v0 + t (8 bf16); the 16 threads of a half-warp cover one
 // 128-element scale block, whose amax is a 4-step xor-shuffle reduction inside
 // the half-warp. Codes leave as 8-byte stores (coalesced, 1 KB per block
-// iteration); the half-warp's first thread stores the block's four scale bytes.
+// iteration); the half-warp's first thread stores the block's scale byte.
 #include <algorithm>
 
 #include "fp8_util.cuh"
@@ -80,13 +80,12 @@ quant_rows_kernel(const uint4* __restrict__ src, int row_vecs, int KB,
     uint2 c;
     c.x = fp8x2(f[0] * inv, f[1] * inv) | (fp8x2(f[2] * inv, f[3] * inv) << 16);
     c.y = fp8x2(f[4] * inv, f[5] * inv) | (fp8x2(f[6] * inv, f[7] * inv) << 16);
-    const uint32_t sbytes = (uint32_t)(p + 127) * 0x01010101u;
+    const uint8_t sbyte = (uint8_t)(p + 127);
     const int kb = v / 16;
     for (int d = 0; d < nd; ++d) {
       const int64_t r = DISPATCH ? (int64_t)s_dst[d] : row;
       *reinterpret_cast<uint2*>(q + r * H + (int64_t)v * 8) = c;
-      if ((threadIdx.x & 15) == 0)
-        *reinterpret_cast<uint32_t*>(sf + sf_offset(r, kb, KB)) = sbytes;
+      if ((threadIdx.x & 15) == 0) sf[sf_offset(r, kb, KB)] = sbyte;
     }
   }
 }

@@ -303,16 +303,17 @@ moe_status_t moe_layer_forward_x(const moe_config_t* cfg, const void* x, const v
  * consecutive elements of a row along the contraction dimension; the scale is a
  * power of two 2^p stored as the byte p + 127 (UE8M0), p the smallest integer
  * >= -127 with max|block| <= 448 * 2^p.
- * Scale layout (what the tensor cores read): for each block of 128 rows and each
- * 128-element k block, a 512-byte chunk at ((r / 128) * (cols / 128) + kb) * 512;
- * row r owns bytes 16*(r % 32) + 4*((r % 128) / 32) + {0,1,2,3} of it, all four
- * holding its scale byte. A [rows, cols] matrix has moe_fp8_scale_bytes(rows, cols)
- * bytes of scales; bytes of rows past `rows` are never written.
+ * Scale layout (what the tensor cores read): with KG = ceil(cols / 512), for each
+ * block of 128 rows and each group of four 128-element k blocks a 512-byte chunk
+ * at ((r / 128) * KG + kb / 4) * 512; row r's scale for k block kb is byte
+ * 16*(r % 32) + 4*((r % 128) / 32) + kb % 4 of it. A [rows, cols] matrix has
+ * moe_fp8_scale_bytes(rows, cols) bytes of scales; bytes of rows (or k blocks)
+ * past the matrix are never written.
  * The whole fp8 path requires bf16 activations, H % 256 == 0, F % 128 == 0,
  * row_align % 128 == 0, n_shared == 0 and E <= 512 (else MOE_ERR_UNSUPPORTED).
  * ------------------------------------------------------------------------- */
 
-/* ceil(rows / 128) * (cols / 128) * 512, or -1 if rows < 0 or cols is not a
+/* ceil(rows / 128) * ceil(cols / 512) * 512, or -1 if rows < 0 or cols is not a
  * positive multiple of 128. */
 int64_t moe_fp8_scale_bytes(int64_t rows, int64_t cols);
 

@@ -108,43 +108,36 @@ def dequantize_rows(codes: np.ndarray, p: np.ndarray) -> np.ndarray:
 
 
 def _scale_positions(rows: int, KB: int) -> np.ndarray:
-    """Byte offset of the first of the four copies of scale (r, kb): [rows, KB]."""
+    """Byte offset of scale (r, kb): [rows, KB]."""
+    KG = -(-KB // 4)
     r = np.arange(rows, dtype=np.int64)[:, None]
     kb = np.arange(KB, dtype=np.int64)[None, :]
-    return ((r // 128) * KB + kb) * 512 + 16 * (r % 32) + 4 * ((r % 128) // 32)
+    return ((r // 128) * KG + kb // 4) * 512 + 16 * (r % 32) + 4 * ((r % 128) // 32) + kb % 4
 
 
 def scales_blocked(p: np.ndarray, row_blocks: int | None = None, pad: int | None = None) -> np.ndarray:
     """The scale bytes (p + 127) in the byte layout the library's kernels read.
 
-    For each block of 128 rows rb and each 128-element k block kb there is a
-    512-byte chunk at offset (rb * KB + kb) * 512; row r = 128*rb + 32*j + i
-    (i < 32, j < 4) owns bytes 16*i + 4*j + s for s = 0..3, all four holding
-    its scale byte (the tensor cores read one scale per 32 elements; a 1 x 128
-    block's scale is repeated for its four 32-element parts).  Rows past the
-    matrix get the byte `pad` (None leaves them 0).  This is an interface layout
-    of the library, written out here so that the kernels' scale output can be
-    compared byte for byte."""
+    With KG = ceil(KB / 4), for each block of 128 rows rb and each group of
+    four 128-element k blocks g there is a 512-byte chunk at offset
+    (rb * KG + g) * 512; the scale of row r = 128*rb + 32*j + i (i < 32,
+    j < 4) for k block kb = 4*g + s is byte 16*i + 4*j + s of it (the position
+    the tensor cores read it from after copying the chunk into tensor memory).
+    Bytes of rows or k blocks past the matrix get `pad` (None leaves them 0).
+    This is an interface layout of the library, written out here so that the
+    kernels' scale output can be compared byte for byte."""
     p = np.asarray(p, dtype=np.int64)
     rows, KB = p.shape
     RB = -(-rows // 128) if row_blocks is None else row_blocks
-    out = np.full(RB * KB * 512, 0 if pad is None else pad, dtype=np.uint8)
-    pos = _scale_positions(rows, KB)
-    for s in range(4):
-        out[pos + s] = (p + 127).astype(np.uint8)
+    out = np.full(RB * (-(-KB // 4)) * 512, 0 if pad is None else pad, dtype=np.uint8)
+    out[_scale_positions(rows, KB)] = (p + 127).astype(np.uint8)
     return out
 
 
 def scales_from_blocked(buf: np.ndarray, rows: int, KB: int) -> np.ndarray:
-    """Inverse of scales_blocked for the first `rows` rows: p [rows, KB].
-    Raises if a row's four copies of a scale disagree."""
+    """Inverse of scales_blocked for the first `rows` rows: p [rows, KB]."""
     buf = np.asarray(buf, dtype=np.uint8)
-    pos = _scale_positions(rows, KB)
-    q = np.stack([buf[pos + s] for s in range(4)])
-    if not np.all(q == q[0]):
-        bad = np.argwhere(np.any(q != q[0], axis=0))[0]
-        raise ValueError(f"row {bad[0]} block {bad[1]}: scale copies differ {q[:, bad[0], bad[1]].tolist()}")
-    return q[0].astype(np.int64) - 127
+    return buf[_scale_positions(rows, KB)].astype(np.int64) - 127
 
 
 def dispatch_fp8(x_bf16: np.ndarray, token_slot: np.ndarray, R_max: int):

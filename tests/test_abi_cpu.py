@@ -172,8 +172,9 @@ def test_status_strings():
 
 def test_fp8_scale_bytes():
     assert M.moe_fp8_scale_bytes(1, 128) == 512
-    assert M.moe_fp8_scale_bytes(128, 256) == 1024
-    assert M.moe_fp8_scale_bytes(129, 7168) == 2 * 56 * 512
+    assert M.moe_fp8_scale_bytes(128, 512) == 512
+    assert M.moe_fp8_scale_bytes(128, 640) == 1024
+    assert M.moe_fp8_scale_bytes(129, 7168) == 2 * 14 * 512
     assert M.moe_fp8_scale_bytes(0, 128) == 0
     assert M.moe_fp8_scale_bytes(10, 100) == -1 and M.moe_fp8_scale_bytes(-1, 128) == -1
 

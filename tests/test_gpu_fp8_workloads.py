@@ -31,7 +31,7 @@ def _expert_scales(buf, e, rows_per_expert, cols):
     """Scale exponents of expert e's rows of a weight matrix quantised as
     [E * rows_per_expert, cols] (its row blocks are contiguous chunks)."""
     KB = cols // 128
-    per = rows_per_expert // 128 * KB * 512
+    per = rows_per_expert // 128 * (-(-KB // 4)) * 512   # the expert's chunks are contiguous
     return Q.scales_from_blocked(np_u8(buf[e * per:(e + 1) * per]), rows_per_expert, KB)
 
 

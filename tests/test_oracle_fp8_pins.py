@@ -100,16 +100,16 @@ def test_quantize_matches_torch_conversion():
 
 
 def test_scale_layout_by_independent_inversion():
-    rows, KB = 300, 3
+    rows, KB = 300, 6
     p = np.arange(rows * KB, dtype=np.int64).reshape(rows, KB) % 200 - 100
     buf = Q.scales_blocked(p, pad=127)
-    assert buf.size == 3 * KB * 512
+    assert buf.size == 3 * 2 * 512
     # walk the bytes and invert the position formula independently
     for off in range(buf.size):
         chunk, o = divmod(off, 512)
-        rb, kb = divmod(chunk, KB)
-        row = 128 * rb + 32 * ((o % 16) // 4) + o // 16
-        want = p[row, kb] + 127 if row < rows else 127
+        rb, g = divmod(chunk, 2)
+        row, kb = 128 * rb + 32 * ((o % 16) // 4) + o // 16, 4 * g + o % 4
+        want = p[row, kb] + 127 if row < rows and kb < KB else 127
         assert buf[off] == want, (off, row, kb)
     assert np.array_equal(Q.scales_from_blocked(buf, rows, KB), p)
 
