@@ -125,6 +125,10 @@ MLP_CASES = [
     (600, 256, 8, 2, 384, 8, 2.0, "zipf"),        # empty experts
     (128, 256, 64, 8, 128, 8, 2.0, "normal"),     # many tiny experts
     (1200, 1024, 8, 2, 1024, 2, 1.25, "normal"),  # several M and N tiles per expert
+    # >= 192 rows per expert: many full 128-row tiles per expert
+    (2048, 256, 4, 2, 256, 2, 1.25, "normal"),    # ragged last tile per expert
+    (1500, 512, 6, 2, 384, 3, 1.0, "zipf"),       # skewed experts, some at capacity
+    (3000, 256, 12, 2, 256, 4, 2.0, "hot"),       # one hot expert over many tiles
 ]
 
 
@@ -166,6 +170,7 @@ def test_expert_mlp_fp8(cuda_ok, T, H, E, K, F, S, cf, kind):
     W.small_case(512, 256, 8, 2, 256, 2, 1.25, "bf16", 128),
     W.small_case(700, 512, 12, 3, 384, 4, 0.8, "bf16", 128, bias="zipf1.2"),
     W.small_case(200, 256, 8, 2, 128, 2, 0.0, "bf16", 128),          # C = 0: nothing kept
+    W.small_case(1024, 512, 4, 2, 256, 2, 1.25, "bf16", 128),        # 512 rows per expert
 ], ids=lambda w: w.name)
 def test_layer_forward_fp8(cuda_ok, wl):
     C = O.capacity(wl.T, wl.K, wl.E, wl.cf)
