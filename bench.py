@@ -328,7 +328,8 @@ def algorithmic(layer: Layer, totals, counts):
         "dispatch_bytes": (T * H * s + (N + Ns) * H * (1 + 4 / 128) + T * K * 4) if layer.fp8
         else (T + N + Ns) * H * s + T * K * 4,
         "combine_bytes": (N + Ns + T) * H * s + T * K * 8,
-        "route_bytes": T * E * 4 + T * K * 12,
+        # logits read; topk_idx, topk_w, token_slot written; row_src; per-expert tables
+        "route_bytes": T * E * 4 + T * K * 12 + int(totals[3]) * 4 + E * 12,
     }
 
 
@@ -494,7 +495,11 @@ def main(argv=None):
     hbm_bound = alg["mlp_bytes"] / (hbm * 1e9) > alg["mlp_flops"] / (tensor_peak * 1e12)
     kernels = {
         "router_us": ph["router"] * 1e3 if args.router else None,
+        "phase_timing": "CUDA events between the piecewise entry points on the launching "
+                        "stream, L2 flushed first; each phase includes its launch gap "
+                        "(kernel-only ncu times: profiles/)",
         "route_us": ph["route"] * 1e3,
+        "route_gbs": alg["route_bytes"] / (ph["route"] * 1e-3) / 1e9,
         "dispatch_us": ph["dispatch"] * 1e3,
         "dispatch_gbs": alg["dispatch_bytes"] / (ph["dispatch"] * 1e-3) / 1e9,
         "expert_mlp_us": ph["expert_mlp"] * 1e3,
