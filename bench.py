@@ -338,6 +338,7 @@ def cpu_oracle_sample(wl: W.Workload, tokens: int, seed: int, inp_host=None):
     (capacity scaled to that batch). Returns (seconds, tokens)."""
     from oracle import moe_oracle as O
     import torch as _t
+    tokens = min(tokens, wl.T)
     if inp_host is None:
         inp_host = W.make_inputs(wl, seed=seed, device="cpu")
 
@@ -360,6 +361,7 @@ def cpu_oracle_sample_fp8(wl: W.Workload, tokens: int, layer: "Layer"):
     with the oracle's). Returns (seconds, tokens)."""
     from oracle import moe_oracle as O
     from oracle import moe_oracle_fp8 as Q
+    tokens = min(tokens, wl.T)
     E, F, H = wl.E, wl.F, wl.H
     gq, gs, dq, ds = (t.cpu().numpy() for t in layer.wq)
     ge = Q.scales_from_blocked(gs, E * 2 * F, H // 128).reshape(E, 2 * F, H // 128)
@@ -382,26 +384,42 @@ def cpu_cores():
         return len(os.sched_getaffinity(0))
 
 
+REFERENCE_BUDGET_S = 120.0   # timed CPU work of the reference arm, at most
+
+
 def run_reference(args, wl: W.Workload, world, rank):
+    """The CPU oracle, timed. One oracle call on the first `cpu_tokens` tokens is
+    one step. Most of a call's cost is fixed (every expert's weights are widened
+    to float64), so no sample size keeps hundreds of steps within minutes: the
+    arm runs the requested warm-ups within 20 s (at least one), then times
+    steps until it has done the requested number or spent REFERENCE_BUDGET_S,
+    and reports the numbers it ran."""
     if rank != 0:
         return 0
-    tokens = args.cpu_tokens
+    tokens = min(args.cpu_tokens, wl.T)
     inp_host = W.make_inputs(wl, seed=0, device="cpu")
-    for _ in range(args.warmup):
-        cpu_oracle_sample(wl, tokens, 0, inp_host)
-    secs = [cpu_oracle_sample(wl, tokens, 0, inp_host)[0] for _ in range(args.steps)]
+    warm, t_warm = 0, 0.0   # the requested warm-ups, within 20 s (at least one)
+    while warm < args.warmup and (warm == 0 or t_warm < 20.0):
+        t_warm += cpu_oracle_sample(wl, tokens, 0, inp_host)[0]
+        warm += 1
+    secs = []
+    while len(secs) < args.steps and (not secs or sum(secs) < REFERENCE_BUDGET_S):
+        secs.append(cpu_oracle_sample(wl, tokens, 0, inp_host)[0])
     ms = float(np.mean(secs)) * 1e3
     value = tokens / (ms / 1e3)
     cores = cpu_cores()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "n_gpus": world, "steps": len(secs), "warmup": warm, "ms_per_step": ms,
+        "requested_steps": args.steps, "requested_warmup": args.warmup,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.act,
         "data": "synthetic", "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E,
                                         "K": wl.K, "F": wl.F, "S": wl.S, "cf": wl.cf},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": f"whole layer (float64 numpy oracle) on the first {tokens} "
-                                   f"tokens of the workload per step, capacity scaled to that batch"},
+                                   f"tokens of the workload per step, capacity scaled to that "
+                                   f"batch; {len(secs)} timed steps (at most the requested "
+                                   f"number, stopped after {REFERENCE_BUDGET_S:.0f} s of timed work)"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -411,11 +429,11 @@ def run_reference(args, wl: W.Workload, world, rank):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mixtral", choices=sorted(W.WORKLOADS))
-    ap.add_argument("--cpu-tokens", type=int, default=256,
+    ap.add_argument("--cpu-tokens", type=int, default=512,
                     help="tokens of the CPU-oracle sample per step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--router", action="store_true",
@@ -522,14 +540,16 @@ def main(argv=None):
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        if args.fp8:
-            secs, tok = cpu_oracle_sample_fp8(wl, args.cpu_tokens, layer)
-        else:
-            secs, tok = cpu_oracle_sample(wl, args.cpu_tokens, 0)
+        # two samples (about 10-30 s of oracle work on the Mixtral shape), on
+        # this replica's own inputs copied to the host once
+        host = None if args.fp8 else {k: layer.inp[k].cpu() for k in ("logits", "x", "w_gu", "w_d")}
+        runs = [cpu_oracle_sample_fp8(wl, args.cpu_tokens, layer) if args.fp8
+                else cpu_oracle_sample(wl, args.cpu_tokens, 0, host) for _ in range(2)]
+        secs, tok = sum(r[0] for r in runs), sum(r[1] for r in runs)
         cpu = {"value": tok / secs, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
-               "sample": f"whole layer ({'fp8 ' if args.fp8 else ''}float64 numpy oracle) on the "
-                         f"first {tok} tokens of the workload, capacity scaled to that batch; "
-                         f"{secs:.1f} s"}
+               "sample": f"whole layer ({'fp8 ' if args.fp8 else ''}float64 numpy oracle), two "
+                         f"calls, each on the first {args.cpu_tokens} tokens of the workload "
+                         f"with capacity scaled to that batch; {secs:.1f} s in total"}
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
