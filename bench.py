@@ -190,20 +190,21 @@ class Layer:
         self.out = torch.empty(wl.T, wl.H, dtype=wl.torch_act, device=device)
         self.aux = None
 
-    def forward(self, x=None, logits=None):
+    def forward(self, x=None, logits=None, out=None):
         x = self.inp["x"] if x is None else x
+        out = self.out if out is None else out
         if self.fp8:
             logits = self.inp["logits"] if logits is None else logits
-            self.aux = self.M.moe_layer_forward_fp8(self.cfg, logits, x, *self.wq, self.out, self.ws)
+            self.aux = self.M.moe_layer_forward_fp8(self.cfg, logits, x, *self.wq, out, self.ws)
         elif self.router:   # from hidden states: router projection + selection-only bias
             self.aux = self.M.moe_layer_forward_x(self.cfg, x, self.inp["w_g"],
                                                   self.inp["sel_bias"], self.inp["w_gu"],
-                                                  self.inp["w_d"], self.out, self.ws,
+                                                  self.inp["w_d"], out, self.ws,
                                                   flags=self.flags)
         else:
             logits = self.inp["logits"] if logits is None else logits
             self.aux = self.M.moe_layer_forward(self.cfg, logits, x, self.inp["w_gu"],
-                                                self.inp["w_d"], self.out, self.ws,
+                                                self.inp["w_d"], out, self.ws,
                                                 flags=self.flags)
 
     def views(self):
@@ -289,6 +290,60 @@ def e2e_steps(layer: Layer, steps, warmup, flush_buf, stream):
     h2d = (0 if layer.router else h_logits.numel() * 4) + h_x.numel() * h_x.element_size()
     d2h = h_out.numel() * h_out.element_size()
     return times, h2d, d2h
+
+
+def e2e_pipelined(layer: Layer, steps, warmup, flush_buf, stream):
+    """The same C call with host copies, as a serving loop runs it: each step
+    copies its inputs from pinned host memory and its output back, but on their
+    own streams into / out of one of two device buffers, so step i+1's input
+    copy and step i-1's output copy overlap step i's layer (events order every
+    buffer's reuse). L2 is flushed on the compute stream before every layer.
+    Returns the device time of the `steps` timed steps (ms), first input copy
+    to last output copy."""
+    inp = layer.inp
+    h_logits = inp["logits"].cpu().pin_memory()
+    h_x = inp["x"].cpu().pin_memory()
+    h_out = [torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory() for _ in range(2)]
+    d_logits = [torch.empty_like(inp["logits"]) for _ in range(2)]
+    d_x = [torch.empty_like(inp["x"]) for _ in range(2)]
+    d_out = [torch.empty_like(layer.out) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    for b in range(2):
+        ev_done[b].record(stream)
+        ev_out[b].record(stream)
+
+    def run(n):
+        for i in range(n):
+            b = i % 2
+            s_in.wait_event(ev_done[b])          # the layer two steps back has read d_x[b]
+            with torch.cuda.stream(s_in):
+                if not layer.router:
+                    d_logits[b].copy_(h_logits, non_blocking=True)
+                d_x[b].copy_(h_x, non_blocking=True)
+            ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            stream.wait_event(ev_out[b])         # d_out[b] from two steps back is on the host
+            flush_buf.add_(1.0)
+            layer.forward(x=d_x[b], logits=d_logits[b], out=d_out[b])
+            ev_done[b].record(stream)
+            s_out.wait_event(ev_done[b])
+            with torch.cuda.stream(s_out):
+                h_out[b].copy_(d_out[b], non_blocking=True)
+            ev_out[b].record(s_out)
+
+    run(warmup)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    s_in.wait_event(start)
+    run(steps)
+    stream.wait_event(ev_out[(steps - 1) % 2])
+    end.record(stream)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end)
 
 
 def mlp_tile_rows(layer: Layer) -> int:
@@ -494,7 +549,9 @@ def main(argv=None):
     value = world * wl.T / (ms / 1e3)
 
     e2e_t, h2d, d2h = e2e_steps(layer, args.steps, args.warmup, flush_buf, stream)
-    e2e_ms = max_over_ranks(float(np.sum(e2e_t)), world, device) / args.steps
+    e2e_serial_ms = max_over_ranks(float(np.sum(e2e_t)), world, device) / args.steps
+    e2e_ms = max_over_ranks(e2e_pipelined(layer, args.steps, args.warmup, flush_buf, stream),
+                            world, device) / args.steps
 
     ph = phase_times(layer, max(args.steps // 2, 3), flush_buf, stream)
     st = layer.M.moe_get_device_status(layer.ws)
@@ -564,7 +621,13 @@ def main(argv=None):
                    "n_shared": wl.n_shared,
                    "payload": "e4m3, 1x128 blocks, UE8M0 scales; bf16 combine" if args.fp8 else wl.act},
         "e2e": {"value": world * wl.T / (e2e_ms / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "mode": "pipelined: per-step copies from/to pinned host memory on their own "
+                        "streams and two device buffers, overlapping the neighbouring steps' "
+                        "layer; L2 flushed before every layer",
+                "serial": {"value": world * wl.T / (e2e_serial_ms / 1e3),
+                           "ms_per_step": e2e_serial_ms,
+                           "mode": "copy in, layer, copy out, one after the other"}},
         "gpu_launches": (KERNELS_PER_STEP + (1 if args.router else 0)) * args.steps,
         "roofline": ({"bound": "hbm", "kernel": "expert_mlp (gate/up + down grouped GEMMs)",
                       "achieved": mlp_gbs, "peak": hbm, "unit": "GB/s", "frac": mlp_gbs / hbm,
