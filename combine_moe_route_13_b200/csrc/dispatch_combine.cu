@@ -28,7 +28,7 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) { return __ldcs(p); }
 
 __global__ void __launch_bounds__(DC_THREADS)
 dispatch_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ token_slot,
-                uint4* __restrict__ xp, int K, int row_vecs, long long sh_row0) {
+                uint4* __restrict__ xp, int K, int row_vecs, long long sh_row0, int slot_end) {
   __shared__ int s_slot[MAX_K + 1];
   __shared__ int s_any;
   const int t = blockIdx.x;
@@ -39,7 +39,8 @@ dispatch_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ token_s
   pdl_trigger();
   __syncthreads();
   if (threadIdx.x < K) {
-    const int s = token_slot[(size_t)t * K + threadIdx.x];
+    int s = token_slot[(size_t)t * K + threadIdx.x];
+    if (s >= slot_end) s = -1;   // outside the grouped buffer: treated as dropped
     s_slot[threadIdx.x] = s;
     if (s >= 0) atomicOr(&s_any, 1);
   } else if (threadIdx.x == K && KD > K) {
@@ -138,14 +139,15 @@ template <bool BF16>
 __global__ void __launch_bounds__(DC_THREADS)
 combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ token_slot,
                const float* __restrict__ topk_w, uint4* __restrict__ out, int K, int row_vecs,
-               long long sh_row0) {
+               long long sh_row0, int slot_end) {
   __shared__ int s_slot[MAX_K];
   __shared__ float s_w[MAX_K];
   const int t = blockIdx.x;
   pdl_wait();
   pdl_trigger();
   if (threadIdx.x < K) {
-    s_slot[threadIdx.x] = token_slot[(size_t)t * K + threadIdx.x];
+    const int sl = token_slot[(size_t)t * K + threadIdx.x];
+    s_slot[threadIdx.x] = sl < slot_end ? sl : -1;   // outside the grouped buffer: dropped
     s_w[threadIdx.x] = topk_w[(size_t)t * K + threadIdx.x];
   }
   __syncthreads();
@@ -220,7 +222,8 @@ template <bool BF16>
 __global__ void __launch_bounds__(DC_THREADS)
 combine_wait_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ token_slot,
                     const float* __restrict__ topk_w, uint4* __restrict__ out, int K,
-                    int row_vecs, long long sh_row0, const uint32_t* row_ready, uint32_t target,
+                    int row_vecs, long long sh_row0, int slot_end, const uint32_t* row_ready,
+                    uint32_t target,
                     unsigned long long timeout_ns, uint32_t* status) {
   __shared__ int s_slot[MAX_K + 1];
   __shared__ float s_w[MAX_K];
@@ -229,7 +232,8 @@ combine_wait_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ tok
   const int t = blockIdx.x;
   const int KW = sh_row0 >= 0 ? K + 1 : K;   // rows to wait for, the shared one last
   if (threadIdx.x < K) {
-    s_slot[threadIdx.x] = token_slot[(size_t)t * K + threadIdx.x];
+    const int sl = token_slot[(size_t)t * K + threadIdx.x];
+    s_slot[threadIdx.x] = sl < slot_end ? sl : -1;   // outside the grouped buffer: dropped
     s_w[threadIdx.x] = topk_w[(size_t)t * K + threadIdx.x];
   } else if (threadIdx.x == K && KW > K) {
     s_slot[K] = (int)(sh_row0 + t);
@@ -311,7 +315,7 @@ cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t*
   const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
   return launch_pdl(dispatch_kernel, dim3(c.T), dim3(DC_THREADS), 0, s,
                     static_cast<const uint4*>(x), slot, static_cast<uint4*>(xp), c.K, row_vecs,
-                    (long long)sh_row0);
+                    (long long)sh_row0, (int)routed_rows(c));
 }
 
 cudaError_t launch_combine(const moe_config_t& c, const void* y, const int32_t* slot,
@@ -320,7 +324,8 @@ cudaError_t launch_combine(const moe_config_t& c, const void* y, const int32_t* 
   const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
   auto kernel = c.act_dtype == MOE_BF16 ? combine_kernel<true> : combine_kernel<false>;
   return launch_pdl(kernel, dim3(c.T), dim3(DC_THREADS), 0, s, static_cast<const uint4*>(y), slot,
-                    w, static_cast<uint4*>(out), c.K, row_vecs, (long long)sh_row0);
+                    w, static_cast<uint4*>(out), c.K, row_vecs, (long long)sh_row0,
+                    (int)routed_rows(c));
 }
 
 cudaError_t launch_combine_wait(const moe_config_t& c, const void* y, const int32_t* slot,
@@ -331,7 +336,8 @@ cudaError_t launch_combine_wait(const moe_config_t& c, const void* y, const int3
   const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
   auto kernel = c.act_dtype == MOE_BF16 ? combine_wait_kernel<true> : combine_wait_kernel<false>;
   return launch_pdl(kernel, dim3(c.T), dim3(DC_THREADS), 0, s, static_cast<const uint4*>(y), slot,
-                    w, static_cast<uint4*>(out), c.K, row_vecs, (long long)sh_row0, row_ready,
+                    w, static_cast<uint4*>(out), c.K, row_vecs, (long long)sh_row0,
+                    (int)routed_rows(c), row_ready,
                     target, timeout_ns, status);
 }
 

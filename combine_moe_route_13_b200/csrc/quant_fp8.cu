@@ -37,7 +37,7 @@ template <bool DISPATCH>
 __global__ void __launch_bounds__(QT)
 quant_rows_kernel(const uint4* __restrict__ src, int row_vecs, int KB,
                   const int32_t* __restrict__ token_slot, int K, uint8_t* __restrict__ q,
-                  uint8_t* __restrict__ sf) {
+                  uint8_t* __restrict__ sf, int slot_end) {
   __shared__ int s_dst[MAX_K];
   __shared__ int s_n;
   const int64_t row = blockIdx.x;
@@ -48,7 +48,7 @@ quant_rows_kernel(const uint4* __restrict__ src, int row_vecs, int KB,
       int n = 0;
       for (int k = 0; k < K; ++k) {
         const int s = token_slot[row * K + k];
-        if (s >= 0) s_dst[n++] = s;
+        if (s >= 0 && s < slot_end) s_dst[n++] = s;   // others are dropped
       }
       s_n = n;
     }
@@ -97,14 +97,15 @@ cudaError_t launch_quantize_fp8(const void* src, int64_t rows, int64_t cols, uin
   if (rows == 0) return cudaSuccess;
   return launch_pdl(quant_rows_kernel<false>, dim3((unsigned)rows), dim3(QT), 0, s,
                     static_cast<const uint4*>(src), (int)(cols / 8), (int)(cols / FP8_BLOCK),
-                    (const int32_t*)nullptr, 0, q, sf);
+                    (const int32_t*)nullptr, 0, q, sf, 0);
 }
 
 cudaError_t launch_dispatch_fp8(const moe_config_t& c, const void* x, const int32_t* slot,
                                 uint8_t* xq, uint8_t* xs, cudaStream_t s) {
   if (c.T == 0) return cudaSuccess;
   return launch_pdl(quant_rows_kernel<true>, dim3(c.T), dim3(QT), 0, s,
-                    static_cast<const uint4*>(x), c.H / 8, c.H / FP8_BLOCK, slot, c.K, xq, xs);
+                    static_cast<const uint4*>(x), c.H / 8, c.H / FP8_BLOCK, slot, c.K, xq, xs,
+                    (int)routed_rows(c));
 }
 
 }  // namespace moe

@@ -33,6 +33,10 @@
  *     read with moe_get_device_status.
  *   - Shapes the kernels do not support return MOE_ERR_UNSUPPORTED; nothing is
  *     ever computed another way.
+ *   - token_slot tables passed by the caller (moe_dispatch, moe_dispatch_fp8,
+ *     moe_combine, moe_combine_wait): an entry that is negative or not below the
+ *     routed rows min(T*K, E*C) + E*(A-1) is treated as a dropped assignment;
+ *     nothing is written or read for it.
  *
  * Symbols: T tokens, H hidden size, E experts, K experts per token, F SwiGLU
  * width, S owner segments, C capacity per expert, A row alignment, R_max rows

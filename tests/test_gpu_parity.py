@@ -247,3 +247,63 @@ def test_empty_batch(cuda_ok):
     assert v["totals"].cpu().tolist() == [0, 0, 0, 0]
     assert torch.all(v["expert_counts"] == 0)
     assert torch.all(v["row_src"] == -1)
+
+
+def test_out_of_range_slots_are_treated_as_dropped(cuda_ok):
+    # caller-supplied tables: entries beyond the routed rows (or below -1) must
+    # not be written or read; the kernels treat them as dropped assignments
+    T, H, E, K, S, A = 300, 256, 8, 2, 2, 8
+    C = O.capacity(T, K, E, 1.0)
+    cfg = cfg_for(T, H, E, K, 64, S, C, A, "bf16")
+    r = run_route(cfg, logits_for(T, E, "normal", 21).to(DEV))
+    R = M.moe_max_rows(cfg)
+    slot = r["token_slot"].clone()
+    bad = torch.zeros_like(slot, dtype=torch.bool)
+    bad[::7, 0] = True
+    slot[bad] = torch.tensor([R, R + 5, 1 << 30, -7], dtype=torch.int32,
+                             device=DEV).repeat(int(bad.sum()) // 4 + 1)[:int(bad.sum())]
+    x = torch.randn(T, H, generator=torch.Generator().manual_seed(6)).to(torch.bfloat16).to(DEV)
+    guard = 64
+    xp_full = torch.full((R + guard, H), 3, dtype=torch.bfloat16, device=DEV)
+    M.moe_dispatch(cfg, x, slot, xp_full[:R])
+    torch.cuda.synchronize()
+    assert torch.all(xp_full[R:] == 3)                         # nothing past the buffer
+    ref_slot = slot.cpu().numpy().copy()
+    ref_slot[(ref_slot < 0) | (ref_slot >= R)] = -1
+    ref = O.dispatch(act_np(x), ref_slot, R)
+    kept = np.zeros(R, bool)
+    kept[ref_slot[ref_slot >= 0]] = True
+    assert np.array_equal(act_np(xp_full[:R])[kept], ref[kept])
+    y = torch.randn(R, H, generator=torch.Generator().manual_seed(7)).to(torch.bfloat16).to(DEV)
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=DEV)
+    M.moe_combine(cfg, y, slot, r["topk_w"], out)
+    torch.cuda.synchronize()
+    ref_out = O.combine(act_np(y), ref_slot, r["topk_w"].cpu().numpy(), O.ACT_BF16)
+    assert_close_act(act_np(out), ref_out, O.ACT_BF16, "combine with dropped entries")
+
+
+def _random_route_cases(n, seed):
+    rng = np.random.default_rng(seed)
+    cases = []
+    for _ in range(n):
+        E = int(rng.choice([1, 2, 3, 8, 16, 40, 64, 96, 256, 384, 1024]))
+        K = int(rng.integers(1, min(E, 32) + 1))
+        divisors = [d for d in (1, 2, 3, 4, 8, 16) if E % d == 0]
+        S = int(rng.choice(divisors))
+        T = int(rng.choice([0, 1, 7, 127, 128, 129, 500, 1000, 3001]))
+        A = int(rng.choice([1, 2, 8, 16, 128]))
+        cf = float(rng.choice([-1.0, 0.0, 0.3, 0.75, 1.0, 1.25, 2.0]))
+        kind = str(rng.choice(["normal", "zipf", "hot", "tied"]))
+        cases.append((T, E, K, S, cf, A, kind))
+    return cases
+
+
+@pytest.mark.parametrize("T,E,K,S,cf,A,kind", _random_route_cases(40, 2024))
+def test_route_random_sweep(cuda_ok, T, E, K, S, cf, A, kind):
+    # seeded random sweep over (T, E, K, S, A, cf, logit kind), overflow and cf -> 0 included
+    C = O.capacity(T, K, E, cf)
+    lg = logits_for(T, E, kind, T * 3 + E * 5 + K)
+    cfg = cfg_for(T, 64, E, K, 64, S, C, A, "bf16")
+    gpu = host(run_route(cfg, lg.to(DEV)))
+    ref = O.route(lg.numpy(), K, C, A, S)
+    assert_route_equal(gpu, ref, ref["R_max"])
