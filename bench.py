@@ -256,12 +256,15 @@ def phase_times(layer: Layer, steps, flush_buf, stream):
         lambda: M.moe_combine(cfg, v["y"], v["token_slot"], v["topk_w"], layer.out),
     )
     acc = {n: [] for n in names}
+    nvtx = torch.cuda.nvtx   # host ranges per phase, for nsys-style timelines
     for _ in range(steps + 1):
         flush_l2(flush_buf)
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
         ev[0].record(stream)
         for i, c in enumerate(calls):
+            nvtx.range_push(names[i])
             c()
+            nvtx.range_pop()
             ev[i + 1].record(stream)
         torch.cuda.synchronize()
         for i, n in enumerate(names):

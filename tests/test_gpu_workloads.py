@@ -100,3 +100,31 @@ def test_workload_full_size(cuda_ok, name, n_shared):
     assert_close_act(got, ref_out, wl.act, "out")
     del inp, ws, out
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("mode", ["bf16", "bf16_overlap", "fp8"])
+def test_layer_is_deterministic_run_to_run(cuda_ok, mode):
+    # no atomics on any output path: two runs of the whole layer on the same
+    # inputs give the same bits (catches races in the scans, scatter and tiles)
+    wl = W.WORKLOADS["skewed"]
+    dev = torch.device("cuda")
+    C = M.moe_capacity(wl.T, wl.K, wl.E, wl.cf)
+    cfg = M.make_config(wl.T, wl.H, wl.E, wl.K, wl.F, wl.S, C, wl.row_align, wl.act)
+    inp = W.make_inputs(wl, seed=3, device=dev)
+    ws = M.alloc_workspace(M.moe_workspace_bytes(cfg), dev)
+    outs = []
+    if mode == "fp8":
+        gq, gs = M.quantize_fp8(inp["w_gu"])
+        dq, ds = M.quantize_fp8(inp["w_d"])
+    for _ in range(2):
+        out = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device=dev)
+        ws.zero_()
+        if mode == "fp8":
+            M.moe_layer_forward_fp8(cfg, inp["logits"], inp["x"], gq, gs, dq, ds, out, ws)
+        else:
+            flags = M.MOE_FLAG_OVERLAP if mode == "bf16_overlap" else M.MOE_FLAG_NONE
+            M.moe_layer_forward(cfg, inp["logits"], inp["x"], inp["w_gu"], inp["w_d"], out, ws,
+                                flags=flags)
+        assert M.moe_get_device_status(ws) == M.MOE_OK
+        outs.append(out.view(torch.int16).clone())
+    assert torch.equal(outs[0], outs[1])
