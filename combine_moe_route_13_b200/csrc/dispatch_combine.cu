@@ -134,7 +134,9 @@ __device__ __forceinline__ void store_acc(uint4* dst, int v0, int row_vecs, cons
 }
 
 // out[t] = sum_k w[t,k] * y[slot[t,k]] with fp32 accumulation in k order,
-// plus y[sh_row0 + t] when sh_row0 >= 0 (the shared expert).
+// plus y[sh_row0 + t] when sh_row0 >= 0 (the shared expert). Warp 0 first packs
+// the token's kept assignments (in k order), so the gather loops over kept rows
+// only: with heavy overflow most of a token's K slots are dropped.
 template <bool BF16>
 __global__ void __launch_bounds__(DC_THREADS)
 combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ token_slot,
@@ -142,15 +144,28 @@ combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ token_sl
                long long sh_row0, int slot_end) {
   __shared__ int s_slot[MAX_K];
   __shared__ float s_w[MAX_K];
+  __shared__ int s_n;
   const int t = blockIdx.x;
   pdl_wait();
   pdl_trigger();
-  if (threadIdx.x < K) {
-    const int sl = token_slot[(size_t)t * K + threadIdx.x];
-    s_slot[threadIdx.x] = sl < slot_end ? sl : -1;   // outside the grouped buffer: dropped
-    s_w[threadIdx.x] = topk_w[(size_t)t * K + threadIdx.x];
+  if (threadIdx.x < 32) {   // warp 0 packs the kept assignments, in k order
+    int sl = -1;
+    float wt = 0.f;
+    if ((int)threadIdx.x < K) {
+      sl = token_slot[(size_t)t * K + threadIdx.x];
+      wt = topk_w[(size_t)t * K + threadIdx.x];
+    }
+    const bool keep = sl >= 0 && sl < slot_end;   // outside the grouped buffer: dropped
+    const unsigned m = __ballot_sync(0xffffffffu, keep);
+    if (keep) {
+      const int pos = __popc(m & ((1u << threadIdx.x) - 1u));
+      s_slot[pos] = sl;
+      s_w[pos] = wt;
+    }
+    if (threadIdx.x == 0) s_n = __popc(m);
   }
   __syncthreads();
+  K = s_n;   // from here on: the kept rows only
   constexpr int LANES = BF16 ? 8 : 4;
   uint4* dst = out + (size_t)t * row_vecs;
   for (int v0 = threadIdx.x; v0 < row_vecs; v0 += DC_THREADS * 2) {
