@@ -242,18 +242,31 @@ combine_wait_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ tok
                     unsigned long long timeout_ns, uint32_t* status) {
   __shared__ int s_slot[MAX_K + 1];
   __shared__ float s_w[MAX_K];
-  __shared__ int s_ok;
+  __shared__ int s_ok, s_n;
   pdl_trigger();   // no griddepcontrol.wait: the ready counters carry the dependency
   const int t = blockIdx.x;
-  const int KW = sh_row0 >= 0 ? K + 1 : K;   // rows to wait for, the shared one last
-  if (threadIdx.x < K) {
-    const int sl = token_slot[(size_t)t * K + threadIdx.x];
-    s_slot[threadIdx.x] = sl < slot_end ? sl : -1;   // outside the grouped buffer: dropped
-    s_w[threadIdx.x] = topk_w[(size_t)t * K + threadIdx.x];
-  } else if (threadIdx.x == K && KW > K) {
-    s_slot[K] = (int)(sh_row0 + t);
+  if (threadIdx.x < 32) {   // warp 0 packs the kept assignments (k order), shared row last
+    int sl = -1;
+    float wt = 0.f;
+    if ((int)threadIdx.x < K) {
+      sl = token_slot[(size_t)t * K + threadIdx.x];
+      wt = topk_w[(size_t)t * K + threadIdx.x];
+    }
+    const bool keep = sl >= 0 && sl < slot_end;   // outside the grouped buffer: dropped
+    const unsigned m = __ballot_sync(0xffffffffu, keep);
+    if (keep) {
+      const int pos = __popc(m & ((1u << threadIdx.x) - 1u));
+      s_slot[pos] = sl;
+      s_w[pos] = wt;
+    }
+    if (threadIdx.x == 0) {
+      s_n = __popc(m);
+      if (sh_row0 >= 0) s_slot[s_n] = (int)(sh_row0 + t);
+    }
   }
   __syncthreads();
+  K = s_n;                                   // from here on: the kept rows only
+  const int KW = sh_row0 >= 0 ? K + 1 : K;   // rows to wait for, the shared one last
   if (threadIdx.x == 0) {
     int ok = 1;
     const unsigned long long t0 = globaltimer();
