@@ -178,14 +178,18 @@ def down_fp8_rows(hq, h_exp, wq_d_e, wd_exp_e):
     return O.f64_to_bf16_bits(dequantize_rows(hq, h_exp) @ dequantize_rows(wq_d_e, wd_exp_e).T)
 
 
-def layer_forward_fp8(logits, x_bf16, wq_gu, wgu_exp, wq_d, wd_exp, K, C, A, S):
+def layer_forward_fp8(logits, x_bf16, wq_gu, wgu_exp, wq_d, wd_exp, K, C, A, S, n_shared=0):
     """route -> fp8 dispatch -> fp8 expert MLP -> bf16 combine.
-    wq_gu [E,2F,H] codes with wgu_exp [E,2F,H/128]; wq_d [E,H,F] with wd_exp [E,H,F/128].
+    wq_gu [E',2F,H] codes with wgu_exp [E',2F,H/128]; wq_d [E',H,F] with
+    wd_exp [E',H,F/128], E' = E + n_shared.  With n_shared = 1 the last expert is
+    the shared expert: every token's quantised row goes through it and its bf16
+    output is added with weight 1 (the combine of the bf16 layer).
     Returns (out bf16 bits [T,H], intermediates)."""
     r = O.route(logits, K, C, A, S)
     R = r["R_max"]
     xq, xe = dispatch_fp8(x_bf16, r["token_slot"], R)
-    E, twoF, H = wq_gu.shape
+    Ew, twoF, H = wq_gu.shape
+    E = Ew - n_shared
     F = twoF // 2
     hq = np.zeros((R, F), np.uint8)
     he = np.full((R, F // BLOCK), P_MIN, np.int64)
@@ -198,6 +202,11 @@ def layer_forward_fp8(logits, x_bf16, wq_gu, wgu_exp, wq_d, wd_exp, K, C, A, S):
         sl = slice(int(off[e]), int(off[e]) + n)
         hq[sl], he[sl], y[sl], _ = expert_mlp_fp8_rows(xq[sl], xe[sl], wq_gu[e], wgu_exp[e],
                                                        wq_d[e], wd_exp[e])
-    out = O.combine(y, r["token_slot"], r["topk_w"], O.ACT_BF16)
-    r.update(xq=xq, x_exp=xe, hq=hq, h_exp=he, y=y)
+    y_sh = hq_sh = he_sh = None
+    if n_shared:
+        tq, te = quantize_rows(O.bf16_bits_to_f64(x_bf16))
+        hq_sh, he_sh, y_sh, _ = expert_mlp_fp8_rows(tq, te, wq_gu[E], wgu_exp[E], wq_d[E], wd_exp[E])
+    out = O.combine(y, r["token_slot"], r["topk_w"], O.ACT_BF16, y_shared=y_sh)
+    r.update(xq=xq, x_exp=xe, hq=hq, h_exp=he, y=y, y_shared=y_sh, hq_shared=hq_sh,
+             h_exp_shared=he_sh)
     return out, r

@@ -213,3 +213,26 @@ def test_layer_forward_fp8_combines_in_bf16():
     out, r = Q.layer_forward_fp8(lg, x, gq, ge, dq, de, K, T, 1, 2)
     ref = O.combine(r["y"], r["token_slot"], r["topk_w"], O.ACT_BF16)
     assert np.array_equal(out, ref)
+
+
+def test_fp8_shared_expert_is_the_dense_fp8_mlp_of_every_token():
+    # every routed assignment dropped (C = 0): the layer is the shared expert
+    # alone, i.e. the torch float8 pipeline applied to all tokens
+    rng = np.random.default_rng(10)
+    T, H, F, E, K = 48, 256, 256, 4, 2
+    x = O.f64_to_bf16_bits(rng.standard_normal((T, H)))
+    gq, ge = Q.quantize_rows(rng.standard_normal(((E + 1) * 2 * F, H)) * 0.05)
+    dq, de = Q.quantize_rows(rng.standard_normal(((E + 1) * H, F)) * 0.05)
+    gq, ge = gq.reshape(E + 1, 2 * F, H), ge.reshape(E + 1, 2 * F, 2)
+    dq, de = dq.reshape(E + 1, H, F), de.reshape(E + 1, H, 2)
+    lg = rng.standard_normal((T, E))
+    out, r = Q.layer_forward_fp8(lg, x, gq, ge, dq, de, K, 0, 1, 2, n_shared=1)
+    xq, xe = Q.quantize_rows(O.bf16_bits_to_f64(x))
+    _, _, ry = _torch_mlp_fp8(xq, xe, gq[E], ge[E], dq[E], de[E])
+    assert np.array_equal(out, ry)
+    # with routing kept, out = routed combine + shared output
+    out2, r2 = Q.layer_forward_fp8(lg, x, gq, ge, dq, de, K, T, 1, 2, n_shared=1)
+    routed = O.combine(r2["y"], r2["token_slot"], r2["topk_w"], O.ACT_BF16,
+                       y_shared=r2["y_shared"])
+    assert np.array_equal(out2, routed)
+    assert not np.array_equal(out2, O.combine(r2["y"], r2["token_slot"], r2["topk_w"], O.ACT_BF16))
