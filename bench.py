@@ -420,7 +420,7 @@ def cpu_oracle_sample_fp8(wl: W.Workload, tokens: int, layer: "Layer"):
     from oracle import moe_oracle as O
     from oracle import moe_oracle_fp8 as Q
     tokens = min(tokens, wl.T)
-    E, F, H = wl.E, wl.F, wl.H
+    E, F, H = wl.E + wl.n_shared, wl.F, wl.H
     gq, gs, dq, ds = (t.cpu().numpy() for t in layer.wq)
     ge = Q.scales_from_blocked(gs, E * 2 * F, H // 128).reshape(E, 2 * F, H // 128)
     de = Q.scales_from_blocked(ds, E * H, F // 128).reshape(E, H, F // 128)
@@ -428,7 +428,7 @@ def cpu_oracle_sample_fp8(wl: W.Workload, tokens: int, layer: "Layer"):
     x = layer.inp["x"][:tokens].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
     C = O.capacity(tokens, wl.K, wl.E, wl.cf)
     t0 = time.perf_counter()
-    Q.layer_forward_fp8(lg, x, gq, ge, dq, de, wl.K, C, wl.row_align, wl.S)
+    Q.layer_forward_fp8(lg, x, gq, ge, dq, de, wl.K, C, wl.row_align, wl.S, n_shared=wl.n_shared)
     return time.perf_counter() - t0, tokens
 
 

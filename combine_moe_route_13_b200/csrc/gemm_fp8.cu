@@ -176,7 +176,7 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                  uint8_t* __restrict__ out_sf, int N_out, int Kdim, int b_rows_per_expert,
                  int b_second_off, const int32_t* __restrict__ offsets,
                  const int32_t* __restrict__ counts, int E, int C, long long R_max,
-                 uint32_t* __restrict__ status) {
+                 uint32_t* __restrict__ status, int sh_rows, int sh_row0) {
   constexpr int BN_OUT = (MODE == 0) ? 128 : 256;   // output columns per tile
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = saddr(smem_raw);
@@ -185,9 +185,12 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   const uint32_t sf_smem = base + STAGES * OPER_BYTES;          // scale chunks of each stage
   const uint32_t staging = sf_smem + STAGES * SF_STAGE;         // 1024-aligned
   Ctl* ctl = reinterpret_cast<Ctl*>(smem + (staging - base) + STAGING_BYTES);
-  int* P = reinterpret_cast<int*>(ctl + 1);   // [E+1] M-tile prefix
-  int* row_off = P + (E + 1);                 // [E+1] first row of each expert, and R
-  int* kept_s = row_off + (E + 1);            // [E]
+  // Groups: the E routed experts, then (sh_rows > 0) the shared expert: its
+  // sh_rows rows start at sh_row0 and its weights are expert E's.
+  const int G = sh_rows > 0 ? E + 1 : E;
+  int* P = reinterpret_cast<int*>(ctl + 1);   // [G+1] M-tile prefix
+  int* row_off = P + (G + 1);                 // [G+1] first row of each group, and its end
+  int* kept_s = row_off + (G + 1);            // [G]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int NT = (N_out + BN_OUT - 1) / BN_OUT;
@@ -215,16 +218,23 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   }
   pdl_wait();
   pdl_trigger();
-  {  // per-expert kept rows, first row and M-tile prefix (block scan)
-    const int chunk = (E + NUM_THREADS - 1) / NUM_THREADS;
+  {  // per-group kept rows, first row and M-tile prefix (block scan)
+    const int chunk = (G + NUM_THREADS - 1) / NUM_THREADS;
     const int e0 = threadIdx.x * chunk;
     int local = 0;
     for (int i = 0; i < chunk; ++i) {
       const int e = e0 + i;
-      if (e < E) {
-        const int k = max(0, min(counts[e], C));
+      if (e < G) {
+        int k = e < E ? max(0, min(counts[e], C)) : sh_rows;
+        const int off = e < E ? offsets[e] : sh_row0;
+        // a caller table whose rows leave the buffer or start off a 128-row
+        // block (the scale chunks are per 128 rows) empties the expert
+        if (k > 0 && (off < 0 || (off & 127) != 0 || (long long)off + k > R_max)) {
+          atomicCAS(status, 0u, (uint32_t)MOE_ERR_DEVICE_INPUT);
+          k = 0;
+        }
         kept_s[e] = k;
-        row_off[e] = offsets[e];
+        row_off[e] = off;
         local += (k + BM - 1) / BM;
       }
     }
@@ -240,28 +250,28 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     for (int w = 0; w < warp; ++w) run += ctl->wsum[w];
     for (int i = 0; i < chunk; ++i) {
       const int e = e0 + i;
-      if (e < E) {
+      if (e < G) {
         P[e] = run;
         run += (kept_s[e] + BM - 1) / BM;
       }
     }
     if (threadIdx.x == NUM_THREADS - 1) {
-      P[E] = run;
-      row_off[E] = offsets[E];
+      P[G] = run;
+      row_off[G] = G > E ? sh_row0 + sh_rows : offsets[E];
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
-  const int total = P[E] * NT;
+  const int total = P[G] * NT;
 
   if (warp == 0) {
     if (lane == 0) {  // ------------------------------------------------ TMA producer
       int it = 0;
       for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
         int m, n;
-        const int e = decode_tile(tile, NT, P, E, m, n);
+        const int e = decode_tile(tile, NT, P, G, m, n);
         const int a_row = row_off[e] + m * BM;           // a multiple of 128
         const int b_row0 = e * b_rows_per_expert + n * BN_OUT;
         const uint8_t* sa_rows = sfa + (size_t)(a_row / 128) * KG * SF_CHUNK;
@@ -345,7 +355,7 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     int tcount = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
       int m, n;
-      const int e = decode_tile(tile, NT, P, E, m, n);
+      const int e = decode_tile(tile, NT, P, G, m, n);
       const int first = m * BM;
       const int rows = min(BM, kept_s[e] - first);
       const long long row0 = (long long)row_off[e] + first;
@@ -483,7 +493,8 @@ cudaError_t launch_one(int grid, size_t smem, cudaStream_t s, const CUtensorMap&
                        const CUtensorMap& b, const CUtensorMap& o, const uint8_t* sfa,
                        const uint8_t* sfb, void* out, uint8_t* out_sf, int N_out, int Kdim,
                        int b_rows, int b_second, const int32_t* offsets, const int32_t* counts,
-                       int E, int C, long long R_max, uint32_t* status) {
+                       int E, int C, long long R_max, uint32_t* status, int sh_rows,
+                       int sh_row0) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3(NUM_THREADS);
@@ -495,7 +506,8 @@ cudaError_t launch_one(int grid, size_t smem, cudaStream_t s, const CUtensorMap&
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, fp8_grouped_gemm<MODE>, a, b, o, sfa, sfb, out, out_sf, N_out,
-                            Kdim, b_rows, b_second, offsets, counts, E, C, R_max, status);
+                            Kdim, b_rows, b_second, offsets, counts, E, C, R_max, status, sh_rows,
+                            sh_row0);
 }
 
 }  // namespace f8
@@ -507,14 +519,18 @@ moe_status_t launch_mlp_fp8(const moe_config_t& c, const uint8_t* xq, const uint
                             cudaStream_t s) {
   using namespace f8;
   if (R_max == 0) return MOE_OK;
+  const int n_sh = c.n_shared ? 1 : 0;
+  const int G = c.E + n_sh;   // routed experts + the shared expert (last in the weights)
   CUtensorMap mx, mwgu, mh, mwd, my;
   if (!make_map_u8(&mx, xq, (uint64_t)c.H, (uint64_t)R_max) ||
-      !make_map_u8(&mwgu, wq_gu, (uint64_t)c.H, (uint64_t)c.E * 2 * c.F) ||
+      !make_map_u8(&mwgu, wq_gu, (uint64_t)c.H, (uint64_t)G * 2 * c.F) ||
       !make_map_u8(&mh, hq, (uint64_t)c.F, (uint64_t)R_max) ||
-      !make_map_u8(&mwd, wq_d, (uint64_t)c.F, (uint64_t)c.E * c.H) ||
+      !make_map_u8(&mwd, wq_d, (uint64_t)c.F, (uint64_t)G * c.H) ||
       !tc::make_map(&my, y, (uint64_t)c.H, (uint64_t)R_max))
     return MOE_ERR_CUDA;
-  const size_t smem = smem_bytes(c.E);
+  const int sh_rows = n_sh ? c.T : 0;
+  const int sh_row0 = n_sh ? (int)shared_row0(c) : 0;
+  const size_t smem = smem_bytes(G);
   if (cudaFuncSetAttribute(fp8_grouped_gemm<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess ||
       cudaFuncSetAttribute(fp8_grouped_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -524,14 +540,15 @@ moe_status_t launch_mlp_fp8(const moe_config_t& c, const uint8_t* xq, const uint
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return MOE_ERR_CUDA;
-  const int64_t mt_bound = ceil_div(R_max, BM) + c.E;   // >= sum_e M tiles
+  const int64_t mt_bound = ceil_div(R_max, BM) + G;   // >= sum over groups of M tiles
   const int g0 = (int)std::min<int64_t>(sms, mt_bound * ceil_div(c.F, 128));
   const int g1 = (int)std::min<int64_t>(sms, mt_bound * ceil_div(c.H, 256));
   cudaError_t e = launch_one<0>(g0, smem, s, mx, mwgu, mh, xs, ws_gu, hq, hs, c.F, c.H, 2 * c.F,
-                                c.F, offsets, counts, c.E, c.capacity, (long long)R_max, status);
+                                c.F, offsets, counts, c.E, c.capacity, (long long)R_max, status,
+                                sh_rows, sh_row0);
   if (e == cudaSuccess)
     e = launch_one<1>(g1, smem, s, mh, mwd, my, hs, ws_d, y, nullptr, c.H, c.F, c.H, 128, offsets,
-                      counts, c.E, c.capacity, (long long)R_max, status);
+                      counts, c.E, c.capacity, (long long)R_max, status, sh_rows, sh_row0);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -191,11 +191,17 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       const int e = e0 + i;
       if (e < G) {
         // dense_rows > 0: one group of dense_rows rows starting at row 0
-        const int k = dense_rows > 0 ? dense_rows
-                      : e < E        ? max(0, min(counts[e], C))
-                                     : sh_rows;
+        int k = dense_rows > 0 ? dense_rows
+                : e < E        ? max(0, min(counts[e], C))
+                               : sh_rows;
+        const int off = dense_rows > 0 ? 0 : (e < E ? offsets[e] : sh_out_row);
+        // a caller table whose rows leave the buffer empties the expert
+        if (k > 0 && (off < 0 || (long long)off + k > R_max)) {
+          atomicCAS(status, 0u, (uint32_t)MOE_ERR_DEVICE_INPUT);
+          k = 0;
+        }
         kept_s[e] = k;
-        row_off[e] = dense_rows > 0 ? 0 : (e < E ? offsets[e] : sh_out_row);
+        row_off[e] = off;
         local += (k + CF::TILE_ROWS - 1) / CF::TILE_ROWS;
       }
     }

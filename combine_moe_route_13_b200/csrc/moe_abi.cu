@@ -58,7 +58,7 @@ moe_status_t validate_fp8(const moe_config_t* c) {
   moe_status_t st = validate(c, true);
   if (st != MOE_OK) return st;
   if (c->act_dtype != MOE_BF16 || c->H % 256 != 0 || c->F % FP8_BLOCK != 0 ||
-      c->row_align % 128 != 0 || c->n_shared != 0 || c->E > 512)
+      c->row_align % 128 != 0 || c->E > 512)
     return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
@@ -448,7 +448,8 @@ moe_status_t moe_layer_forward_fp8(const moe_config_t* cfg, const float* logits,
   st = launch_mlp_fp8(*cfg, a.xq, a.xs, a.expert_offsets, a.expert_counts, wq_gu, ws_gu, wq_d,
                       ws_d, a.hq, a.hs, a.y, R, static_cast<uint32_t*>(ws), s);
   if (st != MOE_OK) return st;
-  return cuda_status(launch_combine(*cfg, a.y, a.token_slot, a.topk_w, -1, out, s));
+  return cuda_status(
+      launch_combine(*cfg, a.y, a.token_slot, a.topk_w, sh_row0_or_none(*cfg), out, s));
 }
 
 moe_status_t moe_get_device_status(void* ws, moe_status_t* status, void* stream) {

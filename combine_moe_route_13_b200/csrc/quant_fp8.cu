@@ -31,14 +31,15 @@ __device__ __forceinline__ void bf16x8_to_float(const uint4& q, float (&f)[8]) {
   }
 }
 
-// DISPATCH: destinations are the kept slots of token row blockIdx.x;
-// otherwise the destination is the row itself.
+// DISPATCH: destinations are the kept slots of token row blockIdx.x (and its
+// shared-expert row when sh_row0 >= 0); otherwise the destination is the row
+// itself.
 template <bool DISPATCH>
 __global__ void __launch_bounds__(QT)
 quant_rows_kernel(const uint4* __restrict__ src, int row_vecs, int KB,
                   const int32_t* __restrict__ token_slot, int K, uint8_t* __restrict__ q,
-                  uint8_t* __restrict__ sf, int slot_end) {
-  __shared__ int s_dst[MAX_K];
+                  uint8_t* __restrict__ sf, int slot_end, long long sh_row0) {
+  __shared__ int s_dst[MAX_K + 1];
   __shared__ int s_n;
   const int64_t row = blockIdx.x;
   pdl_wait();
@@ -50,6 +51,7 @@ quant_rows_kernel(const uint4* __restrict__ src, int row_vecs, int KB,
         const int s = token_slot[row * K + k];
         if (s >= 0 && s < slot_end) s_dst[n++] = s;   // others are dropped
       }
+      if (sh_row0 >= 0) s_dst[n++] = (int)(sh_row0 + row);   // the shared expert's row
       s_n = n;
     }
     __syncthreads();
@@ -97,7 +99,7 @@ cudaError_t launch_quantize_fp8(const void* src, int64_t rows, int64_t cols, uin
   if (rows == 0) return cudaSuccess;
   return launch_pdl(quant_rows_kernel<false>, dim3((unsigned)rows), dim3(QT), 0, s,
                     static_cast<const uint4*>(src), (int)(cols / 8), (int)(cols / FP8_BLOCK),
-                    (const int32_t*)nullptr, 0, q, sf, 0);
+                    (const int32_t*)nullptr, 0, q, sf, 0, -1LL);
 }
 
 cudaError_t launch_dispatch_fp8(const moe_config_t& c, const void* x, const int32_t* slot,
@@ -105,7 +107,7 @@ cudaError_t launch_dispatch_fp8(const moe_config_t& c, const void* x, const int3
   if (c.T == 0) return cudaSuccess;
   return launch_pdl(quant_rows_kernel<true>, dim3(c.T), dim3(QT), 0, s,
                     static_cast<const uint4*>(x), c.H / 8, c.H / FP8_BLOCK, slot, c.K, xq, xs,
-                    (int)routed_rows(c));
+                    (int)routed_rows(c), c.n_shared ? (long long)shared_row0(c) : -1LL);
 }
 
 }  // namespace moe

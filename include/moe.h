@@ -314,7 +314,9 @@ moe_status_t moe_layer_forward_x(const moe_config_t* cfg, const void* x, const v
  * moe_fp8_scale_bytes(rows, cols) bytes of scales; bytes of rows (or k blocks)
  * past the matrix are never written.
  * The whole fp8 path requires bf16 activations, H % 256 == 0, F % 128 == 0,
- * row_align % 128 == 0, n_shared == 0 and E <= 512 (else MOE_ERR_UNSUPPORTED).
+ * row_align % 128 == 0 and E <= 512 (else MOE_ERR_UNSUPPORTED). A shared expert
+ * (n_shared = 1) works as in the bf16 path: its weights are the last of the
+ * quantised arrays and its rows [R_sh, R_sh + T) of xq / hq / y are the tokens.
  * ------------------------------------------------------------------------- */
 
 /* ceil(rows / 128) * ceil(cols / 512) * 512, or -1 if rows < 0 or cols is not a
@@ -329,8 +331,9 @@ moe_status_t moe_quantize_fp8(const void* src, int64_t rows, int64_t cols, uint8
 
 /* Dispatch with the fp8 payload: each token row of x [T,H] bf16 is quantised once
  * and its codes and scales written to every kept row token_slot[t,k] of
- * xq [R_max,H] (e4m3) and xs (moe_fp8_scale_bytes(R_max, H) bytes). Rows no slot
- * points at are not written. */
+ * xq [R_max,H] (e4m3) and xs (moe_fp8_scale_bytes(R_max, H) bytes), and to its
+ * shared-expert row R_sh + t when n_shared = 1. Rows no slot points at are not
+ * written. */
 moe_status_t moe_dispatch_fp8(const moe_config_t* cfg, const void* x, const int32_t* token_slot,
                               uint8_t* xq, uint8_t* xs, void* stream);
 
@@ -339,9 +342,11 @@ moe_status_t moe_dispatch_fp8(const moe_config_t* cfg, const void* x, const int3
  *   h[r] = silu(xq[r] Wg_e^T) * (xq[r] Wu_e^T), quantised to hq[r] (e4m3) and hs
  *          (scales of the [R_max, F] matrix) from its fp32 value,
  *   y[r] = hq[r] W_d,e^T rounded to bf16,
- * with every operand taken as scale * e4m3 value. wq_gu [E,2F,H] e4m3 with scales
- * ws_gu of the [E*2F, H] matrix; wq_d [E,H,F] with ws_d of [E*H, F] (from
- * moe_quantize_fp8). y [R_max,H] bf16. ws: any workspace with a status word. */
+ * with every operand taken as scale * e4m3 value. wq_gu [E',2F,H] e4m3 with scales
+ * ws_gu of the [E'*2F, H] matrix; wq_d [E',H,F] with ws_d of [E'*H, F] (from
+ * moe_quantize_fp8), E' = E + n_shared. y [R_max,H] bf16. ws: any workspace with
+ * a status word. A caller offsets table whose expert leaves [0, R_max) or starts
+ * off a multiple of 128 skips that expert and records MOE_ERR_DEVICE_INPUT. */
 moe_status_t moe_expert_mlp_fp8(const moe_config_t* cfg, const uint8_t* xq, const uint8_t* xs,
                                 const int32_t* expert_offsets, const int32_t* expert_counts,
                                 const uint8_t* wq_gu, const uint8_t* ws_gu, const uint8_t* wq_d,

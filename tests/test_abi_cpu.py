@@ -184,7 +184,6 @@ def test_fp8_scale_bytes():
     (dict(H=4224), M.MOE_ERR_UNSUPPORTED),          # H % 256 != 0
     (dict(F=14400), M.MOE_ERR_UNSUPPORTED),         # F % 128 != 0
     (dict(row_align=64), M.MOE_ERR_UNSUPPORTED),
-    (dict(n_shared=1), M.MOE_ERR_UNSUPPORTED),
     (dict(E=640, K=2, S=8), M.MOE_ERR_UNSUPPORTED),
 ])
 def test_fp8_configs_outside_the_kernels_are_rejected(kw, code):

@@ -215,3 +215,79 @@ def test_layer_forward_fp8(cuda_ok, wl):
         assert fro <= 1e-2, f"whole chain: relative Frobenius error {fro:.3e}"
     else:
         assert not np.any(gd)
+
+
+@pytest.mark.parametrize("corruption", ["past_the_buffer", "off_a_128_row_block"])
+def test_expert_mlp_fp8_rejects_bad_offsets(cuda_ok, corruption):
+    # the fp8 GEMMs read scale chunks per 128 rows with untiled bulk copies, so a
+    # caller offsets table is checked first: an expert whose rows leave the
+    # buffer or start off a 128-row block is skipped and reported
+    T, H, E, K, F, S = 1200, 256, 8, 2, 256, 2
+    C = O.capacity(T, K, E, 1.25)
+    cfg = _cfg(T, H, E, K, F, S, C)
+    r = run_route(cfg, _logits(T, E, "normal", 31).to(DEV))
+    R = M.moe_max_rows(cfg)
+    x = torch.randn(T, H, generator=torch.Generator().manual_seed(32)).to(torch.bfloat16).to(DEV)
+    (gq, gs, dq, ds), _ = _weights_fp8(E, F, H, 33)
+    xq = torch.zeros(R, H, dtype=torch.uint8, device=DEV)
+    xs = torch.zeros(M.moe_fp8_scale_bytes(R, H), dtype=torch.uint8, device=DEV)
+    M.moe_dispatch_fp8(cfg, x, r["token_slot"], xq, xs)
+
+    def run(offsets):
+        hq = torch.zeros(R, F, dtype=torch.uint8, device=DEV)
+        hs = torch.zeros(M.moe_fp8_scale_bytes(R, F), dtype=torch.uint8, device=DEV)
+        y = torch.zeros(R, H, dtype=torch.bfloat16, device=DEV)
+        ws = M.alloc_workspace(256)
+        M.moe_expert_mlp_fp8(cfg, xq, xs, offsets, r["expert_counts"], gq, gs, dq, ds, hq, hs, y, ws)
+        return y, M.moe_get_device_status(ws)
+
+    y_ok, st = run(r["expert_offsets"])
+    assert st == M.MOE_OK
+    bad = r["expert_offsets"].clone()
+    bad[5] = R + 4096 if corruption == "past_the_buffer" else bad[5] + 8
+    y_bad, st = run(bad)
+    assert st == M.MOE_ERR_DEVICE_INPUT
+    off = r["expert_offsets"].cpu().numpy()
+    kept = np.minimum(r["expert_counts"].cpu().numpy(), C)
+    for e in range(E):
+        if e == 5 or kept[e] == 0:
+            continue
+        sl = slice(int(off[e]), int(off[e]) + int(kept[e]))
+        assert torch.equal(y_bad[sl].view(torch.int16), y_ok[sl].view(torch.int16)), e
+
+
+def test_layer_forward_fp8_with_shared_expert(cuda_ok):
+    # the shared expert (n_shared = 1) on the fp8 path: its rows of xq are the
+    # tokens' quantisation, its h / y rows follow the fp8 oracle, and the
+    # combine adds its output with weight 1
+    wl = W.small_case(700, 512, 8, 2, 256, 2, 1.25, "bf16", 128, n_shared=1)
+    C = O.capacity(wl.T, wl.K, wl.E, wl.cf)
+    cfg = M.make_config(T=wl.T, H=wl.H, E=wl.E, K=wl.K, F=wl.F, S=wl.S, capacity=C,
+                        row_align=wl.row_align, act="bf16", n_shared=1)
+    inp = W.make_inputs(wl, seed=77, device=DEV)
+    (gq, gs, dq, ds), (gq_n, ge, dq_n, de) = _weights_fp8(wl.E + 1, wl.F, wl.H, 78)
+    ws = M.alloc_workspace(M.moe_workspace_bytes(cfg))
+    out = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device=DEV)
+    aux = M.moe_layer_forward_fp8(cfg, inp["logits"], inp["x"], gq, gs, dq, ds, out, ws)
+    assert M.moe_get_device_status(ws) == M.MOE_OK
+    v, f = M.layer_views(cfg, ws, aux), M.fp8_views(cfg, ws, aux)
+    x_n = act_np(inp["x"])
+    ref_out, ref = Q.layer_forward_fp8(inp["logits"].cpu().numpy(), x_n, gq_n, ge, dq_n, de,
+                                       wl.K, C, wl.row_align, wl.S, n_shared=1)
+    R_r, R_sh, Rt = ref["R_max"], M.shared_row0(cfg), M.moe_max_rows(cfg)
+    assert Rt == R_sh + wl.T
+    xq_n, hq_n, y_n = np_u8(f["xq"]), np_u8(f["hq"]), act_np(v["y"])
+    xe = Q.scales_from_blocked(np_u8(f["xs"]), Rt, wl.H // 128)
+    he = Q.scales_from_blocked(np_u8(f["hs"]), Rt, wl.F // 128)
+    kept = ref["row_src"] >= 0
+    assert np.array_equal(xq_n[:R_r][kept], ref["xq"][kept])
+    tq, te = Q.quantize_rows(O.bf16_bits_to_f64(x_n))
+    assert np.array_equal(xq_n[R_sh:], tq) and np.array_equal(xe[R_sh:], te)
+    assert_h_close(hq_n[R_sh:], he[R_sh:], ref["hq_shared"], ref["h_exp_shared"], "h shared")
+    assert_close_act(y_n[R_sh:], Q.down_fp8_rows(hq_n[R_sh:], he[R_sh:], dq_n[wl.E], de[wl.E]),
+                     O.ACT_BF16, "y shared")
+    assert_h_close(hq_n[:R_r][kept], he[:R_r][kept], ref["hq"][kept], ref["h_exp"][kept], "h")
+    got = O.combine(y_n, ref["token_slot"], ref["topk_w"], O.ACT_BF16, y_shared=y_n[R_sh:])
+    assert_close_act(act_np(out), got, O.ACT_BF16, "out")
+    gd, rd = O.bf16_bits_to_f64(act_np(out)), O.bf16_bits_to_f64(ref_out)
+    assert np.linalg.norm(gd - rd) / np.linalg.norm(rd) <= 1e-2

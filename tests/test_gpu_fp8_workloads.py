@@ -35,12 +35,14 @@ def _expert_scales(buf, e, rows_per_expert, cols):
     return Q.scales_from_blocked(np_u8(buf[e * per:(e + 1) * per]), rows_per_expert, KB)
 
 
-@pytest.mark.parametrize("name", ["mixtral", "dsv3", "skewed", "kimi"])
-def test_workload_full_size_fp8(cuda_ok, name):
-    wl = W.WORKLOADS[name]
+@pytest.mark.parametrize("name,n_shared", [("mixtral", 0), ("dsv3", 0), ("skewed", 0),
+                                           ("kimi", 0), ("dsv3", 1)])
+def test_workload_full_size_fp8(cuda_ok, name, n_shared):
+    wl = W.WORKLOADS[name].with_(n_shared=n_shared)
     dev = torch.device("cuda")
     C = M.moe_capacity(wl.T, wl.K, wl.E, wl.cf)
-    cfg = M.make_config(wl.T, wl.H, wl.E, wl.K, wl.F, wl.S, C, wl.row_align, wl.act)
+    cfg = M.make_config(wl.T, wl.H, wl.E, wl.K, wl.F, wl.S, C, wl.row_align, wl.act,
+                        n_shared=n_shared)
     inp = W.make_inputs(wl, seed=0, device=dev)
     gq, gs = M.quantize_fp8(inp["w_gu"])
     dq, ds = M.quantize_fp8(inp["w_d"])
@@ -75,6 +77,13 @@ def test_workload_full_size_fp8(cuda_ok, name):
     experts = {int(nonempty[np.argmax(kept[nonempty])]), int(nonempty[np.argmin(kept[nonempty])]),
                int(rng.choice(nonempty))}
     hs_all = Q.scales_from_blocked(np_u8(f["hs"]), R, F // 128)
+    if n_shared:
+        experts.add(wl.E)   # the shared expert: its rows are the tokens, from shared_row0 on
+    R_sh = M.shared_row0(cfg)
+    Rt = M.moe_max_rows(cfg)
+    if n_shared:
+        hs_all = Q.scales_from_blocked(np_u8(f["hs"]), Rt, F // 128)
+        xs_all = Q.scales_from_blocked(np_u8(f["xs"]), Rt, H // 128)
     for e in sorted(experts):
         # the expert's weights: codes and scales against the oracle's quantisation
         wgu = O.bf16_bits_to_f64(act_np(inp["w_gu"][e]))
@@ -85,11 +94,15 @@ def test_workload_full_size_fp8(cuda_ok, name):
         assert np.array_equal(_expert_scales(gs, e, 2 * F, H), ge_ref)
         assert np.array_equal(np_u8(dq[e]), dq_ref)
         assert np.array_equal(_expert_scales(ds, e, H, F), de_ref)
-        n = int(kept[e])
-        rows = off[e] + np.unique(np.concatenate([np.arange(min(3, n)), np.arange(max(0, n - 3), n),
+        n = int(kept[e]) if e < wl.E else wl.T
+        first = off[e] if e < wl.E else R_sh
+        rows = first + np.unique(np.concatenate([np.arange(min(3, n)), np.arange(max(0, n - 3), n),
                                                   rng.integers(0, n, 6)]))
         ridx = torch.from_numpy(rows).to(dev)
         xq_rows = np_u8(f["xq"][ridx])
+        if e == wl.E:   # the shared expert's dispatch: the tokens' own quantisation
+            tq, te = Q.quantize_rows(O.bf16_bits_to_f64(act_np(inp["x"][ridx - R_sh])))
+            assert np.array_equal(xq_rows, tq) and np.array_equal(xs_all[rows], te)
         hq_ref, he_ref, _, _ = Q.expert_mlp_fp8_rows(xq_rows, xs_all[rows], gq_ref, ge_ref, dq_ref,
                                                      de_ref)
         hq_rows = np_u8(f["hq"][ridx])
@@ -105,7 +118,8 @@ def test_workload_full_size_fp8(cuda_ok, name):
     remap[need] = np.arange(len(need))
     slot_sub = np.where(slot >= 0, remap[np.maximum(slot, 0)], -1).astype(np.int32)
     y_sub = act_np(v["y"][torch.from_numpy(need).to(dev)])
-    ref_out = O.combine(y_sub, slot_sub, ref["topk_w"][toks], O.ACT_BF16)
+    y_sh = act_np(v["y"][torch.from_numpy(R_sh + toks).to(dev)]) if n_shared else None
+    ref_out = O.combine(y_sub, slot_sub, ref["topk_w"][toks], O.ACT_BF16, y_shared=y_sh)
     assert_close_act(act_np(out[torch.from_numpy(toks).to(dev)]), ref_out, O.ACT_BF16, "out")
     del inp, ws, out, gq, gs, dq, ds
     torch.cuda.empty_cache()

@@ -307,3 +307,23 @@ def test_route_random_sweep(cuda_ok, T, E, K, S, cf, A, kind):
     gpu = host(run_route(cfg, lg.to(DEV)))
     ref = O.route(lg.numpy(), K, C, A, S)
     assert_route_equal(gpu, ref, ref["R_max"])
+
+
+def test_expert_mlp_rejects_out_of_range_offsets(cuda_ok):
+    # a caller offsets table pointing an expert past the buffer: the GEMMs record
+    # MOE_ERR_DEVICE_INPUT, skip that expert and compute the others as before
+    cfg, r, inp, xp, h, y = _run_mlp(1200, 256, 8, 2, 256, 2, 1.25, 128, "normal", "bf16")
+    R = M.moe_max_rows(cfg)
+    bad = r["expert_offsets"].clone()
+    bad[3] = R + 4096
+    h2, y2 = torch.zeros_like(h), torch.zeros_like(y)
+    ws = M.alloc_workspace(256)
+    M.moe_expert_mlp(cfg, xp, bad, r["expert_counts"], inp["w_gu"], inp["w_d"], h2, y2, ws)
+    assert M.moe_get_device_status(ws) == M.MOE_ERR_DEVICE_INPUT
+    off = r["expert_offsets"].cpu().numpy()
+    kept = np.minimum(r["expert_counts"].cpu().numpy(), cfg.capacity)
+    for e in range(8):
+        if e == 3 or kept[e] == 0:
+            continue
+        sl = slice(int(off[e]), int(off[e]) + int(kept[e]))
+        assert torch.equal(y2[sl].view(torch.int16), y[sl].view(torch.int16)), e
