@@ -35,7 +35,12 @@ EXPORTS = ("moe_capacity", "moe_max_rows", "moe_check_config", "moe_route_worksp
            "moe_status_string", "moe_version", "moe_route_topk_noalloc", "moe_combine_wait",
            "moe_route_topk_biased", "moe_router_logits", "moe_layer_forward_x",
            "moe_fp8_scale_bytes", "moe_quantize_fp8", "moe_dispatch_fp8", "moe_expert_mlp_fp8",
-           "moe_layer_forward_fp8")
+           "moe_layer_forward_fp8") + (
+    # include/moe_ep.h
+           "moe_ep_recv_rows", "moe_ep_symmetric_bytes", "moe_ep_workspace_bytes", "moe_ep_check",
+           "moe_ep_aux", "moe_ep_symmetric_init", "moe_ep_route", "moe_ep_dispatch",
+           "moe_ep_expert_mlp", "moe_ep_combine", "moe_ep_layer_forward", "moe_ep_sym_alloc",
+           "moe_ep_sym_free", "moe_ipc_get_handle", "moe_ipc_open", "moe_ipc_close")
 
 
 class MoeError(RuntimeError):
@@ -61,8 +66,22 @@ class MoeLayerAux(ctypes.Structure):
         "xq", "xs", "hq", "hs")]
 
 
+class MoeEp(ctypes.Structure):
+    _fields_ = [("world", ctypes.c_int32), ("rank", ctypes.c_int32), ("epoch", ctypes.c_uint32),
+                ("timeout_us", ctypes.c_uint32)]
+
+
+class MoeEpAux(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "topk_idx", "expert_counts", "overflow", "expert_offsets", "segment_offsets",
+        "token_slot", "row_src", "totals", "topk_w", "counts_all", "flags", "send_dst_row",
+        "recv_offsets", "recv_counts", "xr", "h", "y")]
+
+
 _P = ctypes.c_void_p
 _CFG = ctypes.POINTER(MoeConfig)
+_EP = ctypes.POINTER(MoeEp)
+_SZ = ctypes.c_size_t
 
 
 def _load():
@@ -101,6 +120,23 @@ def _load():
         "moe_layer_forward_fp8": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P,
                                                  ctypes.c_uint32, _P, ctypes.c_size_t,
                                                  ctypes.POINTER(MoeLayerAux), _P]),
+        "moe_ep_recv_rows": (ctypes.c_int64, [_CFG, ctypes.c_int32]),
+        "moe_ep_symmetric_bytes": (_SZ, [_CFG, ctypes.c_int32]),
+        "moe_ep_workspace_bytes": (_SZ, [_CFG, ctypes.c_int32]),
+        "moe_ep_check": (ctypes.c_int, [_CFG, _EP]),
+        "moe_ep_aux": (ctypes.c_int, [_CFG, _EP, _P, _P, ctypes.POINTER(MoeEpAux)]),
+        "moe_ep_symmetric_init": (ctypes.c_int, [_CFG, ctypes.c_int32, _P, _SZ, _P]),
+        "moe_ep_route": (ctypes.c_int, [_CFG, _EP, _P, _P, _P, _P, _SZ, _P]),
+        "moe_ep_dispatch": (ctypes.c_int, [_CFG, _EP, _P, _P, _P, _P, _SZ, _P]),
+        "moe_ep_expert_mlp": (ctypes.c_int, [_CFG, _EP, _P, _P, _P, _P, _P, _SZ, _P]),
+        "moe_ep_combine": (ctypes.c_int, [_CFG, _EP, _P, _P, _P, _P, _SZ, _P]),
+        "moe_ep_layer_forward": (ctypes.c_int, [_CFG, _EP, _P, _P, _P, _P, _P, _P, _P,
+                                                ctypes.POINTER(MoeEpAux), _P, _SZ, _P]),
+        "moe_ep_sym_alloc": (ctypes.c_int, [_SZ, ctypes.POINTER(ctypes.c_void_p)]),
+        "moe_ep_sym_free": (ctypes.c_int, [_P]),
+        "moe_ipc_get_handle": (ctypes.c_int, [_P, ctypes.c_char_p]),
+        "moe_ipc_open": (ctypes.c_int, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_void_p)]),
+        "moe_ipc_close": (ctypes.c_int, [_P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -431,4 +467,160 @@ def layer_views(cfg: MoeConfig, ws: torch.Tensor, aux: MoeLayerAux) -> dict:
         "h": view(aux.h, R * cfg.F * es, dt, (R, cfg.F)),
         "y": view(aux.y, R * cfg.H * es, dt, (R, cfg.H)),
         "logits": view(aux.logits, TK // max(cfg.K, 1) * cfg.E * 4, torch.float32, (cfg.T, cfg.E)),
+    }
+
+
+# ---------------------------------------------------------------- expert parallelism (moe_ep.h)
+
+def make_ep(world: int, rank: int, epoch: int, timeout_us: int = 0) -> MoeEp:
+    return MoeEp(int(world), int(rank), int(epoch), int(timeout_us))
+
+
+def _addr(buf, name) -> int:
+    """Device address of a CUDA tensor, or an address given as an int (a
+    region mapped by moe_ipc_open or allocated by moe_ep_sym_alloc)."""
+    if isinstance(buf, int):
+        return buf
+    return _ptr(buf, name=name)
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
+def moe_ep_recv_rows(cfg: MoeConfig, world: int) -> int:
+    return int(LIB.moe_ep_recv_rows(ctypes.byref(cfg), int(world)))
+
+
+def moe_ep_symmetric_bytes(cfg: MoeConfig, world: int) -> int:
+    return int(LIB.moe_ep_symmetric_bytes(ctypes.byref(cfg), int(world)))
+
+
+def moe_ep_workspace_bytes(cfg: MoeConfig, world: int) -> int:
+    return int(LIB.moe_ep_workspace_bytes(ctypes.byref(cfg), int(world)))
+
+
+def moe_ep_check(cfg: MoeConfig, ep: MoeEp) -> int:
+    return int(LIB.moe_ep_check(ctypes.byref(cfg), ctypes.byref(ep)))
+
+
+def moe_ep_aux(cfg, ep, sym, ws) -> MoeEpAux:
+    aux = MoeEpAux()
+    _check(LIB.moe_ep_aux(ctypes.byref(cfg), ctypes.byref(ep), _addr(sym, "sym"),
+                          _ptr(ws, name="ws"), ctypes.byref(aux)), "moe_ep_aux")
+    return aux
+
+
+def moe_ep_symmetric_init(cfg, world, sym, sym_bytes=None, stream=None):
+    n = _nbytes(sym) if sym_bytes is None else int(sym_bytes)
+    _check(LIB.moe_ep_symmetric_init(ctypes.byref(cfg), int(world), _addr(sym, "sym"), n,
+                                     _stream(stream)), "moe_ep_symmetric_init")
+
+
+def _peers(peers):
+    return _ptr(peers, torch.int64, "peers")
+
+
+def moe_ep_route(cfg, ep, logits, sym, peers, ws, stream=None):
+    _check(LIB.moe_ep_route(ctypes.byref(cfg), ctypes.byref(ep),
+                            _ptr(logits, torch.float32, "logits"), _addr(sym, "sym"),
+                            _peers(peers), _ptr(ws, name="ws"), _nbytes(ws), _stream(stream)),
+           "moe_ep_route")
+
+
+def moe_ep_dispatch(cfg, ep, x, sym, peers, ws, stream=None):
+    _check(LIB.moe_ep_dispatch(ctypes.byref(cfg), ctypes.byref(ep), _ptr(x, act_dtype(cfg), "x"),
+                               _addr(sym, "sym"), _peers(peers), _ptr(ws, name="ws"), _nbytes(ws),
+                               _stream(stream)), "moe_ep_dispatch")
+
+
+def moe_ep_expert_mlp(cfg, ep, w_gu_local, w_d_local, sym, peers, ws, stream=None):
+    dt = act_dtype(cfg)
+    _check(LIB.moe_ep_expert_mlp(ctypes.byref(cfg), ctypes.byref(ep),
+                                 _ptr(w_gu_local, dt, "w_gu_local"), _ptr(w_d_local, dt, "w_d_local"),
+                                 _addr(sym, "sym"), _peers(peers), _ptr(ws, name="ws"),
+                                 _nbytes(ws), _stream(stream)), "moe_ep_expert_mlp")
+
+
+def moe_ep_combine(cfg, ep, sym, peers, out, ws, stream=None):
+    _check(LIB.moe_ep_combine(ctypes.byref(cfg), ctypes.byref(ep), _addr(sym, "sym"),
+                              _peers(peers), _ptr(out, act_dtype(cfg), "out"), _ptr(ws, name="ws"),
+                              _nbytes(ws), _stream(stream)), "moe_ep_combine")
+
+
+def moe_ep_layer_forward(cfg, ep, logits, x, w_gu_local, w_d_local, sym, peers, out, ws,
+                         stream=None) -> MoeEpAux:
+    dt = act_dtype(cfg)
+    aux = MoeEpAux()
+    _check(LIB.moe_ep_layer_forward(
+        ctypes.byref(cfg), ctypes.byref(ep), _ptr(logits, torch.float32, "logits"),
+        _ptr(x, dt, "x"), _ptr(w_gu_local, dt, "w_gu_local"), _ptr(w_d_local, dt, "w_d_local"),
+        _addr(sym, "sym"), _peers(peers), _ptr(out, dt, "out"), ctypes.byref(aux),
+        _ptr(ws, name="ws"), _nbytes(ws), _stream(stream)), "moe_ep_layer_forward")
+    return aux
+
+
+def moe_ep_sym_alloc(nbytes: int) -> int:
+    p = ctypes.c_void_p()
+    _check(LIB.moe_ep_sym_alloc(int(nbytes), ctypes.byref(p)), "moe_ep_sym_alloc")
+    return int(p.value)
+
+
+def moe_ep_sym_free(addr: int):
+    _check(LIB.moe_ep_sym_free(int(addr)), "moe_ep_sym_free")
+
+
+def moe_ipc_get_handle(addr: int) -> bytes:
+    buf = ctypes.create_string_buffer(64)
+    _check(LIB.moe_ipc_get_handle(int(addr), buf), "moe_ipc_get_handle")
+    return buf.raw
+
+
+def moe_ipc_open(handle: bytes) -> int:
+    if len(handle) != 64:
+        raise ValueError("a CUDA IPC handle has 64 bytes")
+    p = ctypes.c_void_p()
+    _check(LIB.moe_ipc_open(handle, ctypes.byref(p)), "moe_ipc_open")
+    return int(p.value)
+
+
+def moe_ipc_close(addr: int):
+    _check(LIB.moe_ipc_close(int(addr)), "moe_ipc_close")
+
+
+def ep_views(cfg: MoeConfig, world: int, sym: torch.Tensor, ws: torch.Tensor,
+             aux: MoeEpAux) -> dict:
+    """torch views of one rank's intermediates (sym and ws given as tensors)."""
+    El = cfg.E // world
+    R = moe_ep_recv_rows(cfg, world)
+    dt = act_dtype(cfg)
+    es = 4 if dt == torch.float32 else 2
+    TK = cfg.T * cfg.K
+    Rl = moe_max_rows(make_config(cfg.T, cfg.H, cfg.E, cfg.K, cfg.F, cfg.S, cfg.capacity,
+                                  cfg.row_align, cfg.act_dtype))
+
+    def view(buf, ptr, nbytes, dtype, shape):
+        off = ptr - buf.data_ptr()
+        assert 0 <= off and off + nbytes <= _nbytes(buf)
+        return buf[off:off + nbytes].view(dtype).view(shape)
+
+    i32 = torch.int32
+    return {
+        "topk_idx": view(ws, aux.topk_idx, TK * 4, i32, (cfg.T, cfg.K)),
+        "topk_w": view(ws, aux.topk_w, TK * 4, torch.float32, (cfg.T, cfg.K)),
+        "expert_counts": view(ws, aux.expert_counts, cfg.E * 4, i32, (cfg.E,)),
+        "overflow": view(ws, aux.overflow, cfg.E * 4, i32, (cfg.E,)),
+        "expert_offsets": view(ws, aux.expert_offsets, (cfg.E + 1) * 4, i32, (cfg.E + 1,)),
+        "segment_offsets": view(ws, aux.segment_offsets, (cfg.S + 1) * 4, i32, (cfg.S + 1,)),
+        "token_slot": view(ws, aux.token_slot, TK * 4, i32, (cfg.T, cfg.K)),
+        "row_src": view(ws, aux.row_src, Rl * 4, i32, (Rl,)),
+        "totals": view(ws, aux.totals, 16, i32, (4,)),
+        "send_dst_row": view(ws, aux.send_dst_row, cfg.E * 4, i32, (cfg.E,)),
+        "recv_offsets": view(ws, aux.recv_offsets, (El + 1) * 4, i32, (El + 1,)),
+        "recv_counts": view(ws, aux.recv_counts, El * 4, i32, (El,)),
+        "counts_all": view(sym, aux.counts_all, world * cfg.E * 4, i32, (world, cfg.E)),
+        "flags": view(sym, aux.flags, 3 * world * 4, i32, (3, world)),
+        "xr": view(sym, aux.xr, R * cfg.H * es, dt, (R, cfg.H)),
+        "h": view(ws, aux.h, R * cfg.F * es, dt, (R, cfg.F)),
+        "y": view(sym, aux.y, R * cfg.H * es, dt, (R, cfg.H)),
     }

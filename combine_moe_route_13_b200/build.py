@@ -21,9 +21,10 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmoe.so")
 SOURCES = ["moe_abi.cu", "route.cu", "dispatch_combine.cu", "gemm_simt.cu", "gemm_tc.cu",
-           "route_noalloc.cu", "quant_fp8.cu", "gemm_fp8.cu"]
-HEADERS = [os.path.join(CSRC, h) for h in ("moe_internal.h", "tc_ptx.cuh", "fp8_util.cuh")] + \
-    [os.path.join(ROOT, "include", "moe.h")]
+           "route_noalloc.cu", "quant_fp8.cu", "gemm_fp8.cu", "ep.cu"]
+HEADERS = [os.path.join(CSRC, h) for h in ("moe_internal.h", "tc_ptx.cuh", "fp8_util.cuh",
+                                         "vec_util.cuh")] + \
+    [os.path.join(ROOT, "include", h) for h in ("moe.h", "moe_ep.h")]
 GENCODE = "arch=compute_100a,code=sm_100a"
 
 

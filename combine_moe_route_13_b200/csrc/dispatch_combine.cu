@@ -17,6 +17,7 @@
 #include <cuda_bf16.h>
 
 #include "moe_internal.h"
+#include "vec_util.cuh"
 
 namespace moe {
 namespace {
@@ -68,20 +69,6 @@ dispatch_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ token_s
       }
     }
   }
-}
-
-__device__ __forceinline__ void unpack_bf16x8(const uint4& q, float (&f)[8]) {
-  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-  }
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&b);
 }
 
 template <bool BF16>

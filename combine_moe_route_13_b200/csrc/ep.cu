@@ -1,0 +1,732 @@
+// Expert parallelism: the layer split over W ranks, rank d owning the experts
+// [d*E/W, (d+1)*E/W), with every exchange done by this library's kernels
+// over peer memory (plain loads and stores through peer pointers; no
+// multicast objects, no library collectives).
+//
+// Follows:
+//  - "Enabling trillion-parameter models on AWS EFA", "Буферы отправки и
+//    получения": counts per expert are exchanged first; from them senders
+//    find where their rows go and receivers where each sender's rows land.
+//    Inside a node the receive buffers are mapped into the peers, which write
+//    into them directly.
+//  - "Efficient and portable Mixture-of-Experts communication", "Draagbare
+//    kernels": send halves that never block, receive halves that wait for
+//    their data; a fixed per-sender bound gives every sender a unique
+//    destination address with no synchronisation among senders; the received
+//    rows are already in the expert GEMM's layout.
+//  - "Mixture-of-Experts acceleration through overlap": flags published by
+//    the producer and polled by the consumer.
+//
+// Kernels, in the order of a step on one rank:
+//   publish   every rank's counts table gets this rank's E counts; COUNTS flag
+//   plan      wait for all COUNTS flags; kept = min(count, C); scans give
+//             send_dst_row[E], recv_offsets[E/W+1], recv_counts[E/W]
+//   dispatch  one block per token: its row is read once and written to the
+//             owners of its kept experts; the last block to finish sets every
+//             owner's DISPATCH flag for this rank
+//   wait      one thread: all DISPATCH flags (then the grouped GEMM of
+//             moe_expert_mlp over the local experts)
+//   signal    every rank's Y flag for this rank, after the GEMM
+//   wait      all Y flags
+//   combine   one block per token: the owners' y rows of its kept
+//             assignments, read in place, weighted sum in k order
+// Flags hold the step number (epoch) and are compared as "reached", so they
+// are never reset. Every wait is bounded; see moe_ep.h for the error rules.
+#include <algorithm>
+#include <climits>
+#include <cstring>
+
+#include "moe_internal.h"
+#include "vec_util.cuh"
+#include "../../include/moe_ep.h"
+
+namespace moe {
+namespace {
+
+constexpr int EP_THREADS = 128;
+constexpr int EP_UNROLL = 4;
+constexpr int MAX_W = 64;
+constexpr int PLAN_THREADS = 1024;   // >= MAX_E: one thread per expert
+enum : int { FLAG_COUNTS = 0, FLAG_DISPATCH = 1, FLAG_Y = 2, NUM_FLAGS = 3 };
+
+struct SymLayout {
+  size_t counts = 0, flags = 0, xr = 0, y = 0, total = 0;
+};
+
+struct EpWs {
+  size_t blk_cnt = 0, topk_idx = 0, topk_w = 0, counts = 0, overflow = 0, offsets = 0;
+  size_t segoff = 0, totals = 0, slot = 0, row_src = 0;
+  size_t send_dst = 0, recv_off = 0, recv_cnt = 0, done = 0, h = 0, total = 0;
+};
+
+int64_t recv_rows(const moe_config_t& c, int W) {
+  const int64_t El = c.E / W;
+  return std::min<int64_t>((int64_t)W * c.T * std::min<int64_t>(c.K, El),
+                           El * W * (int64_t)c.capacity) +
+         El * (c.row_align - 1);
+}
+
+// The grouped GEMM's view of a rank: its E/W local experts, each with up to
+// W*C received rows, R_recv rows in all (max_rows of this config = R_recv).
+moe_config_t local_cfg(const moe_config_t& c, int W) {
+  moe_config_t l = c;
+  l.T = W * c.T;
+  l.E = c.E / W;
+  l.K = std::min(c.K, c.E / W);
+  l.S = 1;
+  l.capacity = W * c.capacity;
+  l.n_shared = 0;
+  return l;
+}
+
+SymLayout sym_layout(const moe_config_t& c, int W) {
+  SymLayout L;
+  const int64_t R = recv_rows(c, W);
+  const size_t as = act_size(c.act_dtype);
+  size_t p = 0;
+  L.counts = p; p += align256((size_t)W * c.E * 4);
+  L.flags = p;  p += align256((size_t)NUM_FLAGS * W * 4);
+  L.xr = p;     p += align256((size_t)R * c.H * as);
+  L.y = p;      p += align256((size_t)R * c.H * as);
+  L.total = p;
+  return L;
+}
+
+EpWs ep_ws_layout(const moe_config_t& c, int W) {
+  EpWs L;
+  const int64_t nblk = ceil_div(c.T, ROUTE_TB);
+  const int64_t TK = (int64_t)c.T * c.K;
+  const int El = c.E / W;
+  size_t p = 256;   // status word
+  L.blk_cnt = p;   p += align256((size_t)std::max<int64_t>(nblk, 1) * c.E * 4);
+  L.topk_idx = p;  p += align256((size_t)TK * 4);
+  L.topk_w = p;    p += align256((size_t)TK * 4);
+  L.counts = p;    p += align256((size_t)c.E * 4);
+  L.overflow = p;  p += align256((size_t)c.E * 4);
+  L.offsets = p;   p += align256((size_t)(c.E + 1) * 4);
+  L.segoff = p;    p += align256((size_t)(c.S + 1) * 4);
+  L.totals = p;    p += align256(16);
+  L.slot = p;      p += align256((size_t)TK * 4);
+  L.row_src = p;   p += align256((size_t)routed_rows(c) * 4);
+  L.send_dst = p;  p += align256((size_t)c.E * 4);
+  L.recv_off = p;  p += align256((size_t)(El + 1) * 4);
+  L.recv_cnt = p;  p += align256((size_t)El * 4);
+  L.done = p;      p += 256;
+  L.h = p;         p += align256((size_t)recv_rows(c, W) * c.F * act_size(c.act_dtype));
+  L.total = p;
+  return L;
+}
+
+moe_status_t ep_validate(const moe_config_t* c, const moe_ep_t* ep) {
+  if (!c || !ep) return MOE_ERR_INVALID_ARG;
+  moe_status_t st = validate(c, true);
+  if (st != MOE_OK) return st;
+  const int W = ep->world;
+  if (W < 1 || ep->rank < 0 || ep->rank >= W) return MOE_ERR_INVALID_ARG;
+  if (W > MAX_W) return MOE_ERR_UNSUPPORTED;
+  if (c->E % W != 0 || c->S % W != 0) return MOE_ERR_INVALID_ARG;
+  if (c->n_shared != 0) return MOE_ERR_UNSUPPORTED;
+  if ((int64_t)W * c->T > INT_MAX / 2 || (int64_t)W * c->capacity > INT_MAX / 2)
+    return MOE_ERR_UNSUPPORTED;
+  if (recv_rows(*c, W) > INT_MAX / 2) return MOE_ERR_UNSUPPORTED;
+  const moe_config_t l = local_cfg(*c, W);
+  return validate(&l, true);
+}
+
+moe_status_t ws_check(const moe_config_t& c, int W, const void* ws, size_t ws_bytes) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < ep_ws_layout(c, W).total)
+    return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+moe_status_t cuda_st(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+unsigned long long timeout_ns(const moe_ep_t& ep) {
+  return ep.timeout_us ? (unsigned long long)ep.timeout_us * 1000ull : WAIT_LIMIT_NS;
+}
+
+// ---------------------------------------------------------------------------
+// device side
+
+__device__ __forceinline__ uint32_t ld_acquire_sys(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_sys(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ep_globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ bool reached(uint32_t v, uint32_t epoch) {
+  return (int32_t)(v - epoch) >= 0;
+}
+
+__device__ __forceinline__ uint32_t* peer_flags(void* const* peers, int d, size_t flags_off) {
+  return reinterpret_cast<uint32_t*>(static_cast<char*>(peers[d]) + flags_off);
+}
+
+// One thread: wait until flags[0..W) have reached `epoch` (acquire). Gives up
+// after timeout_ns, or at once when an earlier wait of this rank gave up,
+// recording MOE_ERR_TIMEOUT.
+__device__ bool wait_all(const uint32_t* flags, int W, uint32_t epoch,
+                         unsigned long long timeout_ns, uint32_t* status) {
+  const unsigned long long t0 = ep_globaltimer();
+  for (int s = 0; s < W; ++s) {
+    unsigned sleep_ns = 32;
+    while (!reached(ld_acquire_sys(flags + s), epoch)) {
+      if (*(volatile uint32_t*)status == (uint32_t)MOE_ERR_TIMEOUT ||
+          ep_globaltimer() - t0 > timeout_ns) {
+        atomicCAS(status, 0u, (uint32_t)MOE_ERR_TIMEOUT);
+        return false;
+      }
+      __nanosleep(sleep_ns);
+      if (sleep_ns < 2048) sleep_ns *= 2;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ bool timed_out(const uint32_t* status) {
+  return *(volatile const uint32_t*)status == (uint32_t)MOE_ERR_TIMEOUT;
+}
+
+// Block d writes this rank's counts into rank d's table, then sets rank d's
+// COUNTS flag for this rank (release, after a system-scope fence that orders
+// the whole block's writes before it).
+// Block 0 also zeroes the dispatch's completion counter for this step.
+__global__ void ep_publish_kernel(const int32_t* __restrict__ counts, int E, int W, int rank,
+                                  void* const* __restrict__ peers, size_t counts_off,
+                                  size_t flags_off, uint32_t epoch, uint32_t* done) {
+  pdl_wait();
+  pdl_trigger();
+  const int d = blockIdx.x;
+  if (d == 0 && threadIdx.x == 0) *done = 0u;
+  int32_t* dst = reinterpret_cast<int32_t*>(static_cast<char*>(peers[d]) + counts_off) +
+                 (size_t)rank * E;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) dst[e] = counts[e];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence_system();
+    st_release_sys(peer_flags(peers, d, flags_off) + FLAG_COUNTS * W + rank, epoch);
+  }
+}
+
+// One thread per expert e. tot = sum over senders of kept[s][e], pre = the
+// part of it from senders before this rank; the aligned totals are scanned
+// over all experts and each owner's scan restarts at its first expert.
+__global__ void __launch_bounds__(PLAN_THREADS)
+ep_plan_kernel(const int32_t* __restrict__ counts_all, const uint32_t* flags, int E, int W,
+               int rank, int C, int A, uint32_t epoch, unsigned long long timeout_ns,
+               uint32_t* status, int32_t* __restrict__ send_dst, int32_t* __restrict__ recv_off,
+               int32_t* __restrict__ recv_cnt) {
+  __shared__ long long s_scan[PLAN_THREADS];
+  __shared__ int s_ok;
+  pdl_wait();
+  pdl_trigger();
+  if (threadIdx.x == 0) s_ok = wait_all(flags + FLAG_COUNTS * W, W, epoch, timeout_ns, status);
+  __syncthreads();
+  const int e = threadIdx.x;
+  const int El = E / W;
+  long long tot = 0, pre = 0;
+  if (e < E && s_ok) {
+    for (int s = 0; s < W; ++s) {
+      // written by the peers: read from L2, never from a stale L1 line
+      const int c = min(max(__ldcg(counts_all + (size_t)s * E + e), 0), C);
+      tot += c;
+      if (s < rank) pre += c;
+    }
+  }
+  const long long aligned = (tot + A - 1) / A * A;
+  s_scan[e] = e < E ? aligned : 0;
+  __syncthreads();
+  for (int off = 1; off < PLAN_THREADS; off <<= 1) {
+    const long long v = e >= off ? s_scan[e - off] : 0;
+    __syncthreads();
+    s_scan[e] += v;
+    __syncthreads();
+  }
+  if (e < E) {
+    const int d = e / El;
+    const int first = d * El;
+    const long long first_excl = first == 0 ? 0 : s_scan[first - 1];
+    const long long base = s_scan[e] - aligned - first_excl;
+    // after a timeout every count reads as 0: nothing is sent or computed
+    send_dst[e] = (int32_t)(base + pre);
+    if (d == rank) {
+      recv_off[e - first] = (int32_t)base;
+      recv_cnt[e - first] = (int32_t)tot;
+      if (e == first + El - 1) recv_off[El] = (int32_t)(s_scan[e] - first_excl);
+    }
+  }
+}
+
+// One block per token. Warp 0 finds the destination of each kept assignment
+// (k order); the row is read once and stored to each destination. Every block
+// then counts itself done; the last one publishes this rank's DISPATCH flag to
+// every owner. After a timeout of this rank nothing is written or published.
+__global__ void __launch_bounds__(EP_THREADS)
+ep_dispatch_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ topk_idx,
+                   const int32_t* __restrict__ token_slot, const int32_t* __restrict__ offsets,
+                   const int32_t* __restrict__ send_dst, void* const* __restrict__ peers,
+                   size_t xr_off, size_t flags_off, int T, int K, int E, int El, int W, int rank,
+                   int row_vecs, int slot_end, long long n_recv, uint32_t epoch,
+                   uint32_t* status, uint32_t* done) {
+  __shared__ uint4* s_dst[MAX_K];
+  __shared__ int s_n, s_skip;
+  const int t = blockIdx.x;
+  pdl_wait();
+  pdl_trigger();
+  if (threadIdx.x == 0) s_skip = timed_out(status);
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int k = threadIdx.x;
+    uint4* dp = nullptr;
+    if (!s_skip && t < T && k < K) {
+      const int sl = token_slot[(size_t)t * K + k];
+      if (sl >= 0 && sl < slot_end) {
+        const int e = topk_idx[(size_t)t * K + k];
+        const long long row = (e >= 0 && e < E) ? (long long)send_dst[e] + (sl - offsets[e]) : -1;
+        if (row >= 0 && row < n_recv)
+          dp = reinterpret_cast<uint4*>(static_cast<char*>(peers[e / El]) + xr_off) +
+               row * row_vecs;
+        else
+          atomicCAS(status, 0u, (uint32_t)MOE_ERR_DEVICE_INPUT);
+      }
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, dp != nullptr);
+    if (dp) s_dst[__popc(m & ((1u << k) - 1u))] = dp;
+    if (k == 0) s_n = __popc(m);
+  }
+  __syncthreads();
+  const int n = s_n;
+  if (n > 0) {
+    const uint4* src = x + (size_t)t * row_vecs;
+    for (int v0 = threadIdx.x; v0 < row_vecs; v0 += EP_THREADS * EP_UNROLL) {
+      uint4 d[EP_UNROLL];
+#pragma unroll
+      for (int u = 0; u < EP_UNROLL; ++u) {
+        const int v = v0 + u * EP_THREADS;
+        if (v < row_vecs) d[u] = __ldcs(src + v);
+      }
+      for (int j = 0; j < n; ++j) {
+        uint4* dst = s_dst[j];
+#pragma unroll
+        for (int u = 0; u < EP_UNROLL; ++u) {
+          const int v = v0 + u * EP_THREADS;
+          if (v < row_vecs) dst[v] = d[u];
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence_system();   // this block's stores, before its count
+    const uint32_t prev = atomicAdd(done, 1u);
+    if (prev == gridDim.x - 1) {   // every block's stores are ordered before this point
+      __threadfence_system();
+      *done = 0u;   // ready for the next step (stream-ordered)
+      if (!s_skip)
+        for (int d = 0; d < W; ++d)
+          st_release_sys(peer_flags(peers, d, flags_off) + FLAG_DISPATCH * W + rank, epoch);
+    }
+  }
+}
+
+__global__ void ep_wait_kernel(const uint32_t* flags, int W, uint32_t epoch,
+                               unsigned long long timeout_ns, uint32_t* status) {
+  pdl_wait();
+  pdl_trigger();
+  if (threadIdx.x == 0) wait_all(flags, W, epoch, timeout_ns, status);
+}
+
+// After the grouped GEMM (pdl_wait: the GEMM has finished and its stores are
+// visible): every rank's flag `which` for this rank. Not after a timeout.
+__global__ void ep_signal_kernel(void* const* __restrict__ peers, size_t flags_off, int which,
+                                 int W, int rank, uint32_t epoch, const uint32_t* status) {
+  pdl_wait();
+  pdl_trigger();
+  const int d = threadIdx.x;
+  if (d < W && !timed_out(status)) {
+    __threadfence_system();
+    st_release_sys(peer_flags(peers, d, flags_off) + which * W + rank, epoch);
+  }
+}
+
+// out[t] = sum over kept k (k order) of w[t,k] * y_owner[row], fp32 FMA from
+// 0, one rounding: the arithmetic of the one-rank combine, with the rows read
+// in place from their owners.
+template <bool BF16>
+__global__ void __launch_bounds__(EP_THREADS)
+ep_combine_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ token_slot,
+                  const float* __restrict__ topk_w, const int32_t* __restrict__ offsets,
+                  const int32_t* __restrict__ send_dst, void* const* __restrict__ peers,
+                  size_t y_off, uint4* __restrict__ out, int K, int E, int El, int row_vecs,
+                  int slot_end, long long n_recv, uint32_t* status) {
+  __shared__ const uint4* s_src[MAX_K];
+  __shared__ float s_w[MAX_K];
+  __shared__ int s_n;
+  const int t = blockIdx.x;
+  pdl_wait();
+  pdl_trigger();
+  if (threadIdx.x < 32) {
+    const int k = threadIdx.x;
+    const uint4* sp = nullptr;
+    float wt = 0.f;
+    if (k < K) {
+      const int sl = token_slot[(size_t)t * K + k];
+      wt = topk_w[(size_t)t * K + k];
+      if (sl >= 0 && sl < slot_end) {
+        const int e = topk_idx[(size_t)t * K + k];
+        const long long row = (e >= 0 && e < E) ? (long long)send_dst[e] + (sl - offsets[e]) : -1;
+        if (row >= 0 && row < n_recv)
+          sp = reinterpret_cast<const uint4*>(static_cast<char*>(peers[e / El]) + y_off) +
+               row * row_vecs;
+        else
+          atomicCAS(status, 0u, (uint32_t)MOE_ERR_DEVICE_INPUT);
+      }
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, sp != nullptr);
+    if (sp) {
+      const int pos = __popc(m & ((1u << k) - 1u));
+      s_src[pos] = sp;
+      s_w[pos] = wt;
+    }
+    if (k == 0) s_n = __popc(m);
+  }
+  __syncthreads();
+  const int n = s_n;
+  constexpr int LANES = BF16 ? 8 : 4;
+  uint4* dst = out + (size_t)t * row_vecs;
+  for (int v0 = threadIdx.x; v0 < row_vecs; v0 += EP_THREADS * 2) {
+    float acc[2][LANES];
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int i = 0; i < LANES; ++i) acc[u][i] = 0.f;
+    for (int k = 0; k < n; k += 4) {
+      uint4 d[4][2];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int v = v0 + u * EP_THREADS;
+          // rows written by another kernel, possibly on another GPU: read via L2
+          d[j][u] = (k + j < n && v < row_vecs) ? __ldcg(s_src[k + j] + v)
+                                                : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (k + j >= n) continue;
+        const float wk = s_w[k + j];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (BF16) {
+            float f[8];
+            unpack_bf16x8(d[j][u], f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[u][i] = fmaf(wk, f[i], acc[u][i]);
+          } else {
+            acc[u][0] = fmaf(wk, __uint_as_float(d[j][u].x), acc[u][0]);
+            acc[u][1] = fmaf(wk, __uint_as_float(d[j][u].y), acc[u][1]);
+            acc[u][2] = fmaf(wk, __uint_as_float(d[j][u].z), acc[u][2]);
+            acc[u][3] = fmaf(wk, __uint_as_float(d[j][u].w), acc[u][3]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int v = v0 + u * EP_THREADS;
+      if (v >= row_vecs) continue;
+      uint4 o;
+      if (BF16) {
+        o.x = pack_bf16x2(acc[u][0], acc[u][1]);
+        o.y = pack_bf16x2(acc[u][2], acc[u][3]);
+        o.z = pack_bf16x2(acc[u][4], acc[u][5]);
+        o.w = pack_bf16x2(acc[u][6], acc[u][7]);
+      } else {
+        o.x = __float_as_uint(acc[u][0]);
+        o.y = __float_as_uint(acc[u][1]);
+        o.z = __float_as_uint(acc[u][2]);
+        o.w = __float_as_uint(acc[u][3]);
+      }
+      __stcs(dst + v, o);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+
+struct Ptrs {
+  int32_t *topk_idx, *counts, *overflow, *offsets, *segoff, *slot, *row_src, *totals, *blk;
+  float* topk_w;
+  int32_t *send_dst, *recv_off, *recv_cnt;
+  uint32_t *status, *done;
+  char* h;
+};
+
+Ptrs ws_ptrs(const moe_config_t& c, int W, void* ws) {
+  const EpWs L = ep_ws_layout(c, W);
+  char* b = static_cast<char*>(ws);
+  Ptrs p;
+  p.status = reinterpret_cast<uint32_t*>(b);
+  p.blk = reinterpret_cast<int32_t*>(b + L.blk_cnt);
+  p.topk_idx = reinterpret_cast<int32_t*>(b + L.topk_idx);
+  p.topk_w = reinterpret_cast<float*>(b + L.topk_w);
+  p.counts = reinterpret_cast<int32_t*>(b + L.counts);
+  p.overflow = reinterpret_cast<int32_t*>(b + L.overflow);
+  p.offsets = reinterpret_cast<int32_t*>(b + L.offsets);
+  p.segoff = reinterpret_cast<int32_t*>(b + L.segoff);
+  p.totals = reinterpret_cast<int32_t*>(b + L.totals);
+  p.slot = reinterpret_cast<int32_t*>(b + L.slot);
+  p.row_src = reinterpret_cast<int32_t*>(b + L.row_src);
+  p.send_dst = reinterpret_cast<int32_t*>(b + L.send_dst);
+  p.recv_off = reinterpret_cast<int32_t*>(b + L.recv_off);
+  p.recv_cnt = reinterpret_cast<int32_t*>(b + L.recv_cnt);
+  p.done = reinterpret_cast<uint32_t*>(b + L.done);
+  p.h = b + L.h;
+  return p;
+}
+
+moe_status_t common_checks(const moe_config_t* cfg, const moe_ep_t* ep, const void* sym,
+                           void* const* peers, const void* ws, size_t ws_bytes) {
+  moe_status_t st = ep_validate(cfg, ep);
+  if (st != MOE_OK) return st;
+  if (ep->epoch == 0u || !sym || !peers) return MOE_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(sym) & 255u) return MOE_ERR_INVALID_ARG;
+  return ws_check(*cfg, ep->world, ws, ws_bytes);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int64_t moe_ep_recv_rows(const moe_config_t* cfg, int32_t world) {
+  moe_ep_t ep = {world, 0, 1u, 0u};
+  if (ep_validate(cfg, &ep) != MOE_OK) return -1;
+  return recv_rows(*cfg, world);
+}
+
+size_t moe_ep_symmetric_bytes(const moe_config_t* cfg, int32_t world) {
+  moe_ep_t ep = {world, 0, 1u, 0u};
+  if (ep_validate(cfg, &ep) != MOE_OK) return 0;
+  return sym_layout(*cfg, world).total;
+}
+
+size_t moe_ep_workspace_bytes(const moe_config_t* cfg, int32_t world) {
+  moe_ep_t ep = {world, 0, 1u, 0u};
+  if (ep_validate(cfg, &ep) != MOE_OK) return 0;
+  return ep_ws_layout(*cfg, world).total;
+}
+
+moe_status_t moe_ep_check(const moe_config_t* cfg, const moe_ep_t* ep) {
+  moe_status_t st = ep_validate(cfg, ep);
+  if (st != MOE_OK) return st;
+  return ep->epoch == 0u ? MOE_ERR_INVALID_ARG : MOE_OK;
+}
+
+moe_status_t moe_ep_aux(const moe_config_t* cfg, const moe_ep_t* ep, void* sym, void* ws,
+                        moe_ep_aux_t* aux) {
+  moe_status_t st = ep_validate(cfg, ep);
+  if (st != MOE_OK) return st;
+  if (!sym || !ws || !aux) return MOE_ERR_INVALID_ARG;
+  const Ptrs p = ws_ptrs(*cfg, ep->world, ws);
+  const SymLayout S = sym_layout(*cfg, ep->world);
+  char* sb = static_cast<char*>(sym);
+  moe_ep_aux_t a = {};
+  a.topk_idx = p.topk_idx;
+  a.expert_counts = p.counts;
+  a.overflow = p.overflow;
+  a.expert_offsets = p.offsets;
+  a.segment_offsets = p.segoff;
+  a.token_slot = p.slot;
+  a.row_src = p.row_src;
+  a.totals = p.totals;
+  a.topk_w = p.topk_w;
+  a.counts_all = reinterpret_cast<int32_t*>(sb + S.counts);
+  a.flags = reinterpret_cast<uint32_t*>(sb + S.flags);
+  a.send_dst_row = p.send_dst;
+  a.recv_offsets = p.recv_off;
+  a.recv_counts = p.recv_cnt;
+  a.xr = sb + S.xr;
+  a.h = p.h;
+  a.y = sb + S.y;
+  *aux = a;
+  return MOE_OK;
+}
+
+moe_status_t moe_ep_symmetric_init(const moe_config_t* cfg, int32_t world, void* sym,
+                                   size_t sym_bytes, void* stream) {
+  moe_ep_t ep = {world, 0, 1u, 0u};
+  moe_status_t st = ep_validate(cfg, &ep);
+  if (st != MOE_OK) return st;
+  const SymLayout S = sym_layout(*cfg, world);
+  if (!sym || (reinterpret_cast<uintptr_t>(sym) & 255u)) return MOE_ERR_INVALID_ARG;
+  if (sym_bytes < S.total) return MOE_ERR_WORKSPACE;
+  return cuda_st(cudaMemsetAsync(sym, 0, S.xr, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_ep_route(const moe_config_t* cfg, const moe_ep_t* ep, const float* logits,
+                          void* sym, void* const* peers, void* ws, size_t ws_bytes,
+                          void* stream) {
+  moe_status_t st = common_checks(cfg, ep, sym, peers, ws, ws_bytes);
+  if (st != MOE_OK) return st;
+  if (cfg->T > 0 && !logits) return MOE_ERR_INVALID_ARG;
+  const moe_config_t& c = *cfg;
+  const int W = ep->world;
+  const Ptrs p = ws_ptrs(c, W, ws);
+  const SymLayout S = sym_layout(c, W);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = cuda_st(launch_route(c, logits, p.topk_idx, p.topk_w, p.counts, p.overflow, p.offsets,
+                            p.segoff, p.slot, p.row_src, p.totals, p.blk, routed_rows(c), s));
+  if (st != MOE_OK) return st;
+  return cuda_st(launch_pdl(ep_publish_kernel, dim3(W), dim3(256), 0, s,
+                            (const int32_t*)p.counts, c.E, W, ep->rank, peers, S.counts, S.flags,
+                            ep->epoch, p.done));
+}
+
+moe_status_t moe_ep_dispatch(const moe_config_t* cfg, const moe_ep_t* ep, const void* x,
+                             void* sym, void* const* peers, void* ws, size_t ws_bytes,
+                             void* stream) {
+  moe_status_t st = common_checks(cfg, ep, sym, peers, ws, ws_bytes);
+  if (st != MOE_OK) return st;
+  if (cfg->T > 0 && (!x || !aligned16(x))) return MOE_ERR_INVALID_ARG;
+  const moe_config_t& c = *cfg;
+  const int W = ep->world;
+  const Ptrs p = ws_ptrs(c, W, ws);
+  const SymLayout S = sym_layout(c, W);
+  char* sb = static_cast<char*>(sym);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = cuda_st(launch_pdl(ep_plan_kernel, dim3(1), dim3(PLAN_THREADS), 0, s,
+                          (const int32_t*)(sb + S.counts), (const uint32_t*)(sb + S.flags), c.E,
+                          W, ep->rank, c.capacity, c.row_align, ep->epoch, timeout_ns(*ep),
+                          p.status, p.send_dst, p.recv_off, p.recv_cnt));
+  if (st != MOE_OK) return st;
+  const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
+  // at least one block, so that the DISPATCH flags are published with T = 0 too
+  return cuda_st(launch_pdl(ep_dispatch_kernel, dim3((unsigned)std::max(c.T, 1)),
+                            dim3(EP_THREADS), 0, s, static_cast<const uint4*>(x),
+                            (const int32_t*)p.topk_idx, (const int32_t*)p.slot,
+                            (const int32_t*)p.offsets, (const int32_t*)p.send_dst, peers, S.xr,
+                            S.flags, c.T, c.K, c.E, c.E / W, W, ep->rank, row_vecs,
+                            (int)routed_rows(c), (long long)recv_rows(c, W), ep->epoch, p.status,
+                            p.done));
+}
+
+moe_status_t moe_ep_expert_mlp(const moe_config_t* cfg, const moe_ep_t* ep,
+                               const void* w_gu_local, const void* w_d_local, void* sym,
+                               void* const* peers, void* ws, size_t ws_bytes, void* stream) {
+  moe_status_t st = common_checks(cfg, ep, sym, peers, ws, ws_bytes);
+  if (st != MOE_OK) return st;
+  if (!w_gu_local || !w_d_local || !aligned16(w_gu_local) || !aligned16(w_d_local))
+    return MOE_ERR_INVALID_ARG;
+  const moe_config_t& c = *cfg;
+  const int W = ep->world;
+  const Ptrs p = ws_ptrs(c, W, ws);
+  const SymLayout S = sym_layout(c, W);
+  char* sb = static_cast<char*>(sym);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = cuda_st(launch_pdl(ep_wait_kernel, dim3(1), dim3(32), 0, s,
+                          (const uint32_t*)(sb + S.flags) + FLAG_DISPATCH * W, W, ep->epoch,
+                          timeout_ns(*ep), p.status));
+  if (st != MOE_OK) return st;
+  const moe_config_t l = local_cfg(c, W);
+  const int64_t R = recv_rows(c, W);
+  if (c.act_dtype == MOE_BF16)
+    st = launch_mlp_bf16_tc(l, sb + S.xr, p.recv_off, p.recv_cnt, w_gu_local, w_d_local, p.h,
+                            sb + S.y, R, p.status, s);
+  else
+    st = cuda_st(launch_mlp_f32(l, reinterpret_cast<const float*>(sb + S.xr), p.recv_off,
+                                p.recv_cnt, static_cast<const float*>(w_gu_local),
+                                static_cast<const float*>(w_d_local),
+                                reinterpret_cast<float*>(p.h), reinterpret_cast<float*>(sb + S.y),
+                                R, s));
+  if (st != MOE_OK) return st;
+  return cuda_st(launch_pdl(ep_signal_kernel, dim3(1), dim3(MAX_W), 0, s, peers, S.flags,
+                            (int)FLAG_Y, W, ep->rank, ep->epoch, (const uint32_t*)p.status));
+}
+
+moe_status_t moe_ep_combine(const moe_config_t* cfg, const moe_ep_t* ep, void* sym,
+                            void* const* peers, void* out, void* ws, size_t ws_bytes,
+                            void* stream) {
+  moe_status_t st = common_checks(cfg, ep, sym, peers, ws, ws_bytes);
+  if (st != MOE_OK) return st;
+  if (cfg->T > 0 && (!out || !aligned16(out))) return MOE_ERR_INVALID_ARG;
+  const moe_config_t& c = *cfg;
+  const int W = ep->world;
+  const Ptrs p = ws_ptrs(c, W, ws);
+  const SymLayout S = sym_layout(c, W);
+  char* sb = static_cast<char*>(sym);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = cuda_st(launch_pdl(ep_wait_kernel, dim3(1), dim3(32), 0, s,
+                          (const uint32_t*)(sb + S.flags) + FLAG_Y * W, W, ep->epoch,
+                          timeout_ns(*ep), p.status));
+  if (st != MOE_OK || c.T == 0) return st;
+  const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
+  auto kernel = c.act_dtype == MOE_BF16 ? ep_combine_kernel<true> : ep_combine_kernel<false>;
+  return cuda_st(launch_pdl(kernel, dim3(c.T), dim3(EP_THREADS), 0, s,
+                            (const int32_t*)p.topk_idx, (const int32_t*)p.slot,
+                            (const float*)p.topk_w, (const int32_t*)p.offsets,
+                            (const int32_t*)p.send_dst, peers, S.y, static_cast<uint4*>(out),
+                            c.K, c.E, c.E / W, row_vecs, (int)routed_rows(c),
+                            (long long)recv_rows(c, W), p.status));
+}
+
+moe_status_t moe_ep_layer_forward(const moe_config_t* cfg, const moe_ep_t* ep,
+                                  const float* logits, const void* x, const void* w_gu_local,
+                                  const void* w_d_local, void* sym, void* const* peers,
+                                  void* out, moe_ep_aux_t* aux, void* ws, size_t ws_bytes,
+                                  void* stream) {
+  moe_status_t st = common_checks(cfg, ep, sym, peers, ws, ws_bytes);
+  if (st != MOE_OK) return st;
+  if (aux && (st = moe_ep_aux(cfg, ep, sym, ws, aux)) != MOE_OK) return st;
+  if ((st = moe_ep_route(cfg, ep, logits, sym, peers, ws, ws_bytes, stream)) != MOE_OK) return st;
+  if ((st = moe_ep_dispatch(cfg, ep, x, sym, peers, ws, ws_bytes, stream)) != MOE_OK) return st;
+  if ((st = moe_ep_expert_mlp(cfg, ep, w_gu_local, w_d_local, sym, peers, ws, ws_bytes,
+                              stream)) != MOE_OK)
+    return st;
+  return moe_ep_combine(cfg, ep, sym, peers, out, ws, ws_bytes, stream);
+}
+
+moe_status_t moe_ep_sym_alloc(size_t bytes, void** ptr) {
+  if (!ptr || bytes == 0) return MOE_ERR_INVALID_ARG;
+  return cuda_st(cudaMalloc(ptr, bytes));
+}
+
+moe_status_t moe_ep_sym_free(void* ptr) { return cuda_st(cudaFree(ptr)); }
+
+moe_status_t moe_ipc_get_handle(void* ptr, uint8_t handle[64]) {
+  static_assert(sizeof(cudaIpcMemHandle_t) == 64, "CUDA IPC handles are 64 bytes");
+  if (!ptr || !handle) return MOE_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t h;
+  if (cudaIpcGetMemHandle(&h, ptr) != cudaSuccess) return MOE_ERR_CUDA;
+  std::memcpy(handle, &h, sizeof(h));
+  return MOE_OK;
+}
+
+moe_status_t moe_ipc_open(const uint8_t handle[64], void** ptr) {
+  if (!handle || !ptr) return MOE_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t h;
+  std::memcpy(&h, handle, sizeof(h));
+  return cuda_st(cudaIpcOpenMemHandle(ptr, h, cudaIpcMemLazyEnablePeerAccess));
+}
+
+moe_status_t moe_ipc_close(void* ptr) {
+  if (!ptr) return MOE_ERR_INVALID_ARG;
+  return cuda_st(cudaIpcCloseMemHandle(ptr));
+}
+
+}  // extern "C"

@@ -1,0 +1,176 @@
+"""Host-side checks of the expert-parallel ABI (no GPU needed): sizes against
+the oracle, validation, the ctypes mirrors of the header's structs, argument
+errors caught before any launch, and the handle exchange of a process group
+(gloo, two ranks)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import combine_moe_route_13_b200 as M
+from combine_moe_route_13_b200 import ep as EP
+from oracle import moe_oracle as O
+from oracle import moe_oracle_ep as P
+import workloads as W
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "moe_ep.h")
+
+
+def cfg_of(name, **kw):
+    w = W.WORKLOADS[name]
+    d = dict(T=w.T, H=w.H, E=w.E, K=w.K, F=w.F, S=w.S,
+             capacity=O.capacity(w.T, w.K, w.E, w.cf), row_align=w.row_align, act=w.act)
+    d.update(kw)
+    return M.make_config(**d)
+
+
+@pytest.mark.parametrize("name,world", [("mixtral", 2), ("mixtral", 8), ("dsv3", 8), ("dsv3", 4),
+                                        ("skewed", 8), ("kimi", 16), ("tiny", 2), ("mixtral", 1)])
+def test_recv_rows_match_oracle(name, world):
+    c = cfg_of(name)
+    assert M.moe_ep_recv_rows(c, world) == P.recv_rows_max(c.T, c.K, c.E, c.capacity,
+                                                            c.row_align, world)
+    R = M.moe_ep_recv_rows(c, world)
+    es = 4 if c.act_dtype == M.MOE_F32 else 2
+    sym = M.moe_ep_symmetric_bytes(c, world)
+    assert sym >= 2 * R * c.H * es + world * c.E * 4 + 3 * world * 4
+    assert M.moe_ep_workspace_bytes(c, world) >= R * c.F * es
+
+
+def test_one_rank_sizes_equal_the_one_rank_layer():
+    c = cfg_of("mixtral")
+    assert M.moe_ep_recv_rows(c, 1) == M.moe_max_rows(c)
+
+
+@pytest.mark.parametrize("kw,world,rank,epoch,code", [
+    (dict(), 3, 0, 1, M.MOE_ERR_INVALID_ARG),            # E % W
+    (dict(S=2), 4, 0, 1, M.MOE_ERR_INVALID_ARG),         # S % W
+    (dict(), 0, 0, 1, M.MOE_ERR_INVALID_ARG),
+    (dict(), 2, 2, 1, M.MOE_ERR_INVALID_ARG),            # rank >= W
+    (dict(), 2, -1, 1, M.MOE_ERR_INVALID_ARG),
+    (dict(), 2, 0, 0, M.MOE_ERR_INVALID_ARG),            # epoch 0
+    (dict(n_shared=1), 2, 0, 1, M.MOE_ERR_UNSUPPORTED),
+    (dict(H=4100), 2, 0, 1, M.MOE_ERR_UNSUPPORTED),      # what the one-rank GEMM rejects
+    (dict(), 2, 1, 7, M.MOE_OK),
+])
+def test_check(kw, world, rank, epoch, code):
+    c = cfg_of("mixtral", **kw)
+    assert M.moe_ep_check(c, M.make_ep(world, rank, epoch)) == code
+
+
+def test_too_many_ranks_unsupported():
+    c = M.make_config(T=64, H=256, E=128, K=2, F=256, S=128, capacity=8)
+    assert M.moe_ep_check(c, M.make_ep(128, 0, 1)) == M.MOE_ERR_UNSUPPORTED
+    assert M.moe_ep_check(c, M.make_ep(64, 63, 1)) == M.MOE_OK
+    assert M.moe_ep_recv_rows(c, 128) == -1
+    assert M.moe_ep_symmetric_bytes(c, 128) == 0
+
+
+def _fields(struct):
+    src = open(HEADER).read()
+    body = re.search(r"typedef struct \{([^{}]*)\} " + struct + ";", src).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    return re.findall(r"\*?\b([A-Za-z_]+)\s*[,;]", body)
+
+
+def test_structs_match_header():
+    assert [n for n, _ in M.MoeEp._fields_] == _fields("moe_ep_t")
+    assert ctypes.sizeof(M.MoeEp) == 16
+    assert [n for n, _ in M.MoeEpAux._fields_] == _fields("moe_ep_aux_t")
+
+
+def test_aux_layout_is_inside_the_buffers():
+    c = cfg_of("mixtral")
+    world = 4
+    sym, ws = 1 << 40, 1 << 41   # host-only: nothing is dereferenced
+    aux = M.MoeEpAux()
+    ep = M.make_ep(world, 2, 1)
+    assert M.LIB.moe_ep_aux(ctypes.byref(c), ctypes.byref(ep), sym, ws, ctypes.byref(aux)) == M.MOE_OK
+    nsym = M.moe_ep_symmetric_bytes(c, world)
+    nws = M.moe_ep_workspace_bytes(c, world)
+    R = M.moe_ep_recv_rows(c, world)
+    for f in ("counts_all", "flags", "xr", "y"):
+        assert sym <= getattr(aux, f) < sym + nsym, f
+    assert aux.y + R * c.H * 2 <= sym + nsym
+    for f in ("topk_idx", "expert_counts", "token_slot", "send_dst_row", "recv_offsets",
+              "recv_counts", "h"):
+        v = getattr(aux, f)
+        assert ws + 256 <= v < ws + nws and v % 256 == 0, f
+    assert aux.h + R * c.F * 2 <= ws + nws
+
+
+def test_entry_points_reject_bad_arguments_before_any_launch():
+    lib = M.LIB
+    c = cfg_of("tiny", S=2)
+    ep = M.make_ep(2, 0, 1)
+    big = 1 << 30
+    fake = 1 << 40
+    # no symmetric region / peers
+    assert lib.moe_ep_route(ctypes.byref(c), ctypes.byref(ep), fake, None, fake, fake, big, None) \
+        == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_dispatch(ctypes.byref(c), ctypes.byref(ep), fake, fake, None, fake, big,
+                               None) == M.MOE_ERR_INVALID_ARG
+    # workspace too small, or misaligned
+    assert lib.moe_ep_combine(ctypes.byref(c), ctypes.byref(ep), fake, fake, fake, fake, 256,
+                              None) == M.MOE_ERR_WORKSPACE
+    assert lib.moe_ep_expert_mlp(ctypes.byref(c), ctypes.byref(ep), fake, fake, fake, fake,
+                                 fake + 16, big, None) == M.MOE_ERR_WORKSPACE
+    # weights missing
+    assert lib.moe_ep_expert_mlp(ctypes.byref(c), ctypes.byref(ep), None, fake, fake, fake, fake,
+                                 big, None) == M.MOE_ERR_INVALID_ARG
+    # epoch 0 and a bad config
+    ep0 = M.make_ep(2, 0, 0)
+    assert lib.moe_ep_route(ctypes.byref(c), ctypes.byref(ep0), fake, fake, fake, fake, big,
+                            None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_layer_forward(None, ctypes.byref(ep), fake, fake, fake, fake, fake, fake,
+                                    fake, None, fake, big, None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_symmetric_init(ctypes.byref(c), 2, fake, 16, None) == M.MOE_ERR_WORKSPACE
+    assert lib.moe_ipc_open(None, None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_sym_alloc(0, None) == M.MOE_ERR_INVALID_ARG
+
+
+# ---------------------------------------------------------------- handle exchange (gloo)
+
+def _exchange_worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        own = bytes([rank]) * 64
+        opened = []
+
+        def open_handle(h):
+            opened.append(h[0])
+            return 1000 + h[0]
+
+        addrs = EP.exchange_addresses(own, 7 + rank, open_handle)
+        q.put((rank, addrs, opened))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_handle_exchange_two_ranks():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_exchange_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = dict()
+    for _ in range(2):
+        r, addrs, opened = q.get(timeout=120)
+        got[r] = (addrs, opened)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    # rank r keeps its own address and opens the other rank's handle, in rank order
+    assert got[0] == ([7, 1001], [1])
+    assert got[1] == ([1000, 8], [0])
