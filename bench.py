@@ -484,6 +484,131 @@ def run_reference(args, wl: W.Workload, world, rank):
     return 0
 
 
+def run_ep_emulated(args, wl: W.Workload, world_ep: int):
+    """The expert-parallel layer with `world_ep` ranks emulated on this one GPU
+    (EpOnOneDevice): every rank has its own T tokens, E/W experts and buffers,
+    and the four steps run for every rank in turn. The timed step is all
+    ranks' layers, so value = W*T tokens per step time. The exchanges move
+    through this GPU's HBM instead of NVLink; the line reports each phase's
+    time and bytes so that the NVLink time of a real group can be put beside
+    it (remote bytes / link bandwidth)."""
+    import combine_moe_route_13_b200 as M
+    from combine_moe_route_13_b200.ep import EpOnOneDevice
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    peaks = load_peaks()
+    Wn = world_ep
+    C = M.moe_capacity(wl.T, wl.K, wl.E, wl.cf)
+    cfg = M.make_config(wl.T, wl.H, wl.E, wl.K, wl.F, wl.S, C, wl.row_align, wl.act)
+    st = M.moe_ep_check(cfg, M.make_ep(Wn, 0, 1))
+    if st != M.MOE_OK:
+        raise SystemExit(f"unsupported expert-parallel workload: {M.status_string(st)}")
+    full = W.make_inputs(wl, seed=0, device=device)
+    inps = [full] + [W.make_inputs(wl, seed=r, device=device, weights=False) for r in range(1, Wn)]
+    El = wl.E // Wn
+    wg = [full["w_gu"][r * El:(r + 1) * El] for r in range(Wn)]
+    wd = [full["w_d"][r * El:(r + 1) * El] for r in range(Wn)]
+    logits = [i["logits"] for i in inps]
+    xs = [i["x"] for i in inps]
+    outs = [torch.empty(wl.T, wl.H, dtype=wl.torch_act, device=device) for _ in range(Wn)]
+    emu = EpOnOneDevice(cfg, Wn, device)
+    flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        emu.forward(logits, xs, wg, wd, outs)
+
+    step()
+    torch.cuda.synchronize()
+    for r in range(Wn):
+        if emu.status(r) != M.MOE_OK:
+            raise SystemExit(f"rank {r}: {M.status_string(emu.status(r))}")
+    N = [int(emu.views(r)["totals"][1]) for r in range(Wn)]
+    clocks = Clocks(0)
+    clocks.start()
+    times = time_steps(step, args.steps, args.warmup, flush_buf, stream)
+    clk = clocks.stop()
+    ms = float(np.mean(times))
+
+    # phases, all ranks each: events between the four steps
+    c = cfg
+    ph = {n: [] for n in ("route", "dispatch", "expert_mlp", "combine")}
+    for it in range(max(args.steps // 4, 3) + 1):
+        flush_l2(flush_buf)
+        emu.epoch += 1
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        ev[0].record(stream)
+        for r in range(Wn):
+            M.moe_ep_route(c, emu.ep(r), logits[r], emu.sym[r], emu.peers, emu.ws[r])
+        ev[1].record(stream)
+        for r in range(Wn):
+            M.moe_ep_dispatch(c, emu.ep(r), xs[r], emu.sym[r], emu.peers, emu.ws[r])
+        ev[2].record(stream)
+        for r in range(Wn):
+            M.moe_ep_expert_mlp(c, emu.ep(r), wg[r], wd[r], emu.sym[r], emu.peers, emu.ws[r])
+        ev[3].record(stream)
+        for r in range(Wn):
+            M.moe_ep_combine(c, emu.ep(r), emu.sym[r], emu.peers, outs[r], emu.ws[r])
+        ev[4].record(stream)
+        torch.cuda.synchronize()
+        if it:
+            for i, n in enumerate(ph):
+                ph[n].append(ev[i].elapsed_time(ev[i + 1]))
+    ph = {n: float(np.mean(v)) for n, v in ph.items()}
+    for r in range(Wn):
+        if emu.status(r) != M.MOE_OK:
+            raise SystemExit(f"rank {r} after timing: {M.status_string(emu.status(r))}")
+    s_ = 4 if wl.act == "f32" else 2
+    Nt = sum(N)
+    T, H, F, K = wl.T, wl.H, wl.F, wl.K
+    disp_bytes = Wn * (T * H * s_ + T * K * 8) + Nt * H * s_
+    comb_bytes = Wn * (T * H * s_ + T * K * 12) + Nt * H * s_
+    # rows whose owner is another rank: they would cross NVLink in a real group
+    remote = 0
+    for r in range(Wn):
+        v = emu.views(r)
+        kept = np.minimum(v["expert_counts"].cpu().numpy(), C)
+        remote += int(kept.sum() - kept[r * El:(r + 1) * El].sum())
+    flops = 6.0 * Nt * H * F
+    hbm = peaks["hbm_gbs"]
+    tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    mlp_tflops = flops / (ph["expert_mlp"] * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": Wn * T / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if wl.act == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": f"{wl.name}_ep{Wn}_one_device", "T_per_rank": T, "H": H,
+                   "E": wl.E, "K": K, "F": F, "S": wl.S, "cf": wl.cf, "capacity": C,
+                   "row_align": wl.row_align, "ranks": Wn, "effective_tokens": Nt,
+                   "parallelism": f"ep{Wn} emulated on one GPU (exchanges through local HBM)",
+                   "l2": "flushed (256 MB write) before every step"},
+        "e2e": None,
+        "gpu_launches": None,
+        "roofline": {"bound": "tensor", "kernel": "expert_mlp (all ranks' grouped GEMMs)",
+                     "achieved": mlp_tflops, "peak": tensor_peak, "unit": "TFLOP/s",
+                     "frac": mlp_tflops / tensor_peak,
+                     "peak_kind": f"bf16_tflops_sustained ({peaks['source']})", "traffic": None},
+        "kernels": {
+            "phase_timing": "CUDA events around each step for all ranks (wait kernels included)",
+            "route_us": ph["route"] * 1e3,
+            "dispatch_us": ph["dispatch"] * 1e3,
+            "dispatch_gbs": disp_bytes / (ph["dispatch"] * 1e-3) / 1e9,
+            "expert_mlp_us": ph["expert_mlp"] * 1e3,
+            "expert_mlp_tflops": mlp_tflops,
+            "combine_us": ph["combine"] * 1e3,
+            "combine_gbs": comb_bytes / (ph["combine"] * 1e-3) / 1e9,
+            "remote_rows": remote,
+            "remote_bytes_each_way": remote * H * s_,
+            "nvlink_us_each_way_at_770_gbs_per_gpu": remote * H * s_ / Wn / 770e9 * 1e6,
+        },
+        "clocks": clk,
+        "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -503,6 +628,8 @@ def main(argv=None):
                     help="fp8 block-scaled payload and expert GEMMs (moe_layer_forward_fp8)")
     ap.add_argument("--shared", action="store_true",
                     help="add one shared expert of the routed width (as DeepSeek-V3 and Kimi-K2 have)")
+    ap.add_argument("--ep-emulate", type=int, default=0, metavar="W",
+                    help="expert-parallel layer with W ranks emulated on this one GPU")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         raise SystemExit("--warmup must be >= 3")
@@ -514,6 +641,10 @@ def main(argv=None):
     world, rank, local = dist_env()
     if args.impl == "reference":
         return run_reference(args, wl, world, rank)
+    if args.ep_emulate:
+        if world > 1 or args.fp8 or args.shared:
+            raise SystemExit("--ep-emulate runs on one GPU, bf16/f32, without a shared expert")
+        return run_ep_emulated(args, wl, args.ep_emulate)
 
     import torch.distributed as dist
     if world > 1:
