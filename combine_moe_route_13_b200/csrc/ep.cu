@@ -22,8 +22,8 @@
 //   plan      wait for all COUNTS flags; kept = min(count, C); scans give
 //             send_dst_row[E], recv_offsets[E/W+1], recv_counts[E/W]
 //   dispatch  one block per token: its row is read once and written to the
-//             owners of its kept experts; the last block to finish sets every
-//             owner's DISPATCH flag for this rank
+//             owners of its kept experts
+//   signal    every owner's DISPATCH flag for this rank, after the dispatch
 //   wait      one thread: all DISPATCH flags (then the grouped GEMM of
 //             moe_expert_mlp over the local experts)
 //   signal    every rank's Y flag for this rank, after the GEMM
@@ -56,7 +56,7 @@ struct SymLayout {
 struct EpWs {
   size_t blk_cnt = 0, topk_idx = 0, topk_w = 0, counts = 0, overflow = 0, offsets = 0;
   size_t segoff = 0, totals = 0, slot = 0, row_src = 0;
-  size_t send_dst = 0, recv_off = 0, recv_cnt = 0, done = 0, h = 0, total = 0;
+  size_t send_dst = 0, recv_off = 0, recv_cnt = 0, h = 0, total = 0;
 };
 
 int64_t recv_rows(const moe_config_t& c, int W) {
@@ -111,7 +111,6 @@ EpWs ep_ws_layout(const moe_config_t& c, int W) {
   L.send_dst = p;  p += align256((size_t)c.E * 4);
   L.recv_off = p;  p += align256((size_t)(El + 1) * 4);
   L.recv_cnt = p;  p += align256((size_t)El * 4);
-  L.done = p;      p += 256;
   L.h = p;         p += align256((size_t)recv_rows(c, W) * c.F * act_size(c.act_dtype));
   L.total = p;
   return L;
@@ -200,14 +199,12 @@ __device__ __forceinline__ bool timed_out(const uint32_t* status) {
 // Block d writes this rank's counts into rank d's table, then sets rank d's
 // COUNTS flag for this rank (release, after a system-scope fence that orders
 // the whole block's writes before it).
-// Block 0 also zeroes the dispatch's completion counter for this step.
 __global__ void ep_publish_kernel(const int32_t* __restrict__ counts, int E, int W, int rank,
                                   void* const* __restrict__ peers, size_t counts_off,
-                                  size_t flags_off, uint32_t epoch, uint32_t* done) {
+                                  size_t flags_off, uint32_t epoch) {
   pdl_wait();
   pdl_trigger();
   const int d = blockIdx.x;
-  if (d == 0 && threadIdx.x == 0) *done = 0u;
   int32_t* dst = reinterpret_cast<int32_t*>(static_cast<char*>(peers[d]) + counts_off) +
                  (size_t)rank * E;
   for (int e = threadIdx.x; e < E; e += blockDim.x) dst[e] = counts[e];
@@ -267,74 +264,70 @@ ep_plan_kernel(const int32_t* __restrict__ counts_all, const uint32_t* flags, in
   }
 }
 
-// One block per token. Warp 0 finds the destination of each kept assignment
-// (k order); the row is read once and stored to each destination. Every block
-// then counts itself done; the last one publishes this rank's DISPATCH flag to
-// every owner. After a timeout of this rank nothing is written or published.
+// One block per token. The peer table is staged in shared memory while warp 0
+// loads the token's slots, experts and their layout entries; warp 0 then packs
+// the destinations of the kept assignments (k order); the row is read once and
+// stored to each destination. After a timeout of this rank nothing is written.
+// The DISPATCH flags are raised by ep_signal_kernel once this grid has
+// finished (its stores are then complete and visible to the signalling grid).
 __global__ void __launch_bounds__(EP_THREADS)
 ep_dispatch_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ topk_idx,
                    const int32_t* __restrict__ token_slot, const int32_t* __restrict__ offsets,
                    const int32_t* __restrict__ send_dst, void* const* __restrict__ peers,
-                   size_t xr_off, size_t flags_off, int T, int K, int E, int El, int W, int rank,
-                   int row_vecs, int slot_end, long long n_recv, uint32_t epoch,
-                   uint32_t* status, uint32_t* done) {
+                   size_t xr_off, int K, int E, int El, int W, int row_vecs, int slot_end,
+                   long long n_recv, uint32_t* status) {
   __shared__ uint4* s_dst[MAX_K];
-  __shared__ int s_n, s_skip;
+  __shared__ char* s_peer[MAX_W];
+  __shared__ int s_n;
   const int t = blockIdx.x;
   pdl_wait();
   pdl_trigger();
-  if (threadIdx.x == 0) s_skip = timed_out(status);
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    const int k = threadIdx.x;
-    uint4* dp = nullptr;
-    if (!s_skip && t < T && k < K) {
+  if (threadIdx.x >= 32 && threadIdx.x < 32 + W)
+    s_peer[threadIdx.x - 32] = static_cast<char*>(peers[threadIdx.x - 32]);
+  const int k = threadIdx.x;
+  long long row = -1;
+  int d = 0;
+  if (k < 32) {
+    const bool skip = __shfl_sync(0xffffffffu, k == 0 ? (int)timed_out(status) : 0, 0) != 0;
+    if (!skip && k < K) {
       const int sl = token_slot[(size_t)t * K + k];
+      const int e = topk_idx[(size_t)t * K + k];
       if (sl >= 0 && sl < slot_end) {
-        const int e = topk_idx[(size_t)t * K + k];
-        const long long row = (e >= 0 && e < E) ? (long long)send_dst[e] + (sl - offsets[e]) : -1;
-        if (row >= 0 && row < n_recv)
-          dp = reinterpret_cast<uint4*>(static_cast<char*>(peers[e / El]) + xr_off) +
-               row * row_vecs;
-        else
+        row = (e >= 0 && e < E) ? (long long)send_dst[e] + (sl - offsets[e]) : -1;
+        if (row < 0 || row >= n_recv) {
           atomicCAS(status, 0u, (uint32_t)MOE_ERR_DEVICE_INPUT);
+          row = -1;
+        }
+        d = row >= 0 ? e / El : 0;
       }
     }
-    const unsigned m = __ballot_sync(0xffffffffu, dp != nullptr);
-    if (dp) s_dst[__popc(m & ((1u << k) - 1u))] = dp;
+  }
+  __syncthreads();
+  if (k < 32) {
+    const unsigned m = __ballot_sync(0xffffffffu, row >= 0);
+    if (row >= 0)
+      s_dst[__popc(m & ((1u << k) - 1u))] =
+          reinterpret_cast<uint4*>(s_peer[d] + xr_off) + row * row_vecs;
     if (k == 0) s_n = __popc(m);
   }
   __syncthreads();
   const int n = s_n;
-  if (n > 0) {
-    const uint4* src = x + (size_t)t * row_vecs;
-    for (int v0 = threadIdx.x; v0 < row_vecs; v0 += EP_THREADS * EP_UNROLL) {
-      uint4 d[EP_UNROLL];
+  if (n == 0) return;   // every assignment of this token overflowed
+  const uint4* src = x + (size_t)t * row_vecs;
+  for (int v0 = threadIdx.x; v0 < row_vecs; v0 += EP_THREADS * EP_UNROLL) {
+    uint4 dv[EP_UNROLL];
+#pragma unroll
+    for (int u = 0; u < EP_UNROLL; ++u) {
+      const int v = v0 + u * EP_THREADS;
+      if (v < row_vecs) dv[u] = __ldcs(src + v);
+    }
+    for (int j = 0; j < n; ++j) {
+      uint4* dst = s_dst[j];
 #pragma unroll
       for (int u = 0; u < EP_UNROLL; ++u) {
         const int v = v0 + u * EP_THREADS;
-        if (v < row_vecs) d[u] = __ldcs(src + v);
+        if (v < row_vecs) dst[v] = dv[u];
       }
-      for (int j = 0; j < n; ++j) {
-        uint4* dst = s_dst[j];
-#pragma unroll
-        for (int u = 0; u < EP_UNROLL; ++u) {
-          const int v = v0 + u * EP_THREADS;
-          if (v < row_vecs) dst[v] = d[u];
-        }
-      }
-    }
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence_system();   // this block's stores, before its count
-    const uint32_t prev = atomicAdd(done, 1u);
-    if (prev == gridDim.x - 1) {   // every block's stores are ordered before this point
-      __threadfence_system();
-      *done = 0u;   // ready for the next step (stream-ordered)
-      if (!s_skip)
-        for (int d = 0; d < W; ++d)
-          st_release_sys(peer_flags(peers, d, flags_off) + FLAG_DISPATCH * W + rank, epoch);
     }
   }
 }
@@ -346,8 +339,9 @@ __global__ void ep_wait_kernel(const uint32_t* flags, int W, uint32_t epoch,
   if (threadIdx.x == 0) wait_all(flags, W, epoch, timeout_ns, status);
 }
 
-// After the grouped GEMM (pdl_wait: the GEMM has finished and its stores are
-// visible): every rank's flag `which` for this rank. Not after a timeout.
+// After the dispatch or the grouped GEMM (pdl_wait: that grid has finished and
+// its stores are visible to this one): every rank's flag `which` for this rank,
+// released at system scope after a system fence. Not after a timeout.
 __global__ void ep_signal_kernel(void* const* __restrict__ peers, size_t flags_off, int which,
                                  int W, int rank, uint32_t epoch, const uint32_t* status) {
   pdl_wait();
@@ -367,35 +361,40 @@ __global__ void __launch_bounds__(EP_THREADS)
 ep_combine_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ token_slot,
                   const float* __restrict__ topk_w, const int32_t* __restrict__ offsets,
                   const int32_t* __restrict__ send_dst, void* const* __restrict__ peers,
-                  size_t y_off, uint4* __restrict__ out, int K, int E, int El, int row_vecs,
-                  int slot_end, long long n_recv, uint32_t* status) {
+                  size_t y_off, uint4* __restrict__ out, int K, int E, int El, int W,
+                  int row_vecs, int slot_end, long long n_recv, uint32_t* status) {
   __shared__ const uint4* s_src[MAX_K];
   __shared__ float s_w[MAX_K];
+  __shared__ char* s_peer[MAX_W];
   __shared__ int s_n;
   const int t = blockIdx.x;
   pdl_wait();
   pdl_trigger();
-  if (threadIdx.x < 32) {
-    const int k = threadIdx.x;
-    const uint4* sp = nullptr;
-    float wt = 0.f;
-    if (k < K) {
-      const int sl = token_slot[(size_t)t * K + k];
-      wt = topk_w[(size_t)t * K + k];
-      if (sl >= 0 && sl < slot_end) {
-        const int e = topk_idx[(size_t)t * K + k];
-        const long long row = (e >= 0 && e < E) ? (long long)send_dst[e] + (sl - offsets[e]) : -1;
-        if (row >= 0 && row < n_recv)
-          sp = reinterpret_cast<const uint4*>(static_cast<char*>(peers[e / El]) + y_off) +
-               row * row_vecs;
-        else
-          atomicCAS(status, 0u, (uint32_t)MOE_ERR_DEVICE_INPUT);
+  if (threadIdx.x >= 32 && threadIdx.x < 32 + W)
+    s_peer[threadIdx.x - 32] = static_cast<char*>(peers[threadIdx.x - 32]);
+  const int k = threadIdx.x;
+  long long row = -1;
+  int d = 0;
+  float wt = 0.f;
+  if (k < K) {
+    const int sl = token_slot[(size_t)t * K + k];
+    const int e = topk_idx[(size_t)t * K + k];
+    wt = topk_w[(size_t)t * K + k];
+    if (sl >= 0 && sl < slot_end) {
+      row = (e >= 0 && e < E) ? (long long)send_dst[e] + (sl - offsets[e]) : -1;
+      if (row < 0 || row >= n_recv) {
+        atomicCAS(status, 0u, (uint32_t)MOE_ERR_DEVICE_INPUT);
+        row = -1;
       }
+      d = row >= 0 ? e / El : 0;
     }
-    const unsigned m = __ballot_sync(0xffffffffu, sp != nullptr);
-    if (sp) {
+  }
+  __syncthreads();
+  if (k < 32) {   // pack the kept assignments, k order
+    const unsigned m = __ballot_sync(0xffffffffu, row >= 0);
+    if (row >= 0) {
       const int pos = __popc(m & ((1u << k) - 1u));
-      s_src[pos] = sp;
+      s_src[pos] = reinterpret_cast<const uint4*>(s_peer[d] + y_off) + row * row_vecs;
       s_w[pos] = wt;
     }
     if (k == 0) s_n = __popc(m);
@@ -469,7 +468,7 @@ struct Ptrs {
   int32_t *topk_idx, *counts, *overflow, *offsets, *segoff, *slot, *row_src, *totals, *blk;
   float* topk_w;
   int32_t *send_dst, *recv_off, *recv_cnt;
-  uint32_t *status, *done;
+  uint32_t* status;
   char* h;
 };
 
@@ -491,7 +490,6 @@ Ptrs ws_ptrs(const moe_config_t& c, int W, void* ws) {
   p.send_dst = reinterpret_cast<int32_t*>(b + L.send_dst);
   p.recv_off = reinterpret_cast<int32_t*>(b + L.recv_off);
   p.recv_cnt = reinterpret_cast<int32_t*>(b + L.recv_cnt);
-  p.done = reinterpret_cast<uint32_t*>(b + L.done);
   p.h = b + L.h;
   return p;
 }
@@ -595,7 +593,7 @@ moe_status_t moe_ep_route(const moe_config_t* cfg, const moe_ep_t* ep, const flo
   if (st != MOE_OK) return st;
   return cuda_st(launch_pdl(ep_publish_kernel, dim3(W), dim3(256), 0, s,
                             (const int32_t*)p.counts, c.E, W, ep->rank, peers, S.counts, S.flags,
-                            ep->epoch, p.done));
+                            ep->epoch));
 }
 
 moe_status_t moe_ep_dispatch(const moe_config_t* cfg, const moe_ep_t* ep, const void* x,
@@ -616,14 +614,17 @@ moe_status_t moe_ep_dispatch(const moe_config_t* cfg, const moe_ep_t* ep, const 
                           p.status, p.send_dst, p.recv_off, p.recv_cnt));
   if (st != MOE_OK) return st;
   const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
-  // at least one block, so that the DISPATCH flags are published with T = 0 too
-  return cuda_st(launch_pdl(ep_dispatch_kernel, dim3((unsigned)std::max(c.T, 1)),
-                            dim3(EP_THREADS), 0, s, static_cast<const uint4*>(x),
-                            (const int32_t*)p.topk_idx, (const int32_t*)p.slot,
-                            (const int32_t*)p.offsets, (const int32_t*)p.send_dst, peers, S.xr,
-                            S.flags, c.T, c.K, c.E, c.E / W, W, ep->rank, row_vecs,
-                            (int)routed_rows(c), (long long)recv_rows(c, W), ep->epoch, p.status,
-                            p.done));
+  if (c.T > 0) {
+    st = cuda_st(launch_pdl(ep_dispatch_kernel, dim3((unsigned)c.T), dim3(EP_THREADS), 0, s,
+                            static_cast<const uint4*>(x), (const int32_t*)p.topk_idx,
+                            (const int32_t*)p.slot, (const int32_t*)p.offsets,
+                            (const int32_t*)p.send_dst, peers, S.xr, c.K, c.E, c.E / W, W,
+                            row_vecs, (int)routed_rows(c), (long long)recv_rows(c, W), p.status));
+    if (st != MOE_OK) return st;
+  }
+  return cuda_st(launch_pdl(ep_signal_kernel, dim3(1), dim3(MAX_W), 0, s, peers, S.flags,
+                            (int)FLAG_DISPATCH, W, ep->rank, ep->epoch,
+                            (const uint32_t*)p.status));
 }
 
 moe_status_t moe_ep_expert_mlp(const moe_config_t* cfg, const moe_ep_t* ep,
@@ -681,7 +682,7 @@ moe_status_t moe_ep_combine(const moe_config_t* cfg, const moe_ep_t* ep, void* s
                             (const int32_t*)p.topk_idx, (const int32_t*)p.slot,
                             (const float*)p.topk_w, (const int32_t*)p.offsets,
                             (const int32_t*)p.send_dst, peers, S.y, static_cast<uint4*>(out),
-                            c.K, c.E, c.E / W, row_vecs, (int)routed_rows(c),
+                            c.K, c.E, c.E / W, W, row_vecs, (int)routed_rows(c),
                             (long long)recv_rows(c, W), p.status));
 }
 
