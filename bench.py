@@ -155,11 +155,21 @@ def max_over_ranks(x: float, world: int, device) -> float:
     return float(t.item())
 
 
+def flush_buffer(device) -> torch.Tensor:
+    """Two L2-sized halves for flush_l2."""
+    return torch.zeros(2 * L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+
+
 def flush_l2(buf: torch.Tensor):
-    """Evict L2 (a write larger than L2), then keep the GPU busy for ~0.2 ms
-    so that the host has queued the next step's launches before the GPU
-    reaches them: the timed region then holds device time only."""
-    buf.add_(1)
+    """Evict L2: write one half of buf (256 MB, larger than L2), then read the
+    other half, so that the write's dirty lines are written back here and not
+    during the timed kernels, and L2 is left holding clean lines of data the
+    step never touches. Then keep the GPU busy for ~0.2 ms so that the host
+    has queued the next step's launches before the GPU reaches them: the
+    timed region then holds device time only."""
+    w, r = buf.chunk(2)
+    w.add_(1)
+    r.sum()
     if hasattr(torch.cuda, "_sleep"):
         torch.cuda._sleep(400_000)
 
@@ -512,7 +522,7 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
     xs = [i["x"] for i in inps]
     outs = [torch.empty(wl.T, wl.H, dtype=wl.torch_act, device=device) for _ in range(Wn)]
     emu = EpOnOneDevice(cfg, Wn, device)
-    flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    flush_buf = flush_buffer(device)
     stream = torch.cuda.current_stream()
 
     def step():
@@ -582,7 +592,7 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
                    "E": wl.E, "K": K, "F": F, "S": wl.S, "cf": wl.cf, "capacity": C,
                    "row_align": wl.row_align, "ranks": Wn, "effective_tokens": Nt,
                    "parallelism": f"ep{Wn} emulated on one GPU (exchanges through local HBM)",
-                   "l2": "flushed (256 MB write) before every step"},
+                   "l2": "flushed before every step: 256 MB written, then another 256 MB read"},
         "e2e": None,
         "gpu_launches": None,
         "roofline": {"bound": "tensor", "kernel": "expert_mlp (all ranks' grouped GEMMs)",
@@ -656,7 +666,7 @@ def main(argv=None):
 
     layer = Layer(wl, seed=rank, device=device, overlap=args.overlap, router=args.router,
                   fp8=args.fp8)
-    flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    flush_buf = flush_buffer(device)
     stream = torch.cuda.current_stream()
 
     layer.forward()
@@ -750,7 +760,7 @@ def main(argv=None):
         "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "K": wl.K, "F": wl.F,
                    "S": wl.S, "cf": wl.cf, "capacity": layer.C, "row_align": wl.row_align,
                    "effective_tokens": alg["N"], "overflow": int(totals[2]),
-                   "l2": "flushed (256 MB write) before every step", "parallelism": f"replicas{world}",
+                   "l2": "flushed before every step: 256 MB written, then another 256 MB read", "parallelism": f"replicas{world}",
                    "overlap": bool(args.overlap), "router_projection": bool(args.router),
                    "n_shared": wl.n_shared,
                    "payload": "e4m3, 1x128 blocks, UE8M0 scales; bf16 combine" if args.fp8 else wl.act},
