@@ -160,7 +160,7 @@ def flush_buffer(device) -> torch.Tensor:
     return torch.zeros(2 * L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
 
 
-def flush_l2(buf: torch.Tensor):
+def flush_l2(buf: torch.Tensor, sleep_cycles: int = 400_000):
     """Evict L2: write one half of buf (256 MB, larger than L2), then read the
     other half, so that the write's dirty lines are written back here and not
     during the timed kernels, and L2 is left holding clean lines of data the
@@ -171,7 +171,7 @@ def flush_l2(buf: torch.Tensor):
     w.add_(1)
     r.sum()
     if hasattr(torch.cuda, "_sleep"):
-        torch.cuda._sleep(400_000)
+        torch.cuda._sleep(sleep_cycles)
 
 
 class Layer:
@@ -268,7 +268,10 @@ def phase_times(layer: Layer, steps, flush_buf, stream):
     acc = {n: [] for n in names}
     nvtx = torch.cuda.nvtx   # host ranges per phase, for nsys-style timelines
     for _ in range(steps + 1):
-        flush_l2(flush_buf)
+        # a longer idle wait than the whole-step timing's: the piecewise calls
+        # cost more host time, and every phase must already be queued when the
+        # GPU reaches it, or its time would include the host's
+        flush_l2(flush_buf, 4_000_000)
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
         ev[0].record(stream)
         for i, c in enumerate(calls):

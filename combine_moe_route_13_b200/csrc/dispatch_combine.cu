@@ -7,9 +7,10 @@
 // ("Диспетчеризация и комбинирование"): a token's K expert outputs are read
 // back and summed with the router weights.
 //
-// Both are pure HBM streams. One block per token row; each thread moves
-// 16-byte vectors (8 bf16 or 4 fp32), several per iteration so that enough
-// loads are in flight. A dispatched row is read once and written K times;
+// Both are pure HBM streams. Each block strides over token rows (the grid is
+// the blocks resident at once, so the PDL dependency wait runs once per
+// block); each thread moves 16-byte vectors (8 bf16 or 4 fp32), several per
+// iteration so that enough loads are in flight. A dispatched row is read once and written K times;
 // a combined row reads its K expert rows and is written once. A shared
 // expert adds one row per token to both (its copy of x, its output row).
 #include <algorithm>
@@ -29,43 +30,43 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) { return __ldcs(p); }
 
 __global__ void __launch_bounds__(DC_THREADS)
 dispatch_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ token_slot,
-                uint4* __restrict__ xp, int K, int row_vecs, long long sh_row0, int slot_end) {
+                uint4* __restrict__ xp, int T, int K, int row_vecs, long long sh_row0,
+                int slot_end) {
   __shared__ int s_slot[MAX_K + 1];
-  __shared__ int s_any;
-  const int t = blockIdx.x;
-  // the shared expert's row of this token is one more destination
+  // the shared expert's row of a token is one more destination
   const int KD = sh_row0 >= 0 ? K + 1 : K;
-  if (threadIdx.x == 0) s_any = 0;
   pdl_wait();
   pdl_trigger();
-  __syncthreads();
-  if (threadIdx.x < K) {
-    int s = token_slot[(size_t)t * K + threadIdx.x];
-    if (s >= slot_end) s = -1;   // outside the grouped buffer: treated as dropped
-    s_slot[threadIdx.x] = s;
-    if (s >= 0) atomicOr(&s_any, 1);
-  } else if (threadIdx.x == K && KD > K) {
-    s_slot[K] = (int)(sh_row0 + t);
-    s_any = 1;
-  }
-  __syncthreads();
-  if (!s_any) return;   // every assignment of this token overflowed: nothing to copy
-  const uint4* src = x + (size_t)t * row_vecs;
-  for (int v0 = threadIdx.x; v0 < row_vecs; v0 += DC_THREADS * DC_UNROLL) {
-    uint4 d[DC_UNROLL];
-#pragma unroll
-    for (int u = 0; u < DC_UNROLL; ++u) {
-      const int v = v0 + u * DC_THREADS;
-      if (v < row_vecs) d[u] = ld_stream(src + v);
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    __syncthreads();   // the previous token's readers of s_slot are done
+    bool kept = false;
+    if (threadIdx.x < K) {
+      int s = token_slot[(size_t)t * K + threadIdx.x];
+      if (s >= slot_end) s = -1;   // outside the grouped buffer: treated as dropped
+      s_slot[threadIdx.x] = s;
+      kept = s >= 0;
+    } else if (threadIdx.x == K && KD > K) {
+      s_slot[K] = (int)(sh_row0 + t);
+      kept = true;
     }
-    for (int k = 0; k < KD; ++k) {
-      const int s = s_slot[k];
-      if (s < 0) continue;
-      uint4* dst = xp + (size_t)s * row_vecs;
+    if (!__syncthreads_or(kept)) continue;   // every assignment overflowed: nothing to copy
+    const uint4* src = x + (size_t)t * row_vecs;
+    for (int v0 = threadIdx.x; v0 < row_vecs; v0 += DC_THREADS * DC_UNROLL) {
+      uint4 d[DC_UNROLL];
 #pragma unroll
       for (int u = 0; u < DC_UNROLL; ++u) {
         const int v = v0 + u * DC_THREADS;
-        if (v < row_vecs) dst[v] = d[u];
+        if (v < row_vecs) d[u] = ld_stream(src + v);
+      }
+      for (int k = 0; k < KD; ++k) {
+        const int s = s_slot[k];
+        if (s < 0) continue;
+        uint4* dst = xp + (size_t)s * row_vecs;
+#pragma unroll
+        for (int u = 0; u < DC_UNROLL; ++u) {
+          const int v = v0 + u * DC_THREADS;
+          if (v < row_vecs) dst[v] = d[u];
+        }
       }
     }
   }
@@ -127,76 +128,77 @@ __device__ __forceinline__ void store_acc(uint4* dst, int v0, int row_vecs, cons
 template <bool BF16>
 __global__ void __launch_bounds__(DC_THREADS)
 combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ token_slot,
-               const float* __restrict__ topk_w, uint4* __restrict__ out, int K, int row_vecs,
-               long long sh_row0, int slot_end) {
+               const float* __restrict__ topk_w, uint4* __restrict__ out, int T, int K,
+               int row_vecs, long long sh_row0, int slot_end) {
   __shared__ int s_slot[MAX_K];
   __shared__ float s_w[MAX_K];
   __shared__ int s_n;
-  const int t = blockIdx.x;
   pdl_wait();
   pdl_trigger();
-  if (threadIdx.x < 32) {   // warp 0 packs the kept assignments, in k order
-    int sl = -1;
-    float wt = 0.f;
-    if ((int)threadIdx.x < K) {
-      sl = token_slot[(size_t)t * K + threadIdx.x];
-      wt = topk_w[(size_t)t * K + threadIdx.x];
-    }
-    const bool keep = sl >= 0 && sl < slot_end;   // outside the grouped buffer: dropped
-    const unsigned m = __ballot_sync(0xffffffffu, keep);
-    if (keep) {
-      const int pos = __popc(m & ((1u << threadIdx.x) - 1u));
-      s_slot[pos] = sl;
-      s_w[pos] = wt;
-    }
-    if (threadIdx.x == 0) s_n = __popc(m);
-  }
-  __syncthreads();
-  K = s_n;   // from here on: the kept rows only
   constexpr int LANES = BF16 ? 8 : 4;
-  uint4* dst = out + (size_t)t * row_vecs;
-  for (int v0 = threadIdx.x; v0 < row_vecs; v0 += DC_THREADS * 2) {
-    Acc<BF16> acc;
-#pragma unroll
-    for (int u = 0; u < 2; ++u)
-#pragma unroll
-      for (int i = 0; i < LANES; ++i) acc[u][i] = 0.f;
-    int k = 0;
-    // groups of 4 experts: issue the loads, then accumulate in k order
-    for (; k < K; k += 4) {
-      uint4 d[4][2];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int s = (k + j < K) ? s_slot[k + j] : -1;
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int v = v0 + u * DC_THREADS;
-          if (s >= 0 && v < row_vecs) d[j][u] = __ldg(y + (size_t)s * row_vecs + v);
-          else d[j][u] = make_uint4(0u, 0u, 0u, 0u);
-        }
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    __syncthreads();          // the previous token's readers of s_slot, s_w, s_n are done
+    if (threadIdx.x < 32) {   // warp 0 packs the kept assignments, in k order
+      int sl = -1;
+      float wt = 0.f;
+      if ((int)threadIdx.x < K) {
+        sl = token_slot[(size_t)t * K + threadIdx.x];
+        wt = topk_w[(size_t)t * K + threadIdx.x];
       }
+      const bool keep = sl >= 0 && sl < slot_end;   // outside the grouped buffer: dropped
+      const unsigned m = __ballot_sync(0xffffffffu, keep);
+      if (keep) {
+        const int pos = __popc(m & ((1u << threadIdx.x) - 1u));
+        s_slot[pos] = sl;
+        s_w[pos] = wt;
+      }
+      if (threadIdx.x == 0) s_n = __popc(m);
+    }
+    __syncthreads();
+    const int n = s_n;   // from here on: the kept rows only
+    uint4* dst = out + (size_t)t * row_vecs;
+    for (int v0 = threadIdx.x; v0 < row_vecs; v0 += DC_THREADS * 2) {
+      Acc<BF16> acc;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if (k + j >= K || s_slot[k + j] < 0) continue;
-        const float wk = s_w[k + j];
+      for (int u = 0; u < 2; ++u)
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          if (BF16) {
-            float f[8];
-            unpack_bf16x8(d[j][u], f);
+        for (int i = 0; i < LANES; ++i) acc[u][i] = 0.f;
+      // groups of 4 experts: issue the loads, then accumulate in k order
+      for (int k = 0; k < n; k += 4) {
+        uint4 d[4][2];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[u][i] = fmaf(wk, f[i], acc[u][i]);
-          } else {
-            acc[u][0] = fmaf(wk, __uint_as_float(d[j][u].x), acc[u][0]);
-            acc[u][1] = fmaf(wk, __uint_as_float(d[j][u].y), acc[u][1]);
-            acc[u][2] = fmaf(wk, __uint_as_float(d[j][u].z), acc[u][2]);
-            acc[u][3] = fmaf(wk, __uint_as_float(d[j][u].w), acc[u][3]);
+        for (int j = 0; j < 4; ++j) {
+          const int s = (k + j < n) ? s_slot[k + j] : -1;
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int v = v0 + u * DC_THREADS;
+            if (s >= 0 && v < row_vecs) d[j][u] = __ldg(y + (size_t)s * row_vecs + v);
+            else d[j][u] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (k + j >= n) continue;
+          const float wk = s_w[k + j];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            if (BF16) {
+              float f[8];
+              unpack_bf16x8(d[j][u], f);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) acc[u][i] = fmaf(wk, f[i], acc[u][i]);
+            } else {
+              acc[u][0] = fmaf(wk, __uint_as_float(d[j][u].x), acc[u][0]);
+              acc[u][1] = fmaf(wk, __uint_as_float(d[j][u].y), acc[u][1]);
+              acc[u][2] = fmaf(wk, __uint_as_float(d[j][u].z), acc[u][2]);
+              acc[u][3] = fmaf(wk, __uint_as_float(d[j][u].w), acc[u][3]);
+            }
           }
         }
       }
+      if (sh_row0 >= 0) add_row<BF16, false>(y + (size_t)(sh_row0 + t) * row_vecs, v0, row_vecs, acc);
+      store_acc<BF16>(dst, v0, row_vecs, acc);
     }
-    if (sh_row0 >= 0) add_row<BF16, false>(y + (size_t)(sh_row0 + t) * row_vecs, v0, row_vecs, acc);
-    store_acc<BF16>(dst, v0, row_vecs, acc);
   }
 }
 
@@ -328,9 +330,10 @@ cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t*
                             int64_t sh_row0, cudaStream_t s) {
   if (c.T == 0) return cudaSuccess;
   const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
-  return launch_pdl(dispatch_kernel, dim3(c.T), dim3(DC_THREADS), 0, s,
-                    static_cast<const uint4*>(x), slot, static_cast<uint4*>(xp), c.K, row_vecs,
-                    (long long)sh_row0, (int)routed_rows(c));
+  return launch_pdl(dispatch_kernel, dim3(resident_grid(dispatch_kernel, DC_THREADS, c.T)),
+                    dim3(DC_THREADS), 0, s, static_cast<const uint4*>(x), slot,
+                    static_cast<uint4*>(xp), c.T, c.K, row_vecs, (long long)sh_row0,
+                    (int)routed_rows(c));
 }
 
 cudaError_t launch_combine(const moe_config_t& c, const void* y, const int32_t* slot,
@@ -338,9 +341,9 @@ cudaError_t launch_combine(const moe_config_t& c, const void* y, const int32_t* 
   if (c.T == 0) return cudaSuccess;
   const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
   auto kernel = c.act_dtype == MOE_BF16 ? combine_kernel<true> : combine_kernel<false>;
-  return launch_pdl(kernel, dim3(c.T), dim3(DC_THREADS), 0, s, static_cast<const uint4*>(y), slot,
-                    w, static_cast<uint4*>(out), c.K, row_vecs, (long long)sh_row0,
-                    (int)routed_rows(c));
+  return launch_pdl(kernel, dim3(resident_grid(kernel, DC_THREADS, c.T)), dim3(DC_THREADS), 0, s,
+                    static_cast<const uint4*>(y), slot, w, static_cast<uint4*>(out), c.T, c.K,
+                    row_vecs, (long long)sh_row0, (int)routed_rows(c));
 }
 
 cudaError_t launch_combine_wait(const moe_config_t& c, const void* y, const int32_t* slot,

@@ -21,14 +21,14 @@
 //   publish   every rank's counts table gets this rank's E counts; COUNTS flag
 //   plan      wait for all COUNTS flags; kept = min(count, C); scans give
 //             send_dst_row[E], recv_offsets[E/W+1], recv_counts[E/W]
-//   dispatch  one block per token: its row is read once and written to the
-//             owners of its kept experts
+//   dispatch  blocks stride over tokens: a row is read once and written to
+//             the owners of its kept experts
 //   signal    every owner's DISPATCH flag for this rank, after the dispatch
 //   wait      one thread: all DISPATCH flags (then the grouped GEMM of
 //             moe_expert_mlp over the local experts)
 //   signal    every rank's Y flag for this rank, after the GEMM
 //   wait      all Y flags
-//   combine   one block per token: the owners' y rows of its kept
+//   combine   blocks stride over tokens: the owners' y rows of a token's kept
 //             assignments, read in place, weighted sum in k order
 // Flags hold the step number (epoch) and are compared as "reached", so they
 // are never reset. Every wait is bounded; see moe_ep.h for the error rules.
@@ -264,9 +264,10 @@ ep_plan_kernel(const int32_t* __restrict__ counts_all, const uint32_t* flags, in
   }
 }
 
-// One block per token. The peer table is staged in shared memory while warp 0
-// loads the token's slots, experts and their layout entries; warp 0 then packs
-// the destinations of the kept assignments (k order); the row is read once and
+// Blocks stride over the tokens (a grid of the blocks resident at once). The
+// peer table is staged in shared memory once per block; for each token warp 0
+// loads its slots, experts and their layout entries and packs the
+// destinations of the kept assignments (k order); the row is read once and
 // stored to each destination. After a timeout of this rank nothing is written.
 // The DISPATCH flags are raised by ep_signal_kernel once this grid has
 // finished (its stores are then complete and visible to the signalling grid).
@@ -274,59 +275,56 @@ __global__ void __launch_bounds__(EP_THREADS)
 ep_dispatch_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ topk_idx,
                    const int32_t* __restrict__ token_slot, const int32_t* __restrict__ offsets,
                    const int32_t* __restrict__ send_dst, void* const* __restrict__ peers,
-                   size_t xr_off, int K, int E, int El, int W, int row_vecs, int slot_end,
+                   size_t xr_off, int T, int K, int E, int El, int W, int row_vecs, int slot_end,
                    long long n_recv, uint32_t* status) {
   __shared__ uint4* s_dst[MAX_K];
   __shared__ char* s_peer[MAX_W];
-  __shared__ int s_n;
-  const int t = blockIdx.x;
+  __shared__ int s_n, s_skip;
   pdl_wait();
   pdl_trigger();
-  if (threadIdx.x >= 32 && threadIdx.x < 32 + W)
-    s_peer[threadIdx.x - 32] = static_cast<char*>(peers[threadIdx.x - 32]);
+  if (threadIdx.x < W) s_peer[threadIdx.x] = static_cast<char*>(peers[threadIdx.x]);
+  if (threadIdx.x == 0) s_skip = timed_out(status);
+  __syncthreads();
+  if (s_skip) return;   // the same decision for every thread of the block
   const int k = threadIdx.x;
-  long long row = -1;
-  int d = 0;
-  if (k < 32) {
-    const bool skip = __shfl_sync(0xffffffffu, k == 0 ? (int)timed_out(status) : 0, 0) != 0;
-    if (!skip && k < K) {
-      const int sl = token_slot[(size_t)t * K + k];
-      const int e = topk_idx[(size_t)t * K + k];
-      if (sl >= 0 && sl < slot_end) {
-        row = (e >= 0 && e < E) ? (long long)send_dst[e] + (sl - offsets[e]) : -1;
-        if (row < 0 || row >= n_recv) {
-          atomicCAS(status, 0u, (uint32_t)MOE_ERR_DEVICE_INPUT);
-          row = -1;
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    __syncthreads();   // the previous token's readers of s_dst and s_n are done
+    if (k < 32) {
+      uint4* dp = nullptr;
+      if (k < K) {
+        const int sl = token_slot[(size_t)t * K + k];
+        const int e = topk_idx[(size_t)t * K + k];
+        if (sl >= 0 && sl < slot_end) {
+          const long long row =
+              (e >= 0 && e < E) ? (long long)send_dst[e] + (sl - offsets[e]) : -1;
+          if (row >= 0 && row < n_recv)
+            dp = reinterpret_cast<uint4*>(s_peer[e / El] + xr_off) + row * row_vecs;
+          else
+            atomicCAS(status, 0u, (uint32_t)MOE_ERR_DEVICE_INPUT);
         }
-        d = row >= 0 ? e / El : 0;
       }
+      const unsigned m = __ballot_sync(0xffffffffu, dp != nullptr);
+      if (dp) s_dst[__popc(m & ((1u << k) - 1u))] = dp;
+      if (k == 0) s_n = __popc(m);
     }
-  }
-  __syncthreads();
-  if (k < 32) {
-    const unsigned m = __ballot_sync(0xffffffffu, row >= 0);
-    if (row >= 0)
-      s_dst[__popc(m & ((1u << k) - 1u))] =
-          reinterpret_cast<uint4*>(s_peer[d] + xr_off) + row * row_vecs;
-    if (k == 0) s_n = __popc(m);
-  }
-  __syncthreads();
-  const int n = s_n;
-  if (n == 0) return;   // every assignment of this token overflowed
-  const uint4* src = x + (size_t)t * row_vecs;
-  for (int v0 = threadIdx.x; v0 < row_vecs; v0 += EP_THREADS * EP_UNROLL) {
-    uint4 dv[EP_UNROLL];
-#pragma unroll
-    for (int u = 0; u < EP_UNROLL; ++u) {
-      const int v = v0 + u * EP_THREADS;
-      if (v < row_vecs) dv[u] = __ldcs(src + v);
-    }
-    for (int j = 0; j < n; ++j) {
-      uint4* dst = s_dst[j];
+    __syncthreads();
+    const int n = s_n;
+    if (n == 0) continue;   // every assignment of this token overflowed
+    const uint4* src = x + (size_t)t * row_vecs;
+    for (int v0 = threadIdx.x; v0 < row_vecs; v0 += EP_THREADS * EP_UNROLL) {
+      uint4 dv[EP_UNROLL];
 #pragma unroll
       for (int u = 0; u < EP_UNROLL; ++u) {
         const int v = v0 + u * EP_THREADS;
-        if (v < row_vecs) dst[v] = dv[u];
+        if (v < row_vecs) dv[u] = __ldcs(src + v);
+      }
+      for (int j = 0; j < n; ++j) {
+        uint4* dst = s_dst[j];
+#pragma unroll
+        for (int u = 0; u < EP_UNROLL; ++u) {
+          const int v = v0 + u * EP_THREADS;
+          if (v < row_vecs) dst[v] = dv[u];
+        }
       }
     }
   }
@@ -361,102 +359,101 @@ __global__ void __launch_bounds__(EP_THREADS)
 ep_combine_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ token_slot,
                   const float* __restrict__ topk_w, const int32_t* __restrict__ offsets,
                   const int32_t* __restrict__ send_dst, void* const* __restrict__ peers,
-                  size_t y_off, uint4* __restrict__ out, int K, int E, int El, int W,
+                  size_t y_off, uint4* __restrict__ out, int T, int K, int E, int El, int W,
                   int row_vecs, int slot_end, long long n_recv, uint32_t* status) {
   __shared__ const uint4* s_src[MAX_K];
   __shared__ float s_w[MAX_K];
   __shared__ char* s_peer[MAX_W];
   __shared__ int s_n;
-  const int t = blockIdx.x;
   pdl_wait();
   pdl_trigger();
-  if (threadIdx.x >= 32 && threadIdx.x < 32 + W)
-    s_peer[threadIdx.x - 32] = static_cast<char*>(peers[threadIdx.x - 32]);
-  const int k = threadIdx.x;
-  long long row = -1;
-  int d = 0;
-  float wt = 0.f;
-  if (k < K) {
-    const int sl = token_slot[(size_t)t * K + k];
-    const int e = topk_idx[(size_t)t * K + k];
-    wt = topk_w[(size_t)t * K + k];
-    if (sl >= 0 && sl < slot_end) {
-      row = (e >= 0 && e < E) ? (long long)send_dst[e] + (sl - offsets[e]) : -1;
-      if (row < 0 || row >= n_recv) {
-        atomicCAS(status, 0u, (uint32_t)MOE_ERR_DEVICE_INPUT);
-        row = -1;
-      }
-      d = row >= 0 ? e / El : 0;
-    }
-  }
-  __syncthreads();
-  if (k < 32) {   // pack the kept assignments, k order
-    const unsigned m = __ballot_sync(0xffffffffu, row >= 0);
-    if (row >= 0) {
-      const int pos = __popc(m & ((1u << k) - 1u));
-      s_src[pos] = reinterpret_cast<const uint4*>(s_peer[d] + y_off) + row * row_vecs;
-      s_w[pos] = wt;
-    }
-    if (k == 0) s_n = __popc(m);
-  }
-  __syncthreads();
-  const int n = s_n;
+  if (threadIdx.x < W) s_peer[threadIdx.x] = static_cast<char*>(peers[threadIdx.x]);
   constexpr int LANES = BF16 ? 8 : 4;
-  uint4* dst = out + (size_t)t * row_vecs;
-  for (int v0 = threadIdx.x; v0 < row_vecs; v0 += EP_THREADS * 2) {
-    float acc[2][LANES];
-#pragma unroll
-    for (int u = 0; u < 2; ++u)
-#pragma unroll
-      for (int i = 0; i < LANES; ++i) acc[u][i] = 0.f;
-    for (int k = 0; k < n; k += 4) {
-      uint4 d[4][2];
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int v = v0 + u * EP_THREADS;
-          // rows written by another kernel, possibly on another GPU: read via L2
-          d[j][u] = (k + j < n && v < row_vecs) ? __ldcg(s_src[k + j] + v)
-                                                : make_uint4(0u, 0u, 0u, 0u);
+  const int k = threadIdx.x;
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    __syncthreads();   // s_peer staged; the previous token's readers of s_src, s_w, s_n done
+    if (k < 32) {      // warp 0 packs the kept assignments, k order
+      const uint4* sp = nullptr;
+      float wt = 0.f;
+      if (k < K) {
+        const int sl = token_slot[(size_t)t * K + k];
+        const int e = topk_idx[(size_t)t * K + k];
+        wt = topk_w[(size_t)t * K + k];
+        if (sl >= 0 && sl < slot_end) {
+          const long long row =
+              (e >= 0 && e < E) ? (long long)send_dst[e] + (sl - offsets[e]) : -1;
+          if (row >= 0 && row < n_recv)
+            sp = reinterpret_cast<const uint4*>(s_peer[e / El] + y_off) + row * row_vecs;
+          else
+            atomicCAS(status, 0u, (uint32_t)MOE_ERR_DEVICE_INPUT);
         }
+      }
+      const unsigned m = __ballot_sync(0xffffffffu, sp != nullptr);
+      if (sp) {
+        const int pos = __popc(m & ((1u << k) - 1u));
+        s_src[pos] = sp;
+        s_w[pos] = wt;
+      }
+      if (k == 0) s_n = __popc(m);
+    }
+    __syncthreads();
+    const int n = s_n;
+    uint4* dst = out + (size_t)t * row_vecs;
+    for (int v0 = threadIdx.x; v0 < row_vecs; v0 += EP_THREADS * 2) {
+      float acc[2][LANES];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if (k + j >= n) continue;
-        const float wk = s_w[k + j];
+      for (int u = 0; u < 2; ++u)
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          if (BF16) {
-            float f[8];
-            unpack_bf16x8(d[j][u], f);
+        for (int i = 0; i < LANES; ++i) acc[u][i] = 0.f;
+      for (int kk = 0; kk < n; kk += 4) {
+        uint4 d[4][2];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[u][i] = fmaf(wk, f[i], acc[u][i]);
-          } else {
-            acc[u][0] = fmaf(wk, __uint_as_float(d[j][u].x), acc[u][0]);
-            acc[u][1] = fmaf(wk, __uint_as_float(d[j][u].y), acc[u][1]);
-            acc[u][2] = fmaf(wk, __uint_as_float(d[j][u].z), acc[u][2]);
-            acc[u][3] = fmaf(wk, __uint_as_float(d[j][u].w), acc[u][3]);
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int v = v0 + u * EP_THREADS;
+            // rows written by another kernel, possibly on another GPU: read via L2
+            d[j][u] = (kk + j < n && v < row_vecs) ? __ldcg(s_src[kk + j] + v)
+                                                  : make_uint4(0u, 0u, 0u, 0u);
+          }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (kk + j >= n) continue;
+          const float wk = s_w[kk + j];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            if (BF16) {
+              float f[8];
+              unpack_bf16x8(d[j][u], f);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) acc[u][i] = fmaf(wk, f[i], acc[u][i]);
+            } else {
+              acc[u][0] = fmaf(wk, __uint_as_float(d[j][u].x), acc[u][0]);
+              acc[u][1] = fmaf(wk, __uint_as_float(d[j][u].y), acc[u][1]);
+              acc[u][2] = fmaf(wk, __uint_as_float(d[j][u].z), acc[u][2]);
+              acc[u][3] = fmaf(wk, __uint_as_float(d[j][u].w), acc[u][3]);
+            }
           }
         }
       }
-    }
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int v = v0 + u * EP_THREADS;
-      if (v >= row_vecs) continue;
-      uint4 o;
-      if (BF16) {
-        o.x = pack_bf16x2(acc[u][0], acc[u][1]);
-        o.y = pack_bf16x2(acc[u][2], acc[u][3]);
-        o.z = pack_bf16x2(acc[u][4], acc[u][5]);
-        o.w = pack_bf16x2(acc[u][6], acc[u][7]);
-      } else {
-        o.x = __float_as_uint(acc[u][0]);
-        o.y = __float_as_uint(acc[u][1]);
-        o.z = __float_as_uint(acc[u][2]);
-        o.w = __float_as_uint(acc[u][3]);
+      for (int u = 0; u < 2; ++u) {
+        const int v = v0 + u * EP_THREADS;
+        if (v >= row_vecs) continue;
+        uint4 o;
+        if (BF16) {
+          o.x = pack_bf16x2(acc[u][0], acc[u][1]);
+          o.y = pack_bf16x2(acc[u][2], acc[u][3]);
+          o.z = pack_bf16x2(acc[u][4], acc[u][5]);
+          o.w = pack_bf16x2(acc[u][6], acc[u][7]);
+        } else {
+          o.x = __float_as_uint(acc[u][0]);
+          o.y = __float_as_uint(acc[u][1]);
+          o.z = __float_as_uint(acc[u][2]);
+          o.w = __float_as_uint(acc[u][3]);
+        }
+        __stcs(dst + v, o);
       }
-      __stcs(dst + v, o);
     }
   }
 }
@@ -615,11 +612,13 @@ moe_status_t moe_ep_dispatch(const moe_config_t* cfg, const moe_ep_t* ep, const 
   if (st != MOE_OK) return st;
   const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
   if (c.T > 0) {
-    st = cuda_st(launch_pdl(ep_dispatch_kernel, dim3((unsigned)c.T), dim3(EP_THREADS), 0, s,
-                            static_cast<const uint4*>(x), (const int32_t*)p.topk_idx,
-                            (const int32_t*)p.slot, (const int32_t*)p.offsets,
-                            (const int32_t*)p.send_dst, peers, S.xr, c.K, c.E, c.E / W, W,
-                            row_vecs, (int)routed_rows(c), (long long)recv_rows(c, W), p.status));
+    st = cuda_st(launch_pdl(ep_dispatch_kernel,
+                            dim3(resident_grid(ep_dispatch_kernel, EP_THREADS, c.T)),
+                            dim3(EP_THREADS), 0, s, static_cast<const uint4*>(x),
+                            (const int32_t*)p.topk_idx, (const int32_t*)p.slot,
+                            (const int32_t*)p.offsets, (const int32_t*)p.send_dst, peers, S.xr,
+                            c.T, c.K, c.E, c.E / W, W, row_vecs, (int)routed_rows(c),
+                            (long long)recv_rows(c, W), p.status));
     if (st != MOE_OK) return st;
   }
   return cuda_st(launch_pdl(ep_signal_kernel, dim3(1), dim3(MAX_W), 0, s, peers, S.flags,
@@ -678,12 +677,12 @@ moe_status_t moe_ep_combine(const moe_config_t* cfg, const moe_ep_t* ep, void* s
   if (st != MOE_OK || c.T == 0) return st;
   const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
   auto kernel = c.act_dtype == MOE_BF16 ? ep_combine_kernel<true> : ep_combine_kernel<false>;
-  return cuda_st(launch_pdl(kernel, dim3(c.T), dim3(EP_THREADS), 0, s,
-                            (const int32_t*)p.topk_idx, (const int32_t*)p.slot,
-                            (const float*)p.topk_w, (const int32_t*)p.offsets,
-                            (const int32_t*)p.send_dst, peers, S.y, static_cast<uint4*>(out),
-                            c.K, c.E, c.E / W, W, row_vecs, (int)routed_rows(c),
-                            (long long)recv_rows(c, W), p.status));
+  return cuda_st(launch_pdl(kernel, dim3(resident_grid(kernel, EP_THREADS, c.T)),
+                            dim3(EP_THREADS), 0, s, (const int32_t*)p.topk_idx,
+                            (const int32_t*)p.slot, (const float*)p.topk_w,
+                            (const int32_t*)p.offsets, (const int32_t*)p.send_dst, peers, S.y,
+                            static_cast<uint4*>(out), c.T, c.K, c.E, c.E / W, W, row_vecs,
+                            (int)routed_rows(c), (long long)recv_rows(c, W), p.status));
 }
 
 moe_status_t moe_ep_layer_forward(const moe_config_t* cfg, const moe_ep_t* ep,

