@@ -35,7 +35,13 @@ Readings where the pages are silent (listed in the design notes):
   sender's own row order (token order);
 * the expert output of a row is returned to the token's rank and combined
   there exactly as in the one-rank layer (weights in k order, dropped
-  assignments contribute zero).
+  assignments contribute zero);
+* a shared expert (n_shared = 1) is held by every rank and applied to the
+  rank's own tokens, its output added with weight 1 after the routed terms
+  (the pages run it while the dispatch transfers are in flight: "Enabling
+  trillion-parameter models on AWS EFA", "Диспетчеризация и комбинирование";
+  "Efficient and portable Mixture-of-Experts communication", "Draagbare
+  kernels").
 
 Consequence used as the pin: for every rank, the expert-parallel layer equals
 the one-rank layer of that rank's tokens over all E experts.
@@ -109,9 +115,11 @@ def ep_plan(counts_all: np.ndarray, C: int, A: int, rank: int):
     }
 
 
-def ep_layer_forward(logits, x, w_gu, w_d, K: int, C: int, A: int, S: int, act: str, W: int):
-    """W ranks: logits[r] [T,E], x[r] [T,H]; w_gu [E,2F,H], w_d [E,H,F] (all E
-    experts; rank d uses its own E/W).  Steps:
+def ep_layer_forward(logits, x, w_gu, w_d, K: int, C: int, A: int, S: int, act: str, W: int,
+                     n_shared: int = 0):
+    """W ranks: logits[r] [T,E], x[r] [T,H]; w_gu [E',2F,H], w_d [E',H,F] with
+    E' = E + n_shared (all experts; rank d uses its own E/W routed experts,
+    and every rank the shared expert, the last one, on its own tokens).  Steps:
       1. every rank routes its own tokens (the one-rank route);
       2. the per-expert counts are exchanged (counts_all[s] = rank s's counts);
       3. every rank lays out its sends and its receive buffer (ep_plan);
@@ -119,9 +127,10 @@ def ep_layer_forward(logits, x, w_gu, w_d, K: int, C: int, A: int, S: int, act: 
          send_dst_row_s[e] + (slot - off_s[e]) of owner(e)'s receive buffer;
       5. every owner runs its local experts' SwiGLU on their receive rows;
       6. combine: rank s sums, in k order, w[t,k] times the owner's output
-         row of each kept assignment (found by the same address as in 4).
+         row of each kept assignment (found by the same address as in 4),
+         then adds its shared expert's output with weight 1 (n_shared = 1).
     Returns (outs [W arrays T x H], per-rank intermediates)."""
-    E = w_gu.shape[0]
+    E = w_gu.shape[0] - n_shared
     El = E // W
     T = np.asarray(logits[0]).shape[0]
     H = np.asarray(x[0]).shape[1]
@@ -148,6 +157,8 @@ def ep_layer_forward(logits, x, w_gu, w_d, K: int, C: int, A: int, S: int, act: 
                             w_gu[d * El:(d + 1) * El], w_d[d * El:(d + 1) * El], act)
         hs.append(h)
         ys.append(y)
+    y_sh = [O.expert_mlp_rows(np.asarray(x[s]), w_gu[E], w_d[E], act)[1] if n_shared else None
+            for s in range(W)]
     outs = []
     for s in range(W):
         r = routes[s]
@@ -157,7 +168,9 @@ def ep_layer_forward(logits, x, w_gu, w_d, K: int, C: int, A: int, S: int, act: 
             for t in np.nonzero(r["token_slot"][:, k] >= 0)[0]:
                 d, row = dest_row(s, t, k)
                 acc[t] += w[t, k] * O.act_to_f64(ys[d][row:row + 1], act)[0]
+        if n_shared:
+            acc += O.act_to_f64(y_sh[s], act)
         outs.append(O.f64_to_act(acc, act))
     inter = [dict(routes[r], **plans[r], counts_all=counts_all.astype(np.int32), xr=xr[r],
-                  h=hs[r], y=ys[r], R_recv=Rr) for r in range(W)]
+                  h=hs[r], y=ys[r], y_shared=y_sh[r], R_recv=Rr) for r in range(W)]
     return outs, inter

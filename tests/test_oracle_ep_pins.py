@@ -19,13 +19,13 @@ from oracle import moe_oracle as O
 from oracle import moe_oracle_ep as P
 
 
-def _inputs(W, T, H, E, K, F, act, seed, bias=0.0):
+def _inputs(W, T, H, E, K, F, act, seed, bias=0.0, n_shared=0):
     rng = np.random.default_rng(seed)
     logits = [(rng.standard_normal((T, E)) + bias * np.log(np.arange(1, E + 1))).astype(np.float32)
               for _ in range(W)]
     xs = [rng.standard_normal((T, H)).astype(np.float32) for _ in range(W)]
-    w_gu = (rng.standard_normal((E, 2 * F, H)) * 0.1).astype(np.float32)
-    w_d = (rng.standard_normal((E, H, F)) * 0.1).astype(np.float32)
+    w_gu = (rng.standard_normal((E + n_shared, 2 * F, H)) * 0.1).astype(np.float32)
+    w_d = (rng.standard_normal((E + n_shared, H, F)) * 0.1).astype(np.float32)
     if act == O.ACT_BF16:
         xs = [O.f64_to_bf16_bits(x.astype(np.float64)) for x in xs]
         w_gu = O.f64_to_bf16_bits(w_gu.astype(np.float64))
@@ -131,6 +131,19 @@ def test_every_rank_equals_the_one_rank_layer(act, W, T, E, K, cf, A, bias):
         ref, _ = O.layer_forward(logits[r], xs[r], w_gu, w_d, K, C, A, W, act)
         assert np.array_equal(outs[r], ref), f"rank {r}"
         assert inter[r]["recv_offsets"][-1] <= inter[r]["R_recv"]
+
+
+@pytest.mark.parametrize("act", [O.ACT_F32, O.ACT_BF16])
+def test_shared_expert_every_rank_equals_the_one_rank_layer(act):
+    W, T, H, E, K, F = 3, 16, 16, 6, 2, 12
+    logits, xs, w_gu, w_d = _inputs(W, T, H, E, K, F, act, seed=77, n_shared=1)
+    C = O.capacity(T, K, E, 1.0)
+    outs, inter = P.ep_layer_forward(logits, xs, w_gu, w_d, K, C, 4, W, act, W, n_shared=1)
+    plain, _ = P.ep_layer_forward(logits, xs, w_gu[:E], w_d[:E], K, C, 4, W, act, W)
+    for r in range(W):
+        ref, _ = O.layer_forward(logits[r], xs[r], w_gu, w_d, K, C, 4, W, act, n_shared=1)
+        assert np.array_equal(outs[r], ref), f"rank {r}"
+        assert not np.array_equal(outs[r], plain[r])
 
 
 def test_planted_mistakes_are_caught():
