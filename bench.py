@@ -512,15 +512,22 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
     peaks = load_peaks()
     Wn = world_ep
     C = M.moe_capacity(wl.T, wl.K, wl.E, wl.cf)
-    cfg = M.make_config(wl.T, wl.H, wl.E, wl.K, wl.F, wl.S, C, wl.row_align, wl.act)
+    cfg = M.make_config(wl.T, wl.H, wl.E, wl.K, wl.F, wl.S, C, wl.row_align, wl.act,
+                        n_shared=wl.n_shared)
     st = M.moe_ep_check(cfg, M.make_ep(Wn, 0, 1))
     if st != M.MOE_OK:
         raise SystemExit(f"unsupported expert-parallel workload: {M.status_string(st)}")
     full = W.make_inputs(wl, seed=0, device=device)
     inps = [full] + [W.make_inputs(wl, seed=r, device=device, weights=False) for r in range(1, Wn)]
     El = wl.E // Wn
-    wg = [full["w_gu"][r * El:(r + 1) * El] for r in range(Wn)]
-    wd = [full["w_d"][r * El:(r + 1) * El] for r in range(Wn)]
+
+    def local(w):   # each rank's experts, then the shared expert (every rank holds it)
+        if not wl.n_shared:
+            return [w[r * El:(r + 1) * El] for r in range(Wn)]
+        return [torch.cat([w[r * El:(r + 1) * El], w[wl.E:]]).contiguous() for r in range(Wn)]
+
+    wg, wd = local(full["w_gu"]), local(full["w_d"])
+    del full["w_gu"], full["w_d"]
     logits = [i["logits"] for i in inps]
     xs = [i["x"] for i in inps]
     outs = [torch.empty(wl.T, wl.H, dtype=wl.torch_act, device=device) for _ in range(Wn)]
@@ -558,7 +565,8 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
             M.moe_ep_dispatch(c, emu.ep(r), xs[r], emu.sym[r], emu.peers, emu.ws[r])
         ev[2].record(stream)
         for r in range(Wn):
-            M.moe_ep_expert_mlp(c, emu.ep(r), wg[r], wd[r], emu.sym[r], emu.peers, emu.ws[r])
+            M.moe_ep_expert_mlp(c, emu.ep(r), xs[r] if wl.n_shared else None, wg[r], wd[r],
+                                emu.sym[r], emu.peers, emu.ws[r])
         ev[3].record(stream)
         for r in range(Wn):
             M.moe_ep_combine(c, emu.ep(r), emu.sym[r], emu.peers, outs[r], emu.ws[r])
@@ -582,7 +590,7 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
         v = emu.views(r)
         kept = np.minimum(v["expert_counts"].cpu().numpy(), C)
         remote += int(kept.sum() - kept[r * El:(r + 1) * El].sum())
-    flops = 6.0 * Nt * H * F
+    flops = 6.0 * (Nt + Wn * T * wl.n_shared) * H * F
     hbm = peaks["hbm_gbs"]
     tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     mlp_tflops = flops / (ph["expert_mlp"] * 1e-3) / 1e12
@@ -594,6 +602,7 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
         "config": {"workload": f"{wl.name}_ep{Wn}_one_device", "T_per_rank": T, "H": H,
                    "E": wl.E, "K": K, "F": F, "S": wl.S, "cf": wl.cf, "capacity": C,
                    "row_align": wl.row_align, "ranks": Wn, "effective_tokens": Nt,
+                   "n_shared": wl.n_shared,
                    "parallelism": f"ep{Wn} emulated on one GPU (exchanges through local HBM)",
                    "l2": "flushed before every step: 256 MB written, then another 256 MB read"},
         "e2e": None,
@@ -655,8 +664,8 @@ def main(argv=None):
     if args.impl == "reference":
         return run_reference(args, wl, world, rank)
     if args.ep_emulate:
-        if world > 1 or args.fp8 or args.shared:
-            raise SystemExit("--ep-emulate runs on one GPU, bf16/f32, without a shared expert")
+        if world > 1 or args.fp8:
+            raise SystemExit("--ep-emulate runs on one GPU, bf16 or fp32")
         return run_ep_emulated(args, wl, args.ep_emulate)
 
     import torch.distributed as dist

@@ -75,7 +75,7 @@ class MoeEpAux(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "topk_idx", "expert_counts", "overflow", "expert_offsets", "segment_offsets",
         "token_slot", "row_src", "totals", "topk_w", "counts_all", "flags", "send_dst_row",
-        "recv_offsets", "recv_counts", "xr", "h", "y")]
+        "recv_offsets", "recv_counts", "xr", "h", "y", "h_shared", "y_shared")]
 
 
 _P = ctypes.c_void_p
@@ -128,7 +128,7 @@ def _load():
         "moe_ep_symmetric_init": (ctypes.c_int, [_CFG, ctypes.c_int32, _P, _SZ, _P]),
         "moe_ep_route": (ctypes.c_int, [_CFG, _EP, _P, _P, _P, _P, _SZ, _P]),
         "moe_ep_dispatch": (ctypes.c_int, [_CFG, _EP, _P, _P, _P, _P, _SZ, _P]),
-        "moe_ep_expert_mlp": (ctypes.c_int, [_CFG, _EP, _P, _P, _P, _P, _P, _SZ, _P]),
+        "moe_ep_expert_mlp": (ctypes.c_int, [_CFG, _EP, _P, _P, _P, _P, _P, _P, _SZ, _P]),
         "moe_ep_combine": (ctypes.c_int, [_CFG, _EP, _P, _P, _P, _P, _SZ, _P]),
         "moe_ep_layer_forward": (ctypes.c_int, [_CFG, _EP, _P, _P, _P, _P, _P, _P, _P,
                                                 ctypes.POINTER(MoeEpAux), _P, _SZ, _P]),
@@ -534,9 +534,10 @@ def moe_ep_dispatch(cfg, ep, x, sym, peers, ws, stream=None):
                                _stream(stream)), "moe_ep_dispatch")
 
 
-def moe_ep_expert_mlp(cfg, ep, w_gu_local, w_d_local, sym, peers, ws, stream=None):
+def moe_ep_expert_mlp(cfg, ep, x, w_gu_local, w_d_local, sym, peers, ws, stream=None):
+    """x: this rank's tokens, read only for the shared expert (None without one)."""
     dt = act_dtype(cfg)
-    _check(LIB.moe_ep_expert_mlp(ctypes.byref(cfg), ctypes.byref(ep),
+    _check(LIB.moe_ep_expert_mlp(ctypes.byref(cfg), ctypes.byref(ep), _ptr(x, dt, "x"),
                                  _ptr(w_gu_local, dt, "w_gu_local"), _ptr(w_d_local, dt, "w_d_local"),
                                  _addr(sym, "sym"), _peers(peers), _ptr(ws, name="ws"),
                                  _nbytes(ws), _stream(stream)), "moe_ep_expert_mlp")
@@ -597,7 +598,7 @@ def ep_views(cfg: MoeConfig, world: int, sym: torch.Tensor, ws: torch.Tensor,
     es = 4 if dt == torch.float32 else 2
     TK = cfg.T * cfg.K
     Rl = moe_max_rows(make_config(cfg.T, cfg.H, cfg.E, cfg.K, cfg.F, cfg.S, cfg.capacity,
-                                  cfg.row_align, cfg.act_dtype))
+                                  cfg.row_align, cfg.act_dtype))   # the routed rows
 
     def view(buf, ptr, nbytes, dtype, shape):
         off = ptr - buf.data_ptr()
@@ -623,4 +624,8 @@ def ep_views(cfg: MoeConfig, world: int, sym: torch.Tensor, ws: torch.Tensor,
         "xr": view(sym, aux.xr, R * cfg.H * es, dt, (R, cfg.H)),
         "h": view(ws, aux.h, R * cfg.F * es, dt, (R, cfg.F)),
         "y": view(sym, aux.y, R * cfg.H * es, dt, (R, cfg.H)),
+        "h_shared": view(ws, aux.h_shared, cfg.T * cfg.F * es, dt, (cfg.T, cfg.F))
+        if aux.h_shared else None,
+        "y_shared": view(ws, aux.y_shared, cfg.T * cfg.H * es, dt, (cfg.T, cfg.H))
+        if aux.y_shared else None,
     }

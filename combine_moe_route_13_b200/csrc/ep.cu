@@ -24,12 +24,15 @@
 //   dispatch  blocks stride over tokens: a row is read once and written to
 //             the owners of its kept experts
 //   signal    every owner's DISPATCH flag for this rank, after the dispatch
+//   (shared)  with a shared expert: its GEMM on this rank's own tokens, which
+//             needs nothing from the peers and overlaps their dispatch
 //   wait      one thread: all DISPATCH flags (then the grouped GEMM of
 //             moe_expert_mlp over the local experts)
 //   signal    every rank's Y flag for this rank, after the GEMM
 //   wait      all Y flags
 //   combine   blocks stride over tokens: the owners' y rows of a token's kept
-//             assignments, read in place, weighted sum in k order
+//             assignments, read in place, weighted sum in k order, plus the
+//             rank's own shared-expert row with weight 1
 // Flags hold the step number (epoch) and are compared as "reached", so they
 // are never reset. Every wait is bounded; see moe_ep.h for the error rules.
 #include <algorithm>
@@ -56,7 +59,7 @@ struct SymLayout {
 struct EpWs {
   size_t blk_cnt = 0, topk_idx = 0, topk_w = 0, counts = 0, overflow = 0, offsets = 0;
   size_t segoff = 0, totals = 0, slot = 0, row_src = 0;
-  size_t send_dst = 0, recv_off = 0, recv_cnt = 0, h = 0, total = 0;
+  size_t send_dst = 0, recv_off = 0, recv_cnt = 0, h = 0, h_sh = 0, y_sh = 0, total = 0;
 };
 
 int64_t recv_rows(const moe_config_t& c, int W) {
@@ -112,6 +115,10 @@ EpWs ep_ws_layout(const moe_config_t& c, int W) {
   L.recv_off = p;  p += align256((size_t)(El + 1) * 4);
   L.recv_cnt = p;  p += align256((size_t)El * 4);
   L.h = p;         p += align256((size_t)recv_rows(c, W) * c.F * act_size(c.act_dtype));
+  if (c.n_shared) {   // the shared expert's h and y for this rank's own tokens
+    L.h_sh = p;    p += align256((size_t)c.T * c.F * act_size(c.act_dtype));
+    L.y_sh = p;    p += align256((size_t)c.T * c.H * act_size(c.act_dtype));
+  }
   L.total = p;
   return L;
 }
@@ -124,7 +131,7 @@ moe_status_t ep_validate(const moe_config_t* c, const moe_ep_t* ep) {
   if (W < 1 || ep->rank < 0 || ep->rank >= W) return MOE_ERR_INVALID_ARG;
   if (W > MAX_W) return MOE_ERR_UNSUPPORTED;
   if (c->E % W != 0 || c->S % W != 0) return MOE_ERR_INVALID_ARG;
-  if (c->n_shared != 0) return MOE_ERR_UNSUPPORTED;
+  if (c->n_shared != 0 && c->act_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if ((int64_t)W * c->T > INT_MAX / 2 || (int64_t)W * c->capacity > INT_MAX / 2)
     return MOE_ERR_UNSUPPORTED;
   if (recv_rows(*c, W) > INT_MAX / 2) return MOE_ERR_UNSUPPORTED;
@@ -359,8 +366,9 @@ __global__ void __launch_bounds__(EP_THREADS)
 ep_combine_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ token_slot,
                   const float* __restrict__ topk_w, const int32_t* __restrict__ offsets,
                   const int32_t* __restrict__ send_dst, void* const* __restrict__ peers,
-                  size_t y_off, uint4* __restrict__ out, int T, int K, int E, int El, int W,
-                  int row_vecs, int slot_end, long long n_recv, uint32_t* status) {
+                  size_t y_off, const uint4* __restrict__ y_sh, uint4* __restrict__ out, int T,
+                  int K, int E, int El, int W, int row_vecs, int slot_end, long long n_recv,
+                  uint32_t* status) {
   __shared__ const uint4* s_src[MAX_K];
   __shared__ float s_w[MAX_K];
   __shared__ char* s_peer[MAX_W];
@@ -436,6 +444,25 @@ ep_combine_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restric
           }
         }
       }
+      if (y_sh) {   // the shared expert's row, weight 1, after the routed terms
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int v = v0 + u * EP_THREADS;
+          if (v >= row_vecs) continue;
+          const uint4 q = __ldg(y_sh + (size_t)t * row_vecs + v);
+          if (BF16) {
+            float f[8];
+            unpack_bf16x8(q, f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[u][i] += f[i];
+          } else {
+            acc[u][0] += __uint_as_float(q.x);
+            acc[u][1] += __uint_as_float(q.y);
+            acc[u][2] += __uint_as_float(q.z);
+            acc[u][3] += __uint_as_float(q.w);
+          }
+        }
+      }
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int v = v0 + u * EP_THREADS;
@@ -466,7 +493,7 @@ struct Ptrs {
   float* topk_w;
   int32_t *send_dst, *recv_off, *recv_cnt;
   uint32_t* status;
-  char* h;
+  char *h, *h_sh, *y_sh;   // h_sh / y_sh: nullptr without a shared expert
 };
 
 Ptrs ws_ptrs(const moe_config_t& c, int W, void* ws) {
@@ -488,6 +515,8 @@ Ptrs ws_ptrs(const moe_config_t& c, int W, void* ws) {
   p.recv_off = reinterpret_cast<int32_t*>(b + L.recv_off);
   p.recv_cnt = reinterpret_cast<int32_t*>(b + L.recv_cnt);
   p.h = b + L.h;
+  p.h_sh = c.n_shared ? b + L.h_sh : nullptr;
+  p.y_sh = c.n_shared ? b + L.y_sh : nullptr;
   return p;
 }
 
@@ -559,6 +588,8 @@ moe_status_t moe_ep_aux(const moe_config_t* cfg, const moe_ep_t* ep, void* sym, 
   a.xr = sb + S.xr;
   a.h = p.h;
   a.y = sb + S.y;
+  a.h_shared = p.h_sh;
+  a.y_shared = p.y_sh;
   *aux = a;
   return MOE_OK;
 }
@@ -626,19 +657,29 @@ moe_status_t moe_ep_dispatch(const moe_config_t* cfg, const moe_ep_t* ep, const 
                             (const uint32_t*)p.status));
 }
 
-moe_status_t moe_ep_expert_mlp(const moe_config_t* cfg, const moe_ep_t* ep,
+moe_status_t moe_ep_expert_mlp(const moe_config_t* cfg, const moe_ep_t* ep, const void* x,
                                const void* w_gu_local, const void* w_d_local, void* sym,
                                void* const* peers, void* ws, size_t ws_bytes, void* stream) {
   moe_status_t st = common_checks(cfg, ep, sym, peers, ws, ws_bytes);
   if (st != MOE_OK) return st;
   if (!w_gu_local || !w_d_local || !aligned16(w_gu_local) || !aligned16(w_d_local))
     return MOE_ERR_INVALID_ARG;
+  if (cfg->n_shared && cfg->T > 0 && (!x || !aligned16(x))) return MOE_ERR_INVALID_ARG;
   const moe_config_t& c = *cfg;
   const int W = ep->world;
   const Ptrs p = ws_ptrs(c, W, ws);
   const SymLayout S = sym_layout(c, W);
   char* sb = static_cast<char*>(sym);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (c.n_shared) {
+    // the shared expert on this rank's own tokens first: it needs nothing from
+    // the peers, so it runs while their rows are still arriving
+    const int El = c.E / W;
+    const char* wg = static_cast<const char*>(w_gu_local) + (size_t)El * 2 * c.F * c.H * 2;
+    const char* wd = static_cast<const char*>(w_d_local) + (size_t)El * c.H * c.F * 2;
+    st = launch_shared_mlp_bf16_tc(c, x, wg, wd, p.h_sh, p.y_sh, p.status, s);
+    if (st != MOE_OK) return st;
+  }
   st = cuda_st(launch_pdl(ep_wait_kernel, dim3(1), dim3(32), 0, s,
                           (const uint32_t*)(sb + S.flags) + FLAG_DISPATCH * W, W, ep->epoch,
                           timeout_ns(*ep), p.status));
@@ -681,7 +722,8 @@ moe_status_t moe_ep_combine(const moe_config_t* cfg, const moe_ep_t* ep, void* s
                             dim3(EP_THREADS), 0, s, (const int32_t*)p.topk_idx,
                             (const int32_t*)p.slot, (const float*)p.topk_w,
                             (const int32_t*)p.offsets, (const int32_t*)p.send_dst, peers, S.y,
-                            static_cast<uint4*>(out), c.T, c.K, c.E, c.E / W, W, row_vecs,
+                            reinterpret_cast<const uint4*>(p.y_sh), static_cast<uint4*>(out),
+                            c.T, c.K, c.E, c.E / W, W, row_vecs,
                             (int)routed_rows(c), (long long)recv_rows(c, W), p.status));
 }
 
@@ -695,7 +737,7 @@ moe_status_t moe_ep_layer_forward(const moe_config_t* cfg, const moe_ep_t* ep,
   if (aux && (st = moe_ep_aux(cfg, ep, sym, ws, aux)) != MOE_OK) return st;
   if ((st = moe_ep_route(cfg, ep, logits, sym, peers, ws, ws_bytes, stream)) != MOE_OK) return st;
   if ((st = moe_ep_dispatch(cfg, ep, x, sym, peers, ws, ws_bytes, stream)) != MOE_OK) return st;
-  if ((st = moe_ep_expert_mlp(cfg, ep, w_gu_local, w_d_local, sym, peers, ws, ws_bytes,
+  if ((st = moe_ep_expert_mlp(cfg, ep, x, w_gu_local, w_d_local, sym, peers, ws, ws_bytes,
                               stream)) != MOE_OK)
     return st;
   return moe_ep_combine(cfg, ep, sym, peers, out, ws, ws_bytes, stream);

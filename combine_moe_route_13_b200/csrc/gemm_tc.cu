@@ -603,6 +603,26 @@ moe_status_t launch_router_logits_tc(const moe_config_t& c, const void* x, const
   return tc::launch_router<1>(c, x, w_g, logits, status, s);
 }
 
+moe_status_t launch_shared_mlp_bf16_tc(const moe_config_t& c, const void* x, const void* w_gu_sh,
+                                       const void* w_d_sh, void* h, void* y, uint32_t* status,
+                                       cudaStream_t s) {
+  if (c.T == 0) return MOE_OK;
+  // no routed groups (E = 0): the kernel's only group is the shared one, T rows
+  // from row 0 of x, of h and of y, with the weights of expert 0 of w_gu_sh / w_d_sh
+  moe_config_t l = c;
+  l.E = 0;
+  l.K = 1;
+  l.S = 1;
+  l.capacity = 0;
+  l.row_align = 1;
+  l.n_shared = 1;
+  if (c.T >= 192)
+    return tc::launch_mlp<2>(l, x, nullptr, nullptr, w_gu_sh, w_d_sh, h, y, c.T, status, s,
+                             nullptr, x);
+  return tc::launch_mlp<1>(l, x, nullptr, nullptr, w_gu_sh, w_d_sh, h, y, c.T, status, s, nullptr,
+                           x);
+}
+
 moe_status_t launch_mlp_bf16_tc(const moe_config_t& c, const void* xp, const int32_t* offsets,
                                 const int32_t* counts, const void* w_gu, const void* w_d,
                                 void* h, void* y, int64_t R_max, uint32_t* status,

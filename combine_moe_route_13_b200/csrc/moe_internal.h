@@ -137,6 +137,14 @@ moe_status_t launch_mlp_bf16_tc(const moe_config_t& c, const void* xp, const int
                                 cudaStream_t s, uint32_t* row_ready = nullptr,
                                 const void* x_shared = nullptr);
 
+// The shared expert alone, bf16 on tcgen05: h[T,F] = silu(x Wg^T) * (x Wu^T),
+// y[T,H] = h Wd^T for the T rows of x, with w_gu_sh [2F,H] and w_d_sh [H,F]
+// (one expert). Same kernels and arithmetic as the shared group of
+// launch_mlp_bf16_tc.
+moe_status_t launch_shared_mlp_bf16_tc(const moe_config_t& c, const void* x, const void* w_gu_sh,
+                                       const void* w_d_sh, void* h, void* y, uint32_t* status,
+                                       cudaStream_t s);
+
 // Router projection logits[T,E] = x[T,H] w_g[E,H]^T (fp32 out): tcgen05 for
 // bf16, FFMA for fp32.
 moe_status_t launch_router_logits_tc(const moe_config_t& c, const void* x, const void* w_g,

@@ -116,8 +116,8 @@ class EpOnOneDevice:
         for r in range(W):
             B.moe_ep_dispatch(c, self.ep(r), x[r], self.sym[r], self.peers, self.ws[r], stream)
         for r in range(W):
-            B.moe_ep_expert_mlp(c, self.ep(r), w_gu_local[r], w_d_local[r], self.sym[r],
-                                self.peers, self.ws[r], stream)
+            B.moe_ep_expert_mlp(c, self.ep(r), x[r] if c.n_shared else None, w_gu_local[r],
+                                w_d_local[r], self.sym[r], self.peers, self.ws[r], stream)
         for r in range(W):
             B.moe_ep_combine(c, self.ep(r), self.sym[r], self.peers, out[r], self.ws[r], stream)
 

@@ -28,12 +28,18 @@
  *      derive the layout (below); write each kept token row straight into its
  *      owner's receive buffer xr; when every row is written, set each owner's
  *      DISPATCH flag for this rank.
- *   3. moe_ep_expert_mlp: wait for every rank's DISPATCH flag; run the grouped
- *      SwiGLU (the tcgen05 kernel of moe_expert_mlp) over the local experts'
- *      received rows into y; set every rank's Y flag for this rank.
+ *   3. moe_ep_expert_mlp: with a shared expert, first its SwiGLU on this rank's
+ *      own tokens (x), which needs nothing from the peers and so runs while
+ *      their rows are in flight (the pages multiply the shared experts while
+ *      the dispatch transfers are pending: EFA page, "Диспетчеризация и
+ *      комбинирование"; pplx-kernels page, "Draagbare kernels"); then wait
+ *      for every rank's DISPATCH flag; run the grouped SwiGLU (the tcgen05
+ *      kernel of moe_expert_mlp) over the local experts' received rows into y;
+ *      set every rank's Y flag for this rank.
  *   4. moe_ep_combine: wait for every rank's Y flag; out[t] = sum over kept k,
  *      in k order, of w[t,k] * (the owner's y row of that assignment), read
- *      from the owner's memory; fp32 accumulation, one rounding (as moe_combine).
+ *      from the owner's memory, plus (n_shared = 1) the rank's own shared-expert
+ *      row with weight 1; fp32 accumulation, one rounding (as moe_combine).
  *   Every rank's out equals moe_layer_forward of its own tokens over all E
  *   experts (the same rows meet the same weights in the same order).
  *
@@ -50,7 +56,8 @@
  * Memory. Each rank allocates one symmetric region of moe_ep_symmetric_bytes
  * (counts table [W][E] int32, flags [3][W] uint32, xr [R_recv][H], y [R_recv][H])
  * that its peers write into (counts, flags, xr) and read from (y), and a private
- * workspace of moe_ep_workspace_bytes (status word, route outputs, layout, h).
+ * workspace of moe_ep_workspace_bytes (status word, route outputs, layout, h,
+ * and with a shared expert its h and y for this rank's tokens).
  * `sym` is this rank's region as a pointer of this process; `peers` is a DEVICE
  * array of W pointers: peers[r] = rank r's region as mapped into this process
  * (peers[rank] = sym). Regions are zeroed once with moe_ep_symmetric_init on
@@ -75,8 +82,9 @@
  * buffer is not written and records MOE_ERR_DEVICE_INPUT.
  *
  * Limits: everything moe_expert_mlp supports for bf16 (tcgen05) plus
- * n_shared = 0, E % W == 0, S % W == 0, 1 <= W <= 64; fp32 activations use the
- * CUDA-core grouped GEMM. Else MOE_ERR_UNSUPPORTED (or INVALID_ARG).
+ * E % W == 0, S % W == 0, 1 <= W <= 64; fp32 activations use the CUDA-core
+ * grouped GEMM and take no shared expert. Else MOE_ERR_UNSUPPORTED (or
+ * INVALID_ARG).
  */
 #ifndef MOE_EP_H
 #define MOE_EP_H
@@ -106,6 +114,7 @@ typedef struct {
   int32_t *recv_offsets;   /* [E/W + 1]: local experts' first rows in xr, then the end */
   int32_t *recv_counts;    /* [E/W]: rows each local expert received */
   void *xr, *h, *y;        /* [R_recv][H] (symmetric), [R_recv][F] (private), [R_recv][H] (symmetric) */
+  void *h_shared, *y_shared;   /* [T][F], [T][H] (private): the shared expert on this rank's tokens; NULL without one */
 } moe_ep_aux_t;
 
 /* R_recv (see above); -1 for an invalid config or world. */
@@ -123,14 +132,16 @@ moe_status_t moe_ep_symmetric_init(const moe_config_t* cfg, int32_t world, void*
                                    size_t sym_bytes, void* stream);
 
 /* The four steps and the whole layer (see above). logits [T][E] fp32, x [T][H]
- * act; w_gu_local [E/W][2F][H], w_d_local [E/W][H][F]: this rank's experts in
- * ascending order; out [T][H] act. All device pointers, 16-byte aligned. */
+ * act; w_gu_local [E/W + n_shared][2F][H], w_d_local [E/W + n_shared][H][F]:
+ * this rank's experts in ascending order, then the shared expert; out [T][H]
+ * act. All device pointers, 16-byte aligned. moe_ep_expert_mlp reads x only
+ * for the shared expert (NULL allowed when n_shared = 0). */
 moe_status_t moe_ep_route(const moe_config_t* cfg, const moe_ep_t* ep, const float* logits,
                           void* sym, void* const* peers, void* ws, size_t ws_bytes, void* stream);
 moe_status_t moe_ep_dispatch(const moe_config_t* cfg, const moe_ep_t* ep, const void* x,
                              void* sym, void* const* peers, void* ws, size_t ws_bytes,
                              void* stream);
-moe_status_t moe_ep_expert_mlp(const moe_config_t* cfg, const moe_ep_t* ep,
+moe_status_t moe_ep_expert_mlp(const moe_config_t* cfg, const moe_ep_t* ep, const void* x,
                                const void* w_gu_local, const void* w_d_local, void* sym,
                                void* const* peers, void* ws, size_t ws_bytes, void* stream);
 moe_status_t moe_ep_combine(const moe_config_t* cfg, const moe_ep_t* ep, void* sym,

@@ -54,13 +54,18 @@ def test_one_rank_sizes_equal_the_one_rank_layer():
     (dict(), 2, 2, 1, M.MOE_ERR_INVALID_ARG),            # rank >= W
     (dict(), 2, -1, 1, M.MOE_ERR_INVALID_ARG),
     (dict(), 2, 0, 0, M.MOE_ERR_INVALID_ARG),            # epoch 0
-    (dict(n_shared=1), 2, 0, 1, M.MOE_ERR_UNSUPPORTED),
+    (dict(n_shared=1), 2, 0, 1, M.MOE_OK),               # bf16 with a shared expert
     (dict(H=4100), 2, 0, 1, M.MOE_ERR_UNSUPPORTED),      # what the one-rank GEMM rejects
     (dict(), 2, 1, 7, M.MOE_OK),
 ])
 def test_check(kw, world, rank, epoch, code):
     c = cfg_of("mixtral", **kw)
     assert M.moe_ep_check(c, M.make_ep(world, rank, epoch)) == code
+
+
+def test_shared_expert_needs_bf16():
+    c = cfg_of("tiny", S=2, n_shared=1)   # fp32 activations
+    assert M.moe_ep_check(c, M.make_ep(2, 0, 1)) == M.MOE_ERR_UNSUPPORTED
 
 
 def test_too_many_ranks_unsupported():
@@ -102,6 +107,11 @@ def test_aux_layout_is_inside_the_buffers():
         v = getattr(aux, f)
         assert ws + 256 <= v < ws + nws and v % 256 == 0, f
     assert aux.h + R * c.F * 2 <= ws + nws
+    assert aux.h_shared is None and aux.y_shared is None
+    cs = cfg_of("mixtral", n_shared=1)
+    assert M.LIB.moe_ep_aux(ctypes.byref(cs), ctypes.byref(ep), sym, ws, ctypes.byref(aux)) == M.MOE_OK
+    nws = M.moe_ep_workspace_bytes(cs, world)
+    assert ws < aux.h_shared < aux.y_shared and aux.y_shared + cs.T * cs.H * 2 <= ws + nws
 
 
 def test_entry_points_reject_bad_arguments_before_any_launch():
@@ -118,11 +128,15 @@ def test_entry_points_reject_bad_arguments_before_any_launch():
     # workspace too small, or misaligned
     assert lib.moe_ep_combine(ctypes.byref(c), ctypes.byref(ep), fake, fake, fake, fake, 256,
                               None) == M.MOE_ERR_WORKSPACE
-    assert lib.moe_ep_expert_mlp(ctypes.byref(c), ctypes.byref(ep), fake, fake, fake, fake,
+    assert lib.moe_ep_expert_mlp(ctypes.byref(c), ctypes.byref(ep), None, fake, fake, fake, fake,
                                  fake + 16, big, None) == M.MOE_ERR_WORKSPACE
     # weights missing
-    assert lib.moe_ep_expert_mlp(ctypes.byref(c), ctypes.byref(ep), None, fake, fake, fake, fake,
-                                 big, None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_expert_mlp(ctypes.byref(c), ctypes.byref(ep), None, None, fake, fake, fake,
+                                 fake, big, None) == M.MOE_ERR_INVALID_ARG
+    # a shared expert needs x
+    cs = cfg_of("mixtral", n_shared=1)
+    assert lib.moe_ep_expert_mlp(ctypes.byref(cs), ctypes.byref(ep), None, fake, fake, fake, fake,
+                                 fake, big, None) == M.MOE_ERR_INVALID_ARG
     # epoch 0 and a bad config
     ep0 = M.make_ep(2, 0, 0)
     assert lib.moe_ep_route(ctypes.byref(c), ctypes.byref(ep0), fake, fake, fake, fake, big,

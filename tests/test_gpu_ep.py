@@ -12,6 +12,9 @@ through the same peer table the kernels use across GPUs).
 * out bit for bit equal to the one-rank library layer (moe_layer_forward)
   of the same rank's tokens over all E experts;
 * several steps in a row (epochs), empty and fully dropped batches, E/W < K;
+* a shared expert on every rank's own tokens (its GEMM runs before the wait
+  for the peers' rows): its y against the oracle, out bit for bit equal to
+  the one-rank layer with the shared expert;
 * a wait that runs out: rank 0 alone, its peer never publishing, ends with
   MOE_ERR_TIMEOUT within the bound instead of hanging.
 """
@@ -33,27 +36,33 @@ ROUTE_KEYS = ("topk_idx", "topk_w", "expert_counts", "overflow", "expert_offsets
               "segment_offsets", "token_slot", "row_src", "totals")
 
 
-def make_case(W, T, H, E, K, F, act, seed, bias=0.0):
+def make_case(W, T, H, E, K, F, act, seed, bias=0.0, n_shared=0):
     g = torch.Generator().manual_seed(seed)
     dt = torch.bfloat16 if act == "bf16" else torch.float32
     logits = [torch.randn(T, E, generator=g) + bias * torch.log(torch.arange(1, E + 1).float())
               for _ in range(W)]
     xs = [torch.randn(T, H, generator=g).to(dt) for _ in range(W)]
-    w_gu = (torch.randn(E, 2 * F, H, generator=g) * 0.05).to(dt)
-    w_d = (torch.randn(E, H, F, generator=g) * 0.05).to(dt)
+    w_gu = (torch.randn(E + n_shared, 2 * F, H, generator=g) * 0.05).to(dt)
+    w_d = (torch.randn(E + n_shared, H, F, generator=g) * 0.05).to(dt)
     return logits, xs, w_gu, w_d
 
 
+def local_weights(w, W, E, n_shared, dev=DEV):
+    """Each rank's experts, then the shared expert (every rank holds it)."""
+    El = E // W
+    w = w.to(dev)
+    if not n_shared:
+        return [w[r * El:(r + 1) * El] for r in range(W)]
+    return [torch.cat([w[r * El:(r + 1) * El], w[E:E + 1]]).contiguous() for r in range(W)]
+
+
 def run_ep(cfg, W, logits, xs, w_gu, w_d, emu=None):
-    El = cfg.E // W
     emu = emu or EpOnOneDevice(cfg, W, DEV)
     dt = M.act_dtype(cfg)
-    wg = w_gu.to(DEV)
-    wd = w_d.to(DEV)
     outs = [torch.full((cfg.T, cfg.H), float("nan"), dtype=dt, device=DEV) for _ in range(W)]
     emu.forward([l.to(DEV) for l in logits], [x.to(DEV) for x in xs],
-                [wg[r * El:(r + 1) * El] for r in range(W)],
-                [wd[r * El:(r + 1) * El] for r in range(W)], outs)
+                local_weights(w_gu, W, cfg.E, cfg.n_shared),
+                local_weights(w_d, W, cfg.E, cfg.n_shared), outs)
     torch.cuda.synchronize()
     return emu, outs
 
@@ -192,7 +201,7 @@ def test_a_peer_that_never_publishes_times_out(cuda_ok):
     # rank 0 alone: rank 1 never publishes its counts, dispatches or signals
     M.moe_ep_route(cfg, ep, logits[0].to(DEV), emu.sym[0], emu.peers, emu.ws[0])
     M.moe_ep_dispatch(cfg, ep, xs[0].to(DEV), emu.sym[0], emu.peers, emu.ws[0])
-    M.moe_ep_expert_mlp(cfg, ep, wg, wd, emu.sym[0], emu.peers, emu.ws[0])
+    M.moe_ep_expert_mlp(cfg, ep, None, wg, wd, emu.sym[0], emu.peers, emu.ws[0])
     M.moe_ep_combine(cfg, ep, emu.sym[0], emu.peers, out, emu.ws[0])
     torch.cuda.synchronize()
     elapsed = time.perf_counter() - t0
@@ -204,3 +213,33 @@ def test_a_peer_that_never_publishes_times_out(cuda_ok):
         f = emu.views(r)["flags"].cpu().numpy()
         assert f[1, 0] == 0 and f[2, 0] == 0
     assert int(v["recv_counts"].sum()) == 0
+
+
+@pytest.mark.parametrize("W,T,H,E,K,F,cf", [
+    (2, 256, 256, 8, 2, 256, 1.25),
+    (4, 300, 512, 16, 4, 384, 0.5),     # overflow: some tokens keep only the shared term
+    (8, 64, 256, 64, 8, 128, 1.5),
+    (2, 200, 256, 8, 2, 256, 0.0),      # C = 0: the shared expert alone
+])
+def test_ep_shared_expert(cuda_ok, W, T, H, E, K, F, cf):
+    C = O.capacity(T, K, E, cf)
+    cfg = M.make_config(T=T, H=H, E=E, K=K, F=F, S=W, capacity=C, row_align=128, act="bf16",
+                        n_shared=1)
+    logits, xs, w_gu, w_d = make_case(W, T, H, E, K, F, "bf16", seed=T + E, n_shared=1)
+    emu, outs = run_ep(cfg, W, logits, xs, w_gu, w_d)
+    ref_outs, inter = P.ep_layer_forward([l.numpy() for l in logits], [act_np(x) for x in xs],
+                                         act_np(w_gu), act_np(w_d), K, C, 128, W, "bf16", W,
+                                         n_shared=1)
+    for r in range(W):
+        assert emu.status(r) == M.MOE_OK
+        v = emu.views(r)
+        # the shared expert's y on this rank's tokens against the oracle's SwiGLU
+        _, y_ref = O.expert_mlp_rows(act_np(xs[r]), act_np(w_gu[E]), act_np(w_d[E]), "bf16")
+        assert_close_act(act_np(v["y_shared"]), y_ref, "bf16", f"y_shared rank {r}")
+        # bit for bit the one-rank layer with the shared expert
+        ref = one_rank_layer(cfg, logits[r], xs[r], w_gu, w_d)
+        g, w = act_np(outs[r]), act_np(ref)
+        assert np.array_equal(g, w), f"rank {r}: {(g != w).sum()} elements differ"
+        gd, rd = O.act_to_f64(g, "bf16"), O.act_to_f64(ref_outs[r], "bf16")
+        fro = np.linalg.norm(gd - rd) / np.linalg.norm(rd)
+        assert fro <= 1e-2, f"chain rank {r}: relative Frobenius error {fro:.3e}"
