@@ -591,9 +591,16 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
         kept = np.minimum(v["expert_counts"].cpu().numpy(), C)
         remote += int(kept.sum() - kept[r * El:(r + 1) * El].sum())
     flops = 6.0 * (Nt + Wn * T * wl.n_shared) * H * F
+    # bytes the expert MLPs must move at least: every local expert with rows
+    # (and each rank's shared expert) read once, its rows in, h out and back, y out
+    active = sum(int(np.count_nonzero(emu.views(r)["recv_counts"].cpu().numpy()))
+                 for r in range(Wn)) + Wn * wl.n_shared
+    mlp_bytes = 3.0 * active * H * F * s_ + (Nt + Wn * T * wl.n_shared) * (2 * H + 2 * F) * s_
     hbm = peaks["hbm_gbs"]
     tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     mlp_tflops = flops / (ph["expert_mlp"] * 1e-3) / 1e12
+    mlp_gbs = mlp_bytes / (ph["expert_mlp"] * 1e-3) / 1e9
+    hbm_bound = mlp_bytes / (hbm * 1e9) > flops / (tensor_peak * 1e12)
     line = {
         "metric": METRIC, "value": Wn * T / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -607,10 +614,16 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
                    "l2": "flushed before every step: 256 MB written, then another 256 MB read"},
         "e2e": None,
         "gpu_launches": None,
-        "roofline": {"bound": "tensor", "kernel": "expert_mlp (all ranks' grouped GEMMs)",
-                     "achieved": mlp_tflops, "peak": tensor_peak, "unit": "TFLOP/s",
-                     "frac": mlp_tflops / tensor_peak,
-                     "peak_kind": f"bf16_tflops_sustained ({peaks['source']})", "traffic": None},
+        "roofline": ({"bound": "hbm", "kernel": "expert_mlp (all ranks' grouped GEMMs)",
+                      "achieved": mlp_gbs, "peak": hbm, "unit": "GB/s", "frac": mlp_gbs / hbm,
+                      "peak_kind": f"hbm_gbs ({peaks['source']})",
+                      "tensor_frac": mlp_tflops / tensor_peak}
+                     if hbm_bound else
+                     {"bound": "tensor", "kernel": "expert_mlp (all ranks' grouped GEMMs)",
+                      "achieved": mlp_tflops, "peak": tensor_peak, "unit": "TFLOP/s",
+                      "frac": mlp_tflops / tensor_peak,
+                      "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
+                      "hbm_frac": mlp_gbs / hbm}) | {"traffic": None},
         "kernels": {
             "phase_timing": "CUDA events around each step for all ranks (wait kernels included)",
             "route_us": ph["route"] * 1e3,
