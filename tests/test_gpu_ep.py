@@ -243,3 +243,68 @@ def test_ep_shared_expert(cuda_ok, W, T, H, E, K, F, cf):
         gd, rd = O.act_to_f64(g, "bf16"), O.act_to_f64(ref_outs[r], "bf16")
         fro = np.linalg.norm(gd - rd) / np.linalg.norm(rd)
         assert fro <= 1e-2, f"chain rank {r}: relative Frobenius error {fro:.3e}"
+
+
+def test_ep_random_sweep(cuda_ok):
+    # seeded random shapes: ranks, experts per rank, K, capacity factor, alignment,
+    # dtype; every rank bit for bit the one-rank layer, layout bit for bit the oracle's
+    rng = np.random.default_rng(2024)
+    for case in range(16):
+        W = int(rng.choice([2, 3, 4, 8]))
+        El = int(rng.integers(1, 9))
+        E = W * El
+        K = int(rng.integers(1, min(E, 8) + 1))
+        act = "bf16" if rng.random() < 0.75 else "f32"
+        H = int(rng.choice([128, 256, 384])) if act == "bf16" else int(rng.choice([64, 96, 128]))
+        F = int(rng.choice([128, 192, 256]))
+        T = int(rng.integers(1, 200))
+        cf = float(rng.choice([0.3, 0.8, 1.0, 1.5, 4.0]))
+        A = int(rng.choice([1, 8, 128])) if act == "f32" else 128
+        C = O.capacity(T, K, E, cf)
+        cfg = M.make_config(T=T, H=H, E=E, K=K, F=F, S=W, capacity=C, row_align=A, act=act)
+        logits, xs, w_gu, w_d = make_case(W, T, H, E, K, F, act, seed=case,
+                                          bias=float(rng.choice([0.0, -2.4])))
+        emu, outs = run_ep(cfg, W, logits, xs, w_gu, w_d)
+        counts_all = np.stack([O.route(l.numpy(), K, C, A, W)["expert_counts"] for l in logits])
+        for r in range(W):
+            assert emu.status(r) == M.MOE_OK, (case, r)
+            v = emu.views(r)
+            plan = P.ep_plan(counts_all, C, A, r)
+            for k in ("send_dst_row", "recv_offsets", "recv_counts"):
+                assert np.array_equal(v[k].cpu().numpy(), plan[k]), (case, r, k)
+            ref = one_rank_layer(cfg, logits[r], xs[r], w_gu, w_d)
+            assert torch.equal(outs[r], ref), (case, W, T, E, K, act, A, r)
+
+
+def test_a_rank_that_leaves_between_steps_times_the_others_out(cuda_ok):
+    # two good steps, then rank 1 stops taking part: rank 0's next step records
+    # MOE_ERR_TIMEOUT within its bound, and nothing of rank 0 reaches rank 1
+    W, T, H, E, K, F = 2, 96, 256, 8, 2, 256
+    C = O.capacity(T, K, E, 1.25)
+    cfg = M.make_config(T=T, H=H, E=E, K=K, F=F, S=2, capacity=C, row_align=128, act="bf16")
+    emu = EpOnOneDevice(cfg, W, DEV, timeout_us=5000)
+    emu_out = None
+    for step in range(2):
+        logits, xs, w_gu, w_d = make_case(W, T, H, E, K, F, "bf16", seed=50 + step)
+        emu, emu_out = run_ep(cfg, W, logits, xs, w_gu, w_d, emu)
+        for r in range(W):
+            assert emu.status(r) == M.MOE_OK
+            assert torch.equal(emu_out[r], one_rank_layer(cfg, logits[r], xs[r], w_gu, w_d))
+    emu.epoch += 1
+    ep = emu.ep(0)
+    logits, xs, w_gu, w_d = make_case(W, T, H, E, K, F, "bf16", seed=99)
+    wg, wd = local_weights(w_gu, W, E, 0), local_weights(w_d, W, E, 0)
+    out = torch.zeros(T, H, dtype=torch.bfloat16, device=DEV)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    M.moe_ep_route(cfg, ep, logits[0].to(DEV), emu.sym[0], emu.peers, emu.ws[0])
+    M.moe_ep_dispatch(cfg, ep, xs[0].to(DEV), emu.sym[0], emu.peers, emu.ws[0])
+    M.moe_ep_expert_mlp(cfg, ep, None, wg[0], wd[0], emu.sym[0], emu.peers, emu.ws[0])
+    M.moe_ep_combine(cfg, ep, emu.sym[0], emu.peers, out, emu.ws[0])
+    torch.cuda.synchronize()
+    assert time.perf_counter() - t0 < 5.0
+    assert emu.status(0) == M.MOE_ERR_TIMEOUT
+    assert emu.status(1) == M.MOE_OK
+    f1 = emu.views(1)["flags"].cpu().numpy()
+    assert f1[0, 0] == emu.epoch          # rank 0's counts did arrive
+    assert f1[1, 0] == emu.epoch - 1 and f1[2, 0] == emu.epoch - 1   # nothing after that
