@@ -526,7 +526,16 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
             return [w[r * El:(r + 1) * El] for r in range(Wn)]
         return [torch.cat([w[r * El:(r + 1) * El], w[wl.E:]]).contiguous() for r in range(Wn)]
 
-    wg, wd = local(full["w_gu"]), local(full["w_d"])
+    fp8 = bool(args.fp8)
+    if fp8:   # weights quantised once, before any timing; each rank takes its slice
+        gq, gs = M.quantize_fp8(full["w_gu"])
+        dq, ds = M.quantize_fp8(full["w_d"])
+        lg = M.ep_local_fp8_weights(gq, gs, Wn, wl.E, 2 * wl.F, wl.H)
+        ld = M.ep_local_fp8_weights(dq, ds, Wn, wl.E, wl.H, wl.F)
+        wq = [lg[r] + ld[r] for r in range(Wn)]
+        wg = wd = None
+    else:
+        wg, wd = local(full["w_gu"]), local(full["w_d"])
     del full["w_gu"], full["w_d"]
     logits = [i["logits"] for i in inps]
     xs = [i["x"] for i in inps]
@@ -536,7 +545,10 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
     stream = torch.cuda.current_stream()
 
     def step():
-        emu.forward(logits, xs, wg, wd, outs)
+        if fp8:
+            emu.forward_fp8(logits, xs, wq, outs)
+        else:
+            emu.forward(logits, xs, wg, wd, outs)
 
     step()
     torch.cuda.synchronize()
@@ -562,11 +574,17 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
             M.moe_ep_route(c, emu.ep(r), logits[r], emu.sym[r], emu.peers, emu.ws[r])
         ev[1].record(stream)
         for r in range(Wn):
-            M.moe_ep_dispatch(c, emu.ep(r), xs[r], emu.sym[r], emu.peers, emu.ws[r])
+            if fp8:
+                M.moe_ep_dispatch_fp8(c, emu.ep(r), xs[r], emu.sym[r], emu.peers, emu.ws[r])
+            else:
+                M.moe_ep_dispatch(c, emu.ep(r), xs[r], emu.sym[r], emu.peers, emu.ws[r])
         ev[2].record(stream)
         for r in range(Wn):
-            M.moe_ep_expert_mlp(c, emu.ep(r), xs[r] if wl.n_shared else None, wg[r], wd[r],
-                                emu.sym[r], emu.peers, emu.ws[r])
+            if fp8:
+                M.moe_ep_expert_mlp_fp8(c, emu.ep(r), *wq[r], emu.sym[r], emu.peers, emu.ws[r])
+            else:
+                M.moe_ep_expert_mlp(c, emu.ep(r), xs[r] if wl.n_shared else None, wg[r], wd[r],
+                                    emu.sym[r], emu.peers, emu.ws[r])
         ev[3].record(stream)
         for r in range(Wn):
             M.moe_ep_combine(c, emu.ep(r), emu.sym[r], emu.peers, outs[r], emu.ws[r])
@@ -582,7 +600,9 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
     s_ = 4 if wl.act == "f32" else 2
     Nt = sum(N)
     T, H, F, K = wl.T, wl.H, wl.F, wl.K
-    disp_bytes = Wn * (T * H * s_ + T * K * 8) + Nt * H * s_
+    # fp8 rows: H code bytes and H/128 scale bytes instead of 2H
+    row_out = H * (1 + 1 / 128) if fp8 else H * s_
+    disp_bytes = Wn * (T * H * s_ + T * K * 8) + Nt * row_out
     comb_bytes = Wn * (T * H * s_ + T * K * 12) + Nt * H * s_
     # rows whose owner is another rank: they would cross NVLink in a real group
     remote = 0
@@ -595,9 +615,15 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
     # (and each rank's shared expert) read once, its rows in, h out and back, y out
     active = sum(int(np.count_nonzero(emu.views(r)["recv_counts"].cpu().numpy()))
                  for r in range(Wn)) + Wn * wl.n_shared
-    mlp_bytes = 3.0 * active * H * F * s_ + (Nt + Wn * T * wl.n_shared) * (2 * H + 2 * F) * s_
+    ws_ = 1 if fp8 else s_   # weight, xp and h element size
+    mlp_bytes = (3.0 * active * H * F * ws_ * (1 + (4 / 128 if fp8 else 0))
+                 + (Nt + Wn * T * wl.n_shared) * (H * ws_ + 2 * F * ws_ + H * s_))
     hbm = peaks["hbm_gbs"]
     tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    peak_kind = f"bf16_tflops_sustained ({peaks['source']})"
+    if fp8:   # fp8 dense rate = 2 x bf16 (nominal 4.5 / 2.25 PFLOP/s)
+        tensor_peak *= 2.0
+        peak_kind += " x 2 (nominal fp8/bf16 ratio)"
     mlp_tflops = flops / (ph["expert_mlp"] * 1e-3) / 1e12
     mlp_gbs = mlp_bytes / (ph["expert_mlp"] * 1e-3) / 1e9
     hbm_bound = mlp_bytes / (hbm * 1e9) > flops / (tensor_peak * 1e12)
@@ -605,7 +631,7 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
         "metric": METRIC, "value": Wn * T / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if wl.act == "bf16" else "f32", "data": "synthetic",
+        "dtype": ("fp8" if fp8 else "bf16") if wl.act == "bf16" else "f32", "data": "synthetic",
         "config": {"workload": f"{wl.name}_ep{Wn}_one_device", "T_per_rank": T, "H": H,
                    "E": wl.E, "K": K, "F": F, "S": wl.S, "cf": wl.cf, "capacity": C,
                    "row_align": wl.row_align, "ranks": Wn, "effective_tokens": Nt,
@@ -621,8 +647,7 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
                      if hbm_bound else
                      {"bound": "tensor", "kernel": "expert_mlp (all ranks' grouped GEMMs)",
                       "achieved": mlp_tflops, "peak": tensor_peak, "unit": "TFLOP/s",
-                      "frac": mlp_tflops / tensor_peak,
-                      "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
+                      "frac": mlp_tflops / tensor_peak, "peak_kind": peak_kind,
                       "hbm_frac": mlp_gbs / hbm}) | {"traffic": None},
         "kernels": {
             "phase_timing": "CUDA events around each step for all ranks (wait kernels included)",
@@ -634,8 +659,10 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
             "combine_us": ph["combine"] * 1e3,
             "combine_gbs": comb_bytes / (ph["combine"] * 1e-3) / 1e9,
             "remote_rows": remote,
-            "remote_bytes_each_way": remote * H * s_,
-            "nvlink_us_each_way_at_770_gbs_per_gpu": remote * H * s_ / Wn / 770e9 * 1e6,
+            "remote_bytes_dispatch": remote * row_out,
+            "remote_bytes_combine": remote * H * s_,
+            "nvlink_us_at_770_gbs_per_gpu": {"dispatch": remote * row_out / Wn / 770e9 * 1e6,
+                                              "combine": remote * H * s_ / Wn / 770e9 * 1e6},
         },
         "clocks": clk,
         "cpu_baseline": None,
@@ -677,8 +704,8 @@ def main(argv=None):
     if args.impl == "reference":
         return run_reference(args, wl, world, rank)
     if args.ep_emulate:
-        if world > 1 or args.fp8:
-            raise SystemExit("--ep-emulate runs on one GPU, bf16 or fp32")
+        if world > 1:
+            raise SystemExit("--ep-emulate runs on one GPU")
         return run_ep_emulated(args, wl, args.ep_emulate)
 
     import torch.distributed as dist

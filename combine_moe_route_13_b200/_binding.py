@@ -40,7 +40,8 @@ EXPORTS = ("moe_capacity", "moe_max_rows", "moe_check_config", "moe_route_worksp
            "moe_ep_recv_rows", "moe_ep_symmetric_bytes", "moe_ep_workspace_bytes", "moe_ep_check",
            "moe_ep_aux", "moe_ep_symmetric_init", "moe_ep_route", "moe_ep_dispatch",
            "moe_ep_expert_mlp", "moe_ep_combine", "moe_ep_layer_forward", "moe_ep_sym_alloc",
-           "moe_ep_sym_free", "moe_ipc_get_handle", "moe_ipc_open", "moe_ipc_close")
+           "moe_ep_sym_free", "moe_ipc_get_handle", "moe_ipc_open", "moe_ipc_close",
+           "moe_ep_dispatch_fp8", "moe_ep_expert_mlp_fp8", "moe_ep_layer_forward_fp8")
 
 
 class MoeError(RuntimeError):
@@ -75,7 +76,8 @@ class MoeEpAux(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "topk_idx", "expert_counts", "overflow", "expert_offsets", "segment_offsets",
         "token_slot", "row_src", "totals", "topk_w", "counts_all", "flags", "send_dst_row",
-        "recv_offsets", "recv_counts", "xr", "h", "y", "h_shared", "y_shared")]
+        "recv_offsets", "recv_counts", "xr", "h", "y", "h_shared", "y_shared",
+        "xq", "xs", "hq", "hs")]
 
 
 _P = ctypes.c_void_p
@@ -132,6 +134,10 @@ def _load():
         "moe_ep_combine": (ctypes.c_int, [_CFG, _EP, _P, _P, _P, _P, _SZ, _P]),
         "moe_ep_layer_forward": (ctypes.c_int, [_CFG, _EP, _P, _P, _P, _P, _P, _P, _P,
                                                 ctypes.POINTER(MoeEpAux), _P, _SZ, _P]),
+        "moe_ep_dispatch_fp8": (ctypes.c_int, [_CFG, _EP, _P, _P, _P, _P, _SZ, _P]),
+        "moe_ep_expert_mlp_fp8": (ctypes.c_int, [_CFG, _EP, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+        "moe_ep_layer_forward_fp8": (ctypes.c_int, [_CFG, _EP, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                                    ctypes.POINTER(MoeEpAux), _P, _SZ, _P]),
         "moe_ep_sym_alloc": (ctypes.c_int, [_SZ, ctypes.POINTER(ctypes.c_void_p)]),
         "moe_ep_sym_free": (ctypes.c_int, [_P]),
         "moe_ipc_get_handle": (ctypes.c_int, [_P, ctypes.c_char_p]),
@@ -561,6 +567,44 @@ def moe_ep_layer_forward(cfg, ep, logits, x, w_gu_local, w_d_local, sym, peers, 
     return aux
 
 
+def moe_ep_dispatch_fp8(cfg, ep, x, sym, peers, ws, stream=None):
+    _check(LIB.moe_ep_dispatch_fp8(ctypes.byref(cfg), ctypes.byref(ep),
+                                   _ptr(x, torch.bfloat16, "x"), _addr(sym, "sym"), _peers(peers),
+                                   _ptr(ws, name="ws"), _nbytes(ws), _stream(stream)),
+           "moe_ep_dispatch_fp8")
+
+
+def moe_ep_expert_mlp_fp8(cfg, ep, wq_gu_local, ws_gu_local, wq_d_local, ws_d_local, sym, peers,
+                          ws, stream=None):
+    _check(LIB.moe_ep_expert_mlp_fp8(
+        ctypes.byref(cfg), ctypes.byref(ep), _ptr(wq_gu_local, U8, "wq_gu_local"),
+        _ptr(ws_gu_local, U8, "ws_gu_local"), _ptr(wq_d_local, U8, "wq_d_local"),
+        _ptr(ws_d_local, U8, "ws_d_local"), _addr(sym, "sym"), _peers(peers), _ptr(ws, name="ws"),
+        _nbytes(ws), _stream(stream)), "moe_ep_expert_mlp_fp8")
+
+
+def moe_ep_layer_forward_fp8(cfg, ep, logits, x, wq_gu_local, ws_gu_local, wq_d_local,
+                             ws_d_local, sym, peers, out, ws, stream=None) -> MoeEpAux:
+    aux = MoeEpAux()
+    _check(LIB.moe_ep_layer_forward_fp8(
+        ctypes.byref(cfg), ctypes.byref(ep), _ptr(logits, torch.float32, "logits"),
+        _ptr(x, torch.bfloat16, "x"), _ptr(wq_gu_local, U8, "wq_gu_local"),
+        _ptr(ws_gu_local, U8, "ws_gu_local"), _ptr(wq_d_local, U8, "wq_d_local"),
+        _ptr(ws_d_local, U8, "ws_d_local"), _addr(sym, "sym"), _peers(peers),
+        _ptr(out, torch.bfloat16, "out"), ctypes.byref(aux), _ptr(ws, name="ws"), _nbytes(ws),
+        _stream(stream)), "moe_ep_layer_forward_fp8")
+    return aux
+
+
+def ep_local_fp8_weights(wq, sf, world: int, E: int, rows_per_expert: int, cols: int) -> list:
+    """Each rank's slice of weights quantised by quantize_fp8 over all E experts
+    ([E, rows_per_expert, cols] codes and their blocked scales): (codes, scales)
+    per rank. rows_per_expert must be a multiple of 128 (the scale row blocks)."""
+    El = E // world
+    per = rows_per_expert // 128 * ((cols // 128 + 3) // 4) * 512   # scale bytes per expert
+    return [(wq[r * El:(r + 1) * El], sf[r * El * per:(r + 1) * El * per]) for r in range(world)]
+
+
 def moe_ep_sym_alloc(nbytes: int) -> int:
     p = ctypes.c_void_p()
     _check(LIB.moe_ep_sym_alloc(int(nbytes), ctypes.byref(p)), "moe_ep_sym_alloc")
@@ -628,4 +672,8 @@ def ep_views(cfg: MoeConfig, world: int, sym: torch.Tensor, ws: torch.Tensor,
         if aux.h_shared else None,
         "y_shared": view(ws, aux.y_shared, cfg.T * cfg.H * es, dt, (cfg.T, cfg.H))
         if aux.y_shared else None,
+        "xq": view(sym, aux.xq, R * cfg.H, U8, (R, cfg.H)) if aux.xq else None,
+        "xs": view(sym, aux.xs, moe_fp8_scale_bytes(R, cfg.H), U8, (-1,)) if aux.xs else None,
+        "hq": view(ws, aux.hq, R * cfg.F, U8, (R, cfg.F)) if aux.hq else None,
+        "hs": view(ws, aux.hs, moe_fp8_scale_bytes(R, cfg.F), U8, (-1,)) if aux.hs else None,
     }

@@ -39,6 +39,7 @@
 #include <climits>
 #include <cstring>
 
+#include "fp8_util.cuh"
 #include "moe_internal.h"
 #include "vec_util.cuh"
 #include "../../include/moe_ep.h"
@@ -82,6 +83,15 @@ moe_config_t local_cfg(const moe_config_t& c, int W) {
   return l;
 }
 
+// Bytes of an fp8 payload of `rows` rows of `cols` values: the codes, then (from
+// the next 256-byte boundary) the scale bytes; 0 where cols is not a multiple
+// of the scale block. The fp8 layer keeps xq/xs in the xr region and hq/hs in
+// the h region.
+size_t fp8_bytes(int64_t rows, int64_t cols) {
+  if (cols % FP8_BLOCK != 0) return 0;
+  return align256((size_t)rows * cols) + (size_t)sf_bytes(rows, cols);
+}
+
 SymLayout sym_layout(const moe_config_t& c, int W) {
   SymLayout L;
   const int64_t R = recv_rows(c, W);
@@ -89,7 +99,7 @@ SymLayout sym_layout(const moe_config_t& c, int W) {
   size_t p = 0;
   L.counts = p; p += align256((size_t)W * c.E * 4);
   L.flags = p;  p += align256((size_t)NUM_FLAGS * W * 4);
-  L.xr = p;     p += align256((size_t)R * c.H * as);
+  L.xr = p;     p += align256(std::max<size_t>((size_t)R * c.H * as, fp8_bytes(R, c.H)));
   L.y = p;      p += align256((size_t)R * c.H * as);
   L.total = p;
   return L;
@@ -114,7 +124,8 @@ EpWs ep_ws_layout(const moe_config_t& c, int W) {
   L.send_dst = p;  p += align256((size_t)c.E * 4);
   L.recv_off = p;  p += align256((size_t)(El + 1) * 4);
   L.recv_cnt = p;  p += align256((size_t)El * 4);
-  L.h = p;         p += align256((size_t)recv_rows(c, W) * c.F * act_size(c.act_dtype));
+  L.h = p;         p += align256(std::max<size_t>((size_t)recv_rows(c, W) * c.F * act_size(c.act_dtype),
+                                                 fp8_bytes(recv_rows(c, W), c.F)));
   if (c.n_shared) {   // the shared expert's h and y for this rank's own tokens
     L.h_sh = p;    p += align256((size_t)c.T * c.F * act_size(c.act_dtype));
     L.y_sh = p;    p += align256((size_t)c.T * c.H * act_size(c.act_dtype));
@@ -137,6 +148,16 @@ moe_status_t ep_validate(const moe_config_t* c, const moe_ep_t* ep) {
   if (recv_rows(*c, W) > INT_MAX / 2) return MOE_ERR_UNSUPPORTED;
   const moe_config_t l = local_cfg(*c, W);
   return validate(&l, true);
+}
+
+// The fp8 expert-parallel layer: the fp8 grouped GEMM's limits on each rank's
+// local experts, and no shared expert.
+moe_status_t ep_validate_fp8(const moe_config_t* c, const moe_ep_t* ep) {
+  moe_status_t st = ep_validate(c, ep);
+  if (st != MOE_OK) return st;
+  if (c->n_shared != 0) return MOE_ERR_UNSUPPORTED;
+  const moe_config_t l = local_cfg(*c, ep->world);
+  return validate_fp8(&l);
 }
 
 moe_status_t ws_check(const moe_config_t& c, int W, const void* ws, size_t ws_bytes) {
@@ -332,6 +353,93 @@ ep_dispatch_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ topk
           const int v = v0 + u * EP_THREADS;
           if (v < row_vecs) dst[v] = dv[u];
         }
+      }
+    }
+  }
+}
+
+// The fp8 form of ep_dispatch_kernel: each kept token row is read once and
+// quantised once, with the arithmetic of the one-rank fp8 dispatch (e4m3 codes,
+// one UE8M0 scale per 128 values: a half-warp's 16 threads cover one block),
+// and its codes and scale bytes are stored to each destination row of the
+// owners' xq / xs.
+__global__ void __launch_bounds__(EP_THREADS)
+ep_dispatch_fp8_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ topk_idx,
+                       const int32_t* __restrict__ token_slot, const int32_t* __restrict__ offsets,
+                       const int32_t* __restrict__ send_dst, void* const* __restrict__ peers,
+                       size_t xq_off, size_t xs_off, int T, int K, int E, int El, int W,
+                       int row_vecs, int slot_end, long long n_recv, uint32_t* status) {
+  __shared__ char* s_base[MAX_K];
+  __shared__ long long s_row[MAX_K];
+  __shared__ char* s_peer[MAX_W];
+  __shared__ int s_n, s_skip;
+  pdl_wait();
+  pdl_trigger();
+  if (threadIdx.x < W) s_peer[threadIdx.x] = static_cast<char*>(peers[threadIdx.x]);
+  if (threadIdx.x == 0) s_skip = timed_out(status);
+  __syncthreads();
+  if (s_skip) return;   // the same decision for every thread of the block
+  const int k = threadIdx.x;
+  const int64_t H = (int64_t)row_vecs * 8;
+  const int KB = row_vecs / 16;
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    __syncthreads();   // the previous token's readers of s_base, s_row, s_n are done
+    if (k < 32) {
+      long long row = -1;
+      int d = 0;
+      if (k < K) {
+        const int sl = token_slot[(size_t)t * K + k];
+        const int e = topk_idx[(size_t)t * K + k];
+        if (sl >= 0 && sl < slot_end) {
+          row = (e >= 0 && e < E) ? (long long)send_dst[e] + (sl - offsets[e]) : -1;
+          if (row < 0 || row >= n_recv) {
+            atomicCAS(status, 0u, (uint32_t)MOE_ERR_DEVICE_INPUT);
+            row = -1;
+          }
+          d = row >= 0 ? e / El : 0;
+        }
+      }
+      const unsigned m = __ballot_sync(0xffffffffu, row >= 0);
+      if (row >= 0) {
+        const int pos = __popc(m & ((1u << k) - 1u));
+        s_base[pos] = s_peer[d];
+        s_row[pos] = row;
+      }
+      if (k == 0) s_n = __popc(m);
+    }
+    __syncthreads();
+    const int n = s_n;
+    if (n == 0) continue;   // every assignment of this token overflowed
+    const uint4* src = x + (size_t)t * row_vecs;
+    // row_vecs is a multiple of 16 and v0 of 128: a half-warp is all valid or all not
+    for (int v0 = 0; v0 < row_vecs; v0 += EP_THREADS) {
+      const int v = v0 + (int)threadIdx.x;
+      const bool valid = v < row_vecs;
+      float f[8];
+      if (valid) {
+        unpack_bf16x8(__ldcs(src + v), f);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = 0.f;
+      }
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+      for (int o = 1; o < 16; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      if (!valid) continue;
+      const int p = fp8_scale_exp(amax);
+      const float inv = fp8_inv_scale(p);
+      uint2 c;
+      c.x = fp8x2(f[0] * inv, f[1] * inv) | (fp8x2(f[2] * inv, f[3] * inv) << 16);
+      c.y = fp8x2(f[4] * inv, f[5] * inv) | (fp8x2(f[6] * inv, f[7] * inv) << 16);
+      const uint8_t sbyte = (uint8_t)(p + 127);
+      const int kb = v / 16;
+      for (int j = 0; j < n; ++j) {
+        char* base = s_base[j];
+        const long long r = s_row[j];
+        *reinterpret_cast<uint2*>(base + xq_off + r * H + (int64_t)v * 8) = c;
+        if ((threadIdx.x & 15) == 0) base[xs_off + sf_offset(r, kb, KB)] = (char)sbyte;
       }
     }
   }
@@ -590,6 +698,13 @@ moe_status_t moe_ep_aux(const moe_config_t* cfg, const moe_ep_t* ep, void* sym, 
   a.y = sb + S.y;
   a.h_shared = p.h_sh;
   a.y_shared = p.y_sh;
+  if (cfg->H % FP8_BLOCK == 0 && cfg->F % FP8_BLOCK == 0) {   // the fp8 layer's payload
+    const int64_t R = recv_rows(*cfg, ep->world);
+    a.xq = reinterpret_cast<uint8_t*>(sb + S.xr);
+    a.xs = reinterpret_cast<uint8_t*>(sb + S.xr + align256((size_t)R * cfg->H));
+    a.hq = reinterpret_cast<uint8_t*>(p.h);
+    a.hs = reinterpret_cast<uint8_t*>(p.h + align256((size_t)R * cfg->F));
+  }
   *aux = a;
   return MOE_OK;
 }
@@ -739,6 +854,94 @@ moe_status_t moe_ep_layer_forward(const moe_config_t* cfg, const moe_ep_t* ep,
   if ((st = moe_ep_dispatch(cfg, ep, x, sym, peers, ws, ws_bytes, stream)) != MOE_OK) return st;
   if ((st = moe_ep_expert_mlp(cfg, ep, x, w_gu_local, w_d_local, sym, peers, ws, ws_bytes,
                               stream)) != MOE_OK)
+    return st;
+  return moe_ep_combine(cfg, ep, sym, peers, out, ws, ws_bytes, stream);
+}
+
+moe_status_t moe_ep_dispatch_fp8(const moe_config_t* cfg, const moe_ep_t* ep, const void* x,
+                                 void* sym, void* const* peers, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  moe_status_t st = ep_validate_fp8(cfg, ep);
+  if (st != MOE_OK) return st;
+  if ((st = common_checks(cfg, ep, sym, peers, ws, ws_bytes)) != MOE_OK) return st;
+  if (cfg->T > 0 && (!x || !aligned16(x))) return MOE_ERR_INVALID_ARG;
+  const moe_config_t& c = *cfg;
+  const int W = ep->world;
+  const Ptrs p = ws_ptrs(c, W, ws);
+  const SymLayout S = sym_layout(c, W);
+  const int64_t R = recv_rows(c, W);
+  char* sb = static_cast<char*>(sym);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = cuda_st(launch_pdl(ep_plan_kernel, dim3(1), dim3(PLAN_THREADS), 0, s,
+                          (const int32_t*)(sb + S.counts), (const uint32_t*)(sb + S.flags), c.E,
+                          W, ep->rank, c.capacity, c.row_align, ep->epoch, timeout_ns(*ep),
+                          p.status, p.send_dst, p.recv_off, p.recv_cnt));
+  if (st != MOE_OK) return st;
+  if (c.T > 0) {
+    st = cuda_st(launch_pdl(ep_dispatch_fp8_kernel,
+                            dim3(resident_grid(ep_dispatch_fp8_kernel, EP_THREADS, c.T)),
+                            dim3(EP_THREADS), 0, s, static_cast<const uint4*>(x),
+                            (const int32_t*)p.topk_idx, (const int32_t*)p.slot,
+                            (const int32_t*)p.offsets, (const int32_t*)p.send_dst, peers, S.xr,
+                            S.xr + align256((size_t)R * c.H), c.T, c.K, c.E, c.E / W, W,
+                            c.H / 8, (int)routed_rows(c), (long long)R, p.status));
+    if (st != MOE_OK) return st;
+  }
+  return cuda_st(launch_pdl(ep_signal_kernel, dim3(1), dim3(MAX_W), 0, s, peers, S.flags,
+                            (int)FLAG_DISPATCH, W, ep->rank, ep->epoch,
+                            (const uint32_t*)p.status));
+}
+
+moe_status_t moe_ep_expert_mlp_fp8(const moe_config_t* cfg, const moe_ep_t* ep,
+                                   const uint8_t* wq_gu_local, const uint8_t* ws_gu_local,
+                                   const uint8_t* wq_d_local, const uint8_t* ws_d_local,
+                                   void* sym, void* const* peers, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  moe_status_t st = ep_validate_fp8(cfg, ep);
+  if (st != MOE_OK) return st;
+  if ((st = common_checks(cfg, ep, sym, peers, ws, ws_bytes)) != MOE_OK) return st;
+  for (const void* w : {(const void*)wq_gu_local, (const void*)ws_gu_local,
+                        (const void*)wq_d_local, (const void*)ws_d_local})
+    if (!w || !aligned16(w)) return MOE_ERR_INVALID_ARG;
+  const moe_config_t& c = *cfg;
+  const int W = ep->world;
+  const Ptrs p = ws_ptrs(c, W, ws);
+  const SymLayout S = sym_layout(c, W);
+  const int64_t R = recv_rows(c, W);
+  char* sb = static_cast<char*>(sym);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = cuda_st(launch_pdl(ep_wait_kernel, dim3(1), dim3(32), 0, s,
+                          (const uint32_t*)(sb + S.flags) + FLAG_DISPATCH * W, W, ep->epoch,
+                          timeout_ns(*ep), p.status));
+  if (st != MOE_OK) return st;
+  const moe_config_t l = local_cfg(c, W);
+  const uint8_t* xq = reinterpret_cast<const uint8_t*>(sb + S.xr);
+  const uint8_t* xs = xq + align256((size_t)R * c.H);
+  uint8_t* hq = reinterpret_cast<uint8_t*>(p.h);
+  uint8_t* hs = hq + align256((size_t)R * c.F);
+  st = launch_mlp_fp8(l, xq, xs, p.recv_off, p.recv_cnt, wq_gu_local, ws_gu_local, wq_d_local,
+                      ws_d_local, hq, hs, sb + S.y, R, p.status, s);
+  if (st != MOE_OK) return st;
+  return cuda_st(launch_pdl(ep_signal_kernel, dim3(1), dim3(MAX_W), 0, s, peers, S.flags,
+                            (int)FLAG_Y, W, ep->rank, ep->epoch, (const uint32_t*)p.status));
+}
+
+moe_status_t moe_ep_layer_forward_fp8(const moe_config_t* cfg, const moe_ep_t* ep,
+                                      const float* logits, const void* x,
+                                      const uint8_t* wq_gu_local, const uint8_t* ws_gu_local,
+                                      const uint8_t* wq_d_local, const uint8_t* ws_d_local,
+                                      void* sym, void* const* peers, void* out,
+                                      moe_ep_aux_t* aux, void* ws, size_t ws_bytes,
+                                      void* stream) {
+  moe_status_t st = ep_validate_fp8(cfg, ep);
+  if (st != MOE_OK) return st;
+  if ((st = common_checks(cfg, ep, sym, peers, ws, ws_bytes)) != MOE_OK) return st;
+  if (aux && (st = moe_ep_aux(cfg, ep, sym, ws, aux)) != MOE_OK) return st;
+  if ((st = moe_ep_route(cfg, ep, logits, sym, peers, ws, ws_bytes, stream)) != MOE_OK) return st;
+  if ((st = moe_ep_dispatch_fp8(cfg, ep, x, sym, peers, ws, ws_bytes, stream)) != MOE_OK)
+    return st;
+  if ((st = moe_ep_expert_mlp_fp8(cfg, ep, wq_gu_local, ws_gu_local, wq_d_local, ws_d_local, sym,
+                                  peers, ws, ws_bytes, stream)) != MOE_OK)
     return st;
   return moe_ep_combine(cfg, ep, sym, peers, out, ws, ws_bytes, stream);
 }

@@ -121,6 +121,22 @@ class EpOnOneDevice:
         for r in range(W):
             B.moe_ep_combine(c, self.ep(r), self.sym[r], self.peers, out[r], self.ws[r], stream)
 
+    def forward_fp8(self, logits: Sequence, x: Sequence, wq: Sequence, out: Sequence,
+                    stream=None):
+        """One step of every rank with the fp8 payload; wq[r] = (codes and scales
+        of rank r's gate/up weights, codes and scales of its down weights)."""
+        self.epoch += 1
+        c, W = self.cfg, self.world
+        for r in range(W):
+            B.moe_ep_route(c, self.ep(r), logits[r], self.sym[r], self.peers, self.ws[r], stream)
+        for r in range(W):
+            B.moe_ep_dispatch_fp8(c, self.ep(r), x[r], self.sym[r], self.peers, self.ws[r], stream)
+        for r in range(W):
+            B.moe_ep_expert_mlp_fp8(c, self.ep(r), *wq[r], self.sym[r], self.peers, self.ws[r],
+                                    stream)
+        for r in range(W):
+            B.moe_ep_combine(c, self.ep(r), self.sym[r], self.peers, out[r], self.ws[r], stream)
+
     def views(self, rank: int) -> dict:
         aux = B.moe_ep_aux(self.cfg, self.ep(rank) if self.epoch else B.make_ep(self.world, rank, 1),
                            self.sym[rank], self.ws[rank])

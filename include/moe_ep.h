@@ -115,6 +115,8 @@ typedef struct {
   int32_t *recv_counts;    /* [E/W]: rows each local expert received */
   void *xr, *h, *y;        /* [R_recv][H] (symmetric), [R_recv][F] (private), [R_recv][H] (symmetric) */
   void *h_shared, *y_shared;   /* [T][F], [T][H] (private): the shared expert on this rank's tokens; NULL without one */
+  uint8_t *xq, *xs;        /* fp8 layer: codes [R_recv][H] and scales, inside xr's region (symmetric) */
+  uint8_t *hq, *hs;        /* fp8 layer: codes [R_recv][F] and scales, inside h's region (private) */
 } moe_ep_aux_t;
 
 /* R_recv (see above); -1 for an invalid config or world. */
@@ -152,6 +154,40 @@ moe_status_t moe_ep_layer_forward(const moe_config_t* cfg, const moe_ep_t* ep,
                                   const void* w_d_local, void* sym, void* const* peers,
                                   void* out, moe_ep_aux_t* aux, void* ws, size_t ws_bytes,
                                   void* stream);
+
+/* fp8 payload (the pages' production precision for the dispatch, with a bf16
+ * combine: EFA page, "Оценка"; block scale factors travel beside the tokens:
+ * pplx-kernels page, "Dispatch"). The route and the combine are the bf16
+ * layer's (moe_ep_route, moe_ep_combine).
+ *   moe_ep_dispatch_fp8: as moe_ep_dispatch, but each kept token row is
+ *     quantised once (e4m3 codes, one UE8M0 scale per 128 values, the format
+ *     and scale layout of moe_dispatch_fp8 in moe.h) and its codes and scales
+ *     are written into the owner's xq / xs (the bytes crossing to a peer halve).
+ *   moe_ep_expert_mlp_fp8: as moe_ep_expert_mlp with the block-scaled fp8
+ *     grouped GEMMs of moe_expert_mlp_fp8 on the local experts (h quantised
+ *     to fp8 in the gate/up epilogue, y in bf16). wq_gu_local [E/W][2F][H] and
+ *     wq_d_local [E/W][H][F] are codes of this rank's experts, ws_gu_local /
+ *     ws_d_local their scales in the blocked layout (for the experts of rank d,
+ *     the contiguous slice of moe_quantize_fp8's scales of all experts that
+ *     starts at chunk row d*(E/W)*2F/128, resp. d*(E/W)*H/128).
+ * Limits: those of moe_layer_forward_fp8 on each rank's local experts
+ * (bf16 activations, H % 256 == 0, F % 128 == 0, A % 128 == 0), and no
+ * shared expert; else MOE_ERR_UNSUPPORTED. */
+moe_status_t moe_ep_dispatch_fp8(const moe_config_t* cfg, const moe_ep_t* ep, const void* x,
+                                 void* sym, void* const* peers, void* ws, size_t ws_bytes,
+                                 void* stream);
+moe_status_t moe_ep_expert_mlp_fp8(const moe_config_t* cfg, const moe_ep_t* ep,
+                                   const uint8_t* wq_gu_local, const uint8_t* ws_gu_local,
+                                   const uint8_t* wq_d_local, const uint8_t* ws_d_local,
+                                   void* sym, void* const* peers, void* ws, size_t ws_bytes,
+                                   void* stream);
+moe_status_t moe_ep_layer_forward_fp8(const moe_config_t* cfg, const moe_ep_t* ep,
+                                      const float* logits, const void* x,
+                                      const uint8_t* wq_gu_local, const uint8_t* ws_gu_local,
+                                      const uint8_t* wq_d_local, const uint8_t* ws_d_local,
+                                      void* sym, void* const* peers, void* out,
+                                      moe_ep_aux_t* aux, void* ws, size_t ws_bytes,
+                                      void* stream);
 
 /* Setup (not the hot path): a symmetric region another process can map.
  * moe_ep_sym_alloc: cudaMalloc of `bytes` on the current device (its own

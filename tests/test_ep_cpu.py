@@ -68,6 +68,22 @@ def test_shared_expert_needs_bf16():
     assert M.moe_ep_check(c, M.make_ep(2, 0, 1)) == M.MOE_ERR_UNSUPPORTED
 
 
+@pytest.mark.parametrize("kw,code", [
+    (dict(), M.MOE_OK),
+    (dict(n_shared=1), M.MOE_ERR_UNSUPPORTED),
+    (dict(H=4160), M.MOE_ERR_UNSUPPORTED),      # H % 256 != 0
+    (dict(F=14400), M.MOE_ERR_UNSUPPORTED),     # F % 128 != 0
+])
+def test_fp8_entry_points_check_the_fp8_limits(kw, code):
+    c = cfg_of("mixtral", **kw)
+    ep = M.make_ep(2, 0, 1)
+    big, fake = 1 << 40, 1 << 40
+    got = M.LIB.moe_ep_dispatch_fp8(ctypes.byref(c), ctypes.byref(ep), fake, fake, fake, None,
+                                    big, None)
+    # with a valid configuration the missing workspace is the first error found
+    assert got == (M.MOE_ERR_WORKSPACE if code == M.MOE_OK else code)
+
+
 def test_too_many_ranks_unsupported():
     c = M.make_config(T=64, H=256, E=128, K=2, F=256, S=128, capacity=8)
     assert M.moe_ep_check(c, M.make_ep(128, 0, 1)) == M.MOE_ERR_UNSUPPORTED
