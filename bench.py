@@ -639,7 +639,9 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
                    "parallelism": f"ep{Wn} emulated on one GPU (exchanges through local HBM)",
                    "l2": "flushed before every step: 256 MB written, then another 256 MB read"},
         "e2e": None,
-        "gpu_launches": None,
+        # per rank and step: route 3, publish, plan, dispatch, signal, wait, 2 GEMMs,
+        # signal, wait, combine (+2 GEMMs of the shared expert)
+        "gpu_launches": (13 + 2 * wl.n_shared) * Wn * args.steps,
         "roofline": ({"bound": "hbm", "kernel": "expert_mlp (all ranks' grouped GEMMs)",
                       "achieved": mlp_gbs, "peak": hbm, "unit": "GB/s", "frac": mlp_gbs / hbm,
                       "peak_kind": f"hbm_gbs ({peaks['source']})",
