@@ -41,7 +41,8 @@ EXPORTS = ("moe_capacity", "moe_max_rows", "moe_check_config", "moe_route_worksp
            "moe_ep_aux", "moe_ep_symmetric_init", "moe_ep_route", "moe_ep_dispatch",
            "moe_ep_expert_mlp", "moe_ep_combine", "moe_ep_layer_forward", "moe_ep_sym_alloc",
            "moe_ep_sym_free", "moe_ipc_get_handle", "moe_ipc_open", "moe_ipc_close",
-           "moe_ep_dispatch_fp8", "moe_ep_expert_mlp_fp8", "moe_ep_layer_forward_fp8")
+           "moe_ep_dispatch_fp8", "moe_ep_expert_mlp_fp8", "moe_ep_layer_forward_fp8",
+           "moe_ep_workspace_init")
 
 
 class MoeError(RuntimeError):
@@ -128,6 +129,7 @@ def _load():
         "moe_ep_check": (ctypes.c_int, [_CFG, _EP]),
         "moe_ep_aux": (ctypes.c_int, [_CFG, _EP, _P, _P, ctypes.POINTER(MoeEpAux)]),
         "moe_ep_symmetric_init": (ctypes.c_int, [_CFG, ctypes.c_int32, _P, _SZ, _P]),
+        "moe_ep_workspace_init": (ctypes.c_int, [_CFG, ctypes.c_int32, _P, _SZ, _P]),
         "moe_ep_route": (ctypes.c_int, [_CFG, _EP, _P, _P, _P, _P, _SZ, _P]),
         "moe_ep_dispatch": (ctypes.c_int, [_CFG, _EP, _P, _P, _P, _P, _SZ, _P]),
         "moe_ep_expert_mlp": (ctypes.c_int, [_CFG, _EP, _P, _P, _P, _P, _P, _P, _SZ, _P]),
@@ -521,6 +523,11 @@ def moe_ep_symmetric_init(cfg, world, sym, sym_bytes=None, stream=None):
     n = _nbytes(sym) if sym_bytes is None else int(sym_bytes)
     _check(LIB.moe_ep_symmetric_init(ctypes.byref(cfg), int(world), _addr(sym, "sym"), n,
                                      _stream(stream)), "moe_ep_symmetric_init")
+
+
+def moe_ep_workspace_init(cfg, world, ws, stream=None):
+    _check(LIB.moe_ep_workspace_init(ctypes.byref(cfg), int(world), _ptr(ws, name="ws"),
+                                     _nbytes(ws), _stream(stream)), "moe_ep_workspace_init")
 
 
 def _peers(peers):

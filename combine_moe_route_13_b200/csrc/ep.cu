@@ -34,7 +34,10 @@
 //             assignments, read in place, weighted sum in k order, plus the
 //             rank's own shared-expert row with weight 1
 // Flags hold the step number (epoch) and are compared as "reached", so they
-// are never reset. Every wait is bounded; see moe_ep.h for the error rules.
+// are never reset. The step number is the caller's, or (epoch 0) one past a
+// step counter in the workspace that the last wait of every step advances, so
+// that a captured step can be replayed. Every wait is bounded; see moe_ep.h
+// for the error rules.
 #include <algorithm>
 #include <climits>
 #include <cstring>
@@ -60,7 +63,8 @@ struct SymLayout {
 struct EpWs {
   size_t blk_cnt = 0, topk_idx = 0, topk_w = 0, counts = 0, overflow = 0, offsets = 0;
   size_t segoff = 0, totals = 0, slot = 0, row_src = 0;
-  size_t send_dst = 0, recv_off = 0, recv_cnt = 0, h = 0, h_sh = 0, y_sh = 0, total = 0;
+  size_t send_dst = 0, recv_off = 0, recv_cnt = 0, epoch = 0, h = 0, h_sh = 0, y_sh = 0;
+  size_t total = 0;
 };
 
 int64_t recv_rows(const moe_config_t& c, int W) {
@@ -124,6 +128,7 @@ EpWs ep_ws_layout(const moe_config_t& c, int W) {
   L.send_dst = p;  p += align256((size_t)c.E * 4);
   L.recv_off = p;  p += align256((size_t)(El + 1) * 4);
   L.recv_cnt = p;  p += align256((size_t)El * 4);
+  L.epoch = p;     p += 256;   // the device-resident step counter
   L.h = p;         p += align256(std::max<size_t>((size_t)recv_rows(c, W) * c.F * act_size(c.act_dtype),
                                                  fp8_bytes(recv_rows(c, W), c.F)));
   if (c.n_shared) {   // the shared expert's h and y for this rank's own tokens
@@ -195,6 +200,18 @@ __device__ __forceinline__ bool reached(uint32_t v, uint32_t epoch) {
   return (int32_t)(v - epoch) >= 0;
 }
 
+// This step's number: the caller's (value > 0), or one past the rank's
+// device-resident step counter (value 0), which the Y wait of the combine
+// advances at the end of every step, so that a captured step can be replayed.
+struct Epoch {
+  uint32_t value;
+  const uint32_t* counter;
+};
+
+__device__ __forceinline__ uint32_t step_epoch(const Epoch& e) {
+  return e.value ? e.value : *(volatile const uint32_t*)e.counter + 1u;
+}
+
 __device__ __forceinline__ uint32_t* peer_flags(void* const* peers, int d, size_t flags_off) {
   return reinterpret_cast<uint32_t*>(static_cast<char*>(peers[d]) + flags_off);
 }
@@ -229,7 +246,7 @@ __device__ __forceinline__ bool timed_out(const uint32_t* status) {
 // the whole block's writes before it).
 __global__ void ep_publish_kernel(const int32_t* __restrict__ counts, int E, int W, int rank,
                                   void* const* __restrict__ peers, size_t counts_off,
-                                  size_t flags_off, uint32_t epoch) {
+                                  size_t flags_off, Epoch epoch) {
   pdl_wait();
   pdl_trigger();
   const int d = blockIdx.x;
@@ -239,7 +256,7 @@ __global__ void ep_publish_kernel(const int32_t* __restrict__ counts, int E, int
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence_system();
-    st_release_sys(peer_flags(peers, d, flags_off) + FLAG_COUNTS * W + rank, epoch);
+    st_release_sys(peer_flags(peers, d, flags_off) + FLAG_COUNTS * W + rank, step_epoch(epoch));
   }
 }
 
@@ -248,14 +265,15 @@ __global__ void ep_publish_kernel(const int32_t* __restrict__ counts, int E, int
 // over all experts and each owner's scan restarts at its first expert.
 __global__ void __launch_bounds__(PLAN_THREADS)
 ep_plan_kernel(const int32_t* __restrict__ counts_all, const uint32_t* flags, int E, int W,
-               int rank, int C, int A, uint32_t epoch, unsigned long long timeout_ns,
+               int rank, int C, int A, Epoch epoch, unsigned long long timeout_ns,
                uint32_t* status, int32_t* __restrict__ send_dst, int32_t* __restrict__ recv_off,
                int32_t* __restrict__ recv_cnt) {
   __shared__ long long s_scan[PLAN_THREADS];
   __shared__ int s_ok;
   pdl_wait();
   pdl_trigger();
-  if (threadIdx.x == 0) s_ok = wait_all(flags + FLAG_COUNTS * W, W, epoch, timeout_ns, status);
+  if (threadIdx.x == 0)
+    s_ok = wait_all(flags + FLAG_COUNTS * W, W, step_epoch(epoch), timeout_ns, status);
   __syncthreads();
   const int e = threadIdx.x;
   const int El = E / W;
@@ -445,24 +463,30 @@ ep_dispatch_fp8_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ 
   }
 }
 
-__global__ void ep_wait_kernel(const uint32_t* flags, int W, uint32_t epoch,
-                               unsigned long long timeout_ns, uint32_t* status) {
+// advance (the last wait of a step): then move the rank's step counter on
+// (device-resident numbering only).
+__global__ void ep_wait_kernel(const uint32_t* flags, int W, Epoch epoch,
+                               unsigned long long timeout_ns, uint32_t* status, uint32_t* advance) {
   pdl_wait();
   pdl_trigger();
-  if (threadIdx.x == 0) wait_all(flags, W, epoch, timeout_ns, status);
+  if (threadIdx.x == 0) {
+    const uint32_t e = step_epoch(epoch);
+    wait_all(flags, W, e, timeout_ns, status);
+    if (advance && !epoch.value) *advance = e;
+  }
 }
 
 // After the dispatch or the grouped GEMM (pdl_wait: that grid has finished and
 // its stores are visible to this one): every rank's flag `which` for this rank,
 // released at system scope after a system fence. Not after a timeout.
 __global__ void ep_signal_kernel(void* const* __restrict__ peers, size_t flags_off, int which,
-                                 int W, int rank, uint32_t epoch, const uint32_t* status) {
+                                 int W, int rank, Epoch epoch, const uint32_t* status) {
   pdl_wait();
   pdl_trigger();
   const int d = threadIdx.x;
   if (d < W && !timed_out(status)) {
     __threadfence_system();
-    st_release_sys(peer_flags(peers, d, flags_off) + which * W + rank, epoch);
+    st_release_sys(peer_flags(peers, d, flags_off) + which * W + rank, step_epoch(epoch));
   }
 }
 
@@ -600,7 +624,7 @@ struct Ptrs {
   int32_t *topk_idx, *counts, *overflow, *offsets, *segoff, *slot, *row_src, *totals, *blk;
   float* topk_w;
   int32_t *send_dst, *recv_off, *recv_cnt;
-  uint32_t* status;
+  uint32_t *status, *epoch;
   char *h, *h_sh, *y_sh;   // h_sh / y_sh: nullptr without a shared expert
 };
 
@@ -622,6 +646,7 @@ Ptrs ws_ptrs(const moe_config_t& c, int W, void* ws) {
   p.send_dst = reinterpret_cast<int32_t*>(b + L.send_dst);
   p.recv_off = reinterpret_cast<int32_t*>(b + L.recv_off);
   p.recv_cnt = reinterpret_cast<int32_t*>(b + L.recv_cnt);
+  p.epoch = reinterpret_cast<uint32_t*>(b + L.epoch);
   p.h = b + L.h;
   p.h_sh = c.n_shared ? b + L.h_sh : nullptr;
   p.y_sh = c.n_shared ? b + L.y_sh : nullptr;
@@ -632,7 +657,7 @@ moe_status_t common_checks(const moe_config_t* cfg, const moe_ep_t* ep, const vo
                            void* const* peers, const void* ws, size_t ws_bytes) {
   moe_status_t st = ep_validate(cfg, ep);
   if (st != MOE_OK) return st;
-  if (ep->epoch == 0u || !sym || !peers) return MOE_ERR_INVALID_ARG;
+  if (!sym || !peers) return MOE_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(sym) & 255u) return MOE_ERR_INVALID_ARG;
   return ws_check(*cfg, ep->world, ws, ws_bytes);
 }
@@ -667,7 +692,7 @@ size_t moe_ep_workspace_bytes(const moe_config_t* cfg, int32_t world) {
 moe_status_t moe_ep_check(const moe_config_t* cfg, const moe_ep_t* ep) {
   moe_status_t st = ep_validate(cfg, ep);
   if (st != MOE_OK) return st;
-  return ep->epoch == 0u ? MOE_ERR_INVALID_ARG : MOE_OK;
+  return MOE_OK;
 }
 
 moe_status_t moe_ep_aux(const moe_config_t* cfg, const moe_ep_t* ep, void* sym, void* ws,
@@ -709,6 +734,18 @@ moe_status_t moe_ep_aux(const moe_config_t* cfg, const moe_ep_t* ep, void* sym, 
   return MOE_OK;
 }
 
+moe_status_t moe_ep_workspace_init(const moe_config_t* cfg, int32_t world, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  moe_ep_t ep = {world, 0, 1u, 0u};
+  moe_status_t st = ep_validate(cfg, &ep);
+  if (st != MOE_OK) return st;
+  if ((st = ws_check(*cfg, world, ws, ws_bytes)) != MOE_OK) return st;
+  const EpWs L = ep_ws_layout(*cfg, world);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = cuda_st(cudaMemsetAsync(ws, 0, 4, s))) != MOE_OK) return st;   // status word
+  return cuda_st(cudaMemsetAsync(static_cast<char*>(ws) + L.epoch, 0, 4, s));   // step counter
+}
+
 moe_status_t moe_ep_symmetric_init(const moe_config_t* cfg, int32_t world, void* sym,
                                    size_t sym_bytes, void* stream) {
   moe_ep_t ep = {world, 0, 1u, 0u};
@@ -736,7 +773,7 @@ moe_status_t moe_ep_route(const moe_config_t* cfg, const moe_ep_t* ep, const flo
   if (st != MOE_OK) return st;
   return cuda_st(launch_pdl(ep_publish_kernel, dim3(W), dim3(256), 0, s,
                             (const int32_t*)p.counts, c.E, W, ep->rank, peers, S.counts, S.flags,
-                            ep->epoch));
+                            Epoch{ep->epoch, p.epoch}));
 }
 
 moe_status_t moe_ep_dispatch(const moe_config_t* cfg, const moe_ep_t* ep, const void* x,
@@ -753,7 +790,8 @@ moe_status_t moe_ep_dispatch(const moe_config_t* cfg, const moe_ep_t* ep, const 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   st = cuda_st(launch_pdl(ep_plan_kernel, dim3(1), dim3(PLAN_THREADS), 0, s,
                           (const int32_t*)(sb + S.counts), (const uint32_t*)(sb + S.flags), c.E,
-                          W, ep->rank, c.capacity, c.row_align, ep->epoch, timeout_ns(*ep),
+                          W, ep->rank, c.capacity, c.row_align, Epoch{ep->epoch, p.epoch},
+                          timeout_ns(*ep),
                           p.status, p.send_dst, p.recv_off, p.recv_cnt));
   if (st != MOE_OK) return st;
   const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
@@ -768,7 +806,7 @@ moe_status_t moe_ep_dispatch(const moe_config_t* cfg, const moe_ep_t* ep, const 
     if (st != MOE_OK) return st;
   }
   return cuda_st(launch_pdl(ep_signal_kernel, dim3(1), dim3(MAX_W), 0, s, peers, S.flags,
-                            (int)FLAG_DISPATCH, W, ep->rank, ep->epoch,
+                            (int)FLAG_DISPATCH, W, ep->rank, Epoch{ep->epoch, p.epoch},
                             (const uint32_t*)p.status));
 }
 
@@ -796,8 +834,9 @@ moe_status_t moe_ep_expert_mlp(const moe_config_t* cfg, const moe_ep_t* ep, cons
     if (st != MOE_OK) return st;
   }
   st = cuda_st(launch_pdl(ep_wait_kernel, dim3(1), dim3(32), 0, s,
-                          (const uint32_t*)(sb + S.flags) + FLAG_DISPATCH * W, W, ep->epoch,
-                          timeout_ns(*ep), p.status));
+                          (const uint32_t*)(sb + S.flags) + FLAG_DISPATCH * W, W,
+                          Epoch{ep->epoch, p.epoch}, timeout_ns(*ep), p.status,
+                          (uint32_t*)nullptr));
   if (st != MOE_OK) return st;
   const moe_config_t l = local_cfg(c, W);
   const int64_t R = recv_rows(c, W);
@@ -812,7 +851,8 @@ moe_status_t moe_ep_expert_mlp(const moe_config_t* cfg, const moe_ep_t* ep, cons
                                 R, s));
   if (st != MOE_OK) return st;
   return cuda_st(launch_pdl(ep_signal_kernel, dim3(1), dim3(MAX_W), 0, s, peers, S.flags,
-                            (int)FLAG_Y, W, ep->rank, ep->epoch, (const uint32_t*)p.status));
+                            (int)FLAG_Y, W, ep->rank, Epoch{ep->epoch, p.epoch},
+                            (const uint32_t*)p.status));
 }
 
 moe_status_t moe_ep_combine(const moe_config_t* cfg, const moe_ep_t* ep, void* sym,
@@ -828,8 +868,9 @@ moe_status_t moe_ep_combine(const moe_config_t* cfg, const moe_ep_t* ep, void* s
   char* sb = static_cast<char*>(sym);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   st = cuda_st(launch_pdl(ep_wait_kernel, dim3(1), dim3(32), 0, s,
-                          (const uint32_t*)(sb + S.flags) + FLAG_Y * W, W, ep->epoch,
-                          timeout_ns(*ep), p.status));
+                          (const uint32_t*)(sb + S.flags) + FLAG_Y * W, W,
+                          Epoch{ep->epoch, p.epoch}, timeout_ns(*ep), p.status,
+                          p.epoch));   // the step's last wait moves the step counter on
   if (st != MOE_OK || c.T == 0) return st;
   const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
   auto kernel = c.act_dtype == MOE_BF16 ? ep_combine_kernel<true> : ep_combine_kernel<false>;
@@ -874,7 +915,8 @@ moe_status_t moe_ep_dispatch_fp8(const moe_config_t* cfg, const moe_ep_t* ep, co
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   st = cuda_st(launch_pdl(ep_plan_kernel, dim3(1), dim3(PLAN_THREADS), 0, s,
                           (const int32_t*)(sb + S.counts), (const uint32_t*)(sb + S.flags), c.E,
-                          W, ep->rank, c.capacity, c.row_align, ep->epoch, timeout_ns(*ep),
+                          W, ep->rank, c.capacity, c.row_align, Epoch{ep->epoch, p.epoch},
+                          timeout_ns(*ep),
                           p.status, p.send_dst, p.recv_off, p.recv_cnt));
   if (st != MOE_OK) return st;
   if (c.T > 0) {
@@ -888,7 +930,7 @@ moe_status_t moe_ep_dispatch_fp8(const moe_config_t* cfg, const moe_ep_t* ep, co
     if (st != MOE_OK) return st;
   }
   return cuda_st(launch_pdl(ep_signal_kernel, dim3(1), dim3(MAX_W), 0, s, peers, S.flags,
-                            (int)FLAG_DISPATCH, W, ep->rank, ep->epoch,
+                            (int)FLAG_DISPATCH, W, ep->rank, Epoch{ep->epoch, p.epoch},
                             (const uint32_t*)p.status));
 }
 
@@ -911,8 +953,9 @@ moe_status_t moe_ep_expert_mlp_fp8(const moe_config_t* cfg, const moe_ep_t* ep,
   char* sb = static_cast<char*>(sym);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   st = cuda_st(launch_pdl(ep_wait_kernel, dim3(1), dim3(32), 0, s,
-                          (const uint32_t*)(sb + S.flags) + FLAG_DISPATCH * W, W, ep->epoch,
-                          timeout_ns(*ep), p.status));
+                          (const uint32_t*)(sb + S.flags) + FLAG_DISPATCH * W, W,
+                          Epoch{ep->epoch, p.epoch}, timeout_ns(*ep), p.status,
+                          (uint32_t*)nullptr));
   if (st != MOE_OK) return st;
   const moe_config_t l = local_cfg(c, W);
   const uint8_t* xq = reinterpret_cast<const uint8_t*>(sb + S.xr);
@@ -923,7 +966,8 @@ moe_status_t moe_ep_expert_mlp_fp8(const moe_config_t* cfg, const moe_ep_t* ep,
                       ws_d_local, hq, hs, sb + S.y, R, p.status, s);
   if (st != MOE_OK) return st;
   return cuda_st(launch_pdl(ep_signal_kernel, dim3(1), dim3(MAX_W), 0, s, peers, S.flags,
-                            (int)FLAG_Y, W, ep->rank, ep->epoch, (const uint32_t*)p.status));
+                            (int)FLAG_Y, W, ep->rank, Epoch{ep->epoch, p.epoch},
+                            (const uint32_t*)p.status));
 }
 
 moe_status_t moe_ep_layer_forward_fp8(const moe_config_t* cfg, const moe_ep_t* ep,

@@ -60,6 +60,7 @@ class EpGroup:
                                         group)
         self.peers = torch.tensor(self.addrs, dtype=torch.int64, device=self.device)
         self.ws = B.alloc_workspace(B.moe_ep_workspace_bytes(cfg, self.world), self.device)
+        B.moe_ep_workspace_init(cfg, self.world, self.ws)
         B.moe_ep_symmetric_init(cfg, self.world, self.sym, self.sym_bytes)
         torch.cuda.synchronize()
         dist.barrier(group=group)   # every region zeroed before any rank writes into one
@@ -83,12 +84,17 @@ class EpGroup:
 
 
 class EpOnOneDevice:
-    """W ranks on one device (see the module doc)."""
+    """W ranks on one device (see the module doc). device_epoch: number the
+    steps with the ranks' device-resident step counters (epoch 0) instead of
+    host-side step numbers, so that a step can be captured in a CUDA graph and
+    replayed."""
 
-    def __init__(self, cfg: B.MoeConfig, world: int, device="cuda", timeout_us: int = 0):
+    def __init__(self, cfg: B.MoeConfig, world: int, device="cuda", timeout_us: int = 0,
+                 device_epoch: bool = False):
         self.cfg = cfg
         self.world = int(world)
         self.timeout_us = int(timeout_us)
+        self.device_epoch = bool(device_epoch)
         st = B.moe_ep_check(cfg, B.make_ep(self.world, 0, 1, self.timeout_us))
         if st != B.MOE_OK:
             raise B.MoeError(st, "EpOnOneDevice")
@@ -100,10 +106,13 @@ class EpOnOneDevice:
                                   device=device)
         for s in self.sym:
             B.moe_ep_symmetric_init(cfg, self.world, s)
+        for w in self.ws:
+            B.moe_ep_workspace_init(cfg, self.world, w)
         self.epoch = 0
 
     def ep(self, rank: int) -> B.MoeEp:
-        return B.make_ep(self.world, rank, self.epoch, self.timeout_us)
+        return B.make_ep(self.world, rank, 0 if self.device_epoch else self.epoch,
+                         self.timeout_us)
 
     def forward(self, logits: Sequence, x: Sequence, w_gu_local: Sequence, w_d_local: Sequence,
                 out: Sequence, stream=None):
@@ -138,8 +147,8 @@ class EpOnOneDevice:
             B.moe_ep_combine(c, self.ep(r), self.sym[r], self.peers, out[r], self.ws[r], stream)
 
     def views(self, rank: int) -> dict:
-        aux = B.moe_ep_aux(self.cfg, self.ep(rank) if self.epoch else B.make_ep(self.world, rank, 1),
-                           self.sym[rank], self.ws[rank])
+        aux = B.moe_ep_aux(self.cfg, B.make_ep(self.world, rank, 1), self.sym[rank],
+                           self.ws[rank])
         return B.ep_views(self.cfg, self.world, self.sym[rank], self.ws[rank], aux)
 
     def status(self, rank: int) -> int:

@@ -66,8 +66,13 @@
  * region that another process can map (CUDA IPC; no multicast objects).
  *
  * Steps and reuse. `epoch` is the step number: 1 for the first step, one more
- * for each further step, the same on all ranks. No barrier is needed between
- * steps. A rank starts step e+1 (writing peers' counts and xr) only after its
+ * for each further step, the same on all ranks. epoch = 0 asks for the step
+ * counter kept in the private workspace instead: the step's number is then one
+ * past the counter, and the Y wait of moe_ep_combine (the step's last wait)
+ * advances the counter, so that a step captured in a CUDA graph can be
+ * replayed (every rank must then run its four steps in order, every step).
+ * moe_ep_workspace_init zeroes the counter and the status word. No barrier is
+ * needed between steps. A rank starts step e+1 (writing peers' counts and xr) only after its
  * combine of step e has seen every owner's Y flag of step e, and an owner sets
  * that flag after its GEMM of step e, the last reader of its counts and xr of
  * step e. An owner overwrites its y in step e+1 only after every rank's
@@ -98,7 +103,7 @@ extern "C" {
 typedef struct {
   int32_t world;        /* W ranks */
   int32_t rank;         /* this rank, 0 <= rank < W */
-  uint32_t epoch;       /* step number, >= 1, the same on every rank */
+  uint32_t epoch;       /* step number (>= 1, the same on every rank), or 0: the device-resident step counter */
   uint32_t timeout_us;  /* bound of each wait on a peer's flag; 0 = 2 000 000 */
 } moe_ep_t;
 
@@ -129,6 +134,10 @@ moe_status_t moe_ep_check(const moe_config_t* cfg, const moe_ep_t* ep);
 /* Fill *aux from sym and ws (host only, no device work). */
 moe_status_t moe_ep_aux(const moe_config_t* cfg, const moe_ep_t* ep, void* sym, void* ws,
                         moe_ep_aux_t* aux);
+/* Zero the status word and the step counter of a private workspace
+ * (stream-ordered); once, before the first step. */
+moe_status_t moe_ep_workspace_init(const moe_config_t* cfg, int32_t world, void* ws,
+                                   size_t ws_bytes, void* stream);
 /* Zero the counts table and flags of this rank's region (stream-ordered). */
 moe_status_t moe_ep_symmetric_init(const moe_config_t* cfg, int32_t world, void* sym,
                                    size_t sym_bytes, void* stream);

@@ -53,7 +53,7 @@ def test_one_rank_sizes_equal_the_one_rank_layer():
     (dict(), 0, 0, 1, M.MOE_ERR_INVALID_ARG),
     (dict(), 2, 2, 1, M.MOE_ERR_INVALID_ARG),            # rank >= W
     (dict(), 2, -1, 1, M.MOE_ERR_INVALID_ARG),
-    (dict(), 2, 0, 0, M.MOE_ERR_INVALID_ARG),            # epoch 0
+    (dict(), 2, 0, 0, M.MOE_OK),                         # epoch 0: the device step counter
     (dict(n_shared=1), 2, 0, 1, M.MOE_OK),               # bf16 with a shared expert
     (dict(H=4100), 2, 0, 1, M.MOE_ERR_UNSUPPORTED),      # what the one-rank GEMM rejects
     (dict(), 2, 1, 7, M.MOE_OK),
@@ -153,13 +153,11 @@ def test_entry_points_reject_bad_arguments_before_any_launch():
     cs = cfg_of("mixtral", n_shared=1)
     assert lib.moe_ep_expert_mlp(ctypes.byref(cs), ctypes.byref(ep), None, fake, fake, fake, fake,
                                  fake, big, None) == M.MOE_ERR_INVALID_ARG
-    # epoch 0 and a bad config
-    ep0 = M.make_ep(2, 0, 0)
-    assert lib.moe_ep_route(ctypes.byref(c), ctypes.byref(ep0), fake, fake, fake, fake, big,
-                            None) == M.MOE_ERR_INVALID_ARG
+    # a bad config
     assert lib.moe_ep_layer_forward(None, ctypes.byref(ep), fake, fake, fake, fake, fake, fake,
                                     fake, None, fake, big, None) == M.MOE_ERR_INVALID_ARG
     assert lib.moe_ep_symmetric_init(ctypes.byref(c), 2, fake, 16, None) == M.MOE_ERR_WORKSPACE
+    assert lib.moe_ep_workspace_init(ctypes.byref(c), 2, fake, 256, None) == M.MOE_ERR_WORKSPACE
     assert lib.moe_ipc_open(None, None) == M.MOE_ERR_INVALID_ARG
     assert lib.moe_ep_sym_alloc(0, None) == M.MOE_ERR_INVALID_ARG
 
