@@ -111,7 +111,7 @@ SymLayout sym_layout(const moe_config_t& c, int W) {
 
 EpWs ep_ws_layout(const moe_config_t& c, int W) {
   EpWs L;
-  const int64_t nblk = ceil_div(c.T, ROUTE_TB);
+  const int64_t nblk = route_blocks(c.T);
   const int64_t TK = (int64_t)c.T * c.K;
   const int El = c.E / W;
   size_t p = 256;   // status word

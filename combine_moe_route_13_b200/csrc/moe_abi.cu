@@ -65,7 +65,7 @@ moe_status_t validate_fp8(const moe_config_t* c) {
 
 WsLayout ws_layout(const moe_config_t& c) {
   WsLayout L;
-  const int64_t nblk = ceil_div(c.T, ROUTE_TB);
+  const int64_t nblk = route_blocks(c.T);
   const int64_t TK = (int64_t)c.T * c.K;
   const int64_t R = max_rows(c);
   const size_t as = act_size(c.act_dtype);

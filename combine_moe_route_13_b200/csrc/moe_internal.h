@@ -12,10 +12,15 @@
 
 namespace moe {
 
-// Tokens handled by one block of the route kernel (the unit of the per-block
-// expert histograms). The per-block expert bitmap has ROUTE_TB/32 words per
-// expert.
-constexpr int ROUTE_TB = 128;
+// Tokens handled by one block of the route's top-K kernel (the unit of the
+// per-block expert histograms; the block's expert bitmap has tb/32 words per
+// expert): the smallest of 32, 64, 128 that keeps the blocks within one wave
+// of two 1024-thread blocks per SM (296 on the 148 SMs), else 128, so that a
+// small batch still spreads over the SMs instead of leaving most of them idle
+// (a batch of 1,024 tokens is 32 blocks of 32 tokens, not 8 of 128).
+constexpr int ROUTE_TB_MAX = 128;
+inline int route_tb(int64_t T) { return T <= 32 * 296 ? 32 : (T <= 64 * 296 ? 64 : 128); }
+inline int64_t route_blocks(int64_t T) { return (T + route_tb(T) - 1) / route_tb(T); }
 constexpr int MAX_E = 1024;
 constexpr int MAX_K = 32;
 // Rows per ready counter of the overlapped combine (the GEMM half-tile height).

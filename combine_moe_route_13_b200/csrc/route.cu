@@ -4,7 +4,8 @@
 // "Enabling trillion-parameter models on AWS EFA", "Диспетчеризация и
 // комбинирование": the dispatch counts tokens per expert with shared-memory
 // atomics inside a block and turns the counts into packing offsets with a
-// cumulative sum. Here every block of ROUTE_TB tokens builds a bitmap
+// cumulative sum. Here every block of tb tokens (32, 64 or 128, by batch
+// size) builds a bitmap
 // [expert][token-in-block] in shared memory with atomicOr; popcounts of the
 // bitmap give both the block's histogram and, for each assignment, its rank
 // among the block's earlier tokens of the same expert. A scan over blocks then
@@ -38,8 +39,6 @@
 namespace moe {
 namespace {
 
-constexpr int WORDS = ROUTE_TB / 32;   // bitmap words per expert
-
 // Order-preserving map of a float to uint32 (larger float -> larger key);
 // -0.0 is first folded into +0.0 so that the two compare equal, as floats do.
 // Keys of finite values and of -inf are > 0.
@@ -65,14 +64,15 @@ __device__ __forceinline__ void load_logits(const float* __restrict__ row, int E
 template <int VPL, int THREADS, bool BIAS>
 __global__ void __launch_bounds__(THREADS)
 route_topk_kernel(const float* __restrict__ logits, const float* __restrict__ sel_bias, int T,
-                  int E, int K, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+                  int E, int K, int tb, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                   int32_t* __restrict__ local_rank, int32_t* __restrict__ blk_cnt) {
   extern __shared__ uint32_t smem_u[];
+  const int WORDS = tb / 32;                                   // bitmap words per expert
   uint32_t* bitmap = smem_u;                                   // [E][WORDS]
-  int32_t* idx_s = reinterpret_cast<int32_t*>(smem_u + E * WORDS);  // [ROUTE_TB][K]
+  int32_t* idx_s = reinterpret_cast<int32_t*>(smem_u + E * WORDS);  // [tb][K]
 
-  const int tb0 = blockIdx.x * ROUTE_TB;
-  const int ntok = min(ROUTE_TB, T - tb0);
+  const int tb0 = blockIdx.x * tb;
+  const int ntok = min(tb, T - tb0);
   for (int i = threadIdx.x; i < E * WORDS; i += blockDim.x) bitmap[i] = 0u;
   pdl_wait();
   pdl_trigger();
@@ -260,7 +260,8 @@ __device__ __forceinline__ void expert_offsets_smem(int E, int C, int A,
 }
 
 __global__ void __launch_bounds__(256)
-route_slot_kernel(int T, int K, int E, int S, int C, int A, int nblk, int64_t R_max, int64_t R_sh,
+route_slot_kernel(int T, int K, int E, int S, int C, int A, int nblk, int tb, int64_t R_max,
+                  int64_t R_sh,
                   const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ blk_base,
                   const int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                   int32_t* __restrict__ segoff, int32_t* __restrict__ totals,
@@ -291,7 +292,7 @@ route_slot_kernel(int T, int K, int E, int S, int C, int A, int nblk, int64_t R_
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < TK; i += stride) {
     const int t = (int)(i / K);
     const int e = topk_idx[i];
-    const int pos = blk_base[(size_t)e * nblk + t / ROUTE_TB] + slot[i];
+    const int pos = blk_base[(size_t)e * nblk + t / tb] + slot[i];
     int s = -1;
     if (pos < C) {
       s = off_s[e] + pos;
@@ -322,16 +323,16 @@ route_slot_kernel(int T, int K, int E, int S, int C, int A, int nblk, int64_t R_
 
 template <int VPL>
 cudaError_t launch_topk(int nblk, size_t smem, cudaStream_t s, const float* logits,
-                        const float* sel_bias, int T, int E, int K, int32_t* idx, float* w,
+                        const float* sel_bias, int T, int E, int K, int tb, int32_t* idx, float* w,
                         int32_t* rank, int32_t* blk) {
   // 32 warps (4 tokens each) while the register budget allows: 16 warps for
   // E > 256, 8 for E > 512
   constexpr int THREADS = VPL >= 32 ? 256 : (VPL >= 16 ? 512 : 1024);
   if (sel_bias)
     return launch_pdl(route_topk_kernel<VPL, THREADS, true>, dim3(nblk), dim3(THREADS), smem, s,
-                      logits, sel_bias, T, E, K, idx, w, rank, blk);
+                      logits, sel_bias, T, E, K, tb, idx, w, rank, blk);
   return launch_pdl(route_topk_kernel<VPL, THREADS, false>, dim3(nblk), dim3(THREADS), smem, s,
-                    logits, sel_bias, T, E, K, idx, w, rank, blk);
+                    logits, sel_bias, T, E, K, tb, idx, w, rank, blk);
 }
 
 }  // namespace
@@ -341,18 +342,19 @@ cudaError_t launch_route(const moe_config_t& c, const float* logits, int32_t* to
                          int32_t* segoff, int32_t* slot, int32_t* row_src, int32_t* totals,
                          int32_t* blk_cnt, int64_t R_max, cudaStream_t s,
                          uint32_t* row_ready, const float* sel_bias) {
-  const int nblk = (int)ceil_div(c.T, ROUTE_TB);
+  const int tb = route_tb(c.T);
+  const int nblk = (int)route_blocks(c.T);
   const int64_t n_ready = row_ready ? ceil_div(R_max, READY_ROWS) : 0;
   if (nblk > 0) {
-    const size_t smem = (size_t)c.E * WORDS * 4 + (size_t)ROUTE_TB * c.K * 4;
+    const size_t smem = (size_t)c.E * (tb / 32) * 4 + (size_t)tb * c.K * 4;
     const int vpl = (int)ceil_div(c.E, 32);
     cudaError_t e;
-    if (vpl <= 1) e = launch_topk<1>(nblk, smem, s, logits, sel_bias, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
-    else if (vpl <= 2) e = launch_topk<2>(nblk, smem, s, logits, sel_bias, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
-    else if (vpl <= 4) e = launch_topk<4>(nblk, smem, s, logits, sel_bias, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
-    else if (vpl <= 8) e = launch_topk<8>(nblk, smem, s, logits, sel_bias, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
-    else if (vpl <= 16) e = launch_topk<16>(nblk, smem, s, logits, sel_bias, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
-    else e = launch_topk<32>(nblk, smem, s, logits, sel_bias, c.T, c.E, c.K, topk_idx, topk_w, slot, blk_cnt);
+    if (vpl <= 1) e = launch_topk<1>(nblk, smem, s, logits, sel_bias, c.T, c.E, c.K, tb, topk_idx, topk_w, slot, blk_cnt);
+    else if (vpl <= 2) e = launch_topk<2>(nblk, smem, s, logits, sel_bias, c.T, c.E, c.K, tb, topk_idx, topk_w, slot, blk_cnt);
+    else if (vpl <= 4) e = launch_topk<4>(nblk, smem, s, logits, sel_bias, c.T, c.E, c.K, tb, topk_idx, topk_w, slot, blk_cnt);
+    else if (vpl <= 8) e = launch_topk<8>(nblk, smem, s, logits, sel_bias, c.T, c.E, c.K, tb, topk_idx, topk_w, slot, blk_cnt);
+    else if (vpl <= 16) e = launch_topk<16>(nblk, smem, s, logits, sel_bias, c.T, c.E, c.K, tb, topk_idx, topk_w, slot, blk_cnt);
+    else e = launch_topk<32>(nblk, smem, s, logits, sel_bias, c.T, c.E, c.K, tb, topk_idx, topk_w, slot, blk_cnt);
     if (e != cudaSuccess) return e;
   }
   cudaError_t e = launch_pdl(route_scan_kernel, dim3((unsigned)ceil_div(c.E, 32)), dim3(1024), 0, s,
@@ -361,7 +363,7 @@ cudaError_t launch_route(const moe_config_t& c, const float* logits, int32_t* to
   const int64_t work = std::max<int64_t>((int64_t)c.T * c.K, R_max);
   int grid = (int)std::min<int64_t>(std::max<int64_t>(ceil_div(work, 256), 1), 148 * 8);
   return launch_pdl(route_slot_kernel, dim3(grid), dim3(256), 0, s, c.T, c.K, c.E, c.S, c.capacity,
-                    c.row_align, nblk, R_max, shared_row0(c), (const int32_t*)topk_idx, (const int32_t*)blk_cnt,
+                    c.row_align, nblk, tb, R_max, shared_row0(c), (const int32_t*)topk_idx, (const int32_t*)blk_cnt,
                     (const int32_t*)counts, offsets, segoff, totals, slot, row_src, row_ready,
                     n_ready);
 }

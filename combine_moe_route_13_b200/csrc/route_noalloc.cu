@@ -62,7 +62,7 @@ extern "C" moe_status_t moe_route_topk_noalloc(
   if (cfg->T > 0 && (!logits || !topk_idx || !topk_w || !token_slot)) return MOE_ERR_INVALID_ARG;
   const int64_t R = max_rows(*cfg);
   if (R > 0 && !row_src) return MOE_ERR_INVALID_ARG;
-  const int64_t need = std::max<int64_t>(ceil_div(cfg->T, ROUTE_TB), 1) * cfg->E * 4;
+  const int64_t need = std::max<int64_t>(route_blocks(cfg->T), 1) * cfg->E * 4;
   if (need > (int64_t)NOALLOC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE;
   int32_t* scratch = nullptr;
   if (scratch_on_current_device(&scratch) != cudaSuccess) return MOE_ERR_CUDA;

@@ -195,11 +195,12 @@ moe_status_t moe_router_logits(const moe_config_t* cfg, const void* x, const voi
  * and output buffers, or code paths where an allocation could fail at a bad
  * moment. This entry point takes the same arguments as moe_route_topk without
  * ws/ws_bytes and produces identical results. Its scratch (the per-block expert
- * histograms, ceil(T/128) * E * 4 bytes) lives in a fixed device array of
+ * histograms, ceil(T/b) * E * 4 bytes, b the tokens of a route block: 32 for
+ * T <= 9472, 64 for T <= 18944, else 128) lives in a fixed device array of
  * MOE_NOALLOC_SCRATCH_BYTES (1 MiB) inside the library, which every GPU that
  * loads the library holds until the process exits.
  *   - It calls no cudaMalloc, cudaFree or allocating library routine.
- *   - Configurations needing more scratch than 1 MiB (ceil(T/128) * E > 262144)
+ *   - Configurations needing more scratch than 1 MiB (ceil(T/b) * E > 262144)
  *     return MOE_ERR_WORKSPACE and launch nothing.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) and caches it; make that first call before any
