@@ -41,7 +41,8 @@
  *      from the owner's memory, plus (n_shared = 1) the rank's own shared-expert
  *      row with weight 1; fp32 accumulation, one rounding (as moe_combine).
  *   Every rank's out equals moe_layer_forward of its own tokens over all E
- *   experts (the same rows meet the same weights in the same order).
+ *   experts (and the shared expert, if any): the same rows meet the same
+ *   weights in the same order.
  *
  * Layout. kept[s][e] = min(count of rank s for expert e, C). On owner d, local
  * expert j (e = d*E/W + j) receives recv_counts[j] = sum_s kept[s][e] rows from
@@ -71,20 +72,24 @@
  * past the counter, and the Y wait of moe_ep_combine (the step's last wait)
  * advances the counter, so that a step captured in a CUDA graph can be
  * replayed (every rank must then run its four steps in order, every step).
- * moe_ep_workspace_init zeroes the counter and the status word. No barrier is
- * needed between steps. A rank starts step e+1 (writing peers' counts and xr) only after its
- * combine of step e has seen every owner's Y flag of step e, and an owner sets
- * that flag after its GEMM of step e, the last reader of its counts and xr of
- * step e. An owner overwrites its y in step e+1 only after every rank's
- * DISPATCH flag of step e+1, which each rank sets after its combine of step e,
- * the reader of that y. (The combine reads the owners' y in place.)
+ * moe_ep_workspace_init zeroes the counter and the status word.
+ * No barrier is needed between steps. A rank starts step e+1 (writing peers'
+ * counts and xr) only after its combine of step e has seen every owner's Y
+ * flag of step e, and an owner sets that flag after its GEMM of step e, the
+ * last reader of its counts and xr of step e. An owner overwrites its y in step
+ * e+1 only after every rank's DISPATCH flag of step e+1, which each rank sets
+ * after its combine of step e, the reader of that y. (The combine reads the
+ * owners' y in place.)
  *
  * Errors. Arguments: return codes as in moe.h. Every wait on a peer's flag is
  * bounded by timeout_us (0 = 2 s); one that runs out records MOE_ERR_TIMEOUT in
  * the status word (moe_get_device_status on the private workspace), and the
- * later waits of the step then give up at once; the outputs of such a step are
- * unspecified. A row whose computed destination falls outside the receive
- * buffer is not written and records MOE_ERR_DEVICE_INPUT.
+ * later waits then give up at once; the rank sends nothing more and raises no
+ * flag, so its peers time out too instead of waiting. The outputs of such a
+ * step are unspecified, and the group must be set up again
+ * (moe_ep_workspace_init, moe_ep_symmetric_init and a barrier on every rank)
+ * before its next step. A row whose computed destination falls outside the
+ * receive buffer is not written and records MOE_ERR_DEVICE_INPUT.
  *
  * Limits: everything moe_expert_mlp supports for bf16 (tcgen05) plus
  * E % W == 0, S % W == 0, 1 <= W <= 64; fp32 activations use the CUDA-core
