@@ -41,19 +41,24 @@ def exchange_addresses(own_handle: bytes, own_addr: int, open_handle: Callable[[
 
 class EpGroup:
     """This process's rank of a W-GPU expert-parallel layer (W = the process
-    group's size). torch.cuda's current device must be this rank's GPU."""
+    group's size). `device` is this rank's GPU (default: torch.cuda's current
+    device). device_epoch: number the steps with the device-resident step
+    counter (epoch 0), so that a step can be captured in a CUDA graph."""
 
-    def __init__(self, cfg: B.MoeConfig, group=None, timeout_us: int = 0):
+    def __init__(self, cfg: B.MoeConfig, group=None, timeout_us: int = 0, device=None,
+                 device_epoch: bool = False):
         import torch.distributed as dist
         self.cfg = cfg
         self.group = group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
         self.timeout_us = int(timeout_us)
+        self.device_epoch = bool(device_epoch)
         st = B.moe_ep_check(cfg, B.make_ep(self.world, self.rank, 1, self.timeout_us))
         if st != B.MOE_OK:
             raise B.MoeError(st, "EpGroup")
-        self.device = torch.device("cuda", torch.cuda.current_device())
+        self.device = (torch.device("cuda", torch.cuda.current_device()) if device is None
+                       else torch.device(device))
         self.sym_bytes = B.moe_ep_symmetric_bytes(cfg, self.world)
         self.sym = B.moe_ep_sym_alloc(self.sym_bytes)
         self.addrs = exchange_addresses(B.moe_ipc_get_handle(self.sym), self.sym, B.moe_ipc_open,
@@ -62,19 +67,34 @@ class EpGroup:
         self.ws = B.alloc_workspace(B.moe_ep_workspace_bytes(cfg, self.world), self.device)
         B.moe_ep_workspace_init(cfg, self.world, self.ws)
         B.moe_ep_symmetric_init(cfg, self.world, self.sym, self.sym_bytes)
-        torch.cuda.synchronize()
+        self._sync()
         dist.barrier(group=group)   # every region zeroed before any rank writes into one
         self.epoch = 0
 
+    def _sync(self):
+        if self.device.type == "cuda":
+            torch.cuda.synchronize(self.device)
+
+    def _ep(self) -> B.MoeEp:
+        return B.make_ep(self.world, self.rank, 0 if self.device_epoch else self.epoch,
+                         self.timeout_us)
+
     def forward(self, logits, x, w_gu_local, w_d_local, out, stream=None) -> B.MoeEpAux:
+        """One step of this rank's layer (every rank calls it once per step)."""
         self.epoch += 1
-        ep = B.make_ep(self.world, self.rank, self.epoch, self.timeout_us)
-        return B.moe_ep_layer_forward(self.cfg, ep, logits, x, w_gu_local, w_d_local, self.sym,
-                                      self.peers, out, self.ws, stream)
+        return B.moe_ep_layer_forward(self.cfg, self._ep(), logits, x, w_gu_local, w_d_local,
+                                      self.sym, self.peers, out, self.ws, stream)
+
+    def forward_fp8(self, logits, x, wq, out, stream=None) -> B.MoeEpAux:
+        """One step with the fp8 payload; wq = (codes and scales of this rank's
+        gate/up weights, codes and scales of its down weights)."""
+        self.epoch += 1
+        return B.moe_ep_layer_forward_fp8(self.cfg, self._ep(), logits, x, *wq, self.sym,
+                                          self.peers, out, self.ws, stream)
 
     def close(self):
         import torch.distributed as dist
-        torch.cuda.synchronize()
+        self._sync()
         dist.barrier(group=self.group)   # nobody reads a region after it is unmapped
         for r, a in enumerate(self.addrs):
             if r != self.rank:

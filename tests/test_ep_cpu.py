@@ -202,3 +202,74 @@ def test_handle_exchange_two_ranks():
     # rank r keeps its own address and opens the other rank's handle, in rank order
     assert got[0] == ([7, 1001], [1])
     assert got[1] == ([1000, 8], [0])
+
+
+# ---------------------------------------------------------------- EpGroup host logic (gloo)
+
+def _group_worker(rank, world, port, q, device_epoch):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from combine_moe_route_13_b200 import _binding as B
+        calls = []
+        fake = {
+            "moe_ep_check": lambda cfg, ep: B.MOE_OK,
+            "moe_ep_symmetric_bytes": lambda cfg, w: 4096,
+            "moe_ep_workspace_bytes": lambda cfg, w: 1024,
+            "moe_ep_sym_alloc": lambda n: 1000 + rank,
+            "moe_ipc_get_handle": lambda addr: bytes([addr % 256]) * 64,
+            "moe_ipc_open": lambda h: calls.append(("open", h[0])) or 2000 + h[0],
+            "moe_ipc_close": lambda addr: calls.append(("close", addr)),
+            "moe_ep_sym_free": lambda addr: calls.append(("free", addr)),
+            "moe_ep_workspace_init": lambda cfg, w, ws: calls.append(("ws_init", w)),
+            "moe_ep_symmetric_init": lambda cfg, w, sym, n: calls.append(("sym_init", sym, n)),
+            "moe_ep_layer_forward": lambda cfg, ep, *a: calls.append(
+                ("forward", ep.world, ep.rank, ep.epoch)),
+        }
+        for k, v in fake.items():
+            setattr(B, k, v)
+        cfg = M.make_config(T=64, H=256, E=8, K=2, F=256, S=2, capacity=20)
+        g = EP.EpGroup(cfg, device="cpu", device_epoch=device_epoch)
+        peers = g.peers.tolist()
+        for _ in range(3):
+            g.forward(None, None, None, None, None)
+        g.close()
+        q.put((rank, g.addrs, peers, calls))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("device_epoch", [False, True])
+def test_ep_group_setup_steps_and_close_two_ranks(device_epoch):
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_group_worker, args=(r, 2, port, q, device_epoch))
+             for r in range(2)]
+    for p in procs:
+        p.start()
+    got = {}
+    for _ in range(2):
+        r, addrs, peers, calls = q.get(timeout=120)
+        got[r] = (addrs, peers, calls)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for r in range(2):
+        addrs, peers, calls = got[r]
+        other = 1 - r
+        # own region kept, the other rank's region opened from its handle, in rank order
+        want = [1000 + r if i == r else 2000 + (1000 + other) % 256 for i in range(2)]
+        assert addrs == [] and peers == want      # addrs cleared by close()
+        names = [c[0] for c in calls]
+        assert names == ["open", "ws_init", "sym_init", "forward", "forward", "forward",
+                         "close", "free"]
+        assert calls[2] == ("sym_init", 1000 + r, 4096)
+        epochs = [c[3] for c in calls if c[0] == "forward"]
+        assert epochs == ([0, 0, 0] if device_epoch else [1, 2, 3])
+        assert all(c[1:3] == (2, r) for c in calls if c[0] == "forward")
+        assert calls[-2] == ("close", want[other]) and calls[-1] == ("free", 1000 + r)
