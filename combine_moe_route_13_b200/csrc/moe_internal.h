@@ -18,7 +18,6 @@ namespace moe {
 // of two 1024-thread blocks per SM (296 on the 148 SMs), else 128, so that a
 // small batch still spreads over the SMs instead of leaving most of them idle
 // (a batch of 1,024 tokens is 32 blocks of 32 tokens, not 8 of 128).
-constexpr int ROUTE_TB_MAX = 128;
 inline int route_tb(int64_t T) { return T <= 32 * 296 ? 32 : (T <= 64 * 296 ? 64 : 128); }
 inline int64_t route_blocks(int64_t T) { return (T + route_tb(T) - 1) / route_tb(T); }
 constexpr int MAX_E = 1024;
