@@ -211,3 +211,14 @@ def test_fp8_entry_points_reject_bad_arguments():
                                      M.MOE_FLAG_OVERLAP, fake, 1 << 40, None, None) == M.MOE_ERR_UNSUPPORTED
     assert lib.moe_layer_forward_fp8(ctypes.byref(cfg), fake, fake, fake, fake, fake, fake, fake,
                                      0, fake, 1024, None, None) == M.MOE_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("T,b", [(1, 32), (9472, 32), (9473, 64), (18944, 64), (18945, 128),
+                                 (131072, 128)])
+def test_route_workspace_follows_the_route_block_size(T, b):
+    # the route's scratch is ceil(T/b) * E int32 counters, b the tokens of a
+    # top-K block: 32 up to 9472 tokens, 64 up to 18944, else 128 (moe.h)
+    E = 64
+    cfg = M.make_config(T=T, H=64, E=E, K=2, F=64, S=1, capacity=8)
+    nblk = -(-T // b)
+    assert M.moe_route_workspace_bytes(cfg) == 256 + (-(-(nblk * E * 4) // 256)) * 256
