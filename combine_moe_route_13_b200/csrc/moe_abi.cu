@@ -104,7 +104,7 @@ using namespace moe;
 
 extern "C" {
 
-int32_t moe_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+int32_t moe_version(void) { return 1 * 10000 + 1 * 100 + 0; }   // 1.1: moe_ep.h
 
 const char* moe_status_string(moe_status_t s) {
   switch (s) {

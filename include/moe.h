@@ -371,7 +371,8 @@ moe_status_t moe_get_device_status(void* ws, moe_status_t* status, void* stream)
 /* Static text for a status code. */
 const char* moe_status_string(moe_status_t status);
 
-/* Library version as major*10000 + minor*100 + patch. */
+/* Library version as major*10000 + minor*100 + patch (1.1.0: the
+ * expert-parallel entry points of moe_ep.h added). */
 int32_t moe_version(void);
 
 #ifdef __cplusplus
