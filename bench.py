@@ -1,21 +1,33 @@
 """Benchmark of the single-GPU MoE layer (route -> dispatch -> expert MLP -> combine).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mixtral] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload kimi] [--impl ours|reference]
 
 One step = one moe_layer_forward over one batch of T tokens of the workload
-(default: the Mixtral-shaped layer, T=4096, H=4096, E=8, top-2, F=14336, bf16).
-Inputs are synthetic and seeded. Rank 0 prints one JSON line.
+(default: the Kimi-K2-shaped prefill layer, T=32768, H=7168, E=384, top-8,
+F=2048, bf16, 33.8 GB of expert weights: the largest configuration that fits
+one GPU). Inputs are synthetic and seeded. Rank 0 prints one JSON line.
 
-Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
-on the launching stream; L2 is flushed (a 256 MB write) before every step,
-outside the events. A barrier and a device synchronisation bracket the timed
-region; with several ranks every rank runs its own replica of the layer on its
-own tokens (weak scaling, no data-path collective) and the time is the maximum
-over ranks. `e2e` repeats the measurement through the same C ABI call with the
-step's inputs copied from pinned host memory and the output copied back inside
-the timed region. A second pass calls the four piecewise entry points with
-events between them to attribute time to route, dispatch, expert MLP and
-combine; the expert MLP (the grouped GEMMs, the dominant cost) gives `roofline`.
+Timing (16 warm-up and 32 timed steps by default, the DistributedMoE README's
+protocol, "Результаты экспериментов"): every step is bracketed by CUDA events
+on the launching stream, L2 is flushed (256 MB written, 256 MB read) before
+every step outside the events, and the step time is the median over the timed
+steps (the mean is reported beside it). A barrier and a device
+synchronisation bracket the timed region; with several ranks every rank runs
+its own replica of the layer on its own tokens (weak scaling, no data-path
+collective) and the time is the maximum over ranks.
+
+Inside the same clock-sampled region, right after the fused steps, the same
+number of steps runs through the four piecewise entry points with events
+between them: route, dispatch, expert MLP and combine. Their median times
+give the per-kernel GB/s and `roofline` (the expert MLP: the grouped GEMMs,
+the dominant cost), taken at the clocks the fused steps ran at. The peak is
+the measured burst bf16 rate unless the region was at least a second of
+load with the power cap active, then the measured sustained rate; both
+fractions are printed.
+
+`e2e` repeats the measurement through the same C ABI call with the step's
+inputs copied from pinned host memory and the output copied back inside the
+timed region.
 
 `--impl reference` times the CPU oracle on this host's cores instead, on a
 bounded sample of the same workload per step.
@@ -109,6 +121,14 @@ class Clocks:
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return
+        # nvidia-smi takes a moment to start: wait (at most 3 s) for its first
+        # sample, so that the record covers the whole timed region
+        t0 = time.time()
+        while time.time() - t0 < 3.0 and self.proc.poll() is None:
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.02)
 
     def stop(self):
         if self.proc is None:
@@ -238,7 +258,9 @@ def time_steps(fn, steps, warmup, flush_buf, stream):
 
 
 def phase_times(layer: Layer, steps, flush_buf, stream):
-    """Per-phase device times (ms, mean over steps) through the piecewise entry points."""
+    """Per-phase device times (ms, one list per phase over `steps` steps)
+    through the piecewise entry points, and the per-step totals (first pass
+    untimed, a warm-up)."""
     M = layer.M
     v = layer.views()
     cfg, inp = layer.cfg, layer.inp
@@ -266,8 +288,9 @@ def phase_times(layer: Layer, steps, flush_buf, stream):
         lambda: M.moe_combine(cfg, v["y"], v["token_slot"], v["topk_w"], layer.out),
     )
     acc = {n: [] for n in names}
+    totals = []
     nvtx = torch.cuda.nvtx   # host ranges per phase, for nsys-style timelines
-    for _ in range(steps + 1):
+    for it in range(steps + 1):
         # a longer idle wait than the whole-step timing's: the piecewise calls
         # cost more host time, and every phase must already be queued when the
         # GPU reaches it, or its time would include the host's
@@ -280,9 +303,11 @@ def phase_times(layer: Layer, steps, flush_buf, stream):
             nvtx.range_pop()
             ev[i + 1].record(stream)
         torch.cuda.synchronize()
-        for i, n in enumerate(names):
-            acc[n].append(ev[i].elapsed_time(ev[i + 1]))
-    return {n: float(np.mean(acc[n][1:])) for n in names}   # first pass is a warm-up
+        if it:   # the first pass is a warm-up
+            for i, n in enumerate(names):
+                acc[n].append(ev[i].elapsed_time(ev[i + 1]))
+            totals.append(ev[0].elapsed_time(ev[-1]))
+    return acc, totals
 
 
 def e2e_steps(layer: Layer, steps, warmup, flush_buf, stream):
@@ -404,45 +429,91 @@ def algorithmic(layer: Layer, totals, counts):
     }
 
 
-def cpu_oracle_sample(wl: W.Workload, tokens: int, seed: int, inp_host=None):
+def _np_act(t: torch.Tensor) -> np.ndarray:
+    """A tensor on any device as the oracle's host array (bf16 as uint16 bits)."""
+    t = t.detach().cpu().contiguous()
+    return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+
+
+class ExpertWeights:
+    """An [E, rows, cols] weight tensor (on the GPU or the host) that hands the
+    oracle one expert's matrix at a time, copied to host memory when the
+    oracle indexes it: the oracle touches only the experts its sample routes
+    to, so a 34 GB weight set need not sit in host memory. The seconds spent
+    copying are kept in `copy_s` (the caller subtracts them: they are not the
+    oracle's work)."""
+
+    def __init__(self, t: torch.Tensor, clock=None):
+        self.t = t
+        self.shape = tuple(t.shape)
+        self.clock = clock if clock is not None else [0.0]
+
+    @property
+    def copy_s(self) -> float:
+        return self.clock[0]
+
+    def __len__(self):
+        return self.shape[0]
+
+    def __getitem__(self, i):
+        if isinstance(i, slice):
+            return ExpertWeights(self.t[i], self.clock)
+        t0 = time.perf_counter()
+        a = _np_act(self.t[i])
+        self.clock[0] += time.perf_counter() - t0
+        return a
+
+
+# tokens of the CPU-oracle sample per call, by workload: about 5-20 s per call
+# on 8-16 host cores (the oracle widens every routed expert's weights to
+# float64: about 0.2 s per expert of the 7168 x 2048 shapes)
+CPU_TOKENS = {"tiny": 64, "mixtral": 512, "dsv3": 16, "skewed": 512, "kimi": 16,
+              "kimi_seg": 64}
+
+
+def cpu_tokens_for(wl: W.Workload, requested) -> int:
+    if requested:
+        return min(int(requested), wl.T)
+    base = wl.name.replace("_shared", "").replace("_fp8", "")
+    return min(CPU_TOKENS.get(base, 64), wl.T)
+
+
+def cpu_oracle_sample(wl: W.Workload, tokens: int, inp):
     """The oracle's whole layer on the first `tokens` tokens of the workload
-    (capacity scaled to that batch). Returns (seconds, tokens)."""
+    (capacity scaled to that batch). `inp` holds the workload's tensors on any
+    device; the weights reach the oracle one expert at a time. Returns
+    (seconds of oracle work, tokens)."""
     from oracle import moe_oracle as O
-    import torch as _t
     tokens = min(tokens, wl.T)
-    if inp_host is None:
-        inp_host = W.make_inputs(wl, seed=seed, device="cpu")
-
-    def np_act(t):
-        t = t.contiguous()
-        return t.view(_t.int16).numpy().view(np.uint16) if t.dtype == _t.bfloat16 else t.numpy()
-
-    lg = inp_host["logits"][:tokens].numpy()
-    x = np_act(inp_host["x"][:tokens])
-    w_gu, w_d = np_act(inp_host["w_gu"]), np_act(inp_host["w_d"])
+    lg = inp["logits"][:tokens].cpu().numpy()
+    x = _np_act(inp["x"][:tokens])
+    w_gu, w_d = ExpertWeights(inp["w_gu"]), ExpertWeights(inp["w_d"])
     C = O.capacity(tokens, wl.K, wl.E, wl.cf)
     t0 = time.perf_counter()
     O.layer_forward(lg, x, w_gu, w_d, wl.K, C, wl.row_align, wl.S, wl.act, n_shared=wl.n_shared)
-    return time.perf_counter() - t0, tokens
+    secs = time.perf_counter() - t0 - w_gu.copy_s - w_d.copy_s
+    return secs, tokens
 
 
 def cpu_oracle_sample_fp8(wl: W.Workload, tokens: int, layer: "Layer"):
     """The fp8 oracle's whole layer on the first `tokens` tokens, with the
     expert weights as the library quantised them (its quantiser is bit-exact
-    with the oracle's). Returns (seconds, tokens)."""
+    with the oracle's); the codes reach the oracle one expert at a time.
+    Returns (seconds of oracle work, tokens)."""
     from oracle import moe_oracle as O
     from oracle import moe_oracle_fp8 as Q
     tokens = min(tokens, wl.T)
     E, F, H = wl.E + wl.n_shared, wl.F, wl.H
-    gq, gs, dq, ds = (t.cpu().numpy() for t in layer.wq)
-    ge = Q.scales_from_blocked(gs, E * 2 * F, H // 128).reshape(E, 2 * F, H // 128)
-    de = Q.scales_from_blocked(ds, E * H, F // 128).reshape(E, H, F // 128)
+    gq, gs, dq, ds = layer.wq
+    ge = Q.scales_from_blocked(gs.cpu().numpy(), E * 2 * F, H // 128).reshape(E, 2 * F, H // 128)
+    de = Q.scales_from_blocked(ds.cpu().numpy(), E * H, F // 128).reshape(E, H, F // 128)
+    gq, dq = ExpertWeights(gq), ExpertWeights(dq)
     lg = layer.inp["logits"][:tokens].cpu().numpy()
-    x = layer.inp["x"][:tokens].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    x = _np_act(layer.inp["x"][:tokens])
     C = O.capacity(tokens, wl.K, wl.E, wl.cf)
     t0 = time.perf_counter()
     Q.layer_forward_fp8(lg, x, gq, ge, dq, de, wl.K, C, wl.row_align, wl.S, n_shared=wl.n_shared)
-    return time.perf_counter() - t0, tokens
+    return time.perf_counter() - t0 - gq.copy_s - dq.copy_s, tokens
 
 
 def cpu_cores():
@@ -460,28 +531,33 @@ REFERENCE_BUDGET_S = 120.0   # timed CPU work of the reference arm, at most
 
 def run_reference(args, wl: W.Workload, world, rank):
     """The CPU oracle, timed. One oracle call on the first `cpu_tokens` tokens is
-    one step. Most of a call's cost is fixed (every expert's weights are widened
-    to float64), so no sample size keeps hundreds of steps within minutes: the
-    arm runs the requested warm-ups within 20 s (at least one), then times
-    steps until it has done the requested number or spent REFERENCE_BUDGET_S,
-    and reports the numbers it ran."""
+    one step. Most of a call's cost is fixed (every routed expert's weights are
+    widened to float64), so no sample size keeps hundreds of steps within
+    minutes: the arm runs the requested warm-ups within 20 s (at least one),
+    then times steps until it has done the requested number or spent
+    REFERENCE_BUDGET_S, and reports the numbers it ran. The inputs are drawn
+    with the GPU arm's recipe and seed, on the GPU when there is one (the same
+    values the GPU arm computes on; only their generation uses it), else on
+    the host."""
     if rank != 0:
         return 0
-    tokens = min(args.cpu_tokens, wl.T)
-    inp_host = W.make_inputs(wl, seed=0, device="cpu")
+    tokens = cpu_tokens_for(wl, args.cpu_tokens)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = W.make_inputs(wl, seed=0, device=dev)
     warm, t_warm = 0, 0.0   # the requested warm-ups, within 20 s (at least one)
     while warm < args.warmup and (warm == 0 or t_warm < 20.0):
-        t_warm += cpu_oracle_sample(wl, tokens, 0, inp_host)[0]
+        t_warm += cpu_oracle_sample(wl, tokens, inp)[0]
         warm += 1
     secs = []
     while len(secs) < args.steps and (not secs or sum(secs) < REFERENCE_BUDGET_S):
-        secs.append(cpu_oracle_sample(wl, tokens, 0, inp_host)[0])
-    ms = float(np.mean(secs)) * 1e3
+        secs.append(cpu_oracle_sample(wl, tokens, inp)[0])
+    ms = float(np.median(secs)) * 1e3
     value = tokens / (ms / 1e3)
     cores = cpu_cores()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": world, "steps": len(secs), "warmup": warm, "ms_per_step": ms,
+        "ms_per_step_mean": float(np.mean(secs)) * 1e3,
         "requested_steps": args.steps, "requested_warmup": args.warmup,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.act,
         "data": "synthetic", "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E,
@@ -489,8 +565,9 @@ def run_reference(args, wl: W.Workload, world, rank):
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": f"whole layer (float64 numpy oracle) on the first {tokens} "
                                    f"tokens of the workload per step, capacity scaled to that "
-                                   f"batch; {len(secs)} timed steps (at most the requested "
-                                   f"number, stopped after {REFERENCE_BUDGET_S:.0f} s of timed work)"},
+                                   f"batch; median of {len(secs)} timed steps (at most the "
+                                   f"requested number, stopped after {REFERENCE_BUDGET_S:.0f} s "
+                                   f"of timed work)"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -540,7 +617,9 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
     logits = [i["logits"] for i in inps]
     xs = [i["x"] for i in inps]
     outs = [torch.empty(wl.T, wl.H, dtype=wl.torch_act, device=device) for _ in range(Wn)]
-    emu = EpOnOneDevice(cfg, Wn, device)
+    ep_flags = (M.MOE_EP_TILE_SIGNAL if args.ep_tiles else 0) | \
+        (M.MOE_EP_REMOTE_FIRST if args.ep_remote_first else 0)
+    emu = EpOnOneDevice(cfg, Wn, device, flags=ep_flags)
     flush_buf = flush_buffer(device)
     stream = torch.cuda.current_stream()
 
@@ -560,7 +639,7 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
     clocks.start()
     times = time_steps(step, args.steps, args.warmup, flush_buf, stream)
     clk = clocks.stop()
-    ms = float(np.mean(times))
+    ms = float(np.median(times))
 
     # phases, all ranks each: events between the four steps
     c = cfg
@@ -593,7 +672,7 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
         if it:
             for i, n in enumerate(ph):
                 ph[n].append(ev[i].elapsed_time(ev[i + 1]))
-    ph = {n: float(np.mean(v)) for n, v in ph.items()}
+    ph = {n: float(np.median(v)) for n, v in ph.items()}
     for r in range(Wn):
         if emu.status(r) != M.MOE_OK:
             raise SystemExit(f"rank {r} after timing: {M.status_string(emu.status(r))}")
@@ -619,17 +698,14 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
     mlp_bytes = (3.0 * active * H * F * ws_ * (1 + (4 / 128 if fp8 else 0))
                  + (Nt + Wn * T * wl.n_shared) * (H * ws_ + 2 * F * ws_ + H * s_))
     hbm = peaks["hbm_gbs"]
-    tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    peak_kind = f"bf16_tflops_sustained ({peaks['source']})"
-    if fp8:   # fp8 dense rate = 2 x bf16 (nominal 4.5 / 2.25 PFLOP/s)
-        tensor_peak *= 2.0
-        peak_kind += " x 2 (nominal fp8/bf16 ratio)"
+    tensor_peak, peak_kind, _, _ = choose_peak(peaks, clk, float(np.sum(times)) / 1e3, fp8)
     mlp_tflops = flops / (ph["expert_mlp"] * 1e-3) / 1e12
     mlp_gbs = mlp_bytes / (ph["expert_mlp"] * 1e-3) / 1e9
     hbm_bound = mlp_bytes / (hbm * 1e9) > flops / (tensor_peak * 1e12)
     line = {
         "metric": METRIC, "value": Wn * T / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "ms_per_step_mean": float(np.mean(times)),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": ("fp8" if fp8 else "bf16") if wl.act == "bf16" else "f32", "data": "synthetic",
         "config": {"workload": f"{wl.name}_ep{Wn}_one_device", "T_per_rank": T, "H": H,
@@ -637,6 +713,7 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
                    "row_align": wl.row_align, "ranks": Wn, "effective_tokens": Nt,
                    "n_shared": wl.n_shared,
                    "parallelism": f"ep{Wn} emulated on one GPU (exchanges through local HBM)",
+                   "tile_signal": bool(args.ep_tiles), "remote_first": bool(args.ep_remote_first),
                    "l2": "flushed before every step: 256 MB written, then another 256 MB read"},
         "e2e": None,
         # per rank and step: route 3, publish, plan, dispatch, signal, wait, 2 GEMMs,
@@ -673,15 +750,31 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
     return 0
 
 
+def choose_peak(peaks, clk, region_s, fp8: bool):
+    """The tensor peak the expert MLP is measured against: the measured burst
+    bf16 rate, or the measured sustained rate when the timed region held at
+    least a second of load and the clock record shows the power cap. fp8: 2x
+    (the nominal dense fp8/bf16 ratio, 4.5 / 2.25 PFLOP/s)."""
+    capped = bool(clk) and "sw_power_cap" in clk.get("reasons", [])
+    sustained = capped and region_s >= 1.0 and "bf16_tflops_sustained" in peaks
+    mult = 2.0 if fp8 else 1.0
+    burst = peaks["bf16_tflops"] * mult
+    sus = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * mult
+    kind = ("bf16_tflops_sustained" if sustained else "bf16_tflops (burst)") + \
+        f" ({peaks['source']})" + (" x 2 (nominal fp8/bf16 ratio)" if fp8 else "")
+    return (sus if sustained else burst), kind, burst, sus
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=32)
+    ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="mixtral", choices=sorted(W.WORKLOADS))
-    ap.add_argument("--cpu-tokens", type=int, default=512,
-                    help="tokens of the CPU-oracle sample per step")
+    ap.add_argument("--workload", default="kimi", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--cpu-tokens", type=int, default=None,
+                    help="tokens of the CPU-oracle sample per call (default: by workload, "
+                         "about 5-20 s of oracle work per call)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--router", action="store_true",
                     help="start from hidden states: router projection x W_g^T and a "
@@ -694,7 +787,14 @@ def main(argv=None):
                     help="add one shared expert of the routed width (as DeepSeek-V3 and Kimi-K2 have)")
     ap.add_argument("--ep-emulate", type=int, default=0, metavar="W",
                     help="expert-parallel layer with W ranks emulated on this one GPU")
+    ap.add_argument("--ep-tiles", action="store_true",
+                    help="with --ep-emulate: tile-signalled owner GEMMs and combine "
+                         "(MOE_EP_TILE_SIGNAL)")
+    ap.add_argument("--ep-remote-first", action="store_true",
+                    help="with --ep-tiles: remote-first tile order (MOE_EP_REMOTE_FIRST)")
     args = ap.parse_args(argv)
+    if args.ep_remote_first:
+        args.ep_tiles = True
     if args.warmup < 3 and args.impl == "ours":
         raise SystemExit("--warmup must be >= 3")
     wl = W.WORKLOADS[args.workload]
@@ -736,46 +836,52 @@ def main(argv=None):
             dist.barrier()
         torch.cuda.synchronize()
 
+    # One clock-sampled region: the fused steps (the headline), then as many
+    # steps through the piecewise entry points (the per-kernel split).
     clocks = Clocks(device.index if device.index is not None else 0)
     barrier()
     clocks.start()
     times = time_steps(layer.forward, args.steps, args.warmup, flush_buf, stream)
+    ph_lists, ph_totals = phase_times(layer, args.steps, flush_buf, stream)
     barrier()
     clk = clocks.stop()
-    total_ms = max_over_ranks(float(np.sum(times)), world, device)
-    ms = total_ms / args.steps
+    ms = max_over_ranks(float(np.median(times)), world, device)
+    ms_mean = max_over_ranks(float(np.mean(times)), world, device)
     value = world * wl.T / (ms / 1e3)
+    ph = {n: max_over_ranks(float(np.median(v)), world, device) if v else 0.0
+          for n, v in ph_lists.items()}
+    ph_step = max_over_ranks(float(np.median(ph_totals)), world, device)
+    region_s = (float(np.sum(times)) + float(np.sum(ph_totals))) / 1e3
 
     e2e_t, h2d, d2h = e2e_steps(layer, args.steps, args.warmup, flush_buf, stream)
-    e2e_serial_ms = max_over_ranks(float(np.sum(e2e_t)), world, device) / args.steps
+    e2e_serial_ms = max_over_ranks(float(np.median(e2e_t)), world, device)
     e2e_ms = max_over_ranks(e2e_pipelined(layer, args.steps, args.warmup, flush_buf, stream),
                             world, device) / args.steps
 
-    ph = phase_times(layer, max(args.steps // 2, 3), flush_buf, stream)
     st = layer.M.moe_get_device_status(layer.ws)
     if st != layer.M.MOE_OK:
         raise SystemExit(f"device status after timing: {layer.M.status_string(st)}")
 
     hbm = peaks["hbm_gbs"]
-    tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    peak_kind = f"bf16_tflops_sustained ({peaks['source']})"
-    if args.fp8:   # fp8 dense rate = 2 x bf16 (nominal 4.5 / 2.25 PFLOP/s)
-        tensor_peak *= 2.0
-        peak_kind += " x 2 (nominal fp8/bf16 ratio)"
-    mlp_tflops = alg["mlp_flops"] / (ph["expert_mlp"] * 1e-3) / 1e12
-    mlp_gbs = alg["mlp_bytes"] / (ph["expert_mlp"] * 1e-3) / 1e9
+    tensor_peak, peak_kind, peak_burst, peak_sus = choose_peak(peaks, clk, region_s, args.fp8)
+    mlp_ms = ph["expert_mlp"]
+    mlp_tflops = alg["mlp_flops"] / (mlp_ms * 1e-3) / 1e12
+    mlp_gbs = alg["mlp_bytes"] / (mlp_ms * 1e-3) / 1e9
     # the binding roofline of the expert MLP: tensor time or HBM time, whichever is longer
     hbm_bound = alg["mlp_bytes"] / (hbm * 1e9) > alg["mlp_flops"] / (tensor_peak * 1e12)
     kernels = {
         "router_us": ph["router"] * 1e3 if args.router else None,
-        "phase_timing": "CUDA events between the piecewise entry points on the launching "
-                        "stream, L2 flushed first; each phase includes its launch gap "
-                        "(kernel-only ncu times: profiles/)",
+        "phase_timing": "median over the timed steps of CUDA events between the piecewise "
+                        "entry points on the launching stream, run right after the fused "
+                        "steps inside the same clock-sampled region, L2 flushed before every "
+                        "step; each phase includes its launch gap (kernel-only ncu times: "
+                        "profiles/)",
+        "piecewise_step_ms": ph_step,
         "route_us": ph["route"] * 1e3,
         "route_gbs": alg["route_bytes"] / (ph["route"] * 1e-3) / 1e9,
         "dispatch_us": ph["dispatch"] * 1e3,
         "dispatch_gbs": alg["dispatch_bytes"] / (ph["dispatch"] * 1e-3) / 1e9,
-        "expert_mlp_us": ph["expert_mlp"] * 1e3,
+        "expert_mlp_us": mlp_ms * 1e3,
         "expert_mlp_tflops": mlp_tflops,
         "expert_mlp_gbs": mlp_gbs,
         "combine_us": ph["combine"] * 1e3,
@@ -783,10 +889,16 @@ def main(argv=None):
     }
     kernels["dispatch_hbm_frac"] = kernels["dispatch_gbs"] / hbm
     kernels["combine_hbm_frac"] = kernels["combine_gbs"] / hbm
-    kernels["expert_mlp_tensor_frac_burst"] = mlp_tflops / (peaks["bf16_tflops"] * (2.0 if args.fp8 else 1.0))
-    kernels["expert_mlp_executed_tflops"] = alg["mlp_executed_flops"] / (ph["expert_mlp"] * 1e-3) / 1e12
+    kernels["expert_mlp_tensor_frac_burst"] = mlp_tflops / peak_burst
+    kernels["expert_mlp_tensor_frac_sustained"] = mlp_tflops / peak_sus
+    kernels["expert_mlp_share_of_piecewise_step"] = mlp_ms / ph_step
+    kernels["expert_mlp_within_fused_step"] = bool(mlp_ms <= ms)
+    kernels["expert_mlp_executed_tflops"] = alg["mlp_executed_flops"] / (mlp_ms * 1e-3) / 1e12
     kernels["expert_mlp_tile_rows"] = alg["tile_rows"]
     kernels["expert_mlp_executed_rows"] = alg["executed_rows"]
+    if clk and clk.get("sm_mhz"):
+        # rate per SM clock: compare with the peaks' own clocks at equal frequency
+        kernels["expert_mlp_tflops_per_ghz"] = mlp_tflops / (clk["sm_mhz"] / 1e3)
 
     if rank != 0:
         if world > 1:
@@ -795,26 +907,47 @@ def main(argv=None):
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        # two samples (about 10-30 s of oracle work on the Mixtral shape), on
-        # this replica's own inputs copied to the host once
-        host = None if args.fp8 else {k: layer.inp[k].cpu() for k in ("logits", "x", "w_gu", "w_d")}
-        runs = [cpu_oracle_sample_fp8(wl, args.cpu_tokens, layer) if args.fp8
-                else cpu_oracle_sample(wl, args.cpu_tokens, 0, host) for _ in range(2)]
+        # about 10-30 s of oracle work on this replica's own inputs: two calls
+        # when one takes under 10 s
+        tokens = cpu_tokens_for(wl, args.cpu_tokens)
+        runs = []
+        while len(runs) < 2 and sum(r[0] for r in runs) < 10.0:
+            runs.append(cpu_oracle_sample_fp8(wl, tokens, layer) if args.fp8
+                        else cpu_oracle_sample(wl, tokens, layer.inp))
         secs, tok = sum(r[0] for r in runs), sum(r[1] for r in runs)
         cpu = {"value": tok / secs, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
-               "sample": f"whole layer ({'fp8 ' if args.fp8 else ''}float64 numpy oracle), two "
-                         f"calls, each on the first {args.cpu_tokens} tokens of the workload "
-                         f"with capacity scaled to that batch; {secs:.1f} s in total"}
+               "sample": f"whole layer ({'fp8 ' if args.fp8 else ''}float64 numpy oracle), "
+                         f"{len(runs)} call(s), each on the first {tokens} tokens of the "
+                         f"workload with capacity scaled to that batch; {secs:.1f} s of oracle "
+                         f"work in total"}
+    roof = ({"bound": "hbm", "kernel": "expert_mlp (gate/up + down grouped GEMMs)",
+             "achieved": mlp_gbs, "peak": hbm, "unit": "GB/s", "frac": mlp_gbs / hbm,
+             "peak_kind": f"hbm_gbs ({peaks['source']})",
+             "tensor_frac": mlp_tflops / tensor_peak}
+            if hbm_bound else
+            {"bound": "tensor", "kernel": "expert_mlp (gate/up + down grouped GEMMs)",
+             "achieved": mlp_tflops, "peak": tensor_peak, "unit": "TFLOP/s",
+             "frac": mlp_tflops / tensor_peak, "peak_kind": peak_kind,
+             "frac_burst": mlp_tflops / peak_burst, "frac_sustained": mlp_tflops / peak_sus,
+             "hbm_frac": mlp_gbs / hbm})
+    roof.update({"time_us": mlp_ms * 1e3, "flops": alg["mlp_flops"],
+                 "algorithmic_bytes": alg["mlp_bytes"],
+                 "sm_mhz": clk.get("sm_mhz") if clk else None,
+                 "timed_region_s": region_s,
+                 "traffic": measured_traffic(wl.name),
+                 "traffic_unit": "bytes per moe_expert_mlp call (ncu dram read+write)"})
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "ms_per_step_mean": ms_mean,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": ("fp8" if args.fp8 else "bf16") if wl.act == "bf16" else "f32",
         "data": "synthetic",
         "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "K": wl.K, "F": wl.F,
                    "S": wl.S, "cf": wl.cf, "capacity": layer.C, "row_align": wl.row_align,
                    "effective_tokens": alg["N"], "overflow": int(totals[2]),
-                   "l2": "flushed before every step: 256 MB written, then another 256 MB read", "parallelism": f"replicas{world}",
+                   "l2": "flushed before every step: 256 MB written, then another 256 MB read",
+                   "parallelism": f"replicas{world}",
                    "overlap": bool(args.overlap), "router_projection": bool(args.router),
                    "n_shared": wl.n_shared,
                    "payload": "e4m3, 1x128 blocks, UE8M0 scales; bf16 combine" if args.fp8 else wl.act},
@@ -825,19 +958,11 @@ def main(argv=None):
                         "layer; L2 flushed before every layer",
                 "serial": {"value": world * wl.T / (e2e_serial_ms / 1e3),
                            "ms_per_step": e2e_serial_ms,
-                           "mode": "copy in, layer, copy out, one after the other"}},
+                           "mode": "copy in, layer, copy out, one after the other (median)"}},
+        # the fused steps' launches (the piecewise steps, in the same clock
+        # window, launch as many again)
         "gpu_launches": (KERNELS_PER_STEP + (1 if args.router else 0)) * args.steps,
-        "roofline": ({"bound": "hbm", "kernel": "expert_mlp (gate/up + down grouped GEMMs)",
-                      "achieved": mlp_gbs, "peak": hbm, "unit": "GB/s", "frac": mlp_gbs / hbm,
-                      "peak_kind": f"hbm_gbs ({peaks['source']})",
-                      "tensor_frac": mlp_tflops / tensor_peak}
-                     if hbm_bound else
-                     {"bound": "tensor", "kernel": "expert_mlp (gate/up + down grouped GEMMs)",
-                      "achieved": mlp_tflops, "peak": tensor_peak, "unit": "TFLOP/s",
-                      "frac": mlp_tflops / tensor_peak, "peak_kind": peak_kind,
-                      "hbm_frac": mlp_gbs / hbm}) | {
-                     "traffic": measured_traffic(wl.name),
-                     "traffic_unit": "bytes per moe_expert_mlp call (ncu dram read+write)"},
+        "roofline": roof,
         "kernels": kernels,
         "effective_tokens_per_s": world * alg["N"] / (ms / 1e3),
         "clocks": clk,

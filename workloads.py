@@ -15,6 +15,8 @@ Workloads (shapes from the pages' settings, synthetic values):
   Zipf-skewed router (the "cross-rank skewed" routing mode of the
   "MoE Expert Parallel Benchmark" page, Step 1)
 * ``kimi``    bf16 prefill, T=32768, H=7168, E=384, K=8, F=2048, S=16, cf=1.25
+* ``kimi_seg`` one owner segment of ``kimi``: T=2048, E=24, S=1, the same
+  rows per expert and capacity (a profiling case of a few GB)
 
 Value recipe (all from one ``torch.Generator`` seeded with ``seed``, drawn in
 this order): router logits N(0,1) [T,E] fp32; per-expert logit bias (dsv3:
@@ -65,6 +67,10 @@ WORKLOADS = {
     "dsv3": Workload("dsv3", 1024, 7168, 256, 8, 2048, 8, 1.5, "bf16", bias="normal0.1"),
     "skewed": Workload("skewed", 16384, 2048, 64, 6, 1408, 8, 1.0, "bf16", bias="zipf1.2"),
     "kimi": Workload("kimi", 32768, 7168, 384, 8, 2048, 16, 1.25, "bf16"),
+    # one owner segment of the Kimi-K2 shape (24 experts) with the same rows
+    # per expert (T*K/E = 683) and capacity (854): the case the profiler
+    # captures, 2.1 GB of weights instead of 33.8 GB
+    "kimi_seg": Workload("kimi_seg", 2048, 7168, 24, 8, 2048, 1, 1.25, "bf16"),
 }
 
 
