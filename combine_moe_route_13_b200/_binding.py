@@ -14,7 +14,9 @@ import os
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libmoe.so")
+# MOE_LIBRARY selects another build of the same library: a file name inside
+# this package (libmoe_check.so, the bounds-checked build) or an absolute path.
+LIB_PATH = os.path.join(HERE, os.environ.get("MOE_LIBRARY", "") or "libmoe.so")
 
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = 1
@@ -35,7 +37,7 @@ EXPORTS = ("moe_capacity", "moe_max_rows", "moe_check_config", "moe_route_worksp
            "moe_status_string", "moe_version", "moe_route_topk_noalloc", "moe_combine_wait",
            "moe_route_topk_biased", "moe_router_logits", "moe_layer_forward_x",
            "moe_fp8_scale_bytes", "moe_quantize_fp8", "moe_dispatch_fp8", "moe_expert_mlp_fp8",
-           "moe_layer_forward_fp8") + (
+           "moe_layer_forward_fp8", "moe_debug_bounds_failures") + (
     # include/moe_ep.h
            "moe_ep_recv_rows", "moe_ep_symmetric_bytes", "moe_ep_workspace_bytes", "moe_ep_check",
            "moe_ep_aux", "moe_ep_symmetric_init", "moe_ep_route", "moe_ep_dispatch",
@@ -70,7 +72,11 @@ class MoeLayerAux(ctypes.Structure):
 
 class MoeEp(ctypes.Structure):
     _fields_ = [("world", ctypes.c_int32), ("rank", ctypes.c_int32), ("epoch", ctypes.c_uint32),
-                ("timeout_us", ctypes.c_uint32)]
+                ("timeout_us", ctypes.c_uint32), ("flags", ctypes.c_uint32)]
+
+
+MOE_EP_TILE_SIGNAL = 1
+MOE_EP_REMOTE_FIRST = 2
 
 
 class MoeEpAux(ctypes.Structure):
@@ -78,7 +84,7 @@ class MoeEpAux(ctypes.Structure):
         "topk_idx", "expert_counts", "overflow", "expert_offsets", "segment_offsets",
         "token_slot", "row_src", "totals", "topk_w", "counts_all", "flags", "send_dst_row",
         "recv_offsets", "recv_counts", "xr", "h", "y", "h_shared", "y_shared",
-        "xq", "xs", "hq", "hs")]
+        "xq", "xs", "hq", "hs", "recv_split", "y_ready")]
 
 
 _P = ctypes.c_void_p
@@ -89,7 +95,7 @@ _SZ = ctypes.c_size_t
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libmoe.so is not built ({LIB_PATH}); run "
+        raise ImportError(f"{os.path.basename(LIB_PATH)} is not built ({LIB_PATH}); run "
                           "`python combine_moe_route_13_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     sig = {
@@ -108,6 +114,9 @@ def _load():
         "moe_get_device_status": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int), _P]),
         "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "moe_version": (ctypes.c_int32, []),
+        "moe_debug_bounds_failures": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32),
+                                                     ctypes.POINTER(ctypes.c_uint32),
+                                                     ctypes.c_int32]),
         "moe_route_topk_noalloc": (ctypes.c_int, [_CFG] + [_P] * 10 + [_P]),
         "moe_combine_wait": (ctypes.c_int, [_CFG, _P, _P, _P, _P, ctypes.c_uint32, _P,
                                             ctypes.c_uint32, _P, ctypes.c_size_t, _P]),
@@ -353,6 +362,15 @@ def moe_version() -> int:
     return int(LIB.moe_version())
 
 
+def moe_debug_bounds_failures(reset: bool = False):
+    """(failures, first failing source line) of the bounds-checked build;
+    raises MoeError(MOE_ERR_UNSUPPORTED) on the release build."""
+    n, line = ctypes.c_uint32(0), ctypes.c_uint32(0)
+    _check(LIB.moe_debug_bounds_failures(ctypes.byref(n), ctypes.byref(line), int(bool(reset))),
+           "moe_debug_bounds_failures")
+    return int(n.value), int(line.value)
+
+
 # ---------------------------------------------------------------- fp8 block-scaled path
 
 U8 = torch.uint8
@@ -480,8 +498,8 @@ def layer_views(cfg: MoeConfig, ws: torch.Tensor, aux: MoeLayerAux) -> dict:
 
 # ---------------------------------------------------------------- expert parallelism (moe_ep.h)
 
-def make_ep(world: int, rank: int, epoch: int, timeout_us: int = 0) -> MoeEp:
-    return MoeEp(int(world), int(rank), int(epoch), int(timeout_us))
+def make_ep(world: int, rank: int, epoch: int, timeout_us: int = 0, flags: int = 0) -> MoeEp:
+    return MoeEp(int(world), int(rank), int(epoch), int(timeout_us), int(flags))
 
 
 def _addr(buf, name) -> int:
@@ -603,13 +621,24 @@ def moe_ep_layer_forward_fp8(cfg, ep, logits, x, wq_gu_local, ws_gu_local, wq_d_
     return aux
 
 
-def ep_local_fp8_weights(wq, sf, world: int, E: int, rows_per_expert: int, cols: int) -> list:
+def ep_local_fp8_weights(wq, sf, world: int, E: int, rows_per_expert: int, cols: int,
+                         n_shared: int = 0) -> list:
     """Each rank's slice of weights quantised by quantize_fp8 over all E experts
-    ([E, rows_per_expert, cols] codes and their blocked scales): (codes, scales)
-    per rank. rows_per_expert must be a multiple of 128 (the scale row blocks)."""
+    ([E + n_shared, rows_per_expert, cols] codes and their blocked scales):
+    (codes, scales) per rank, with the shared expert (the last one, held by
+    every rank) appended when n_shared = 1. rows_per_expert must be a multiple
+    of 128 (the scale row blocks), so that each expert's scales are one
+    contiguous byte range."""
     El = E // world
     per = rows_per_expert // 128 * ((cols // 128 + 3) // 4) * 512   # scale bytes per expert
-    return [(wq[r * El:(r + 1) * El], sf[r * El * per:(r + 1) * El * per]) for r in range(world)]
+    out = []
+    for r in range(world):
+        q, f = wq[r * El:(r + 1) * El], sf[r * El * per:(r + 1) * El * per]
+        if n_shared:
+            q = torch.cat([q, wq[E:E + 1]]).contiguous()
+            f = torch.cat([f, sf[E * per:(E + 1) * per]]).contiguous()
+        out.append((q, f))
+    return out
 
 
 def moe_ep_sym_alloc(nbytes: int) -> int:
@@ -683,4 +712,6 @@ def ep_views(cfg: MoeConfig, world: int, sym: torch.Tensor, ws: torch.Tensor,
         "xs": view(sym, aux.xs, moe_fp8_scale_bytes(R, cfg.H), U8, (-1,)) if aux.xs else None,
         "hq": view(ws, aux.hq, R * cfg.F, U8, (R, cfg.F)) if aux.hq else None,
         "hs": view(ws, aux.hs, moe_fp8_scale_bytes(R, cfg.F), U8, (-1,)) if aux.hs else None,
+        "recv_split": view(ws, aux.recv_split, El * (world + 1) * 4, i32, (El, world + 1)),
+        "y_ready": view(sym, aux.y_ready, 2 * ((R + 127) // 128) * 4, i32, (2, (R + 127) // 128)),
     }

@@ -35,6 +35,7 @@ dispatch_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ token_s
   __shared__ int s_slot[MAX_K + 1];
   // the shared expert's row of a token is one more destination
   const int KD = sh_row0 >= 0 ? K + 1 : K;
+  MOE_CHECK(KD <= MAX_K + 1 && K <= DC_THREADS);
   pdl_wait();
   pdl_trigger();
   for (int t = blockIdx.x; t < T; t += gridDim.x) {

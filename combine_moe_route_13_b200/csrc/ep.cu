@@ -57,13 +57,14 @@ constexpr int PLAN_THREADS = 1024;   // >= MAX_E: one thread per expert
 enum : int { FLAG_COUNTS = 0, FLAG_DISPATCH = 1, FLAG_Y = 2, NUM_FLAGS = 3 };
 
 struct SymLayout {
-  size_t counts = 0, flags = 0, xr = 0, y = 0, total = 0;
+  size_t counts = 0, flags = 0, yready = 0, xr = 0, y = 0, total = 0;
 };
 
 struct EpWs {
   size_t blk_cnt = 0, topk_idx = 0, topk_w = 0, counts = 0, overflow = 0, offsets = 0;
   size_t segoff = 0, totals = 0, slot = 0, row_src = 0;
-  size_t send_dst = 0, recv_off = 0, recv_cnt = 0, epoch = 0, h = 0, h_sh = 0, y_sh = 0;
+  size_t send_dst = 0, recv_off = 0, recv_cnt = 0, split = 0, epoch = 0, h = 0, h_sh = 0, y_sh = 0;
+  size_t x_sh = 0;   // fp8 layer with a shared expert: this rank's quantised tokens
   size_t total = 0;
 };
 
@@ -73,6 +74,9 @@ int64_t recv_rows(const moe_config_t& c, int W) {
                            El * W * (int64_t)c.capacity) +
          El * (c.row_align - 1);
 }
+
+// 128-row blocks of a receive buffer: the ready counters of one bank.
+int64_t ready_blocks(const moe_config_t& c, int W) { return ceil_div(recv_rows(c, W), READY_ROWS); }
 
 // The grouped GEMM's view of a rank: its E/W local experts, each with up to
 // W*C received rows, R_recv rows in all (max_rows of this config = R_recv).
@@ -103,6 +107,7 @@ SymLayout sym_layout(const moe_config_t& c, int W) {
   size_t p = 0;
   L.counts = p; p += align256((size_t)W * c.E * 4);
   L.flags = p;  p += align256((size_t)NUM_FLAGS * W * 4);
+  L.yready = p; p += align256((size_t)2 * ready_blocks(c, W) * 4);
   L.xr = p;     p += align256(std::max<size_t>((size_t)R * c.H * as, fp8_bytes(R, c.H)));
   L.y = p;      p += align256((size_t)R * c.H * as);
   L.total = p;
@@ -128,12 +133,15 @@ EpWs ep_ws_layout(const moe_config_t& c, int W) {
   L.send_dst = p;  p += align256((size_t)c.E * 4);
   L.recv_off = p;  p += align256((size_t)(El + 1) * 4);
   L.recv_cnt = p;  p += align256((size_t)El * 4);
+  L.split = p;     p += align256((size_t)El * (W + 1) * 4);
   L.epoch = p;     p += 256;   // the device-resident step counter
   L.h = p;         p += align256(std::max<size_t>((size_t)recv_rows(c, W) * c.F * act_size(c.act_dtype),
                                                  fp8_bytes(recv_rows(c, W), c.F)));
   if (c.n_shared) {   // the shared expert's h and y for this rank's own tokens
-    L.h_sh = p;    p += align256((size_t)c.T * c.F * act_size(c.act_dtype));
+    L.h_sh = p;    p += align256(std::max<size_t>((size_t)c.T * c.F * act_size(c.act_dtype),
+                                                  fp8_bytes(c.T, c.F)));
     L.y_sh = p;    p += align256((size_t)c.T * c.H * act_size(c.act_dtype));
+    L.x_sh = p;    p += align256(fp8_bytes(c.T, c.H));   // codes + scales (fp8 layer)
   }
   L.total = p;
   return L;
@@ -147,20 +155,25 @@ moe_status_t ep_validate(const moe_config_t* c, const moe_ep_t* ep) {
   if (W < 1 || ep->rank < 0 || ep->rank >= W) return MOE_ERR_INVALID_ARG;
   if (W > MAX_W) return MOE_ERR_UNSUPPORTED;
   if (c->E % W != 0 || c->S % W != 0) return MOE_ERR_INVALID_ARG;
-  if (c->n_shared != 0 && c->act_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if ((int64_t)W * c->T > INT_MAX / 2 || (int64_t)W * c->capacity > INT_MAX / 2)
     return MOE_ERR_UNSUPPORTED;
   if (recv_rows(*c, W) > INT_MAX / 2) return MOE_ERR_UNSUPPORTED;
+  if (ep->flags & ~(MOE_EP_TILE_SIGNAL | MOE_EP_REMOTE_FIRST)) return MOE_ERR_INVALID_ARG;
+  if ((ep->flags & MOE_EP_REMOTE_FIRST) && !(ep->flags & MOE_EP_TILE_SIGNAL))
+    return MOE_ERR_INVALID_ARG;
+  if ((ep->flags & MOE_EP_TILE_SIGNAL) &&
+      (c->act_dtype != MOE_BF16 || c->row_align % READY_ROWS != 0))
+    return MOE_ERR_UNSUPPORTED;
   const moe_config_t l = local_cfg(*c, W);
   return validate(&l, true);
 }
 
 // The fp8 expert-parallel layer: the fp8 grouped GEMM's limits on each rank's
-// local experts, and no shared expert.
+// local experts (and on its shared expert), untagged steps only.
 moe_status_t ep_validate_fp8(const moe_config_t* c, const moe_ep_t* ep) {
   moe_status_t st = ep_validate(c, ep);
   if (st != MOE_OK) return st;
-  if (c->n_shared != 0) return MOE_ERR_UNSUPPORTED;
+  if (ep->flags != 0) return MOE_ERR_UNSUPPORTED;
   const moe_config_t l = local_cfg(*c, ep->world);
   return validate_fp8(&l);
 }
@@ -243,12 +256,17 @@ __device__ __forceinline__ bool timed_out(const uint32_t* status) {
 
 // Block d writes this rank's counts into rank d's table, then sets rank d's
 // COUNTS flag for this rank (release, after a system-scope fence that orders
-// the whole block's writes before it).
+// the whole block's writes before it). A rank that has timed out writes
+// nothing into its peers' memory.
 __global__ void ep_publish_kernel(const int32_t* __restrict__ counts, int E, int W, int rank,
                                   void* const* __restrict__ peers, size_t counts_off,
-                                  size_t flags_off, Epoch epoch) {
+                                  size_t flags_off, Epoch epoch, const uint32_t* status) {
+  __shared__ int s_skip;
   pdl_wait();
   pdl_trigger();
+  if (threadIdx.x == 0) s_skip = timed_out(status);
+  __syncthreads();
+  if (s_skip) return;   // the same decision for every thread of the block
   const int d = blockIdx.x;
   int32_t* dst = reinterpret_cast<int32_t*>(static_cast<char*>(peers[d]) + counts_off) +
                  (size_t)rank * E;
@@ -267,7 +285,7 @@ __global__ void __launch_bounds__(PLAN_THREADS)
 ep_plan_kernel(const int32_t* __restrict__ counts_all, const uint32_t* flags, int E, int W,
                int rank, int C, int A, Epoch epoch, unsigned long long timeout_ns,
                uint32_t* status, int32_t* __restrict__ send_dst, int32_t* __restrict__ recv_off,
-               int32_t* __restrict__ recv_cnt) {
+               int32_t* __restrict__ recv_cnt, int32_t* __restrict__ split) {
   __shared__ long long s_scan[PLAN_THREADS];
   __shared__ int s_ok;
   pdl_wait();
@@ -277,14 +295,19 @@ ep_plan_kernel(const int32_t* __restrict__ counts_all, const uint32_t* flags, in
   __syncthreads();
   const int e = threadIdx.x;
   const int El = E / W;
+  MOE_CHECK(E <= PLAN_THREADS && W <= MAX_W);
   long long tot = 0, pre = 0;
-  if (e < E && s_ok) {
+  // a local expert's row split by sender: its senders' blocks in rank order
+  int32_t* sp = (e < E && e / El == rank) ? split + (size_t)(e - rank * El) * (W + 1) : nullptr;
+  if (e < E) {
     for (int s = 0; s < W; ++s) {
+      if (sp) sp[s] = (int32_t)tot;
       // written by the peers: read from L2, never from a stale L1 line
-      const int c = min(max(__ldcg(counts_all + (size_t)s * E + e), 0), C);
+      const int c = s_ok ? min(max(__ldcg(counts_all + (size_t)s * E + e), 0), C) : 0;
       tot += c;
       if (s < rank) pre += c;
     }
+    if (sp) sp[W] = (int32_t)tot;
   }
   const long long aligned = (tot + A - 1) / A * A;
   s_scan[e] = e < E ? aligned : 0;
@@ -343,7 +366,7 @@ ep_dispatch_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ topk
         if (sl >= 0 && sl < slot_end) {
           const long long row =
               (e >= 0 && e < E) ? (long long)send_dst[e] + (sl - offsets[e]) : -1;
-          if (row >= 0 && row < n_recv)
+          if (row >= 0 && row < n_recv && MOE_CHECKED(e / El < W))
             dp = reinterpret_cast<uint4*>(s_peer[e / El] + xr_off) + row * row_vecs;
           else
             atomicCAS(status, 0u, (uint32_t)MOE_ERR_DEVICE_INPUT);
@@ -476,6 +499,24 @@ __global__ void ep_wait_kernel(const uint32_t* flags, int W, Epoch epoch,
   }
 }
 
+// Before the down GEMM of a tile-signalled step: wait for every sender's
+// DISPATCH flag (each is raised after that rank's combine of the previous
+// step, the last reader of this owner's y and of the other bank of its ready
+// counters), then zero that other bank, which the next step counts into.
+__global__ void ep_wait_zero_kernel(const uint32_t* flags, int W, Epoch epoch,
+                                    unsigned long long timeout_ns, uint32_t* status,
+                                    uint32_t* yready, int nblk) {
+  __shared__ int s_ok;
+  pdl_wait();
+  pdl_trigger();
+  const uint32_t e = step_epoch(epoch);
+  if (threadIdx.x == 0) s_ok = wait_all(flags, W, e, timeout_ns, status);
+  __syncthreads();
+  if (!s_ok) return;
+  uint32_t* other = yready + (size_t)((e + 1u) & 1u) * nblk;
+  for (int i = threadIdx.x; i < nblk; i += blockDim.x) other[i] = 0u;
+}
+
 // After the dispatch or the grouped GEMM (pdl_wait: that grid has finished and
 // its stores are visible to this one): every rank's flag `which` for this rank,
 // released at system scope after a system fence. Not after a timeout.
@@ -492,7 +533,12 @@ __global__ void ep_signal_kernel(void* const* __restrict__ peers, size_t flags_o
 
 // out[t] = sum over kept k (k order) of w[t,k] * y_owner[row], fp32 FMA from
 // 0, one rounding: the arithmetic of the one-rank combine, with the rows read
-// in place from their owners.
+// in place from their owners. After a timeout of this rank nothing is read
+// from the peers and `out` is left as it was.
+// ready_target > 0 (tile signalling): before a token is combined, each kept
+// row's 128-row block must have reached ready_target in its owner's ready
+// counters (bank = step & 1; acquire at system scope, all waits bounded by one
+// deadline); a token whose wait runs out is not written, nor is any later one.
 template <bool BF16>
 __global__ void __launch_bounds__(EP_THREADS)
 ep_combine_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ token_slot,
@@ -500,20 +546,27 @@ ep_combine_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restric
                   const int32_t* __restrict__ send_dst, void* const* __restrict__ peers,
                   size_t y_off, const uint4* __restrict__ y_sh, uint4* __restrict__ out, int T,
                   int K, int E, int El, int W, int row_vecs, int slot_end, long long n_recv,
-                  uint32_t* status) {
+                  uint32_t* status, size_t ready_off, int ready_nblk, uint32_t ready_target,
+                  Epoch epoch, unsigned long long timeout_ns) {
   __shared__ const uint4* s_src[MAX_K];
   __shared__ float s_w[MAX_K];
   __shared__ char* s_peer[MAX_W];
-  __shared__ int s_n;
+  __shared__ int s_n, s_skip;
   pdl_wait();
   pdl_trigger();
   if (threadIdx.x < W) s_peer[threadIdx.x] = static_cast<char*>(peers[threadIdx.x]);
+  if (threadIdx.x == 0) s_skip = timed_out(status);
+  __syncthreads();
+  if (s_skip) return;   // the same decision for every thread of the block
   constexpr int LANES = BF16 ? 8 : 4;
   const int k = threadIdx.x;
+  const size_t bank = ready_target ? (size_t)(step_epoch(epoch) & 1u) * ready_nblk : 0;
+  const unsigned long long deadline = ep_globaltimer() + timeout_ns;
   for (int t = blockIdx.x; t < T; t += gridDim.x) {
     __syncthreads();   // s_peer staged; the previous token's readers of s_src, s_w, s_n done
     if (k < 32) {      // warp 0 packs the kept assignments, k order
       const uint4* sp = nullptr;
+      const uint32_t* ready = nullptr;
       float wt = 0.f;
       if (k < K) {
         const int sl = token_slot[(size_t)t * K + k];
@@ -522,21 +575,44 @@ ep_combine_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restric
         if (sl >= 0 && sl < slot_end) {
           const long long row =
               (e >= 0 && e < E) ? (long long)send_dst[e] + (sl - offsets[e]) : -1;
-          if (row >= 0 && row < n_recv)
+          if (row >= 0 && row < n_recv) {
             sp = reinterpret_cast<const uint4*>(s_peer[e / El] + y_off) + row * row_vecs;
-          else
+            if (ready_target)
+              ready = reinterpret_cast<const uint32_t*>(s_peer[e / El] + ready_off) + bank +
+                      row / READY_ROWS;
+          } else {
             atomicCAS(status, 0u, (uint32_t)MOE_ERR_DEVICE_INPUT);
+          }
         }
       }
+      // each lane waits for its own row's block on its owner
+      bool ok = true;
+      if (ready) {
+        unsigned ns = 32;
+        while (ld_acquire_sys(ready) < ready_target) {
+          if (timed_out(status) || ep_globaltimer() > deadline) {
+            atomicCAS(status, 0u, (uint32_t)MOE_ERR_TIMEOUT);
+            ok = false;
+            break;
+          }
+          __nanosleep(ns);
+          if (ns < 1024) ns *= 2;
+        }
+      }
+      const bool all_ok = __all_sync(0xffffffffu, ok);
       const unsigned m = __ballot_sync(0xffffffffu, sp != nullptr);
       if (sp) {
         const int pos = __popc(m & ((1u << k) - 1u));
         s_src[pos] = sp;
         s_w[pos] = wt;
       }
-      if (k == 0) s_n = __popc(m);
+      if (k == 0) {
+        s_n = __popc(m);
+        s_skip = !all_ok;
+      }
     }
     __syncthreads();
+    if (s_skip) return;   // a wait ran out: this token and the rest stay unwritten
     const int n = s_n;
     uint4* dst = out + (size_t)t * row_vecs;
     for (int v0 = threadIdx.x; v0 < row_vecs; v0 += EP_THREADS * 2) {
@@ -623,9 +699,9 @@ ep_combine_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restric
 struct Ptrs {
   int32_t *topk_idx, *counts, *overflow, *offsets, *segoff, *slot, *row_src, *totals, *blk;
   float* topk_w;
-  int32_t *send_dst, *recv_off, *recv_cnt;
+  int32_t *send_dst, *recv_off, *recv_cnt, *split;
   uint32_t *status, *epoch;
-  char *h, *h_sh, *y_sh;   // h_sh / y_sh: nullptr without a shared expert
+  char *h, *h_sh, *y_sh, *x_sh;   // h_sh / y_sh / x_sh: nullptr without a shared expert
 };
 
 Ptrs ws_ptrs(const moe_config_t& c, int W, void* ws) {
@@ -646,10 +722,12 @@ Ptrs ws_ptrs(const moe_config_t& c, int W, void* ws) {
   p.send_dst = reinterpret_cast<int32_t*>(b + L.send_dst);
   p.recv_off = reinterpret_cast<int32_t*>(b + L.recv_off);
   p.recv_cnt = reinterpret_cast<int32_t*>(b + L.recv_cnt);
+  p.split = reinterpret_cast<int32_t*>(b + L.split);
   p.epoch = reinterpret_cast<uint32_t*>(b + L.epoch);
   p.h = b + L.h;
   p.h_sh = c.n_shared ? b + L.h_sh : nullptr;
   p.y_sh = c.n_shared ? b + L.y_sh : nullptr;
+  p.x_sh = c.n_shared ? b + L.x_sh : nullptr;
   return p;
 }
 
@@ -723,6 +801,8 @@ moe_status_t moe_ep_aux(const moe_config_t* cfg, const moe_ep_t* ep, void* sym, 
   a.y = sb + S.y;
   a.h_shared = p.h_sh;
   a.y_shared = p.y_sh;
+  a.recv_split = p.split;
+  a.y_ready = reinterpret_cast<uint32_t*>(sb + S.yready);
   if (cfg->H % FP8_BLOCK == 0 && cfg->F % FP8_BLOCK == 0) {   // the fp8 layer's payload
     const int64_t R = recv_rows(*cfg, ep->world);
     a.xq = reinterpret_cast<uint8_t*>(sb + S.xr);
@@ -773,7 +853,7 @@ moe_status_t moe_ep_route(const moe_config_t* cfg, const moe_ep_t* ep, const flo
   if (st != MOE_OK) return st;
   return cuda_st(launch_pdl(ep_publish_kernel, dim3(W), dim3(256), 0, s,
                             (const int32_t*)p.counts, c.E, W, ep->rank, peers, S.counts, S.flags,
-                            Epoch{ep->epoch, p.epoch}));
+                            Epoch{ep->epoch, p.epoch}, (const uint32_t*)p.status));
 }
 
 moe_status_t moe_ep_dispatch(const moe_config_t* cfg, const moe_ep_t* ep, const void* x,
@@ -792,7 +872,7 @@ moe_status_t moe_ep_dispatch(const moe_config_t* cfg, const moe_ep_t* ep, const 
                           (const int32_t*)(sb + S.counts), (const uint32_t*)(sb + S.flags), c.E,
                           W, ep->rank, c.capacity, c.row_align, Epoch{ep->epoch, p.epoch},
                           timeout_ns(*ep),
-                          p.status, p.send_dst, p.recv_off, p.recv_cnt));
+                          p.status, p.send_dst, p.recv_off, p.recv_cnt, p.split));
   if (st != MOE_OK) return st;
   const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
   if (c.T > 0) {
@@ -828,18 +908,67 @@ moe_status_t moe_ep_expert_mlp(const moe_config_t* cfg, const moe_ep_t* ep, cons
     // the shared expert on this rank's own tokens first: it needs nothing from
     // the peers, so it runs while their rows are still arriving
     const int El = c.E / W;
-    const char* wg = static_cast<const char*>(w_gu_local) + (size_t)El * 2 * c.F * c.H * 2;
-    const char* wd = static_cast<const char*>(w_d_local) + (size_t)El * c.H * c.F * 2;
-    st = launch_shared_mlp_bf16_tc(c, x, wg, wd, p.h_sh, p.y_sh, p.status, s);
+    const size_t as = act_size(c.act_dtype);
+    const char* wg = static_cast<const char*>(w_gu_local) + (size_t)El * 2 * c.F * c.H * as;
+    const char* wd = static_cast<const char*>(w_d_local) + (size_t)El * c.H * c.F * as;
+    if (c.act_dtype == MOE_BF16) {
+      st = launch_shared_mlp_bf16_tc(c, x, wg, wd, p.h_sh, p.y_sh, p.status, s);
+    } else if (c.T > 0) {
+      // the CUDA-core grouped SwiGLU with no routed group: its shared group is
+      // rows [0, T) of x, with expert 0 of the shared expert's weights
+      moe_config_t l = c;
+      l.E = 0;
+      l.K = 1;
+      l.S = 1;
+      l.capacity = 0;
+      l.row_align = 1;
+      l.n_shared = 1;
+      st = cuda_st(launch_mlp_f32(l, static_cast<const float*>(x), nullptr, nullptr,
+                                  reinterpret_cast<const float*>(wg),
+                                  reinterpret_cast<const float*>(wd),
+                                  reinterpret_cast<float*>(p.h_sh),
+                                  reinterpret_cast<float*>(p.y_sh), c.T, s));
+    }
     if (st != MOE_OK) return st;
   }
-  st = cuda_st(launch_pdl(ep_wait_kernel, dim3(1), dim3(32), 0, s,
-                          (const uint32_t*)(sb + S.flags) + FLAG_DISPATCH * W, W,
+  const moe_config_t l = local_cfg(c, W);
+  const int64_t R = recv_rows(c, W);
+  const uint32_t* dispatch_flags = (const uint32_t*)(sb + S.flags) + FLAG_DISPATCH * W;
+  if (ep->flags & MOE_EP_TILE_SIGNAL) {
+    // gate/up: each CTA waits only for the senders of its rows; then every
+    // sender (y and the other ready bank are free), then down, publishing y's
+    // blocks as they are stored
+    EpTiles t;
+    t.arrive = dispatch_flags;
+    t.split = p.split;
+    t.counter = p.epoch;
+    t.epoch = ep->epoch;
+    t.W = W;
+    t.rank = ep->rank;
+    t.remote_first = (ep->flags & MOE_EP_REMOTE_FIRST) ? 1 : 0;
+    t.wait_ns = timeout_ns(*ep);
+    st = launch_mlp_bf16_tc_ep(l, 1, sb + S.xr, p.recv_off, p.recv_cnt, w_gu_local, w_d_local,
+                               p.h, sb + S.y, R, p.status, s, t);
+    if (st != MOE_OK) return st;
+    const int nblk = (int)ready_blocks(c, W);
+    st = cuda_st(launch_pdl(ep_wait_zero_kernel, dim3(1), dim3(1024), 0, s, dispatch_flags, W,
+                            Epoch{ep->epoch, p.epoch}, timeout_ns(*ep), p.status,
+                            reinterpret_cast<uint32_t*>(sb + S.yready), nblk));
+    if (st != MOE_OK) return st;
+    t.arrive = nullptr;
+    t.yready = reinterpret_cast<uint32_t*>(sb + S.yready);
+    t.ready_blocks = nblk;
+    st = launch_mlp_bf16_tc_ep(l, 2, sb + S.xr, p.recv_off, p.recv_cnt, w_gu_local, w_d_local,
+                               p.h, sb + S.y, R, p.status, s, t);
+    if (st != MOE_OK) return st;
+    return cuda_st(launch_pdl(ep_signal_kernel, dim3(1), dim3(MAX_W), 0, s, peers, S.flags,
+                              (int)FLAG_Y, W, ep->rank, Epoch{ep->epoch, p.epoch},
+                              (const uint32_t*)p.status));
+  }
+  st = cuda_st(launch_pdl(ep_wait_kernel, dim3(1), dim3(32), 0, s, dispatch_flags, W,
                           Epoch{ep->epoch, p.epoch}, timeout_ns(*ep), p.status,
                           (uint32_t*)nullptr));
   if (st != MOE_OK) return st;
-  const moe_config_t l = local_cfg(c, W);
-  const int64_t R = recv_rows(c, W);
   if (c.act_dtype == MOE_BF16)
     st = launch_mlp_bf16_tc(l, sb + S.xr, p.recv_off, p.recv_cnt, w_gu_local, w_d_local, p.h,
                             sb + S.y, R, p.status, s);
@@ -867,20 +996,32 @@ moe_status_t moe_ep_combine(const moe_config_t* cfg, const moe_ep_t* ep, void* s
   const SymLayout S = sym_layout(c, W);
   char* sb = static_cast<char*>(sym);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = cuda_st(launch_pdl(ep_wait_kernel, dim3(1), dim3(32), 0, s,
-                          (const uint32_t*)(sb + S.flags) + FLAG_Y * W, W,
-                          Epoch{ep->epoch, p.epoch}, timeout_ns(*ep), p.status,
-                          p.epoch));   // the step's last wait moves the step counter on
-  if (st != MOE_OK || c.T == 0) return st;
-  const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
-  auto kernel = c.act_dtype == MOE_BF16 ? ep_combine_kernel<true> : ep_combine_kernel<false>;
-  return cuda_st(launch_pdl(kernel, dim3(resident_grid(kernel, EP_THREADS, c.T)),
+  const bool tiles = (ep->flags & MOE_EP_TILE_SIGNAL) != 0;
+  auto y_wait = [&]() {   // the step's last wait moves the step counter on
+    return cuda_st(launch_pdl(ep_wait_kernel, dim3(1), dim3(32), 0, s,
+                              (const uint32_t*)(sb + S.flags) + FLAG_Y * W, W,
+                              Epoch{ep->epoch, p.epoch}, timeout_ns(*ep), p.status, p.epoch));
+  };
+  if (!tiles) {
+    st = y_wait();
+    if (st != MOE_OK || c.T == 0) return st;
+  }
+  if (c.T > 0) {
+    const int row_vecs = (int)((int64_t)c.H * act_size(c.act_dtype) / 16);
+    auto kernel = c.act_dtype == MOE_BF16 ? ep_combine_kernel<true> : ep_combine_kernel<false>;
+    st = cuda_st(launch_pdl(kernel, dim3(resident_grid(kernel, EP_THREADS, c.T)),
                             dim3(EP_THREADS), 0, s, (const int32_t*)p.topk_idx,
                             (const int32_t*)p.slot, (const float*)p.topk_w,
                             (const int32_t*)p.offsets, (const int32_t*)p.send_dst, peers, S.y,
                             reinterpret_cast<const uint4*>(p.y_sh), static_cast<uint4*>(out),
                             c.T, c.K, c.E, c.E / W, W, row_vecs,
-                            (int)routed_rows(c), (long long)recv_rows(c, W), p.status));
+                            (int)routed_rows(c), (long long)recv_rows(c, W), p.status, S.yready,
+                            (int)ready_blocks(c, W), tiles ? ready_target(c) : 0u,
+                            Epoch{ep->epoch, p.epoch}, timeout_ns(*ep)));
+    if (st != MOE_OK) return st;
+  }
+  // tile signalling: the Y flags still order the next step's writes into the peers
+  return tiles ? y_wait() : MOE_OK;
 }
 
 moe_status_t moe_ep_layer_forward(const moe_config_t* cfg, const moe_ep_t* ep,
@@ -917,7 +1058,7 @@ moe_status_t moe_ep_dispatch_fp8(const moe_config_t* cfg, const moe_ep_t* ep, co
                           (const int32_t*)(sb + S.counts), (const uint32_t*)(sb + S.flags), c.E,
                           W, ep->rank, c.capacity, c.row_align, Epoch{ep->epoch, p.epoch},
                           timeout_ns(*ep),
-                          p.status, p.send_dst, p.recv_off, p.recv_cnt));
+                          p.status, p.send_dst, p.recv_off, p.recv_cnt, p.split));
   if (st != MOE_OK) return st;
   if (c.T > 0) {
     st = cuda_st(launch_pdl(ep_dispatch_fp8_kernel,
@@ -929,9 +1070,15 @@ moe_status_t moe_ep_dispatch_fp8(const moe_config_t* cfg, const moe_ep_t* ep, co
                             c.H / 8, (int)routed_rows(c), (long long)R, p.status));
     if (st != MOE_OK) return st;
   }
-  return cuda_st(launch_pdl(ep_signal_kernel, dim3(1), dim3(MAX_W), 0, s, peers, S.flags,
-                            (int)FLAG_DISPATCH, W, ep->rank, Epoch{ep->epoch, p.epoch},
-                            (const uint32_t*)p.status));
+  st = cuda_st(launch_pdl(ep_signal_kernel, dim3(1), dim3(MAX_W), 0, s, peers, S.flags,
+                          (int)FLAG_DISPATCH, W, ep->rank, Epoch{ep->epoch, p.epoch},
+                          (const uint32_t*)p.status));
+  if (st != MOE_OK || !c.n_shared || c.T == 0) return st;
+  // the shared expert's input: this rank's own token rows, quantised with the
+  // dispatch's arithmetic (codes and blocked scales, rows from 0), after the
+  // flags so that the peers' transfers are not held up by it
+  uint8_t* xq_sh = reinterpret_cast<uint8_t*>(p.x_sh);
+  return cuda_st(launch_quantize_fp8(x, c.T, c.H, xq_sh, xq_sh + align256((size_t)c.T * c.H), s));
 }
 
 moe_status_t moe_ep_expert_mlp_fp8(const moe_config_t* cfg, const moe_ep_t* ep,
@@ -952,6 +1099,28 @@ moe_status_t moe_ep_expert_mlp_fp8(const moe_config_t* cfg, const moe_ep_t* ep,
   const int64_t R = recv_rows(c, W);
   char* sb = static_cast<char*>(sym);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (c.n_shared && c.T > 0) {
+    // the shared expert on this rank's own tokens first (codes and scales of
+    // the last local expert; it needs nothing from the peers)
+    const int El = c.E / W;
+    const int64_t kg_gu = ceil_div(c.H / FP8_BLOCK, 4), kg_d = ceil_div(c.F / FP8_BLOCK, 4);
+    moe_config_t l = c;
+    l.E = 0;
+    l.K = 1;
+    l.S = 1;
+    l.capacity = 0;
+    l.row_align = 128;
+    l.n_shared = 1;
+    const uint8_t* xq_sh = reinterpret_cast<const uint8_t*>(p.x_sh);
+    uint8_t* hq_sh = reinterpret_cast<uint8_t*>(p.h_sh);
+    st = launch_mlp_fp8(
+        l, xq_sh, xq_sh + align256((size_t)c.T * c.H), nullptr, nullptr,
+        wq_gu_local + (size_t)El * 2 * c.F * c.H,
+        ws_gu_local + (size_t)El * 2 * c.F / 128 * kg_gu * SF_CHUNK,
+        wq_d_local + (size_t)El * c.H * c.F, ws_d_local + (size_t)El * c.H / 128 * kg_d * SF_CHUNK,
+        hq_sh, hq_sh + align256((size_t)c.T * c.F), p.y_sh, c.T, p.status, s);
+    if (st != MOE_OK) return st;
+  }
   st = cuda_st(launch_pdl(ep_wait_kernel, dim3(1), dim3(32), 0, s,
                           (const uint32_t*)(sb + S.flags) + FLAG_DISPATCH * W, W,
                           Epoch{ep->epoch, p.epoch}, timeout_ns(*ep), p.status,

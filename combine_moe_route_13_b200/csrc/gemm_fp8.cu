@@ -60,7 +60,14 @@ constexpr int B_HALF = 128 * BK;                // 16 KB
 constexpr int OPER_BYTES = A_BYTES + 2 * B_HALF;
 constexpr int SF_STAGE = 3 * SF_CHUNK;          // A, B rows 0-127, B rows 128-255
 constexpr int STAGES = 4;
-constexpr int NUM_THREADS = 192;
+// Threads: warp 0 TMA, warp 1 MMA, then the epilogue warps: eight for gate/up
+// (two per TMEM lane quarter, each taking half of the tile's columns, so that
+// a thread holds its 64 gate and 64 up accumulators in registers and TMEM is
+// released before the SwiGLU and the quantisation run), four for down.
+template <int MODE>
+__host__ __device__ constexpr int epi_warps() { return MODE == 0 ? 8 : 4; }
+template <int MODE>
+__host__ __device__ constexpr int num_threads() { return 64 + 32 * epi_warps<MODE>(); }
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL0 = 256;
 constexpr uint32_t SF_COLS = 12;                // per scale slot: 4 (A) + 8 (B)
@@ -74,7 +81,8 @@ struct Ctl {
   uint64_t tfull, tempty, drain;
   uint32_t tmem_base;
   int abort;
-  int wsum[8];
+  int wsum[16];
+  float amax[2][2][128];   // gate/up: [tile parity][column half][row] partial amax of h
 };
 
 size_t smem_bytes(int E) {
@@ -168,8 +176,14 @@ __device__ __forceinline__ void stage_row(uint32_t staging, int r, const uint4 (
   }
 }
 
+// Named barrier of the epilogue warps.
 template <int MODE>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__device__ __forceinline__ void epi_bar() {
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * epi_warps<MODE>()) : "memory");
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(num_threads<MODE>(), 1)
 fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmOut, const uint8_t* __restrict__ sfa,
                  const uint8_t* __restrict__ sfb, void* __restrict__ out_v,
@@ -178,6 +192,8 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                  const int32_t* __restrict__ counts, int E, int C, long long R_max,
                  uint32_t* __restrict__ status, int sh_rows, int sh_row0) {
   constexpr int BN_OUT = (MODE == 0) ? 128 : 256;   // output columns per tile
+  constexpr int NUM_THREADS = num_threads<MODE>();
+  constexpr int EPI_WARPS = epi_warps<MODE>();
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = saddr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -197,6 +213,9 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   const int KB = Kdim / BK;
   const int KG = (KB + 3) / 4;   // k groups (scale chunks per row block)
   volatile int* abort_flag = &ctl->abort;
+  // drains wait for copies and MMAs already issued even after an abort (bounded
+  // by DRAIN_NS): shared memory and TMEM must not be released under them
+  volatile int no_abort = 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -204,7 +223,7 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       mbar_init(saddr(&ctl->empty[s]), 1);
     }
     mbar_init(saddr(&ctl->tfull), 1);
-    mbar_init(saddr(&ctl->tempty), 4);
+    mbar_init(saddr(&ctl->tempty), EPI_WARPS);
     mbar_init(saddr(&ctl->drain), 1);
     ctl->abort = 0;
     fence_mbar_init();
@@ -272,6 +291,7 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
         int m, n;
         const int e = decode_tile(tile, NT, P, G, m, n);
+        MOE_CHECK(e >= 0 && e < G && n >= 0 && n < NT && m >= 0 && m * BM < max(kept_s[e], 1));
         const int a_row = row_off[e] + m * BM;           // a multiple of 128
         const int b_row0 = e * b_rows_per_expert + n * BN_OUT;
         const uint8_t* sa_rows = sfa + (size_t)(a_row / 128) * KG * SF_CHUNK;
@@ -302,7 +322,7 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         if (!ok) break;
       }
       for (int i = max(0, it - STAGES); i < it; ++i)
-        wait_phase(saddr(&ctl->full[i % STAGES]), (uint32_t)(i / STAGES) & 1u, abort_flag, status,
+        wait_phase(saddr(&ctl->full[i % STAGES]), (uint32_t)(i / STAGES) & 1u, &no_abort, status,
                    DRAIN_NS);
     }
   } else if (warp == 1) {
@@ -325,6 +345,7 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           const uint32_t sa = base + s * OPER_BYTES;
           const uint32_t ss = sf_smem + s * SF_STAGE;
           const int sg = sf_group_of_stage(kb, KG);
+          MOE_CHECK(SF_COL0 + 2 * SF_COLS <= TMEM_COLS && s >= 0 && s < STAGES);
           if (sg >= 0) {   // this stage brought the scales of k group sg
             const uint32_t slot = tmem + SF_COL0 + (uint32_t)(sg & 1) * SF_COLS;
             sf_copy(slot, sf_desc(ss));
@@ -346,16 +367,19 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         tc_commit<1>(saddr(&ctl->tfull));
       }
       tc_commit<1>(saddr(&ctl->drain));
-      wait_phase(saddr(&ctl->drain), 0u, abort_flag, status, DRAIN_NS);
+      wait_phase(saddr(&ctl->drain), 0u, &no_abort, status, DRAIN_NS);
     }
   } else {  // -------------------------------------------------------- epilogue
     const int q = warp & 3;                 // TMEM lane quarter of this warp
     const int r_in = q * 32 + lane;         // row of the tile
+    const int half = (warp - 2) >> 2;       // gate/up: which 64 of the tile's 128 h columns
     const int KBo = N_out / FP8_BLOCK;      // scale blocks of an output row (MODE 0)
     int tcount = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
       int m, n;
       const int e = decode_tile(tile, NT, P, G, m, n);
+      MOE_CHECK(e >= 0 && e < G && n >= 0 && n < NT && m >= 0 && m * BM < max(kept_s[e], 1) &&
+                r_in < BM);
       const int first = m * BM;
       const int rows = min(BM, kept_s[e] - first);
       const long long row0 = (long long)row_off[e] + first;
@@ -377,49 +401,69 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const bool staged = rows > 0 && row0 >= 0 && row0 + BM <= row_off[e + 1] && row0 + BM <= R_max;
       const uint32_t t0 = tmem + ((uint32_t)(q * 32) << 16);
       if (MODE == 0) {
-        float h[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t g[32], u[32];
-          tmem_ld32(t0 + (uint32_t)(c * 32), g);
-          tmem_ld32(t0 + 128u + (uint32_t)(c * 32), u);
-          tmem_ld_wait();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) h[c * 32 + k] = silu_mul(g[k], u[k]);
-        }
+        // this thread's 64 gate and 64 up accumulators (columns 64*half of
+        // each), loaded before anything is computed so that TMEM is released
+        // as early as possible
+        uint32_t g[64], u[64];
+        const uint32_t cg = t0 + (uint32_t)(64 * half);
+        tmem_ld32(cg, *reinterpret_cast<uint32_t(*)[32]>(g));
+        tmem_ld32(cg + 32u, *reinterpret_cast<uint32_t(*)[32]>(g + 32));
+        tmem_ld32(cg + 128u, *reinterpret_cast<uint32_t(*)[32]>(u));
+        tmem_ld32(cg + 160u, *reinterpret_cast<uint32_t(*)[32]>(u + 32));
+        tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_local(saddr(&ctl->tempty));   // TMEM free for the next tile
+        float h[64];
         float amax = 0.f;
 #pragma unroll
-        for (int k = 0; k < 128; ++k) amax = fmaxf(amax, fabsf(h[k]));
+        for (int k = 0; k < 64; ++k) {
+          h[k] = silu_mul(g[k], u[k]);
+          amax = fmaxf(amax, fabsf(h[k]));
+        }
+        // the h block is the tile's 128 columns: amax over both halves of the row
+        float* am = ctl->amax[tcount & 1][0];
+        am[half * 128 + r_in] = amax;
+        epi_bar<MODE>();
+        amax = fmaxf(amax, am[(half ^ 1) * 128 + r_in]);
         const int p = fp8_scale_exp(amax);
         const float inv = fp8_inv_scale(p);
-        uint4 o[8];
+        uint4 o[4];
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
+        for (int v = 0; v < 4; ++v) {
           const float* hv = h + 16 * v;
           o[v].x = fp8x2(hv[0] * inv, hv[1] * inv) | (fp8x2(hv[2] * inv, hv[3] * inv) << 16);
           o[v].y = fp8x2(hv[4] * inv, hv[5] * inv) | (fp8x2(hv[6] * inv, hv[7] * inv) << 16);
           o[v].z = fp8x2(hv[8] * inv, hv[9] * inv) | (fp8x2(hv[10] * inv, hv[11] * inv) << 16);
           o[v].w = fp8x2(hv[12] * inv, hv[13] * inv) | (fp8x2(hv[14] * inv, hv[15] * inv) << 16);
         }
-        if (row_ok) out_sf[sf_offset(grow, n, KBo)] = (uint8_t)(p + 127);
+        if (half == 0 && row_ok && MOE_CHECKED(n < KBo))
+          out_sf[sf_offset(grow, n, KBo)] = (uint8_t)(p + 127);
         if (staged) {
           if (threadIdx.x == 64) bulk_wait_read_all();   // the previous box has left smem
-          epilogue_bar();
-          stage_row(staging, r_in, o);
+          epi_bar<MODE>();
+          // 16-byte chunks 4*half .. 4*half+3 of row r_in, at the 128-byte
+          // swizzle's positions
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const int c = 4 * half + v;
+            const uint32_t a = staging + (uint32_t)(r_in * 128 + ((c ^ (r_in & 7)) << 4));
+            MOE_CHECK(r_in * 128 + 128 <= STAGING_BYTES);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(o[v].x),
+                         "r"(o[v].y), "r"(o[v].z), "r"(o[v].w)
+                         : "memory");
+          }
           fence_proxy_async_smem();
-          epilogue_bar();
+          epi_bar<MODE>();
           if (threadIdx.x == 64) {
             tma_store_2d(&tmOut, n * BN_OUT, (int)row0, staging);
             bulk_commit();
           }
         } else if (row_ok) {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(out_v) + grow * N_out +
-                                                (long long)n * BN_OUT);
+                                                (long long)n * BN_OUT + 64 * half);
 #pragma unroll
-          for (int v = 0; v < 8; ++v) dst[v] = o[v];
+          for (int v = 0; v < 4; ++v) dst[v] = o[v];
         }
       } else {
         uint32_t pk[128];   // 256 bf16 of this row
@@ -447,10 +491,10 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                               pk[c * 32 + 4 * v + 3]);
           if (staged) {
             if (threadIdx.x == 64) bulk_wait_read_all();
-            epilogue_bar();
+            epi_bar<MODE>();
             stage_row(staging, r_in, o);
             fence_proxy_async_smem();
-            epilogue_bar();
+            epi_bar<MODE>();
             if (threadIdx.x == 64) {
               tma_store_2d(&tmOut, col, (int)row0, staging);
               bulk_commit();
@@ -497,7 +541,7 @@ cudaError_t launch_one(int grid, size_t smem, cudaStream_t s, const CUtensorMap&
                        int sh_row0) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.blockDim = dim3(num_threads<MODE>());
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];

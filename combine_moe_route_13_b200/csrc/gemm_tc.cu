@@ -96,7 +96,7 @@ constexpr int STAGING_BYTES = 128 * 64 * 2;   // one 128-row x 64-column bf16 ou
 template <int CG>
 size_t smem_bytes(int E) {
   return 1024 + (size_t)Cfg<CG>::STAGES * Cfg<CG>::STAGE_BYTES + STAGING_BYTES + sizeof(Ctl) +
-         (size_t)(3 * E + 2) * 4;
+         (size_t)(6 * E + 8) * 4;
 }
 
 // silu(g) * u = g * u / (1 + exp(-g)), with the fast exponential and the fast
@@ -108,21 +108,101 @@ __device__ __forceinline__ float silu_mul(uint32_t g_bits, uint32_t u_bits) {
   return __fdividef(g * __uint_as_float(u_bits), 1.0f + __expf(-g));
 }
 
-// Tile t -> (expert, m tile, n tile). Expert e owns tiles [NT*P[e], NT*P[e+1])
-// where P is the prefix of its M-tile counts; inside, n-major then m.
-__device__ __forceinline__ void decode_tile(int tile, int NT, const int* P, int E, int& e, int& m,
-                                            int& n) {
-  const int g = tile / NT;
-  int lo = 0, hi = E;   // P[lo] <= g < P[hi]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (P[mid] <= g) lo = mid; else hi = mid;
+// Tile t -> (group, m tile, n tile). The tiles come in two sets: first every
+// group's M tiles outside [ml0[e], ml0[e] + nl[e]), then those inside (nl = 0
+// everywhere puts every tile in the first set). In each set a group owns a
+// contiguous range, n-major then m inside; P is the prefix of the groups' M
+// tiles and PB the prefix of nl, so the first set's prefix is P - PB.
+__device__ __forceinline__ void decode_tile(int tile, int NT, const int* P, const int* PB,
+                                            const int* ml0, int G, int& e, int& m, int& n) {
+  const int totalA = (P[G] - PB[G]) * NT;
+  int lo = 0, hi = G;
+  if (tile < totalA) {
+    const int g = tile / NT;   // P[lo] - PB[lo] <= g < P[hi] - PB[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (P[mid] - PB[mid] <= g) lo = mid; else hi = mid;
+    }
+    e = lo;
+    const int base = P[e] - PB[e];
+    const int mt = (P[e + 1] - PB[e + 1]) - base;
+    const int local = tile - NT * base;
+    n = local / mt;
+    const int mm = local - n * mt;
+    m = mm < ml0[e] ? mm : mm + (PB[e + 1] - PB[e]);
+  } else {
+    const int t2 = tile - totalA;
+    const int g = t2 / NT;     // PB[lo] <= g < PB[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (PB[mid] <= g) lo = mid; else hi = mid;
+    }
+    e = lo;
+    const int nl = PB[e + 1] - PB[e];
+    const int local = t2 - NT * PB[e];
+    n = local / nl;
+    m = ml0[e] + (local - n * nl);
   }
-  e = lo;
-  const int mt = P[e + 1] - P[e];
-  const int local = tile - NT * P[e];
-  n = local / mt;
-  m = local - n * mt;
+}
+
+// Exclusive prefix of `v` over the block's threads (all threads call it);
+// wsum: one int per warp of shared memory. Returns the prefix; *total the sum.
+__device__ __forceinline__ int block_exclusive(int v, int* wsum, int warp, int lane, int* total) {
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  int run = incl - v, tot = 0;
+  for (int w = 0; w < NUM_THREADS / 32; ++w) {
+    if (w < warp) run += wsum[w];
+    tot += wsum[w];
+  }
+  __syncthreads();   // wsum may be reused
+  *total = tot;
+  return run;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_sys_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_add_sys(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.sys.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Raise the abort flag of the other CTA of the pair (its shared memory).
+__device__ __forceinline__ void abort_peer_cta(uint32_t abort_local, uint32_t peer) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(map_to_rank(abort_local, peer)), "r"(1u)
+               : "memory");
+}
+
+// Wait until the flag has reached `epoch` (acquire at system scope). Gives up
+// when the CTA aborts, when an earlier wait of this step gave up (the status
+// word holds MOE_ERR_TIMEOUT), or after limit_ns, recording MOE_ERR_TIMEOUT
+// and raising the abort flag.
+__device__ __noinline__ bool wait_arrival(const uint32_t* flag, uint32_t epoch,
+                                          volatile int* abort_flag, uint32_t* status,
+                                          unsigned long long limit_ns) {
+  if ((int32_t)(ld_acquire_sys_u32(flag) - epoch) >= 0) return true;
+  const unsigned long long t0 = globaltimer();
+  unsigned ns = 64;
+  while (true) {
+    if (*abort_flag) return false;
+    if ((int32_t)(ld_acquire_sys_u32(flag) - epoch) >= 0) return true;
+    if (*(volatile uint32_t*)status == (uint32_t)MOE_ERR_TIMEOUT || globaltimer() - t0 > limit_ns) {
+      atomicCAS(status, 0u, (uint32_t)MOE_ERR_TIMEOUT);
+      *abort_flag = 1;
+      return false;
+    }
+    __nanosleep(ns);
+    if (ns < 1024) ns *= 2;
+  }
 }
 
 template <int MODE, int CG>
@@ -133,7 +213,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 int b_second_off, const int32_t* __restrict__ offsets,
                 const int32_t* __restrict__ counts, int E, int C, long long R_max,
                 uint32_t* __restrict__ status, uint32_t* __restrict__ row_ready,
-                int dense_rows, int sh_rows, int sh_a_row, int sh_out_row) {
+                int dense_rows, int sh_rows, int sh_a_row, int sh_out_row, const EpTiles ept) {
   using CF = Cfg<CG>;
   constexpr int STAGES = CF::STAGES;
   constexpr int BN_OUT = (MODE == 0) ? 128 : 256;   // output columns per tile
@@ -149,8 +229,10 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   // sh_rows rows are read from tmA2 at row sh_a_row and written at sh_out_row.
   const int G = sh_rows > 0 ? E + 1 : E;
   int* P = reinterpret_cast<int*>(ctl + 1);   // [G+1] M-tile prefix
-  int* row_off = P + (G + 1);                 // [G+1] first output row of each group, and its end
+  int* PB = P + (G + 1);                      // [G+1] prefix of the tiles ordered last
+  int* row_off = PB + (G + 1);                // [G+1] first output row of each group, and its end
   int* kept_s = row_off + (G + 1);            // [G]
+  int* ml0 = kept_s + G;                      // [G] first M tile ordered last
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;   // position in the pair
@@ -159,6 +241,9 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   const int NT = (N_out + BN_OUT - 1) / BN_OUT;
   const int KB = Kdim / BK;
   volatile int* abort_flag = &ctl->abort;
+  // drains wait for copies and MMAs already issued even after an abort (bounded
+  // by DRAIN_NS): shared memory and TMEM must not be released under them
+  volatile int no_abort = 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -183,10 +268,13 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   }
   pdl_wait();      // everything above touched only this CTA's shared memory and TMEM
   pdl_trigger();
-  {  // per-group kept rows, first row and M-tile prefix (block scan)
+  // this step's number (tile-signalled expert-parallel GEMMs only)
+  const uint32_t step = ept.epoch ? ept.epoch
+                                  : (ept.counter ? *(volatile const uint32_t*)ept.counter + 1u : 0u);
+  {  // per-group kept rows, first row and M-tile prefix (block scans)
     const int chunk = (G + NUM_THREADS - 1) / NUM_THREADS;
     const int e0 = threadIdx.x * chunk;
-    int local = 0;
+    int local = 0, localB = 0;
     for (int i = 0; i < chunk; ++i) {
       const int e = e0 + i;
       if (e < G) {
@@ -202,28 +290,42 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         }
         kept_s[e] = k;
         row_off[e] = off;
-        local += (k + CF::TILE_ROWS - 1) / CF::TILE_ROWS;
+        const int mt = (k + CF::TILE_ROWS - 1) / CF::TILE_ROWS;
+        local += mt;
+        // remote-first order: the M tiles whose rows are all this owner's own
+        // (one contiguous block of the expert's rows) are ordered last
+        int first_local = 0, n_local = 0;
+        if (ept.remote_first && ept.split != nullptr && e < E && k > 0) {
+          const int* sp = ept.split + (size_t)e * (ept.W + 1);
+          const int lo = min(max(sp[ept.rank], 0), k), hi = min(max(sp[ept.rank + 1], lo), k);
+          const int m_lo = (lo + CF::TILE_ROWS - 1) / CF::TILE_ROWS;
+          const int m_hi = hi >= k ? mt : hi / CF::TILE_ROWS;
+          if (m_hi > m_lo) {
+            first_local = m_lo;
+            n_local = m_hi - m_lo;
+          }
+        }
+        ml0[e] = first_local;
+        PB[e] = n_local;   // replaced by its prefix below
+        localB += n_local;
       }
     }
-    int incl = local;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int o = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += o;
-    }
-    if (lane == 31) ctl->wsum[warp] = incl;
-    __syncthreads();
-    int run = incl - local;
-    for (int w = 0; w < warp; ++w) run += ctl->wsum[w];
+    int tot = 0, totB = 0;
+    int run = block_exclusive(local, ctl->wsum, warp, lane, &tot);
+    int runB = block_exclusive(localB, ctl->wsum, warp, lane, &totB);
     for (int i = 0; i < chunk; ++i) {
       const int e = e0 + i;
       if (e < G) {
         P[e] = run;
         run += (kept_s[e] + CF::TILE_ROWS - 1) / CF::TILE_ROWS;
+        const int n_local = PB[e];
+        PB[e] = runB;
+        runB += n_local;
       }
     }
     if (threadIdx.x == NUM_THREADS - 1) {
-      P[G] = run;
+      P[G] = tot;
+      PB[G] = totB;
       row_off[G] = dense_rows > 0 ? dense_rows : (G > E ? sh_out_row + sh_rows : offsets[E]);
     }
   }
@@ -237,14 +339,40 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   if (warp == 0) {
     if (lane == 0) {  // ------------------------------------------------ TMA producer
       int it = 0;
+      uint64_t seen = 0;   // senders whose DISPATCH flag of this step has been seen
+      bool ok = true;
       for (int tile = cluster_id; tile < total; tile += n_clusters) {
         int e, m, n;
-        decode_tile(tile, NT, P, G, e, m, n);
+        decode_tile(tile, NT, P, PB, ml0, G, e, m, n);
+        MOE_CHECK(e >= 0 && e < G && n >= 0 && n < NT && m >= 0 &&
+                  m * CF::TILE_ROWS < max(kept_s[e], 1));
         const bool shared_group = e >= E;
         const CUtensorMap* mapA = shared_group ? &tmA2 : &tmA;
         const int a_row = (shared_group ? sh_a_row : row_off[e]) + m * CF::TILE_ROWS + (int)rank * BM;
         const int b_row0 = e * b_rows_per_expert + n * N_STEP;
-        bool ok = true;
+        if (MODE == 0 && ept.arrive != nullptr && !shared_group) {
+          // this CTA's rows of the tile: wait for every sender that owns some of them
+          const int lo = m * CF::TILE_ROWS + (int)rank * BM;
+          const int hi = min(lo + BM, kept_s[e]);
+          const int* sp = ept.split + (size_t)e * (ept.W + 1);
+          bool waited = false;
+          for (int s = 0; s < ept.W && ok && lo < hi; ++s) {
+            if ((seen >> s) & 1ull) continue;
+            const int a = sp[s], b = sp[s + 1];
+            if (b > a && a < hi && b > lo) {
+              ok = wait_arrival(ept.arrive + s, step, abort_flag, status, ept.wait_ns);
+              seen |= 1ull << s;
+              waited = true;
+            }
+          }
+          if (!ok) {
+            if (CG == 2) abort_peer_cta(saddr(&ctl->abort), rank ^ 1u);
+            break;
+          }
+          // the rows were written by the peers' generic stores: order the
+          // acquire above before this CTA's TMA (async proxy) reads them
+          if (waited) fence_proxy_async_global();
+        }
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
@@ -253,6 +381,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             break;
           }
           const uint32_t sa = base + s * CF::STAGE_BYTES;
+          MOE_CHECK(s >= 0 && s < STAGES && a_row >= 0);
           const uint32_t fb_local = saddr(&ctl->full[s]);
           const uint32_t fb = (CG == 2) ? map_to_rank(fb_local, 0) : fb_local;
           if (leader) mbar_expect_tx(fb_local, CF::STAGE_BYTES * CG);
@@ -266,11 +395,12 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         }
         if (!ok) break;
       }
+      (void)seen;
       // the copies of the last STAGES stages must land before the CTA exits
       // (the leader's barriers also count the peer's copies)
       if (leader)
         for (int i = max(0, it - STAGES); i < it; ++i)
-          wait_phase(saddr(&ctl->full[i % STAGES]), (uint32_t)(i / STAGES) & 1u, abort_flag,
+          wait_phase(saddr(&ctl->full[i % STAGES]), (uint32_t)(i / STAGES) & 1u, &no_abort,
                      status, DRAIN_NS);
     }
   } else if (warp == 1) {
@@ -281,6 +411,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         const uint32_t tph = (uint32_t)(tcount >> 1) & 1u;
         if (!wait_phase(saddr(&ctl->tempty[b]), tph ^ 1u, abort_flag, status, WAIT_NS)) break;
         tc_fence_after();
+        MOE_CHECK(b * UMMA_N + UMMA_N <= (int)TMEM_COLS);
         const uint32_t d = tmem + (uint32_t)(b * UMMA_N);
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb, ++it) {
@@ -305,7 +436,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       }
       // every MMA this thread issued must finish before TMEM is released
       tc_commit<CG>(saddr(&ctl->drain));
-      wait_phase(saddr(&ctl->drain), 0u, abort_flag, status, DRAIN_NS);
+      wait_phase(saddr(&ctl->drain), 0u, &no_abort, status, DRAIN_NS);
     }
   } else {  // -------------------------------------------------------- epilogue
     const int q = warp & 3;                 // TMEM sub-partition of this warp
@@ -315,7 +446,9 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     int tcount = 0;
     for (int tile = cluster_id; tile < total; tile += n_clusters, ++tcount) {
       int e, m, n;
-      decode_tile(tile, NT, P, G, e, m, n);
+      decode_tile(tile, NT, P, PB, ml0, G, e, m, n);
+      MOE_CHECK(e >= 0 && e < G && n >= 0 && n < NT && m >= 0 &&
+                m * CF::TILE_ROWS < max(kept_s[e], 1) && r_in < BM);
       const int first = m * CF::TILE_ROWS + (int)rank * BM;   // first row of this half tile
       const int rows = min(BM, kept_s[e] - first);
       const long long grow = (long long)row_off[e] + first + r_in;
@@ -366,6 +499,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 #pragma unroll 1
       for (int c = 0; c < CHUNKS; ++c) {
         uint4 o[8];
+        MOE_CHECK(c * 64 + 64 + (MODE == 0 ? 128 : 0) <= UMMA_N);
         if (MODE == 0) {   // gate in TMEM columns [c*64, +64), up in [128 + c*64, +64)
           uint32_t g[64], u[64];
           tmem_ld64(t0 + (uint32_t)(c * 64), g);
@@ -395,6 +529,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         if (staged) {
           if (threadIdx.x == 64) bulk_wait_read_all();   // the previous box has left smem
           epilogue_bar();
+          MOE_CHECK((r_in + 1) * 128 <= STAGING_BYTES && col + 64 <= N_out);
           // row r_in of the box, 16-byte chunk v at position v ^ (r_in % 8):
           // the 128-byte swizzle the output tensor map uses
 #pragma unroll
@@ -422,7 +557,20 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         const uint32_t tb = tempty_leader0 + (uint32_t)(b * sizeof(uint64_t));
         if (CG == 2) mbar_arrive_cluster(tb); else mbar_arrive_local(tb);
       }
-      if (row_ready != nullptr && rows > 0) {
+      if (MODE == 1 && ept.yready != nullptr && rows > 0) {
+        // The same publication at system scope, into this step's bank of the
+        // expert-parallel ready counters (read by the peers' combines).
+        __threadfence_system();
+        if (threadIdx.x == 64) {
+          bulk_wait_all();
+          fence_proxy_async_global();
+        }
+        epilogue_bar();
+        if (threadIdx.x == 64 && MOE_CHECKED(row0 / READY_ROWS < ept.ready_blocks))
+          red_release_add_sys(ept.yready + (size_t)(step & 1u) * ept.ready_blocks +
+                                  row0 / READY_ROWS,
+                              1u);
+      } else if (row_ready != nullptr && rows > 0) {
         // Publish this half tile: its 128 rows (one ready block: the rows are
         // aligned to 128) have one more N tile stored. The staged TMA stores
         // are waited for by their issuing thread and every thread fences its
@@ -433,7 +581,8 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
           fence_proxy_async_global();
         }
         epilogue_bar();
-        if (threadIdx.x == 64) red_release_add(row_ready + (row0 / READY_ROWS), 1u);
+        if (threadIdx.x == 64 && MOE_CHECKED(row0 >= 0 && row0 < R_max))
+          red_release_add(row_ready + (row0 / READY_ROWS), 1u);
       }
     }
     if (threadIdx.x == 64) bulk_wait_all();   // staged stores complete before the CTA exits
@@ -520,7 +669,8 @@ template <int CG>
 moe_status_t launch_mlp(const moe_config_t& c, const void* xp, const int32_t* offsets,
                         const int32_t* counts, const void* w_gu, const void* w_d, void* h,
                         void* y, int64_t R_max, uint32_t* status, cudaStream_t s,
-                        uint32_t* row_ready, const void* x_shared) {
+                        uint32_t* row_ready, const void* x_shared, int modes = 3,
+                        const EpTiles& ept = EpTiles{}) {
   const int n_sh = c.n_shared ? 1 : 0;
   const int G = c.E + n_sh;   // routed experts + the shared expert (last in the weights)
   CUtensorMap mx, mwgu, mh, mwd, my, mxs;
@@ -553,16 +703,18 @@ moe_status_t launch_mlp(const moe_config_t& c, const void* xp, const int32_t* of
   const int g1 = (int)std::min<int64_t>(units, t1) * CG;
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[2];
-  fill_launch<0, CG>(cfg, attr, g0, smem, s);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, tc_grouped_gemm<0, CG>, mx, mwgu, mh, mxs, h, c.F,
-                                     c.H, 2 * c.F, c.F, offsets, counts, c.E, c.capacity,
-                                     (long long)R_max, status, (uint32_t*)nullptr, 0, sh_rows,
-                                     sh_a_row, sh_row0);
-  if (e == cudaSuccess) {
+  cudaError_t e = cudaSuccess;
+  if (modes & 1) {
+    fill_launch<0, CG>(cfg, attr, g0, smem, s);
+    e = cudaLaunchKernelEx(&cfg, tc_grouped_gemm<0, CG>, mx, mwgu, mh, mxs, h, c.F, c.H, 2 * c.F,
+                           c.F, offsets, counts, c.E, c.capacity, (long long)R_max, status,
+                           (uint32_t*)nullptr, 0, sh_rows, sh_a_row, sh_row0, ept);
+  }
+  if (e == cudaSuccess && (modes & 2)) {
     fill_launch<1, CG>(cfg, attr, g1, smem, s);
     e = cudaLaunchKernelEx(&cfg, tc_grouped_gemm<1, CG>, mh, mwd, my, mh, y, c.H, c.F, c.H, 128,
                            offsets, counts, c.E, c.capacity, (long long)R_max, status, row_ready,
-                           0, sh_rows, sh_row0, sh_row0);
+                           0, sh_rows, sh_row0, sh_row0, ept);
   }
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -590,7 +742,7 @@ moe_status_t launch_router(const moe_config_t& c, const void* x, const void* w_g
   const cudaError_t e = cudaLaunchKernelEx(
       &cfg, tc_grouped_gemm<2, CG>, mx, mg, mx, mx, (void*)logits, c.E, c.H, 0, 128,
       (const int32_t*)nullptr, (const int32_t*)nullptr, 1, c.T, (long long)c.T, status,
-      (uint32_t*)nullptr, c.T, 0, 0, 0);
+      (uint32_t*)nullptr, c.T, 0, 0, 0, EpTiles{});
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -621,6 +773,22 @@ moe_status_t launch_shared_mlp_bf16_tc(const moe_config_t& c, const void* x, con
                              nullptr, x);
   return tc::launch_mlp<1>(l, x, nullptr, nullptr, w_gu_sh, w_d_sh, h, y, c.T, status, s, nullptr,
                            x);
+}
+
+moe_status_t launch_mlp_bf16_tc_ep(const moe_config_t& c, int modes, const void* xr,
+                                   const int32_t* offsets, const int32_t* counts,
+                                   const void* w_gu, const void* w_d, void* h, void* y,
+                                   int64_t R_max, uint32_t* status, cudaStream_t s,
+                                   const EpTiles& t) {
+  if (R_max == 0) return MOE_OK;
+  moe_config_t l = c;
+  l.n_shared = 0;
+  const int64_t rows_per_expert = std::min<int64_t>((int64_t)c.T * c.K, (int64_t)c.E * c.capacity) / c.E;
+  if (rows_per_expert >= 192)
+    return tc::launch_mlp<2>(l, xr, offsets, counts, w_gu, w_d, h, y, R_max, status, s, nullptr,
+                             nullptr, modes, t);
+  return tc::launch_mlp<1>(l, xr, offsets, counts, w_gu, w_d, h, y, R_max, status, s, nullptr,
+                           nullptr, modes, t);
 }
 
 moe_status_t launch_mlp_bf16_tc(const moe_config_t& c, const void* xp, const int32_t* offsets,

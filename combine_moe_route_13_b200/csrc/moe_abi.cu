@@ -102,9 +102,37 @@ static moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_O
 
 using namespace moe;
 
+#ifdef MOE_CHECK_BOUNDS
+namespace moe {
+__device__ unsigned int g_moe_bounds[2] = {0u, 0u};
+}
+#endif
+
 extern "C" {
 
-int32_t moe_version(void) { return 1 * 10000 + 1 * 100 + 0; }   // 1.1: moe_ep.h
+moe_status_t moe_debug_bounds_failures(uint32_t* failures, uint32_t* first_line, int32_t reset) {
+#ifdef MOE_CHECK_BOUNDS
+  if (!failures || !first_line) return MOE_ERR_INVALID_ARG;
+  unsigned int v[2] = {0u, 0u};
+  if (cudaDeviceSynchronize() != cudaSuccess ||
+      cudaMemcpyFromSymbol(v, moe::g_moe_bounds, sizeof(v)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  *failures = v[0];
+  *first_line = v[1];
+  if (reset) {
+    const unsigned int z[2] = {0u, 0u};
+    if (cudaMemcpyToSymbol(moe::g_moe_bounds, z, sizeof(z)) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+#else
+  (void)failures;
+  (void)first_line;
+  (void)reset;
+  return MOE_ERR_UNSUPPORTED;
+#endif
+}
+
+int32_t moe_version(void) { return 1 * 10000 + 2 * 100 + 0; }   // 1.2: tile-signalled moe_ep.h
 
 const char* moe_status_string(moe_status_t s) {
   switch (s) {

@@ -85,6 +85,29 @@ int resident_grid(void (*kernel)(KArgs...), int threads, int64_t work) {
   return (int)std::max<int64_t>(1, std::min<int64_t>(work, (int64_t)sms * per));
 }
 
+// Bounds-checked build (-DMOE_CHECK_BOUNDS, relocatable device code: the
+// library variant libmoe_check.so). MOE_CHECK(c) checks an internal index
+// invariant of a kernel (a decoded tile, a TMEM column, a shared-memory
+// staging offset, a table index); a failed check counts itself and records
+// the first failing source line in g_moe_bounds (read with
+// moe_debug_bounds_failures), and the guarded access is skipped where the
+// kernel uses MOE_CHECKED(c) as its condition. In the release build both
+// compile to nothing (MOE_CHECKED(c) is true).
+#if defined(MOE_CHECK_BOUNDS) && defined(__CUDACC__)
+extern __device__ unsigned int g_moe_bounds[2];   // failures, first failing line
+__device__ __forceinline__ void moe_bounds_fail(unsigned line) {
+  if (atomicAdd(&g_moe_bounds[0], 1u) == 0u) atomicExch(&g_moe_bounds[1], line);
+}
+#define MOE_CHECK(c)                                       \
+  do {                                                     \
+    if (!(c)) ::moe::moe_bounds_fail((unsigned)__LINE__);  \
+  } while (0)
+#define MOE_CHECKED(c) ((c) ? true : (::moe::moe_bounds_fail((unsigned)__LINE__), false))
+#else
+#define MOE_CHECK(c) ((void)0)
+#define MOE_CHECKED(c) true
+#endif
+
 #ifdef __CUDACC__
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {
@@ -140,6 +163,42 @@ moe_status_t launch_mlp_bf16_tc(const moe_config_t& c, const void* xp, const int
                                 void* h, void* y, int64_t R_max, uint32_t* status,
                                 cudaStream_t s, uint32_t* row_ready = nullptr,
                                 const void* x_shared = nullptr);
+
+// Tile signalling of an expert-parallel owner's grouped GEMMs ("Mixture-of-
+// Experts acceleration through overlap": the GEMM consumes rows as they arrive
+// and publishes output tiles through flags the consumer polls).
+//   Gate/up (arrive != nullptr): before a CTA loads its rows of a tile, it
+//   waits until every sender owning some of those rows has raised its
+//   DISPATCH flag of this step (acquire at system scope, bounded by wait_ns;
+//   a wait that runs out records MOE_ERR_TIMEOUT and ends the kernel).
+//   Down (yready != nullptr): each stored 128-row x 256-column tile adds 1 to
+//   its block's counter in bank (step & 1) of yready (release at system
+//   scope), so that a block is final when its counter reaches ceil(H / 256).
+//   remote_first: tiles holding rows of other senders run before the tiles
+//   that hold only this owner's own rows (the outputs other ranks read
+//   first), each set in the usual (expert, N tile, M tile) order.
+// The step number is `epoch`, or one past *counter when epoch is 0.
+struct EpTiles {
+  const uint32_t* arrive = nullptr;   // [W] this owner's DISPATCH flags, by sender
+  const int32_t* split = nullptr;     // [E_local][W+1]: sender s's first row within each local
+                                      // expert's rows; [W] = the expert's received rows
+  const uint32_t* counter = nullptr;
+  uint32_t epoch = 0;
+  int W = 0, rank = 0;
+  int remote_first = 0;
+  unsigned long long wait_ns = 0;
+  uint32_t* yready = nullptr;         // [2][ready_blocks]
+  int ready_blocks = 0;
+};
+
+// One or both launches (modes: bit 0 gate/up, bit 1 down) of the bf16 grouped
+// GEMM of launch_mlp_bf16_tc over an expert-parallel owner's local experts
+// (no shared group), tile-signalled by `t`.
+moe_status_t launch_mlp_bf16_tc_ep(const moe_config_t& c, int modes, const void* xr,
+                                   const int32_t* offsets, const int32_t* counts,
+                                   const void* w_gu, const void* w_d, void* h, void* y,
+                                   int64_t R_max, uint32_t* status, cudaStream_t s,
+                                   const EpTiles& t);
 
 // The shared expert alone, bf16 on tcgen05: h[T,F] = silu(x Wg^T) * (x Wu^T),
 // y[T,H] = h Wd^T for the T rows of x, with w_gu_sh [2F,H] and w_d_sh [H,F]

@@ -145,7 +145,8 @@ route_topk_kernel(const float* __restrict__ logits, const float* __restrict__ se
       topk_idx[(size_t)t * K + lane] = my_i;
       topk_w[(size_t)t * K + lane] = ex / sum;
       idx_s[tl * K + lane] = my_i;
-      atomicOr(&bitmap[my_i * WORDS + (tl >> 5)], 1u << (tl & 31));
+      if (MOE_CHECKED(my_i >= 0 && my_i < E && tl < tb))
+        atomicOr(&bitmap[my_i * WORDS + (tl >> 5)], 1u << (tl & 31));
     }
   }
   __syncthreads();
@@ -158,6 +159,7 @@ route_topk_kernel(const float* __restrict__ logits, const float* __restrict__ se
   }
   for (int i = threadIdx.x; i < ntok * K; i += blockDim.x) {
     const int tl = i / K;
+    MOE_CHECK(idx_s[i] >= 0 && idx_s[i] < E);
     const uint32_t* bm = bitmap + idx_s[i] * WORDS;
     const int w = tl >> 5;
     int r = __popc(bm[w] & ((1u << (tl & 31)) - 1u));

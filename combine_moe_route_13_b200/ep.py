@@ -43,10 +43,12 @@ class EpGroup:
     """This process's rank of a W-GPU expert-parallel layer (W = the process
     group's size). `device` is this rank's GPU (default: torch.cuda's current
     device). device_epoch: number the steps with the device-resident step
-    counter (epoch 0), so that a step can be captured in a CUDA graph."""
+    counter (epoch 0), so that a step can be captured in a CUDA graph.
+    flags: MOE_EP_TILE_SIGNAL [| MOE_EP_REMOTE_FIRST] for the tile-signalled
+    layer (the same on every rank)."""
 
     def __init__(self, cfg: B.MoeConfig, group=None, timeout_us: int = 0, device=None,
-                 device_epoch: bool = False):
+                 device_epoch: bool = False, flags: int = 0):
         import torch.distributed as dist
         self.cfg = cfg
         self.group = group
@@ -54,7 +56,8 @@ class EpGroup:
         self.rank = dist.get_rank(group)
         self.timeout_us = int(timeout_us)
         self.device_epoch = bool(device_epoch)
-        st = B.moe_ep_check(cfg, B.make_ep(self.world, self.rank, 1, self.timeout_us))
+        self.flags = int(flags)
+        st = B.moe_ep_check(cfg, B.make_ep(self.world, self.rank, 1, self.timeout_us, self.flags))
         if st != B.MOE_OK:
             raise B.MoeError(st, "EpGroup")
         self.device = (torch.device("cuda", torch.cuda.current_device()) if device is None
@@ -77,7 +80,7 @@ class EpGroup:
 
     def _ep(self) -> B.MoeEp:
         return B.make_ep(self.world, self.rank, 0 if self.device_epoch else self.epoch,
-                         self.timeout_us)
+                         self.timeout_us, self.flags)
 
     def forward(self, logits, x, w_gu_local, w_d_local, out, stream=None) -> B.MoeEpAux:
         """One step of this rank's layer (every rank calls it once per step)."""
@@ -107,15 +110,16 @@ class EpOnOneDevice:
     """W ranks on one device (see the module doc). device_epoch: number the
     steps with the ranks' device-resident step counters (epoch 0) instead of
     host-side step numbers, so that a step can be captured in a CUDA graph and
-    replayed."""
+    replayed. flags: MOE_EP_TILE_SIGNAL [| MOE_EP_REMOTE_FIRST]."""
 
     def __init__(self, cfg: B.MoeConfig, world: int, device="cuda", timeout_us: int = 0,
-                 device_epoch: bool = False):
+                 device_epoch: bool = False, flags: int = 0):
         self.cfg = cfg
         self.world = int(world)
         self.timeout_us = int(timeout_us)
         self.device_epoch = bool(device_epoch)
-        st = B.moe_ep_check(cfg, B.make_ep(self.world, 0, 1, self.timeout_us))
+        self.flags = int(flags)
+        st = B.moe_ep_check(cfg, B.make_ep(self.world, 0, 1, self.timeout_us, self.flags))
         if st != B.MOE_OK:
             raise B.MoeError(st, "EpOnOneDevice")
         nsym = B.moe_ep_symmetric_bytes(cfg, self.world)
@@ -132,7 +136,7 @@ class EpOnOneDevice:
 
     def ep(self, rank: int) -> B.MoeEp:
         return B.make_ep(self.world, rank, 0 if self.device_epoch else self.epoch,
-                         self.timeout_us)
+                         self.timeout_us, self.flags)
 
     def forward(self, logits: Sequence, x: Sequence, w_gu_local: Sequence, w_d_local: Sequence,
                 out: Sequence, stream=None):

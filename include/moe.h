@@ -139,6 +139,15 @@ moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Route: steps "top-K + weights", "histogram + capacity + overflow" and
  * "owner-aligned offsets + permutation".
+ * Defining passages: the pplx-kernels page, "Introductie" (each token's router
+ * distribution picks its top-K experts, whose outputs are averaged with the
+ * router's weights); the EFA page, "Диспетчеризация и комбинирование" (tokens
+ * per expert counted with shared-memory atomics inside a block, a cumulative
+ * sum turned into offsets, tokens packed contiguously per destination);
+ * "MoE Expert Parallel Benchmark", Step 2 (overflow = max(assigned - capacity,
+ * 0), effective tokens = sum of assigned - overflow); "Mixture-of-Experts
+ * acceleration through overlap" (the buffer ordered by owner, every tile
+ * inside one owner's rows).
  *   logits          [T,E] fp32, device, read only. Any bias is already added.
  *   topk_idx        [T,K] int32 out: experts by (logit descending, index ascending).
  *   topk_w          [T,K] fp32 out: softmax over the K selected logits.
@@ -204,7 +213,10 @@ moe_status_t moe_router_logits(const moe_config_t* cfg, const void* x, const voi
  *     return MOE_ERR_WORKSPACE and launch nothing.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) and caches it; make that first call before any
- *     stream capture on that device.
+ *     stream capture on that device. The cached address belongs to that
+ *     device's current context: after cudaDeviceReset (which unloads the
+ *     library's kernels and their array) it is stale, so do not call this
+ *     entry point again in a process that has reset the device.
  *   - Every call shares the one array, which keeps the last call's contents;
  *     the kernels write every scratch entry before reading it, so nothing needs
  *     to start at zero. Calls whose kernels overlap on the GPU (different
@@ -225,7 +237,11 @@ moe_status_t moe_route_topk_noalloc(const moe_config_t* cfg, const float* logits
 moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* token_slot,
                           void* xp, void* stream);
 
-/* Grouped SwiGLU expert MLP. For every expert e and every row r in
+/* Grouped SwiGLU expert MLP (the EFA page, "MoE all-to-all через EFA": the
+ * experts' grouped GEMM runs between dispatch and combine on the packed rows;
+ * the DistributedMoE README, "Результаты экспериментов": one grouped GEMM
+ * instead of many small per-expert GEMMs; the SwiGLU form of the expert is this
+ * library's reading, the pages give none). For every expert e and every row r in
  * [off_e, off_e + min(count_e, C)):
  *   h[r] = silu(xp[r] Wg_e^T) * (xp[r] Wu_e^T)   (fp32 accumulate, rounded to act)
  *   y[r] = h[r] W_d,e^T                          (fp32 accumulate, rounded to act)
@@ -276,7 +292,10 @@ moe_status_t moe_combine_wait(const moe_config_t* cfg, const void* y, const int3
                               uint32_t ready_target, void* out, uint32_t timeout_us, void* ws,
                               size_t ws_bytes, void* stream);
 
-/* The whole layer on `stream`: route -> dispatch -> expert MLP -> combine, with
+/* The whole layer on `stream`: route -> dispatch -> expert MLP -> combine (the
+ * cycle of the pplx-kernels page, "Introductie", "Dispatch" and "Combine", and
+ * of the EFA page, "MoE all-to-all через EFA": dispatch to the experts, the
+ * experts' grouped GEMM, combine back to token order by weighted average), with
  * every intermediate in the workspace (moe_workspace_bytes). `aux` may be NULL;
  * otherwise it receives the workspace pointers of the intermediates. No host
  * synchronisation: the per-expert counts stay on the device. With n_shared = 1 and
@@ -368,11 +387,22 @@ moe_status_t moe_layer_forward_fp8(const moe_config_t* cfg, const float* logits,
  * it to MOE_OK. Returns MOE_ERR_CUDA if the synchronisation or copy failed. */
 moe_status_t moe_get_device_status(void* ws, moe_status_t* status, void* stream);
 
+/* Debugging aid (no counterpart on the pages). In the bounds-checked build of
+ * the library (libmoe_check.so, compiled with -DMOE_CHECK_BOUNDS) every kernel
+ * checks its internal index invariants (decoded tiles, TMEM columns,
+ * shared-memory staging offsets, table indices); a failed check is counted
+ * and skips the access it guards instead of stopping the kernel. This call
+ * synchronises the device and returns the count and the source line of the
+ * first failure on the current device, then zeroes them when reset != 0. The
+ * release build returns MOE_ERR_UNSUPPORTED. */
+moe_status_t moe_debug_bounds_failures(uint32_t* failures, uint32_t* first_line, int32_t reset);
+
 /* Static text for a status code. */
 const char* moe_status_string(moe_status_t status);
 
 /* Library version as major*10000 + minor*100 + patch (1.1.0: the
- * expert-parallel entry points of moe_ep.h added). */
+ * expert-parallel entry points of moe_ep.h added; 1.2.0: their tile-signalled
+ * form, moe_ep_t.flags). */
 int32_t moe_version(void);
 
 #ifdef __cplusplus

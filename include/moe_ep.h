@@ -55,7 +55,8 @@
  * rows (moe_ep_recv_rows).
  *
  * Memory. Each rank allocates one symmetric region of moe_ep_symmetric_bytes
- * (counts table [W][E] int32, flags [3][W] uint32, xr [R_recv][H], y [R_recv][H])
+ * (counts table [W][E] int32, flags [3][W] uint32, ready counters
+ * [2][ceil(R_recv/128)] uint32, xr [R_recv][H], y [R_recv][H])
  * that its peers write into (counts, flags, xr) and read from (y), and a private
  * workspace of moe_ep_workspace_bytes (status word, route outputs, layout, h,
  * and with a shared expert its h and y for this rank's tokens).
@@ -84,9 +85,11 @@
  * Errors. Arguments: return codes as in moe.h. Every wait on a peer's flag is
  * bounded by timeout_us (0 = 2 s); one that runs out records MOE_ERR_TIMEOUT in
  * the status word (moe_get_device_status on the private workspace), and the
- * later waits then give up at once; the rank sends nothing more and raises no
- * flag, so its peers time out too instead of waiting. The outputs of such a
- * step are unspecified, and the group must be set up again
+ * later waits then give up at once; the rank writes nothing more into its
+ * peers' memory (no counts, rows or flags) and reads nothing more from it, so
+ * its peers time out too instead of waiting. Its combine then leaves `out`
+ * untouched (whatever the caller's buffer held before the step); its other
+ * outputs of such a step are unspecified, and the group must be set up again
  * (moe_ep_workspace_init, moe_ep_symmetric_init and a barrier on every rank)
  * before its next step. A row whose computed destination falls outside the
  * receive buffer is not written and records MOE_ERR_DEVICE_INPUT.
@@ -105,11 +108,36 @@
 extern "C" {
 #endif
 
+/* Tile signalling ("Mixture-of-Experts acceleration through overlap": a
+ * persistent GEMM that consumes rows as they arrive and publishes its output
+ * tiles through flags that the consumer polls; remote-first tile order).
+ * MOE_EP_TILE_SIGNAL (bf16, row_align % 128 == 0; else MOE_ERR_UNSUPPORTED):
+ *   - moe_ep_expert_mlp does not wait for every sender before its grouped
+ *     GEMM: each CTA of the gate/up GEMM waits, before it loads its 128 rows of
+ *     a tile, only for the DISPATCH flags of the senders whose rows those are
+ *     (inside a local expert the senders' blocks follow in rank order). Before
+ *     the down GEMM it waits for every sender (an owner overwrites y only after
+ *     every rank's combine of the previous step has read it), and the down GEMM
+ *     publishes each 128-row block of y through a ready counter in the
+ *     symmetric region (one more per stored 256-column tile, released at
+ *     system scope; two banks, by step parity).
+ *   - moe_ep_combine does not wait for every owner's Y flag first: a token is
+ *     combined as soon as the ready counters of its kept rows' blocks on their
+ *     owners reach ceil(H/256). The Y flags are waited for after the combine
+ *     (they still order the next step's writes into the peers).
+ *   Results are bit for bit those of the untagged layer.
+ * MOE_EP_REMOTE_FIRST (with MOE_EP_TILE_SIGNAL): the owner's GEMMs run the
+ *   tiles that hold other senders' rows first and the tiles holding only its
+ *   own rows last, so that the rows other ranks read are finished first. */
+#define MOE_EP_TILE_SIGNAL 1u
+#define MOE_EP_REMOTE_FIRST 2u
+
 typedef struct {
   int32_t world;        /* W ranks */
   int32_t rank;         /* this rank, 0 <= rank < W */
   uint32_t epoch;       /* step number (>= 1, the same on every rank), or 0: the device-resident step counter */
   uint32_t timeout_us;  /* bound of each wait on a peer's flag; 0 = 2 000 000 */
+  uint32_t flags;       /* MOE_EP_TILE_SIGNAL | MOE_EP_REMOTE_FIRST, or 0; the same on every rank */
 } moe_ep_t;
 
 /* Where the layer keeps its per-rank intermediates (host-side pointer values
@@ -127,6 +155,10 @@ typedef struct {
   void *h_shared, *y_shared;   /* [T][F], [T][H] (private): the shared expert on this rank's tokens; NULL without one */
   uint8_t *xq, *xs;        /* fp8 layer: codes [R_recv][H] and scales, inside xr's region (symmetric) */
   uint8_t *hq, *hs;        /* fp8 layer: codes [R_recv][F] and scales, inside h's region (private) */
+  int32_t *recv_split;     /* [E/W][W+1]: first row of sender s's block inside each local
+                              expert's rows, and [W] = the rows it received (private) */
+  uint32_t *y_ready;       /* [2][ceil(R_recv/128)]: ready counters of y's 128-row blocks,
+                              bank (step & 1) (symmetric; MOE_EP_TILE_SIGNAL) */
 } moe_ep_aux_t;
 
 /* R_recv (see above); -1 for an invalid config or world. */

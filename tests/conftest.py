@@ -19,3 +19,16 @@ def cuda_ok():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return True
+
+
+def pytest_sessionfinish(session, exitstatus):
+    # Under the bounds-checked library (MOE_LIBRARY=libmoe_check.so), write the
+    # device's bounds-check failure count and first failing line to the file
+    # MOE_BOUNDS_REPORT names (test_gpu_check_bounds.py reads it).
+    path = os.environ.get("MOE_BOUNDS_REPORT")
+    if not path:
+        return
+    import combine_moe_route_13_b200 as M
+    n, line = M.moe_debug_bounds_failures()
+    with open(path, "w") as f:
+        f.write(f"{n} {line}\n")

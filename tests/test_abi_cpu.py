@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_version():
-    assert M.moe_version() == 10100
+    assert M.moe_version() == 10200
 
 
 @pytest.mark.parametrize("name", list(W.WORKLOADS))

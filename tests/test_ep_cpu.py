@@ -63,14 +63,39 @@ def test_check(kw, world, rank, epoch, code):
     assert M.moe_ep_check(c, M.make_ep(world, rank, epoch)) == code
 
 
-def test_shared_expert_needs_bf16():
-    c = cfg_of("tiny", S=2, n_shared=1)   # fp32 activations
-    assert M.moe_ep_check(c, M.make_ep(2, 0, 1)) == M.MOE_ERR_UNSUPPORTED
+@pytest.mark.parametrize("kw,flags,code", [
+    (dict(), M.MOE_EP_TILE_SIGNAL, M.MOE_OK),
+    (dict(), M.MOE_EP_TILE_SIGNAL | M.MOE_EP_REMOTE_FIRST, M.MOE_OK),
+    (dict(n_shared=1), M.MOE_EP_TILE_SIGNAL, M.MOE_OK),
+    (dict(), M.MOE_EP_REMOTE_FIRST, M.MOE_ERR_INVALID_ARG),    # the order knob alone
+    (dict(), 4, M.MOE_ERR_INVALID_ARG),                        # an unknown flag
+    (dict(row_align=64), M.MOE_EP_TILE_SIGNAL, M.MOE_ERR_UNSUPPORTED),   # 128-row blocks
+])
+def test_check_tile_signal_flags(kw, flags, code):
+    # moe_ep.h: tile signalling needs bf16 and row_align % 128 == 0
+    c = cfg_of("mixtral", **kw)
+    assert M.moe_ep_check(c, M.make_ep(2, 0, 1, 0, flags)) == code
+
+
+def test_tile_signal_needs_bf16_and_not_fp8():
+    c = cfg_of("tiny", S=2, row_align=128)   # fp32 activations
+    assert M.moe_ep_check(c, M.make_ep(2, 0, 1, 0, M.MOE_EP_TILE_SIGNAL)) == M.MOE_ERR_UNSUPPORTED
+    c = cfg_of("mixtral")
+    ep = M.make_ep(2, 0, 1, 0, M.MOE_EP_TILE_SIGNAL)
+    fake = 1 << 40
+    got = M.LIB.moe_ep_dispatch_fp8(ctypes.byref(c), ctypes.byref(ep), fake, fake, fake, None,
+                                    1 << 40, None)
+    assert got == M.MOE_ERR_UNSUPPORTED
+
+
+def test_shared_expert_with_fp32_activations():
+    c = cfg_of("tiny", S=2, n_shared=1)   # fp32: the CUDA-core GEMM runs the shared expert
+    assert M.moe_ep_check(c, M.make_ep(2, 0, 1)) == M.MOE_OK
 
 
 @pytest.mark.parametrize("kw,code", [
     (dict(), M.MOE_OK),
-    (dict(n_shared=1), M.MOE_ERR_UNSUPPORTED),
+    (dict(n_shared=1), M.MOE_OK),               # each rank's shared expert in fp8
     (dict(H=4160), M.MOE_ERR_UNSUPPORTED),      # H % 256 != 0
     (dict(F=14400), M.MOE_ERR_UNSUPPORTED),     # F % 128 != 0
 ])
@@ -101,7 +126,7 @@ def _fields(struct):
 
 def test_structs_match_header():
     assert [n for n, _ in M.MoeEp._fields_] == _fields("moe_ep_t")
-    assert ctypes.sizeof(M.MoeEp) == 16
+    assert ctypes.sizeof(M.MoeEp) == 20
     assert [n for n, _ in M.MoeEpAux._fields_] == _fields("moe_ep_aux_t")
 
 
@@ -115,11 +140,13 @@ def test_aux_layout_is_inside_the_buffers():
     nsym = M.moe_ep_symmetric_bytes(c, world)
     nws = M.moe_ep_workspace_bytes(c, world)
     R = M.moe_ep_recv_rows(c, world)
-    for f in ("counts_all", "flags", "xr", "y"):
+    for f in ("counts_all", "flags", "y_ready", "xr", "y"):
         assert sym <= getattr(aux, f) < sym + nsym, f
+    # the ready counters (2 banks of ceil(R/128)) lie before xr, inside the zeroed head
+    assert aux.y_ready + 2 * ((R + 127) // 128) * 4 <= aux.xr
     assert aux.y + R * c.H * 2 <= sym + nsym
     for f in ("topk_idx", "expert_counts", "token_slot", "send_dst_row", "recv_offsets",
-              "recv_counts", "h"):
+              "recv_counts", "recv_split", "h"):
         v = getattr(aux, f)
         assert ws + 256 <= v < ws + nws and v % 256 == 0, f
     assert aux.h + R * c.F * 2 <= ws + nws

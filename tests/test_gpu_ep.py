@@ -95,6 +95,16 @@ def test_ep_layer_matches_oracle(cuda_ok, W, T, H, E, K, F, cf, A, act, bias):
     cfg = M.make_config(T=T, H=H, E=E, K=K, F=F, S=S, capacity=C, row_align=A, act=act)
     logits, xs, w_gu, w_d = make_case(W, T, H, E, K, F, act, seed=W * 1000 + T, bias=bias)
     emu, outs = run_ep(cfg, W, logits, xs, w_gu, w_d)
+    assert_ep_matches_oracle(emu, outs, logits, xs, w_gu, w_d, K, C, A, S, act, W)
+
+
+def assert_ep_matches_oracle(emu, outs, logits, xs, w_gu, w_d, K, C, A, S, act, W):
+    """Every rank of an emulated step against the expert-parallel oracle: route,
+    counts table and layout bit for bit, received rows bit for bit, y against
+    the oracle's SwiGLU of the GPU's own received rows, out against the
+    oracle's weighted sum of the GPU's own y rows, and the whole chain by
+    relative Frobenius error."""
+    E = w_gu.shape[0]
     for r in range(W):
         assert emu.status(r) == M.MOE_OK, f"rank {r}: {M.status_string(emu.status(r))}"
     np_act = act_np
@@ -165,6 +175,27 @@ def test_ep_equals_one_rank_layer_over_several_steps(cuda_ok, W, T, H, E, K, F, 
                 bad = np.argwhere(g != w)
                 raise AssertionError(f"step {step} rank {r}: {len(bad)} elements differ, "
                                      f"first {bad[:3].tolist()}")
+
+
+@pytest.mark.parametrize("W,T,H,E,K,F,cf,A", [
+    (2, 100, 128, 8, 2, 256, 1.25, 1),
+    (4, 90, 64, 8, 3, 96, 0.7, 4),
+])
+def test_ep_fp32_with_a_shared_expert(cuda_ok, W, T, H, E, K, F, cf, A):
+    # fp32: the shared expert runs on the CUDA-core grouped GEMM over the rank's
+    # own tokens; against the oracle and bit for bit the one-rank fp32 layer
+    C = O.capacity(T, K, E, cf)
+    cfg = M.make_config(T=T, H=H, E=E, K=K, F=F, S=W, capacity=C, row_align=A, act="f32",
+                        n_shared=1)
+    logits, xs, w_gu, w_d = make_case(W, T, H, E, K, F, "f32", seed=W * 13 + T, n_shared=1)
+    emu, outs = run_ep(cfg, W, logits, xs, w_gu, w_d)
+    ref_outs, _ = P.ep_layer_forward([l.numpy() for l in logits], [act_np(x) for x in xs],
+                                     act_np(w_gu), act_np(w_d), K, C, A, W, "f32", W, n_shared=1)
+    for r in range(W):
+        assert emu.status(r) == M.MOE_OK
+        assert_close_act(act_np(outs[r]), ref_outs[r], "f32", f"out rank {r}")
+        ref = one_rank_layer(cfg, logits[r], xs[r], w_gu, w_d)
+        assert torch.equal(outs[r], ref), f"rank {r}: {(outs[r] != ref).sum().item()} differ"
 
 
 def test_ep_layer_forward_one_rank(cuda_ok):
@@ -294,7 +325,9 @@ def test_a_rank_that_leaves_between_steps_times_the_others_out(cuda_ok):
     ep = emu.ep(0)
     logits, xs, w_gu, w_d = make_case(W, T, H, E, K, F, "bf16", seed=99)
     wg, wd = local_weights(w_gu, W, E, 0), local_weights(w_d, W, E, 0)
-    out = torch.zeros(T, H, dtype=torch.bfloat16, device=DEV)
+    # a sentinel the timed-out combine must leave in place (include/moe_ep.h:
+    # after a timeout the rank reads nothing from its peers and `out` is untouched)
+    out = torch.full((T, H), 7.0, dtype=torch.bfloat16, device=DEV)
     torch.cuda.synchronize()
     t0 = time.perf_counter()
     M.moe_ep_route(cfg, ep, logits[0].to(DEV), emu.sym[0], emu.peers, emu.ws[0])
@@ -303,8 +336,14 @@ def test_a_rank_that_leaves_between_steps_times_the_others_out(cuda_ok):
     M.moe_ep_combine(cfg, ep, emu.sym[0], emu.peers, out, emu.ws[0])
     torch.cuda.synchronize()
     assert time.perf_counter() - t0 < 5.0
+    # a further step of the timed-out rank (its status word still holds the
+    # timeout: reading it would reset it) publishes nothing into its peer
+    M.moe_ep_route(cfg, M.make_ep(W, 0, emu.epoch + 1, 5000),
+                   logits[0].to(DEV), emu.sym[0], emu.peers, emu.ws[0])
+    torch.cuda.synchronize()
     assert emu.status(0) == M.MOE_ERR_TIMEOUT
     assert emu.status(1) == M.MOE_OK
     f1 = emu.views(1)["flags"].cpu().numpy()
-    assert f1[0, 0] == emu.epoch          # rank 0's counts did arrive
+    assert f1[0, 0] == emu.epoch          # rank 0's counts of the timed-out step did arrive
     assert f1[1, 0] == emu.epoch - 1 and f1[2, 0] == emu.epoch - 1   # nothing after that
+    assert torch.all(out == 7.0)

@@ -8,7 +8,9 @@
   (moe_layer_forward_fp8) of its tokens over all E experts, which the fp8
   tests check against the fp8 oracle; and the whole chain within a relative
   Frobenius error of 1e-2 of the fp8 oracle's layer on two ranks;
-* at the Mixtral shape with two ranks, bit for bit the one-rank fp8 layer.
+* at the Mixtral shape with two ranks, bit for bit the one-rank fp8 layer;
+* with a shared expert (every rank applies it to its own tokens), bit for bit
+  the one-rank fp8 layer with the shared expert.
 """
 import numpy as np
 import pytest
@@ -38,18 +40,19 @@ def fp8_one_rank(cfg, logits, x, wq):
     return out
 
 
-def run_case(W, T, H, E, K, F, cf, seed, check_rows=True):
+def run_case(W, T, H, E, K, F, cf, seed, check_rows=True, n_shared=0):
     C = O.capacity(T, K, E, cf)
-    cfg = M.make_config(T=T, H=H, E=E, K=K, F=F, S=W, capacity=C, row_align=128, act="bf16")
+    cfg = M.make_config(T=T, H=H, E=E, K=K, F=F, S=W, capacity=C, row_align=128, act="bf16",
+                        n_shared=n_shared)
     g = torch.Generator().manual_seed(seed)
     logits = [torch.randn(T, E, generator=g).to(DEV) for _ in range(W)]
     xs = [torch.randn(T, H, generator=g).to(torch.bfloat16).to(DEV) for _ in range(W)]
-    w_gu = (torch.randn(E, 2 * F, H, generator=g) * 0.05).to(torch.bfloat16).to(DEV)
-    w_d = (torch.randn(E, H, F, generator=g) * 0.05).to(torch.bfloat16).to(DEV)
+    w_gu = (torch.randn(E + n_shared, 2 * F, H, generator=g) * 0.05).to(torch.bfloat16).to(DEV)
+    w_d = (torch.randn(E + n_shared, H, F, generator=g) * 0.05).to(torch.bfloat16).to(DEV)
     gq, gs = M.quantize_fp8(w_gu)
     dq, ds = M.quantize_fp8(w_d)
-    loc_gu = M.ep_local_fp8_weights(gq, gs, W, E, 2 * F, H)
-    loc_d = M.ep_local_fp8_weights(dq, ds, W, E, H, F)
+    loc_gu = M.ep_local_fp8_weights(gq, gs, W, E, 2 * F, H, n_shared)
+    loc_d = M.ep_local_fp8_weights(dq, ds, W, E, H, F, n_shared)
     wq = [loc_gu[r] + loc_d[r] for r in range(W)]
     emu = EpOnOneDevice(cfg, W, DEV)
     outs = [torch.full((T, H), float("nan"), dtype=torch.bfloat16, device=DEV) for _ in range(W)]
@@ -93,6 +96,16 @@ def run_case(W, T, H, E, K, F, cf, seed, check_rows=True):
 ])
 def test_ep_fp8_layer(cuda_ok, W, T, H, E, K, F, cf):
     run_case(W, T, H, E, K, F, cf, seed=W * 31 + T)
+
+
+@pytest.mark.parametrize("W,T,H,E,K,F,cf", [
+    (2, 256, 256, 8, 2, 256, 1.25),
+    (4, 300, 512, 16, 4, 384, 0.5),     # overflow: the shared expert still reaches every token
+])
+def test_ep_fp8_layer_with_a_shared_expert(cuda_ok, W, T, H, E, K, F, cf):
+    # every rank runs the shared expert on its own tokens, quantised with the
+    # dispatch's arithmetic: bit for bit the one-rank fp8 layer with a shared expert
+    run_case(W, T, H, E, K, F, cf, seed=W * 37 + T, n_shared=1)
 
 
 def test_ep_fp8_chain_against_the_fp8_oracle(cuda_ok):

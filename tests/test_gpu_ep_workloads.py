@@ -4,7 +4,12 @@ times): every rank's route bit for bit against the oracle, the exchanged
 counts and the layout bit for bit against the oracle's plan, sampled received
 rows bit for bit against the senders' token rows, and every rank's output
 bit for bit equal to the one-rank library layer over all E experts (which the
-one-rank tests check against the oracle)."""
+one-rank tests check against the oracle). Sampled tokens of every rank are
+also checked against the oracle directly, token by token: the owners' y rows
+of their kept assignments against the oracle's SwiGLU of the token row with
+that expert's weights, the token's output against the oracle's weighted sum
+of those GPU y rows, and against the oracle's own chain by relative Frobenius
+error (the tolerances of the one-rank layer tests)."""
 import numpy as np
 import pytest
 import torch
@@ -14,7 +19,7 @@ from combine_moe_route_13_b200.ep import EpOnOneDevice
 from oracle import moe_oracle as O
 from oracle import moe_oracle_ep as P
 import workloads as W
-from _gpu_common import act_np, assert_route_equal, host
+from _gpu_common import act_np, assert_close_act, assert_route_equal, host
 
 pytestmark = pytest.mark.gpu
 ROUTE_KEYS = ("topk_idx", "topk_w", "expert_counts", "overflow", "expert_offsets",
@@ -64,6 +69,45 @@ def test_workload_full_size_ep(cuda_ok, name, world):
                 e = int(r["topk_idx"][t, k])
                 row = int(send[e]) + int(r["token_slot"][t, k]) - int(r["expert_offsets"][e])
                 assert torch.equal(xr[row], inps[s]["x"][t]), (d, s, t, k)
+    # sampled tokens against the oracle, one token at a time
+    w_gu_h, w_d_h = {}, {}
+    for s in range(world):
+        r = routes[s]
+        toks = rng.choice(wl.T, 6, replace=False)
+        g_y, o_y, g_out, o_out, o_chain = [], [], [], [], []
+        for t in toks:
+            rows_gpu, rows_ref = [], []
+            for k in range(wl.K):
+                sl = int(r["token_slot"][t, k])
+                if sl < 0:
+                    continue
+                e = int(r["topk_idx"][t, k])
+                d = e // El
+                send = P.ep_plan(counts_all, C, wl.row_align, s)["send_dst_row"]
+                row = int(send[e]) + sl - int(r["expert_offsets"][e])
+                if e not in w_gu_h:
+                    w_gu_h[e], w_d_h[e] = act_np(full["w_gu"][e]), act_np(full["w_d"][e])
+                _, y_ref = O.expert_mlp_rows(act_np(inps[s]["x"][t:t + 1]), w_gu_h[e], w_d_h[e],
+                                             wl.act)
+                rows_gpu.append(act_np(emu.views(d)["y"][row:row + 1]))
+                rows_ref.append(y_ref)
+            slot1 = np.full((1, wl.K), -1, np.int32)
+            kept_k = [k for k in range(wl.K) if r["token_slot"][t, k] >= 0]
+            slot1[0, kept_k] = np.arange(len(kept_k))
+            w1 = r["topk_w"][t:t + 1]
+            ygpu = np.concatenate(rows_gpu) if rows_gpu else np.zeros((0, wl.H), np.uint16)
+            yref = np.concatenate(rows_ref) if rows_ref else np.zeros((0, wl.H), np.uint16)
+            g_y.append(ygpu)
+            o_y.append(yref)
+            g_out.append(act_np(outs[s][t:t + 1]))
+            o_out.append(O.combine(ygpu, slot1, w1, wl.act))
+            o_chain.append(O.combine(yref, slot1, w1, wl.act))
+        assert_close_act(np.concatenate(g_y), np.concatenate(o_y), wl.act, f"rank {s} y")
+        assert_close_act(np.concatenate(g_out), np.concatenate(o_out), wl.act, f"rank {s} out")
+        g = O.act_to_f64(np.concatenate(g_out), wl.act)
+        c = O.act_to_f64(np.concatenate(o_chain), wl.act)
+        fro = np.sqrt(np.sum((g - c) ** 2)) / max(np.sqrt(np.sum(c * c)), 1e-300)
+        assert fro <= 1e-2, f"rank {s}: whole chain relative Frobenius error {fro:.3e}"
     # every rank's output equals the one-rank layer of its tokens over all E experts
     ws = M.alloc_workspace(M.moe_workspace_bytes(cfg), dev)
     ref_out = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device=dev)

@@ -357,6 +357,35 @@ def test_round_trip_identity_experts(act, K, equal):
     assert out.dtype == x.dtype and np.array_equal(out, x)
 
 
+def bf16_nearest_bits(s: float) -> int:
+    """The bf16 value nearest to the float64 s (ties to the even significand),
+    by exact rational arithmetic: |s| = k * 2^(e-8) + r with 128 <= k < 256 (8
+    significant bits); normal range only, which the values here stay in."""
+    from fractions import Fraction
+    import math
+    if s == 0.0:
+        return 0x8000 if math.copysign(1.0, s) < 0 else 0
+    _, e = math.frexp(abs(s))                 # 2^(e-1) <= |s| < 2^e
+    q = Fraction(abs(s)) / Fraction(2) ** (e - 8)
+    k = math.floor(q)
+    rem = q - k
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and k % 2 == 1):
+        k += 1
+    v = math.ldexp(k, e - 8) * (1.0 if s > 0 else -1.0)
+    return int(np.array([v], dtype=np.float32).view(np.uint32)[0] >> 16)
+
+
+def test_bf16_nearest_bits_by_hand():
+    # 1 + 2^-8 lies halfway between 1 and 1 + 2^-7: ties to even -> 1.0 (0x3F80);
+    # 1 + 3*2^-8 lies halfway between 1 + 2^-7 and 1 + 2^-6 -> 1 + 2^-6 (0x3F82);
+    # just above the first halfway point rounds up (0x3F81)
+    assert bf16_nearest_bits(1.0 + 2 ** -8) == 0x3F80
+    assert bf16_nearest_bits(1.0 + 3 * 2 ** -8) == 0x3F82
+    assert bf16_nearest_bits(1.0 + 2 ** -8 + 2 ** -40) == 0x3F81
+    assert bf16_nearest_bits(-2.0) == 0xC000
+    assert bf16_nearest_bits(-0.0) == 0x8000
+
+
 @pytest.mark.parametrize("act", [O.ACT_F32, O.ACT_BF16])
 def test_combine_is_the_explicit_weighted_sum(act):
     T, K, H, R = 12, 3, 5, 40
@@ -376,8 +405,7 @@ def test_combine_is_the_explicit_weighted_sum(act):
             if act == O.ACT_F32:
                 assert out[t, j] == np.float32(s)
             else:
-                assert out[t, j] == bf16_bits_of(torch.tensor([s], dtype=torch.float64))[0] or \
-                    abs(O.bf16_bits_to_f64(out[t:t + 1, j])[0] - s) <= abs(s) * 2 ** -8
+                assert out[t, j] == bf16_nearest_bits(s), (t, j, s)
 
 
 # ----------------------------------------------------------------------------

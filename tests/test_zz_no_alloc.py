@@ -5,8 +5,12 @@ device array inside the library instead of a caller workspace.
 
 Checks, through the C ABI: two calls in a row (different inputs, so that the
 shared scratch is reused) give exactly what moe_route_topk gives with its own
-workspace, and a configuration needing more scratch than the array holds is
-refused without launching anything. This file is collected last on purpose.
+workspace and what the oracle's route gives (indices, counts, offsets and the
+permutation bit for bit, weights within the router-weight tolerance), for each
+of the three route block sizes (32, 64 and 128 tokens) and for a configuration
+whose scratch fills the array exactly; a configuration needing more scratch
+than the array holds is refused without launching anything. This file is
+collected last on purpose.
 """
 import numpy as np
 import pytest
@@ -36,8 +40,13 @@ def _route_both(cfg, logits):
             {k: v.cpu().numpy() for k, v in ref.items()})
 
 
-@pytest.mark.parametrize("T,E,K,S,cf,A", [(4096, 64, 6, 8, 1.0, 128), (32768, 384, 8, 16, 1.25, 128)])
-def test_noalloc_route_matches_workspace_route_twice(cuda_ok, T, E, K, S, cf, A):
+# route blocks of 32 tokens (T <= 9472), 64 (T <= 18944) and 128 (above); the
+# last case needs ceil(32768/128) * 1024 * 4 B = 1 MiB: the array exactly
+@pytest.mark.parametrize("T,E,K,S,cf,A", [(4096, 64, 6, 8, 1.0, 128),
+                                          (16384, 64, 6, 8, 1.0, 128),
+                                          (32768, 384, 8, 16, 1.25, 128),
+                                          (32768, 1024, 8, 16, 1.25, 128)])
+def test_noalloc_route_matches_workspace_route_and_oracle_twice(cuda_ok, T, E, K, S, cf, A):
     C = O.capacity(T, K, E, cf)
     cfg = M.make_config(T, 64, E, K, 64, S, C, A, "bf16")
     R = M.moe_max_rows(cfg)
@@ -48,6 +57,10 @@ def test_noalloc_route_matches_workspace_route_twice(cuda_ok, T, E, K, S, cf, A)
         got, ref = _route_both(cfg, lg.cuda())
         assert_route_equal(got, ref, R)
         assert np.array_equal(got["topk_w"], ref["topk_w"])
+        # and the oracle's route of the same logits (weights: fp32 exp vs float64)
+        o = O.route(lg.numpy(), K, C, A, S)
+        assert o["R_max"] == R
+        assert_route_equal(got, o, R)
 
 
 def test_noalloc_route_refuses_configs_beyond_its_scratch(cuda_ok):
