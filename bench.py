@@ -16,14 +16,14 @@ synchronisation bracket the timed region; with several ranks every rank runs
 its own replica of the layer on its own tokens (weak scaling, no data-path
 collective) and the time is the maximum over ranks.
 
-Inside the same clock-sampled region, right after the fused steps, the same
-number of steps runs through the four piecewise entry points with events
-between them: route, dispatch, expert MLP and combine. Their median times
-give the per-kernel GB/s and `roofline` (the expert MLP: the grouped GEMMs,
-the dominant cost), taken at the clocks the fused steps ran at. The peak is
-the measured burst bf16 rate unless the region was at least a second of
-load with the power cap active, then the measured sustained rate; both
-fractions are printed.
+Every timed fused step is followed by one step through the four piecewise
+entry points with events between them (route, dispatch, expert MLP, combine),
+alternating inside the same clock-sampled region, so that both see the same
+clocks and power budget. The piecewise medians give the per-kernel GB/s and
+`roofline` (the expert MLP: the grouped GEMMs, the dominant cost). The peak
+is the measured burst bf16 rate unless the region held a second of load at
+the power cap with the SM clock held below 90% of its maximum, then the
+measured sustained rate; both fractions are printed.
 
 `e2e` repeats the measurement through the same C ABI call with the step's
 inputs copied from pinned host memory and the output copied back inside the
@@ -257,10 +257,8 @@ def time_steps(fn, steps, warmup, flush_buf, stream):
     return [a.elapsed_time(b) for a, b in evs]
 
 
-def phase_times(layer: Layer, steps, flush_buf, stream):
-    """Per-phase device times (ms, one list per phase over `steps` steps)
-    through the piecewise entry points, and the per-step totals (first pass
-    untimed, a warm-up)."""
+def piecewise_calls(layer: Layer):
+    """The step through the piecewise entry points: (names, calls)."""
     M = layer.M
     v = layer.views()
     cfg, inp = layer.cfg, layer.inp
@@ -287,27 +285,49 @@ def phase_times(layer: Layer, steps, flush_buf, stream):
                                   inp["w_gu"], inp["w_d"], v["h"], v["y"], layer.ws)),
         lambda: M.moe_combine(cfg, v["y"], v["token_slot"], v["topk_w"], layer.out),
     )
-    acc = {n: [] for n in names}
-    totals = []
+    return names, calls
+
+
+def time_interleaved(layer: Layer, steps, warmup, flush_buf, stream):
+    """Fused steps (the headline) and piecewise steps (the per-kernel split),
+    alternating, so that both run under the same clocks and power budget:
+    each iteration flushes L2 and times one moe_layer_forward, then flushes
+    again and times the piecewise entry points with an event after each.
+    Returns (fused step times, {phase: times}, piecewise step times), in ms."""
+    names, calls = piecewise_calls(layer)
     nvtx = torch.cuda.nvtx   # host ranges per phase, for nsys-style timelines
-    for it in range(steps + 1):
-        # a longer idle wait than the whole-step timing's: the piecewise calls
-        # cost more host time, and every phase must already be queued when the
-        # GPU reaches it, or its time would include the host's
-        flush_l2(flush_buf, 4_000_000)
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
+
+    def piecewise(ev):
         ev[0].record(stream)
         for i, c in enumerate(calls):
             nvtx.range_push(names[i])
             c()
             nvtx.range_pop()
             ev[i + 1].record(stream)
-        torch.cuda.synchronize()
-        if it:   # the first pass is a warm-up
-            for i, n in enumerate(names):
-                acc[n].append(ev[i].elapsed_time(ev[i + 1]))
-            totals.append(ev[0].elapsed_time(ev[-1]))
-    return acc, totals
+
+    def events(n):
+        return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+    for _ in range(warmup):
+        flush_l2(flush_buf)
+        layer.forward()
+        flush_l2(flush_buf)
+        piecewise(events(len(calls) + 1))
+    torch.cuda.synchronize()
+    fused = [events(2) for _ in range(steps)]
+    pieces = [events(len(calls) + 1) for _ in range(steps)]
+    for i in range(steps):
+        flush_l2(flush_buf)
+        fused[i][0].record(stream)
+        layer.forward()
+        fused[i][1].record(stream)
+        flush_l2(flush_buf)
+        piecewise(pieces[i])
+    torch.cuda.synchronize()
+    times = [a.elapsed_time(b) for a, b in fused]
+    acc = {n: [ev[k].elapsed_time(ev[k + 1]) for ev in pieces] for k, n in enumerate(names)}
+    totals = [ev[0].elapsed_time(ev[-1]) for ev in pieces]
+    return times, acc, totals
 
 
 def e2e_steps(layer: Layer, steps, warmup, flush_buf, stream):
@@ -752,10 +772,13 @@ def run_ep_emulated(args, wl: W.Workload, world_ep: int):
 
 def choose_peak(peaks, clk, region_s, fp8: bool):
     """The tensor peak the expert MLP is measured against: the measured burst
-    bf16 rate, or the measured sustained rate when the timed region held at
-    least a second of load and the clock record shows the power cap. fp8: 2x
-    (the nominal dense fp8/bf16 ratio, 4.5 / 2.25 PFLOP/s)."""
-    capped = bool(clk) and "sw_power_cap" in clk.get("reasons", [])
+    bf16 rate, or the measured sustained rate (taken under the 1000 W power
+    cap) when the timed region held at least a second of load, the clock
+    record shows the power cap, and the median SM clock under load sat below
+    90% of the maximum: the conditions the sustained rate was measured in.
+    fp8: 2x (the nominal dense fp8/bf16 ratio, 4.5 / 2.25 PFLOP/s)."""
+    capped = bool(clk) and "sw_power_cap" in clk.get("reasons", []) and \
+        clk.get("sm_mhz", 0) < 0.9 * clk.get("sm_max_mhz", 1e9)
     sustained = capped and region_s >= 1.0 and "bf16_tflops_sustained" in peaks
     mult = 2.0 if fp8 else 1.0
     burst = peaks["bf16_tflops"] * mult
@@ -841,8 +864,8 @@ def main(argv=None):
     clocks = Clocks(device.index if device.index is not None else 0)
     barrier()
     clocks.start()
-    times = time_steps(layer.forward, args.steps, args.warmup, flush_buf, stream)
-    ph_lists, ph_totals = phase_times(layer, args.steps, flush_buf, stream)
+    times, ph_lists, ph_totals = time_interleaved(layer, args.steps, args.warmup, flush_buf,
+                                                  stream)
     barrier()
     clk = clocks.stop()
     ms = max_over_ranks(float(np.median(times)), world, device)
@@ -872,10 +895,10 @@ def main(argv=None):
     kernels = {
         "router_us": ph["router"] * 1e3 if args.router else None,
         "phase_timing": "median over the timed steps of CUDA events between the piecewise "
-                        "entry points on the launching stream, run right after the fused "
-                        "steps inside the same clock-sampled region, L2 flushed before every "
-                        "step; each phase includes its launch gap (kernel-only ncu times: "
-                        "profiles/)",
+                        "entry points on the launching stream; each timed step is one fused "
+                        "step then one piecewise step, alternating inside the same "
+                        "clock-sampled region, L2 flushed before each; each phase includes "
+                        "its launch gap (kernel-only ncu times: profiles/)",
         "piecewise_step_ms": ph_step,
         "route_us": ph["route"] * 1e3,
         "route_gbs": alg["route_bytes"] / (ph["route"] * 1e-3) / 1e9,
