@@ -7,11 +7,14 @@
 // is read once as bf16, quantised once, and its codes and scales written to
 // each of its kept rows.
 //
-// Blocks of 128 threads stride over the source rows. Thread t handles the 16-byte
-// vector v = v0 + t (8 bf16); the 16 threads of a half-warp cover one
-// 128-element scale block, whose amax is a 4-step xor-shuffle reduction inside
-// the half-warp. Codes leave as 8-byte stores (coalesced, 1 KB per block
-// iteration); the half-warp's first thread stores the block's scale byte.
+// Blocks of 128 threads stride over the source rows. Thread t handles 16
+// consecutive values (two 16-byte vectors of bf16, both loaded before either is
+// used); the 8 threads of a warp's eighth cover one 128-element scale block,
+// whose amax is a 3-step xor-shuffle reduction, and a warp covers four scale
+// blocks: the four scale bytes a row's 512-value chunk owns are adjacent in the
+// blocked layout (one UE8M0 byte per 32-k part of the MMA, see fp8_util.cuh),
+// so lane 0 gathers them and stores one 4-byte word. Codes leave as 16-byte
+// stores (2 KB per block iteration and destination).
 #include <algorithm>
 
 #include "fp8_util.cuh"
@@ -44,51 +47,71 @@ quant_rows_kernel(const uint4* __restrict__ src, int64_t rows, int row_vecs, int
   pdl_wait();
   pdl_trigger();
   const int64_t H = (int64_t)row_vecs * 8;
+  const int lane = threadIdx.x & 31;
   for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
     if (DISPATCH) {
       __syncthreads();   // the previous row's readers of s_dst and s_n are done
-      if (threadIdx.x == 0) {
-        int n = 0;
-        for (int k = 0; k < K; ++k) {
-          const int s = token_slot[row * K + k];
-          if (s >= 0 && s < slot_end) s_dst[n++] = s;   // others are dropped
+      if (threadIdx.x < 32) {   // warp 0 packs the kept destinations, k order
+        int s = -1;
+        if (lane < K) s = token_slot[row * K + lane];
+        const bool keep = s >= 0 && s < slot_end;   // others are dropped
+        const unsigned m = __ballot_sync(0xffffffffu, keep);
+        if (keep) s_dst[__popc(m & ((1u << lane) - 1u))] = s;
+        if (lane == 0) {
+          int n = __popc(m);
+          if (sh_row0 >= 0) s_dst[n++] = (int)(sh_row0 + row);   // the shared expert's row
+          s_n = n;
         }
-        if (sh_row0 >= 0) s_dst[n++] = (int)(sh_row0 + row);   // the shared expert's row
-        s_n = n;
       }
       __syncthreads();
       if (s_n == 0) continue;   // every assignment of this token overflowed
     }
     const int nd = DISPATCH ? s_n : 1;
     const uint4* x = src + row * row_vecs;
-    // row_vecs is a multiple of 16 and v0 of 128: a half-warp is all valid or all not
-    for (int v0 = 0; v0 < row_vecs; v0 += QT) {
-      const int v = v0 + (int)threadIdx.x;
+    // 16 values (two vectors) per thread, 2048 per block iteration; H is a
+    // multiple of 128, so an 8-thread scale block is all valid or all not
+    for (int v0 = 0; v0 < row_vecs; v0 += 2 * QT) {
+      const int v = v0 + 2 * (int)threadIdx.x;   // this thread's first vector
       const bool valid = v < row_vecs;
-      float f[8];
+      float f[16];
       if (valid) {
-        bf16x8_to_float(__ldcs(x + v), f);
+        const uint4 a = __ldcs(x + v), b = __ldcs(x + v + 1);
+        float fa[8], fb[8];
+        bf16x8_to_float(a, fa);
+        bf16x8_to_float(b, fb);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          f[i] = fa[i];
+          f[8 + i] = fb[i];
+        }
       } else {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) f[i] = 0.f;
+        for (int i = 0; i < 16; ++i) f[i] = 0.f;
       }
       float amax = 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+      for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
 #pragma unroll
-      for (int o = 1; o < 16; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      if (!valid) continue;
+      for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
       const int p = fp8_scale_exp(amax);
       const float inv = fp8_inv_scale(p);
-      uint2 c;
+      uint4 c;
       c.x = fp8x2(f[0] * inv, f[1] * inv) | (fp8x2(f[2] * inv, f[3] * inv) << 16);
       c.y = fp8x2(f[4] * inv, f[5] * inv) | (fp8x2(f[6] * inv, f[7] * inv) << 16);
-      const uint8_t sbyte = (uint8_t)(p + 127);
-      const int kb = v / 16;
+      c.z = fp8x2(f[8] * inv, f[9] * inv) | (fp8x2(f[10] * inv, f[11] * inv) << 16);
+      c.w = fp8x2(f[12] * inv, f[13] * inv) | (fp8x2(f[14] * inv, f[15] * inv) << 16);
+      // the warp's four scale bytes (scale blocks kb0 .. kb0+3) into one word
+      const uint32_t sb = (uint32_t)(p + 127);
+      const uint32_t word = __shfl_sync(0xffffffffu, sb, 0) | (__shfl_sync(0xffffffffu, sb, 8) << 8) |
+                            (__shfl_sync(0xffffffffu, sb, 16) << 16) |
+                            (__shfl_sync(0xffffffffu, sb, 24) << 24);
+      const int kb0 = (v - 2 * lane) / 16;   // the warp's first scale block
       for (int d = 0; d < nd; ++d) {
         const int64_t r = DISPATCH ? (int64_t)s_dst[d] : row;
-        *reinterpret_cast<uint2*>(q + r * H + (int64_t)v * 8) = c;
-        if ((threadIdx.x & 15) == 0) sf[sf_offset(r, kb, KB)] = sbyte;
+        if (valid) *reinterpret_cast<uint4*>(q + r * H + (int64_t)v * 8) = c;
+        // a warp's first scale block is valid whenever any of its lanes is
+        if (lane == 0 && kb0 < KB && MOE_CHECKED(kb0 % 4 == 0))
+          *reinterpret_cast<uint32_t*>(sf + sf_offset(r, kb0, KB)) = word;
       }
     }
   }

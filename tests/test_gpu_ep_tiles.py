@@ -57,6 +57,8 @@ CASES = [
     (2, 700, 256, 8, 3, 256, 0.8, 1),    # overflow, a shared expert
     (8, 128, 256, 64, 8, 128, 1.5, 0),   # eight senders inside one pair tile
     (8, 64, 256, 64, 8, 128, 1.5, 0),    # small experts: 128-row one-CTA tiles
+    (2, 0, 256, 8, 2, 256, 1.25, 0),     # empty batch on every rank
+    (2, 200, 256, 8, 2, 256, 0.0, 0),    # C = 0: every assignment dropped
 ]
 
 
