@@ -244,6 +244,14 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   // drains wait for copies and MMAs already issued even after an abort (bounded
   // by DRAIN_NS): shared memory and TMEM must not be released under them
   volatile int no_abort = 0;
+  // With arrival waits (tile-signalled gate/up) one CTA of a pair may hold its
+  // loads back for as long as a sender is late (up to ept.wait_ns), and every
+  // other wait of the pair (the leader's MMA on the stage barriers, the
+  // epilogues, the leader's final drain of stage barriers that count the peer's
+  // copies) must outlast that.
+  const bool arrivals = MODE == 0 && ept.arrive != nullptr;
+  const unsigned long long wait_ns =
+      arrivals ? (ept.wait_ns + DRAIN_NS > WAIT_NS ? ept.wait_ns + DRAIN_NS : WAIT_NS) : WAIT_NS;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -376,7 +384,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!wait_phase(saddr(&ctl->empty[s]), ph ^ 1u, abort_flag, status, WAIT_NS)) {
+          if (!wait_phase(saddr(&ctl->empty[s]), ph ^ 1u, abort_flag, status, wait_ns)) {
             ok = false;
             break;
           }
@@ -397,11 +405,17 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       }
       (void)seen;
       // the copies of the last STAGES stages must land before the CTA exits
-      // (the leader's barriers also count the peer's copies)
+      // (the leader's barriers also count the peer's copies, which a pair CTA
+      // waiting for a late sender issues only then: with arrival waits the
+      // drain allows for that, unless the pair has aborted, when only this
+      // CTA's own copies, already issued, are left to land)
       if (leader)
-        for (int i = max(0, it - STAGES); i < it; ++i)
-          wait_phase(saddr(&ctl->full[i % STAGES]), (uint32_t)(i / STAGES) & 1u, &no_abort,
-                     status, DRAIN_NS);
+        for (int i = max(0, it - STAGES); i < it; ++i) {
+          const uint32_t fb = saddr(&ctl->full[i % STAGES]);
+          const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
+          if (!arrivals || !wait_phase(fb, ph, abort_flag, status, wait_ns))
+            wait_phase(fb, ph, &no_abort, status, DRAIN_NS);
+        }
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {  // ---------------------------------------- MMA issuer
@@ -409,7 +423,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       for (int tile = cluster_id; tile < total; tile += n_clusters, ++tcount) {
         const int b = tcount & 1;
         const uint32_t tph = (uint32_t)(tcount >> 1) & 1u;
-        if (!wait_phase(saddr(&ctl->tempty[b]), tph ^ 1u, abort_flag, status, WAIT_NS)) break;
+        if (!wait_phase(saddr(&ctl->tempty[b]), tph ^ 1u, abort_flag, status, wait_ns)) break;
         tc_fence_after();
         MOE_CHECK(b * UMMA_N + UMMA_N <= (int)TMEM_COLS);
         const uint32_t d = tmem + (uint32_t)(b * UMMA_N);
@@ -417,7 +431,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!wait_phase(saddr(&ctl->full[s]), ph, abort_flag, status, WAIT_NS)) {
+          if (!wait_phase(saddr(&ctl->full[s]), ph, abort_flag, status, wait_ns)) {
             ok = false;
             break;
           }
@@ -455,7 +469,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       const int b = tcount & 1;
       const uint32_t tph = (uint32_t)(tcount >> 1) & 1u;
       int ok = 1;
-      if (lane == 0) ok = wait_phase(saddr(&ctl->tfull[b]), tph, abort_flag, status, WAIT_NS);
+      if (lane == 0) ok = wait_phase(saddr(&ctl->tfull[b]), tph, abort_flag, status, wait_ns);
       __syncwarp();
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;

@@ -11,9 +11,10 @@ W ranks emulated on one device:
   block of y that holds rows, 0 elsewhere;
 * a sender that never dispatches: the owner's gate/up GEMM gives up within its
   bound with MOE_ERR_TIMEOUT (no hang), and the device stays usable;
-* a sender that is late: its DISPATCH flag is set from the host while the
-  owner's GEMM already runs and waits for it; the GEMM then finishes and the
-  layer is bit for bit the one-rank layer.
+* a sender that is late: its DISPATCH flag is set from the host (a copy on
+  another stream) 0.3 s after the owner's GEMM started waiting for it; the
+  GEMM (whose pair CTAs, epilogues and final drain all outlast the wait)
+  then finishes and the layer is bit for bit the one-rank layer.
 """
 import time
 
@@ -154,12 +155,12 @@ def test_owner_gemm_waits_for_a_late_sender(cuda_ok):
         M.moe_ep_expert_mlp(cfg, emu.ep(0), None, wg[0], wd[0], emu.sym[0], emu.peers,
                             emu.ws[0])
         end.record()
-    time.sleep(0.2)                               # the GEMM is running and waiting
+    time.sleep(0.3)                               # the GEMM is running and waiting
     with torch.cuda.stream(s_copy):               # a copy engine raises the flag
         flag.copy_(late, non_blocking=True)
     torch.cuda.synchronize()
     assert emu.status(0) == M.MOE_OK
-    assert start.elapsed_time(end) >= 100.0       # it did wait for the late sender
+    assert start.elapsed_time(end) >= 250.0       # it did wait for the late sender
     with torch.cuda.stream(s_gemm):
         M.moe_ep_expert_mlp(cfg, emu.ep(1), None, wg[1], wd[1], emu.sym[1], emu.peers,
                             emu.ws[1])
