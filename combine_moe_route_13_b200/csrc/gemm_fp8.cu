@@ -57,9 +57,21 @@ constexpr int BK = 128;                         // k per stage (bytes of a swizz
 constexpr int UMMA_N = 256;
 constexpr int A_BYTES = BM * BK;                // 16 KB
 constexpr int B_HALF = 128 * BK;                // 16 KB
-constexpr int OPER_BYTES = A_BYTES + 2 * B_HALF;
 constexpr int SF_STAGE = 3 * SF_CHUNK;          // A, B rows 0-127, B rows 128-255
-constexpr int STAGES = 4;
+constexpr int MAX_STAGES = 6;
+// CG = 1: one CTA per tile of 128 rows, loading A and both halves of B (four
+// stages of 48 KB). CG = 2: a pair of CTAs on two SMs shares one
+// tcgen05.mma.cta_group::2 of M = 256; each CTA loads its own 128 rows of A
+// and its own half of B (32 KB per stage, six stages: half the operand bytes
+// per k step and CTA, 1.5x the k steps of lookahead in the same shared
+// memory), and the scale chunks of its A rows and of all 256 B rows (every
+// CTA's TMEM holds the full B scales, as the one-CTA M = 128 MMA does).
+template <int CG>
+struct F8 {
+  static constexpr int STAGES = CG == 2 ? 6 : 4;
+  static constexpr int OPER_BYTES = A_BYTES + (CG == 2 ? 1 : 2) * B_HALF;
+  static constexpr int TILE_ROWS = BM * CG;
+};
 // Threads: warp 0 TMA, warp 1 MMA, then the epilogue warps: eight for gate/up
 // (two per TMEM lane quarter, each taking half of the tile's columns, so that
 // a thread holds its 64 gate and 64 up accumulators in registers and TMEM is
@@ -76,8 +88,8 @@ constexpr unsigned long long WAIT_NS = 2000000000ull;
 constexpr unsigned long long DRAIN_NS = 200000000ull;
 
 struct Ctl {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[MAX_STAGES];
+  uint64_t empty[MAX_STAGES];
   uint64_t tfull, tempty, drain;
   uint32_t tmem_base;
   int abort;
@@ -85,18 +97,20 @@ struct Ctl {
   float amax[2][2][128];   // gate/up: [tile parity][column half][row] partial amax of h
 };
 
+template <int CG>
 size_t smem_bytes(int E) {
-  return 1024 + (size_t)STAGES * (OPER_BYTES + SF_STAGE) + STAGING_BYTES + sizeof(Ctl) +
-         (size_t)(3 * E + 2) * 4;
+  return 1024 + (size_t)F8<CG>::STAGES * (F8<CG>::OPER_BYTES + SF_STAGE) + STAGING_BYTES +
+         sizeof(Ctl) + (size_t)(3 * E + 2) * 4;
 }
 
 // Instruction descriptor of tcgen05.mma.kind::mxf8f6f4.block_scale: B scale
 // byte j (bits 4-5), A and B e4m3 (format 0 at bits 7-9, 10-12), both
 // K-major, N >> 3 at bits 17-22, UE8M0 scales (bit 23), M >> 4 at bits 24-28,
 // A scale byte j (bits 29-30), dense K = 32 (bit 31 = 0).
+template <int CG>
 __host__ __device__ constexpr uint32_t idesc_fp8(uint32_t j) {
-  return (j << 4) | ((uint32_t)(UMMA_N >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24) |
-         (j << 29);
+  return (j << 4) | ((uint32_t)(UMMA_N >> 3) << 17) | (1u << 23) |
+         ((uint32_t)((BM * CG) >> 4) << 24) | (j << 29);
 }
 
 // Global -> shared bulk copy (no tensor map), completion counted on `bar`.
@@ -121,21 +135,37 @@ __device__ __forceinline__ uint64_t sf_desc(uint32_t a) {
 }
 
 // 32 rows x 128 bits of shared memory into 4 TMEM columns, the same rows in
-// each of the four 32-lane quarters.
+// each of the four 32-lane quarters. CG = 2 (issued by the pair's first CTA):
+// each CTA's chunk at that shared-memory address into its own TMEM.
+template <int CG>
 __device__ __forceinline__ void sf_copy(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-               : "memory");
+  if (CG == 2)
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+                 : "memory");
+  else
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+                 : "memory");
 }
 
+template <int CG>
 __device__ __forceinline__ void mma_fp8(uint32_t d, uint64_t ad, uint64_t bd, uint32_t idesc,
                                         uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::
-          "r"(d),
-      "l"(ad), "l"(bd), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
-      : "memory");
+  if (CG == 2)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::
+            "r"(d),
+        "l"(ad), "l"(bd), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::
+            "r"(d),
+        "l"(ad), "l"(bd), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
 }
 
 __device__ __forceinline__ float silu_mul(uint32_t g_bits, uint32_t u_bits) {
@@ -182,15 +212,23 @@ __device__ __forceinline__ void epi_bar() {
   asm volatile("bar.sync 1, %0;" ::"n"(32 * epi_warps<MODE>()) : "memory");
 }
 
-template <int MODE>
+// Scale chunks (512 bytes: 128 rows x four k blocks) by tensor map (CG = 2):
+// the scale buffer seen as [chunks][128] uint32, one chunk per box, so that
+// both CTAs' copies count on the pair's first CTA's barrier like the
+// operands (tmSFA, tmSFB); CG = 1 uses plain bulk copies from sfa / sfb.
+template <int MODE, int CG>
 __global__ void __launch_bounds__(num_threads<MODE>(), 1)
 fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const __grid_constant__ CUtensorMap tmOut, const uint8_t* __restrict__ sfa,
+                 const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ CUtensorMap tmSFA,
+                 const __grid_constant__ CUtensorMap tmSFB, const uint8_t* __restrict__ sfa,
                  const uint8_t* __restrict__ sfb, void* __restrict__ out_v,
                  uint8_t* __restrict__ out_sf, int N_out, int Kdim, int b_rows_per_expert,
                  int b_second_off, const int32_t* __restrict__ offsets,
                  const int32_t* __restrict__ counts, int E, int C, long long R_max,
                  uint32_t* __restrict__ status, int sh_rows, int sh_row0) {
+  using CF = F8<CG>;
+  constexpr int STAGES = CF::STAGES;
+  constexpr int OPER_BYTES = CF::OPER_BYTES;
   constexpr int BN_OUT = (MODE == 0) ? 128 : 256;   // output columns per tile
   constexpr int NUM_THREADS = num_threads<MODE>();
   constexpr int EPI_WARPS = epi_warps<MODE>();
@@ -209,6 +247,9 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   int* kept_s = row_off + (G + 1);            // [G]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;   // position in the pair
+  const bool leader = rank == 0;
+  const int cta_group = blockIdx.x / CG, n_groups = gridDim.x / CG;
   const int NT = (N_out + BN_OUT - 1) / BN_OUT;
   const int KB = Kdim / BK;
   const int KG = (KB + 3) / 4;   // k groups (scale chunks per row block)
@@ -223,17 +264,21 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       mbar_init(saddr(&ctl->empty[s]), 1);
     }
     mbar_init(saddr(&ctl->tfull), 1);
-    mbar_init(saddr(&ctl->tempty), EPI_WARPS);
+    mbar_init(saddr(&ctl->tempty), EPI_WARPS * CG);   // both CTAs' epilogues (on the first)
     mbar_init(saddr(&ctl->drain), 1);
     ctl->abort = 0;
     fence_mbar_init();
     prefetch_map(&tmA);
     prefetch_map(&tmB);
     prefetch_map(&tmOut);
+    if (CG == 2) {
+      prefetch_map(&tmSFA);
+      prefetch_map(&tmSFB);
+    }
   }
   if (warp == 1) {
-    tmem_alloc<1>(saddr(&ctl->tmem_base), TMEM_COLS);
-    tmem_relinquish<1>();
+    tmem_alloc<CG>(saddr(&ctl->tmem_base), TMEM_COLS);
+    tmem_relinquish<CG>();
   }
   pdl_wait();
   pdl_trigger();
@@ -254,7 +299,7 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
         kept_s[e] = k;
         row_off[e] = off;
-        local += (k + BM - 1) / BM;
+        local += (k + CF::TILE_ROWS - 1) / CF::TILE_ROWS;
       }
     }
     int incl = local;
@@ -271,7 +316,7 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const int e = e0 + i;
       if (e < G) {
         P[e] = run;
-        run += (kept_s[e] + BM - 1) / BM;
+        run += (kept_s[e] + CF::TILE_ROWS - 1) / CF::TILE_ROWS;
       }
     }
     if (threadIdx.x == NUM_THREADS - 1) {
@@ -281,6 +326,7 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   }
   tc_fence_before();
   __syncthreads();
+  if (CG == 2) cluster_sync();   // both CTAs' barriers exist before anyone signals them
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
   const int total = P[G] * NT;
@@ -288,11 +334,13 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   if (warp == 0) {
     if (lane == 0) {  // ------------------------------------------------ TMA producer
       int it = 0;
-      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      for (int tile = cta_group; tile < total; tile += n_groups) {
         int m, n;
         const int e = decode_tile(tile, NT, P, G, m, n);
-        MOE_CHECK(e >= 0 && e < G && n >= 0 && n < NT && m >= 0 && m * BM < max(kept_s[e], 1));
-        const int a_row = row_off[e] + m * BM;           // a multiple of 128
+        MOE_CHECK(e >= 0 && e < G && n >= 0 && n < NT && m >= 0 &&
+                  m * CF::TILE_ROWS < max(kept_s[e], 1));
+        // this CTA's 128 rows of A (a multiple of 128)
+        const int a_row = row_off[e] + m * CF::TILE_ROWS + (int)rank * BM;
         const int b_row0 = e * b_rows_per_expert + n * BN_OUT;
         const uint8_t* sa_rows = sfa + (size_t)(a_row / 128) * KG * SF_CHUNK;
         const uint8_t* sb0_rows = sfb + (size_t)(b_row0 / 128) * KG * SF_CHUNK;
@@ -307,28 +355,44 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           }
           const uint32_t sa = base + s * OPER_BYTES;
           const uint32_t ss = sf_smem + s * SF_STAGE;
-          const uint32_t fb = saddr(&ctl->full[s]);
+          const uint32_t fb_local = saddr(&ctl->full[s]);
+          // the pair's copies all count on the first CTA's barrier
+          const uint32_t fb = (CG == 2) ? map_to_rank(fb_local, 0) : fb_local;
           const int sg = sf_group_of_stage(kb, KG);
-          mbar_expect_tx(fb, OPER_BYTES + (sg >= 0 ? SF_STAGE : 0));
-          tma_load_2d<1>(sa, &tmA, kb * BK, a_row, fb);
-          tma_load_2d<1>(sa + A_BYTES, &tmB, kb * BK, b_row0, fb);
-          tma_load_2d<1>(sa + A_BYTES + B_HALF, &tmB, kb * BK, b_row0 + b_second_off, fb);
-          if (sg >= 0) {
-            bulk_load(ss, sa_rows + (size_t)sg * SF_CHUNK, SF_CHUNK, fb);
-            bulk_load(ss + SF_CHUNK, sb0_rows + (size_t)sg * SF_CHUNK, SF_CHUNK, fb);
-            bulk_load(ss + 2 * SF_CHUNK, sb1_rows + (size_t)sg * SF_CHUNK, SF_CHUNK, fb);
+          if (leader) mbar_expect_tx(fb_local, (OPER_BYTES + (sg >= 0 ? SF_STAGE : 0)) * CG);
+          MOE_CHECK(s >= 0 && s < STAGES && a_row >= 0);
+          tma_load_2d<CG>(sa, &tmA, kb * BK, a_row, fb);
+          if (CG == 2) {   // this CTA's half of B: gate rows or up rows (gate/up), 128 rows (down)
+            tma_load_2d<CG>(sa + A_BYTES, &tmB, kb * BK, b_row0 + (int)rank * b_second_off, fb);
+            if (sg >= 0) {
+              tma_load_2d<CG>(ss, &tmSFA, 0, (a_row / 128) * KG + sg, fb);
+              tma_load_2d<CG>(ss + SF_CHUNK, &tmSFB, 0, (b_row0 / 128) * KG + sg, fb);
+              tma_load_2d<CG>(ss + 2 * SF_CHUNK, &tmSFB, 0,
+                              ((b_row0 + b_second_off) / 128) * KG + sg, fb);
+            }
+          } else {
+            tma_load_2d<CG>(sa + A_BYTES, &tmB, kb * BK, b_row0, fb);
+            tma_load_2d<CG>(sa + A_BYTES + B_HALF, &tmB, kb * BK, b_row0 + b_second_off, fb);
+            if (sg >= 0) {
+              bulk_load(ss, sa_rows + (size_t)sg * SF_CHUNK, SF_CHUNK, fb);
+              bulk_load(ss + SF_CHUNK, sb0_rows + (size_t)sg * SF_CHUNK, SF_CHUNK, fb);
+              bulk_load(ss + 2 * SF_CHUNK, sb1_rows + (size_t)sg * SF_CHUNK, SF_CHUNK, fb);
+            }
           }
         }
         if (!ok) break;
       }
-      for (int i = max(0, it - STAGES); i < it; ++i)
-        wait_phase(saddr(&ctl->full[i % STAGES]), (uint32_t)(i / STAGES) & 1u, &no_abort, status,
-                   DRAIN_NS);
+      // the copies of the last STAGES stages land before the CTA exits (the
+      // first CTA's barriers also count the peer's copies)
+      if (leader)
+        for (int i = max(0, it - STAGES); i < it; ++i)
+          wait_phase(saddr(&ctl->full[i % STAGES]), (uint32_t)(i / STAGES) & 1u, &no_abort,
+                     status, DRAIN_NS);
     }
   } else if (warp == 1) {
-    if (lane == 0) {  // ---------------------------------------------- MMA issuer
+    if (lane == 0 && leader) {  // ------------------------------------ MMA issuer
       int it = 0, tcount = 0;
-      for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
+      for (int tile = cta_group; tile < total; tile += n_groups, ++tcount) {
         if (!wait_phase(saddr(&ctl->tempty), ((uint32_t)tcount & 1u) ^ 1u, abort_flag, status,
                         WAIT_NS))
           break;
@@ -348,25 +412,25 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           MOE_CHECK(SF_COL0 + 2 * SF_COLS <= TMEM_COLS && s >= 0 && s < STAGES);
           if (sg >= 0) {   // this stage brought the scales of k group sg
             const uint32_t slot = tmem + SF_COL0 + (uint32_t)(sg & 1) * SF_COLS;
-            sf_copy(slot, sf_desc(ss));
-            sf_copy(slot + 4, sf_desc(ss + SF_CHUNK));
-            sf_copy(slot + 8, sf_desc(ss + 2 * SF_CHUNK));
+            sf_copy<CG>(slot, sf_desc(ss));
+            sf_copy<CG>(slot + 4, sf_desc(ss + SF_CHUNK));
+            sf_copy<CG>(slot + 8, sf_desc(ss + 2 * SF_CHUNK));
           }
           const uint32_t cur = tmem + SF_COL0 + (uint32_t)((kb >> 2) & 1) * SF_COLS;
           const uint32_t sel = (uint32_t)(kb & 3);   // scale byte of this k block
-          const uint32_t idesc = idesc_fp8(sel);
+          const uint32_t idesc = idesc_fp8<CG>(sel);
           const uint64_t ad = sw128_desc(sa);
           const uint64_t bd = sw128_desc(sa + A_BYTES);
 #pragma unroll
           for (uint32_t j = 0; j < 4; ++j)
-            mma_fp8(tmem, ad + 2 * j, bd + 2 * j, idesc, cur | (sel << 30),
-                    (cur + 4) | (sel << 30), (kb | (int)j) != 0 ? 1u : 0u);
-          tc_commit<1>(saddr(&ctl->empty[s]));
+            mma_fp8<CG>(tmem, ad + 2 * j, bd + 2 * j, idesc, cur | (sel << 30),
+                        (cur + 4) | (sel << 30), (kb | (int)j) != 0 ? 1u : 0u);
+          tc_commit<CG>(saddr(&ctl->empty[s]));
         }
         if (!ok) break;
-        tc_commit<1>(saddr(&ctl->tfull));
+        tc_commit<CG>(saddr(&ctl->tfull));
       }
-      tc_commit<1>(saddr(&ctl->drain));
+      tc_commit<CG>(saddr(&ctl->drain));
       wait_phase(saddr(&ctl->drain), 0u, &no_abort, status, DRAIN_NS);
     }
   } else {  // -------------------------------------------------------- epilogue
@@ -374,13 +438,16 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const int r_in = q * 32 + lane;         // row of the tile
     const int half = (warp - 2) >> 2;       // gate/up: which 64 of the tile's 128 h columns
     const int KBo = N_out / FP8_BLOCK;      // scale blocks of an output row (MODE 0)
+    // TMEM is released on the pair's first CTA's barrier
+    const uint32_t tempty_lead = (CG == 2) ? map_to_rank(saddr(&ctl->tempty), 0)
+                                           : saddr(&ctl->tempty);
     int tcount = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
+    for (int tile = cta_group; tile < total; tile += n_groups, ++tcount) {
       int m, n;
       const int e = decode_tile(tile, NT, P, G, m, n);
-      MOE_CHECK(e >= 0 && e < G && n >= 0 && n < NT && m >= 0 && m * BM < max(kept_s[e], 1) &&
-                r_in < BM);
-      const int first = m * BM;
+      MOE_CHECK(e >= 0 && e < G && n >= 0 && n < NT && m >= 0 &&
+                m * CF::TILE_ROWS < max(kept_s[e], 1) && r_in < BM);
+      const int first = m * CF::TILE_ROWS + (int)rank * BM;   // this CTA's 128 rows
       const int rows = min(BM, kept_s[e] - first);
       const long long row0 = (long long)row_off[e] + first;
       const long long grow = row0 + r_in;
@@ -413,7 +480,9 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_local(saddr(&ctl->tempty));   // TMEM free for the next tile
+        if (lane == 0) {   // TMEM free for the next tile
+          if (CG == 2) mbar_arrive_cluster(tempty_lead); else mbar_arrive_local(tempty_lead);
+        }
         float h[64];
         float amax = 0.f;
 #pragma unroll
@@ -478,7 +547,9 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_local(saddr(&ctl->tempty));
+        if (lane == 0) {
+          if (CG == 2) mbar_arrive_cluster(tempty_lead); else mbar_arrive_local(tempty_lead);
+        }
         __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(out_v) + (row_ok ? grow : 0) * (long long)N_out;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -512,9 +583,10 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 
   tc_fence_before();
   __syncthreads();
+  if (CG == 2) cluster_sync();   // no CTA leaves while its peer may still signal it
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc<1>(tmem, TMEM_COLS);
+    tmem_dealloc<CG>(tmem, TMEM_COLS);
   }
 }
 
@@ -532,26 +604,115 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t row
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE>
+// The scale chunks of a blocked scale buffer ([rows/128][KG][512 bytes]) as a
+// 2-D uint32 tensor [chunks][128]: one chunk per box, no swizzle.
+bool make_map_sf(CUtensorMap* map, const void* base, int64_t rows, int64_t kdim) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+  if (!enc) return false;
+  const int64_t chunks = ceil_div(rows, 128) * ceil_div(kdim / FP8_BLOCK, 4);
+  const cuuint64_t dims[2] = {SF_CHUNK / 4, (cuuint64_t)chunks};
+  const cuuint64_t strides[1] = {SF_CHUNK};
+  const cuuint32_t box[2] = {SF_CHUNK / 4, 1};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE, int CG>
 cudaError_t launch_one(int grid, size_t smem, cudaStream_t s, const CUtensorMap& a,
-                       const CUtensorMap& b, const CUtensorMap& o, const uint8_t* sfa,
-                       const uint8_t* sfb, void* out, uint8_t* out_sf, int N_out, int Kdim,
-                       int b_rows, int b_second, const int32_t* offsets, const int32_t* counts,
-                       int E, int C, long long R_max, uint32_t* status, int sh_rows,
-                       int sh_row0) {
+                       const CUtensorMap& b, const CUtensorMap& o, const CUtensorMap& msfa,
+                       const CUtensorMap& msfb, const uint8_t* sfa, const uint8_t* sfb, void* out,
+                       uint8_t* out_sf, int N_out, int Kdim, int b_rows, int b_second,
+                       const int32_t* offsets, const int32_t* counts, int E, int C,
+                       long long R_max, uint32_t* status, int sh_rows, int sh_row0) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3(num_threads<MODE>());
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = CG;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, fp8_grouped_gemm<MODE>, a, b, o, sfa, sfb, out, out_sf, N_out,
-                            Kdim, b_rows, b_second, offsets, counts, E, C, R_max, status, sh_rows,
-                            sh_row0);
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, fp8_grouped_gemm<MODE, CG>, a, b, o, msfa, msfb, sfa, sfb, out,
+                            out_sf, N_out, Kdim, b_rows, b_second, offsets, counts, E, C, R_max,
+                            status, sh_rows, sh_row0);
+}
+
+// Co-resident CTAs (CG = 1) or CTA pairs (CG = 2) of one launch.
+template <int MODE, int CG>
+int resident_groups(size_t smem) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  if (CG == 1) return sms;
+  cudaLaunchConfig_t q = {};
+  q.gridDim = dim3((unsigned)(sms & ~1));
+  q.blockDim = dim3(num_threads<MODE>());
+  q.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  q.attrs = attr;
+  q.numAttrs = 1;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, fp8_grouped_gemm<MODE, CG>, &q) != cudaSuccess)
+    return 0;
+  return clusters;
+}
+
+template <int CG>
+moe_status_t launch_mlp(const moe_config_t& c, const uint8_t* xq, const uint8_t* xs,
+                        const int32_t* offsets, const int32_t* counts, const uint8_t* wq_gu,
+                        const uint8_t* ws_gu, const uint8_t* wq_d, const uint8_t* ws_d,
+                        uint8_t* hq, uint8_t* hs, void* y, int64_t R_max, uint32_t* status,
+                        cudaStream_t s) {
+  const int n_sh = c.n_shared ? 1 : 0;
+  const int G = c.E + n_sh;   // routed experts + the shared expert (last in the weights)
+  CUtensorMap mx, mwgu, mh, mwd, my, sx, sgu, shh, sd;
+  if (!make_map_u8(&mx, xq, (uint64_t)c.H, (uint64_t)R_max) ||
+      !make_map_u8(&mwgu, wq_gu, (uint64_t)c.H, (uint64_t)G * 2 * c.F) ||
+      !make_map_u8(&mh, hq, (uint64_t)c.F, (uint64_t)R_max) ||
+      !make_map_u8(&mwd, wq_d, (uint64_t)c.F, (uint64_t)G * c.H) ||
+      !tc::make_map(&my, y, (uint64_t)c.H, (uint64_t)R_max))
+    return MOE_ERR_CUDA;
+  if (CG == 2) {
+    if (!make_map_sf(&sx, xs, R_max, c.H) || !make_map_sf(&sgu, ws_gu, (int64_t)G * 2 * c.F, c.H) ||
+        !make_map_sf(&shh, hs, R_max, c.F) || !make_map_sf(&sd, ws_d, (int64_t)G * c.H, c.F))
+      return MOE_ERR_CUDA;
+  } else {   // not read by the one-CTA kernel
+    sx = sgu = shh = sd = mx;
+  }
+  const int sh_rows = n_sh ? c.T : 0;
+  const int sh_row0 = n_sh ? (int)shared_row0(c) : 0;
+  const size_t smem = smem_bytes<CG>(G);
+  if (cudaFuncSetAttribute(fp8_grouped_gemm<0, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess ||
+      cudaFuncSetAttribute(fp8_grouped_gemm<1, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int u0 = resident_groups<0, CG>(smem), u1 = resident_groups<1, CG>(smem);
+  if (u0 <= 0 || u1 <= 0) return MOE_ERR_CUDA;
+  const int64_t mt_bound = ceil_div(R_max, F8<CG>::TILE_ROWS) + G;   // >= sum of M tiles
+  const int g0 = (int)std::min<int64_t>(u0, mt_bound * ceil_div(c.F, 128)) * CG;
+  const int g1 = (int)std::min<int64_t>(u1, mt_bound * ceil_div(c.H, 256)) * CG;
+  cudaError_t e = launch_one<0, CG>(g0, smem, s, mx, mwgu, mh, sx, sgu, xs, ws_gu, hq, hs, c.F,
+                                    c.H, 2 * c.F, c.F, offsets, counts, c.E, c.capacity,
+                                    (long long)R_max, status, sh_rows, sh_row0);
+  if (e == cudaSuccess)
+    e = launch_one<1, CG>(g1, smem, s, mh, mwd, my, shh, sd, hs, ws_d, y, nullptr, c.H, c.F, c.H,
+                          128, offsets, counts, c.E, c.capacity, (long long)R_max, status,
+                          sh_rows, sh_row0);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace f8
@@ -561,39 +722,17 @@ moe_status_t launch_mlp_fp8(const moe_config_t& c, const uint8_t* xq, const uint
                             const uint8_t* ws_gu, const uint8_t* wq_d, const uint8_t* ws_d,
                             uint8_t* hq, uint8_t* hs, void* y, int64_t R_max, uint32_t* status,
                             cudaStream_t s) {
-  using namespace f8;
   if (R_max == 0) return MOE_OK;
-  const int n_sh = c.n_shared ? 1 : 0;
-  const int G = c.E + n_sh;   // routed experts + the shared expert (last in the weights)
-  CUtensorMap mx, mwgu, mh, mwd, my;
-  if (!make_map_u8(&mx, xq, (uint64_t)c.H, (uint64_t)R_max) ||
-      !make_map_u8(&mwgu, wq_gu, (uint64_t)c.H, (uint64_t)G * 2 * c.F) ||
-      !make_map_u8(&mh, hq, (uint64_t)c.F, (uint64_t)R_max) ||
-      !make_map_u8(&mwd, wq_d, (uint64_t)c.F, (uint64_t)G * c.H) ||
-      !tc::make_map(&my, y, (uint64_t)c.H, (uint64_t)R_max))
-    return MOE_ERR_CUDA;
-  const int sh_rows = n_sh ? c.T : 0;
-  const int sh_row0 = n_sh ? (int)shared_row0(c) : 0;
-  const size_t smem = smem_bytes(G);
-  if (cudaFuncSetAttribute(fp8_grouped_gemm<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess ||
-      cudaFuncSetAttribute(fp8_grouped_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  const int64_t mt_bound = ceil_div(R_max, BM) + G;   // >= sum over groups of M tiles
-  const int g0 = (int)std::min<int64_t>(sms, mt_bound * ceil_div(c.F, 128));
-  const int g1 = (int)std::min<int64_t>(sms, mt_bound * ceil_div(c.H, 256));
-  cudaError_t e = launch_one<0>(g0, smem, s, mx, mwgu, mh, xs, ws_gu, hq, hs, c.F, c.H, 2 * c.F,
-                                c.F, offsets, counts, c.E, c.capacity, (long long)R_max, status,
-                                sh_rows, sh_row0);
-  if (e == cudaSuccess)
-    e = launch_one<1>(g1, smem, s, mh, mwd, my, hs, ws_d, y, nullptr, c.H, c.F, c.H, 128, offsets,
-                      counts, c.E, c.capacity, (long long)R_max, status, sh_rows, sh_row0);
-  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  // 256-row CTA-pair tiles halve each CTA's operand bytes per k step; small
+  // experts (decode-like batches) keep 128-row one-CTA tiles, whose padding
+  // is half as large (as in the bf16 grouped GEMM)
+  const int64_t rows_per_expert =
+      c.E > 0 ? std::min<int64_t>((int64_t)c.T * c.K, (int64_t)c.E * c.capacity) / c.E : c.T;
+  if (rows_per_expert >= 192)
+    return f8::launch_mlp<2>(c, xq, xs, offsets, counts, wq_gu, ws_gu, wq_d, ws_d, hq, hs, y,
+                             R_max, status, s);
+  return f8::launch_mlp<1>(c, xq, xs, offsets, counts, wq_gu, ws_gu, wq_d, ws_d, hq, hs, y, R_max,
+                           status, s);
 }
 
 }  // namespace moe

@@ -125,7 +125,7 @@ MLP_CASES = [
     (600, 256, 8, 2, 384, 8, 2.0, "zipf"),        # empty experts
     (128, 256, 64, 8, 128, 8, 2.0, "normal"),     # many tiny experts
     (1200, 1024, 8, 2, 1024, 2, 1.25, "normal"),  # several M and N tiles per expert
-    # >= 192 rows per expert: many full 128-row tiles per expert
+    # >= 192 rows per expert: 256-row CTA-pair tiles, several per expert
     (2048, 256, 4, 2, 256, 2, 1.25, "normal"),    # ragged last tile per expert
     (1500, 512, 6, 2, 384, 3, 1.0, "zipf"),       # skewed experts, some at capacity
     (3000, 256, 12, 2, 256, 4, 2.0, "hot"),       # one hot expert over many tiles
