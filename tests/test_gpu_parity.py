@@ -73,7 +73,12 @@ def test_route_is_deterministic(cuda_ok):
 
 @pytest.mark.parametrize("act", ["bf16", "f32"])
 @pytest.mark.parametrize("T,H,E,K,S,cf,A", [
-    (300, 256, 8, 2, 2, 1.0, 128), (1000, 128, 17, 5, 1, 0.7, 4), (64, 7168, 4, 2, 2, 1.0, 1)])
+    (300, 256, 8, 2, 2, 1.0, 128), (1000, 128, 17, 5, 1, 0.7, 4), (64, 7168, 4, 2, 2, 1.0, 1),
+    (333, 7168, 32, 8, 8, 0.5, 1),        # 14 KB rows, K = 8, half the assignments dropped
+    (4096, 4096, 32, 8, 4, 1.0, 128),     # 8 KB (bf16) / 16 KB (f32) rows, several tokens per block
+    (4133, 7168, 64, 8, 8, 0.5, 1),       # a ragged token tail
+    (4096, 4096, 16, 10, 2, 0.1, 128),    # most tokens lose every assignment
+])
 def test_dispatch_bit_exact(cuda_ok, act, T, H, E, K, S, cf, A):
     C = O.capacity(T, K, E, cf)
     lg = logits_for(T, E, "hot", 11)
@@ -249,10 +254,38 @@ def test_empty_batch(cuda_ok):
     assert torch.all(v["row_src"] == -1)
 
 
-def test_out_of_range_slots_are_treated_as_dropped(cuda_ok):
+@pytest.mark.parametrize("act", ["bf16", "f32"])
+@pytest.mark.parametrize("T,H,K", [(257, 256, 2), (257, 7168, 8), (4099, 4096, 8)])
+def test_dispatch_shared_expert_rows(cuda_ok, act, T, H, K):
+    # with a shared expert the piecewise dispatch also copies every token to its
+    # shared row shared_row0 + t: one more destination per token
+    E, S, A = 16, 4, 128
+    C = O.capacity(T, K, E, 0.75)
+    cfg = M.make_config(T=T, H=H, E=E, K=K, F=64, S=S, capacity=C, row_align=A, act=act,
+                        n_shared=1)
+    r = run_route(cfg, logits_for(T, E, "zipf", 31).to(DEV))
+    dt = torch.float32 if act == "f32" else torch.bfloat16
+    x = torch.randn(T, H, generator=torch.Generator().manual_seed(8)).to(dt).to(DEV)
+    R = M.moe_max_rows(cfg)
+    xp = torch.full((R, H), 5, dtype=dt, device=DEV)
+    M.moe_dispatch(cfg, x, r["token_slot"], xp)
+    torch.cuda.synchronize()
+    r0 = M.shared_row0(cfg)
+    assert r0 + T <= R
+    assert np.array_equal(act_np(xp[r0:r0 + T]), act_np(x))          # the shared rows
+    ts = r["token_slot"].cpu().numpy()
+    ref = O.dispatch(act_np(x), ts, r0)
+    kept = np.zeros(r0, bool)
+    kept[ts[ts >= 0]] = True
+    assert np.array_equal(act_np(xp[:r0])[kept], ref[kept])          # the routed rows
+    assert np.all(act_np(xp[:r0])[~kept] == act_np(torch.full((1, H), 5, dtype=dt)))
+
+
+@pytest.mark.parametrize("T,H,K", [(300, 256, 2), (4096, 4096, 8)])
+def test_out_of_range_slots_are_treated_as_dropped(cuda_ok, T, H, K):
     # caller-supplied tables: entries beyond the routed rows (or below -1) must
     # not be written or read; the kernels treat them as dropped assignments
-    T, H, E, K, S, A = 300, 256, 8, 2, 2, 8
+    E, S, A = 8, 2, 8
     C = O.capacity(T, K, E, 1.0)
     cfg = cfg_for(T, H, E, K, 64, S, C, A, "bf16")
     r = run_route(cfg, logits_for(T, E, "normal", 21).to(DEV))
