@@ -28,7 +28,7 @@ LIB = os.path.join(HERE, "libmoe.so")
 LIB_CHECK = os.path.join(HERE, "libmoe_check.so")
 SOURCES = ["moe_abi.cu", "route.cu", "dispatch_combine.cu", "gemm_simt.cu", "gemm_tc.cu",
            "route_noalloc.cu", "quant_fp8.cu", "gemm_fp8.cu", "ep.cu"]
-HEADERS = [os.path.join(CSRC, h) for h in ("moe_internal.h", "tc_ptx.cuh", "fp8_util.cuh",
+HEADERS = [os.path.join(CSRC, h) for h in ("moe_internal.h", "tc_ptx.cuh", "tile_sched.cuh", "fp8_util.cuh",
                                          "vec_util.cuh")] + \
     [os.path.join(ROOT, "include", h) for h in ("moe.h", "moe_ep.h")]
 GENCODE = "arch=compute_100a,code=sm_100a"

@@ -169,12 +169,14 @@ moe_status_t ep_validate(const moe_config_t* c, const moe_ep_t* ep) {
 }
 
 // The fp8 expert-parallel layer: the fp8 grouped GEMM's limits on each rank's
-// local experts (and on its shared expert), untagged steps only.
+// local experts (and on its shared expert); with the remote-first order its
+// tables must fit the kernel's shared memory too.
 moe_status_t ep_validate_fp8(const moe_config_t* c, const moe_ep_t* ep) {
   moe_status_t st = ep_validate(c, ep);
   if (st != MOE_OK) return st;
-  if (ep->flags != 0) return MOE_ERR_UNSUPPORTED;
   const moe_config_t l = local_cfg(*c, ep->world);
+  if ((ep->flags & MOE_EP_REMOTE_FIRST) && fp8_ep_smem_bytes(l, true) > 227 * 1024)
+    return MOE_ERR_UNSUPPORTED;
   return validate_fp8(&l);
 }
 
@@ -1121,16 +1123,47 @@ moe_status_t moe_ep_expert_mlp_fp8(const moe_config_t* cfg, const moe_ep_t* ep,
         hq_sh, hq_sh + align256((size_t)c.T * c.F), p.y_sh, c.T, p.status, s);
     if (st != MOE_OK) return st;
   }
-  st = cuda_st(launch_pdl(ep_wait_kernel, dim3(1), dim3(32), 0, s,
-                          (const uint32_t*)(sb + S.flags) + FLAG_DISPATCH * W, W,
-                          Epoch{ep->epoch, p.epoch}, timeout_ns(*ep), p.status,
-                          (uint32_t*)nullptr));
-  if (st != MOE_OK) return st;
+  const uint32_t* dispatch_flags = (const uint32_t*)(sb + S.flags) + FLAG_DISPATCH * W;
   const moe_config_t l = local_cfg(c, W);
   const uint8_t* xq = reinterpret_cast<const uint8_t*>(sb + S.xr);
   const uint8_t* xs = xq + align256((size_t)R * c.H);
   uint8_t* hq = reinterpret_cast<uint8_t*>(p.h);
   uint8_t* hs = hq + align256((size_t)R * c.F);
+  if (ep->flags & MOE_EP_TILE_SIGNAL) {
+    // as the bf16 layer: gate/up waits per CTA for the senders of its rows
+    // (codes and scale chunks), then every sender (y and the other ready bank
+    // are free), then down, publishing y's blocks as they are stored
+    EpTiles t;
+    t.arrive = dispatch_flags;
+    t.split = p.split;
+    t.counter = p.epoch;
+    t.epoch = ep->epoch;
+    t.W = W;
+    t.rank = ep->rank;
+    t.remote_first = (ep->flags & MOE_EP_REMOTE_FIRST) ? 1 : 0;
+    t.wait_ns = timeout_ns(*ep);
+    st = launch_mlp_fp8_ep(l, 1, xq, xs, p.recv_off, p.recv_cnt, wq_gu_local, ws_gu_local,
+                           wq_d_local, ws_d_local, hq, hs, sb + S.y, R, p.status, s, t);
+    if (st != MOE_OK) return st;
+    const int nblk = (int)ready_blocks(c, W);
+    st = cuda_st(launch_pdl(ep_wait_zero_kernel, dim3(1), dim3(1024), 0, s, dispatch_flags, W,
+                            Epoch{ep->epoch, p.epoch}, timeout_ns(*ep), p.status,
+                            reinterpret_cast<uint32_t*>(sb + S.yready), nblk));
+    if (st != MOE_OK) return st;
+    t.arrive = nullptr;
+    t.yready = reinterpret_cast<uint32_t*>(sb + S.yready);
+    t.ready_blocks = nblk;
+    st = launch_mlp_fp8_ep(l, 2, xq, xs, p.recv_off, p.recv_cnt, wq_gu_local, ws_gu_local,
+                           wq_d_local, ws_d_local, hq, hs, sb + S.y, R, p.status, s, t);
+    if (st != MOE_OK) return st;
+    return cuda_st(launch_pdl(ep_signal_kernel, dim3(1), dim3(MAX_W), 0, s, peers, S.flags,
+                              (int)FLAG_Y, W, ep->rank, Epoch{ep->epoch, p.epoch},
+                              (const uint32_t*)p.status));
+  }
+  st = cuda_st(launch_pdl(ep_wait_kernel, dim3(1), dim3(32), 0, s, dispatch_flags, W,
+                          Epoch{ep->epoch, p.epoch}, timeout_ns(*ep), p.status,
+                          (uint32_t*)nullptr));
+  if (st != MOE_OK) return st;
   st = launch_mlp_fp8(l, xq, xs, p.recv_off, p.recv_cnt, wq_gu_local, ws_gu_local, wq_d_local,
                       ws_d_local, hq, hs, sb + S.y, R, p.status, s);
   if (st != MOE_OK) return st;

@@ -42,6 +42,7 @@
 #include "fp8_util.cuh"
 #include "moe_internal.h"
 #include "tc_ptx.cuh"
+#include "tile_sched.cuh"
 
 namespace moe {
 namespace tc {
@@ -97,10 +98,13 @@ struct Ctl {
   float amax[2][2][128];   // gate/up: [tile parity][column half][row] partial amax of h
 };
 
+// Shared memory of a launch over G groups; two_sets: the remote-first tile
+// order's tables too (expert-parallel launches only: they would not fit at the
+// 512-expert limit of the plain layer).
 template <int CG>
-size_t smem_bytes(int E) {
+size_t smem_bytes(int G, bool two_sets = false) {
   return 1024 + (size_t)F8<CG>::STAGES * (F8<CG>::OPER_BYTES + SF_STAGE) + STAGING_BYTES +
-         sizeof(Ctl) + (size_t)(3 * E + 2) * 4;
+         sizeof(Ctl) + (size_t)(3 * G + 2 + (two_sets ? 2 * G + 1 : 0)) * 4;
 }
 
 // Instruction descriptor of tcgen05.mma.kind::mxf8f6f4.block_scale: B scale
@@ -180,7 +184,9 @@ __device__ __forceinline__ int sf_group_of_stage(int kb, int KG) {
   return -1;
 }
 
-__device__ __forceinline__ int decode_tile(int tile, int NT, const int* P, int E, int& m, int& n) {
+// Tile -> (group, m tile, n tile), one set: group e owns tiles
+// [NT*P[e], NT*P[e+1]), n-major then m.
+__device__ __forceinline__ int decode_tile1(int tile, int NT, const int* P, int E, int& m, int& n) {
   const int g = tile / NT;
   int lo = 0, hi = E;
   while (hi - lo > 1) {
@@ -192,6 +198,16 @@ __device__ __forceinline__ int decode_tile(int tile, int NT, const int* P, int E
   n = local / mt;
   m = local - n * mt;
   return lo;
+}
+
+// Either order: with the remote-first tables (PB, ml0) the two-set order of
+// the tile-signalled expert-parallel layer, else one set.
+__device__ __forceinline__ int tile_of(int tile, int NT, const int* P, const int* PB,
+                                       const int* ml0, int G, int& m, int& n) {
+  if (PB == nullptr) return decode_tile1(tile, NT, P, G, m, n);
+  int e;
+  decode_tile(tile, NT, P, PB, ml0, G, e, m, n);
+  return e;
 }
 
 // Write one 128-byte row of the output box into the staging buffer at the
@@ -225,7 +241,7 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                  uint8_t* __restrict__ out_sf, int N_out, int Kdim, int b_rows_per_expert,
                  int b_second_off, const int32_t* __restrict__ offsets,
                  const int32_t* __restrict__ counts, int E, int C, long long R_max,
-                 uint32_t* __restrict__ status, int sh_rows, int sh_row0) {
+                 uint32_t* __restrict__ status, int sh_rows, int sh_row0, const EpTiles ept) {
   using CF = F8<CG>;
   constexpr int STAGES = CF::STAGES;
   constexpr int OPER_BYTES = CF::OPER_BYTES;
@@ -245,6 +261,10 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   int* P = reinterpret_cast<int*>(ctl + 1);   // [G+1] M-tile prefix
   int* row_off = P + (G + 1);                 // [G+1] first row of each group, and its end
   int* kept_s = row_off + (G + 1);            // [G]
+  // remote-first order (tile-signalled expert-parallel gate/up and down)
+  const bool two_sets = ept.remote_first != 0 && ept.split != nullptr;
+  int* PB = two_sets ? kept_s + G : nullptr;  // [G+1] prefix of the M tiles ordered last
+  int* ml0 = two_sets ? PB + (G + 1) : nullptr;   // [G] first M tile ordered last
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;   // position in the pair
@@ -257,6 +277,12 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   // drains wait for copies and MMAs already issued even after an abort (bounded
   // by DRAIN_NS): shared memory and TMEM must not be released under them
   volatile int no_abort = 0;
+  // With arrival waits (tile-signalled gate/up) one CTA of a pair may hold its
+  // loads back for as long as a sender is late (up to ept.wait_ns), and every
+  // other wait of the pair must outlast that.
+  const bool arrivals = MODE == 0 && ept.arrive != nullptr;
+  const unsigned long long wait_ns =
+      arrivals ? (ept.wait_ns + DRAIN_NS > WAIT_NS ? ept.wait_ns + DRAIN_NS : WAIT_NS) : WAIT_NS;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -282,10 +308,13 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   }
   pdl_wait();
   pdl_trigger();
-  {  // per-group kept rows, first row and M-tile prefix (block scan)
+  // this step's number (tile-signalled expert-parallel GEMMs only)
+  const uint32_t step = ept.epoch ? ept.epoch
+                                  : (ept.counter ? *(volatile const uint32_t*)ept.counter + 1u : 0u);
+  {  // per-group kept rows, first row and M-tile prefixes (block scans)
     const int chunk = (G + NUM_THREADS - 1) / NUM_THREADS;
     const int e0 = threadIdx.x * chunk;
-    int local = 0;
+    int local = 0, localB = 0;
     for (int i = 0; i < chunk; ++i) {
       const int e = e0 + i;
       if (e < G) {
@@ -299,28 +328,65 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
         kept_s[e] = k;
         row_off[e] = off;
-        local += (k + CF::TILE_ROWS - 1) / CF::TILE_ROWS;
+        const int mt = (k + CF::TILE_ROWS - 1) / CF::TILE_ROWS;
+        local += mt;
+        if (two_sets) {
+          // remote-first order: the M tiles whose rows are all this owner's
+          // own (one contiguous block of the expert's rows) are ordered last
+          int first_local = 0, n_local = 0;
+          if (e < E && k > 0) {
+            const int* sp = ept.split + (size_t)e * (ept.W + 1);
+            const int lo = min(max(sp[ept.rank], 0), k), hi = min(max(sp[ept.rank + 1], lo), k);
+            const int m_lo = (lo + CF::TILE_ROWS - 1) / CF::TILE_ROWS;
+            const int m_hi = hi >= k ? mt : hi / CF::TILE_ROWS;
+            if (m_hi > m_lo) {
+              first_local = m_lo;
+              n_local = m_hi - m_lo;
+            }
+          }
+          ml0[e] = first_local;
+          PB[e] = n_local;   // replaced by its prefix below
+          localB += n_local;
+        }
       }
     }
-    int incl = local;
+    // exclusive block prefix of v (all threads); *tot: the block's sum
+    auto block_prefix = [&](int v, int* tot) {
+      int incl = v;
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int o = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += o;
-    }
-    if (lane == 31) ctl->wsum[warp] = incl;
-    __syncthreads();
-    int run = incl - local;
-    for (int w = 0; w < warp; ++w) run += ctl->wsum[w];
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      if (lane == 31) ctl->wsum[warp] = incl;
+      __syncthreads();
+      int run = incl - v, t = 0;
+      for (int w = 0; w < NUM_THREADS / 32; ++w) {
+        if (w < warp) run += ctl->wsum[w];
+        t += ctl->wsum[w];
+      }
+      __syncthreads();   // wsum is reused
+      *tot = t;
+      return run;
+    };
+    int tot = 0, totB = 0;
+    int run = block_prefix(local, &tot);
+    int runB = two_sets ? block_prefix(localB, &totB) : 0;
     for (int i = 0; i < chunk; ++i) {
       const int e = e0 + i;
       if (e < G) {
         P[e] = run;
         run += (kept_s[e] + CF::TILE_ROWS - 1) / CF::TILE_ROWS;
+        if (two_sets) {
+          const int n_local = PB[e];
+          PB[e] = runB;
+          runB += n_local;
+        }
       }
     }
     if (threadIdx.x == NUM_THREADS - 1) {
-      P[G] = run;
+      P[G] = tot;
+      if (two_sets) PB[G] = totB;
       row_off[G] = G > E ? sh_row0 + sh_rows : offsets[E];
     }
   }
@@ -334,9 +400,10 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   if (warp == 0) {
     if (lane == 0) {  // ------------------------------------------------ TMA producer
       int it = 0;
+      uint64_t seen = 0;   // senders whose DISPATCH flag of this step has been seen
       for (int tile = cta_group; tile < total; tile += n_groups) {
         int m, n;
-        const int e = decode_tile(tile, NT, P, G, m, n);
+        const int e = tile_of(tile, NT, P, PB, ml0, G, m, n);
         MOE_CHECK(e >= 0 && e < G && n >= 0 && n < NT && m >= 0 &&
                   m * CF::TILE_ROWS < max(kept_s[e], 1));
         // this CTA's 128 rows of A (a multiple of 128)
@@ -346,10 +413,34 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const uint8_t* sb0_rows = sfb + (size_t)(b_row0 / 128) * KG * SF_CHUNK;
         const uint8_t* sb1_rows = sfb + (size_t)((b_row0 + b_second_off) / 128) * KG * SF_CHUNK;
         bool ok = true;
+        if (arrivals && e < E) {
+          // this CTA's rows of the tile (codes and their scale chunk): wait for
+          // every sender that owns some of them
+          const int lo = m * CF::TILE_ROWS + (int)rank * BM;
+          const int hi = min(lo + BM, kept_s[e]);
+          const int* sp = ept.split + (size_t)e * (ept.W + 1);
+          bool waited = false;
+          for (int s = 0; s < ept.W && ok && lo < hi; ++s) {
+            if ((seen >> s) & 1ull) continue;
+            const int a = sp[s], b = sp[s + 1];
+            if (b > a && a < hi && b > lo) {
+              ok = wait_arrival(ept.arrive + s, step, abort_flag, status, ept.wait_ns);
+              seen |= 1ull << s;
+              waited = true;
+            }
+          }
+          if (!ok) {
+            if (CG == 2) abort_peer_cta(saddr(&ctl->abort), rank ^ 1u);
+            break;
+          }
+          // the rows were written by the peers' generic stores: order the
+          // acquire above before this CTA's TMA (async proxy) reads them
+          if (waited) fence_proxy_async_global();
+        }
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!wait_phase(saddr(&ctl->empty[s]), ph ^ 1u, abort_flag, status, WAIT_NS)) {
+          if (!wait_phase(saddr(&ctl->empty[s]), ph ^ 1u, abort_flag, status, wait_ns)) {
             ok = false;
             break;
           }
@@ -382,26 +473,33 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
         if (!ok) break;
       }
+      (void)seen;
       // the copies of the last STAGES stages land before the CTA exits (the
-      // first CTA's barriers also count the peer's copies)
+      // first CTA's barriers also count the peer's copies, which a pair CTA
+      // waiting for a late sender issues only then: with arrival waits the
+      // drain allows for that, unless the pair has aborted, when only this
+      // CTA's own copies, already issued, are left to land)
       if (leader)
-        for (int i = max(0, it - STAGES); i < it; ++i)
-          wait_phase(saddr(&ctl->full[i % STAGES]), (uint32_t)(i / STAGES) & 1u, &no_abort,
-                     status, DRAIN_NS);
+        for (int i = max(0, it - STAGES); i < it; ++i) {
+          const uint32_t fb = saddr(&ctl->full[i % STAGES]);
+          const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
+          if (!arrivals || !wait_phase(fb, ph, abort_flag, status, wait_ns))
+            wait_phase(fb, ph, &no_abort, status, DRAIN_NS);
+        }
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {  // ------------------------------------ MMA issuer
       int it = 0, tcount = 0;
       for (int tile = cta_group; tile < total; tile += n_groups, ++tcount) {
         if (!wait_phase(saddr(&ctl->tempty), ((uint32_t)tcount & 1u) ^ 1u, abort_flag, status,
-                        WAIT_NS))
+                        wait_ns))
           break;
         tc_fence_after();
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!wait_phase(saddr(&ctl->full[s]), ph, abort_flag, status, WAIT_NS)) {
+          if (!wait_phase(saddr(&ctl->full[s]), ph, abort_flag, status, wait_ns)) {
             ok = false;
             break;
           }
@@ -444,7 +542,7 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     int tcount = 0;
     for (int tile = cta_group; tile < total; tile += n_groups, ++tcount) {
       int m, n;
-      const int e = decode_tile(tile, NT, P, G, m, n);
+      const int e = tile_of(tile, NT, P, PB, ml0, G, m, n);
       MOE_CHECK(e >= 0 && e < G && n >= 0 && n < NT && m >= 0 &&
                 m * CF::TILE_ROWS < max(kept_s[e], 1) && r_in < BM);
       const int first = m * CF::TILE_ROWS + (int)rank * BM;   // this CTA's 128 rows
@@ -453,7 +551,7 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const long long grow = row0 + r_in;
       int ok = 1;
       if (lane == 0) ok = wait_phase(saddr(&ctl->tfull), (uint32_t)tcount & 1u, abort_flag, status,
-                                     WAIT_NS);
+                                     wait_ns);
       __syncwarp();
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
@@ -576,6 +674,23 @@ fp8_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             for (int v = 0; v < 8; ++v) dst[v] = o[v];
           }
         }
+        if (ept.yready != nullptr && rows > 0) {
+          // Publish this half tile at system scope, into this step's bank of
+          // the expert-parallel ready counters (read by the peers' combines):
+          // its 128 rows (one ready block) have one more N tile stored. The
+          // staged stores are waited for by their issuing thread, every
+          // thread fences its own stores, then one release add.
+          __threadfence_system();
+          if (threadIdx.x == 64) {
+            bulk_wait_all();
+            fence_proxy_async_global();
+          }
+          epi_bar<MODE>();
+          if (threadIdx.x == 64 && MOE_CHECKED(row0 >= 0 && row0 / READY_ROWS < ept.ready_blocks))
+            red_release_add_sys(ept.yready + (size_t)(step & 1u) * ept.ready_blocks +
+                                    (size_t)(row0 / READY_ROWS),
+                                1u);
+        }
       }
     }
     if (threadIdx.x == 64) bulk_wait_all();   // staged stores complete before the CTA exits
@@ -625,7 +740,8 @@ cudaError_t launch_one(int grid, size_t smem, cudaStream_t s, const CUtensorMap&
                        const CUtensorMap& msfb, const uint8_t* sfa, const uint8_t* sfb, void* out,
                        uint8_t* out_sf, int N_out, int Kdim, int b_rows, int b_second,
                        const int32_t* offsets, const int32_t* counts, int E, int C,
-                       long long R_max, uint32_t* status, int sh_rows, int sh_row0) {
+                       long long R_max, uint32_t* status, int sh_rows, int sh_row0,
+                       const EpTiles& ept) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3(num_threads<MODE>());
@@ -642,7 +758,7 @@ cudaError_t launch_one(int grid, size_t smem, cudaStream_t s, const CUtensorMap&
   cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, fp8_grouped_gemm<MODE, CG>, a, b, o, msfa, msfb, sfa, sfb, out,
                             out_sf, N_out, Kdim, b_rows, b_second, offsets, counts, E, C, R_max,
-                            status, sh_rows, sh_row0);
+                            status, sh_rows, sh_row0, ept);
 }
 
 // Co-resident CTAs (CG = 1) or CTA pairs (CG = 2) of one launch.
@@ -675,7 +791,7 @@ moe_status_t launch_mlp(const moe_config_t& c, const uint8_t* xq, const uint8_t*
                         const int32_t* offsets, const int32_t* counts, const uint8_t* wq_gu,
                         const uint8_t* ws_gu, const uint8_t* wq_d, const uint8_t* ws_d,
                         uint8_t* hq, uint8_t* hs, void* y, int64_t R_max, uint32_t* status,
-                        cudaStream_t s) {
+                        cudaStream_t s, int modes = 3, const EpTiles& ept = EpTiles{}) {
   const int n_sh = c.n_shared ? 1 : 0;
   const int G = c.E + n_sh;   // routed experts + the shared expert (last in the weights)
   CUtensorMap mx, mwgu, mh, mwd, my, sx, sgu, shh, sd;
@@ -694,7 +810,7 @@ moe_status_t launch_mlp(const moe_config_t& c, const uint8_t* xq, const uint8_t*
   }
   const int sh_rows = n_sh ? c.T : 0;
   const int sh_row0 = n_sh ? (int)shared_row0(c) : 0;
-  const size_t smem = smem_bytes<CG>(G);
+  const size_t smem = smem_bytes<CG>(G, ept.remote_first != 0 && ept.split != nullptr);
   if (cudaFuncSetAttribute(fp8_grouped_gemm<0, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess ||
       cudaFuncSetAttribute(fp8_grouped_gemm<1, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -705,13 +821,19 @@ moe_status_t launch_mlp(const moe_config_t& c, const uint8_t* xq, const uint8_t*
   const int64_t mt_bound = ceil_div(R_max, F8<CG>::TILE_ROWS) + G;   // >= sum of M tiles
   const int g0 = (int)std::min<int64_t>(u0, mt_bound * ceil_div(c.F, 128)) * CG;
   const int g1 = (int)std::min<int64_t>(u1, mt_bound * ceil_div(c.H, 256)) * CG;
-  cudaError_t e = launch_one<0, CG>(g0, smem, s, mx, mwgu, mh, sx, sgu, xs, ws_gu, hq, hs, c.F,
-                                    c.H, 2 * c.F, c.F, offsets, counts, c.E, c.capacity,
-                                    (long long)R_max, status, sh_rows, sh_row0);
-  if (e == cudaSuccess)
+  // gate/up: the arrival waits only; down: the ready-counter publication only
+  EpTiles t0 = ept, t1 = ept;
+  t0.yready = nullptr;
+  t1.arrive = nullptr;
+  cudaError_t e = cudaSuccess;
+  if (modes & 1)
+    e = launch_one<0, CG>(g0, smem, s, mx, mwgu, mh, sx, sgu, xs, ws_gu, hq, hs, c.F, c.H, 2 * c.F,
+                          c.F, offsets, counts, c.E, c.capacity, (long long)R_max, status,
+                          sh_rows, sh_row0, t0);
+  if (e == cudaSuccess && (modes & 2))
     e = launch_one<1, CG>(g1, smem, s, mh, mwd, my, shh, sd, hs, ws_d, y, nullptr, c.H, c.F, c.H,
                           128, offsets, counts, c.E, c.capacity, (long long)R_max, status,
-                          sh_rows, sh_row0);
+                          sh_rows, sh_row0, t1);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -733,6 +855,31 @@ moe_status_t launch_mlp_fp8(const moe_config_t& c, const uint8_t* xq, const uint
                              R_max, status, s);
   return f8::launch_mlp<1>(c, xq, xs, offsets, counts, wq_gu, ws_gu, wq_d, ws_d, hq, hs, y, R_max,
                            status, s);
+}
+
+size_t fp8_ep_smem_bytes(const moe_config_t& c, bool two_sets) {
+  const int64_t rows_per_expert =
+      c.E > 0 ? std::min<int64_t>((int64_t)c.T * c.K, (int64_t)c.E * c.capacity) / c.E : c.T;
+  return rows_per_expert >= 192 ? f8::smem_bytes<2>(c.E, two_sets)
+                                : f8::smem_bytes<1>(c.E, two_sets);
+}
+
+moe_status_t launch_mlp_fp8_ep(const moe_config_t& c, int modes, const uint8_t* xq,
+                               const uint8_t* xs, const int32_t* offsets, const int32_t* counts,
+                               const uint8_t* wq_gu, const uint8_t* ws_gu, const uint8_t* wq_d,
+                               const uint8_t* ws_d, uint8_t* hq, uint8_t* hs, void* y,
+                               int64_t R_max, uint32_t* status, cudaStream_t s,
+                               const EpTiles& t) {
+  if (R_max == 0) return MOE_OK;
+  moe_config_t l = c;
+  l.n_shared = 0;
+  const int64_t rows_per_expert =
+      c.E > 0 ? std::min<int64_t>((int64_t)c.T * c.K, (int64_t)c.E * c.capacity) / c.E : c.T;
+  if (rows_per_expert >= 192)
+    return f8::launch_mlp<2>(l, xq, xs, offsets, counts, wq_gu, ws_gu, wq_d, ws_d, hq, hs, y,
+                             R_max, status, s, modes, t);
+  return f8::launch_mlp<1>(l, xq, xs, offsets, counts, wq_gu, ws_gu, wq_d, ws_d, hq, hs, y, R_max,
+                           status, s, modes, t);
 }
 
 }  // namespace moe

@@ -227,6 +227,20 @@ moe_status_t launch_mlp_fp8(const moe_config_t& c, const uint8_t* xq, const uint
                             uint8_t* hq, uint8_t* hs, void* y, int64_t R_max, uint32_t* status,
                             cudaStream_t s);
 
+// Shared memory of launch_mlp_fp8_ep's kernels over c's E experts (two_sets:
+// with the remote-first order's tables).
+size_t fp8_ep_smem_bytes(const moe_config_t& c, bool two_sets);
+
+// One or both launches (modes: bit 0 gate/up, bit 1 down) of the fp8 grouped
+// GEMM of launch_mlp_fp8 over an expert-parallel owner's local experts (no
+// shared group), tile-signalled by `t` as launch_mlp_bf16_tc_ep.
+moe_status_t launch_mlp_fp8_ep(const moe_config_t& c, int modes, const uint8_t* xq,
+                               const uint8_t* xs, const int32_t* offsets, const int32_t* counts,
+                               const uint8_t* wq_gu, const uint8_t* ws_gu, const uint8_t* wq_d,
+                               const uint8_t* ws_d, uint8_t* hq, uint8_t* hs, void* y,
+                               int64_t R_max, uint32_t* status, cudaStream_t s,
+                               const EpTiles& t);
+
 // Ready-counter target of the down GEMM (its number of N tiles).
 inline uint32_t ready_target(const moe_config_t& c) { return (uint32_t)ceil_div(c.H, 256); }
 

@@ -111,7 +111,8 @@ extern "C" {
 /* Tile signalling ("Mixture-of-Experts acceleration through overlap": a
  * persistent GEMM that consumes rows as they arrive and publishes its output
  * tiles through flags that the consumer polls; remote-first tile order).
- * MOE_EP_TILE_SIGNAL (bf16, row_align % 128 == 0; else MOE_ERR_UNSUPPORTED):
+ * MOE_EP_TILE_SIGNAL (bf16 activations: the bf16 and the fp8 layer; row_align
+ *   % 128 == 0; else MOE_ERR_UNSUPPORTED):
  *   - moe_ep_expert_mlp does not wait for every sender before its grouped
  *     GEMM: each CTA of the gate/up GEMM waits, before it loads its 128 rows of
  *     a tile, only for the DISPATCH flags of the senders whose rows those are
@@ -216,9 +217,16 @@ moe_status_t moe_ep_layer_forward(const moe_config_t* cfg, const moe_ep_t* ep,
  *     ws_d_local their scales in the blocked layout (for the experts of rank d,
  *     the contiguous slice of moe_quantize_fp8's scales of all experts that
  *     starts at chunk row d*(E/W)*2F/128, resp. d*(E/W)*H/128).
+ *   With MOE_EP_TILE_SIGNAL the fp8 gate/up GEMM waits per CTA for the
+ *     senders of its rows (their codes and scale chunks) and the fp8 down GEMM
+ *     publishes y's 128-row blocks through the same ready counters as the bf16
+ *     layer; MOE_EP_REMOTE_FIRST orders its tiles the same way.
  * Limits: those of moe_layer_forward_fp8 on each rank's local experts
- * (bf16 activations, H % 256 == 0, F % 128 == 0, A % 128 == 0), and no
- * shared expert; else MOE_ERR_UNSUPPORTED. */
+ * (bf16 activations, H % 256 == 0, F % 128 == 0, A % 128 == 0); with
+ * MOE_EP_REMOTE_FIRST the order's tables (two ints per local expert) must fit
+ * the fp8 GEMM's shared memory beside its stages (about 340 local experts
+ * with 256-row tiles); else MOE_ERR_UNSUPPORTED. A shared expert (n_shared
+ * = 1) is run by every rank on its own tokens, as in the bf16 layer. */
 moe_status_t moe_ep_dispatch_fp8(const moe_config_t* cfg, const moe_ep_t* ep, const void* x,
                                  void* sym, void* const* peers, void* ws, size_t ws_bytes,
                                  void* stream);

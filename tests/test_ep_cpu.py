@@ -77,15 +77,31 @@ def test_check_tile_signal_flags(kw, flags, code):
     assert M.moe_ep_check(c, M.make_ep(2, 0, 1, 0, flags)) == code
 
 
-def test_tile_signal_needs_bf16_and_not_fp8():
+def test_tile_signal_needs_bf16_activations():
     c = cfg_of("tiny", S=2, row_align=128)   # fp32 activations
     assert M.moe_ep_check(c, M.make_ep(2, 0, 1, 0, M.MOE_EP_TILE_SIGNAL)) == M.MOE_ERR_UNSUPPORTED
+    # the fp8 layer (bf16 activations, e4m3 payload) takes both tile flags: with
+    # a valid configuration the missing workspace is the first error found
     c = cfg_of("mixtral")
-    ep = M.make_ep(2, 0, 1, 0, M.MOE_EP_TILE_SIGNAL)
     fake = 1 << 40
-    got = M.LIB.moe_ep_dispatch_fp8(ctypes.byref(c), ctypes.byref(ep), fake, fake, fake, None,
-                                    1 << 40, None)
-    assert got == M.MOE_ERR_UNSUPPORTED
+    for flags in (M.MOE_EP_TILE_SIGNAL, M.MOE_EP_TILE_SIGNAL | M.MOE_EP_REMOTE_FIRST):
+        ep = M.make_ep(2, 0, 1, 0, flags)
+        got = M.LIB.moe_ep_dispatch_fp8(ctypes.byref(c), ctypes.byref(ep), fake, fake, fake, None,
+                                        1 << 40, None)
+        assert got == M.MOE_ERR_WORKSPACE, flags
+
+
+def test_fp8_remote_first_needs_its_tables_to_fit():
+    # the remote-first order's two extra tables per local expert live in the
+    # fp8 GEMM's shared memory: 512 local experts do not fit beside six stages
+    c = M.make_config(T=16384, H=256, E=512, K=8, F=256, S=1, capacity=320, row_align=128)
+    fake = 1 << 40
+    for flags, code in ((M.MOE_EP_TILE_SIGNAL, M.MOE_ERR_WORKSPACE),
+                        (M.MOE_EP_TILE_SIGNAL | M.MOE_EP_REMOTE_FIRST, M.MOE_ERR_UNSUPPORTED)):
+        ep = M.make_ep(1, 0, 1, 0, flags)
+        got = M.LIB.moe_ep_dispatch_fp8(ctypes.byref(c), ctypes.byref(ep), fake, fake, fake, None,
+                                        1 << 40, None)
+        assert got == code, (flags, got)
 
 
 def test_shared_expert_with_fp32_activations():
