@@ -102,6 +102,9 @@ class EpGroup:
         for r, a in enumerate(self.addrs):
             if r != self.rank:
                 B.moe_ipc_close(a)
+        # an exported region is freed only after every importer has closed it
+        # (freeing it while another process still has it open is undefined)
+        dist.barrier(group=self.group)
         B.moe_ep_sym_free(self.sym)
         self.addrs = []
 

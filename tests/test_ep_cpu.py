@@ -4,6 +4,7 @@ errors caught before any launch, and the handle exchange of a process group
 (gloo, two ranks)."""
 import ctypes
 import os
+import time
 import re
 
 import pytest
@@ -263,8 +264,10 @@ def _group_worker(rank, world, port, q, device_epoch):
             "moe_ep_sym_alloc": lambda n: 1000 + rank,
             "moe_ipc_get_handle": lambda addr: bytes([addr % 256]) * 64,
             "moe_ipc_open": lambda h: calls.append(("open", h[0])) or 2000 + h[0],
-            "moe_ipc_close": lambda addr: calls.append(("close", addr)),
-            "moe_ep_sym_free": lambda addr: calls.append(("free", addr)),
+            # rank 1 closes its import late: every rank's free must still wait for it
+            "moe_ipc_close": lambda addr: (time.sleep(0.2 if rank == 1 else 0.0),
+                                           calls.append(("close", addr, time.monotonic()))),
+            "moe_ep_sym_free": lambda addr: calls.append(("free", addr, time.monotonic())),
             "moe_ep_workspace_init": lambda cfg, w, ws: calls.append(("ws_init", w)),
             "moe_ep_symmetric_init": lambda cfg, w, sym, n: calls.append(("sym_init", sym, n)),
             "moe_ep_layer_forward": lambda cfg, ep, *a: calls.append(
@@ -315,4 +318,9 @@ def test_ep_group_setup_steps_and_close_two_ranks(device_epoch):
         epochs = [c[3] for c in calls if c[0] == "forward"]
         assert epochs == ([0, 0, 0] if device_epoch else [1, 2, 3])
         assert all(c[1:3] == (2, r) for c in calls if c[0] == "forward")
-        assert calls[-2] == ("close", want[other]) and calls[-1] == ("free", 1000 + r)
+        assert calls[-2][:2] == ("close", want[other]) and calls[-1][:2] == ("free", 1000 + r)
+    # teardown order across the processes: every import is closed before any
+    # exporter frees its region (CLOCK_MONOTONIC is shared by the processes)
+    closes = [c[2] for r in range(2) for c in got[r][2] if c[0] == "close"]
+    frees = [c[2] for r in range(2) for c in got[r][2] if c[0] == "free"]
+    assert max(closes) < min(frees), (closes, frees)
