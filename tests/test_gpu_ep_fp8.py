@@ -8,7 +8,8 @@
   (moe_layer_forward_fp8) of its tokens over all E experts, which the fp8
   tests check against the fp8 oracle; and the whole chain within a relative
   Frobenius error of 1e-2 of the fp8 oracle's layer on two ranks;
-* at the Mixtral shape with two ranks, bit for bit the one-rank fp8 layer;
+* at the Mixtral shape with two ranks (untagged, tile-signalled and
+  remote-first), bit for bit the one-rank fp8 layer;
 * with a shared expert (every rank applies it to its own tokens), bit for bit
   the one-rank fp8 layer with the shared expert.
 """
@@ -122,7 +123,10 @@ def test_ep_fp8_chain_against_the_fp8_oracle(cuda_ok):
         assert fro <= 1e-2, f"rank {r}: relative Frobenius error {fro:.3e}"
 
 
-def test_ep_fp8_mixtral_two_ranks(cuda_ok):
+@pytest.mark.parametrize("flags", [0, M.MOE_EP_TILE_SIGNAL,
+                                   M.MOE_EP_TILE_SIGNAL | M.MOE_EP_REMOTE_FIRST],
+                         ids=["untagged", "tiles", "remote_first"])
+def test_ep_fp8_mixtral_two_ranks(cuda_ok, flags):
     wl = W_.WORKLOADS["mixtral"]
     W = 2
     dev = torch.device("cuda")
@@ -135,7 +139,7 @@ def test_ep_fp8_mixtral_two_ranks(cuda_ok):
     del full["w_gu"], full["w_d"]
     loc_gu = M.ep_local_fp8_weights(gq, gs, W, wl.E, 2 * wl.F, wl.H)
     loc_d = M.ep_local_fp8_weights(dq, ds, W, wl.E, wl.H, wl.F)
-    emu = EpOnOneDevice(cfg, W, dev)
+    emu = EpOnOneDevice(cfg, W, dev, flags=flags)
     outs = [torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device=dev) for _ in range(W)]
     emu.forward_fp8([i["logits"] for i in inps], [i["x"] for i in inps],
                     [loc_gu[r] + loc_d[r] for r in range(W)], outs)

@@ -1,6 +1,6 @@
 """Expert-parallel layer at the workloads' full per-rank sizes, W ranks
-emulated on one device (the launch configuration `bench.py --ep-emulate W`
-times): every rank's route bit for bit against the oracle, the exchanged
+emulated on one device (the launch configuration `bench.py --ep-emulate W
+[--ep-tiles]` times), untagged and tile-signalled: every rank's route bit for bit against the oracle, the exchanged
 counts and the layout bit for bit against the oracle's plan, sampled received
 rows bit for bit against the senders' token rows, and every rank's output
 bit for bit equal to the one-rank library layer over all E experts (which the
@@ -26,8 +26,15 @@ ROUTE_KEYS = ("topk_idx", "topk_w", "expert_counts", "overflow", "expert_offsets
               "segment_offsets", "token_slot", "row_src", "totals")
 
 
-@pytest.mark.parametrize("name,world", [("mixtral", 2), ("dsv3", 8), ("skewed", 4)])
-def test_workload_full_size_ep(cuda_ok, name, world):
+TILES = M.MOE_EP_TILE_SIGNAL
+REMOTE_FIRST = M.MOE_EP_TILE_SIGNAL | M.MOE_EP_REMOTE_FIRST
+
+
+@pytest.mark.parametrize("name,world,flags", [
+    ("mixtral", 2, 0), ("dsv3", 8, 0), ("skewed", 4, 0),
+    # the tile-signalled layer (MOE_EP_TILE_SIGNAL) at the same sizes
+    ("mixtral", 2, REMOTE_FIRST), ("dsv3", 8, TILES)])
+def test_workload_full_size_ep(cuda_ok, name, world, flags):
     wl = W.WORKLOADS[name]
     dev = torch.device("cuda")
     C = M.moe_capacity(wl.T, wl.K, wl.E, wl.cf)
@@ -35,7 +42,7 @@ def test_workload_full_size_ep(cuda_ok, name, world):
     full = W.make_inputs(wl, seed=0, device=dev)
     inps = [full] + [W.make_inputs(wl, seed=r, device=dev, weights=False) for r in range(1, world)]
     El = wl.E // world
-    emu = EpOnOneDevice(cfg, world, dev)
+    emu = EpOnOneDevice(cfg, world, dev, flags=flags)
     outs = [torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device=dev) for _ in range(world)]
     emu.forward([i["logits"] for i in inps], [i["x"] for i in inps],
                 [full["w_gu"][r * El:(r + 1) * El] for r in range(world)],
