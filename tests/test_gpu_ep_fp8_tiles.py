@@ -190,3 +190,21 @@ def test_fp8_owner_gemm_waits_for_a_late_sender(cuda_ok):
     for r in range(W):
         assert emu.status(r) == M.MOE_OK
         assert torch.equal(outs[r], fp8_one_rank(cfg, logits[r], xs[r], wq))
+
+
+@pytest.mark.parametrize("flags", [TILES, REMOTE_FIRST], ids=["tiles", "remote_first"])
+def test_tile_signalled_fp8_layer_over_many_steps(cuda_ok, flags):
+    # as the bf16 test: sixteen steps on the same inputs, every step bit for bit
+    # the first, which is the one-rank fp8 layer
+    W, T, H, E, K, F = 4, 640, 512, 16, 4, 384
+    cfg, C, logits, xs, wq, wq_local = _case(W, T, H, E, K, F, 1.0, 4243)
+    emu = EpOnOneDevice(cfg, W, DEV, flags=flags)
+    first = _step(emu, cfg, W, logits, xs, wq_local)
+    for r in range(W):
+        assert emu.status(r) == M.MOE_OK
+        assert torch.equal(first[r], fp8_one_rank(cfg, logits[r], xs[r], wq)), r
+    for step in range(1, 16):
+        outs = _step(emu, cfg, W, logits, xs, wq_local)
+        for r in range(W):
+            assert emu.status(r) == M.MOE_OK, (step, r)
+            assert torch.equal(outs[r], first[r]), (step, r)

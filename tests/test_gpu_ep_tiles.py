@@ -170,3 +170,23 @@ def test_owner_gemm_waits_for_a_late_sender(cuda_ok):
     for r in range(W):
         assert emu.status(r) == M.MOE_OK
         assert torch.equal(outs[r], one_rank_layer(cfg, logits[r], xs[r], w_gu, w_d))
+
+
+@pytest.mark.parametrize("flags", [TILES, REMOTE_FIRST], ids=["tiles", "remote_first"])
+def test_tile_signalled_layer_over_many_steps(cuda_ok, flags):
+    # sixteen steps on the same inputs: the two banks of ready counters and the
+    # step-numbered flags alternate and wrap, and every step's output is bit for
+    # bit the first one's, which is the one-rank layer's
+    W, T, H, E, K, F = 4, 640, 512, 16, 4, 384
+    cfg, C = _cfg(W, T, H, E, K, F, 1.0)
+    emu = EpOnOneDevice(cfg, W, DEV, flags=flags)
+    logits, xs, w_gu, w_d = make_case(W, T, H, E, K, F, "bf16", seed=4242)
+    first = _step(emu, cfg, W, logits, xs, w_gu, w_d)
+    for r in range(W):
+        assert emu.status(r) == M.MOE_OK
+        assert torch.equal(first[r], one_rank_layer(cfg, logits[r], xs[r], w_gu, w_d)), r
+    for step in range(1, 16):
+        outs = _step(emu, cfg, W, logits, xs, w_gu, w_d)
+        for r in range(W):
+            assert emu.status(r) == M.MOE_OK, (step, r)
+            assert torch.equal(outs[r], first[r]), (step, r)
